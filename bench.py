@@ -1,0 +1,419 @@
+"""Benchmark of the DP-SGD per-sample clip + sum + noise step on B200.
+
+One step = the whole hot path over one batch: dp_linear_step on every linear of the workload
+(Llama-7B-shaped block by default: 7 linears, B=8, T=2048, bf16).  Each call computes the
+per-sample norms, the clip factors, the clipped sum and the Gaussian noise.  The inputs are
+seeded synthetic tensors, resident in HBM.  They are larger than the 126 MB L2, and the 7
+linears cycle through 2.2 GB, so no L2 flush is needed between steps.
+
+Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+Under torchrun every rank runs an independent replica (the step has no cross-GPU exchange).
+Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "DP clip+sum+noise tokens/s and TFLOP/s as % of B200 roofline, 1 GPU"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="llama7b_block")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--method", default="auto", choices=["auto", "ghost", "explicit"])
+    ap.add_argument("--linears", default="", help="comma-separated subset of the workload's linears")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_model(w):
+    """Algorithmic flops and bytes of one step (per-linear sums; X counted per linear)."""
+    e = 2 if w.dtype == "bf16" else 4
+    N = w.tokens
+    flops = byts = 0.0
+    x_shared_bytes = 0.0
+    seen = set()
+    per_linear = []
+    for lin in w.linears:
+        m, n, r = lin.d_in, lin.d_out, w.r
+        if r:
+            f = 2.0 * N * n * r + 2.0 * N * m * r
+            b = N * m * e + N * n * e + m * r * 4 + n * r * e
+        else:
+            f = 2.0 * N * m * n
+            b = N * m * e + N * n * e + m * n * 4
+        flops += f
+        byts += b
+        x_shared_bytes += b - (N * m * e if lin.x_key in seen else 0)
+        seen.add(lin.x_key)
+        per_linear.append((lin, f, b))
+    return flops, byts, x_shared_bytes, per_linear
+
+
+def ghost_flops(w):
+    """Executed flops of the ghost-norm Gram tiles (upper-triangular 128-token tile pairs)."""
+    tt = math.ceil(w.T / 128)
+    pairs = tt * (tt + 1) // 2
+    return sum(w.B * pairs * 2.0 * 128 * 128 * (lin.d_in + (w.r or lin.d_out)) for lin in w.linears)
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        try:
+            import torch
+
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            target = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+        except Exception:
+            target = str(device_index)
+        self.target = target
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.target, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[3:7]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------------------- reference arm
+
+def oracle_block_sample(w, data, linears, sample=0):
+    """The fp64 oracle on one sample of the given linears; returns (seconds, block-equiv tokens)."""
+    import numpy as np
+
+    import oracle
+    from sample_gradient_clipping_b200 import inputs
+
+    total_mn = sum(l.d_in * (w.r or l.d_out) for l in w.linears)
+    t0 = time.perf_counter()
+    tokens = 0.0
+    for lin in linears:
+        X = inputs.as_f64(data["X"][lin.x_key][sample:sample + 1])
+        dY = inputs.as_f64(data["dY"][lin.name][sample:sample + 1])
+        P = None
+        if w.r:
+            P = oracle.round_to(w.dtype, oracle.projection(lin.d_out, w.r, w.seed, lin.layer_id))
+        oracle.linear_step(X, dY, w.C, w.sigma, w.seed, w.step, lin.layer_id, P)
+        tokens += w.T * lin.d_in * (w.r or lin.d_out) / total_mn
+    del np
+    return time.perf_counter() - t0, tokens
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+
+        return max(i.get("num_threads", 1) for i in threadpool_info()) or 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def run_reference(args, w, rank):
+    if rank != 0:
+        return 0
+    from sample_gradient_clipping_b200 import inputs
+
+    data = inputs.generate(w)
+    lin_cycle = list(w.linears)
+    for s in range(args.warmup):
+        oracle_block_sample(w, data, [lin_cycle[s % len(lin_cycle)]])
+    secs = toks = 0.0
+    for s in range(args.steps):
+        dt, tk = oracle_block_sample(w, data, [lin_cycle[(args.warmup + s) % len(lin_cycle)]])
+        secs += dt
+        toks += tk
+    value = toks / secs
+    cores = blas_threads()
+    sample = (f"each step: the fp64 oracle (norms, clip, sum, noise) on sample 0 ({w.T} tokens) of "
+              f"one linear, cycling through the {len(w.linears)} linears; tokens counted as the "
+              f"linear's share d_in*d_out of the block")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * secs / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "T": w.T, "linears": len(w.linears),
+                   "description": w.description},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------- our arm
+
+def run_ours(args, w, rank, world):
+    import torch
+
+    from sample_gradient_clipping_b200 import _lib, inputs
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    _lib.lib()
+    data = inputs.generate(w)
+    X = {k: v.to(dev) for k, v in data["X"].items()}
+    dY = {k: v.to(dev) for k, v in data["dY"].items()}
+    r = w.r
+    ws_bytes = max(_lib.workspace_size(w.B, w.T, l.d_in, l.d_out, r,
+                                       _lib.DP_BF16 if w.dtype == "bf16" else _lib.DP_F32)
+                   for l in w.linears)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    G = {l.name: torch.empty(l.d_in, r or l.d_out, dtype=torch.float32, device=dev) for l in w.linears}
+    norms = {l.name: torch.empty(w.B, dtype=torch.float32, device=dev) for l in w.linears}
+    stream = torch.cuda.current_stream(dev)
+
+    def step(k):
+        for l in w.linears:
+            _lib.dp_linear_step(X[l.x_key], dY[l.name], w.C, w.sigma, w.seed, w.step + k, l.layer_id,
+                                r=r, method=args.method, norms_out=norms[l.name], G_out=G[l.name],
+                                workspace=ws, stream=stream)
+
+    for k in range(args.warmup):
+        step(k)
+    torch.cuda.synchronize(dev)
+    if _lib.dp_workspace_status(ws, stream) != _lib.DP_OK:
+        raise RuntimeError("an in-kernel wait timed out during warm-up")
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    sampler = ClockSampler(local)
+    _lib.profiling_enable(True)
+    _lib.profiling_collect()
+    barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    launches0 = _lib.kernel_launches()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for k in range(args.steps):
+        step(args.warmup + k)
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    launches = _lib.kernel_launches() - launches0
+    clocks = sampler.stop()
+    prof = _lib.profiling_collect()
+    _lib.profiling_enable(False)
+    ms = ev0.elapsed_time(ev1) / args.steps
+    if _lib.dp_workspace_status(ws, stream) != _lib.DP_OK:
+        raise RuntimeError("an in-kernel wait timed out during the timed steps")
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, w, data, dev, stream, ws, r, _lib, torch, world)
+
+    if rank != 0:
+        return 0
+    pk, pk_kind = peaks()
+    flops, byts, xbytes, per_linear = workload_model(w)
+    tokens = w.tokens * world
+    roof_t_burst = max(flops / (pk["bf16_tflops"] * 1e12), byts / (pk["hbm_gbs"] * 1e9))
+    roof_t_sust = max(flops / (pk["bf16_tflops_sustained"] * 1e12), byts / (pk["hbm_gbs"] * 1e9))
+    step_s = ms / 1e3
+    kinds = {k: v for k, v in prof.items()}
+    dominant = max(kinds, key=lambda k: kinds[k][0]) if kinds else None
+    roofline = None
+    if dominant:
+        d_ms, d_n = kinds[dominant]
+        if dominant == "umma_clipsum":
+            work, unit, bound = flops * args.steps, "TFLOP/s", "tensor"
+        elif dominant == "umma_ghost_norm":
+            work, unit, bound = ghost_flops(w) * args.steps, "TFLOP/s", "tensor"
+        elif dominant == "umma_explicit_norm":
+            work, unit, bound = flops * args.steps, "TFLOP/s", "tensor"
+        else:
+            work, unit, bound = None, None, None
+        if work is not None:
+            achieved = work / (d_ms / 1e3) / 1e12
+            peak = pk["bf16_tflops_sustained"]
+            roofline = {"bound": bound, "kernel": dominant, "achieved": achieved, "peak": peak,
+                        "unit": unit, "frac": achieved / peak, "traffic": None,
+                        "peak_kind": f"{pk_kind} sustained bf16 (kernel timed inside a long step)",
+                        "launches": d_n // args.steps, "avg_launch_ms": d_ms / d_n,
+                        "share_of_step": d_ms / (ms * args.steps)}
+    line = {
+        "metric": METRIC, "value": tokens / step_s, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "T": w.T, "linears": len(w.linears),
+                   "method": args.method, "l2": "inputs larger than L2 (no flush)",
+                   "parallelism": "replicas" if world > 1 else "1 GPU",
+                   "description": w.description},
+        "tflops_alg": flops * world / step_s / 1e12,
+        "step_roofline": {"frac_of_burst": roof_t_burst / step_s, "frac_of_sustained": roof_t_sust / step_s,
+                          "roofline_ms_burst": roof_t_burst * 1e3, "peaks": pk_kind,
+                          "bytes_alg": byts, "bytes_alg_x_shared": xbytes, "flops_alg": flops,
+                          "executed_ghost_flops": ghost_flops(w)},
+        "roofline": roofline,
+        "kernels": {k: {"ms_per_step": v[0] / args.steps, "launches_per_step": v[1] / args.steps}
+                    for k, v in sorted(kinds.items(), key=lambda kv: -kv[1][0])},
+        "gpu_launches": launches,
+        "clocks": clocks,
+        "e2e": e2e,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        secs, toks = oracle_block_sample(w, data, list(w.linears))
+        line["cpu_baseline"] = {
+            "value": toks / secs, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"sample 0 ({w.T} tokens) through all {len(w.linears)} linears with the fp64 "
+                      f"oracle (norms, clip, sum, full noise), {secs:.1f} s"}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_e2e(args, w, data, dev, stream, ws, r, _lib, torch, world):
+    """Same step through the public API from pinned host buffers, copies inside the timing."""
+    hX = {k: v.pin_memory() for k, v in data["X"].items()}
+    hdY = {k: v.pin_memory() for k, v in data["dY"].items()}
+    dX = {k: torch.empty_like(v, device=dev) for k, v in hX.items()}
+    ddY = {k: torch.empty_like(v, device=dev) for k, v in hdY.items()}
+    G = {l.name: torch.empty(l.d_in, r or l.d_out, dtype=torch.float32, device=dev) for l in w.linears}
+    n = {l.name: torch.empty(w.B, dtype=torch.float32, device=dev) for l in w.linears}
+    hG = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in G.items()}
+    hn = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in n.items()}
+    bi = sum(v.numel() * v.element_size() for v in hX.values()) + \
+        sum(v.numel() * v.element_size() for v in hdY.values())
+    bo = sum(v.numel() * v.element_size() for v in hG.values()) + \
+        sum(v.numel() * v.element_size() for v in hn.values())
+
+    def step(k):
+        loaded = set()
+        for l in w.linears:
+            if l.x_key not in loaded:
+                dX[l.x_key].copy_(hX[l.x_key], non_blocking=True)
+                loaded.add(l.x_key)
+            ddY[l.name].copy_(hdY[l.name], non_blocking=True)
+            _lib.dp_linear_step(dX[l.x_key], ddY[l.name], w.C, w.sigma, w.seed, w.step + k, l.layer_id,
+                                r=r, method=args.method, norms_out=n[l.name], G_out=G[l.name],
+                                workspace=ws, stream=stream)
+            hG[l.name].copy_(G[l.name], non_blocking=True)
+            hn[l.name].copy_(n[l.name], non_blocking=True)
+
+    steps = max(1, min(args.steps, 5))
+    for k in range(min(args.warmup, 2)):
+        step(k)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for k in range(steps):
+        step(k)
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = ev0.elapsed_time(ev1) / steps
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    return {"value": w.tokens * world / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": bi,
+            "d2h_bytes_per_step": bo, "ms_per_step": ms, "steps": steps,
+            "result_read_back": "every linear's noisy clipped gradient and per-sample norms"}
+
+
+def main():
+    args = parse()
+    from sample_gradient_clipping_b200 import inputs
+
+    w = inputs.WORKLOADS[args.workload]
+    if args.linears:
+        keep = args.linears.split(",")
+        lins = tuple(l for l in w.linears if l.name in keep)
+        if not lins:
+            raise SystemExit(f"no linear of {w.name} in {keep}")
+        w = dataclasses.replace(w, name=f"{w.name}[{args.linears}]", linears=lins)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, w, rank)
+    if world > 1:
+        import torch
+
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        return run_ours(args, w, rank, world)
+    finally:
+        if world > 1:
+            import torch
+
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,179 @@
+/*
+ * dpclip.h -- C ABI of the B200 (sm_100a) per-sample gradient clipping library.
+ *
+ * The library privatises the weight gradient of one linear layer Y = X W, as DP-SGD does per
+ * layer.  X[B,T,d_in] is the layer input saved by the forward pass and dY[B,T,d_out] the
+ * output gradient.  Sample i's weight gradient is G_i = X_i^T dY_i.  A call of the library
+ * computes, per sample, the Frobenius norm n_i = ||G_i||, clips with c_i = min(1, C / n_i),
+ * sums S = sum_i c_i G_i and adds Gaussian noise of std sigma*C.  Sources:
+ *   - "FlashDP: Private Training Large Language Models with Efficient DP-SGD", Abstract:
+ *     per-sample gradient clipping is the costly step of DP-SGD.  FlashDP computes each
+ *     per-sample gradient once, in one fused task per layer, and matches per-layer clipped
+ *     DP-SGD.
+ *   - "Memory-Efficient Differentially Private Training with Gradient Random Projection"
+ *     (DP-GRAPE), Problem Statement: per-sample gradients are clipped before noise is added.
+ *     Methodology, "Random Projection over SVD" and "Order of Operations": the raw per-sample
+ *     gradient is projected by a random Gaussian matrix regenerated from a seed, and only
+ *     then clipped and noised.
+ *
+ * Conventions for every entry point:
+ *   - Tensor pointers are DEVICE pointers owned by the caller.  Tensors are row-major and
+ *     contiguous, with 16-byte aligned base addresses.
+ *   - X is [B, T, d_in] and dY is [B, T, d_out], both in dtype `dt`.  Token t of sample i
+ *     is row i*T + t.
+ *   - P is [d_out, r] in dtype `dt`.  Every output is fp32.
+ *   - Work is enqueued asynchronously on `stream`, a cudaStream_t passed as void*; NULL is
+ *     the legacy default stream.
+ *   - The library allocates no device memory.  Scratch comes from the caller's `workspace`,
+ *     sized by dp_workspace_size.
+ *   - Arguments are checked on the host before anything is enqueued.  On failure nothing on
+ *     the device is touched and a non-zero dp_status is returned.  Launch failures return
+ *     DP_ERR_CUDA.
+ *   - No kernel traps.  Every wait inside a kernel is bounded: when it runs out, the kernel
+ *     records it in the workspace's status word and returns, and dp_workspace_status then
+ *     reports DP_ERR_TIMEOUT.
+ *   - Shapes:
+ *       B, T, d_in, d_out >= 1;
+ *       d_in, d_out and r are multiples of 8 for bf16 and of 4 for fp32 (rows of 16 bytes);
+ *       B*T < 2^31;
+ *       an output of rows*cols elements has rows*cols <= 2^34, since one Philox counter
+ *       word numbers its blocks of four.
+ *   - Random numbers: Philox4x32-10 (Salmon et al., "Parallel random numbers: as easy as
+ *     1, 2, 3", SC'11), then Box-Muller (1958) in fp64:
+ *       key = (seed mod 2^32, seed >> 32);
+ *       counter = (j, layer_id, step mod 2^32, stream);
+ *       stream 0 = gradient noise, stream 1 = projection;
+ *       u1 = (x_even + 1) 2^-32 and u2 = x_odd 2^-32;
+ *       z_even = sqrt(-2 ln u1) cos(2 pi u2) and z_odd = sqrt(-2 ln u1) sin(2 pi u2).
+ *     Flat element k = row*cols + col of a buffer takes z_{k mod 4} of block j = k div 4.
+ */
+#ifndef DPCLIP_H
+#define DPCLIP_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    DP_OK = 0,
+    DP_ERR_INVALID_ARG = 1,   /* null pointer, bad shape, misalignment, C <= 0, sigma < 0 ... */
+    DP_ERR_UNSUPPORTED = 2,   /* valid request this build does not implement (e.g. fp32 ghost) */
+    DP_ERR_WORKSPACE = 3,     /* workspace smaller than dp_workspace_size() */
+    DP_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed; see dp_last_cuda_error */
+    DP_ERR_TIMEOUT = 5        /* a bounded in-kernel wait ran out (reported by dp_workspace_status) */
+} dp_status;
+
+typedef enum { DP_F32 = 0, DP_BF16 = 1 } dp_dtype;
+
+/* How n_i is computed.  Both methods give the same value up to rounding:
+ *   GHOST    : n_i^2 = sum_{t,s} (x_t . x_s)(dy_t . dy_s), from the two T x T Gram matrices of
+ *              sample i.  This is the ghost-norm identity behind the implicit methods the
+ *              FlashDP Abstract names (GhostClip).
+ *   EXPLICIT : n_i^2 = sum of squares of the tiles of G_i = X_i^T dY_i, formed on chip and
+ *              never stored.
+ *   AUTO     : GHOST when T (d_in + d_out) < 2 d_in d_out, else EXPLICIT.  With projection,
+ *              d_out is replaced by r in this rule.  fp32 inputs always use EXPLICIT. */
+typedef enum { DP_NORM_AUTO = 0, DP_NORM_GHOST = 1, DP_NORM_EXPLICIT = 2 } dp_norm_method;
+
+/* Bytes of workspace needed by every call below for these shapes.  r = 0 means unprojected.
+ * Returns 0 when the shape is invalid.  The workspace must be 256-byte aligned (any
+ * cudaMalloc or torch allocation is). */
+size_t dp_workspace_size(int B, int T, int d_in, int d_out, int r, dp_dtype dt);
+
+/* Per-sample gradient norms n_i = ||X_i^T dY_i||_F, or ||X_i^T dY_i P||_F when P != NULL.
+ * (FlashDP Abstract: per-sample gradient clipping needs each sample's gradient; DP-GRAPE
+ * Methodology: the norm is taken after projection.)
+ *   P      : NULL, or DEVICE [d_out, r] in dtype dt.
+ *   norms  : DEVICE fp32 [B], overwritten. */
+dp_status dp_per_sample_norms(const void* X, const void* dY, const void* P, int r, dp_dtype dt,
+                              int B, int T, int d_in, int d_out, dp_norm_method method,
+                              float* norms, void* workspace, size_t ws_bytes, void* stream);
+
+/* G_sum += sum_i c_i X_i^T dY_i [P], where c_i = 1 if norms[i] <= C and C / norms[i] otherwise.
+ * (FlashDP Abstract: per-layer clipped DP-SGD.)  No noise is added.
+ *   norms  : DEVICE fp32 [B].  These may be this layer's norms, or flat norms
+ *            sqrt(sum_l n_{i,l}^2) that the caller computed over several layers.
+ *   C      : > 0.  +INF means no clipping.
+ *   G_sum  : DEVICE fp32 [d_in, P ? r : d_out], accumulated into, so that several
+ *            microbatches can be summed. */
+dp_status dp_clip_accumulate(const void* X, const void* dY, const void* P, int r, dp_dtype dt,
+                             int B, int T, int d_in, int d_out, const float* norms, float C,
+                             float* G_sum, void* workspace, size_t ws_bytes, void* stream);
+
+/* G[k] += std * z_k for k < rows*cols, with z from Philox stream 0 under (seed, step,
+ * layer_id).  This is the Gaussian noise that follows clipping (DP-GRAPE Problem Statement
+ * and Methodology).  Each element is added in fp64 and rounded once to fp32.
+ *   G    : DEVICE fp32 [rows, cols], updated in place.
+ *   std  : >= 0 and finite; it is sigma * C for a DP-SGD step. */
+dp_status dp_add_noise(float* G, long long rows, long long cols, float std,
+                       unsigned long long seed, unsigned long long step, unsigned layer_id,
+                       void* stream);
+
+/* P[b, j] = z_{b*r + j} / sqrt(r), with z from Philox stream 1 under (seed, step 0,
+ * layer_id): a Gaussian matrix with N(0, 1/r) entries, regenerated from the seed, one per
+ * layer (DP-GRAPE Methodology, "Random Projection over SVD").  The value is formed in fp64,
+ * rounded to fp32, then for bf16 rounded to nearest even.
+ *   P : DEVICE [d_out, r] in dtype dt, overwritten. */
+dp_status dp_projection_matrix(void* P, dp_dtype dt, int d_out, int r,
+                               unsigned long long seed, unsigned layer_id, void* stream);
+
+/* One privatised step for one linear layer (FlashDP Abstract: one fused task per layer):
+ *   norms_out[i] = n_i,
+ *   G_out = sum_i c_i G_i [P] + sigma*C*z (Philox stream 0, (seed, step, layer_id)).
+ * Projection: pass P (DEVICE [d_out, r]).  Or pass P = NULL with r > 0 to regenerate P from
+ * (seed, layer_id) into the workspace, as dp_projection_matrix does.  r = 0 with P = NULL
+ * is the unprojected step.
+ *   C          : > 0.  +INF (no clipping) requires sigma = 0.
+ *   sigma      : >= 0.
+ *   norms_out  : NULL or DEVICE fp32 [B].
+ *   G_out      : DEVICE fp32 [d_in, r or d_out], overwritten. */
+dp_status dp_linear_step(const void* X, const void* dY, const void* P, int r, dp_dtype dt,
+                         int B, int T, int d_in, int d_out, float C, float sigma,
+                         unsigned long long seed, unsigned long long step, unsigned layer_id,
+                         dp_norm_method method, float* norms_out, float* G_out,
+                         void* workspace, size_t ws_bytes, void* stream);
+
+/* The raw Philox4x32-10 words behind every random number of the library (Salmon et al.,
+ * "Parallel random numbers: as easy as 1, 2, 3", SC'11), exposed so that the uint32 stream
+ * can be checked bit for bit: out[4 j + q] = word q of block j under counter
+ * (j, layer_id, step mod 2^32, stream_id) and key (seed mod 2^32, seed >> 32), j < nblocks.
+ *   out : DEVICE uint32 [nblocks, 4], overwritten; nblocks <= 2^32. */
+dp_status dp_philox_blocks(unsigned* out, unsigned long long nblocks, unsigned long long seed,
+                           unsigned long long step, unsigned layer_id, unsigned stream_id,
+                           void* stream);
+
+/* Synchronises `stream`, then reads the status word that the kernels of earlier calls wrote
+ * into `workspace`.  Returns DP_OK, DP_ERR_TIMEOUT (a bounded in-kernel wait ran out; the
+ * results of that call are invalid) or DP_ERR_CUDA.  The word is cleared at the start of
+ * every call that takes a workspace. */
+dp_status dp_workspace_status(const void* workspace, void* stream);
+
+/* Norm method that DP_NORM_AUTO picks for these shapes (DP_NORM_GHOST or DP_NORM_EXPLICIT). */
+dp_norm_method dp_auto_norm_method(int T, int d_in, int d_out, int r, dp_dtype dt);
+
+/* Launch accounting, for measurement.  dp_kernel_launches() is the number of kernels this
+ * library has launched in this process.  Once dp_profiling_enable(1) is called, every later
+ * launch is bracketed by two CUDA events recorded on its own stream.
+ * dp_profiling_collect(total_ms, launches) waits for those events and fills both arrays,
+ * which the caller owns, with dp_profiling_kinds() entries: the device time and launch count
+ * per kernel kind.  dp_profiling_kind_name() names a kind.  It then forgets the records.
+ * dp_profiling_enable(0) stops recording.  Both calls drop records not yet collected. */
+dp_status dp_profiling_enable(int on);
+int dp_profiling_kinds(void);
+const char* dp_profiling_kind_name(int kind);
+dp_status dp_profiling_collect(double* total_ms, long long* launches);
+long long dp_kernel_launches(void);
+
+/* Static description of a status code. */
+const char* dp_status_string(dp_status s);
+
+/* The last CUDA error string seen by this thread's calls, or "" if none. */
+const char* dp_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DPCLIP_H */

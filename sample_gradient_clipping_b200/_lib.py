@@ -1,0 +1,234 @@
+"""ctypes binding of libdpclip.so: the C ABI of include/dpclip.h, one Python function per entry.
+
+This module only marshals arguments.  It turns torch tensors into device pointers and shapes,
+and the current torch stream into a ``cudaStream_t``.  Every step of the computation runs in
+the CUDA library.  When the library is missing this module raises; it never falls back to
+other code.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libdpclip.so")
+
+DP_OK, DP_ERR_INVALID_ARG, DP_ERR_UNSUPPORTED, DP_ERR_WORKSPACE, DP_ERR_CUDA, DP_ERR_TIMEOUT = range(6)
+DP_F32, DP_BF16 = 0, 1
+DP_NORM_AUTO, DP_NORM_GHOST, DP_NORM_EXPLICIT = 0, 1, 2
+METHODS = {"auto": DP_NORM_AUTO, "ghost": DP_NORM_GHOST, "explicit": DP_NORM_EXPLICIT}
+
+_c_void_p, _c_int, _c_float = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+_c_size_t, _c_ll, _c_ull, _c_uint = ctypes.c_size_t, ctypes.c_longlong, ctypes.c_ulonglong, ctypes.c_uint
+
+SIGNATURES = {
+    "dp_workspace_size": (_c_size_t, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_int]),
+    "dp_per_sample_norms": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_int, _c_int,
+                                     _c_int, _c_int, _c_int, _c_void_p, _c_void_p, _c_size_t, _c_void_p]),
+    "dp_clip_accumulate": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_int, _c_int,
+                                    _c_int, _c_int, _c_void_p, _c_float, _c_void_p, _c_void_p,
+                                    _c_size_t, _c_void_p]),
+    "dp_add_noise": (_c_int, [_c_void_p, _c_ll, _c_ll, _c_float, _c_ull, _c_ull, _c_uint, _c_void_p]),
+    "dp_projection_matrix": (_c_int, [_c_void_p, _c_int, _c_int, _c_int, _c_ull, _c_uint, _c_void_p]),
+    "dp_linear_step": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_int, _c_int,
+                                _c_int, _c_int, _c_float, _c_float, _c_ull, _c_ull, _c_uint, _c_int,
+                                _c_void_p, _c_void_p, _c_void_p, _c_size_t, _c_void_p]),
+    "dp_workspace_status": (_c_int, [_c_void_p, _c_void_p]),
+    "dp_philox_blocks": (_c_int, [_c_void_p, _c_ull, _c_ull, _c_ull, _c_uint, _c_uint, _c_void_p]),
+    "dp_auto_norm_method": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_int]),
+    "dp_status_string": (ctypes.c_char_p, [_c_int]),
+    "dp_last_cuda_error": (ctypes.c_char_p, []),
+    "dp_profiling_enable": (_c_int, [_c_int]),
+    "dp_profiling_kinds": (_c_int, []),
+    "dp_profiling_kind_name": (ctypes.c_char_p, [_c_int]),
+    "dp_profiling_collect": (_c_int, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_c_ll)]),
+    "dp_kernel_launches": (_c_ll, []),
+}
+
+_lib = None
+
+
+def lib():
+    """The loaded library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with "
+                "`python -m sample_gradient_clipping_b200.build` (nvcc, sm_100a)")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(handle, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = handle
+    return _lib
+
+
+class DPError(RuntimeError):
+    def __init__(self, status, what):
+        detail = lib().dp_last_cuda_error().decode() if status == DP_ERR_CUDA else ""
+        msg = f"{what}: {lib().dp_status_string(status).decode()}"
+        super().__init__(msg + (f" ({detail})" if detail else ""))
+        self.status = status
+
+
+def check(status, what):
+    if status != DP_OK:
+        raise DPError(status, what)
+
+
+def _dtype_code(t):
+    import torch
+
+    if t.dtype == torch.bfloat16:
+        return DP_BF16
+    if t.dtype == torch.float32:
+        return DP_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _stream(stream):
+    import torch
+
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _bt_dims(X, dY):
+    if X.dim() != 3 or dY.dim() != 3 or X.shape[:2] != dY.shape[:2]:
+        raise ValueError("X must be [B, T, d_in] and dY [B, T, d_out]")
+    if not (X.is_contiguous() and dY.is_contiguous()):
+        raise ValueError("X and dY must be contiguous")
+    if X.dtype != dY.dtype:
+        raise ValueError("X and dY must share a dtype")
+    return int(X.shape[0]), int(X.shape[1]), int(X.shape[2]), int(dY.shape[2])
+
+
+def workspace_size(B, T, d_in, d_out, r=0, dtype_code=DP_BF16):
+    return int(lib().dp_workspace_size(B, T, d_in, d_out, r, dtype_code))
+
+
+def _workspace(X, dY, r, workspace):
+    import torch
+
+    B, T, d_in, d_out = _bt_dims(X, dY)
+    need = workspace_size(B, T, d_in, d_out, r, _dtype_code(X))
+    if need == 0:
+        raise DPError(DP_ERR_INVALID_ARG, "workspace size")
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=X.device)
+    return workspace
+
+
+def dp_per_sample_norms(X, dY, P=None, method="auto", norms=None, workspace=None, stream=None):
+    """Per-sample norms n_i (fp32 [B]) of X_i^T dY_i [P]."""
+    import torch
+
+    B, T, d_in, d_out = _bt_dims(X, dY)
+    r = int(P.shape[1]) if P is not None else 0
+    ws = _workspace(X, dY, r, workspace)
+    if norms is None:
+        norms = torch.empty(B, dtype=torch.float32, device=X.device)
+    check(lib().dp_per_sample_norms(_ptr(X), _ptr(dY), _ptr(P), r, _dtype_code(X), B, T, d_in, d_out,
+                                    METHODS[method], _ptr(norms), _ptr(ws), ws.numel(), _stream(stream)),
+          "dp_per_sample_norms")
+    return norms
+
+
+def dp_clip_accumulate(X, dY, norms, C, G_sum, P=None, workspace=None, stream=None):
+    """G_sum += sum_i c_i X_i^T dY_i [P] with c_i = min(1, C / norms[i])."""
+    B, T, d_in, d_out = _bt_dims(X, dY)
+    r = int(P.shape[1]) if P is not None else 0
+    ws = _workspace(X, dY, r, workspace)
+    check(lib().dp_clip_accumulate(_ptr(X), _ptr(dY), _ptr(P), r, _dtype_code(X), B, T, d_in, d_out,
+                                   _ptr(norms), float(C), _ptr(G_sum), _ptr(ws), ws.numel(),
+                                   _stream(stream)),
+          "dp_clip_accumulate")
+    return G_sum
+
+
+def dp_add_noise(G, std, seed, step, layer_id, stream=None):
+    """G += std * z (Philox stream 0 at (seed, step, layer_id)), in place."""
+    rows = int(G.shape[0])
+    cols = int(G.numel() // max(rows, 1))
+    check(lib().dp_add_noise(_ptr(G), rows, cols, float(std), int(seed), int(step), int(layer_id),
+                             _stream(stream)),
+          "dp_add_noise")
+    return G
+
+
+def dp_projection_matrix(P, seed, layer_id, stream=None):
+    """Fills P[d_out, r] with z / sqrt(r) from Philox stream 1 at (seed, layer_id)."""
+    check(lib().dp_projection_matrix(_ptr(P), _dtype_code(P), int(P.shape[0]), int(P.shape[1]),
+                                     int(seed), int(layer_id), _stream(stream)),
+          "dp_projection_matrix")
+    return P
+
+
+def dp_linear_step(X, dY, C, sigma, seed, step, layer_id, P=None, r=0, method="auto",
+                   norms_out=None, G_out=None, workspace=None, stream=None):
+    """One privatised step; returns (G_out, norms_out)."""
+    import torch
+
+    B, T, d_in, d_out = _bt_dims(X, dY)
+    if P is not None:
+        r = int(P.shape[1])
+    ws = _workspace(X, dY, r, workspace)
+    width = r if r else d_out
+    if G_out is None:
+        G_out = torch.empty(d_in, width, dtype=torch.float32, device=X.device)
+    if norms_out is None:
+        norms_out = torch.empty(B, dtype=torch.float32, device=X.device)
+    check(lib().dp_linear_step(_ptr(X), _ptr(dY), _ptr(P), r, _dtype_code(X), B, T, d_in, d_out,
+                               float(C), float(sigma), int(seed), int(step), int(layer_id),
+                               METHODS[method], _ptr(norms_out), _ptr(G_out), _ptr(ws), ws.numel(),
+                               _stream(stream)),
+          "dp_linear_step")
+    return G_out, norms_out
+
+
+def dp_philox_blocks(nblocks, seed, step, layer_id, stream_id, out=None, device="cuda", stream=None):
+    """Raw Philox4x32-10 words [nblocks, 4] (int32 tensor holding the uint32 bits)."""
+    import torch
+
+    if out is None:
+        out = torch.empty(int(nblocks), 4, dtype=torch.int32, device=device)
+    check(lib().dp_philox_blocks(_ptr(out), int(nblocks), int(seed), int(step), int(layer_id),
+                                 int(stream_id), _stream(stream)),
+          "dp_philox_blocks")
+    return out
+
+
+def dp_workspace_status(workspace, stream=None):
+    return lib().dp_workspace_status(_ptr(workspace), _stream(stream))
+
+
+def auto_norm_method(T, d_in, d_out, r=0, dtype_code=DP_BF16):
+    return {DP_NORM_GHOST: "ghost", DP_NORM_EXPLICIT: "explicit"}[
+        lib().dp_auto_norm_method(T, d_in, d_out, r, dtype_code)]
+
+
+def kernel_launches():
+    """Kernels launched by the library so far in this process."""
+    return int(lib().dp_kernel_launches())
+
+
+def profiling_enable(on=True):
+    check(lib().dp_profiling_enable(1 if on else 0), "dp_profiling_enable")
+
+
+def profiling_collect():
+    """{kernel kind: (device ms, launches)} for the launches recorded since the last collect."""
+    n = int(lib().dp_profiling_kinds())
+    ms = (ctypes.c_double * n)()
+    cnt = (_c_ll * n)()
+    check(lib().dp_profiling_collect(ms, cnt), "dp_profiling_collect")
+    return {lib().dp_profiling_kind_name(k).decode(): (ms[k], cnt[k]) for k in range(n) if cnt[k]}

@@ -1,0 +1,633 @@
+// Host side of the C ABI declared in include/dpclip.h: argument checks, workspace layout,
+// TMA tensor-map encoding, norm-method selection and the launches that make up each call.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "dpclip.h"
+#include "launch_profiler.h"
+#include "rng.cuh"
+#include "simt.cuh"
+#include "umma_gemm.cuh"
+
+using namespace dpclip;
+
+namespace {
+
+thread_local char g_cuda_error[256] = "";
+
+dp_status cuda_fail(cudaError_t e, const char* what) {
+  snprintf(g_cuda_error, sizeof(g_cuda_error), "%s: %s", what, cudaGetErrorString(e));
+  return DP_ERR_CUDA;
+}
+
+#define DP_CUDA(call)                                  \
+  do {                                                 \
+    cudaError_t e_ = (call);                           \
+    if (e_ != cudaSuccess) return cuda_fail(e_, #call); \
+  } while (0)
+
+#define DP_CHECK_LAUNCH(what)                          \
+  do {                                                 \
+    cudaError_t e_ = cudaGetLastError();               \
+    if (e_ != cudaSuccess) return cuda_fail(e_, what); \
+  } while (0)
+
+inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline int ceil_div(long long a, long long b) { return static_cast<int>((a + b - 1) / b); }
+
+int sm_count() {
+  static int counts[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (counts[dev] == 0) {
+    int c = 0;
+    if (cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || c <= 0) c = 148;
+    counts[dev] = c;
+  }
+  return counts[dev];
+}
+
+// ---------------------------------------------------------------- shape rules
+struct Shape {
+  int B, T, m, n, r;  // r = 0: unprojected
+  dp_dtype dt;
+  long long N() const { return static_cast<long long>(B) * T; }
+  int ne() const { return r > 0 ? r : n; }  // width of the clip-space gradient
+};
+
+bool valid_dtype(dp_dtype dt) { return dt == DP_F32 || dt == DP_BF16; }
+
+bool valid_shape(const Shape& s) {
+  if (!valid_dtype(s.dt)) return false;
+  if (s.B < 1 || s.T < 1 || s.m < 1 || s.n < 1 || s.r < 0) return false;
+  const int q = (s.dt == DP_BF16) ? 8 : 4;
+  if (s.m % q || s.n % q || s.r % q) return false;
+  if (s.N() >= (1ll << 31)) return false;
+  if (static_cast<long long>(s.m) * s.ne() > (1ll << 34)) return false;
+  if (s.dt == DP_F32 && s.B > 65535) return false;
+  return true;
+}
+
+struct WsLayout {
+  size_t status = 0, norm2 = 0, c = 0, scaled = 0, z = 0, p = 0, total = 0;
+};
+
+WsLayout ws_layout(const Shape& s) {
+  WsLayout L;
+  size_t off = 256;  // status word(s)
+  L.norm2 = off;
+  off += align256(static_cast<size_t>(s.B) * 8);
+  L.c = off;
+  off += align256(static_cast<size_t>(s.B) * 4);
+  const size_t e = (s.dt == DP_BF16) ? 2 : 4;
+  if (s.dt == DP_BF16) {
+    L.scaled = off;
+    off += align256(static_cast<size_t>(s.N()) * static_cast<size_t>(s.m < s.ne() ? s.m : s.ne()) * 2);
+  }
+  if (s.r > 0) {
+    L.z = off;
+    off += align256(static_cast<size_t>(s.N()) * s.r * e);
+    L.p = off;
+    off += align256(static_cast<size_t>(s.n) * s.r * e);
+  }
+  L.total = off;
+  return L;
+}
+
+dp_norm_method auto_method(const Shape& s) {
+  if (s.dt == DP_F32) return DP_NORM_EXPLICIT;
+  const double ghost = static_cast<double>(s.T) * (static_cast<double>(s.m) + s.ne());
+  const double expl = 2.0 * static_cast<double>(s.m) * s.ne();
+  return ghost < expl ? DP_NORM_GHOST : DP_NORM_EXPLICIT;
+}
+
+// ---------------------------------------------------------------- tensor maps
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+dp_status get_encoder() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  if (!g_encode) {
+    snprintf(g_cuda_error, sizeof(g_cuda_error), "cuTensorMapEncodeTiled unavailable");
+    return DP_ERR_CUDA;
+  }
+  return DP_OK;
+}
+
+// bf16 tensor [outer..., inner] with a box of {64 (inner), box_rows, 1...}, 128-byte swizzle.
+dp_status encode_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                      uint32_t box_rows) {
+  cuuint64_t gdim[3], gstride[2];
+  cuuint32_t box[3], estr[3] = {1, 1, 1};
+  for (int d = 0; d < rank; ++d) gdim[d] = dims[d];
+  uint64_t stride = dims[0] * 2;
+  for (int d = 1; d < rank; ++d) {
+    gstride[d - 1] = stride;
+    stride *= dims[d];
+  }
+  box[0] = 64;
+  box[1] = box_rows;
+  if (rank == 3) box[2] = 1;
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), gdim,
+                        gstride, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    snprintf(g_cuda_error, sizeof(g_cuda_error), "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+    return DP_ERR_CUDA;
+  }
+  return DP_OK;
+}
+
+dp_status map_2d(CUtensorMap* m, const void* base, long long rows, int cols, uint32_t box_rows) {
+  const uint64_t d[2] = {static_cast<uint64_t>(cols), static_cast<uint64_t>(rows)};
+  return encode_bf16(m, base, 2, d, box_rows);
+}
+dp_status map_3d(CUtensorMap* m, const void* base, int B, int T, int cols, uint32_t box_rows) {
+  const uint64_t d[3] = {static_cast<uint64_t>(cols), static_cast<uint64_t>(T), static_cast<uint64_t>(B)};
+  return encode_bf16(m, base, 3, d, box_rows);
+}
+
+// ---------------------------------------------------------------- engine launches
+template <class Cfg>
+dp_status launch_umma(const UmmaParams& p, cudaStream_t stream) {
+  static bool configured[64] = {false};
+  int dev = 0;
+  DP_CUDA(cudaGetDevice(&dev));
+  if (dev >= 0 && dev < 64 && !configured[dev]) {
+    DP_CUDA(cudaFuncSetAttribute(umma_kernel<Cfg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Cfg::SMEM_BYTES));
+    configured[dev] = true;
+  }
+  if (p.num_units <= 0) return DP_OK;
+  const int grid = p.num_units < sm_count() ? p.num_units : sm_count();
+  constexpr int kind = Cfg::EPI == kEpiClipSum        ? kKindClipSum
+                       : Cfg::EPI == kEpiExplicitNorm ? kKindExplicitNorm
+                       : Cfg::EPI == kEpiGhostNorm    ? kKindGhostNorm
+                                                      : kKindProject;
+  LaunchScope scope(kind, stream);
+  umma_kernel<Cfg><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(p);
+  DP_CHECK_LAUNCH("umma_kernel");
+  return DP_OK;
+}
+
+UmmaParams base_params(uint32_t* status) {
+  UmmaParams p;
+  memset(&p, 0, sizeof(p));
+  p.status = status;
+  return p;
+}
+
+int stream_grid(unsigned long long work_items, int threads) {
+  const unsigned long long blocks = (work_items + threads - 1) / threads;
+  const unsigned long long cap = static_cast<unsigned long long>(sm_count()) * 8;
+  return static_cast<int>(blocks < cap ? (blocks > 0 ? blocks : 1) : cap);
+}
+
+// norm2[i] += ||X_i^T Z_i||^2 (bf16 operands; Z is dY or the projected dY, ne columns)
+dp_status bf16_norms(const Shape& s, const void* X, const void* Z, dp_norm_method method,
+                     float* norm2, uint32_t* status, cudaStream_t stream) {
+  UmmaParams p = base_params(status);
+  p.norm2 = norm2;
+  const int ne = s.ne();
+  if (method == DP_NORM_GHOST) {
+    using Cfg = UmmaConfig<128, kEpiGhostNorm>;
+    dp_status st;
+    if ((st = map_3d(&p.tmA0, X, s.B, s.T, s.m, 128)) != DP_OK) return st;
+    p.tmB0 = p.tmA0;
+    if ((st = map_3d(&p.tmA1, Z, s.B, s.T, ne, 128)) != DP_OK) return st;
+    p.tmB1 = p.tmA1;
+    p.t_tiles = ceil_div(s.T, 128);
+    p.pairs_per_sample = p.t_tiles * (p.t_tiles + 1) / 2;
+    p.num_units = s.B * p.pairs_per_sample;
+    p.k_blocks = ceil_div(s.m, 64);
+    p.k_blocks1 = ceil_div(ne, 64);
+    return launch_umma<Cfg>(p, stream);
+  }
+  dp_status st;
+  if ((st = map_3d(&p.tmA0, X, s.B, s.T, s.m, 64)) != DP_OK) return st;
+  if ((st = map_3d(&p.tmB0, Z, s.B, s.T, ne, 64)) != DP_OK) return st;
+  p.k_blocks = ceil_div(s.T, 64);
+  p.m_tiles = ceil_div(s.m, 128);
+  if (ne <= 128) {
+    using Cfg = UmmaConfig<128, kEpiExplicitNorm>;
+    p.n_tiles = ceil_div(ne, 128);
+    p.num_units = s.B * p.m_tiles * p.n_tiles;
+    return launch_umma<Cfg>(p, stream);
+  }
+  using Cfg = UmmaConfig<256, kEpiExplicitNorm>;
+  p.n_tiles = ceil_div(ne, 256);
+  p.num_units = s.B * p.m_tiles * p.n_tiles;
+  return launch_umma<Cfg>(p, stream);
+}
+
+// out (+)= A^T Bm over all N rows (A: [N, m], Bm: [N, ne], both bf16, one already scaled by
+// c_i), plus noise when noise_std != 0.  `accumulate` = 0 overwrites out.
+dp_status bf16_clipsum(const Shape& s, const void* A, const void* Bm, float* out, int accumulate,
+                       double noise_std, unsigned long long seed, unsigned long long step,
+                       unsigned layer_id, uint32_t* status, cudaStream_t stream) {
+  UmmaParams p = base_params(status);
+  const int ne = s.ne();
+  const int BN = ne <= 128 ? 128 : 256;
+  dp_status st;
+  if ((st = map_2d(&p.tmA0, A, s.N(), s.m, 64)) != DP_OK) return st;
+  if ((st = map_2d(&p.tmB0, Bm, s.N(), ne, 64)) != DP_OK) return st;
+  p.m_tiles = ceil_div(s.m, 128);
+  p.n_tiles = ceil_div(ne, BN);
+  p.k_blocks = ceil_div(s.N(), 64);
+  const int tiles = p.m_tiles * p.n_tiles;
+  int splits = 1;
+  if (tiles < sm_count()) {
+    splits = sm_count() / tiles;
+    const int max_splits = p.k_blocks / 4 > 0 ? p.k_blocks / 4 : 1;
+    if (splits > max_splits) splits = max_splits;
+    if (splits < 1) splits = 1;
+  }
+  p.k_blocks_per_split = ceil_div(p.k_blocks, splits);
+  splits = ceil_div(p.k_blocks, p.k_blocks_per_split);  // every split non-empty
+  p.k_splits = splits;
+  p.num_units = tiles * splits;
+  p.out_rows = s.m;
+  p.out_cols = ne;
+  p.out_f32 = out;
+  if (splits > 1 || accumulate) {
+    p.out_mode = (splits > 1) ? kOutAtomicAdd : kOutAdd;
+    if (!accumulate)
+      DP_CUDA(cudaMemsetAsync(out, 0, static_cast<size_t>(s.m) * ne * sizeof(float), stream));
+  } else {
+    p.out_mode = kOutStore;
+  }
+  p.noise_std = noise_std;
+  const PhiloxKey key = philox_key_from_seed(seed);
+  p.key0 = key.k0;
+  p.key1 = key.k1;
+  p.layer_id = layer_id;
+  p.step_lo = static_cast<uint32_t>(step & 0xFFFFFFFFull);
+  if (BN == 128) return launch_umma<UmmaConfig<128, kEpiClipSum>>(p, stream);
+  return launch_umma<UmmaConfig<256, kEpiClipSum>>(p, stream);
+}
+
+// Z[N, r] = dY[N, n] P[n, r], bf16 out.
+dp_status bf16_project(const Shape& s, const void* dY, const void* P, void* Z, uint32_t* status,
+                       cudaStream_t stream) {
+  UmmaParams p = base_params(status);
+  dp_status st;
+  if ((st = map_2d(&p.tmA0, dY, s.N(), s.n, 128)) != DP_OK) return st;
+  if ((st = map_2d(&p.tmB0, P, s.n, s.r, 64)) != DP_OK) return st;
+  p.m_tiles = ceil_div(s.N(), 128);
+  p.k_blocks = ceil_div(s.n, 64);
+  p.k_blocks_per_split = p.k_blocks;
+  p.k_splits = 1;
+  p.out_rows = static_cast<int>(s.N());
+  p.out_cols = s.r;
+  p.out_bf16 = static_cast<__nv_bfloat16*>(Z);
+  if (s.r <= 128) {
+    p.n_tiles = ceil_div(s.r, 128);
+    p.num_units = p.m_tiles * p.n_tiles;
+    return launch_umma<UmmaConfig<128, kEpiStoreBf16>>(p, stream);
+  }
+  p.n_tiles = ceil_div(s.r, 256);
+  p.num_units = p.m_tiles * p.n_tiles;
+  return launch_umma<UmmaConfig<256, kEpiStoreBf16>>(p, stream);
+}
+
+dp_status launch_projection(void* P, dp_dtype dt, int d_out, int r, unsigned long long seed,
+                            unsigned layer_id, cudaStream_t stream) {
+  const unsigned long long total = static_cast<unsigned long long>(d_out) * r;
+  const int grid = stream_grid((total + 3) / 4, 256);
+  const PhiloxKey key = philox_key_from_seed(seed);
+  LaunchScope scope(kKindProjection, stream);
+  if (dt == DP_BF16)
+    projection_kernel<true><<<grid, 256, 0, stream>>>(P, total, r, key, layer_id);
+  else
+    projection_kernel<false><<<grid, 256, 0, stream>>>(P, total, r, key, layer_id);
+  DP_CHECK_LAUNCH("projection_kernel");
+  return DP_OK;
+}
+
+dp_status launch_scale(const void* in, void* out, long long rows, int cols, int T, NormSource src,
+                       float C, cudaStream_t stream) {
+  const unsigned long long vecs = static_cast<unsigned long long>(rows) * (cols / 8);
+  LaunchScope scope(kKindScale, stream);
+  scale_rows_bf16_kernel<<<stream_grid(vecs, 256), 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(in), static_cast<__nv_bfloat16*>(out), rows, cols, T, src, C);
+  DP_CHECK_LAUNCH("scale_rows_bf16_kernel");
+  return DP_OK;
+}
+
+dp_status launch_finalize(NormSource src, int B, float C, float* norms_out, float* c_out,
+                          cudaStream_t stream) {
+  LaunchScope scope(kKindFinalize, stream);
+  finalize_norms_kernel<<<ceil_div(B, 256), 256, 0, stream>>>(src, B, C, norms_out, c_out);
+  DP_CHECK_LAUNCH("finalize_norms_kernel");
+  return DP_OK;
+}
+
+// ---------------------------------------------------------------- common front end
+struct Call {
+  Shape s;
+  WsLayout L;
+  uint8_t* ws;
+  cudaStream_t stream;
+  uint32_t* status() const { return reinterpret_cast<uint32_t*>(ws + L.status); }
+  float* norm2_f32() const { return reinterpret_cast<float*>(ws + L.norm2); }
+  double* norm2_f64() const { return reinterpret_cast<double*>(ws + L.norm2); }
+  float* c() const { return reinterpret_cast<float*>(ws + L.c); }
+};
+
+dp_status check_common(const void* X, const void* dY, const void* P, int r, dp_dtype dt, int B,
+                       int T, int d_in, int d_out, void* workspace, size_t ws_bytes, bool p_from_seed,
+                       Call* call) {
+  if (!X || !dY || !workspace) return DP_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(dY) || (P && !aligned16(P))) return DP_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return DP_ERR_INVALID_ARG;
+  if (P && r < 1) return DP_ERR_INVALID_ARG;
+  if (!P && r != 0 && !p_from_seed) return DP_ERR_INVALID_ARG;
+  call->s = Shape{B, T, d_in, d_out, r, dt};
+  if (!valid_shape(call->s)) return DP_ERR_INVALID_ARG;
+  call->L = ws_layout(call->s);
+  if (ws_bytes < call->L.total) return DP_ERR_WORKSPACE;
+  call->ws = static_cast<uint8_t*>(workspace);
+  return DP_OK;
+}
+
+// Projection front end shared by the calls: returns the clip-space operand (dY or Z = dY P).
+dp_status clip_space_operand(Call& c, const void* dY, const void* P, bool p_from_seed,
+                             unsigned long long seed, unsigned layer_id, const void** Zout) {
+  if (c.s.r == 0) {
+    *Zout = dY;
+    return DP_OK;
+  }
+  const void* Pd = P;
+  dp_status st;
+  if (!P && p_from_seed) {
+    if ((st = launch_projection(c.ws + c.L.p, c.s.dt, c.s.n, c.s.r, seed, layer_id, c.stream)) != DP_OK)
+      return st;
+    Pd = c.ws + c.L.p;
+  }
+  void* Z = c.ws + c.L.z;
+  if (c.s.dt == DP_BF16) {
+    if ((st = bf16_project(c.s, dY, Pd, Z, c.status(), c.stream)) != DP_OK) return st;
+  } else {
+    const long long total = c.s.N() * c.s.r;
+    LaunchScope scope(kKindF32Project, c.stream);
+    f32_project_kernel<<<stream_grid(total, 256), 256, 0, c.stream>>>(
+        static_cast<const float*>(dY), static_cast<const float*>(Pd), static_cast<float*>(Z), c.s.N(),
+        c.s.n, c.s.r);
+    DP_CHECK_LAUNCH("f32_project_kernel");
+  }
+  *Zout = Z;
+  return DP_OK;
+}
+
+dp_status norms_into_ws(Call& c, const void* X, const void* Z, dp_norm_method method) {
+  if (c.s.dt == DP_F32) {
+    dim3 grid(ceil_div(c.s.ne(), kF32Tile), ceil_div(c.s.m, kF32Tile), c.s.B);
+    LaunchScope scope(kKindF32Norm, c.stream);
+    f32_norm_kernel<<<grid, 256, 0, c.stream>>>(static_cast<const float*>(X), static_cast<const float*>(Z),
+                                                 c.s.T, c.s.m, c.s.ne(), c.norm2_f64());
+    DP_CHECK_LAUNCH("f32_norm_kernel");
+    return DP_OK;
+  }
+  return bf16_norms(c.s, X, Z, method, c.norm2_f32(), c.status(), c.stream);
+}
+
+NormSource ws_norm_source(const Call& c) {
+  NormSource src{nullptr, nullptr, nullptr};
+  if (c.s.dt == DP_F32)
+    src.norm2_f64 = c.norm2_f64();
+  else
+    src.norm2_f32 = c.norm2_f32();
+  return src;
+}
+
+// G_out (+)= sum_i c_i X_i^T Z_i (+ noise) for norms given by `src`.
+dp_status clipped_sum(Call& c, const void* X, const void* Z, NormSource src, float C, float* out,
+                      int accumulate, double noise_std, unsigned long long seed,
+                      unsigned long long step, unsigned layer_id) {
+  const Shape& s = c.s;
+  if (s.dt == DP_F32) {
+    dim3 grid(ceil_div(s.ne(), kF32Tile), ceil_div(s.m, kF32Tile));
+    const PhiloxKey key = philox_key_from_seed(seed);
+    LaunchScope scope(kKindF32ClipSum, c.stream);
+    f32_clipsum_kernel<<<grid, 256, 0, c.stream>>>(
+        static_cast<const float*>(X), static_cast<const float*>(Z), s.N(), s.T, s.m, s.ne(), src, C,
+        out, accumulate, noise_std, key, layer_id, static_cast<uint32_t>(step & 0xFFFFFFFFull));
+    DP_CHECK_LAUNCH("f32_clipsum_kernel");
+    return DP_OK;
+  }
+  // Fold c_i into the narrower operand: one extra read + write of N * min(m, ne) bf16.
+  void* scaled = c.ws + c.L.scaled;
+  dp_status st;
+  if (s.ne() <= s.m) {
+    if ((st = launch_scale(Z, scaled, s.N(), s.ne(), s.T, src, C, c.stream)) != DP_OK) return st;
+    return bf16_clipsum(s, X, scaled, out, accumulate, noise_std, seed, step, layer_id, c.status(), c.stream);
+  }
+  if ((st = launch_scale(X, scaled, s.N(), s.m, s.T, src, C, c.stream)) != DP_OK) return st;
+  return bf16_clipsum(s, scaled, Z, out, accumulate, noise_std, seed, step, layer_id, c.status(), c.stream);
+}
+
+dp_status resolve_method(const Shape& s, dp_norm_method method, dp_norm_method* out) {
+  if (method == DP_NORM_AUTO) {
+    *out = auto_method(s);
+    return DP_OK;
+  }
+  if (method != DP_NORM_GHOST && method != DP_NORM_EXPLICIT) return DP_ERR_INVALID_ARG;
+  if (s.dt == DP_F32 && method == DP_NORM_GHOST) return DP_ERR_UNSUPPORTED;
+  *out = method;
+  return DP_OK;
+}
+
+}  // namespace
+
+// ==================================================================== C ABI
+extern "C" {
+
+size_t dp_workspace_size(int B, int T, int d_in, int d_out, int r, dp_dtype dt) {
+  const Shape s{B, T, d_in, d_out, r, dt};
+  if (!valid_shape(s)) return 0;
+  return ws_layout(s).total;
+}
+
+dp_norm_method dp_auto_norm_method(int T, int d_in, int d_out, int r, dp_dtype dt) {
+  return auto_method(Shape{1, T, d_in, d_out, r, dt});
+}
+
+dp_status dp_per_sample_norms(const void* X, const void* dY, const void* P, int r, dp_dtype dt, int B,
+                              int T, int d_in, int d_out, dp_norm_method method, float* norms,
+                              void* workspace, size_t ws_bytes, void* stream) {
+  Call c;
+  dp_status st = check_common(X, dY, P, r, dt, B, T, d_in, d_out, workspace, ws_bytes, false, &c);
+  if (st != DP_OK) return st;
+  if (!norms) return DP_ERR_INVALID_ARG;
+  dp_norm_method m;
+  if ((st = resolve_method(c.s, method, &m)) != DP_OK) return st;
+  if ((st = get_encoder()) != DP_OK && dt == DP_BF16) return st;
+  c.stream = static_cast<cudaStream_t>(stream);
+  DP_CUDA(cudaMemsetAsync(c.ws, 0, c.L.c, c.stream));  // status word + norm accumulators
+  const void* Z;
+  if ((st = clip_space_operand(c, dY, P, false, 0, 0, &Z)) != DP_OK) return st;
+  if ((st = norms_into_ws(c, X, Z, m)) != DP_OK) return st;
+  return launch_finalize(ws_norm_source(c), B, INFINITY, norms, nullptr, c.stream);
+}
+
+dp_status dp_clip_accumulate(const void* X, const void* dY, const void* P, int r, dp_dtype dt, int B,
+                             int T, int d_in, int d_out, const float* norms, float C, float* G_sum,
+                             void* workspace, size_t ws_bytes, void* stream) {
+  Call c;
+  dp_status st = check_common(X, dY, P, r, dt, B, T, d_in, d_out, workspace, ws_bytes, false, &c);
+  if (st != DP_OK) return st;
+  if (!norms || !G_sum || !aligned16(G_sum)) return DP_ERR_INVALID_ARG;
+  if (!(C > 0.0f)) return DP_ERR_INVALID_ARG;  // also rejects NaN
+  if ((st = get_encoder()) != DP_OK && dt == DP_BF16) return st;
+  c.stream = static_cast<cudaStream_t>(stream);
+  DP_CUDA(cudaMemsetAsync(c.ws, 0, 256, c.stream));  // status word
+  const void* Z;
+  if ((st = clip_space_operand(c, dY, P, false, 0, 0, &Z)) != DP_OK) return st;
+  NormSource src{nullptr, nullptr, norms};
+  return clipped_sum(c, X, Z, src, C, G_sum, 1, 0.0, 0, 0, 0);
+}
+
+dp_status dp_add_noise(float* G, long long rows, long long cols, float std, unsigned long long seed,
+                       unsigned long long step, unsigned layer_id, void* stream) {
+  if (!G || !aligned16(G) || rows < 1 || cols < 1) return DP_ERR_INVALID_ARG;
+  if (!(std >= 0.0f) || std::isinf(std)) return DP_ERR_INVALID_ARG;
+  if (rows > (1ll << 34) / cols) return DP_ERR_INVALID_ARG;
+  const unsigned long long total = static_cast<unsigned long long>(rows) * static_cast<unsigned long long>(cols);
+  if (std == 0.0f) return DP_OK;
+  const PhiloxKey key = philox_key_from_seed(seed);
+  LaunchScope scope(kKindNoise, static_cast<cudaStream_t>(stream));
+  noise_add_kernel<<<stream_grid((total + 3) / 4, 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      G, total, static_cast<double>(std), key, layer_id, static_cast<uint32_t>(step & 0xFFFFFFFFull));
+  DP_CHECK_LAUNCH("noise_add_kernel");
+  return DP_OK;
+}
+
+dp_status dp_projection_matrix(void* P, dp_dtype dt, int d_out, int r, unsigned long long seed,
+                               unsigned layer_id, void* stream) {
+  if (!P || !aligned16(P) || !valid_dtype(dt) || d_out < 1 || r < 1) return DP_ERR_INVALID_ARG;
+  const int q = (dt == DP_BF16) ? 8 : 4;
+  if (d_out % q || r % q) return DP_ERR_INVALID_ARG;
+  if (static_cast<long long>(d_out) * r > (1ll << 34)) return DP_ERR_INVALID_ARG;
+  return launch_projection(P, dt, d_out, r, seed, layer_id, static_cast<cudaStream_t>(stream));
+}
+
+dp_status dp_linear_step(const void* X, const void* dY, const void* P, int r, dp_dtype dt, int B, int T,
+                         int d_in, int d_out, float C, float sigma, unsigned long long seed,
+                         unsigned long long step, unsigned layer_id, dp_norm_method method,
+                         float* norms_out, float* G_out, void* workspace, size_t ws_bytes, void* stream) {
+  Call c;
+  dp_status st = check_common(X, dY, P, r, dt, B, T, d_in, d_out, workspace, ws_bytes, true, &c);
+  if (st != DP_OK) return st;
+  if (!G_out || !aligned16(G_out)) return DP_ERR_INVALID_ARG;
+  if (!(C > 0.0f) || !(sigma >= 0.0f) || std::isinf(sigma)) return DP_ERR_INVALID_ARG;
+  if (std::isinf(C) && sigma != 0.0f) return DP_ERR_INVALID_ARG;  // std = sigma * C would be inf
+  dp_norm_method m;
+  if ((st = resolve_method(c.s, method, &m)) != DP_OK) return st;
+  if ((st = get_encoder()) != DP_OK && dt == DP_BF16) return st;
+  c.stream = static_cast<cudaStream_t>(stream);
+  DP_CUDA(cudaMemsetAsync(c.ws, 0, c.L.c, c.stream));  // status word + norm accumulators
+  const void* Z;
+  if ((st = clip_space_operand(c, dY, P, true, seed, layer_id, &Z)) != DP_OK) return st;
+  if ((st = norms_into_ws(c, X, Z, m)) != DP_OK) return st;
+  const NormSource src = ws_norm_source(c);
+  if (norms_out && (st = launch_finalize(src, B, C, norms_out, c.c(), c.stream)) != DP_OK) return st;
+  // sigma = 0 means no noise, also for C = +inf (where sigma * C would be NaN).
+  const double noise_std = (sigma == 0.0f) ? 0.0 : static_cast<double>(sigma) * static_cast<double>(C);
+  return clipped_sum(c, X, Z, src, C, G_out, 0, noise_std, seed, step, layer_id);
+}
+
+dp_status dp_philox_blocks(unsigned* out, unsigned long long nblocks, unsigned long long seed,
+                           unsigned long long step, unsigned layer_id, unsigned stream_id,
+                           void* stream) {
+  if (!out || !aligned16(out) || nblocks < 1 || nblocks > (1ull << 32)) return DP_ERR_INVALID_ARG;
+  LaunchScope scope(kKindPhilox, static_cast<cudaStream_t>(stream));
+  philox_blocks_kernel<<<stream_grid(nblocks, 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      reinterpret_cast<uint4*>(out), nblocks, philox_key_from_seed(seed), layer_id,
+      static_cast<uint32_t>(step & 0xFFFFFFFFull), stream_id);
+  DP_CHECK_LAUNCH("philox_blocks_kernel");
+  return DP_OK;
+}
+
+dp_status dp_workspace_status(const void* workspace, void* stream) {
+  if (!workspace) return DP_ERR_INVALID_ARG;
+  DP_CUDA(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+  uint32_t word = 0;
+  DP_CUDA(cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost));
+  return word ? DP_ERR_TIMEOUT : DP_OK;
+}
+
+const char* dp_status_string(dp_status s) {
+  switch (s) {
+    case DP_OK: return "ok";
+    case DP_ERR_INVALID_ARG: return "invalid argument";
+    case DP_ERR_UNSUPPORTED: return "unsupported";
+    case DP_ERR_WORKSPACE: return "workspace too small";
+    case DP_ERR_CUDA: return "CUDA error";
+    case DP_ERR_TIMEOUT: return "in-kernel wait timed out";
+  }
+  return "unknown status";
+}
+
+const char* dp_last_cuda_error(void) { return g_cuda_error; }
+
+dp_status dp_profiling_enable(int on) {
+  LaunchProfiler& p = profiler();
+  std::lock_guard<std::mutex> g(p.mu);
+  for (auto& r : p.recs) {
+    p.give(r.a);
+    p.give(r.b);
+  }
+  p.recs.clear();
+  p.enabled = (on != 0);
+  return DP_OK;
+}
+
+int dp_profiling_kinds(void) { return kNumKinds; }
+
+const char* dp_profiling_kind_name(int kind) { return kernel_kind_name(kind); }
+
+dp_status dp_profiling_collect(double* total_ms, long long* launches) {
+  if (!total_ms || !launches) return DP_ERR_INVALID_ARG;
+  LaunchProfiler& p = profiler();
+  std::lock_guard<std::mutex> g(p.mu);
+  for (int k = 0; k < kNumKinds; ++k) {
+    total_ms[k] = 0.0;
+    launches[k] = 0;
+  }
+  dp_status st = DP_OK;
+  for (auto& r : p.recs) {
+    float ms = 0.f;
+    cudaError_t e = cudaEventSynchronize(r.b);
+    if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, r.a, r.b);
+    if (e != cudaSuccess) {
+      st = cuda_fail(e, "dp_profiling_collect");
+    } else {
+      total_ms[r.kind] += ms;
+      launches[r.kind] += 1;
+    }
+    p.give(r.a);
+    p.give(r.b);
+  }
+  p.recs.clear();
+  return st;
+}
+
+long long dp_kernel_launches(void) { return profiler().launches.load(); }
+
+}  // extern "C"

@@ -1,0 +1,245 @@
+// CUDA-core kernels of the step: Gaussian noise, the projection matrix, the clip-factor
+// row scaling, and the fp32 path.
+//
+// The noise, projection and scaling kernels are HBM-bound streams: 16-byte vector loads and
+// stores, and grids sized in multiples of the SM count.  The fp32 path keeps fp64
+// accumulators.  A product of two fp32 values is exact in fp64, so the fp32 parity bounds
+// (1e-5 on the sum, 1e-6 on the norms) hold at any T.
+#pragma once
+#include <cuda_bf16.h>
+
+#include <cstdint>
+
+#include "rng.cuh"
+
+namespace dpclip {
+
+// G[k] = fp32(G[k] + std * z_k), z from stream 0.  One thread per Philox block of 4 elements.
+__global__ void noise_add_kernel(float* __restrict__ G, unsigned long long total, double std_dev,
+                                 PhiloxKey key, uint32_t layer_id, uint32_t step_lo) {
+  const unsigned long long nblk = (total + 3) / 4;
+  for (unsigned long long j = blockIdx.x * static_cast<unsigned long long>(blockDim.x) + threadIdx.x;
+       j < nblk; j += static_cast<unsigned long long>(gridDim.x) * blockDim.x) {
+    double z[4];
+    normals4(static_cast<uint32_t>(j), layer_id, step_lo, kStreamNoise, key, z);
+    const unsigned long long k0 = 4 * j;
+    if (k0 + 3 < total) {
+      float4* p = reinterpret_cast<float4*>(G + k0);
+      float4 g = *p;
+      g.x = static_cast<float>(static_cast<double>(g.x) + std_dev * z[0]);
+      g.y = static_cast<float>(static_cast<double>(g.y) + std_dev * z[1]);
+      g.z = static_cast<float>(static_cast<double>(g.z) + std_dev * z[2]);
+      g.w = static_cast<float>(static_cast<double>(g.w) + std_dev * z[3]);
+      *p = g;
+    } else {
+      for (int q = 0; q < 4 && k0 + q < total; ++q)
+        G[k0 + q] = static_cast<float>(static_cast<double>(G[k0 + q]) + std_dev * z[q]);
+    }
+  }
+}
+
+// out[4 j + q] = word q of Philox block j (verification of the raw uint32 stream).
+__global__ void philox_blocks_kernel(uint4* __restrict__ out, unsigned long long nblocks,
+                                     PhiloxKey key, uint32_t layer_id, uint32_t step_lo,
+                                     uint32_t stream_id) {
+  for (unsigned long long j = blockIdx.x * static_cast<unsigned long long>(blockDim.x) + threadIdx.x;
+       j < nblocks; j += static_cast<unsigned long long>(gridDim.x) * blockDim.x)
+    out[j] = philox4x32_10(make_uint4(static_cast<uint32_t>(j), layer_id, step_lo, stream_id), key);
+}
+
+// P[k] = round(z_k / sqrt(r)), z from stream 1 at step 0: fp64 -> fp32 (RN) [-> bf16 (RN)].
+template <bool BF16>
+__global__ void projection_kernel(void* __restrict__ P, unsigned long long total, int r,
+                                  PhiloxKey key, uint32_t layer_id) {
+  const double scale = sqrt(static_cast<double>(r));
+  const unsigned long long nblk = (total + 3) / 4;
+  for (unsigned long long j = blockIdx.x * static_cast<unsigned long long>(blockDim.x) + threadIdx.x;
+       j < nblk; j += static_cast<unsigned long long>(gridDim.x) * blockDim.x) {
+    double z[4];
+    normals4(static_cast<uint32_t>(j), layer_id, 0u, kStreamProjection, key, z);
+    float f[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) f[q] = static_cast<float>(z[q] / scale);
+    const unsigned long long k0 = 4 * j;
+    if (BF16) {
+      __nv_bfloat16* out = static_cast<__nv_bfloat16*>(P);
+      if (k0 + 3 < total) {
+        __nv_bfloat162 lo = __floats2bfloat162_rn(f[0], f[1]);
+        __nv_bfloat162 hi = __floats2bfloat162_rn(f[2], f[3]);
+        uint2 pk;
+        pk.x = *reinterpret_cast<uint32_t*>(&lo);
+        pk.y = *reinterpret_cast<uint32_t*>(&hi);
+        *reinterpret_cast<uint2*>(out + k0) = pk;
+      } else {
+        for (int q = 0; q < 4 && k0 + q < total; ++q) out[k0 + q] = __float2bfloat16_rn(f[q]);
+      }
+    } else {
+      float* out = static_cast<float*>(P);
+      if (k0 + 3 < total) {
+        *reinterpret_cast<float4*>(out + k0) = make_float4(f[0], f[1], f[2], f[3]);
+      } else {
+        for (int q = 0; q < 4 && k0 + q < total; ++q) out[k0 + q] = f[q];
+      }
+    }
+  }
+}
+
+// Clip factor of sample i from either squared-norm accumulators or final norms.
+__device__ __forceinline__ float clip_factor(float norm, float C) {
+  return (norm <= C) ? 1.0f : C / norm;
+}
+
+struct NormSource {
+  const float* norm2_f32;   // bf16 path: fp32 accumulators of n_i^2
+  const double* norm2_f64;  // fp32 path: fp64 accumulators of n_i^2
+  const float* norms;       // caller-given norms
+  __device__ __forceinline__ float norm(int i) const {
+    if (norms) return norms[i];
+    if (norm2_f64) return static_cast<float>(sqrt(norm2_f64[i]));
+    return sqrtf(norm2_f32[i]);
+  }
+};
+
+// norms_out[i] = n_i and c_out[i] = c_i for i < B (either may be null).
+__global__ void finalize_norms_kernel(NormSource src, int B, float C, float* __restrict__ norms_out,
+                                      float* __restrict__ c_out) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < B; i += gridDim.x * blockDim.x) {
+    const float n = src.norm(i);
+    if (norms_out) norms_out[i] = n;
+    if (c_out) c_out[i] = clip_factor(n, C);
+  }
+}
+
+// out[row, :] = bf16(c_{row / T} * in[row, :]) for a [rows, cols] bf16 matrix, 8 elements per
+// thread (cols is a multiple of 8, rows are 16-byte aligned).
+__global__ void scale_rows_bf16_kernel(const __nv_bfloat16* __restrict__ in,
+                                       __nv_bfloat16* __restrict__ out, long long rows, int cols,
+                                       int T, NormSource src, float C) {
+  const int vec_per_row = cols / 8;
+  const long long total = rows * vec_per_row;
+  for (long long v = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; v < total;
+       v += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long row = v / vec_per_row;
+    const float c = clip_factor(src.norm(static_cast<int>(row / T)), C);
+    const uint4 pk = reinterpret_cast<const uint4*>(in)[v];
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&pk);
+    uint4 res;
+    __nv_bfloat162* o = reinterpret_cast<__nv_bfloat162*>(&res);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __bfloat1622float2(h[e]);
+      o[e] = __floats2bfloat162_rn(c * f.x, c * f.y);
+    }
+    reinterpret_cast<uint4*>(out)[v] = res;
+  }
+}
+
+// ------------------------------------------------------------------------------ fp32 path
+// Tiles of 32 rows (a) x 32 columns (b); thread (ty, tx) owns row a0 + ty and the four
+// consecutive columns b0 + 4 tx .. b0 + 4 tx + 3, so one Philox block feeds its noise.
+constexpr int kF32Tile = 32;
+
+// norm2[i] += sum over this tile of G_i[a, b]^2, G_i = X_i^T dY_i accumulated in fp64.
+__global__ void __launch_bounds__(256) f32_norm_kernel(const float* __restrict__ X,
+                                                       const float* __restrict__ dY, int T, int m,
+                                                       int n, double* __restrict__ norm2) {
+  __shared__ float xs[kF32Tile][kF32Tile + 1];  // [t][a]
+  __shared__ float ds[kF32Tile][kF32Tile + 1];  // [t][b]
+  __shared__ double red[8];
+  const int i = blockIdx.z;
+  const int a0 = blockIdx.y * kF32Tile, b0 = blockIdx.x * kF32Tile;
+  const int tx = threadIdx.x % 8, ty = threadIdx.x / 8;
+  const float* Xi = X + static_cast<long long>(i) * T * m;
+  const float* Di = dY + static_cast<long long>(i) * T * n;
+  double acc[4] = {0, 0, 0, 0};
+  for (int t0 = 0; t0 < T; t0 += kF32Tile) {
+    for (int e = threadIdx.x; e < kF32Tile * kF32Tile; e += 256) {
+      const int tt = e / kF32Tile, cc = e % kF32Tile;
+      const int t = t0 + tt;
+      xs[tt][cc] = (t < T && a0 + cc < m) ? Xi[static_cast<long long>(t) * m + a0 + cc] : 0.f;
+      ds[tt][cc] = (t < T && b0 + cc < n) ? Di[static_cast<long long>(t) * n + b0 + cc] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int tt = 0; tt < kF32Tile; ++tt) {
+      const double x = xs[tt][ty];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) acc[q] = fma(x, static_cast<double>(ds[tt][4 * tx + q]), acc[q]);
+    }
+    __syncthreads();
+  }
+  double ss = acc[0] * acc[0] + acc[1] * acc[1] + acc[2] * acc[2] + acc[3] * acc[3];
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
+  if (threadIdx.x % 32 == 0) red[threadIdx.x / 32] = ss;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double s = 0;
+    for (int w = 0; w < 8; ++w) s += red[w];
+    atomicAdd(norm2 + i, s);
+  }
+}
+
+// S[a, b] = sum_t c_{t / T} X[t, a] dY[t, b] over all N = B*T tokens (fp64 accumulation),
+// then out = fp32(S + std * z) (mode store) or out += fp32(S) (mode add).
+__global__ void __launch_bounds__(256) f32_clipsum_kernel(
+    const float* __restrict__ X, const float* __restrict__ dY, long long N, int T, int m, int n,
+    NormSource src, float C, float* __restrict__ out, int add_mode, double noise_std, PhiloxKey key,
+    uint32_t layer_id, uint32_t step_lo) {
+  __shared__ float xs[kF32Tile][kF32Tile + 1];
+  __shared__ float ds[kF32Tile][kF32Tile + 1];
+  __shared__ float cs[kF32Tile];
+  const int a0 = blockIdx.y * kF32Tile, b0 = blockIdx.x * kF32Tile;
+  const int tx = threadIdx.x % 8, ty = threadIdx.x / 8;
+  double acc[4] = {0, 0, 0, 0};
+  for (long long t0 = 0; t0 < N; t0 += kF32Tile) {
+    if (threadIdx.x < kF32Tile) {
+      const long long t = t0 + threadIdx.x;
+      cs[threadIdx.x] = (t < N) ? clip_factor(src.norm(static_cast<int>(t / T)), C) : 0.f;
+    }
+    for (int e = threadIdx.x; e < kF32Tile * kF32Tile; e += 256) {
+      const int tt = e / kF32Tile, cc = e % kF32Tile;
+      const long long t = t0 + tt;
+      xs[tt][cc] = (t < N && a0 + cc < m) ? X[t * m + a0 + cc] : 0.f;
+      ds[tt][cc] = (t < N && b0 + cc < n) ? dY[t * n + b0 + cc] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int tt = 0; tt < kF32Tile; ++tt) {
+      const double x = static_cast<double>(cs[tt]) * static_cast<double>(xs[tt][ty]);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) acc[q] = fma(x, static_cast<double>(ds[tt][4 * tx + q]), acc[q]);
+    }
+    __syncthreads();
+  }
+  const int a = a0 + ty, b = b0 + 4 * tx;
+  if (a >= m || b >= n) return;  // n is a multiple of 4: the four columns are all in range
+  float* dst = out + static_cast<long long>(a) * n + b;
+  if (add_mode) {
+    for (int q = 0; q < 4; ++q) dst[q] += static_cast<float>(acc[q]);
+    return;
+  }
+  if (noise_std != 0.0) {
+    const unsigned long long k = static_cast<unsigned long long>(a) * n + b;
+    double z[4];
+    normals4(static_cast<uint32_t>(k >> 2), layer_id, step_lo, kStreamNoise, key, z);
+    for (int q = 0; q < 4; ++q) acc[q] += noise_std * z[q];
+  }
+  for (int q = 0; q < 4; ++q) dst[q] = static_cast<float>(acc[q]);
+}
+
+// Z[t, j] = fp32(sum_b dY[t, b] P[b, j]) in fp64, one thread per output.
+__global__ void f32_project_kernel(const float* __restrict__ dY, const float* __restrict__ P,
+                                   float* __restrict__ Z, long long N, int n, int r) {
+  const long long total = N * r;
+  for (long long e = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; e < total;
+       e += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long t = e / r;
+    const int j = static_cast<int>(e % r);
+    double acc = 0;
+    for (int b = 0; b < n; ++b)
+      acc = fma(static_cast<double>(dY[t * n + b]), static_cast<double>(P[static_cast<long long>(b) * r + j]), acc);
+    Z[e] = static_cast<float>(acc);
+  }
+}
+
+}  // namespace dpclip

@@ -1,0 +1,431 @@
+// Persistent, warp-specialised tcgen05 contraction engine for sm_100a.
+//
+// One CTA per SM (192 threads) walks a static list of work units:
+//   warp 0      TMA producer: loads 128-byte-swizzled A/B tiles into a STAGES-deep smem ring;
+//   warp 1      MMA issuer: allocates all 512 TMEM columns, one lane issues tcgen05.mma
+//               (M = 128, N = BN, K = 16 per instruction) into a TMEM accumulator;
+//               accumulators are double-buffered so the epilogue of unit u overlaps the
+//               mainloop of unit u + 1;
+//   warps 2..5  epilogue: each thread owns one accumulator row (TMEM lane) and reads it
+//               back 32 columns at a time with tcgen05.ld.
+//
+// The same engine serves the four contractions of the step:
+//   kEpiClipSum      S[a, b] = sum_t Xs[t, a] dYs[t, b] over all B*T tokens (both operands
+//                    MN-major; the clip factor is already folded into one operand), with the
+//                    Philox/Box-Muller noise added in the epilogue before the fp32 store;
+//   kEpiExplicitNorm per (sample, output tile): the tile of G_i = X_i^T dY_i over the
+//                    sample's T tokens, squared and summed on chip into norm2[i];
+//   kEpiGhostNorm    per (sample, upper-triangular pair of 128-token blocks): the X Gram
+//                    tile and the dY Gram tile in two TMEM accumulators; the epilogue sums
+//                    w * Gx * Gy with w = 2 above the diagonal, 1 on it, 0 below;
+//   kEpiStoreBf16    Z = dY P (K-major dY, MN-major P), rounded to bf16.
+//
+// All waits are bounded (ptx.cuh); a wait that runs out sets the CTA's abort flag, records
+// its site in the status word and the CTA drains and exits.
+#pragma once
+#include <cuda_bf16.h>
+
+#include "ptx.cuh"
+#include "rng.cuh"
+
+namespace dpclip {
+
+enum EpiKind : int { kEpiClipSum = 0, kEpiExplicitNorm = 1, kEpiGhostNorm = 2, kEpiStoreBf16 = 3 };
+
+enum OutMode : int { kOutStore = 0, kOutAtomicAdd = 1, kOutAdd = 2 };
+
+struct alignas(64) UmmaParams {
+  CUtensorMap tmA0, tmB0, tmA1, tmB1;  // phase-1 maps are used by the ghost norm only
+  int num_units;
+  int m_tiles, n_tiles;       // output tile grid (128 x BN tiles)
+  int k_blocks;               // 64-deep K blocks of phase 0
+  int k_blocks1;              // 64-deep K blocks of phase 1 (ghost: the dY Gram)
+  int k_splits, k_blocks_per_split;
+  int t_tiles;                // ghost: 128-token blocks per sample
+  int pairs_per_sample;       // ghost: t_tiles (t_tiles + 1) / 2
+  int out_rows, out_cols;     // row-major output, leading dimension out_cols
+  int out_mode;               // OutMode (clip-sum)
+  float* out_f32;
+  __nv_bfloat16* out_bf16;
+  double noise_std;           // 0 disables the noise
+  uint32_t key0, key1, layer_id, step_lo;
+  float* norm2;               // [B] squared-norm accumulators
+  uint32_t* status;
+};
+
+template <int BN_, int EPI_>
+struct UmmaConfig {
+  static constexpr int BM = 128;
+  static constexpr int BN = BN_;
+  static constexpr int BK = 64;  // 64 bf16 = 128 bytes: one swizzle atom row
+  static constexpr int EPI = EPI_;
+  static constexpr bool A_MN = (EPI == kEpiClipSum || EPI == kEpiExplicitNorm);
+  static constexpr bool B_MN = (EPI != kEpiGhostNorm);
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = (196608 / STAGE_BYTES) < 8 ? (196608 / STAGE_BYTES) : 8;
+  static constexpr int ACCS = (EPI == kEpiGhostNorm) ? 2 : 1;  // accumulators per unit
+  static constexpr int ACC_COLS = BN * ACCS;
+  static constexpr int NUM_BUFS = 512 / ACC_COLS;
+  static constexpr int THREADS = 192;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
+  static constexpr uint32_t IDESC = umma_idesc_bf16(BM, BN, A_MN, B_MN);
+  static_assert(NUM_BUFS >= 1, "TMEM budget");
+  static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN");
+};
+
+struct Unit {
+  int m_blk, n_blk, kb_begin, kb_end, sample, split;
+};
+
+template <class Cfg>
+__device__ __forceinline__ Unit decode_unit(const UmmaParams& p, int u) {
+  Unit w{};
+  if (Cfg::EPI == kEpiGhostNorm) {
+    w.sample = u / p.pairs_per_sample;
+    int r = u % p.pairs_per_sample;
+    int row = 0;
+    while (r >= p.t_tiles - row) {
+      r -= p.t_tiles - row;
+      ++row;
+    }
+    w.m_blk = row;
+    w.n_blk = row + r;
+    w.kb_begin = 0;
+    w.kb_end = p.k_blocks;
+    w.split = 0;
+    return w;
+  }
+  const int tiles = p.m_tiles * p.n_tiles;
+  int r = u % tiles;
+  const int outer = u / tiles;
+  // Rasterise in groups of 8 row-tiles so that concurrently running CTAs share operand tiles
+  // in L2.
+  constexpr int G = 8;
+  const int per_group = G * p.n_tiles;
+  const int first_m = (r / per_group) * G;
+  const int gsz = min(G, p.m_tiles - first_m);
+  const int within = r % per_group;
+  w.m_blk = first_m + within % gsz;
+  w.n_blk = within / gsz;
+  if (Cfg::EPI == kEpiExplicitNorm) {
+    w.sample = outer;
+    w.split = 0;
+    w.kb_begin = 0;
+    w.kb_end = p.k_blocks;
+  } else {
+    w.sample = 0;
+    w.split = outer;
+    w.kb_begin = outer * p.k_blocks_per_split;
+    w.kb_end = min(p.k_blocks, w.kb_begin + p.k_blocks_per_split);
+  }
+  return w;
+}
+
+template <class Cfg>
+__device__ __forceinline__ void issue_stage_loads(const UmmaParams& p, const Unit& w, int phase,
+                                                  int kb, uint32_t sA, uint32_t sB,
+                                                  uint32_t bar) {
+  const int k0 = kb * Cfg::BK;
+  if (Cfg::EPI == kEpiClipSum) {
+#pragma unroll
+    for (int h = 0; h < Cfg::BM / 64; ++h)
+      tma_load_2d(sA + h * (Cfg::BK * 128), &p.tmA0, bar, w.m_blk * Cfg::BM + 64 * h, k0);
+#pragma unroll
+    for (int h = 0; h < Cfg::BN / 64; ++h)
+      tma_load_2d(sB + h * (Cfg::BK * 128), &p.tmB0, bar, w.n_blk * Cfg::BN + 64 * h, k0);
+  } else if (Cfg::EPI == kEpiExplicitNorm) {
+#pragma unroll
+    for (int h = 0; h < Cfg::BM / 64; ++h)
+      tma_load_3d(sA + h * (Cfg::BK * 128), &p.tmA0, bar, w.m_blk * Cfg::BM + 64 * h, k0,
+                  w.sample);
+#pragma unroll
+    for (int h = 0; h < Cfg::BN / 64; ++h)
+      tma_load_3d(sB + h * (Cfg::BK * 128), &p.tmB0, bar, w.n_blk * Cfg::BN + 64 * h, k0,
+                  w.sample);
+  } else if (Cfg::EPI == kEpiGhostNorm) {
+    const CUtensorMap* ma = phase ? &p.tmA1 : &p.tmA0;
+    const CUtensorMap* mb = phase ? &p.tmB1 : &p.tmB0;
+    tma_load_3d(sA, ma, bar, k0, w.m_blk * Cfg::BM, w.sample);
+    tma_load_3d(sB, mb, bar, k0, w.n_blk * Cfg::BN, w.sample);
+  } else {  // kEpiStoreBf16: A = dY rows (K-major), B = P (MN-major)
+    tma_load_2d(sA, &p.tmA0, bar, k0, w.m_blk * Cfg::BM);
+#pragma unroll
+    for (int h = 0; h < Cfg::BN / 64; ++h)
+      tma_load_2d(sB + h * (Cfg::BK * 128), &p.tmB0, bar, w.n_blk * Cfg::BN + 64 * h, k0);
+  }
+}
+
+template <class Cfg>
+__device__ __forceinline__ uint64_t operand_desc(uint32_t base, int ks, bool mn_major) {
+  // MN-major: 16 K-rows of 128 bytes per MMA step; MN chunks of 64 elements BK*128 bytes apart.
+  // K-major : 32 bytes (16 bf16) per MMA step inside the 128-byte swizzle row.
+  return mn_major ? umma_desc_sw128(base + ks * 2048, Cfg::BK * 128, 1024)
+                  : umma_desc_sw128(base + ks * 32, 16, 1024);
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+  return v;
+}
+
+template <class Cfg>
+__device__ __forceinline__ void epilogue_unit(const UmmaParams& p, const Unit& w, uint32_t tacc,
+                                              int wq, uint32_t lane) {
+  const int row = wq * 32 + static_cast<int>(lane);
+  if (Cfg::EPI == kEpiClipSum) {
+    const long long grow = static_cast<long long>(w.m_blk) * Cfg::BM + row;
+    const bool row_ok = grow < p.out_rows;
+    const bool noisy = (p.noise_std != 0.0) && (w.split == 0);
+    const PhiloxKey key{p.key0, p.key1};
+#pragma unroll 1
+    for (int c0 = 0; c0 < Cfg::BN; c0 += 32) {
+      float v[32];
+      __syncwarp();
+      tmem_ld32(tacc + c0, v);
+      tmem_ld_wait();
+      const long long gcol0 = static_cast<long long>(w.n_blk) * Cfg::BN + c0;
+      if (!row_ok || gcol0 >= p.out_cols) continue;  // the next tmem_ld32 reconverges first
+      float* dst = p.out_f32 + grow * p.out_cols + gcol0;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (gcol0 + 4 * q >= p.out_cols) break;  // out_cols is a multiple of 4
+        float4 val = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+        if (noisy) {
+          const unsigned long long k = static_cast<unsigned long long>(grow) * p.out_cols + gcol0 + 4 * q;
+          double z[4];
+          normals4(static_cast<uint32_t>(k >> 2), p.layer_id, p.step_lo, kStreamNoise, key, z);
+          val.x = static_cast<float>(static_cast<double>(val.x) + p.noise_std * z[0]);
+          val.y = static_cast<float>(static_cast<double>(val.y) + p.noise_std * z[1]);
+          val.z = static_cast<float>(static_cast<double>(val.z) + p.noise_std * z[2]);
+          val.w = static_cast<float>(static_cast<double>(val.w) + p.noise_std * z[3]);
+        }
+        float4* d4 = reinterpret_cast<float4*>(dst + 4 * q);
+        if (p.out_mode == kOutStore) {
+          *d4 = val;
+        } else if (p.out_mode == kOutAtomicAdd) {
+          atomicAdd(d4, val);
+        } else {
+          float4 o = *d4;
+          o.x += val.x; o.y += val.y; o.z += val.z; o.w += val.w;
+          *d4 = o;
+        }
+      }
+    }
+  } else if (Cfg::EPI == kEpiExplicitNorm) {
+    float ss = 0.f;
+#pragma unroll 1
+    for (int c0 = 0; c0 < Cfg::BN; c0 += 32) {
+      float v[32];
+      tmem_ld32(tacc + c0, v);
+      tmem_ld_wait();
+#pragma unroll
+      for (int e = 0; e < 32; ++e) ss = fmaf(v[e], v[e], ss);
+    }
+    ss = warp_sum(ss);
+    if (lane == 0) atomicAdd(p.norm2 + w.sample, ss);
+  } else if (Cfg::EPI == kEpiGhostNorm) {
+    // Rows and columns past T were zero-filled by TMA, so their Gram entries are 0.
+    const int t = w.m_blk * Cfg::BM + row;
+    float ss = 0.f;
+#pragma unroll 1
+    for (int c0 = 0; c0 < Cfg::BN; c0 += 32) {
+      float gx[32], gy[32];
+      tmem_ld32(tacc + c0, gx);
+      tmem_ld32(tacc + Cfg::BN + c0, gy);
+      tmem_ld_wait();
+      const int s0 = w.n_blk * Cfg::BN + c0;
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const int s = s0 + e;
+        const float wgt = (t < s) ? 2.f : ((t == s) ? 1.f : 0.f);
+        ss = fmaf(wgt * gx[e], gy[e], ss);
+      }
+    }
+    ss = warp_sum(ss);
+    if (lane == 0) atomicAdd(p.norm2 + w.sample, ss);
+  } else {  // kEpiStoreBf16
+    const long long grow = static_cast<long long>(w.m_blk) * Cfg::BM + row;
+#pragma unroll 1
+    for (int c0 = 0; c0 < Cfg::BN; c0 += 32) {
+      float v[32];
+      __syncwarp();
+      tmem_ld32(tacc + c0, v);
+      tmem_ld_wait();
+      const long long gcol0 = static_cast<long long>(w.n_blk) * Cfg::BN + c0;
+      if (grow >= p.out_rows) continue;  // the next tmem_ld32 reconverges first
+      __nv_bfloat16* dst = p.out_bf16 + grow * p.out_cols + gcol0;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        if (gcol0 + 8 * q >= p.out_cols) break;  // out_cols is a multiple of 8
+        uint4 pk;
+        __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&pk);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) h[e] = __floats2bfloat162_rn(v[8 * q + 2 * e], v[8 * q + 2 * e + 1]);
+        *reinterpret_cast<uint4*>(dst + 8 * q) = pk;
+      }
+    }
+  }
+}
+
+template <class Cfg>
+__global__ void __launch_bounds__(Cfg::THREADS, 1) umma_kernel(const __grid_constant__ UmmaParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::STAGES * Cfg::STAGE_BYTES);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + Cfg::STAGES;
+  uint64_t* acc_full = bars + 2 * Cfg::STAGES;
+  uint64_t* acc_empty = acc_full + Cfg::NUM_BUFS;
+  uint64_t* drain = acc_empty + Cfg::NUM_BUFS;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x / 32;
+  const uint32_t lane = lane_id();
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < Cfg::STAGES; ++s) {
+      mbar_init(smem_addr(full + s), 1);
+      mbar_init(smem_addr(empty + s), 1);
+    }
+    for (int b = 0; b < Cfg::NUM_BUFS; ++b) {
+      mbar_init(smem_addr(acc_full + b), 1);
+      mbar_init(smem_addr(acc_empty + b), 4);  // one arrival per epilogue warp
+    }
+    mbar_init(smem_addr(drain), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&p.tmA0);
+    tma_prefetch_desc(&p.tmB0);
+    if (Cfg::EPI == kEpiGhostNorm) {
+      tma_prefetch_desc(&p.tmA1);
+      tma_prefetch_desc(&p.tmB1);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_addr(tmem_slot), 512);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int nphases = (Cfg::EPI == kEpiGhostNorm) ? 2 : 1;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
+        const Unit w = decode_unit<Cfg>(p, u);
+        for (int ph = 0; ok && ph < nphases; ++ph) {
+          const int kb_end = ph ? p.k_blocks1 : w.kb_end;
+          const int kb_begin = ph ? 0 : w.kb_begin;
+          for (int kb = kb_begin; kb < kb_end; ++kb) {
+            if (!mbar_wait_bounded(smem_addr(empty + stage), phase ^ 1u, abort_flag, p.status, 1u)) {
+              ok = false;
+              break;
+            }
+            const uint32_t sA = smem_addr(smem + stage * Cfg::STAGE_BYTES);
+            const uint32_t bar = smem_addr(full + stage);
+            mbar_arrive_expect_tx(bar, Cfg::STAGE_BYTES);
+            issue_stage_loads<Cfg>(p, w, ph, kb, sA, sA + Cfg::A_BYTES, bar);
+            if (++stage == Cfg::STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int buf = 0;
+      uint32_t buf_phase = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
+        const Unit w = decode_unit<Cfg>(p, u);
+        if (!mbar_wait_bounded(smem_addr(acc_empty + buf), buf_phase ^ 1u, abort_flag, p.status, 2u)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        for (int ph = 0; ok && ph < nphases; ++ph) {
+          const uint32_t d_tmem = tmem_base + buf * Cfg::ACC_COLS + ph * Cfg::BN;
+          const int kb_end = ph ? p.k_blocks1 : w.kb_end;
+          const int kb_begin = ph ? 0 : w.kb_begin;
+          for (int kb = kb_begin; kb < kb_end; ++kb) {
+            if (!mbar_wait_bounded(smem_addr(full + stage), phase, abort_flag, p.status, 3u)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t sA = smem_addr(smem + stage * Cfg::STAGE_BYTES);
+            const uint32_t sB = sA + Cfg::A_BYTES;
+#pragma unroll
+            for (int ks = 0; ks < Cfg::BK / 16; ++ks) {
+              umma_bf16(d_tmem, operand_desc<Cfg>(sA, ks, Cfg::A_MN),
+                        operand_desc<Cfg>(sB, ks, Cfg::B_MN), Cfg::IDESC,
+                        (kb > kb_begin || ks > 0) ? 1u : 0u);
+            }
+            umma_commit(smem_addr(empty + stage));  // frees the smem stage once read
+            if (++stage == Cfg::STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+        }
+        if (!ok) break;
+        umma_commit(smem_addr(acc_full + buf));  // accumulator ready for the epilogue
+        if (++buf == Cfg::NUM_BUFS) {
+          buf = 0;
+          buf_phase ^= 1u;
+        }
+      }
+      // Make sure no MMA is still writing TMEM before it is released.
+      umma_commit(smem_addr(drain));
+      const unsigned long long t0 = global_timer_ns();
+      while (!mbar_try_wait(smem_addr(drain), 0u)) {
+        if (global_timer_ns() - t0 > kWaitLimitNs) {
+          if (p.status) atomicCAS(p.status, 0u, 5u);
+          break;
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue warps 2..5
+    const int wq = warp & 3;  // TMEM lane quarter this warp may access
+    int buf = 0;
+    uint32_t buf_phase = 0;
+    for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
+      const Unit w = decode_unit<Cfg>(p, u);
+      if (!mbar_wait_bounded(smem_addr(acc_full + buf), buf_phase, abort_flag, p.status, 4u)) break;
+      tc_fence_after();
+      const uint32_t tacc = tmem_base + buf * Cfg::ACC_COLS + (static_cast<uint32_t>(wq * 32) << 16);
+      epilogue_unit<Cfg>(p, w, tacc, wq, lane);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_addr(acc_empty + buf));
+      if (++buf == Cfg::NUM_BUFS) {
+        buf = 0;
+        buf_phase ^= 1u;
+      }
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+}  // namespace dpclip

@@ -1,0 +1,139 @@
+"""The C ABI without a GPU: the library loads, exports every declared entry point, sizes its
+workspace, and rejects bad arguments on the host before touching the device."""
+import math
+import os
+import re
+
+import pytest
+
+from sample_gradient_clipping_b200 import _lib, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dpclip.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return _lib.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(dp_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_functions()
+    assert len(names) >= 10
+    for name in names:
+        assert hasattr(L, name), name
+    assert set(names) == set(_lib.SIGNATURES), "binding and header disagree"
+
+
+def test_status_strings(L):
+    for code in range(6):
+        assert L.dp_status_string(code)
+    assert L.dp_status_string(0) == b"ok"
+
+
+def test_workspace_size(L):
+    ws = L.dp_workspace_size(8, 2048, 4096, 11008, 0, _lib.DP_BF16)
+    # status + norm2 + c + the scaled copy of the narrower operand (X here: 4096 wide)
+    assert ws >= 8 * 2048 * 4096 * 2
+    assert ws < 8 * 2048 * 4096 * 2 + 4096
+    assert L.dp_workspace_size(64, 128, 1024, 1024, 128, _lib.DP_BF16) >= 64 * 128 * 128 * 2 * 2
+    assert L.dp_workspace_size(0, 1, 8, 8, 0, _lib.DP_BF16) == 0
+    assert L.dp_workspace_size(1, 1, 12, 8, 0, _lib.DP_BF16) == 0     # d_in not a multiple of 8
+    assert L.dp_workspace_size(1, 1, 12, 8, 0, _lib.DP_F32) > 0        # fp32 needs multiples of 4
+
+
+def test_auto_method_rule(L):
+    # ghost iff T (d_in + d_out) < 2 d_in d_out; fp32 is always explicit
+    assert _lib.auto_norm_method(2048, 4096, 4096) == "ghost"
+    assert _lib.auto_norm_method(128, 1024, 1024, 128) == "ghost"
+    assert _lib.auto_norm_method(4096, 64, 64) == "explicit"
+    assert _lib.auto_norm_method(16, 64, 32, 0, _lib.DP_F32) == "explicit"
+
+
+FAKE = 0x10000          # 16-byte aligned, never dereferenced: every case fails on the host
+ODD = FAKE + 4
+
+
+def _step(L, **kw):
+    a = dict(X=FAKE, dY=FAKE, P=None, r=0, dt=_lib.DP_BF16, B=2, T=4, d_in=16, d_out=16, C=1.0,
+             sigma=1.0, seed=0, step=0, layer=0, method=0, norms=None, G=FAKE, ws=FAKE,
+             ws_bytes=1 << 30, stream=None)
+    a.update(kw)
+    return L.dp_linear_step(a["X"], a["dY"], a["P"], a["r"], a["dt"], a["B"], a["T"], a["d_in"],
+                            a["d_out"], a["C"], a["sigma"], a["seed"], a["step"], a["layer"],
+                            a["method"], a["norms"], a["G"], a["ws"], a["ws_bytes"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(X=None), _lib.DP_ERR_INVALID_ARG),
+    (dict(dY=None), _lib.DP_ERR_INVALID_ARG),
+    (dict(G=None), _lib.DP_ERR_INVALID_ARG),
+    (dict(ws=None), _lib.DP_ERR_INVALID_ARG),
+    (dict(X=ODD), _lib.DP_ERR_INVALID_ARG),
+    (dict(G=ODD), _lib.DP_ERR_INVALID_ARG),
+    (dict(ws=FAKE + 16), _lib.DP_ERR_INVALID_ARG),         # workspace must be 256-byte aligned
+    (dict(B=0), _lib.DP_ERR_INVALID_ARG),
+    (dict(T=0), _lib.DP_ERR_INVALID_ARG),
+    (dict(d_in=12), _lib.DP_ERR_INVALID_ARG),
+    (dict(d_out=20), _lib.DP_ERR_INVALID_ARG),
+    (dict(dt=7), _lib.DP_ERR_INVALID_ARG),
+    (dict(C=0.0), _lib.DP_ERR_INVALID_ARG),
+    (dict(C=-1.0), _lib.DP_ERR_INVALID_ARG),
+    (dict(C=float("nan")), _lib.DP_ERR_INVALID_ARG),
+    (dict(sigma=-0.5), _lib.DP_ERR_INVALID_ARG),
+    (dict(sigma=float("inf")), _lib.DP_ERR_INVALID_ARG),
+    (dict(C=math.inf, sigma=1.0), _lib.DP_ERR_INVALID_ARG),  # noise std would be infinite
+    (dict(P=FAKE, r=0), _lib.DP_ERR_INVALID_ARG),
+    (dict(r=12), _lib.DP_ERR_INVALID_ARG),
+    (dict(method=9), _lib.DP_ERR_INVALID_ARG),
+    (dict(dt=_lib.DP_F32, method=_lib.DP_NORM_GHOST), _lib.DP_ERR_UNSUPPORTED),
+    (dict(ws_bytes=512), _lib.DP_ERR_WORKSPACE),
+    (dict(B=1 << 16, T=1 << 15), _lib.DP_ERR_INVALID_ARG),   # B*T >= 2^31
+])
+def test_linear_step_rejects_on_host(L, kw, want):
+    assert _step(L, **kw) == want
+
+
+def test_other_entry_points_reject_on_host(L):
+    E = _lib.DP_ERR_INVALID_ARG
+    assert L.dp_add_noise(None, 4, 4, 1.0, 0, 0, 0, None) == E
+    assert L.dp_add_noise(ODD, 4, 4, 1.0, 0, 0, 0, None) == E
+    assert L.dp_add_noise(FAKE, 0, 4, 1.0, 0, 0, 0, None) == E
+    assert L.dp_add_noise(FAKE, 4, 4, -1.0, 0, 0, 0, None) == E
+    assert L.dp_add_noise(FAKE, 4, 4, float("nan"), 0, 0, 0, None) == E
+    assert L.dp_add_noise(FAKE, 1 << 20, 1 << 20, 1.0, 0, 0, 0, None) == E   # > 2^34 elements
+    assert L.dp_add_noise(FAKE, 4, 4, 0.0, 0, 0, 0, None) == _lib.DP_OK      # std 0: nothing to do
+    assert L.dp_projection_matrix(None, _lib.DP_BF16, 16, 8, 0, 0, None) == E
+    assert L.dp_projection_matrix(FAKE, _lib.DP_BF16, 16, 12, 0, 0, None) == E
+    assert L.dp_projection_matrix(FAKE, 5, 16, 8, 0, 0, None) == E
+    assert L.dp_per_sample_norms(FAKE, FAKE, None, 0, _lib.DP_BF16, 2, 4, 16, 16, 0, None, FAKE,
+                                 1 << 30, None) == E                          # norms is null
+    assert L.dp_per_sample_norms(FAKE, FAKE, None, 8, _lib.DP_BF16, 2, 4, 16, 16, 0, FAKE, FAKE,
+                                 1 << 30, None) == E                          # r without P
+    assert L.dp_clip_accumulate(FAKE, FAKE, None, 0, _lib.DP_BF16, 2, 4, 16, 16, FAKE, 0.0, FAKE,
+                                FAKE, 1 << 30, None) == E                     # C = 0
+    assert L.dp_clip_accumulate(FAKE, FAKE, None, 0, _lib.DP_BF16, 2, 4, 16, 16, None, 1.0, FAKE,
+                                FAKE, 1 << 30, None) == E                     # norms null
+    assert L.dp_workspace_status(None, None) == E
+
+
+def test_binding_raises_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(_lib, "_lib", None)
+    monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        _lib.lib()
+
+
+def test_philox_blocks_rejects_on_host(L):
+    E = _lib.DP_ERR_INVALID_ARG
+    assert L.dp_philox_blocks(None, 4, 0, 0, 0, 0, None) == E
+    assert L.dp_philox_blocks(ODD, 4, 0, 0, 0, 0, None) == E
+    assert L.dp_philox_blocks(FAKE, 0, 0, 0, 0, 0, None) == E
+    assert L.dp_philox_blocks(FAKE, (1 << 32) + 1, 0, 0, 0, 0, None) == E
