@@ -33,8 +33,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
-    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="llama7b_block")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
@@ -77,6 +77,11 @@ def workload_model(w):
     return flops, byts, x_shared_bytes, per_linear
 
 
+def reduce_bytes(w):
+    """Bytes of the clipped-sum reduce over stored per-sample tiles: B bf16 reads + one fp32 write."""
+    return sum(w.B * l.d_in * (w.r or l.d_out) * 2.0 + l.d_in * (w.r or l.d_out) * 4.0 for l in w.linears)
+
+
 def ghost_flops(w):
     """Executed flops of the ghost-norm Gram tiles (upper-triangular 128-token tile pairs)."""
     tt = math.ceil(w.T / 128)
@@ -85,7 +90,7 @@ def ghost_flops(w):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms during the timed region."""
+    """nvidia-smi clocks and throttle reasons sampled every 100 ms during the timed region."""
 
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
@@ -106,7 +111,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", self.target, f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
@@ -223,7 +228,7 @@ def run_ours(args, w, rank, world):
     dY = {k: v.to(dev) for k, v in data["dY"].items()}
     r = w.r
     ws_bytes = max(_lib.workspace_size(w.B, w.T, l.d_in, l.d_out, r,
-                                       _lib.DP_BF16 if w.dtype == "bf16" else _lib.DP_F32)
+                                       _lib.DP_BF16 if w.dtype == "bf16" else _lib.DP_F32, args.method)
                    for l in w.linears)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     G = {l.name: torch.empty(l.d_in, r or l.d_out, dtype=torch.float32, device=dev) for l in w.linears}
@@ -294,16 +299,23 @@ def run_ours(args, w, rank, world):
             work, unit, bound = flops * args.steps, "TFLOP/s", "tensor"
         elif dominant == "umma_ghost_norm":
             work, unit, bound = ghost_flops(w) * args.steps, "TFLOP/s", "tensor"
-        elif dominant == "umma_explicit_norm":
+        elif dominant in ("umma_explicit_norm", "umma_explicit_store"):
             work, unit, bound = flops * args.steps, "TFLOP/s", "tensor"
+        elif dominant == "clip_reduce":
+            work, unit, bound = reduce_bytes(w) * args.steps, "GB/s", "hbm"
         else:
             work, unit, bound = None, None, None
         if work is not None:
-            achieved = work / (d_ms / 1e3) / 1e12
-            peak = pk["bf16_tflops_sustained"]
+            if unit == "GB/s":
+                achieved = work / (d_ms / 1e3) / 1e9
+                peak = pk["hbm_gbs"]
+            else:
+                achieved = work / (d_ms / 1e3) / 1e12
+                peak = pk["bf16_tflops_sustained"]
             roofline = {"bound": bound, "kernel": dominant, "achieved": achieved, "peak": peak,
                         "unit": unit, "frac": achieved / peak, "traffic": None,
-                        "peak_kind": f"{pk_kind} sustained bf16 (kernel timed inside a long step)",
+                        "peak_kind": (f"{pk_kind} HBM copy bandwidth" if unit == "GB/s" else
+                                      f"{pk_kind} sustained bf16 (kernel timed inside a long step)"),
                         "launches": d_n // args.steps, "avg_launch_ms": d_ms / d_n,
                         "share_of_step": d_ms / (ms * args.steps)}
     line = {

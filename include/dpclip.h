@@ -73,14 +73,31 @@ typedef enum { DP_F32 = 0, DP_BF16 = 1 } dp_dtype;
  *              FlashDP Abstract names (GhostClip).
  *   EXPLICIT : n_i^2 = sum of squares of the tiles of G_i = X_i^T dY_i, formed on chip and
  *              never stored.
- *   AUTO     : GHOST when T (d_in + d_out) < 2 d_in d_out, else EXPLICIT.  With projection,
- *              d_out is replaced by r in this rule.  fp32 inputs always use EXPLICIT. */
-typedef enum { DP_NORM_AUTO = 0, DP_NORM_GHOST = 1, DP_NORM_EXPLICIT = 2 } dp_norm_method;
+ *   ONCE     : EXPLICIT, and each tile of G_i is also kept in the workspace in bf16.  The
+ *              clipped sum is then sum_i c_i G_i over those stored tiles, not a second
+ *              contraction, so each per-sample gradient is formed exactly once (FlashDP
+ *              Abstract: "calculating gradients only once").  It needs B*d_in*ne bf16 of
+ *              extra workspace, where ne = d_out, or r with projection.  bf16 only.
+ *   AUTO     : the cheapest of the three by a roofline cost model: flops at 1.4e15/s and
+ *              bytes at 6.5e12/s (ghost: B ceil(T/128)(ceil(T/128)+1)/2 128x128 Gram tile
+ *              pairs plus one scaling pass; explicit: twice the contraction; once: the
+ *              contraction plus the stored tiles read back).  fp32 inputs always use
+ *              EXPLICIT. */
+typedef enum {
+    DP_NORM_AUTO = 0,
+    DP_NORM_GHOST = 1,
+    DP_NORM_EXPLICIT = 2,
+    DP_NORM_ONCE = 3
+} dp_norm_method;
 
-/* Bytes of workspace needed by every call below for these shapes.  r = 0 means unprojected.
- * Returns 0 when the shape is invalid.  The workspace must be 256-byte aligned (any
- * cudaMalloc or torch allocation is). */
+/* Bytes of workspace needed by every call below for these shapes when the norm method is
+ * DP_NORM_AUTO.  r = 0 means unprojected.  Returns 0 when the shape is invalid.  The workspace
+ * must be 256-byte aligned (any cudaMalloc or torch allocation is). */
 size_t dp_workspace_size(int B, int T, int d_in, int d_out, int r, dp_dtype dt);
+
+/* The same for an explicit norm method (DP_NORM_ONCE needs the most). */
+size_t dp_workspace_size_for(int B, int T, int d_in, int d_out, int r, dp_dtype dt,
+                             dp_norm_method method);
 
 /* Per-sample gradient norms n_i = ||X_i^T dY_i||_F, or ||X_i^T dY_i P||_F when P != NULL.
  * (FlashDP Abstract: per-sample gradient clipping needs each sample's gradient; DP-GRAPE
@@ -150,8 +167,8 @@ dp_status dp_philox_blocks(unsigned* out, unsigned long long nblocks, unsigned l
  * every call that takes a workspace. */
 dp_status dp_workspace_status(const void* workspace, void* stream);
 
-/* Norm method that DP_NORM_AUTO picks for these shapes (DP_NORM_GHOST or DP_NORM_EXPLICIT). */
-dp_norm_method dp_auto_norm_method(int T, int d_in, int d_out, int r, dp_dtype dt);
+/* Norm method that DP_NORM_AUTO picks for these shapes (GHOST, EXPLICIT or ONCE). */
+dp_norm_method dp_auto_norm_method(int B, int T, int d_in, int d_out, int r, dp_dtype dt);
 
 /* Launch accounting, for measurement.  dp_kernel_launches() is the number of kernels this
  * library has launched in this process.  Once dp_profiling_enable(1) is called, every later

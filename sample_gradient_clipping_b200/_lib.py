@@ -15,14 +15,17 @@ LIB_PATH = os.path.join(PKG, "libdpclip.so")
 
 DP_OK, DP_ERR_INVALID_ARG, DP_ERR_UNSUPPORTED, DP_ERR_WORKSPACE, DP_ERR_CUDA, DP_ERR_TIMEOUT = range(6)
 DP_F32, DP_BF16 = 0, 1
-DP_NORM_AUTO, DP_NORM_GHOST, DP_NORM_EXPLICIT = 0, 1, 2
-METHODS = {"auto": DP_NORM_AUTO, "ghost": DP_NORM_GHOST, "explicit": DP_NORM_EXPLICIT}
+DP_NORM_AUTO, DP_NORM_GHOST, DP_NORM_EXPLICIT, DP_NORM_ONCE = 0, 1, 2, 3
+METHODS = {"auto": DP_NORM_AUTO, "ghost": DP_NORM_GHOST, "explicit": DP_NORM_EXPLICIT,
+           "once": DP_NORM_ONCE}
+METHOD_NAMES = {v: k for k, v in METHODS.items()}
 
 _c_void_p, _c_int, _c_float = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
 _c_size_t, _c_ll, _c_ull, _c_uint = ctypes.c_size_t, ctypes.c_longlong, ctypes.c_ulonglong, ctypes.c_uint
 
 SIGNATURES = {
     "dp_workspace_size": (_c_size_t, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_int]),
+    "dp_workspace_size_for": (_c_size_t, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int]),
     "dp_per_sample_norms": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_int, _c_int,
                                      _c_int, _c_int, _c_int, _c_void_p, _c_void_p, _c_size_t, _c_void_p]),
     "dp_clip_accumulate": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_int, _c_int,
@@ -35,7 +38,7 @@ SIGNATURES = {
                                 _c_void_p, _c_void_p, _c_void_p, _c_size_t, _c_void_p]),
     "dp_workspace_status": (_c_int, [_c_void_p, _c_void_p]),
     "dp_philox_blocks": (_c_int, [_c_void_p, _c_ull, _c_ull, _c_ull, _c_uint, _c_uint, _c_void_p]),
-    "dp_auto_norm_method": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_int]),
+    "dp_auto_norm_method": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_int]),
     "dp_status_string": (ctypes.c_char_p, [_c_int]),
     "dp_last_cuda_error": (ctypes.c_char_p, []),
     "dp_profiling_enable": (_c_int, [_c_int]),
@@ -112,15 +115,15 @@ def _bt_dims(X, dY):
     return int(X.shape[0]), int(X.shape[1]), int(X.shape[2]), int(dY.shape[2])
 
 
-def workspace_size(B, T, d_in, d_out, r=0, dtype_code=DP_BF16):
-    return int(lib().dp_workspace_size(B, T, d_in, d_out, r, dtype_code))
+def workspace_size(B, T, d_in, d_out, r=0, dtype_code=DP_BF16, method="auto"):
+    return int(lib().dp_workspace_size_for(B, T, d_in, d_out, r, dtype_code, METHODS[method]))
 
 
-def _workspace(X, dY, r, workspace):
+def _workspace(X, dY, r, workspace, method="auto"):
     import torch
 
     B, T, d_in, d_out = _bt_dims(X, dY)
-    need = workspace_size(B, T, d_in, d_out, r, _dtype_code(X))
+    need = workspace_size(B, T, d_in, d_out, r, _dtype_code(X), method)
     if need == 0:
         raise DPError(DP_ERR_INVALID_ARG, "workspace size")
     if workspace is None:
@@ -181,7 +184,7 @@ def dp_linear_step(X, dY, C, sigma, seed, step, layer_id, P=None, r=0, method="a
     B, T, d_in, d_out = _bt_dims(X, dY)
     if P is not None:
         r = int(P.shape[1])
-    ws = _workspace(X, dY, r, workspace)
+    ws = _workspace(X, dY, r, workspace, method)
     width = r if r else d_out
     if G_out is None:
         G_out = torch.empty(d_in, width, dtype=torch.float32, device=X.device)
@@ -211,9 +214,8 @@ def dp_workspace_status(workspace, stream=None):
     return lib().dp_workspace_status(_ptr(workspace), _stream(stream))
 
 
-def auto_norm_method(T, d_in, d_out, r=0, dtype_code=DP_BF16):
-    return {DP_NORM_GHOST: "ghost", DP_NORM_EXPLICIT: "explicit"}[
-        lib().dp_auto_norm_method(T, d_in, d_out, r, dtype_code)]
+def auto_norm_method(B, T, d_in, d_out, r=0, dtype_code=DP_BF16):
+    return METHOD_NAMES[lib().dp_auto_norm_method(B, T, d_in, d_out, r, dtype_code)]
 
 
 def kernel_launches():

@@ -16,6 +16,7 @@
 #include "rng.cuh"
 #include "simt.cuh"
 #include "umma_gemm.cuh"
+#include "umma_gemm_2sm.cuh"
 
 using namespace dpclip;
 
@@ -78,10 +79,23 @@ bool valid_shape(const Shape& s) {
 }
 
 struct WsLayout {
-  size_t status = 0, norm2 = 0, c = 0, scaled = 0, z = 0, p = 0, total = 0;
+  size_t status = 0, norm2 = 0, c = 0, partials = 0, scaled = 0, z = 0, p = 0, gs = 0, total = 0;
+  int partial_stride = 0;  // floats per sample
 };
 
-WsLayout ws_layout(const Shape& s) {
+// Per-warp norm partial slots per sample: 4 per unit of the explicit (128-wide tiles at most)
+// or ghost (upper-triangular 128-token pairs) norm kernel, whichever has more units.
+int partial_slots(const Shape& s) {
+  const long long expl = 4ll * ((s.m + 127) / 128) * ((s.ne() + 127) / 128);
+  const long long pair = 8ll * ((s.m + 255) / 256) * ((s.ne() + 255) / 256);  // two-SM tiles
+  const long long tt = (s.T + 127) / 128;
+  const long long ghost = 4 * tt * (tt + 1) / 2;
+  long long most = expl > ghost ? expl : ghost;
+  if (pair > most) most = pair;
+  return static_cast<int>(most);
+}
+
+WsLayout ws_layout(const Shape& s, dp_norm_method method) {
   WsLayout L;
   size_t off = 256;  // status word(s)
   L.norm2 = off;
@@ -89,6 +103,11 @@ WsLayout ws_layout(const Shape& s) {
   L.c = off;
   off += align256(static_cast<size_t>(s.B) * 4);
   const size_t e = (s.dt == DP_BF16) ? 2 : 4;
+  if (s.dt == DP_BF16) {
+    L.partial_stride = partial_slots(s);
+    L.partials = off;
+    off += align256(static_cast<size_t>(s.B) * L.partial_stride * 4);
+  }
   if (s.dt == DP_BF16) {
     L.scaled = off;
     off += align256(static_cast<size_t>(s.N()) * static_cast<size_t>(s.m < s.ne() ? s.m : s.ne()) * 2);
@@ -99,15 +118,37 @@ WsLayout ws_layout(const Shape& s) {
     L.p = off;
     off += align256(static_cast<size_t>(s.n) * s.r * e);
   }
+  if (method == DP_NORM_ONCE && s.dt == DP_BF16) {
+    L.gs = off;  // per-sample gradient tiles, bf16 [B][d_in][ne]
+    off += align256(static_cast<size_t>(s.B) * s.m * s.ne() * 2);
+  }
   L.total = off;
   return L;
 }
 
+// Roofline cost model of one step for each norm method (seconds at the rates below).
+constexpr double kModelFlops = 1.4e15;  // bf16 tensor flop/s
+constexpr double kModelBytes = 6.5e12;  // HBM byte/s
+
+double model_cost(const Shape& s, dp_norm_method m) {
+  const double N = static_cast<double>(s.N()), d = s.m, ne = s.ne(), B = s.B;
+  const double contraction = 2.0 * N * d * ne / kModelFlops;
+  const double scale_pass = N * (d < ne ? d : ne) * 4.0 / kModelBytes;
+  if (m == DP_NORM_GHOST) {
+    const double tt = std::ceil(s.T / 128.0);
+    return B * tt * (tt + 1) / 2 * 2.0 * 128 * 128 * (d + ne) / kModelFlops + scale_pass + contraction;
+  }
+  if (m == DP_NORM_EXPLICIT) return 2.0 * contraction + scale_pass;
+  const double store = B * d * ne * 2.0 / kModelBytes;  // written while the MMAs run
+  return (contraction > store ? contraction : store) + (B * d * ne * 2.0 + d * ne * 4.0) / kModelBytes;
+}
+
 dp_norm_method auto_method(const Shape& s) {
   if (s.dt == DP_F32) return DP_NORM_EXPLICIT;
-  const double ghost = static_cast<double>(s.T) * (static_cast<double>(s.m) + s.ne());
-  const double expl = 2.0 * static_cast<double>(s.m) * s.ne();
-  return ghost < expl ? DP_NORM_GHOST : DP_NORM_EXPLICIT;
+  dp_norm_method best = DP_NORM_GHOST;
+  for (dp_norm_method m : {DP_NORM_EXPLICIT, DP_NORM_ONCE})
+    if (model_cost(s, m) < model_cost(s, best)) best = m;
+  return best;
 }
 
 // ---------------------------------------------------------------- tensor maps
@@ -164,6 +205,26 @@ dp_status map_3d(CUtensorMap* m, const void* base, int B, int T, int cols, uint3
 }
 
 // ---------------------------------------------------------------- engine launches
+// Two-SM launch: clusters of 2 CTAs (compile-time cluster dims), one pair per 2 SMs.
+template <class Cfg>
+dp_status launch_umma_pair(const UmmaParams& p, cudaStream_t stream) {
+  static bool configured[64] = {false};
+  int dev = 0;
+  DP_CUDA(cudaGetDevice(&dev));
+  if (dev >= 0 && dev < 64 && !configured[dev]) {
+    DP_CUDA(cudaFuncSetAttribute(umma_pair_kernel<Cfg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Cfg::SMEM_BYTES));
+    configured[dev] = true;
+  }
+  if (p.num_units <= 0) return DP_OK;
+  const int pairs_avail = sm_count() / 2;
+  const int pairs = p.num_units < pairs_avail ? p.num_units : pairs_avail;
+  LaunchScope scope(Cfg::EPI == kEpiExplicitStore ? kKindExplicitStore : kKindExplicitNorm, stream);
+  umma_pair_kernel<Cfg><<<2 * pairs, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(p);
+  DP_CHECK_LAUNCH("umma_pair_kernel");
+  return DP_OK;
+}
+
 template <class Cfg>
 dp_status launch_umma(const UmmaParams& p, cudaStream_t stream) {
   static bool configured[64] = {false};
@@ -176,10 +237,11 @@ dp_status launch_umma(const UmmaParams& p, cudaStream_t stream) {
   }
   if (p.num_units <= 0) return DP_OK;
   const int grid = p.num_units < sm_count() ? p.num_units : sm_count();
-  constexpr int kind = Cfg::EPI == kEpiClipSum        ? kKindClipSum
-                       : Cfg::EPI == kEpiExplicitNorm ? kKindExplicitNorm
-                       : Cfg::EPI == kEpiGhostNorm    ? kKindGhostNorm
-                                                      : kKindProject;
+  constexpr int kind = Cfg::EPI == kEpiClipSum         ? kKindClipSum
+                       : Cfg::EPI == kEpiExplicitNorm  ? kKindExplicitNorm
+                       : Cfg::EPI == kEpiExplicitStore ? kKindExplicitStore
+                       : Cfg::EPI == kEpiGhostNorm     ? kKindGhostNorm
+                                                       : kKindProject;
   LaunchScope scope(kind, stream);
   umma_kernel<Cfg><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(p);
   DP_CHECK_LAUNCH("umma_kernel");
@@ -199,11 +261,15 @@ int stream_grid(unsigned long long work_items, int threads) {
   return static_cast<int>(blocks < cap ? (blocks > 0 ? blocks : 1) : cap);
 }
 
-// norm2[i] += ||X_i^T Z_i||^2 (bf16 operands; Z is dY or the projected dY, ne columns)
+// Per-warp partials of ||X_i^T Z_i||^2 (bf16 operands; Z is dY or the projected dY, ne
+// columns) into `partials` ([B][stride]); `count` receives the slots used per sample.  With
+// `store`, the explicit tiles of every G_i are also written there in bf16 ([B][d_in][ne]).
 dp_status bf16_norms(const Shape& s, const void* X, const void* Z, dp_norm_method method,
-                     float* norm2, uint32_t* status, cudaStream_t stream) {
+                     float* partials, int stride, int* count, uint32_t* status, cudaStream_t stream,
+                     __nv_bfloat16* store = nullptr) {
   UmmaParams p = base_params(status);
-  p.norm2 = norm2;
+  p.partials = partials;
+  p.partial_stride = stride;
   const int ne = s.ne();
   if (method == DP_NORM_GHOST) {
     using Cfg = UmmaConfig<128, kEpiGhostNorm>;
@@ -215,6 +281,7 @@ dp_status bf16_norms(const Shape& s, const void* X, const void* Z, dp_norm_metho
     p.t_tiles = ceil_div(s.T, 128);
     p.pairs_per_sample = p.t_tiles * (p.t_tiles + 1) / 2;
     p.num_units = s.B * p.pairs_per_sample;
+    *count = 4 * p.pairs_per_sample;
     p.k_blocks = ceil_div(s.m, 64);
     p.k_blocks1 = ceil_div(ne, 64);
     return launch_umma<Cfg>(p, stream);
@@ -223,18 +290,33 @@ dp_status bf16_norms(const Shape& s, const void* X, const void* Z, dp_norm_metho
   if ((st = map_3d(&p.tmA0, X, s.B, s.T, s.m, 64)) != DP_OK) return st;
   if ((st = map_3d(&p.tmB0, Z, s.B, s.T, ne, 64)) != DP_OK) return st;
   p.k_blocks = ceil_div(s.T, 64);
-  p.m_tiles = ceil_div(s.m, 128);
-  if (ne <= 128) {
-    using Cfg = UmmaConfig<128, kEpiExplicitNorm>;
-    p.n_tiles = ceil_div(ne, 128);
+  p.out_rows = s.m;
+  p.out_cols = ne;
+  p.out_bf16 = store;
+  if (s.m >= 256 && ne >= 256) {
+    // 256 x 256 tiles on SM pairs: half the operand traffic per SM of a 128 x 256 tile.
+    p.m_tiles = ceil_div(s.m, 256);
+    p.n_tiles = ceil_div(ne, 256);
     p.num_units = s.B * p.m_tiles * p.n_tiles;
-    return launch_umma<Cfg>(p, stream);
+    *count = 8 * p.m_tiles * p.n_tiles;
+    if (store) return launch_umma_pair<Umma2Config<kEpiExplicitStore>>(p, stream);
+    return launch_umma_pair<Umma2Config<kEpiExplicitNorm>>(p, stream);
   }
-  using Cfg = UmmaConfig<256, kEpiExplicitNorm>;
-  p.n_tiles = ceil_div(ne, 256);
+  p.m_tiles = ceil_div(s.m, 128);
+  const int bn = ne <= 128 ? 128 : 256;
+  p.n_tiles = ceil_div(ne, bn);
   p.num_units = s.B * p.m_tiles * p.n_tiles;
-  return launch_umma<Cfg>(p, stream);
+  *count = 4 * p.m_tiles * p.n_tiles;
+  if (store) {
+    if (bn == 128) return launch_umma<UmmaConfig<128, kEpiExplicitStore>>(p, stream);
+    return launch_umma<UmmaConfig<256, kEpiExplicitStore>>(p, stream);
+  }
+  if (bn == 128) return launch_umma<UmmaConfig<128, kEpiExplicitNorm>>(p, stream);
+  return launch_umma<UmmaConfig<256, kEpiExplicitNorm>>(p, stream);
 }
+
+dp_status launch_noise(float* G, unsigned long long total, double std_dev, unsigned long long seed,
+                       unsigned long long step, unsigned layer_id, cudaStream_t stream);
 
 // out (+)= A^T Bm over all N rows (A: [N, m], Bm: [N, ne], both bf16, one already scaled by
 // c_i), plus noise when noise_std != 0.  `accumulate` = 0 overwrites out.
@@ -272,14 +354,29 @@ dp_status bf16_clipsum(const Shape& s, const void* A, const void* Bm, float* out
   } else {
     p.out_mode = kOutStore;
   }
-  p.noise_std = noise_std;
+  // With split K the partial sums land by atomics; the noise is then added once, after the
+  // sum is complete, so that it is rounded once as in the unsplit epilogue.
+  const bool fused_noise = (splits == 1);
+  p.noise_std = fused_noise ? noise_std : 0.0;
   const PhiloxKey key = philox_key_from_seed(seed);
   p.key0 = key.k0;
   p.key1 = key.k1;
   p.layer_id = layer_id;
   p.step_lo = static_cast<uint32_t>(step & 0xFFFFFFFFull);
-  if (BN == 128) return launch_umma<UmmaConfig<128, kEpiClipSum>>(p, stream);
-  return launch_umma<UmmaConfig<256, kEpiClipSum>>(p, stream);
+  dp_status st2 = (BN == 128) ? launch_umma<UmmaConfig<128, kEpiClipSum>>(p, stream)
+                              : launch_umma<UmmaConfig<256, kEpiClipSum>>(p, stream);
+  if (st2 != DP_OK || fused_noise || noise_std == 0.0) return st2;
+  return launch_noise(out, static_cast<unsigned long long>(s.m) * ne, noise_std, seed, step, layer_id,
+                      stream);
+}
+
+dp_status launch_noise(float* G, unsigned long long total, double std_dev, unsigned long long seed,
+                       unsigned long long step, unsigned layer_id, cudaStream_t stream) {
+  LaunchScope scope(kKindNoise, stream);
+  noise_add_kernel<<<stream_grid((total + 3) / 4, 256), 256, 0, stream>>>(
+      G, total, std_dev, philox_key_from_seed(seed), layer_id, static_cast<uint32_t>(step & 0xFFFFFFFFull));
+  DP_CHECK_LAUNCH("noise_add_kernel");
+  return DP_OK;
 }
 
 // Z[N, r] = dY[N, n] P[n, r], bf16 out.
@@ -330,11 +427,53 @@ dp_status launch_scale(const void* in, void* out, long long rows, int cols, int 
   return DP_OK;
 }
 
+dp_status launch_norm_partials(const float* partials, int stride, int count, int B, float C,
+                               float* norm2, float* norms_out, float* c_out, cudaStream_t stream) {
+  LaunchScope scope(kKindFinalize, stream);
+  reduce_norm_partials_kernel<<<ceil_div(B, 8), 256, 0, stream>>>(partials, stride, count, B, C, norm2,
+                                                                   norms_out, c_out);
+  DP_CHECK_LAUNCH("reduce_norm_partials_kernel");
+  return DP_OK;
+}
+
 dp_status launch_finalize(NormSource src, int B, float C, float* norms_out, float* c_out,
                           cudaStream_t stream) {
   LaunchScope scope(kKindFinalize, stream);
   finalize_norms_kernel<<<ceil_div(B, 256), 256, 0, stream>>>(src, B, C, norms_out, c_out);
   DP_CHECK_LAUNCH("finalize_norms_kernel");
+  return DP_OK;
+}
+
+template <int BU>
+void reduce_kernel_launch(int grid, size_t smem, cudaStream_t stream, const __nv_bfloat16* gs, int B,
+                          long long mn, NormSource src, float C, float* out, double noise_std,
+                          PhiloxKey key, unsigned layer_id, uint32_t step_lo) {
+  clip_reduce_kernel<BU><<<grid, 256, smem, stream>>>(gs, B, mn, src, C, out, noise_std, key, layer_id,
+                                                      step_lo);
+}
+
+dp_status launch_reduce(const __nv_bfloat16* gs, int B, long long mn, NormSource src, float C,
+                        float* out, double noise_std, unsigned long long seed, unsigned long long step,
+                        unsigned layer_id, cudaStream_t stream) {
+  const int cached = B < kReduceCachedSamples ? B : kReduceCachedSamples;
+  const int grid = stream_grid(static_cast<unsigned long long>(mn / 8), 256);
+  const size_t smem = cached * sizeof(float);
+  const PhiloxKey key = philox_key_from_seed(seed);
+  const uint32_t step_lo = static_cast<uint32_t>(step & 0xFFFFFFFFull);
+  LaunchScope scope(kKindReduce, stream);
+  switch (B) {
+    case 1: reduce_kernel_launch<1>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step_lo); break;
+    case 2: reduce_kernel_launch<2>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step_lo); break;
+    case 3: reduce_kernel_launch<3>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step_lo); break;
+    case 4: reduce_kernel_launch<4>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step_lo); break;
+    case 5: reduce_kernel_launch<5>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step_lo); break;
+    case 6: reduce_kernel_launch<6>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step_lo); break;
+    case 7: reduce_kernel_launch<7>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step_lo); break;
+    case 8: reduce_kernel_launch<8>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step_lo); break;
+    default: reduce_kernel_launch<0>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step_lo); break;
+  }
+  static_assert(kReduceUnrolled == 8, "the switch above unrolls up to 8 samples");
+  DP_CHECK_LAUNCH("clip_reduce_kernel");
   return DP_OK;
 }
 
@@ -348,11 +487,12 @@ struct Call {
   float* norm2_f32() const { return reinterpret_cast<float*>(ws + L.norm2); }
   double* norm2_f64() const { return reinterpret_cast<double*>(ws + L.norm2); }
   float* c() const { return reinterpret_cast<float*>(ws + L.c); }
+  float* partials() const { return reinterpret_cast<float*>(ws + L.partials); }
 };
 
 dp_status check_common(const void* X, const void* dY, const void* P, int r, dp_dtype dt, int B,
                        int T, int d_in, int d_out, void* workspace, size_t ws_bytes, bool p_from_seed,
-                       Call* call) {
+                       dp_norm_method method, Call* call) {
   if (!X || !dY || !workspace) return DP_ERR_INVALID_ARG;
   if (!aligned16(X) || !aligned16(dY) || (P && !aligned16(P))) return DP_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return DP_ERR_INVALID_ARG;
@@ -360,7 +500,7 @@ dp_status check_common(const void* X, const void* dY, const void* P, int r, dp_d
   if (!P && r != 0 && !p_from_seed) return DP_ERR_INVALID_ARG;
   call->s = Shape{B, T, d_in, d_out, r, dt};
   if (!valid_shape(call->s)) return DP_ERR_INVALID_ARG;
-  call->L = ws_layout(call->s);
+  call->L = ws_layout(call->s, method == DP_NORM_AUTO ? auto_method(call->s) : method);
   if (ws_bytes < call->L.total) return DP_ERR_WORKSPACE;
   call->ws = static_cast<uint8_t*>(workspace);
   return DP_OK;
@@ -395,7 +535,10 @@ dp_status clip_space_operand(Call& c, const void* dY, const void* P, bool p_from
   return DP_OK;
 }
 
-dp_status norms_into_ws(Call& c, const void* X, const void* Z, dp_norm_method method) {
+// Per-sample squared norms into the workspace's norm2[B]; for bf16 also norms_out and c
+// when given (the fp32 path writes those in launch_finalize).
+dp_status norms_into_ws(Call& c, const void* X, const void* Z, dp_norm_method method, float C,
+                        float* norms_out, bool store_tiles = false) {
   if (c.s.dt == DP_F32) {
     dim3 grid(ceil_div(c.s.ne(), kF32Tile), ceil_div(c.s.m, kF32Tile), c.s.B);
     LaunchScope scope(kKindF32Norm, c.stream);
@@ -404,7 +547,12 @@ dp_status norms_into_ws(Call& c, const void* X, const void* Z, dp_norm_method me
     DP_CHECK_LAUNCH("f32_norm_kernel");
     return DP_OK;
   }
-  return bf16_norms(c.s, X, Z, method, c.norm2_f32(), c.status(), c.stream);
+  int count = 0;
+  dp_status st = bf16_norms(c.s, X, Z, method, c.partials(), c.L.partial_stride, &count, c.status(),
+                            c.stream, store_tiles ? reinterpret_cast<__nv_bfloat16*>(c.ws + c.L.gs) : nullptr);
+  if (st != DP_OK) return st;
+  return launch_norm_partials(c.partials(), c.L.partial_stride, count, c.s.B, C, c.norm2_f32(), norms_out,
+                              norms_out ? c.c() : nullptr, c.stream);
 }
 
 NormSource ws_norm_source(const Call& c) {
@@ -447,8 +595,9 @@ dp_status resolve_method(const Shape& s, dp_norm_method method, dp_norm_method* 
     *out = auto_method(s);
     return DP_OK;
   }
-  if (method != DP_NORM_GHOST && method != DP_NORM_EXPLICIT) return DP_ERR_INVALID_ARG;
-  if (s.dt == DP_F32 && method == DP_NORM_GHOST) return DP_ERR_UNSUPPORTED;
+  if (method != DP_NORM_GHOST && method != DP_NORM_EXPLICIT && method != DP_NORM_ONCE)
+    return DP_ERR_INVALID_ARG;
+  if (s.dt == DP_F32 && method != DP_NORM_EXPLICIT) return DP_ERR_UNSUPPORTED;
   *out = method;
   return DP_OK;
 }
@@ -461,28 +610,42 @@ extern "C" {
 size_t dp_workspace_size(int B, int T, int d_in, int d_out, int r, dp_dtype dt) {
   const Shape s{B, T, d_in, d_out, r, dt};
   if (!valid_shape(s)) return 0;
-  return ws_layout(s).total;
+  return ws_layout(s, auto_method(s)).total;
 }
 
-dp_norm_method dp_auto_norm_method(int T, int d_in, int d_out, int r, dp_dtype dt) {
-  return auto_method(Shape{1, T, d_in, d_out, r, dt});
+size_t dp_workspace_size_for(int B, int T, int d_in, int d_out, int r, dp_dtype dt,
+                             dp_norm_method method) {
+  const Shape s{B, T, d_in, d_out, r, dt};
+  if (!valid_shape(s)) return 0;
+  if (method != DP_NORM_AUTO && method != DP_NORM_GHOST && method != DP_NORM_EXPLICIT &&
+      method != DP_NORM_ONCE)
+    return 0;
+  return ws_layout(s, method == DP_NORM_AUTO ? auto_method(s) : method).total;
+}
+
+dp_norm_method dp_auto_norm_method(int B, int T, int d_in, int d_out, int r, dp_dtype dt) {
+  const Shape s{B < 1 ? 1 : B, T, d_in, d_out, r, dt};
+  return auto_method(s);
 }
 
 dp_status dp_per_sample_norms(const void* X, const void* dY, const void* P, int r, dp_dtype dt, int B,
                               int T, int d_in, int d_out, dp_norm_method method, float* norms,
                               void* workspace, size_t ws_bytes, void* stream) {
   Call c;
-  dp_status st = check_common(X, dY, P, r, dt, B, T, d_in, d_out, workspace, ws_bytes, false, &c);
+  dp_status st = check_common(X, dY, P, r, dt, B, T, d_in, d_out, workspace, ws_bytes, false,
+                              DP_NORM_GHOST, &c);
   if (st != DP_OK) return st;
   if (!norms) return DP_ERR_INVALID_ARG;
   dp_norm_method m;
   if ((st = resolve_method(c.s, method, &m)) != DP_OK) return st;
+  if (m == DP_NORM_ONCE) m = DP_NORM_EXPLICIT;  // nothing to reuse: the norms are the result
   if ((st = get_encoder()) != DP_OK && dt == DP_BF16) return st;
   c.stream = static_cast<cudaStream_t>(stream);
   DP_CUDA(cudaMemsetAsync(c.ws, 0, c.L.c, c.stream));  // status word + norm accumulators
   const void* Z;
   if ((st = clip_space_operand(c, dY, P, false, 0, 0, &Z)) != DP_OK) return st;
-  if ((st = norms_into_ws(c, X, Z, m)) != DP_OK) return st;
+  if ((st = norms_into_ws(c, X, Z, m, INFINITY, dt == DP_BF16 ? norms : nullptr)) != DP_OK) return st;
+  if (dt == DP_BF16) return DP_OK;
   return launch_finalize(ws_norm_source(c), B, INFINITY, norms, nullptr, c.stream);
 }
 
@@ -490,7 +653,8 @@ dp_status dp_clip_accumulate(const void* X, const void* dY, const void* P, int r
                              int T, int d_in, int d_out, const float* norms, float C, float* G_sum,
                              void* workspace, size_t ws_bytes, void* stream) {
   Call c;
-  dp_status st = check_common(X, dY, P, r, dt, B, T, d_in, d_out, workspace, ws_bytes, false, &c);
+  dp_status st = check_common(X, dY, P, r, dt, B, T, d_in, d_out, workspace, ws_bytes, false,
+                              DP_NORM_GHOST, &c);
   if (st != DP_OK) return st;
   if (!norms || !G_sum || !aligned16(G_sum)) return DP_ERR_INVALID_ARG;
   if (!(C > 0.0f)) return DP_ERR_INVALID_ARG;  // also rejects NaN
@@ -510,12 +674,8 @@ dp_status dp_add_noise(float* G, long long rows, long long cols, float std, unsi
   if (rows > (1ll << 34) / cols) return DP_ERR_INVALID_ARG;
   const unsigned long long total = static_cast<unsigned long long>(rows) * static_cast<unsigned long long>(cols);
   if (std == 0.0f) return DP_OK;
-  const PhiloxKey key = philox_key_from_seed(seed);
-  LaunchScope scope(kKindNoise, static_cast<cudaStream_t>(stream));
-  noise_add_kernel<<<stream_grid((total + 3) / 4, 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      G, total, static_cast<double>(std), key, layer_id, static_cast<uint32_t>(step & 0xFFFFFFFFull));
-  DP_CHECK_LAUNCH("noise_add_kernel");
-  return DP_OK;
+  return launch_noise(G, total, static_cast<double>(std), seed, step, layer_id,
+                      static_cast<cudaStream_t>(stream));
 }
 
 dp_status dp_projection_matrix(void* P, dp_dtype dt, int d_out, int r, unsigned long long seed,
@@ -532,7 +692,9 @@ dp_status dp_linear_step(const void* X, const void* dY, const void* P, int r, dp
                          unsigned long long step, unsigned layer_id, dp_norm_method method,
                          float* norms_out, float* G_out, void* workspace, size_t ws_bytes, void* stream) {
   Call c;
-  dp_status st = check_common(X, dY, P, r, dt, B, T, d_in, d_out, workspace, ws_bytes, true, &c);
+  if (method < DP_NORM_AUTO || method > DP_NORM_ONCE) return DP_ERR_INVALID_ARG;
+  dp_status st = check_common(X, dY, P, r, dt, B, T, d_in, d_out, workspace, ws_bytes, true,
+                              method, &c);
   if (st != DP_OK) return st;
   if (!G_out || !aligned16(G_out)) return DP_ERR_INVALID_ARG;
   if (!(C > 0.0f) || !(sigma >= 0.0f) || std::isinf(sigma)) return DP_ERR_INVALID_ARG;
@@ -544,11 +706,19 @@ dp_status dp_linear_step(const void* X, const void* dY, const void* P, int r, dp
   DP_CUDA(cudaMemsetAsync(c.ws, 0, c.L.c, c.stream));  // status word + norm accumulators
   const void* Z;
   if ((st = clip_space_operand(c, dY, P, true, seed, layer_id, &Z)) != DP_OK) return st;
-  if ((st = norms_into_ws(c, X, Z, m)) != DP_OK) return st;
-  const NormSource src = ws_norm_source(c);
-  if (norms_out && (st = launch_finalize(src, B, C, norms_out, c.c(), c.stream)) != DP_OK) return st;
+  const bool once = (m == DP_NORM_ONCE);
   // sigma = 0 means no noise, also for C = +inf (where sigma * C would be NaN).
   const double noise_std = (sigma == 0.0f) ? 0.0 : static_cast<double>(sigma) * static_cast<double>(C);
+  const long long mn = static_cast<long long>(c.s.m) * c.s.ne();
+  if ((st = norms_into_ws(c, X, Z, once ? DP_NORM_EXPLICIT : m, C, dt == DP_BF16 ? norms_out : nullptr,
+                          once)) != DP_OK)
+    return st;
+  const NormSource src = ws_norm_source(c);
+  if (dt == DP_F32 && norms_out && (st = launch_finalize(src, B, C, norms_out, c.c(), c.stream)) != DP_OK)
+    return st;
+  if (once)
+    return launch_reduce(reinterpret_cast<const __nv_bfloat16*>(c.ws + c.L.gs), B, mn, src, C, G_out,
+                         noise_std, seed, step, layer_id, c.stream);
   return clipped_sum(c, X, Z, src, C, G_out, 0, noise_std, seed, step, layer_id);
 }
 

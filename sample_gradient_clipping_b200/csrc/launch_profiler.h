@@ -26,6 +26,8 @@ enum KernelKind : int {
   kKindExplicitNorm,  // tcgen05 per-sample G_i tiles, squared on chip
   kKindGhostNorm,     // tcgen05 Gram tiles of X_i and dY_i
   kKindProject,       // tcgen05 Z = dY P
+  kKindExplicitStore, // tcgen05 per-sample G_i tiles, squared on chip and stored in bf16
+  kKindReduce,        // sum_i c_i G_i over the stored tiles + noise
   kNumKinds
 };
 
@@ -33,7 +35,7 @@ inline const char* kernel_kind_name(int k) {
   static const char* names[kNumKinds] = {
       "noise_add",  "projection",   "philox_blocks", "scale_rows_bf16", "finalize_norms",
       "f32_norm",   "f32_clipsum",  "f32_project",   "umma_clipsum",    "umma_explicit_norm",
-      "umma_ghost_norm", "umma_project"};
+      "umma_ghost_norm", "umma_project", "umma_explicit_store", "clip_reduce"};
   return (k >= 0 && k < kNumKinds) ? names[k] : "";
 }
 

@@ -84,6 +84,11 @@ __global__ void projection_kernel(void* __restrict__ P, unsigned long long total
   }
 }
 
+// Clip factors that clip_reduce_kernel keeps in shared memory (the rest are recomputed), and
+// the largest sample count whose loads it unrolls.
+constexpr int kReduceCachedSamples = 4096;
+constexpr int kReduceUnrolled = 8;
+
 // Clip factor of sample i from either squared-norm accumulators or final norms.
 __device__ __forceinline__ float clip_factor(float norm, float C) {
   return (norm <= C) ? 1.0f : C / norm;
@@ -99,6 +104,28 @@ struct NormSource {
     return sqrtf(norm2_f32[i]);
   }
 };
+
+// norm2[i] = the sum of sample i's `count` per-warp partials, in a fixed order and in fp64,
+// so the norms (and the clip factors that follow from them) are reproducible bit for bit.
+// One warp per sample.  Also writes norms_out[i] = n_i and c_out[i] = c_i when given.
+__global__ void reduce_norm_partials_kernel(const float* __restrict__ partials, int stride, int count,
+                                            int B, float C, float* __restrict__ norm2,
+                                            float* __restrict__ norms_out, float* __restrict__ c_out) {
+  const int i = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  if (i >= B) return;
+  double acc = 0.0;
+  for (int k = lane; k < count; k += 32) acc += static_cast<double>(partials[static_cast<long long>(i) * stride + k]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
+  if (lane == 0) {
+    const float n2 = static_cast<float>(acc);
+    norm2[i] = n2;
+    const float n = sqrtf(n2);
+    if (norms_out) norms_out[i] = n;
+    if (c_out) c_out[i] = clip_factor(n, C);
+  }
+}
 
 // norms_out[i] = n_i and c_out[i] = c_i for i < B (either may be null).
 __global__ void finalize_norms_kernel(NormSource src, int B, float C, float* __restrict__ norms_out,
@@ -131,6 +158,79 @@ __global__ void scale_rows_bf16_kernel(const __nv_bfloat16* __restrict__ in,
       o[e] = __floats2bfloat162_rn(c * f.x, c * f.y);
     }
     reinterpret_cast<uint4*>(out)[v] = res;
+  }
+}
+
+// out[e] = fp32(sum_i c_i Gs[i][e] + std * z_e) over the per-sample bf16 gradients that the
+// explicit-store pass left in the workspace: the clipped sum without forming any G_i again.
+//
+// Each thread owns 8 consecutive elements: two Philox blocks and four independent fp64
+// Box-Muller pairs.  The loads of all samples are issued first (for B <= kReduceUnrolled the
+// loop is unrolled), the noise is computed while they are in flight, and then the sum is
+// formed.  This keeps both the fp64 pipe and HBM busy instead of alternating between them.
+template <int BU>  // compile-time sample count, or 0 for a runtime loop
+__global__ void __launch_bounds__(256, 3) clip_reduce_kernel(
+    const __nv_bfloat16* __restrict__ Gs, int B, long long mn, NormSource src, float C,
+    float* __restrict__ out, double noise_std, PhiloxKey key, uint32_t layer_id, uint32_t step_lo) {
+  extern __shared__ float c_smem[];
+  const int cached = B < kReduceCachedSamples ? B : kReduceCachedSamples;
+  for (int i = threadIdx.x; i < cached; i += blockDim.x) c_smem[i] = clip_factor(src.norm(i), C);
+  __syncthreads();
+  const long long nvec = mn / 8;  // 16-byte vectors per sample
+  for (long long v = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; v < nvec;
+       v += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const uint4* g = reinterpret_cast<const uint4*>(Gs) + v;
+    float acc[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) acc[q] = 0.f;
+    double z[8];
+    if constexpr (BU > 0) {
+      uint4 pk[BU > 0 ? BU : 1];
+#pragma unroll
+      for (int i = 0; i < BU; ++i) pk[i] = __ldcs(g + static_cast<long long>(i) * nvec);
+      if (noise_std != 0.0) {
+        normals4(static_cast<uint32_t>(2 * v), layer_id, step_lo, kStreamNoise, key,
+                 *reinterpret_cast<double(*)[4]>(z));
+        normals4(static_cast<uint32_t>(2 * v + 1), layer_id, step_lo, kStreamNoise, key,
+                 *reinterpret_cast<double(*)[4]>(z + 4));
+      }
+#pragma unroll
+      for (int i = 0; i < BU; ++i) {
+        const float c = c_smem[i];
+        const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&pk[i]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(hv[e]);
+          acc[2 * e] = fmaf(c, f.x, acc[2 * e]);
+          acc[2 * e + 1] = fmaf(c, f.y, acc[2 * e + 1]);
+        }
+      }
+    } else {
+      for (int i = 0; i < B; ++i) {
+        const float c = i < cached ? c_smem[i] : clip_factor(src.norm(i), C);
+        const uint4 pk = __ldcs(g + static_cast<long long>(i) * nvec);
+        const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&pk);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(hv[e]);
+          acc[2 * e] = fmaf(c, f.x, acc[2 * e]);
+          acc[2 * e + 1] = fmaf(c, f.y, acc[2 * e + 1]);
+        }
+      }
+      if (noise_std != 0.0) {
+        normals4(static_cast<uint32_t>(2 * v), layer_id, step_lo, kStreamNoise, key,
+                 *reinterpret_cast<double(*)[4]>(z));
+        normals4(static_cast<uint32_t>(2 * v + 1), layer_id, step_lo, kStreamNoise, key,
+                 *reinterpret_cast<double(*)[4]>(z + 4));
+      }
+    }
+    if (noise_std != 0.0) {
+#pragma unroll
+      for (int q = 0; q < 8; ++q) acc[q] = static_cast<float>(static_cast<double>(acc[q]) + noise_std * z[q]);
+    }
+    float4* o = reinterpret_cast<float4*>(out) + 2 * v;
+    o[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    o[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
   }
 }
 

@@ -14,11 +14,16 @@
 //                    MN-major; the clip factor is already folded into one operand), with the
 //                    Philox/Box-Muller noise added in the epilogue before the fp32 store;
 //   kEpiExplicitNorm per (sample, output tile): the tile of G_i = X_i^T dY_i over the
-//                    sample's T tokens, squared and summed on chip into norm2[i];
+//                    sample's T tokens, squared and summed on chip; each epilogue warp writes
+//                    its partial to its own slot, and the slots of a sample are summed later
+//                    in a fixed order (norms reproducible bit for bit);
 //   kEpiGhostNorm    per (sample, upper-triangular pair of 128-token blocks): the X Gram
 //                    tile and the dY Gram tile in two TMEM accumulators; the epilogue sums
 //                    w * Gx * Gy with w = 2 above the diagonal, 1 on it, 0 below;
-//   kEpiStoreBf16    Z = dY P (K-major dY, MN-major P), rounded to bf16.
+//   kEpiStoreBf16    Z = dY P (K-major dY, MN-major P), rounded to bf16;
+//   kEpiExplicitStore as kEpiExplicitNorm, and the tile of G_i is also written to HBM in bf16
+//                    so that the clipped sum reuses it instead of forming G_i again
+//                    (each per-sample gradient is formed once).
 //
 // All waits are bounded (ptx.cuh); a wait that runs out sets the CTA's abort flag, records
 // its site in the status word and the CTA drains and exits.
@@ -30,7 +35,16 @@
 
 namespace dpclip {
 
-enum EpiKind : int { kEpiClipSum = 0, kEpiExplicitNorm = 1, kEpiGhostNorm = 2, kEpiStoreBf16 = 3 };
+enum EpiKind : int {
+  kEpiClipSum = 0,
+  kEpiExplicitNorm = 1,
+  kEpiGhostNorm = 2,
+  kEpiStoreBf16 = 3,
+  kEpiExplicitStore = 4
+};
+
+// K-blocks ahead of the smem ring that the clipped-sum producer asks TMA to pull into L2.
+constexpr int kL2PrefetchDistance = 8;
 
 enum OutMode : int { kOutStore = 0, kOutAtomicAdd = 1, kOutAdd = 2 };
 
@@ -49,7 +63,8 @@ struct alignas(64) UmmaParams {
   __nv_bfloat16* out_bf16;
   double noise_std;           // 0 disables the noise
   uint32_t key0, key1, layer_id, step_lo;
-  float* norm2;               // [B] squared-norm accumulators
+  float* partials;            // [B][partial_stride] per-warp squared-norm partials
+  int partial_stride;         // slots per sample: 4 per unit of that sample
   uint32_t* status;
 };
 
@@ -59,7 +74,8 @@ struct UmmaConfig {
   static constexpr int BN = BN_;
   static constexpr int BK = 64;  // 64 bf16 = 128 bytes: one swizzle atom row
   static constexpr int EPI = EPI_;
-  static constexpr bool A_MN = (EPI == kEpiClipSum || EPI == kEpiExplicitNorm);
+  static constexpr bool PER_SAMPLE = (EPI == kEpiExplicitNorm || EPI == kEpiExplicitStore);
+  static constexpr bool A_MN = (EPI == kEpiClipSum || PER_SAMPLE);
   static constexpr bool B_MN = (EPI != kEpiGhostNorm);
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = BN * BK * 2;
@@ -77,6 +93,7 @@ struct UmmaConfig {
 
 struct Unit {
   int m_blk, n_blk, kb_begin, kb_end, sample, split;
+  int local;  // index of the unit among the units of its sample (norm partial slots)
 };
 
 template <class Cfg>
@@ -90,6 +107,7 @@ __device__ __forceinline__ Unit decode_unit(const UmmaParams& p, int u) {
       r -= p.t_tiles - row;
       ++row;
     }
+    w.local = u % p.pairs_per_sample;
     w.m_blk = row;
     w.n_blk = row + r;
     w.kb_begin = 0;
@@ -100,6 +118,7 @@ __device__ __forceinline__ Unit decode_unit(const UmmaParams& p, int u) {
   const int tiles = p.m_tiles * p.n_tiles;
   int r = u % tiles;
   const int outer = u / tiles;
+  w.local = r;
   // Rasterise in groups of 8 row-tiles so that concurrently running CTAs share operand tiles
   // in L2.
   constexpr int G = 8;
@@ -109,7 +128,7 @@ __device__ __forceinline__ Unit decode_unit(const UmmaParams& p, int u) {
   const int within = r % per_group;
   w.m_blk = first_m + within % gsz;
   w.n_blk = within / gsz;
-  if (Cfg::EPI == kEpiExplicitNorm) {
+  if (Cfg::PER_SAMPLE) {
     w.sample = outer;
     w.split = 0;
     w.kb_begin = 0;
@@ -135,7 +154,7 @@ __device__ __forceinline__ void issue_stage_loads(const UmmaParams& p, const Uni
 #pragma unroll
     for (int h = 0; h < Cfg::BN / 64; ++h)
       tma_load_2d(sB + h * (Cfg::BK * 128), &p.tmB0, bar, w.n_blk * Cfg::BN + 64 * h, k0);
-  } else if (Cfg::EPI == kEpiExplicitNorm) {
+  } else if (Cfg::PER_SAMPLE) {
 #pragma unroll
     for (int h = 0; h < Cfg::BM / 64; ++h)
       tma_load_3d(sA + h * (Cfg::BK * 128), &p.tmA0, bar, w.m_blk * Cfg::BM + 64 * h, k0,
@@ -155,6 +174,18 @@ __device__ __forceinline__ void issue_stage_loads(const UmmaParams& p, const Uni
     for (int h = 0; h < Cfg::BN / 64; ++h)
       tma_load_2d(sB + h * (Cfg::BK * 128), &p.tmB0, bar, w.n_blk * Cfg::BN + 64 * h, k0);
   }
+}
+
+// Clipped sum only: pull the A/B boxes of K-block `kb` into L2 ahead of their smem loads.
+// Every k-slice of the long token dimension is first touched by one CTA and then re-read by
+// the others, so its DRAM latency would otherwise stall the MMA.
+template <class Cfg>
+__device__ __forceinline__ void prefetch_stage_l2(const UmmaParams& p, const Unit& w, int kb) {
+  const int k0 = kb * Cfg::BK;
+#pragma unroll
+  for (int h = 0; h < Cfg::BM / 64; ++h) tma_prefetch_l2_2d(&p.tmA0, w.m_blk * Cfg::BM + 64 * h, k0);
+#pragma unroll
+  for (int h = 0; h < Cfg::BN / 64; ++h) tma_prefetch_l2_2d(&p.tmB0, w.n_blk * Cfg::BN + 64 * h, k0);
 }
 
 template <class Cfg>
@@ -214,18 +245,35 @@ __device__ __forceinline__ void epilogue_unit(const UmmaParams& p, const Unit& w
         }
       }
     }
-  } else if (Cfg::EPI == kEpiExplicitNorm) {
+  } else if (Cfg::PER_SAMPLE) {
+    // Rows and columns past d_in / ne were zero-filled by TMA and add nothing.
     float ss = 0.f;
+    const long long grow = static_cast<long long>(w.m_blk) * Cfg::BM + row;
+    const bool row_ok = grow < p.out_rows;
 #pragma unroll 1
     for (int c0 = 0; c0 < Cfg::BN; c0 += 32) {
       float v[32];
+      __syncwarp();
       tmem_ld32(tacc + c0, v);
       tmem_ld_wait();
 #pragma unroll
       for (int e = 0; e < 32; ++e) ss = fmaf(v[e], v[e], ss);
+      if (Cfg::EPI == kEpiExplicitStore && row_ok) {
+        const long long gcol0 = static_cast<long long>(w.n_blk) * Cfg::BN + c0;
+        __nv_bfloat16* dst = p.out_bf16 + (static_cast<long long>(w.sample) * p.out_rows + grow) * p.out_cols + gcol0;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          if (gcol0 + 8 * q >= p.out_cols) break;  // out_cols is a multiple of 8
+          uint4 pk;
+          __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&pk);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) h[e] = __floats2bfloat162_rn(v[8 * q + 2 * e], v[8 * q + 2 * e + 1]);
+          *reinterpret_cast<uint4*>(dst + 8 * q) = pk;
+        }
+      }
     }
     ss = warp_sum(ss);
-    if (lane == 0) atomicAdd(p.norm2 + w.sample, ss);
+    if (lane == 0) p.partials[static_cast<long long>(w.sample) * p.partial_stride + 4 * w.local + wq] = ss;
   } else if (Cfg::EPI == kEpiGhostNorm) {
     // Rows and columns past T were zero-filled by TMA, so their Gram entries are 0.
     const int t = w.m_blk * Cfg::BM + row;
@@ -245,7 +293,7 @@ __device__ __forceinline__ void epilogue_unit(const UmmaParams& p, const Unit& w
       }
     }
     ss = warp_sum(ss);
-    if (lane == 0) atomicAdd(p.norm2 + w.sample, ss);
+    if (lane == 0) p.partials[static_cast<long long>(w.sample) * p.partial_stride + 4 * w.local + wq] = ss;
   } else {  // kEpiStoreBf16
     const long long grow = static_cast<long long>(w.m_blk) * Cfg::BM + row;
 #pragma unroll 1
@@ -336,6 +384,14 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1) umma_kernel(const __grid_cons
             const uint32_t bar = smem_addr(full + stage);
             mbar_arrive_expect_tx(bar, Cfg::STAGE_BYTES);
             issue_stage_loads<Cfg>(p, w, ph, kb, sA, sA + Cfg::A_BYTES, bar);
+            if (Cfg::EPI == kEpiClipSum) {
+              if (kb == kb_begin) {
+                for (int d = 1; d <= kL2PrefetchDistance && kb + d < kb_end; ++d)
+                  prefetch_stage_l2<Cfg>(p, w, kb + d);
+              } else if (kb + kL2PrefetchDistance < kb_end) {
+                prefetch_stage_l2<Cfg>(p, w, kb + kL2PrefetchDistance);
+              }
+            }
             if (++stage == Cfg::STAGES) {
               stage = 0;
               phase ^= 1u;

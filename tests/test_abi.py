@@ -39,22 +39,30 @@ def test_status_strings(L):
 
 
 def test_workspace_size(L):
+    # AUTO picks "once" here: status + norm2 + c + the per-warp norm partials (4 per 128x128
+    # tile) + the scaled narrower operand (4096 wide) + the bf16 per-sample tiles.
     ws = L.dp_workspace_size(8, 2048, 4096, 11008, 0, _lib.DP_BF16)
-    # status + norm2 + c + the scaled copy of the narrower operand (X here: 4096 wide)
-    assert ws >= 8 * 2048 * 4096 * 2
-    assert ws < 8 * 2048 * 4096 * 2 + 4096
+    scaled, tiles = 8 * 2048 * 4096 * 2, 8 * 4096 * 11008 * 2
+    partials = 8 * 4 * 32 * 86 * 4
+    assert scaled + tiles + partials <= ws < scaled + tiles + partials + 4096
+    ghost = L.dp_workspace_size_for(8, 2048, 4096, 11008, 0, _lib.DP_BF16, _lib.DP_NORM_GHOST)
+    assert scaled + partials <= ghost < scaled + partials + 4096
+    assert L.dp_workspace_size_for(8, 2048, 4096, 11008, 0, _lib.DP_BF16, 9) == 0
     assert L.dp_workspace_size(64, 128, 1024, 1024, 128, _lib.DP_BF16) >= 64 * 128 * 128 * 2 * 2
     assert L.dp_workspace_size(0, 1, 8, 8, 0, _lib.DP_BF16) == 0
     assert L.dp_workspace_size(1, 1, 12, 8, 0, _lib.DP_BF16) == 0     # d_in not a multiple of 8
     assert L.dp_workspace_size(1, 1, 12, 8, 0, _lib.DP_F32) > 0        # fp32 needs multiples of 4
 
 
-def test_auto_method_rule(L):
-    # ghost iff T (d_in + d_out) < 2 d_in d_out; fp32 is always explicit
-    assert _lib.auto_norm_method(2048, 4096, 4096) == "ghost"
-    assert _lib.auto_norm_method(128, 1024, 1024, 128) == "ghost"
-    assert _lib.auto_norm_method(4096, 64, 64) == "explicit"
-    assert _lib.auto_norm_method(16, 64, 32, 0, _lib.DP_F32) == "explicit"
+def test_auto_method_cost_model(L):
+    # Long sequences over wide layers: forming each G_i once beats a second contraction.
+    assert _lib.auto_norm_method(8, 2048, 4096, 4096) == "once"
+    assert _lib.auto_norm_method(4, 2048, 5120, 13824) == "once"
+    # Short sequences: the ghost Grams are nearly free.
+    assert _lib.auto_norm_method(64, 16, 4096, 4096) == "ghost"
+    # Very long sequences over narrow layers: the explicit tiles are cheapest.
+    assert _lib.auto_norm_method(2, 8192, 64, 64) in ("explicit", "once")
+    assert _lib.auto_norm_method(4, 16, 64, 32, 0, _lib.DP_F32) == "explicit"
 
 
 FAKE = 0x10000          # 16-byte aligned, never dereferenced: every case fails on the host
@@ -94,7 +102,9 @@ def _step(L, **kw):
     (dict(r=12), _lib.DP_ERR_INVALID_ARG),
     (dict(method=9), _lib.DP_ERR_INVALID_ARG),
     (dict(dt=_lib.DP_F32, method=_lib.DP_NORM_GHOST), _lib.DP_ERR_UNSUPPORTED),
+    (dict(dt=_lib.DP_F32, method=_lib.DP_NORM_ONCE), _lib.DP_ERR_UNSUPPORTED),
     (dict(ws_bytes=512), _lib.DP_ERR_WORKSPACE),
+    (dict(method=_lib.DP_NORM_ONCE, ws_bytes=1024), _lib.DP_ERR_WORKSPACE),   # needs the tiles
     (dict(B=1 << 16, T=1 << 15), _lib.DP_ERR_INVALID_ARG),   # B*T >= 2^31
 ])
 def test_linear_step_rejects_on_host(L, kw, want):

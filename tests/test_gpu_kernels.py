@@ -95,7 +95,7 @@ def _draw(B, T, m, n, dtype="bf16", seed=21, dy_var=None):
 
 
 @pytest.mark.parametrize("shape", NORM_SHAPES, ids=lambda s: "x".join(map(str, s)))
-@pytest.mark.parametrize("method", ["ghost", "explicit"])
+@pytest.mark.parametrize("method", ["ghost", "explicit", "once"])
 def test_norms_bf16(shape, method):
     X, dY = _draw(*shape)
     got = host(_lib.dp_per_sample_norms(X.cuda(), dY.cuda(), method=method))
