@@ -116,12 +116,13 @@ __device__ __forceinline__ void sincos_turn_from_word(uint32_t x, double& c, dou
   const double cos_t = fma(cp, t2, 1.0);
   const double cq = reflect ? sin_t : cos_t;    // cos and sin of the angle within the quadrant
   const double sq = reflect ? cos_t : sin_t;
-  switch (quadrant) {
-    case 0: c = cq; s = sq; break;
-    case 1: c = -sq; s = cq; break;
-    case 2: c = -cq; s = -sq; break;
-    default: c = sq; s = -cq; break;
-  }
+  // Rotate by quadrant * 90 degrees without branches: odd quadrants swap the pair, and the
+  // cosine is negative in quadrants 1 and 2, the sine in quadrants 2 and 3.
+  const bool odd = quadrant & 1u;
+  const double c0 = odd ? sq : cq;
+  const double s0 = odd ? cq : sq;
+  c = (quadrant == 1u || quadrant == 2u) ? -c0 : c0;
+  s = (quadrant >= 2u) ? -s0 : s0;
 }
 
 __device__ __forceinline__ void box_muller_f64(uint32_t x_even, uint32_t x_odd, double& z_even,

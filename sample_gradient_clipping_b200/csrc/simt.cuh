@@ -169,7 +169,7 @@ __global__ void scale_rows_bf16_kernel(const __nv_bfloat16* __restrict__ in,
 // loop is unrolled), the noise is computed while they are in flight, and then the sum is
 // formed.  This keeps both the fp64 pipe and HBM busy instead of alternating between them.
 template <int BU>  // compile-time sample count, or 0 for a runtime loop
-__global__ void __launch_bounds__(256, 3) clip_reduce_kernel(
+__global__ void __launch_bounds__(256, 2) clip_reduce_kernel(
     const __nv_bfloat16* __restrict__ Gs, int B, long long mn, NormSource src, float C,
     float* __restrict__ out, double noise_std, PhiloxKey key, uint32_t layer_id, uint32_t step_lo) {
   extern __shared__ float c_smem[];
@@ -177,17 +177,34 @@ __global__ void __launch_bounds__(256, 3) clip_reduce_kernel(
   for (int i = threadIdx.x; i < cached; i += blockDim.x) c_smem[i] = clip_factor(src.norm(i), C);
   __syncthreads();
   const long long nvec = mn / 8;  // 16-byte vectors per sample
-  for (long long v = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; v < nvec;
-       v += static_cast<long long>(gridDim.x) * blockDim.x) {
+  const long long v0 = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x;
+  uint4 pk_next[BU > 0 ? BU : 1];
+  if constexpr (BU > 0) {
+    if (v0 < nvec) {
+#pragma unroll
+      for (int i = 0; i < BU; ++i)
+        pk_next[i] = __ldcs(reinterpret_cast<const uint4*>(Gs) + v0 + static_cast<long long>(i) * nvec);
+    }
+  }
+  for (long long v = v0; v < nvec; v += static_cast<long long>(gridDim.x) * blockDim.x) {
     const uint4* g = reinterpret_cast<const uint4*>(Gs) + v;
     float acc[8];
 #pragma unroll
     for (int q = 0; q < 8; ++q) acc[q] = 0.f;
     double z[8];
     if constexpr (BU > 0) {
+      // Software pipeline: this iteration's vectors were loaded by the previous iteration
+      // (or the prologue), and the next iteration's loads are issued before the noise of this
+      // one is computed, so HBM stays busy while the fp64 pipe works.
       uint4 pk[BU > 0 ? BU : 1];
 #pragma unroll
-      for (int i = 0; i < BU; ++i) pk[i] = __ldcs(g + static_cast<long long>(i) * nvec);
+      for (int i = 0; i < BU; ++i) pk[i] = pk_next[i];
+      const long long vn = v + static_cast<long long>(gridDim.x) * blockDim.x;
+      if (vn < nvec) {
+        const uint4* gn = reinterpret_cast<const uint4*>(Gs) + vn;
+#pragma unroll
+        for (int i = 0; i < BU; ++i) pk_next[i] = __ldcs(gn + static_cast<long long>(i) * nvec);
+      }
       if (noise_std != 0.0) {
         normals4(static_cast<uint32_t>(2 * v), layer_id, step_lo, kStreamNoise, key,
                  *reinterpret_cast<double(*)[4]>(z));
