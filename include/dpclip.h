@@ -161,6 +161,30 @@ dp_status dp_philox_blocks(unsigned* out, unsigned long long nblocks, unsigned l
                            unsigned long long step, unsigned layer_id, unsigned stream_id,
                            void* stream);
 
+/* dp_per_sample_norms without a workspace, for callers that cannot allocate device memory.
+ * Some callers cannot: code that runs inside another framework's allocator hook or a memory
+ * budget it does not own, or a real-time loop that forbids new device allocations after
+ * start-up.  (The pages have no counterpart of this entry point; it is a convenience of
+ * this library.)
+ *   - Unprojected only (no P), same arguments and results as dp_per_sample_norms.
+ *   - Scratch is a fixed 1 MiB device array inside the library.  Every GPU that loads the
+ *     library holds it until the process exits.  The call refuses shapes whose scratch would
+ *     exceed it with DP_ERR_WORKSPACE (dp_last_cuda_error() gives the sizes).  bf16 needs
+ *     about 512 + 8 B + 4 B * slots bytes, where slots is the largest of
+ *     4 ceil(d_in/128) ceil(d_out/128), 8 ceil(d_in/256) ceil(d_out/256) and
+ *     2 ceil(T/128) (ceil(T/128) + 1); e.g. B <= 63 for 4096 x 4096 linears.
+ *   - It calls no cudaMalloc, cudaFree or other allocating routine.  The first call on each
+ *     device looks up the array's device address (cudaGetSymbolAddress) with that device
+ *     current.  Make that first call before any stream capture.
+ *   - Every call shares the one array, and each call clears what must start at zero.  Calls
+ *     that overlap on the GPU (other streams, other host threads) race on it and give wrong
+ *     norms: serialise them.
+ *   - An in-kernel wait that times out is recorded only inside the array; use the workspace
+ *     entry point when dp_workspace_status is needed. */
+dp_status dp_per_sample_norms_static(const void* X, const void* dY, dp_dtype dt, int B, int T,
+                                     int d_in, int d_out, dp_norm_method method, float* norms,
+                                     void* stream);
+
 /* Synchronises `stream`, then reads the status word that the kernels of earlier calls wrote
  * into `workspace`.  Returns DP_OK, DP_ERR_TIMEOUT (a bounded in-kernel wait ran out; the
  * results of that call are invalid) or DP_ERR_CUDA.  The word is cleared at the start of

@@ -37,6 +37,8 @@ SIGNATURES = {
                                 _c_int, _c_int, _c_float, _c_float, _c_ull, _c_ull, _c_uint, _c_int,
                                 _c_void_p, _c_void_p, _c_void_p, _c_size_t, _c_void_p]),
     "dp_workspace_status": (_c_int, [_c_void_p, _c_void_p]),
+    "dp_per_sample_norms_static": (_c_int, [_c_void_p, _c_void_p, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                            _c_int, _c_void_p, _c_void_p]),
     "dp_philox_blocks": (_c_int, [_c_void_p, _c_ull, _c_ull, _c_ull, _c_uint, _c_uint, _c_void_p]),
     "dp_auto_norm_method": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_int]),
     "dp_status_string": (ctypes.c_char_p, [_c_int]),

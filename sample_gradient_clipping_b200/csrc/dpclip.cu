@@ -602,6 +602,31 @@ dp_status resolve_method(const Shape& s, dp_norm_method method, dp_norm_method* 
   return DP_OK;
 }
 
+// ---------------------------------------------------------------- allocation-free norms
+// Scratch of dp_per_sample_norms_static: a fixed device array instead of a caller workspace.
+// Every GPU that loads this library holds these 1 MiB until the process exits.
+constexpr size_t kStaticScratchBytes = size_t(1) << 20;
+static __device__ __align__(256) unsigned char g_norms_scratch[kStaticScratchBytes];
+
+// Device address of g_norms_scratch on the current device.  In host code the array's name is
+// only a host-side stand-in, so the address must come from cudaGetSymbolAddress, resolved
+// once per device with that device current.
+dp_status static_scratch(unsigned char** out) {
+  static std::mutex mu;
+  static unsigned char* addr[64] = {nullptr};
+  int dev = 0;
+  DP_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return DP_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> g(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    DP_CUDA(cudaGetSymbolAddress(&p, g_norms_scratch));
+    addr[dev] = static_cast<unsigned char*>(p);
+  }
+  *out = addr[dev];
+  return DP_OK;
+}
+
 }  // namespace
 
 // ==================================================================== C ABI
@@ -732,6 +757,54 @@ dp_status dp_philox_blocks(unsigned* out, unsigned long long nblocks, unsigned l
       static_cast<uint32_t>(step & 0xFFFFFFFFull), stream_id);
   DP_CHECK_LAUNCH("philox_blocks_kernel");
   return DP_OK;
+}
+
+dp_status dp_per_sample_norms_static(const void* X, const void* dY, dp_dtype dt, int B, int T,
+                                     int d_in, int d_out, dp_norm_method method, float* norms,
+                                     void* stream) {
+  if (!X || !dY || !norms || !aligned16(X) || !aligned16(dY)) return DP_ERR_INVALID_ARG;
+  const Shape s{B, T, d_in, d_out, 0, dt};
+  if (!valid_shape(s)) return DP_ERR_INVALID_ARG;
+  dp_norm_method m;
+  dp_status st = resolve_method(s, method, &m);
+  if (st != DP_OK) return st;
+  if (m == DP_NORM_ONCE) m = DP_NORM_EXPLICIT;
+  // Layout inside the fixed array: status word, fp64 or fp32 norm accumulators, per-warp
+  // norm partials (bf16).  Anything larger than the array is refused before any launch.
+  const size_t norm2_off = 256;
+  const size_t partials_off = norm2_off + align256(static_cast<size_t>(B) * 8);
+  const int stride = (dt == DP_BF16) ? partial_slots(s) : 0;
+  const size_t total = partials_off + align256(static_cast<size_t>(B) * stride * 4);
+  if (total > kStaticScratchBytes) {
+    snprintf(g_cuda_error, sizeof(g_cuda_error),
+             "dp_per_sample_norms_static: needs %zu bytes of scratch, the fixed array holds %zu", total,
+             kStaticScratchBytes);
+    return DP_ERR_WORKSPACE;
+  }
+  if (dt == DP_BF16 && (st = get_encoder()) != DP_OK) return st;
+  unsigned char* scratch = nullptr;
+  if ((st = static_scratch(&scratch)) != DP_OK) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  // The status word and the fp32 path's atomic accumulators must start at zero.
+  DP_CUDA(cudaMemsetAsync(scratch, 0, partials_off, cs));
+  uint32_t* status = reinterpret_cast<uint32_t*>(scratch);
+  if (dt == DP_F32) {
+    double* norm2 = reinterpret_cast<double*>(scratch + norm2_off);
+    dim3 grid(ceil_div(d_out, kF32Tile), ceil_div(d_in, kF32Tile), B);
+    {
+      LaunchScope scope(kKindF32Norm, cs);
+      f32_norm_kernel<<<grid, 256, 0, cs>>>(static_cast<const float*>(X), static_cast<const float*>(dY), T,
+                                            d_in, d_out, norm2);
+      DP_CHECK_LAUNCH("f32_norm_kernel");
+    }
+    NormSource src{nullptr, norm2, nullptr};
+    return launch_finalize(src, B, INFINITY, norms, nullptr, cs);
+  }
+  float* partials = reinterpret_cast<float*>(scratch + partials_off);
+  float* norm2 = reinterpret_cast<float*>(scratch + norm2_off);
+  int count = 0;
+  if ((st = bf16_norms(s, X, dY, m, partials, stride, &count, status, cs)) != DP_OK) return st;
+  return launch_norm_partials(partials, stride, count, B, INFINITY, norm2, norms, nullptr, cs);
 }
 
 dp_status dp_workspace_status(const void* workspace, void* stream) {
