@@ -77,6 +77,23 @@ def workload_model(w):
     return flops, byts, x_shared_bytes, per_linear
 
 
+def max_over_ranks(value, device, world):
+    """The largest of every rank's value (ranks time their own replica; the job is as slow as
+    its slowest rank).  Every rank must call it at the same point."""
+    if world <= 1:
+        return float(value)
+    import torch
+
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_second(tokens_per_replica, world, ms_per_step):
+    """Whole-job throughput of `world` replicas that each process `tokens_per_replica` per step."""
+    return tokens_per_replica * world / (ms_per_step / 1e3)
+
+
 def reduce_bytes(w):
     """Bytes of the clipped-sum reduce over stored per-sample tiles: B bf16 reads + one fp32 write."""
     return sum(w.B * l.d_in * (w.r or l.d_out) * 2.0 + l.d_in * (w.r or l.d_out) * 4.0 for l in w.linears)
@@ -272,10 +289,7 @@ def run_ours(args, w, rank, world):
     ms = ev0.elapsed_time(ev1) / args.steps
     if _lib.dp_workspace_status(ws, stream) != _lib.DP_OK:
         raise RuntimeError("an in-kernel wait timed out during the timed steps")
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, dev, world)
 
     # ---- end to end through the public API with host buffers
     e2e = None
@@ -286,7 +300,6 @@ def run_ours(args, w, rank, world):
         return 0
     pk, pk_kind = peaks()
     flops, byts, xbytes, per_linear = workload_model(w)
-    tokens = w.tokens * world
     roof_t_burst = max(flops / (pk["bf16_tflops"] * 1e12), byts / (pk["hbm_gbs"] * 1e9))
     roof_t_sust = max(flops / (pk["bf16_tflops_sustained"] * 1e12), byts / (pk["hbm_gbs"] * 1e9))
     step_s = ms / 1e3
@@ -319,7 +332,8 @@ def run_ours(args, w, rank, world):
                         "launches": d_n // args.steps, "avg_launch_ms": d_ms / d_n,
                         "share_of_step": d_ms / (ms * args.steps)}
     line = {
-        "metric": METRIC, "value": tokens / step_s, "unit": "tokens/s", "n_gpus": world,
+        "metric": METRIC, "value": job_tokens_per_second(w.tokens, world, ms), "unit": "tokens/s",
+        "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "T": w.T, "linears": len(w.linears),
@@ -388,12 +402,8 @@ def run_e2e(args, w, data, dev, stream, ws, r, _lib, torch, world):
         step(k)
     ev1.record(stream)
     torch.cuda.synchronize(dev)
-    ms = ev0.elapsed_time(ev1) / steps
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
-    return {"value": w.tokens * world / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": bi,
+    ms = max_over_ranks(ev0.elapsed_time(ev1) / steps, dev, world)
+    return {"value": job_tokens_per_second(w.tokens, world, ms), "unit": "tokens/s", "h2d_bytes_per_step": bi,
             "d2h_bytes_per_step": bo, "ms_per_step": ms, "steps": steps,
             "result_read_back": "every linear's noisy clipped gradient and per-sample norms"}
 
