@@ -57,7 +57,7 @@ import numpy as np
 __all__ = [
     "philox4x32_10", "box_muller", "normals", "normals_at", "noise", "projection",
     "round_to", "per_sample_gradient", "per_sample_norm", "per_sample_norms",
-    "clip_factors", "clipped_sum", "clipped_sum_entries", "linear_step",
+    "clip_factors", "clipped_sum", "clipped_sum_entries", "linear_step", "block_step",
     "NOISE_STREAM", "PROJECTION_STREAM",
 ]
 
@@ -254,3 +254,34 @@ def linear_step(X, dY, C, sigma, seed, step, layer_id, P=None):
     std = float(sigma) * float(C)
     z = noise(S.shape[0], S.shape[1], std, seed, step, layer_id) if sigma != 0 else np.zeros_like(S)
     return {"norms": norms, "c": c, "S": S, "noise": z, "out": S + z}
+
+
+def block_step(layers, C, sigma, seed, step, mode="per_layer"):
+    """One privatised step for a block of linear layers that see the same samples.
+
+    ``layers`` is a list of dicts with X [B,T,d_in], dY [B,T,d_out], layer_id and, for
+    per-layer clipping, C (the layer's bound; ``C`` is then ignored).
+    * mode "per_layer": each layer is clipped with its own bound, as in ``linear_step``
+      (FlashDP Abstract: per-layer clipped DP-SGD).
+    * mode "flat": one clip factor per sample for the whole block,
+      c_i = min(1, C / sqrt(sum_l n_{i,l}^2)), i.e. the sample's gradient over all the
+      block's weights is clipped as one vector; every layer's noise has std sigma * C.
+    Returns {"layers": [per-layer dicts like linear_step], "flat_norms": [B] or None}.
+    """
+    if mode == "per_layer":
+        return {"layers": [linear_step(l["X"], l["dY"], l["C"], sigma, seed, step, l["layer_id"])
+                           for l in layers], "flat_norms": None}
+    if mode != "flat":
+        raise ValueError(mode)
+    if sigma != 0 and not np.isfinite(C):
+        raise ValueError("noise std sigma*C is infinite when C = inf; use sigma = 0")
+    per_layer_norms = [per_sample_norms(l["X"], l["dY"]) for l in layers]
+    flat = np.sqrt(np.sum(np.stack(per_layer_norms) ** 2, axis=0))
+    c = clip_factors(flat, C)
+    out = []
+    for l, n_l in zip(layers, per_layer_norms):
+        S = clipped_sum(l["X"], l["dY"], c)
+        z = (noise(S.shape[0], S.shape[1], float(sigma) * float(C), seed, step, l["layer_id"])
+             if sigma != 0 else np.zeros_like(S))
+        out.append({"norms": n_l, "c": c, "S": S, "noise": z, "out": S + z})
+    return {"layers": out, "flat_norms": flat}

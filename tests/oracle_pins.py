@@ -281,9 +281,38 @@ def pin_bf16_rounding(o):
     assert np.array_equal(o.round_to("f32", f.astype(np.float64)), f.astype(np.float64))
 
 
+def pin_flat_clipping(o, seed=9):
+    """Flat clipping bounds each sample's whole-block gradient by C, and one layer is per-layer."""
+    rng = np.random.default_rng(seed)
+    B, T = 4, 5
+    shapes = [(6, 3), (3, 7), (5, 5)]
+    X = [rng.standard_normal((B, T, m)) for m, _ in shapes]
+    dY = [rng.standard_normal((B, T, n)) * np.array([2.0, 0.05, 1.0, 0.3])[:, None, None]
+          for _, n in shapes]
+    layers = [{"X": x, "dY": d, "layer_id": k, "C": 1.0} for k, (x, d) in enumerate(zip(X, dY))]
+    C = 1.5
+    r = o.block_step(layers, C, 0.0, 1, 0, mode="flat")
+    G = [[o.per_sample_gradient(X[k][i], dY[k][i]) for k in range(3)] for i in range(B)]
+    for i in range(B):
+        whole = np.sqrt(sum(np.sum(g * g) for g in G[i]))          # the sample's block gradient
+        assert abs(r["flat_norms"][i] - whole) <= 1e-12 * whole
+        c_i = r["layers"][0]["c"][i]
+        assert np.sqrt(sum(np.sum((c_i * g) ** 2) for g in G[i])) <= C * (1 + 1e-12)
+        assert (c_i == 1.0) == (whole <= C)
+    # C = inf: every layer gets its plain batch gradient.
+    r_inf = o.block_step(layers, np.inf, 0.0, 1, 0, mode="flat")
+    for k in range(3):
+        plain = X[k].reshape(-1, shapes[k][0]).T @ dY[k].reshape(-1, shapes[k][1])
+        assert np.allclose(r_inf["layers"][k]["S"], plain, rtol=1e-12, atol=1e-12)
+    # A block of one layer: flat clipping is per-layer clipping with the same bound.
+    one = o.block_step([dict(layers[1], C=C)], C, 0.8, 2, 3, mode="flat")["layers"][0]
+    ref = o.linear_step(X[1], dY[1], C, 0.8, 2, 3, 1)
+    assert np.allclose(one["out"], ref["out"], rtol=1e-13, atol=1e-13)
+
+
 ALL_PINS = [
     pin_philox_kat, pin_box_muller_closed_forms, pin_box_muller_mpmath, pin_counter_layout,
     pin_gradient_brute_force, pin_gradient_finite_difference, pin_ghost_identity,
     pin_clip_invariants, pin_sigma_zero_deterministic, pin_noise_is_added_once,
-    pin_projection, pin_normal_statistics, pin_bf16_rounding,
+    pin_projection, pin_normal_statistics, pin_bf16_rounding, pin_flat_clipping,
 ]

@@ -132,10 +132,27 @@ def _mut_bf16_truncates(m):
     m.round_to = bad
 
 
+def _mut_flat_without_square(m):
+    orig = m.block_step
+
+    def bad(layers, C, sigma, seed, step, mode="per_layer"):
+        if mode != "flat":
+            return orig(layers, C, sigma, seed, step, mode)
+        norms = [m.per_sample_norms(l["X"], l["dY"]) for l in layers]
+        flat = np.sum(np.stack(norms), axis=0)            # sum of norms, not of squares
+        c = m.clip_factors(flat, C)
+        out = [{"norms": n, "c": c, "S": m.clipped_sum(l["X"], l["dY"], c)} for l, n in zip(layers, norms)]
+        for o_ in out:
+            o_["noise"] = np.zeros_like(o_["S"]); o_["out"] = o_["S"]
+        return {"layers": out, "flat_norms": flat}
+    m.block_step = bad
+
+
 MUTANTS = [
     _mut_transposed_gradient, _mut_shifted_token, _mut_no_clip, _mut_clip_by_squared_norm,
     _mut_sin_cos_swap, _mut_key_bump_first, _mut_u1_without_offset, _mut_projection_unscaled,
     _mut_project_after_clip, _mut_noise_scaled_by_sigma_only, _mut_bf16_truncates,
+    _mut_flat_without_square,
 ]
 
 _FAST_PINS = [p for p in pins.ALL_PINS if p is not pins.pin_normal_statistics]
