@@ -58,6 +58,7 @@ __all__ = [
     "philox4x32_10", "box_muller", "normals", "normals_at", "noise", "projection",
     "round_to", "per_sample_gradient", "per_sample_norm", "per_sample_norms",
     "clip_factors", "clipped_sum", "clipped_sum_entries", "linear_step", "block_step",
+    "projected_adam",
     "NOISE_STREAM", "PROJECTION_STREAM",
 ]
 
@@ -285,3 +286,27 @@ def block_step(layers, C, sigma, seed, step, mode="per_layer"):
              if sigma != 0 else np.zeros_like(S))
         out.append({"norms": n_l, "c": c, "S": S, "noise": z, "out": S + z})
     return {"layers": out, "flat_norms": flat}
+
+
+def projected_adam(W, R, m, v, P, lr, beta1, beta2, eps, grad_scale, t):
+    """One projected Adam update (DP-GRAPE page, Methodology, "Projected Optimizer States").
+
+    The optimizer state lives in the projected space: m and v are [d_in, r], like the
+    privatised projected gradient R (the noisy clipped sum of R_i = G_i P).  The page gives
+    neither the averaging nor the map back to the weights.  The plainest readings are taken:
+    the gradient estimate is g = grad_scale * R (grad_scale = 1/B averages over the batch),
+    Adam with bias correction at step t >= 1 acts on g, and the r-space update goes back to
+    the weights through P^T:
+        m <- beta1 m + (1 - beta1) g,    v <- beta2 v + (1 - beta2) g^2,
+        U = (m / (1 - beta1^t)) / (sqrt(v / (1 - beta2^t)) + eps),
+        W <- W - lr U P^T.
+    Returns (W, m, v) as new fp64 arrays.
+    """
+    g = float(grad_scale) * np.asarray(R, dtype=np.float64)
+    m = float(beta1) * np.asarray(m, dtype=np.float64) + (1.0 - float(beta1)) * g
+    v = float(beta2) * np.asarray(v, dtype=np.float64) + (1.0 - float(beta2)) * g * g
+    m_hat = m / (1.0 - float(beta1) ** t)
+    v_hat = v / (1.0 - float(beta2) ** t)
+    U = m_hat / (np.sqrt(v_hat) + float(eps))
+    W = np.asarray(W, dtype=np.float64) - float(lr) * (U @ np.asarray(P, dtype=np.float64).T)
+    return W, m, v

@@ -310,9 +310,34 @@ def pin_flat_clipping(o, seed=9):
     assert np.allclose(one["out"], ref["out"], rtol=1e-13, atol=1e-13)
 
 
+def pin_projected_adam(o, seed=10):
+    """With P = I the projected update is plain Adam: torch.optim.Adam in fp64 is the reference."""
+    import torch
+
+    rng = np.random.default_rng(seed)
+    d_in, n = 5, 6
+    W0 = rng.standard_normal((d_in, n))
+    grads = [rng.standard_normal((d_in, n)) for _ in range(3)]
+    lr, b1, b2, eps, scale = 0.01, 0.9, 0.99, 1e-8, 0.25
+    p_t = torch.nn.Parameter(torch.tensor(W0))
+    opt = torch.optim.Adam([p_t], lr=lr, betas=(b1, b2), eps=eps)
+    W, m, v = W0, np.zeros((d_in, n)), np.zeros((d_in, n))
+    for t, R in enumerate(grads, start=1):
+        p_t.grad = torch.tensor(scale * R)
+        opt.step()
+        W, m, v = o.projected_adam(W, R, m, v, np.eye(n), lr, b1, b2, eps, scale, t)
+        assert np.allclose(W, p_t.detach().numpy(), rtol=1e-12, atol=1e-14), t
+    # First step from zero moments: U = g / (|g| + eps), i.e. each weight moves by about lr.
+    R = rng.standard_normal((d_in, 3))
+    P = rng.standard_normal((n, 3))
+    W1, _, _ = o.projected_adam(W0, R, np.zeros_like(R), np.zeros_like(R), P, lr, b1, b2, 0.0, 1.0, 1)
+    assert np.allclose(W1, W0 - lr * np.sign(R) @ P.T, rtol=1e-12, atol=1e-12)
+
+
 ALL_PINS = [
     pin_philox_kat, pin_box_muller_closed_forms, pin_box_muller_mpmath, pin_counter_layout,
     pin_gradient_brute_force, pin_gradient_finite_difference, pin_ghost_identity,
     pin_clip_invariants, pin_sigma_zero_deterministic, pin_noise_is_added_once,
     pin_projection, pin_normal_statistics, pin_bf16_rounding, pin_flat_clipping,
+    pin_projected_adam,
 ]

@@ -148,11 +148,30 @@ def _mut_flat_without_square(m):
     m.block_step = bad
 
 
+def _mut_adam_without_bias_correction(m):
+    def bad(W, R, mm, vv, P, lr, beta1, beta2, eps, grad_scale, t):
+        g = grad_scale * np.asarray(R, float)
+        mm = beta1 * mm + (1 - beta1) * g
+        vv = beta2 * vv + (1 - beta2) * g * g
+        return np.asarray(W, float) - lr * (mm / (np.sqrt(vv) + eps)) @ np.asarray(P, float).T, mm, vv
+    m.projected_adam = bad
+
+
+def _mut_adam_back_projection_transposed(m):
+    orig = m.projected_adam
+
+    def bad(W, R, mm, vv, P, lr, beta1, beta2, eps, grad_scale, t):
+        Wn, mm, vv = orig(np.zeros_like(np.asarray(W, float)), R, mm, vv, P, lr, beta1, beta2, eps, grad_scale, t)
+        return np.asarray(W, float) + Wn[::-1], mm, vv    # a row-flipped update
+    m.projected_adam = bad
+
+
 MUTANTS = [
     _mut_transposed_gradient, _mut_shifted_token, _mut_no_clip, _mut_clip_by_squared_norm,
     _mut_sin_cos_swap, _mut_key_bump_first, _mut_u1_without_offset, _mut_projection_unscaled,
     _mut_project_after_clip, _mut_noise_scaled_by_sigma_only, _mut_bf16_truncates,
-    _mut_flat_without_square,
+    _mut_flat_without_square, _mut_adam_without_bias_correction,
+    _mut_adam_back_projection_transposed,
 ]
 
 _FAST_PINS = [p for p in pins.ALL_PINS if p is not pins.pin_normal_statistics]
