@@ -13,13 +13,14 @@
 //   z_even = sqrt(-2 ln u1) cos(2 pi u2) and z_odd = sqrt(-2 ln u1) sin(2 pi u2).
 // The transform is evaluated in fp64.  A value in fp32 would be off by several 1e-7 near
 // |z| = 6.7, because 2 pi u2 and ln u1 then lose bits.  The logarithm and the sine/cosine take
-// their arguments straight from the 32-bit words.  So the range reduction is exact integer
-// work, and each is a short textbook series (log_u1_from_word, sincos_turn_from_word), with
-// errors near 1e-16.
+// their arguments straight from the 32-bit words, so the range reduction is exact integer
+// work, and each is a table lookup plus a short polynomial (box_muller_f64 below).
 //
 // Counter layout: (j, layer_id, step mod 2^32, stream); key: (seed mod 2^32, seed >> 32).
 #pragma once
 #include <cstdint>
+
+#include "noise_tables.cuh"
 
 namespace dpclip {
 
@@ -55,91 +56,166 @@ __device__ __forceinline__ uint4 philox4x32_10(uint4 c, PhiloxKey k) {
   return c;
 }
 
-// ln(u1) for u1 = (x + 1) 2^-32, in fp64, straight from the integer.
-// y = x + 1 = 2^e f with f in [sqrt(2)/2, sqrt(2)) found exactly from the leading bit, so
-// ln u1 = (e - 32) ln 2 + ln f, and ln f = 2 atanh(s) = 2 (s + s^3/3 + s^5/5 + ...) with
-// s = (f - 1) / (f + 1), |s| <= 0.1716 (the classical atanh series for the logarithm).  Nine
-// terms leave a truncation error below 0.1716^19 / 19 < 3e-16 relative.
-__device__ __forceinline__ double log_u1_from_word(uint32_t x) {
-  const unsigned long long y = static_cast<unsigned long long>(x) + 1ull;  // 1 .. 2^32
-  int e = 63 - __clzll(static_cast<long long>(y));                         // y in [2^e, 2^(e+1))
-  // f = y 2^-e, exact: y < 2^53 and the scale is a power of two.
-  double f = static_cast<double>(y) * __longlong_as_double(static_cast<long long>(1023 - e) << 52);
-  if (f > 1.4142135623730951) {
-    f *= 0.5;
-    ++e;
+// Table-driven Box-Muller (Tang, "Table-driven implementation of the logarithm function in
+// IEEE floating-point arithmetic", ACM TOMS 1990; sine and cosine by the addition formula
+// around tabulated angles).  Every breakpoint value is the double nearest its exact value
+// (gen_noise_tables.py), so each piece is a short polynomial on a small interval.  The noise is
+// issue-bound where it is generated, and this form needs about 40 fp64 operations per pair.
+// Against 50-digit arithmetic on all edge words and 6500 random pairs, |z - z_exact| stays
+// below 5e-13.  The largest errors come at u1 just below 1, where the radius is ~2e-5.
+
+// Where the transform reads its tables.  Global: the module's arrays through the read-only
+// cache.  Shared: eight copies, entry j of copy c at [8 j + c], each thread reading copy
+// threadIdx.x mod 8.  A 128-bit shared load serves 8 threads per pass, so the 8 threads of a
+// pass always read 8 different bank groups, whatever entries they want.
+struct NoiseTablesGlobal {
+  __device__ __forceinline__ double2 ln(uint32_t j) const { return __ldg(&kLnTable[j]); }
+  __device__ __forceinline__ double2 sincos(uint32_t j) const { return __ldg(&kSinCosTable[j]); }
+};
+
+constexpr int kNoiseTableCopies = 8;
+constexpr int kNoiseSharedEntries = 2 * kNoiseTableSize * kNoiseTableCopies;
+constexpr int kNoiseSharedBytes = kNoiseSharedEntries * 16;  // 32 KB
+
+struct NoiseTablesShared {
+  const double2* s;  // kNoiseSharedEntries entries, filled by stage_noise_tables
+  __device__ __forceinline__ double2 ln(uint32_t j) const {
+    return s[j * kNoiseTableCopies + (threadIdx.x & (kNoiseTableCopies - 1))];
   }
-  const double s = (f - 1.0) / (f + 1.0);
-  const double s2 = s * s;
-  double p = 1.0 / 19.0;
-  p = fma(p, s2, 1.0 / 17.0);
-  p = fma(p, s2, 1.0 / 15.0);
-  p = fma(p, s2, 1.0 / 13.0);
-  p = fma(p, s2, 1.0 / 11.0);
-  p = fma(p, s2, 1.0 / 9.0);
-  p = fma(p, s2, 1.0 / 7.0);
-  p = fma(p, s2, 1.0 / 5.0);
-  p = fma(p, s2, 1.0 / 3.0);
-  const double ln_f = 2.0 * s * fma(p, s2, 1.0);
-  return fma(static_cast<double>(e - 32), 0.6931471805599453, ln_f);
+  __device__ __forceinline__ double2 sincos(uint32_t j) const {
+    return s[(kNoiseTableSize + j) * kNoiseTableCopies + (threadIdx.x & (kNoiseTableCopies - 1))];
+  }
+};
+
+// Fills the shared copies; the caller synchronises the block before the first read.
+__device__ __forceinline__ void stage_noise_tables(double2* s) {
+  for (int i = threadIdx.x; i < kNoiseSharedEntries; i += blockDim.x) {
+    const int j = (i / kNoiseTableCopies) % kNoiseTableSize;
+    s[i] = i < kNoiseTableSize * kNoiseTableCopies ? kLnTable[j] : kSinCosTable[j];
+  }
 }
 
-// (cos, sin) of the angle 2 pi x 2^-32, in fp64, from the integer.
-// The quadrant is the top two bits of x.  Within it, the angle fraction f < 2^30 is reflected
-// to f' = 2^30 - f when f > 2^29, so that the reduced angle t = f' 2 pi 2^-32 lies in
-// [0, pi/4]; the reflection swaps sine and cosine, and each quadrant rotates the pair by 90
-// degrees.  All of this is exact integer work.  sin t and cos t are then the Taylor series to
-// t^15 and t^16: the next terms are below (pi/4)^17/17! < 2e-16.
-__device__ __forceinline__ void sincos_turn_from_word(uint32_t x, double& c, double& s) {
-  const uint32_t quadrant = x >> 30;
-  uint32_t f = x & 0x3FFFFFFFu;
-  const bool reflect = f > 0x20000000u;
-  if (reflect) f = 0x40000000u - f;
-  const double t = static_cast<double>(f) * 1.4629180792671596e-09;  // 2 pi / 2^32
-  const double t2 = t * t;
-  double sp = -1.0 / 1307674368000.0;          // -1/15!
-  sp = fma(sp, t2, 1.0 / 6227020800.0);         //  1/13!
-  sp = fma(sp, t2, -1.0 / 39916800.0);          // -1/11!
-  sp = fma(sp, t2, 1.0 / 362880.0);             //  1/9!
-  sp = fma(sp, t2, -1.0 / 5040.0);              // -1/7!
-  sp = fma(sp, t2, 1.0 / 120.0);                //  1/5!
-  sp = fma(sp, t2, -1.0 / 6.0);                 // -1/3!
-  const double sin_t = fma(sp * t2, t, t);
-  double cp = 1.0 / 20922789888000.0;           //  1/16!
-  cp = fma(cp, t2, -1.0 / 87178291200.0);       // -1/14!
-  cp = fma(cp, t2, 1.0 / 479001600.0);          //  1/12!
-  cp = fma(cp, t2, -1.0 / 3628800.0);           // -1/10!
-  cp = fma(cp, t2, 1.0 / 40320.0);              //  1/8!
-  cp = fma(cp, t2, -1.0 / 720.0);               // -1/6!
-  cp = fma(cp, t2, 1.0 / 24.0);                 //  1/4!
-  cp = fma(cp, t2, -0.5);                       // -1/2!
-  const double cos_t = fma(cp, t2, 1.0);
-  const double cq = reflect ? sin_t : cos_t;    // cos and sin of the angle within the quadrant
-  const double sq = reflect ? cos_t : sin_t;
-  // Rotate by quadrant * 90 degrees without branches: odd quadrants swap the pair, and the
-  // cosine is negative in quadrants 1 and 2, the sine in quadrants 2 and 3.
-  const bool odd = quadrant & 1u;
-  const double c0 = odd ? sq : cq;
-  const double s0 = odd ? cq : sq;
-  c = (quadrant == 1u || quadrant == 2u) ? -c0 : c0;
-  s = (quadrant >= 2u) ? -s0 : s0;
+__device__ __forceinline__ float rsqrt_approx(float a) {
+  float r;
+  asm("rsqrt.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(a));
+  return r;
 }
 
-__device__ __forceinline__ void box_muller_f64(uint32_t x_even, uint32_t x_odd, double& z_even,
-                                               double& z_odd) {
-  const double radius = sqrt(-2.0 * log_u1_from_word(x_even));
+// Integer -> double without a conversion instruction: the double with high word 0x43300000
+// and low word u is exactly 2^52 + u, so one subtraction gives u - offset exactly.  Where the
+// noise is generated, conversions share a narrow pipe that would otherwise be the bound.
+constexpr double kTwo52 = 4503599627370496.0;
+__device__ __forceinline__ double u32_minus(uint32_t u, double offset) {
+  return __hiloint2double(0x43300000, static_cast<int>(u)) - (kTwo52 + offset);
+}
+
+// Exact double <-> float moves by bit manipulation for normal, positive values in the float
+// range (2^-126 <= a < 2^128); the float is the double truncated to 24 bits.
+__device__ __forceinline__ float f32_trunc_from_pos_f64(double a) {
+  const int hi = __double2hiint(a);
+  const uint32_t lo = static_cast<uint32_t>(__double2loint(a));
+  return __int_as_float(((hi - (896 << 20)) << 3) | static_cast<int>(lo >> 29));
+}
+__device__ __forceinline__ double f64_from_pos_f32(float f) {
+  const int b = __float_as_int(f);
+  return __hiloint2double((b >> 3) + (896 << 20), b << 29);
+}
+
+// -2 ln(u1), u1 = (x + 1) 2^-32.  x + 1 = 2^k m exactly, m in [1, 2), and with (F, L) the
+// table entry of m's top 7 fraction bits, ln m = L + ln(1 + r) where r = m F - 1 comes from
+// one fused multiply-add and |r| <= 2^-8.  ln(1 + r) is its Taylor series to r^6 (the next
+// term is below 2e-18).  ln 2 is split so that (k - 32) ln 2 adds without rounding error.
+template <class Tab>
+__device__ __forceinline__ double minus_two_ln_u1(uint32_t x, const Tab& tab) {
+  const double d = u32_minus(x, -1.0);             // x + 1, exact
+  const int hi = __double2hiint(d);                // biased exponent 1023 + k, k = 0 .. 32
+  const double m = __hiloint2double((hi & 0x000FFFFF) | 0x3FF00000, __double2loint(d));
+  const double2 FL = tab.ln((static_cast<uint32_t>(hi) >> 13) & (kNoiseTableSize - 1));
+  const double r = fma(m, FL.x, -1.0);
+  double q = fma(r, -1.0 / 6.0, 1.0 / 5.0);
+  q = fma(r, q, -0.25);
+  q = fma(r, q, 1.0 / 3.0);
+  q = fma(r, q, -0.5);
+  const double ln1p_r = fma(r * r, q, r);
+  const double kk = u32_minus(static_cast<uint32_t>(hi) >> 20, 1055.0);  // k - 32
+  return -2.0 * (fma(kk, kLn2Hi, FL.y) + fma(kk, kLn2Lo, ln1p_r));
+}
+
+// sqrt(y) for 2^-126 <= y < 2^128: fp32 reciprocal-square-root seed (relative error ~2^-22),
+// one coupled Newton step on s ~ sqrt(y) and h ~ 1/(2 sqrt(y)) (Goldschmidt), then the
+// residual correction s + (y - s^2) h.
+__device__ __forceinline__ double sqrt_pos_f64(double y) {
+  const double r0 = f64_from_pos_f32(rsqrt_approx(f32_trunc_from_pos_f64(y)));
+  double s = y * r0, h = 0.5 * r0;
+  const double e = fma(-s, h, 0.5);
+  s = fma(s, e, s);
+  h = fma(h, e, h);
+  return fma(fma(-s, s, y), h, s);
+}
+
+// (cos, sin) of 2 pi x 2^-32.  The top 7 bits of x pick the sector centre a_j = 2 pi (j + 1/2)
+// / 128; the other 25 bits, centred, give delta = angle - a_j exactly as an integer times
+// 2 pi 2^-32, |delta| <= pi/128.  sin(delta) to delta^7 and 1 - cos(delta) to delta^6 (next
+// terms below 1e-20 and 4e-18) then enter the addition formulas, written so that the small
+// corrections are added to the tabulated values last.
+template <class Tab>
+__device__ __forceinline__ void sincos_turn(uint32_t x, const Tab& tab, double& c, double& s) {
+  const double delta = u32_minus(x & 0x1FFFFFFu, 16777216.0) * kTurnToRad;
+  const double d2 = delta * delta;
+  double sp = fma(d2, -1.0 / 5040.0, 1.0 / 120.0);
+  sp = fma(d2, sp, -1.0 / 6.0);
+  const double sin_d = fma(delta * d2, sp, delta);
+  double cp = fma(d2, 1.0 / 720.0, -1.0 / 24.0);
+  cp = fma(d2, cp, 0.5);
+  const double one_minus_cos_d = d2 * cp;
+  const double2 SC = tab.sincos(x >> 25);
+  s = SC.x + fma(SC.y, sin_d, -(SC.x * one_minus_cos_d));
+  c = SC.y - fma(SC.x, sin_d, SC.y * one_minus_cos_d);
+}
+
+template <class Tab>
+__device__ __forceinline__ void box_muller_f64(uint32_t x_even, uint32_t x_odd, const Tab& tab,
+                                               double& z_even, double& z_odd) {
+  const double y = minus_two_ln_u1(x_even, tab);
+  // u1 = 1 exactly (x_even = 2^32 - 1) has radius 0; y there is a rounding residue.  Every
+  // other word gives y >= 4.6e-10, inside the range of sqrt_pos_f64.
+  const double radius = x_even == 0xFFFFFFFFu ? 0.0 : sqrt_pos_f64(y);
   double c, s;
-  sincos_turn_from_word(x_odd, c, s);
+  sincos_turn(x_odd, tab, c, s);
   z_even = radius * c;
   z_odd = radius * s;
 }
 
-// The four standard normals of Philox block j: elements 4j .. 4j+3 of the stream.
-__device__ __forceinline__ void normals4(uint32_t j, uint32_t layer_id, uint32_t step_lo,
-                                         uint32_t stream, PhiloxKey key, double (&z)[4]) {
+// Full-precision Box-Muller (CUDA's log, sqrt and sincospi, ~1e-16).  Used where the normals
+// are rounded to a storage type and that rounding must agree with an exact reference bit for
+// bit: the projection matrix P.  A 1e-11 error would move a few P entries across a rounding
+// boundary.
+__device__ __forceinline__ void box_muller_f64_precise(uint32_t x_even, uint32_t x_odd, double& z_even,
+                                                       double& z_odd) {
+  const double u1 = (static_cast<double>(x_even) + 1.0) * 0x1p-32;
+  const double u2 = static_cast<double>(x_odd) * 0x1p-32;
+  const double radius = sqrt(-2.0 * log(u1));
+  double s, c;
+  sincospi(2.0 * u2, &s, &c);
+  z_even = radius * c;
+  z_odd = radius * s;
+}
+
+__device__ __forceinline__ void normals4_precise(uint32_t j, uint32_t layer_id, uint32_t step_lo,
+                                                 uint32_t stream, PhiloxKey key, double (&z)[4]) {
   const uint4 x = philox4x32_10(make_uint4(j, layer_id, step_lo, stream), key);
-  box_muller_f64(x.x, x.y, z[0], z[1]);
-  box_muller_f64(x.z, x.w, z[2], z[3]);
+  box_muller_f64_precise(x.x, x.y, z[0], z[1]);
+  box_muller_f64_precise(x.z, x.w, z[2], z[3]);
+}
+
+// The four standard normals of Philox block j: elements 4j .. 4j+3 of the stream.
+template <class Tab = NoiseTablesGlobal>
+__device__ __forceinline__ void normals4(uint32_t j, uint32_t layer_id, uint32_t step_lo,
+                                         uint32_t stream, PhiloxKey key, double (&z)[4],
+                                         const Tab& tab = Tab{}) {
+  const uint4 x = philox4x32_10(make_uint4(j, layer_id, step_lo, stream), key);
+  box_muller_f64(x.x, x.y, tab, z[0], z[1]);
+  box_muller_f64(x.z, x.w, tab, z[2], z[3]);
 }
 
 }  // namespace dpclip
