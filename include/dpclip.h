@@ -185,6 +185,75 @@ dp_status dp_per_sample_norms_static(const void* X, const void* dY, dp_dtype dt,
                                      int d_in, int d_out, dp_norm_method method, float* norms,
                                      void* stream);
 
+/* ------------------------------------------------------------------ block step
+ * One call for all the linears of a block that see the same samples (e.g. q, k, v, o, gate,
+ * up, down of a transformer block).  Two clipping modes:
+ *   DP_CLIP_PER_LAYER : each layer l is clipped with its own bound layers[l].C and gets noise
+ *                       of std sigma * layers[l].C.  This is per-layer clipped DP-SGD
+ *                       (FlashDP Abstract), the same result as one dp_linear_step per layer.
+ *   DP_CLIP_FLAT      : one clip factor per sample for the whole block,
+ *                       c_i = min(1, C / sqrt(sum_l n_{i,l}^2)).  The sample's gradient over
+ *                       all the block's weights is clipped as one vector, as in textbook
+ *                       DP-SGD.  Every layer's output gets noise of std sigma * C.
+ * Each layer's noise uses its own layer_id in the Philox counter.  Unprojected only.
+ * Layers whose norm method resolves to DP_NORM_GHOST and that point at the same X with the
+ * same d_in and d_out (q/k/v; gate/up) are grouped, up to three, and share one X Gram per
+ * pair of 128-token blocks; their norms are bitwise those of one layer at a time. */
+typedef struct {
+    const void* X;        /* DEVICE [B, T, d_in] in dtype dt */
+    const void* dY;       /* DEVICE [B, T, d_out] in dtype dt */
+    int d_in, d_out;
+    unsigned layer_id;
+    float C;              /* the layer's bound (per-layer mode; ignored in flat mode) */
+    float* G_out;         /* DEVICE fp32 [d_in, d_out], overwritten */
+    float* norms_out;     /* NULL or DEVICE fp32 [B]: the layer's own per-sample norms */
+} dp_layer;
+
+typedef enum { DP_CLIP_PER_LAYER = 0, DP_CLIP_FLAT = 1 } dp_clip_mode;
+
+/* Workspace bytes for dp_block_step with these layers (0 if a layer's shape is invalid).
+ * Flat mode with DP_NORM_ONCE keeps every layer's per-sample tiles: sum_l B d_in d_out bf16;
+ * per-layer mode finishes each layer first and needs one such region, for the largest. */
+size_t dp_block_workspace_size(const dp_layer* layers, int L, int B, int T, dp_dtype dt,
+                               dp_clip_mode mode, dp_norm_method method);
+
+/* layers: HOST array of L descriptors; the tensors they point to are DEVICE memory.
+ * C: the flat bound (> 0; flat mode only).  flat_norms_out: NULL or DEVICE fp32 [B],
+ * sqrt(sum_l n_{i,l}^2) (flat mode only).  Other arguments as for dp_linear_step. */
+dp_status dp_block_step(const dp_layer* layers, int L, dp_dtype dt, int B, int T,
+                        dp_clip_mode mode, float C, float sigma, unsigned long long seed,
+                        unsigned long long step, dp_norm_method method, float* flat_norms_out,
+                        void* workspace, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------ projected Adam
+ * One projected Adam update.  DP-GRAPE page, Methodology, "Projected Optimizer States": the
+ * optimizer state lives in the projected space, O(r x layers) instead of O(d).  The page
+ * gives neither the averaging nor the map back to the weights; the plainest readings are
+ * used:
+ *   g = grad_scale * R                          (grad_scale = 1/B averages over the batch)
+ *   m <- beta1 m + (1 - beta1) g,  v <- beta2 v + (1 - beta2) g^2
+ *   U = (m / (1 - beta1^t)) / (sqrt(v / (1 - beta2^t)) + eps)        (t >= 1)
+ *   W <- W - lr U P^T                           (the r-space update mapped back through P)
+ *   W    : DEVICE fp32 [d_in, d_out], updated in place.
+ *   R    : DEVICE fp32 [d_in, r], the privatised projected gradient (G_out of a projected
+ *          dp_linear_step).
+ *   m, v : DEVICE fp32 [d_in, r], updated in place; zeros before the first step.
+ *   P    : DEVICE [d_out, r] in dtype dt (bf16: U is rounded to bf16 for the tensor cores).
+ *   workspace : DEVICE, 256-byte aligned, >= dp_adam_workspace_size(d_in, r) bytes.
+ * d_in, d_out and r are multiples of 8. */
+size_t dp_adam_workspace_size(int d_in, int r);
+dp_status dp_projected_adam_step(float* W, const float* R, float* m, float* v, const void* P,
+                                 dp_dtype dt, int d_in, int d_out, int r, float lr, float beta1,
+                                 float beta2, float eps, float grad_scale, int t, void* workspace,
+                                 size_t ws_bytes, void* stream);
+
+/* Failure-detection self-test of the bounded in-kernel waits: a one-warp kernel waits on a
+ * barrier that nothing arrives at.  After limit_ns nanoseconds (1 us .. 2 s) it gives up,
+ * records the timeout in the workspace's status word and returns.  dp_workspace_status then
+ * reports DP_ERR_TIMEOUT, and the device stays usable for further calls.
+ *   workspace : DEVICE, 256-byte aligned, at least 256 bytes. */
+dp_status dp_selftest_wait_timeout(void* workspace, unsigned long long limit_ns, void* stream);
+
 /* Synchronises `stream`, then reads the status word that the kernels of earlier calls wrote
  * into `workspace`.  Returns DP_OK, DP_ERR_TIMEOUT (a bounded in-kernel wait ran out; the
  * results of that call are invalid) or DP_ERR_CUDA.  The word is cleared at the start of

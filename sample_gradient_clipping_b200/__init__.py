@@ -5,6 +5,7 @@ holds the ctypes binding (``_lib``), the in-tree build script (``build``) and th
 synthetic workloads (``inputs``).
 """
 from ._lib import (  # noqa: F401
-    DPError, auto_norm_method, dp_add_noise, dp_clip_accumulate, dp_linear_step, dp_philox_blocks,
+    DPError, auto_norm_method, dp_add_noise, dp_block_step, dp_clip_accumulate, dp_linear_step, dp_philox_blocks,
+    dp_projected_adam_step,
     dp_per_sample_norms, dp_projection_matrix, dp_workspace_status, lib, workspace_size,
 )

@@ -23,6 +23,16 @@ METHOD_NAMES = {v: k for k, v in METHODS.items()}
 _c_void_p, _c_int, _c_float = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
 _c_size_t, _c_ll, _c_ull, _c_uint = ctypes.c_size_t, ctypes.c_longlong, ctypes.c_ulonglong, ctypes.c_uint
 
+class DpLayer(ctypes.Structure):
+    """Mirror of the C struct dp_layer (include/dpclip.h)."""
+    _fields_ = [("X", ctypes.c_void_p), ("dY", ctypes.c_void_p), ("d_in", ctypes.c_int),
+                ("d_out", ctypes.c_int), ("layer_id", ctypes.c_uint), ("C", ctypes.c_float),
+                ("G_out", ctypes.c_void_p), ("norms_out", ctypes.c_void_p)]
+
+
+DP_CLIP_PER_LAYER, DP_CLIP_FLAT = 0, 1
+CLIP_MODES = {"per_layer": DP_CLIP_PER_LAYER, "flat": DP_CLIP_FLAT}
+
 SIGNATURES = {
     "dp_workspace_size": (_c_size_t, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_int]),
     "dp_workspace_size_for": (_c_size_t, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int]),
@@ -37,12 +47,22 @@ SIGNATURES = {
                                 _c_int, _c_int, _c_float, _c_float, _c_ull, _c_ull, _c_uint, _c_int,
                                 _c_void_p, _c_void_p, _c_void_p, _c_size_t, _c_void_p]),
     "dp_workspace_status": (_c_int, [_c_void_p, _c_void_p]),
+    "dp_selftest_wait_timeout": (_c_int, [_c_void_p, _c_ull, _c_void_p]),
     "dp_per_sample_norms_static": (_c_int, [_c_void_p, _c_void_p, _c_int, _c_int, _c_int, _c_int, _c_int,
                                             _c_int, _c_void_p, _c_void_p]),
     "dp_philox_blocks": (_c_int, [_c_void_p, _c_ull, _c_ull, _c_ull, _c_uint, _c_uint, _c_void_p]),
     "dp_auto_norm_method": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_int]),
     "dp_status_string": (ctypes.c_char_p, [_c_int]),
     "dp_last_cuda_error": (ctypes.c_char_p, []),
+    "dp_block_workspace_size": (_c_size_t, [ctypes.POINTER(DpLayer), _c_int, _c_int, _c_int, _c_int,
+                                            _c_int, _c_int]),
+    "dp_block_step": (_c_int, [ctypes.POINTER(DpLayer), _c_int, _c_int, _c_int, _c_int, _c_int, _c_float,
+                               _c_float, _c_ull, _c_ull, _c_int, _c_void_p, _c_void_p, _c_size_t,
+                               _c_void_p]),
+    "dp_adam_workspace_size": (_c_size_t, [_c_int, _c_int]),
+    "dp_projected_adam_step": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_int, _c_int,
+                                        _c_int, _c_int, _c_float, _c_float, _c_float, _c_float, _c_float,
+                                        _c_int, _c_void_p, _c_size_t, _c_void_p]),
     "dp_profiling_enable": (_c_int, [_c_int]),
     "dp_profiling_kinds": (_c_int, []),
     "dp_profiling_kind_name": (ctypes.c_char_p, [_c_int]),
@@ -236,3 +256,57 @@ def profiling_collect():
     cnt = (_c_ll * n)()
     check(lib().dp_profiling_collect(ms, cnt), "dp_profiling_collect")
     return {lib().dp_profiling_kind_name(k).decode(): (ms[k], cnt[k]) for k in range(n) if cnt[k]}
+
+
+def dp_block_step(layers, mode="per_layer", C=1.0, sigma=0.0, seed=0, step=0, method="auto",
+                  flat_norms_out=None, workspace=None, stream=None):
+    """One step for a block of linears sharing the batch.
+
+    ``layers``: dicts with X, dY, layer_id, C (per-layer bound), and optional G_out, norms_out.
+    Returns (list of G_out, list of norms_out or None, flat_norms_out or None).
+    """
+    import torch
+
+    first = layers[0]
+    B, T = int(first["X"].shape[0]), int(first["X"].shape[1])
+    dt = _dtype_code(first["X"])
+    arr = (DpLayer * len(layers))()
+    outs, norms = [], []
+    for k, l in enumerate(layers):
+        _, _, d_in, d_out = _bt_dims(l["X"], l["dY"])
+        G = l.get("G_out")
+        if G is None:
+            G = torch.empty(d_in, d_out, dtype=torch.float32, device=l["X"].device)
+        n = l.get("norms_out")
+        arr[k] = DpLayer(_ptr(l["X"]), _ptr(l["dY"]), d_in, d_out, int(l["layer_id"]), float(l.get("C", C)),
+                         _ptr(G), _ptr(n))
+        outs.append(G)
+        norms.append(n)
+    need = int(lib().dp_block_workspace_size(arr, len(layers), B, T, dt, CLIP_MODES[mode], METHODS[method]))
+    if need == 0:
+        raise DPError(DP_ERR_INVALID_ARG, "dp_block_workspace_size")
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=first["X"].device)
+    if mode == "flat" and flat_norms_out is None:
+        flat_norms_out = torch.empty(B, dtype=torch.float32, device=first["X"].device)
+    check(lib().dp_block_step(arr, len(layers), dt, B, T, CLIP_MODES[mode], float(C), float(sigma), int(seed),
+                              int(step), METHODS[method], _ptr(flat_norms_out), _ptr(workspace),
+                              workspace.numel(), _stream(stream)),
+          "dp_block_step")
+    return outs, norms, flat_norms_out
+
+
+def dp_projected_adam_step(W, R, m, v, P, lr, t, beta1=0.9, beta2=0.999, eps=1e-8, grad_scale=1.0,
+                           workspace=None, stream=None):
+    """One projected Adam update: W -= lr * U P^T with Adam moments m, v kept in r-space."""
+    import torch
+
+    d_in, d_out = int(W.shape[0]), int(W.shape[1])
+    r = int(R.shape[1])
+    if workspace is None:
+        workspace = torch.empty(int(lib().dp_adam_workspace_size(d_in, r)), dtype=torch.uint8, device=W.device)
+    check(lib().dp_projected_adam_step(_ptr(W), _ptr(R), _ptr(m), _ptr(v), _ptr(P), _dtype_code(P), d_in, d_out,
+                                       r, float(lr), float(beta1), float(beta2), float(eps), float(grad_scale),
+                                       int(t), _ptr(workspace), workspace.numel(), _stream(stream)),
+          "dp_projected_adam_step")
+    return W, m, v

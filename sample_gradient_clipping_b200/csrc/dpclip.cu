@@ -5,11 +5,13 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "dpclip.h"
 #include "launch_profiler.h"
@@ -241,6 +243,8 @@ dp_status launch_umma(const UmmaParams& p, cudaStream_t stream) {
                        : Cfg::EPI == kEpiExplicitNorm  ? kKindExplicitNorm
                        : Cfg::EPI == kEpiExplicitStore ? kKindExplicitStore
                        : Cfg::EPI == kEpiGhostNorm     ? kKindGhostNorm
+                       : Cfg::EPI == kEpiAxpy          ? kKindAxpy
+                       : Cfg::EPI == kEpiGhostShared   ? kKindGhostShared
                                                        : kKindProject;
   LaunchScope scope(kind, stream);
   umma_kernel<Cfg><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(p);
@@ -315,6 +319,33 @@ dp_status bf16_norms(const Shape& s, const void* X, const void* Z, dp_norm_metho
   return launch_umma<UmmaConfig<256, kEpiExplicitNorm>>(p, stream);
 }
 
+// Ghost-norm partials of k <= 3 linears that read the same X ([B, T, m]) with dY operands
+// Zs[j] of equal width ne: one X Gram per token-block pair serves all of them.  Operand j's
+// partials go to partials + j * op_stride, laid out as for bf16_norms.
+dp_status bf16_norms_ghost_shared(const Shape& s, const void* X, const void* const* Zs, int k,
+                                  float* partials, int stride, long long op_stride, int* count,
+                                  uint32_t* status, cudaStream_t stream) {
+  if (k < 1 || k > kGhostSharedMaxOps) return DP_ERR_INVALID_ARG;
+  UmmaParams p = base_params(status);
+  p.partials = partials;
+  p.partial_stride = stride;
+  p.partial_op_stride = op_stride;
+  p.ghost_ops = k;
+  const int ne = s.ne();
+  dp_status st;
+  if ((st = map_3d(&p.tmA0, X, s.B, s.T, s.m, 128)) != DP_OK) return st;
+  CUtensorMap* maps[kGhostSharedMaxOps] = {&p.tmB0, &p.tmA1, &p.tmB1};
+  for (int j = 0; j < k; ++j)
+    if ((st = map_3d(maps[j], Zs[j], s.B, s.T, ne, 128)) != DP_OK) return st;
+  p.t_tiles = ceil_div(s.T, 128);
+  p.pairs_per_sample = p.t_tiles * (p.t_tiles + 1) / 2;
+  p.num_units = s.B * p.pairs_per_sample;
+  *count = 4 * p.pairs_per_sample;
+  p.k_blocks = ceil_div(s.m, 64);
+  p.k_blocks1 = ceil_div(ne, 64);
+  return launch_umma<UmmaConfig<128, kEpiGhostShared>>(p, stream);
+}
+
 dp_status launch_noise(float* G, unsigned long long total, double std_dev, unsigned long long seed,
                        unsigned long long step, unsigned layer_id, cudaStream_t stream);
 
@@ -373,8 +404,16 @@ dp_status bf16_clipsum(const Shape& s, const void* A, const void* Bm, float* out
 dp_status launch_noise(float* G, unsigned long long total, double std_dev, unsigned long long seed,
                        unsigned long long step, unsigned layer_id, cudaStream_t stream) {
   LaunchScope scope(kKindNoise, stream);
-  noise_add_kernel<<<stream_grid((total + 3) / 4, 256), 256, 0, stream>>>(
-      G, total, std_dev, philox_key_from_seed(seed), layer_id, static_cast<uint32_t>(step & 0xFFFFFFFFull));
+  // Large G: a persistent grid whose blocks stage the 32 KB of Box-Muller tables once each.
+  const PhiloxKey key = philox_key_from_seed(seed);
+  const uint32_t step_lo = static_cast<uint32_t>(step & 0xFFFFFFFFull);
+  if (total >= (1ull << 22)) {
+    const int grid = std::min(stream_grid((total + 3) / 4, 256), sm_count() * 4);
+    noise_add_kernel<true><<<grid, 256, 0, stream>>>(G, total, std_dev, key, layer_id, step_lo);
+  } else {
+    noise_add_kernel<false><<<stream_grid((total + 3) / 4, 256), 256, 0, stream>>>(G, total, std_dev, key,
+                                                                                  layer_id, step_lo);
+  }
   DP_CHECK_LAUNCH("noise_add_kernel");
   return DP_OK;
 }
@@ -452,12 +491,52 @@ void reduce_kernel_launch(int grid, size_t smem, cudaStream_t stream, const __nv
                                                       step_lo);
 }
 
+template <int BU>
+dp_status reduce_tma_launch(cudaStream_t stream, const __nv_bfloat16* gs, long long mn, NormSource src,
+                            float C, float* out, double noise_std, PhiloxKey key, unsigned layer_id,
+                            uint32_t step_lo, uint32_t* status) {
+  using Cfg = ReduceTmaConfig<BU>;
+  static bool configured[64] = {false};
+  int dev = 0;
+  DP_CUDA(cudaGetDevice(&dev));
+  if (dev >= 0 && dev < 64 && !configured[dev]) {
+    DP_CUDA(cudaFuncSetAttribute(clip_reduce_tma_kernel<BU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Cfg::SMEM_BYTES));
+    configured[dev] = true;
+  }
+  const long long chunks = (mn + kReduceChunk - 1) / kReduceChunk;
+  const int grid = static_cast<int>(chunks < sm_count() ? chunks : sm_count());
+  clip_reduce_tma_kernel<BU><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(gs, mn, src, C, out, noise_std,
+                                                                               key, layer_id, step_lo, status);
+  return DP_OK;
+}
+
 dp_status launch_reduce(const __nv_bfloat16* gs, int B, long long mn, NormSource src, float C,
                         float* out, double noise_std, unsigned long long seed, unsigned long long step,
-                        unsigned layer_id, cudaStream_t stream) {
+                        unsigned layer_id, cudaStream_t stream, uint32_t* status) {
+  if (B <= 8) {
+    // Warp-specialised bulk-copy reduce: noise generation overlaps the HBM stream.
+    const PhiloxKey key = philox_key_from_seed(seed);
+    const uint32_t step_lo = static_cast<uint32_t>(step & 0xFFFFFFFFull);
+    LaunchScope scope(kKindReduce, stream);
+    dp_status st;
+    switch (B) {
+      case 1: st = reduce_tma_launch<1>(stream, gs, mn, src, C, out, noise_std, key, layer_id, step_lo, status); break;
+      case 2: st = reduce_tma_launch<2>(stream, gs, mn, src, C, out, noise_std, key, layer_id, step_lo, status); break;
+      case 3: st = reduce_tma_launch<3>(stream, gs, mn, src, C, out, noise_std, key, layer_id, step_lo, status); break;
+      case 4: st = reduce_tma_launch<4>(stream, gs, mn, src, C, out, noise_std, key, layer_id, step_lo, status); break;
+      case 5: st = reduce_tma_launch<5>(stream, gs, mn, src, C, out, noise_std, key, layer_id, step_lo, status); break;
+      case 6: st = reduce_tma_launch<6>(stream, gs, mn, src, C, out, noise_std, key, layer_id, step_lo, status); break;
+      case 7: st = reduce_tma_launch<7>(stream, gs, mn, src, C, out, noise_std, key, layer_id, step_lo, status); break;
+      default: st = reduce_tma_launch<8>(stream, gs, mn, src, C, out, noise_std, key, layer_id, step_lo, status); break;
+    }
+    if (st != DP_OK) return st;
+    DP_CHECK_LAUNCH("clip_reduce_tma_kernel");
+    return DP_OK;
+  }
   const int cached = B < kReduceCachedSamples ? B : kReduceCachedSamples;
-  const int grid = stream_grid(static_cast<unsigned long long>(mn / 8), 256);
-  const size_t smem = cached * sizeof(float);
+  const int grid = std::min(stream_grid(static_cast<unsigned long long>(mn / 8), 256), sm_count() * 2);
+  const size_t smem = kNoiseSharedBytes + cached * sizeof(float);
   const PhiloxKey key = philox_key_from_seed(seed);
   const uint32_t step_lo = static_cast<uint32_t>(step & 0xFFFFFFFFull);
   LaunchScope scope(kKindReduce, stream);
@@ -602,6 +681,235 @@ dp_status resolve_method(const Shape& s, dp_norm_method method, dp_norm_method* 
   return DP_OK;
 }
 
+// ---------------------------------------------------------------- block step
+// One call for the linears of a block.  Linears that read the same X with the same shape and
+// take the ghost norm are grouped (up to three: q/k/v, gate/up), and one X Gram per
+// token-block pair serves the whole group.  Every other linear is a group of one.
+//
+// Workspace: one status word; the flat squared norms [B]; every layer's squared norms [L][B]
+// (fp64 slots, fp32 used for bf16); c[B]; the norm partial slots (three sets when some group
+// shares an X Gram) and the scaled-operand copy, each sized for the largest layer; and the
+// bf16 per-sample tiles of the gradients-once layers.  Flat clipping needs every such layer's
+// tiles at once; per-layer clipping finishes each layer before the next, so one region sized
+// for the largest serves them all.
+struct BlockLayout {
+  size_t flat = 0, norm2 = 0, c = 0, partials = 0, scaled = 0, total = 0;
+  int partial_stride = 0;
+  long long partial_op_stride = 0;       // floats between the partial sets of a shared group
+  std::vector<size_t> tiles;             // per layer; 0 when the layer does not keep tiles
+  std::vector<dp_norm_method> methods;   // resolved per layer
+  std::vector<std::vector<int>> groups;  // layers in call order, grouped as described above
+};
+
+Shape layer_shape(const dp_layer& l, int B, int T, dp_dtype dt) { return Shape{B, T, l.d_in, l.d_out, 0, dt}; }
+
+dp_status block_methods(const dp_layer* layers, int L, int B, int T, dp_dtype dt, dp_norm_method method,
+                        std::vector<dp_norm_method>* out) {
+  out->clear();
+  for (int l = 0; l < L; ++l) {
+    const Shape s = layer_shape(layers[l], B, T, dt);
+    if (!valid_shape(s)) return DP_ERR_INVALID_ARG;
+    dp_norm_method m;
+    dp_status st = resolve_method(s, method, &m);
+    if (st != DP_OK) return st;
+    out->push_back(m);
+  }
+  return DP_OK;
+}
+
+std::vector<std::vector<int>> block_groups(const dp_layer* layers, int L, dp_dtype dt,
+                                           const std::vector<dp_norm_method>& methods) {
+  std::vector<std::vector<int>> groups;
+  std::vector<bool> taken(L, false);
+  for (int l = 0; l < L; ++l) {
+    if (taken[l]) continue;
+    groups.push_back({l});
+    taken[l] = true;
+    if (dt != DP_BF16 || methods[l] != DP_NORM_GHOST) continue;
+    for (int j = l + 1; j < L && static_cast<int>(groups.back().size()) < kGhostSharedMaxOps; ++j) {
+      if (!taken[j] && methods[j] == DP_NORM_GHOST && layers[j].X == layers[l].X &&
+          layers[j].d_in == layers[l].d_in && layers[j].d_out == layers[l].d_out) {
+        groups.back().push_back(j);
+        taken[j] = true;
+      }
+    }
+  }
+  return groups;
+}
+
+BlockLayout block_layout(const dp_layer* layers, int L, int B, int T, dp_dtype dt, dp_clip_mode mode,
+                         const std::vector<dp_norm_method>& methods) {
+  BlockLayout Lb;
+  Lb.methods = methods;
+  Lb.groups = block_groups(layers, L, dt, methods);
+  size_t off = 256;
+  Lb.flat = off;
+  off += align256(static_cast<size_t>(B) * 8);
+  Lb.norm2 = off;
+  off += align256(static_cast<size_t>(L) * B * 8);
+  Lb.c = off;
+  off += align256(static_cast<size_t>(B) * 4);
+  size_t scaled = 0, tiles_most = 0;
+  for (int l = 0; l < L; ++l) {
+    const Shape s = layer_shape(layers[l], B, T, dt);
+    if (dt == DP_BF16) {
+      const int ps = partial_slots(s);
+      if (ps > Lb.partial_stride) Lb.partial_stride = ps;
+      const size_t sc = static_cast<size_t>(s.N()) * static_cast<size_t>(s.m < s.n ? s.m : s.n) * 2;
+      if (methods[l] != DP_NORM_ONCE && sc > scaled) scaled = sc;
+      if (methods[l] == DP_NORM_ONCE)
+        tiles_most = std::max(tiles_most, static_cast<size_t>(B) * layers[l].d_in * layers[l].d_out * 2);
+    }
+  }
+  int sets = 1;
+  for (const auto& g : Lb.groups) sets = std::max(sets, static_cast<int>(g.size()));
+  Lb.partial_op_stride = static_cast<long long>(align256(static_cast<size_t>(B) * Lb.partial_stride * 4) / 4);
+  Lb.partials = off;
+  off += static_cast<size_t>(sets) * Lb.partial_op_stride * 4;
+  Lb.scaled = off;
+  off += align256(scaled);
+  Lb.tiles.assign(L, 0);
+  if (mode == DP_CLIP_PER_LAYER) {
+    if (tiles_most) {
+      for (int l = 0; l < L; ++l)
+        if (dt == DP_BF16 && methods[l] == DP_NORM_ONCE) Lb.tiles[l] = off;
+      off += align256(tiles_most);
+    }
+  } else {
+    for (int l = 0; l < L; ++l) {
+      if (dt == DP_BF16 && methods[l] == DP_NORM_ONCE) {
+        Lb.tiles[l] = off;
+        off += align256(static_cast<size_t>(B) * layers[l].d_in * layers[l].d_out * 2);
+      }
+    }
+  }
+  Lb.total = off;
+  return Lb;
+}
+
+// Squared norms of the layers of one group into their [B] rows of the norm2 block, and each
+// layer's norms_out when given (gradients-once layers also keep their tiles).
+dp_status block_group_norms(const dp_layer* layers, const std::vector<int>& g, dp_dtype dt, int B, int T,
+                            const BlockLayout& Lb, uint8_t* ws, cudaStream_t stream) {
+  dp_status st;
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws);
+  const dp_layer& y0 = layers[g[0]];
+  const Shape s = layer_shape(y0, B, T, dt);
+  if (dt == DP_F32) {
+    double* n2 = reinterpret_cast<double*>(ws + Lb.norm2) + static_cast<size_t>(g[0]) * B;
+    dim3 grid(ceil_div(s.n, kF32Tile), ceil_div(s.m, kF32Tile), B);
+    {
+      LaunchScope scope(kKindF32Norm, stream);
+      f32_norm_kernel<<<grid, 256, 0, stream>>>(static_cast<const float*>(y0.X), static_cast<const float*>(y0.dY),
+                                                 T, s.m, s.n, n2);
+      DP_CHECK_LAUNCH("f32_norm_kernel");
+    }
+    if (y0.norms_out) {
+      NormSource src{nullptr, n2, nullptr};
+      if ((st = launch_finalize(src, B, INFINITY, y0.norms_out, nullptr, stream)) != DP_OK) return st;
+    }
+    return DP_OK;
+  }
+  float* partials = reinterpret_cast<float*>(ws + Lb.partials);
+  int count = 0;
+  if (g.size() > 1) {
+    const void* Zs[kGhostSharedMaxOps] = {};
+    for (size_t j = 0; j < g.size(); ++j) Zs[j] = layers[g[j]].dY;
+    if ((st = bf16_norms_ghost_shared(s, y0.X, Zs, static_cast<int>(g.size()), partials, Lb.partial_stride,
+                                      Lb.partial_op_stride, &count, status, stream)) != DP_OK)
+      return st;
+  } else {
+    const bool once = (Lb.methods[g[0]] == DP_NORM_ONCE);
+    if ((st = bf16_norms(s, y0.X, y0.dY, once ? DP_NORM_EXPLICIT : Lb.methods[g[0]], partials,
+                         Lb.partial_stride, &count, status, stream,
+                         once ? reinterpret_cast<__nv_bfloat16*>(ws + Lb.tiles[g[0]]) : nullptr)) != DP_OK)
+      return st;
+  }
+  for (size_t j = 0; j < g.size(); ++j) {
+    const dp_layer& y = layers[g[j]];
+    float* n2 = reinterpret_cast<float*>(ws + Lb.norm2) + static_cast<size_t>(g[j]) * B;
+    if ((st = launch_norm_partials(partials + j * Lb.partial_op_stride, Lb.partial_stride, count, B, INFINITY,
+                                   n2, y.norms_out, nullptr, stream)) != DP_OK)
+      return st;
+  }
+  return DP_OK;
+}
+
+// Layer l's clipped sum with the clip factors of `src` and bound C, plus noise of std sigma C.
+dp_status block_layer_sum(const dp_layer* layers, int l, dp_dtype dt, int B, int T, NormSource src, float C,
+                          float sigma, unsigned long long seed, unsigned long long step, const BlockLayout& Lb,
+                          uint8_t* ws, cudaStream_t stream) {
+  const dp_layer& y = layers[l];
+  const Shape s = layer_shape(y, B, T, dt);
+  const double noise_std = (sigma == 0.0f) ? 0.0 : static_cast<double>(sigma) * static_cast<double>(C);
+  if (dt == DP_BF16 && Lb.methods[l] == DP_NORM_ONCE)
+    return launch_reduce(reinterpret_cast<const __nv_bfloat16*>(ws + Lb.tiles[l]), B,
+                         static_cast<long long>(s.m) * s.n, src, C, y.G_out, noise_std, seed, step, y.layer_id,
+                         stream, reinterpret_cast<uint32_t*>(ws));
+  Call c;
+  c.s = s;
+  c.L = WsLayout();
+  c.L.scaled = Lb.scaled;
+  c.ws = ws;
+  c.stream = stream;
+  return clipped_sum(c, y.X, y.dY, src, C, y.G_out, 0, noise_std, seed, step, y.layer_id);
+}
+
+NormSource layer_norm_source(const BlockLayout& Lb, uint8_t* ws, int l, int B, dp_dtype dt) {
+  NormSource src{nullptr, nullptr, nullptr};
+  if (dt == DP_F32)
+    src.norm2_f64 = reinterpret_cast<double*>(ws + Lb.norm2) + static_cast<size_t>(l) * B;
+  else
+    src.norm2_f32 = reinterpret_cast<float*>(ws + Lb.norm2) + static_cast<size_t>(l) * B;
+  return src;
+}
+
+dp_status block_step(const dp_layer* layers, int L, dp_dtype dt, int B, int T, dp_clip_mode mode, float C,
+                     float sigma, unsigned long long seed, unsigned long long step, const BlockLayout& Lb,
+                     float* flat_norms_out, uint8_t* ws, cudaStream_t stream) {
+  dp_status st;
+  // Status word, and the fp32 path's atomic norm accumulators, start at zero.
+  DP_CUDA(cudaMemsetAsync(ws, 0, Lb.c, stream));
+  if (mode == DP_CLIP_PER_LAYER) {
+    // Each group: its norms, then each member's clipped sum with its own bound and noise.
+    for (const auto& g : Lb.groups) {
+      if ((st = block_group_norms(layers, g, dt, B, T, Lb, ws, stream)) != DP_OK) return st;
+      for (int l : g) {
+        const NormSource src = layer_norm_source(Lb, ws, l, B, dt);
+        if ((st = block_layer_sum(layers, l, dt, B, T, src, layers[l].C, sigma, seed, step, Lb, ws, stream)) !=
+            DP_OK)
+          return st;
+      }
+    }
+    return DP_OK;
+  }
+  // 1. Every layer's per-sample norms (gradients-once layers also keep their tiles).
+  for (const auto& g : Lb.groups)
+    if ((st = block_group_norms(layers, g, dt, B, T, Lb, ws, stream)) != DP_OK) return st;
+  // 2. The flat squared norms, summed over the layers in order.
+  NormSource src{nullptr, nullptr, nullptr};
+  {
+    LaunchScope scope(kKindFinalize, stream);
+    if (dt == DP_F32) {
+      double* flat = reinterpret_cast<double*>(ws + Lb.flat);
+      flat_norm2_kernel<double><<<ceil_div(B, 256), 256, 0, stream>>>(
+          reinterpret_cast<const double*>(ws + Lb.norm2), L, B, flat, flat_norms_out);
+      src.norm2_f64 = flat;
+    } else {
+      float* flat = reinterpret_cast<float*>(ws + Lb.flat);
+      flat_norm2_kernel<float><<<ceil_div(B, 256), 256, 0, stream>>>(
+          reinterpret_cast<const float*>(ws + Lb.norm2), L, B, flat, flat_norms_out);
+      src.norm2_f32 = flat;
+    }
+    DP_CHECK_LAUNCH("flat_norm2_kernel");
+  }
+  // 3. Every layer's clipped sum with the shared clip factors, plus its own noise.
+  for (int l = 0; l < L; ++l)
+    if ((st = block_layer_sum(layers, l, dt, B, T, src, C, sigma, seed, step, Lb, ws, stream)) != DP_OK)
+      return st;
+  return DP_OK;
+}
+
 // ---------------------------------------------------------------- allocation-free norms
 // Scratch of dp_per_sample_norms_static: a fixed device array instead of a caller workspace.
 // Every GPU that loads this library holds these 1 MiB until the process exits.
@@ -743,7 +1051,7 @@ dp_status dp_linear_step(const void* X, const void* dY, const void* P, int r, dp
     return st;
   if (once)
     return launch_reduce(reinterpret_cast<const __nv_bfloat16*>(c.ws + c.L.gs), B, mn, src, C, G_out,
-                         noise_std, seed, step, layer_id, c.stream);
+                         noise_std, seed, step, layer_id, c.stream, c.status());
   return clipped_sum(c, X, Z, src, C, G_out, 0, noise_std, seed, step, layer_id);
 }
 
@@ -805,6 +1113,104 @@ dp_status dp_per_sample_norms_static(const void* X, const void* dY, dp_dtype dt,
   int count = 0;
   if ((st = bf16_norms(s, X, dY, m, partials, stride, &count, status, cs)) != DP_OK) return st;
   return launch_norm_partials(partials, stride, count, B, INFINITY, norm2, norms, nullptr, cs);
+}
+
+size_t dp_block_workspace_size(const dp_layer* layers, int L, int B, int T, dp_dtype dt,
+                               dp_clip_mode mode, dp_norm_method method) {
+  if (!layers || L < 1) return 0;
+  std::vector<dp_norm_method> methods;
+  if (method < DP_NORM_AUTO || method > DP_NORM_ONCE) return 0;
+  if (mode != DP_CLIP_PER_LAYER && mode != DP_CLIP_FLAT) return 0;
+  if (block_methods(layers, L, B, T, dt, method, &methods) != DP_OK) return 0;
+  return block_layout(layers, L, B, T, dt, mode, methods).total;
+}
+
+dp_status dp_block_step(const dp_layer* layers, int L, dp_dtype dt, int B, int T, dp_clip_mode mode,
+                        float C, float sigma, unsigned long long seed, unsigned long long step,
+                        dp_norm_method method, float* flat_norms_out, void* workspace, size_t ws_bytes,
+                        void* stream) {
+  if (!layers || L < 1 || !workspace) return DP_ERR_INVALID_ARG;
+  if (mode != DP_CLIP_PER_LAYER && mode != DP_CLIP_FLAT) return DP_ERR_INVALID_ARG;
+  if (method < DP_NORM_AUTO || method > DP_NORM_ONCE) return DP_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return DP_ERR_INVALID_ARG;
+  if (!(sigma >= 0.0f) || std::isinf(sigma)) return DP_ERR_INVALID_ARG;
+  for (int l = 0; l < L; ++l) {
+    const dp_layer& y = layers[l];
+    if (!y.X || !y.dY || !y.G_out || !aligned16(y.X) || !aligned16(y.dY) || !aligned16(y.G_out))
+      return DP_ERR_INVALID_ARG;
+    if (mode == DP_CLIP_PER_LAYER && (!(y.C > 0.0f) || (std::isinf(y.C) && sigma != 0.0f)))
+      return DP_ERR_INVALID_ARG;
+  }
+  std::vector<dp_norm_method> methods;
+  dp_status st = block_methods(layers, L, B, T, dt, method, &methods);
+  if (st != DP_OK) return st;
+  if (mode == DP_CLIP_FLAT && (!(C > 0.0f) || (std::isinf(C) && sigma != 0.0f))) return DP_ERR_INVALID_ARG;
+  const BlockLayout Lb = block_layout(layers, L, B, T, dt, mode, methods);
+  if (ws_bytes < Lb.total) return DP_ERR_WORKSPACE;
+  if (dt == DP_BF16 && (st = get_encoder()) != DP_OK) return st;
+  return block_step(layers, L, dt, B, T, mode, C, sigma, seed, step, Lb, flat_norms_out,
+                    static_cast<uint8_t*>(workspace), static_cast<cudaStream_t>(stream));
+}
+
+size_t dp_adam_workspace_size(int d_in, int r) {
+  if (d_in < 1 || r < 1 || r % 8) return 0;
+  return 256 + align256(static_cast<size_t>(d_in) * r * 2);
+}
+
+dp_status dp_projected_adam_step(float* W, const float* R, float* m, float* v, const void* P, dp_dtype dt,
+                                 int d_in, int d_out, int r, float lr, float beta1, float beta2, float eps,
+                                 float grad_scale, int t, void* workspace, size_t ws_bytes, void* stream) {
+  if (!W || !R || !m || !v || !P || !workspace) return DP_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(R) || !aligned16(m) || !aligned16(v) || !aligned16(P)) return DP_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return DP_ERR_INVALID_ARG;
+  if (!valid_dtype(dt)) return DP_ERR_INVALID_ARG;
+  if (d_in < 1 || d_out < 1 || r < 1 || d_in % 8 || d_out % 8 || r % 8) return DP_ERR_INVALID_ARG;
+  if (static_cast<long long>(d_in) * d_out > (1ll << 34)) return DP_ERR_INVALID_ARG;
+  if (t < 1 || !(lr >= 0.0f) || std::isinf(lr) || !(beta1 >= 0.0f && beta1 < 1.0f) ||
+      !(beta2 >= 0.0f && beta2 < 1.0f) || !(eps >= 0.0f) || std::isinf(grad_scale) || grad_scale != grad_scale)
+    return DP_ERR_INVALID_ARG;
+  if (dt != DP_BF16) return DP_ERR_UNSUPPORTED;  // the back-projection runs on bf16 tensor cores
+  if (ws_bytes < dp_adam_workspace_size(d_in, r)) return DP_ERR_WORKSPACE;
+  dp_status st;
+  if ((st = get_encoder()) != DP_OK) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  DP_CUDA(cudaMemsetAsync(ws, 0, 256, cs));  // status word
+  __nv_bfloat16* U = reinterpret_cast<__nv_bfloat16*>(ws + 256);
+  const long long n = static_cast<long long>(d_in) * r;
+  const float bc1 = 1.0f - static_cast<float>(std::pow(static_cast<double>(beta1), t));
+  const float bc2 = 1.0f - static_cast<float>(std::pow(static_cast<double>(beta2), t));
+  {
+    LaunchScope scope(kKindAdam, cs);
+    adam_rspace_kernel<<<stream_grid(static_cast<unsigned long long>(n / 4), 256), 256, 0, cs>>>(
+        R, m, v, U, n, grad_scale, beta1, beta2, eps, bc1, bc2);
+    DP_CHECK_LAUNCH("adam_rspace_kernel");
+  }
+  if (lr == 0.0f) return DP_OK;
+  UmmaParams p = base_params(reinterpret_cast<uint32_t*>(ws));
+  if ((st = map_2d(&p.tmA0, U, d_in, r, 128)) != DP_OK) return st;
+  if ((st = map_2d(&p.tmB0, P, d_out, r, 256)) != DP_OK) return st;
+  p.m_tiles = ceil_div(d_in, 128);
+  p.n_tiles = ceil_div(d_out, 256);
+  p.k_blocks = ceil_div(r, 64);
+  p.k_blocks_per_split = p.k_blocks;
+  p.k_splits = 1;
+  p.num_units = p.m_tiles * p.n_tiles;
+  p.out_rows = d_in;
+  p.out_cols = d_out;
+  p.out_f32 = W;
+  p.alpha = -lr;
+  return launch_umma<UmmaConfig<256, kEpiAxpy>>(p, cs);
+}
+
+dp_status dp_selftest_wait_timeout(void* workspace, unsigned long long limit_ns, void* stream) {
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return DP_ERR_INVALID_ARG;
+  if (limit_ns < 1000ull || limit_ns > kWaitLimitNs) return DP_ERR_INVALID_ARG;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  DP_CUDA(cudaMemsetAsync(workspace, 0, 256, cs));
+  wait_timeout_selftest_kernel<<<1, 32, 0, cs>>>(static_cast<uint32_t*>(workspace), limit_ns);
+  DP_CHECK_LAUNCH("wait_timeout_selftest_kernel");
+  return DP_OK;
 }
 
 dp_status dp_workspace_status(const void* workspace, void* stream) {

@@ -28,6 +28,9 @@ enum KernelKind : int {
   kKindProject,       // tcgen05 Z = dY P
   kKindExplicitStore, // tcgen05 per-sample G_i tiles, squared on chip and stored in bf16
   kKindReduce,        // sum_i c_i G_i over the stored tiles + noise
+  kKindAdam,          // projected Adam moments and update in r-space
+  kKindAxpy,          // tcgen05 W += alpha U P^T
+  kKindGhostShared,   // tcgen05 one X Gram shared by the dY Grams of up to three linears
   kNumKinds
 };
 
@@ -35,7 +38,8 @@ inline const char* kernel_kind_name(int k) {
   static const char* names[kNumKinds] = {
       "noise_add",  "projection",   "philox_blocks", "scale_rows_bf16", "finalize_norms",
       "f32_norm",   "f32_clipsum",  "f32_project",   "umma_clipsum",    "umma_explicit_norm",
-      "umma_ghost_norm", "umma_project", "umma_explicit_store", "clip_reduce"};
+      "umma_ghost_norm", "umma_project", "umma_explicit_store", "clip_reduce", "adam_rspace",
+      "umma_axpy", "umma_ghost_shared"};
   return (k >= 0 && k < kNumKinds) ? names[k] : "";
 }
 

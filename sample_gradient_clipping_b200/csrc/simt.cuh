@@ -9,19 +9,32 @@
 #include <cuda_bf16.h>
 
 #include <cstdint>
+#include <type_traits>
 
+#include "ptx.cuh"
 #include "rng.cuh"
 
 namespace dpclip {
 
 // G[k] = fp32(G[k] + std * z_k), z from stream 0.  One thread per Philox block of 4 elements.
+// STAGED: the Box-Muller tables are copied to shared memory once per block (large G); else
+// they are read through the read-only cache, which saves the copy's latency on small G.
+template <bool STAGED>
 __global__ void noise_add_kernel(float* __restrict__ G, unsigned long long total, double std_dev,
                                  PhiloxKey key, uint32_t layer_id, uint32_t step_lo) {
+  __shared__ double2 tab_s[STAGED ? kNoiseSharedEntries : 1];
+  if constexpr (STAGED) {
+    stage_noise_tables(tab_s);
+    __syncthreads();
+  }
+  using Tab = typename std::conditional<STAGED, NoiseTablesShared, NoiseTablesGlobal>::type;
+  Tab tab;
+  if constexpr (STAGED) tab = NoiseTablesShared{tab_s};
   const unsigned long long nblk = (total + 3) / 4;
   for (unsigned long long j = blockIdx.x * static_cast<unsigned long long>(blockDim.x) + threadIdx.x;
        j < nblk; j += static_cast<unsigned long long>(gridDim.x) * blockDim.x) {
     double z[4];
-    normals4(static_cast<uint32_t>(j), layer_id, step_lo, kStreamNoise, key, z);
+    normals4(static_cast<uint32_t>(j), layer_id, step_lo, kStreamNoise, key, z, tab);
     const unsigned long long k0 = 4 * j;
     if (k0 + 3 < total) {
       float4* p = reinterpret_cast<float4*>(G + k0);
@@ -56,7 +69,7 @@ __global__ void projection_kernel(void* __restrict__ P, unsigned long long total
   for (unsigned long long j = blockIdx.x * static_cast<unsigned long long>(blockDim.x) + threadIdx.x;
        j < nblk; j += static_cast<unsigned long long>(gridDim.x) * blockDim.x) {
     double z[4];
-    normals4(static_cast<uint32_t>(j), layer_id, 0u, kStreamProjection, key, z);
+    normals4_precise(static_cast<uint32_t>(j), layer_id, 0u, kStreamProjection, key, z);
     float f[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) f[q] = static_cast<float>(z[q] / scale);
@@ -127,6 +140,20 @@ __global__ void reduce_norm_partials_kernel(const float* __restrict__ partials, 
   }
 }
 
+// flat[i] = sum_l norm2[l][i] over the L layers of a block, in layer order (fp64), and
+// flat_norms_out[i] = sqrt(flat[i]) when given: the squared norm of each sample's gradient
+// over all the block's weights.
+template <typename T>
+__global__ void flat_norm2_kernel(const T* __restrict__ norm2_layers, int L, int B, T* __restrict__ flat,
+                                  float* __restrict__ flat_norms_out) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < B; i += gridDim.x * blockDim.x) {
+    double acc = 0.0;
+    for (int l = 0; l < L; ++l) acc += static_cast<double>(norm2_layers[static_cast<long long>(l) * B + i]);
+    flat[i] = static_cast<T>(acc);
+    if (flat_norms_out) flat_norms_out[i] = static_cast<float>(sqrt(acc));
+  }
+}
+
 // norms_out[i] = n_i and c_out[i] = c_i for i < B (either may be null).
 __global__ void finalize_norms_kernel(NormSource src, int B, float C, float* __restrict__ norms_out,
                                       float* __restrict__ c_out) {
@@ -165,17 +192,22 @@ __global__ void scale_rows_bf16_kernel(const __nv_bfloat16* __restrict__ in,
 // explicit-store pass left in the workspace: the clipped sum without forming any G_i again.
 //
 // Each thread owns 8 consecutive elements: two Philox blocks and four independent fp64
-// Box-Muller pairs.  The loads of all samples are issued first (for B <= kReduceUnrolled the
+// Box-Muller pairs.  The noise sigma C z is rounded to fp32 once and added to the fp32 sum
+// (one conversion an element instead of two; the result is within 1 ulp of the fp64 sum
+// rounded once).  The loads of all samples are issued first (for B <= kReduceUnrolled the
 // loop is unrolled), the noise is computed while they are in flight, and then the sum is
 // formed.  This keeps both the fp64 pipe and HBM busy instead of alternating between them.
 template <int BU>  // compile-time sample count, or 0 for a runtime loop
 __global__ void __launch_bounds__(256, 2) clip_reduce_kernel(
     const __nv_bfloat16* __restrict__ Gs, int B, long long mn, NormSource src, float C,
     float* __restrict__ out, double noise_std, PhiloxKey key, uint32_t layer_id, uint32_t step_lo) {
-  extern __shared__ float c_smem[];
+  extern __shared__ double2 reduce_smem[];  // noise tables, then the cached clip factors
+  float* c_smem = reinterpret_cast<float*>(reduce_smem + kNoiseSharedEntries);
   const int cached = B < kReduceCachedSamples ? B : kReduceCachedSamples;
   for (int i = threadIdx.x; i < cached; i += blockDim.x) c_smem[i] = clip_factor(src.norm(i), C);
+  if (noise_std != 0.0) stage_noise_tables(reduce_smem);
   __syncthreads();
+  const NoiseTablesShared tab{reduce_smem};
   const long long nvec = mn / 8;  // 16-byte vectors per sample
   const long long v0 = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x;
   uint4 pk_next[BU > 0 ? BU : 1];
@@ -207,9 +239,9 @@ __global__ void __launch_bounds__(256, 2) clip_reduce_kernel(
       }
       if (noise_std != 0.0) {
         normals4(static_cast<uint32_t>(2 * v), layer_id, step_lo, kStreamNoise, key,
-                 *reinterpret_cast<double(*)[4]>(z));
+                 *reinterpret_cast<double(*)[4]>(z), tab);
         normals4(static_cast<uint32_t>(2 * v + 1), layer_id, step_lo, kStreamNoise, key,
-                 *reinterpret_cast<double(*)[4]>(z + 4));
+                 *reinterpret_cast<double(*)[4]>(z + 4), tab);
       }
 #pragma unroll
       for (int i = 0; i < BU; ++i) {
@@ -236,19 +268,184 @@ __global__ void __launch_bounds__(256, 2) clip_reduce_kernel(
       }
       if (noise_std != 0.0) {
         normals4(static_cast<uint32_t>(2 * v), layer_id, step_lo, kStreamNoise, key,
-                 *reinterpret_cast<double(*)[4]>(z));
+                 *reinterpret_cast<double(*)[4]>(z), tab);
         normals4(static_cast<uint32_t>(2 * v + 1), layer_id, step_lo, kStreamNoise, key,
-                 *reinterpret_cast<double(*)[4]>(z + 4));
+                 *reinterpret_cast<double(*)[4]>(z + 4), tab);
       }
     }
     if (noise_std != 0.0) {
 #pragma unroll
-      for (int q = 0; q < 8; ++q) acc[q] = static_cast<float>(static_cast<double>(acc[q]) + noise_std * z[q]);
+      for (int q = 0; q < 8; ++q) acc[q] = acc[q] + __double2float_rn(noise_std * z[q]);
     }
     float4* o = reinterpret_cast<float4*>(out) + 2 * v;
     o[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
     o[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
   }
+}
+
+// Warp-specialised variant of clip_reduce_kernel for B <= 8 samples.
+//   warp 0      : one lane streams chunks of kReduceChunk elements of every sample's bf16
+//                 tiles into a ring of shared-memory stages with 1-D bulk async copies;
+//   warps 1..23 : each thread owns 8 consecutive elements of a chunk.  It first computes
+//                 their fp64 noise, which needs no data, then waits for the stage, forms
+//                 sum_i c_i G_i from shared memory, adds the noise and stores fp32.
+// The copies are issued by one thread with a few instructions each, so HBM stays busy while
+// the compute warps saturate the fp64 pipe.  Waits are bounded as in the tensor-core engine.
+constexpr int kReduceComputeWarps = 23;  // 24 warps at 80 registers fill the register file
+constexpr int kReduceChunk = 8 * 32 * kReduceComputeWarps;
+
+template <int BU>
+struct ReduceTmaConfig {
+  static constexpr int STAGE_BYTES = BU * kReduceChunk * 2;
+  static constexpr int STAGES = (196608 / STAGE_BYTES) < 8 ? (196608 / STAGE_BYTES) : 8;
+  static constexpr int THREADS = 32 * (1 + kReduceComputeWarps);
+  static constexpr int TABLE_OFFSET = STAGES * STAGE_BYTES + 256;  // after the barriers
+  static constexpr int SMEM_BYTES = 1024 + TABLE_OFFSET + kNoiseSharedBytes;
+  static_assert(SMEM_BYTES <= 232448, "dynamic shared memory per block");
+  static_assert(kReduceChunk == 8 * 32 * kReduceComputeWarps, "8 elements per compute thread");
+};
+
+template <int BU>
+__global__ void __launch_bounds__(ReduceTmaConfig<BU>::THREADS, 1) clip_reduce_tma_kernel(
+    const __nv_bfloat16* __restrict__ Gs, long long mn, NormSource src, float C, float* __restrict__ out,
+    double noise_std, PhiloxKey key, uint32_t layer_id, uint32_t step_lo, uint32_t* status) {
+  using Cfg = ReduceTmaConfig<BU>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Cfg::STAGES * Cfg::STAGE_BYTES);
+  uint64_t* empty = full + Cfg::STAGES;
+  float* c_s = reinterpret_cast<float*>(empty + Cfg::STAGES);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(c_s + 8);
+  const int warp = threadIdx.x / 32;
+  const uint32_t lane = lane_id();
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < Cfg::STAGES; ++s) {
+      mbar_init(smem_addr(full + s), 1);
+      mbar_init(smem_addr(empty + s), kReduceComputeWarps);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (threadIdx.x < BU) c_s[threadIdx.x] = clip_factor(src.norm(threadIdx.x), C);
+  double2* tab_s = reinterpret_cast<double2*>(smem + Cfg::TABLE_OFFSET);
+  if (noise_std != 0.0) stage_noise_tables(tab_s);
+  __syncthreads();
+  const NoiseTablesShared tab{tab_s};
+  const long long chunks = (mn + kReduceChunk - 1) / kReduceChunk;
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      for (long long ch = blockIdx.x; ch < chunks; ch += gridDim.x) {
+        if (!mbar_wait_bounded(smem_addr(empty + stage), phase ^ 1u, abort_flag, status, 21u)) break;
+        const long long e0 = ch * kReduceChunk;
+        const long long n = (mn - e0) < kReduceChunk ? (mn - e0) : kReduceChunk;  // multiple of 8
+        const uint32_t bytes = static_cast<uint32_t>(n * 2);
+        const uint32_t bar = smem_addr(full + stage);
+        mbar_arrive_expect_tx(bar, BU * bytes);
+        const uint32_t dst = smem_addr(smem + stage * Cfg::STAGE_BYTES);
+#pragma unroll
+        for (int i = 0; i < BU; ++i)
+          bulk_load(dst + i * kReduceChunk * 2, Gs + static_cast<long long>(i) * mn + e0, bytes, bar);
+        if (++stage == Cfg::STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+  } else {
+    const int t = threadIdx.x - 32;  // 0 .. 32 * kReduceComputeWarps - 1
+    int stage = 0;
+    uint32_t phase = 0;
+    for (long long ch = blockIdx.x; ch < chunks; ch += gridDim.x) {
+      const long long e = ch * kReduceChunk + 8 * t;  // first of this thread's 8 elements
+      double z[8];
+      if (noise_std != 0.0 && e < mn) {
+        normals4(static_cast<uint32_t>(e >> 2), layer_id, step_lo, kStreamNoise, key,
+                 *reinterpret_cast<double(*)[4]>(z), tab);
+        normals4(static_cast<uint32_t>((e >> 2) + 1), layer_id, step_lo, kStreamNoise, key,
+                 *reinterpret_cast<double(*)[4]>(z + 4), tab);
+      }
+      if (!mbar_wait_bounded(smem_addr(full + stage), phase, abort_flag, status, 22u)) break;
+      if (e < mn) {
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        const uint8_t* base = smem + stage * Cfg::STAGE_BYTES + 16 * t;
+#pragma unroll
+        for (int i = 0; i < BU; ++i) {
+          const uint4 pk = *reinterpret_cast<const uint4*>(base + i * kReduceChunk * 2);
+          const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&pk);
+          const float c = c_s[i];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float2 f = __bfloat1622float2(hv[q]);
+            acc[2 * q] = fmaf(c, f.x, acc[2 * q]);
+            acc[2 * q + 1] = fmaf(c, f.y, acc[2 * q + 1]);
+          }
+        }
+        if (noise_std != 0.0) {
+#pragma unroll
+          for (int q = 0; q < 8; ++q) acc[q] = acc[q] + __double2float_rn(noise_std * z[q]);
+        }
+        float4* o = reinterpret_cast<float4*>(out + e);
+        o[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        o[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_addr(empty + stage));
+      if (++stage == Cfg::STAGES) {
+        stage = 0;
+        phase ^= 1u;
+      }
+    }
+  }
+  __syncthreads();
+}
+
+// Projected Adam in r-space: g = scale R; m <- b1 m + (1 - b1) g; v <- b2 v + (1 - b2) g^2;
+// U = (m / bc1) / (sqrt(v / bc2) + eps), written in bf16 for the tensor-core back-projection
+// (bc1 = 1 - b1^t, bc2 = 1 - b2^t).  Four elements per thread.
+__global__ void adam_rspace_kernel(const float* __restrict__ R, float* __restrict__ m, float* __restrict__ v,
+                                   __nv_bfloat16* __restrict__ U, long long n, float scale, float b1, float b2,
+                                   float eps, float bc1, float bc2) {
+  for (long long q = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; 4 * q < n;
+       q += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const float4 r4 = reinterpret_cast<const float4*>(R)[q];
+    float4 m4 = reinterpret_cast<float4*>(m)[q];
+    float4 v4 = reinterpret_cast<float4*>(v)[q];
+    const float gr[4] = {r4.x, r4.y, r4.z, r4.w};
+    float* mm = &m4.x;
+    float* vv = &v4.x;
+    float u[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float g = scale * gr[e];
+      mm[e] = fmaf(b1, mm[e], (1.0f - b1) * g);
+      vv[e] = fmaf(b2, vv[e], (1.0f - b2) * g * g);
+      u[e] = (mm[e] / bc1) / (sqrtf(vv[e] / bc2) + eps);
+    }
+    reinterpret_cast<float4*>(m)[q] = m4;
+    reinterpret_cast<float4*>(v)[q] = v4;
+    __nv_bfloat162 lo = __floats2bfloat162_rn(u[0], u[1]);
+    __nv_bfloat162 hi = __floats2bfloat162_rn(u[2], u[3]);
+    uint2 pk;
+    pk.x = *reinterpret_cast<uint32_t*>(&lo);
+    pk.y = *reinterpret_cast<uint32_t*>(&hi);
+    reinterpret_cast<uint2*>(U)[q] = pk;
+  }
+}
+
+// Failure-detection self-test: one thread waits, with the bounded wait every pipeline uses,
+// on an mbarrier that nothing ever arrives at.  After `limit_ns` the wait gives up, records
+// its site (code 99) in the status word and the kernel returns; the GPU stays usable.
+__global__ void wait_timeout_selftest_kernel(uint32_t* status, unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x != 0) return;
+  abort_flag = 0;
+  mbar_init(smem_addr(&bar), 1);
+  fence_mbar_init();
+  mbar_wait_bounded(smem_addr(&bar), 0u, &abort_flag, status, 99u, limit_ns);
 }
 
 // ------------------------------------------------------------------------------ fp32 path

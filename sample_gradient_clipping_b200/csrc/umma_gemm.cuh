@@ -23,7 +23,12 @@
 //   kEpiStoreBf16    Z = dY P (K-major dY, MN-major P), rounded to bf16;
 //   kEpiExplicitStore as kEpiExplicitNorm, and the tile of G_i is also written to HBM in bf16
 //                    so that the clipped sum reuses it instead of forming G_i again
-//                    (each per-sample gradient is formed once).
+//                    (each per-sample gradient is formed once);
+//   kEpiAxpy         W[a, b] += alpha * sum_k U[a, k] P[b, k] (both K-major): the projected
+//                    optimizer's update mapped back to the weights through P^T;
+//   kEpiGhostShared  the ghost norm of up to three linears that read the same input X (q/k/v,
+//                    gate/up): one X Gram tile and each linear's dY Gram tile in four TMEM
+//                    accumulators, so the X Gram is formed once for the group.
 //
 // All waits are bounded (ptx.cuh); a wait that runs out sets the CTA's abort flag, records
 // its site in the status word and the CTA drains and exits.
@@ -40,8 +45,12 @@ enum EpiKind : int {
   kEpiExplicitNorm = 1,
   kEpiGhostNorm = 2,
   kEpiStoreBf16 = 3,
-  kEpiExplicitStore = 4
+  kEpiExplicitStore = 4,
+  kEpiAxpy = 5,
+  kEpiGhostShared = 6
 };
+
+constexpr int kGhostSharedMaxOps = 3;  // dY operands per shared X Gram (TMEM: 4 x 128 columns)
 
 // K-blocks ahead of the smem ring that the clipped-sum producer asks TMA to pull into L2.
 constexpr int kL2PrefetchDistance = 8;
@@ -63,8 +72,11 @@ struct alignas(64) UmmaParams {
   __nv_bfloat16* out_bf16;
   double noise_std;           // 0 disables the noise
   uint32_t key0, key1, layer_id, step_lo;
+  float alpha;                // axpy: W += alpha * acc
   float* partials;            // [B][partial_stride] per-warp squared-norm partials
   int partial_stride;         // slots per sample: 4 per unit of that sample
+  int ghost_ops;              // shared ghost: dY operands (1..3); phase 1 + k reads operand k
+  long long partial_op_stride;  // shared ghost: floats between the operands' partial arrays
   uint32_t* status;
 };
 
@@ -76,12 +88,15 @@ struct UmmaConfig {
   static constexpr int EPI = EPI_;
   static constexpr bool PER_SAMPLE = (EPI == kEpiExplicitNorm || EPI == kEpiExplicitStore);
   static constexpr bool A_MN = (EPI == kEpiClipSum || PER_SAMPLE);
-  static constexpr bool B_MN = (EPI != kEpiGhostNorm);
+  static constexpr bool GHOST = (EPI == kEpiGhostNorm || EPI == kEpiGhostShared);
+  static constexpr bool B_MN = (!GHOST && EPI != kEpiAxpy);
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = BN * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int STAGES = (196608 / STAGE_BYTES) < 8 ? (196608 / STAGE_BYTES) : 8;
-  static constexpr int ACCS = (EPI == kEpiGhostNorm) ? 2 : 1;  // accumulators per unit
+  static constexpr int ACCS = (EPI == kEpiGhostNorm)     ? 2
+                              : (EPI == kEpiGhostShared) ? 1 + kGhostSharedMaxOps
+                                                         : 1;  // accumulators per unit
   static constexpr int ACC_COLS = BN * ACCS;
   static constexpr int NUM_BUFS = 512 / ACC_COLS;
   static constexpr int THREADS = 192;
@@ -99,7 +114,7 @@ struct Unit {
 template <class Cfg>
 __device__ __forceinline__ Unit decode_unit(const UmmaParams& p, int u) {
   Unit w{};
-  if (Cfg::EPI == kEpiGhostNorm) {
+  if (Cfg::GHOST) {
     w.sample = u / p.pairs_per_sample;
     int r = u % p.pairs_per_sample;
     int row = 0;
@@ -168,6 +183,15 @@ __device__ __forceinline__ void issue_stage_loads(const UmmaParams& p, const Uni
     const CUtensorMap* mb = phase ? &p.tmB1 : &p.tmB0;
     tma_load_3d(sA, ma, bar, k0, w.m_blk * Cfg::BM, w.sample);
     tma_load_3d(sB, mb, bar, k0, w.n_blk * Cfg::BN, w.sample);
+  } else if (Cfg::EPI == kEpiGhostShared) {
+    // Phase 0 reads X (tmA0), phase 1 + k reads dY operand k (tmB0, tmA1, tmB1); both
+    // operands of a Gram tile come from the same map, at the two token blocks of the pair.
+    const CUtensorMap* m = phase == 0 ? &p.tmA0 : phase == 1 ? &p.tmB0 : phase == 2 ? &p.tmA1 : &p.tmB1;
+    tma_load_3d(sA, m, bar, k0, w.m_blk * Cfg::BM, w.sample);
+    tma_load_3d(sB, m, bar, k0, w.n_blk * Cfg::BN, w.sample);
+  } else if (Cfg::EPI == kEpiAxpy) {  // A = U rows, B = P rows, both K-major
+    tma_load_2d(sA, &p.tmA0, bar, k0, w.m_blk * Cfg::BM);
+    tma_load_2d(sB, &p.tmB0, bar, k0, w.n_blk * Cfg::BN);
   } else {  // kEpiStoreBf16: A = dY rows (K-major), B = P (MN-major)
     tma_load_2d(sA, &p.tmA0, bar, k0, w.m_blk * Cfg::BM);
 #pragma unroll
@@ -294,6 +318,64 @@ __device__ __forceinline__ void epilogue_unit(const UmmaParams& p, const Unit& w
     }
     ss = warp_sum(ss);
     if (lane == 0) p.partials[static_cast<long long>(w.sample) * p.partial_stride + 4 * w.local + wq] = ss;
+  } else if (Cfg::EPI == kEpiGhostShared) {
+    const int t = w.m_blk * Cfg::BM + row;
+    float ss[kGhostSharedMaxOps] = {0.f, 0.f, 0.f};
+#pragma unroll 1
+    for (int c0 = 0; c0 < Cfg::BN; c0 += 32) {
+      float gx[32];
+      tmem_ld32(tacc + c0, gx);
+      tmem_ld_wait();
+      const int s0 = w.n_blk * Cfg::BN + c0;
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const int s = s0 + e;
+        gx[e] *= (t < s) ? 2.f : ((t == s) ? 1.f : 0.f);
+      }
+#pragma unroll
+      for (int op = 0; op < kGhostSharedMaxOps; ++op) {
+        if (op < p.ghost_ops) {  // uniform across the CTA
+          float gy[32];
+          tmem_ld32(tacc + (1 + op) * Cfg::BN + c0, gy);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) ss[op] = fmaf(gx[e], gy[e], ss[op]);
+        }
+      }
+    }
+#pragma unroll
+    for (int op = 0; op < kGhostSharedMaxOps; ++op) {
+      if (op < p.ghost_ops) {
+        const float v = warp_sum(ss[op]);
+        if (lane == 0)
+          p.partials[op * p.partial_op_stride + static_cast<long long>(w.sample) * p.partial_stride +
+                     4 * w.local + wq] = v;
+      }
+    }
+  } else if (Cfg::EPI == kEpiAxpy) {
+    const long long grow = static_cast<long long>(w.m_blk) * Cfg::BM + row;
+    const bool row_ok = grow < p.out_rows;
+#pragma unroll 1
+    for (int c0 = 0; c0 < Cfg::BN; c0 += 32) {
+      float v[32];
+      __syncwarp();
+      tmem_ld32(tacc + c0, v);
+      tmem_ld_wait();
+      const long long gcol0 = static_cast<long long>(w.n_blk) * Cfg::BN + c0;
+      if (!row_ok || gcol0 >= p.out_cols) continue;  // the next tmem_ld32 reconverges first
+      float* dst = p.out_f32 + grow * p.out_cols + gcol0;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (gcol0 + 4 * q >= p.out_cols) break;  // out_cols is a multiple of 4
+        float4* d4 = reinterpret_cast<float4*>(dst + 4 * q);
+        float4 o = *d4;
+        o.x = fmaf(p.alpha, v[4 * q], o.x);
+        o.y = fmaf(p.alpha, v[4 * q + 1], o.y);
+        o.z = fmaf(p.alpha, v[4 * q + 2], o.z);
+        o.w = fmaf(p.alpha, v[4 * q + 3], o.w);
+        *d4 = o;
+      }
+    }
   } else {  // kEpiStoreBf16
     const long long grow = static_cast<long long>(w.m_blk) * Cfg::BM + row;
 #pragma unroll 1
@@ -349,7 +431,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1) umma_kernel(const __grid_cons
     fence_mbar_init();
     tma_prefetch_desc(&p.tmA0);
     tma_prefetch_desc(&p.tmB0);
-    if (Cfg::EPI == kEpiGhostNorm) {
+    if (Cfg::GHOST) {
       tma_prefetch_desc(&p.tmA1);
       tma_prefetch_desc(&p.tmB1);
     }
@@ -362,7 +444,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1) umma_kernel(const __grid_cons
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int nphases = (Cfg::EPI == kEpiGhostNorm) ? 2 : 1;
+  const int nphases = (Cfg::EPI == kEpiGhostNorm) ? 2 : (Cfg::EPI == kEpiGhostShared) ? 1 + p.ghost_ops : 1;
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer

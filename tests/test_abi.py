@@ -147,3 +147,63 @@ def test_philox_blocks_rejects_on_host(L):
     assert L.dp_philox_blocks(ODD, 4, 0, 0, 0, 0, None) == E
     assert L.dp_philox_blocks(FAKE, 0, 0, 0, 0, 0, None) == E
     assert L.dp_philox_blocks(FAKE, (1 << 32) + 1, 0, 0, 0, 0, None) == E
+
+
+def test_block_workspace_size_and_host_rejections(L):
+    from sample_gradient_clipping_b200._lib import DpLayer
+    lay = (DpLayer * 2)(DpLayer(FAKE, FAKE, 4096, 4096, 0, 0.3, FAKE, None),
+                        DpLayer(FAKE, FAKE, 4096, 11008, 1, 0.3, FAKE, None))
+    per = L.dp_block_workspace_size(lay, 2, 8, 2048, _lib.DP_BF16, 0, _lib.DP_NORM_ONCE)
+    flat = L.dp_block_workspace_size(lay, 2, 8, 2048, _lib.DP_BF16, 1, _lib.DP_NORM_ONCE)
+    # per-layer mode reuses one tile region sized for the largest layer; flat once keeps every
+    # layer's tiles
+    assert 8 * 2 * 4096 * 11008 <= per <= L.dp_workspace_size_for(8, 2048, 4096, 11008, 0, _lib.DP_BF16,
+                                                                   _lib.DP_NORM_ONCE)
+    assert flat >= 8 * 2 * (4096 * 4096 + 4096 * 11008)
+    assert L.dp_block_workspace_size(lay, 2, 8, 2048, _lib.DP_BF16, 7, 0) == 0
+    assert L.dp_block_workspace_size(lay, 0, 8, 2048, _lib.DP_BF16, 0, 0) == 0
+    E = _lib.DP_ERR_INVALID_ARG
+    args = lambda **k: dict(dict(mode=1, C=1.0, sigma=1.0, ws=FAKE, ws_bytes=1 << 40), **k)
+    def call(**k):
+        a = args(**k)
+        return L.dp_block_step(lay, 2, _lib.DP_BF16, 8, 2048, a["mode"], a["C"], a["sigma"], 0, 0, 0,
+                               None, a["ws"], a["ws_bytes"], None)
+    assert call(mode=5) == E
+    assert call(C=0.0) == E
+    assert call(C=float("inf")) == E                    # flat noise std would be infinite
+    assert call(sigma=-1.0) == E
+    assert call(ws=None) == E
+    assert call(ws_bytes=4096) == _lib.DP_ERR_WORKSPACE
+    bad = (DpLayer * 1)(DpLayer(ODD, FAKE, 64, 64, 0, 1.0, FAKE, None))
+    assert L.dp_block_step(bad, 1, _lib.DP_BF16, 2, 4, 1, 1.0, 0.0, 0, 0, 0, None, FAKE, 1 << 30, None) == E
+
+
+def test_projected_adam_rejects_on_host(L):
+    E = _lib.DP_ERR_INVALID_ARG
+    assert L.dp_adam_workspace_size(128, 64) == 256 + 128 * 64 * 2
+    assert L.dp_adam_workspace_size(128, 12) == 0
+
+    def call(**k):
+        a = dict(W=FAKE, dt=_lib.DP_BF16, d_in=128, d_out=256, r=64, lr=1e-3, b1=0.9, b2=0.999,
+                 eps=1e-8, t=1, ws=FAKE, ws_bytes=1 << 20)
+        a.update(k)
+        return L.dp_projected_adam_step(a["W"], FAKE, FAKE, FAKE, FAKE, a["dt"], a["d_in"], a["d_out"],
+                                        a["r"], a["lr"], a["b1"], a["b2"], a["eps"], 1.0, a["t"], a["ws"],
+                                        a["ws_bytes"], None)
+    assert call(W=None) == E
+    assert call(W=ODD) == E
+    assert call(t=0) == E
+    assert call(b1=1.0) == E
+    assert call(b2=-0.1) == E
+    assert call(lr=-1.0) == E
+    assert call(r=12) == E
+    assert call(dt=_lib.DP_F32) == _lib.DP_ERR_UNSUPPORTED
+    assert call(ws_bytes=100) == _lib.DP_ERR_WORKSPACE
+
+
+def test_selftest_rejects_on_host(L):
+    E = _lib.DP_ERR_INVALID_ARG
+    assert L.dp_selftest_wait_timeout(None, 10**6, None) == E
+    assert L.dp_selftest_wait_timeout(FAKE + 16, 10**6, None) == E
+    assert L.dp_selftest_wait_timeout(FAKE, 10, None) == E              # below 1 us
+    assert L.dp_selftest_wait_timeout(FAKE, 10**10, None) == E          # above the 2 s limit

@@ -1,0 +1,137 @@
+"""dp_block_step against the fp64 oracle: per-layer and flat clipping over a block of linears."""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from sample_gradient_clipping_b200 import _lib, inputs
+from tests.gpu_helpers import TOL, check_clip_decisions, host, noise_tolerance, rel_fro, rel_max
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    _lib.lib()
+
+
+def _block(dtype="bf16", d=256, ffn=512, B=4, T=256, seed=3, lognormal=True):
+    w = inputs.Workload("blk", B=B, T=T, dtype=dtype, linears=inputs._block(0, d, ffn),
+                        C=1.0 / math.sqrt(7.0), sigma=0.6, seed=seed, dy_var="per_layer",
+                        sample_scale="lognormal" if lognormal else "")
+    data = inputs.generate(w)
+    dev = {"X": {k: v.cuda() for k, v in data["X"].items()},
+           "dY": {k: v.cuda() for k, v in data["dY"].items()}}
+    return w, data, dev
+
+
+def _layers(w, dev, C):
+    return [{"X": dev["X"][l.x_key], "dY": dev["dY"][l.name], "layer_id": l.layer_id, "C": C,
+             "norms_out": torch.empty(w.B, dtype=torch.float32, device="cuda")} for l in w.linears]
+
+
+def _oracle_layers(w, data, C):
+    return [{"X": inputs.as_f64(data["X"][l.x_key]), "dY": inputs.as_f64(data["dY"][l.name]),
+             "layer_id": l.layer_id, "C": C} for l in w.linears]
+
+
+@pytest.mark.parametrize("method", ["auto", "ghost", "explicit", "once"])
+def test_flat_clipping_block(method):
+    w, data, dev = _block()
+    C = float(np.float32(1.0))           # the block's bound: sqrt(7) per-layer bounds of 1/sqrt(7)
+    sigma = float(np.float32(w.sigma))
+    tol = TOL["bf16"]
+    outs0, norms0, flat0 = _lib.dp_block_step(_layers(w, dev, C), mode="flat", C=C, sigma=0.0,
+                                              seed=w.seed, step=5, method=method)
+    outs1, _, _ = _lib.dp_block_step(_layers(w, dev, C), mode="flat", C=C, sigma=sigma, seed=w.seed,
+                                     step=5, method=method)
+    torch.cuda.synchronize()
+    ref = oracle.block_step(_oracle_layers(w, data, C), C, 0.0, w.seed, 5, mode="flat")
+    assert rel_max(host(flat0), ref["flat_norms"]) <= tol["norm"]
+    check_clip_decisions(host(flat0), ref["flat_norms"], C)
+    # Samples 0 and 2 exceed the block bound, 1 and 3 do not (lognormal scales 7.7, 0.08, 1.5, 0.57).
+    assert list(host(flat0) > C) == [True, False, True, False]
+    for k, lin in enumerate(w.linears):
+        r = ref["layers"][k]
+        assert rel_max(host(norms0[k]), r["norms"]) <= tol["norm"], lin.name
+        assert rel_fro(host(outs0[k]), r["S"]) <= tol["sum"], (lin.name, rel_fro(host(outs0[k]), r["S"]))
+        a, b = host(outs1[k]), host(outs0[k])
+        want = oracle.noise(a.shape[0], a.shape[1], sigma * C, w.seed, 5, lin.layer_id)
+        assert np.all(np.abs((a - b) - want) <= noise_tolerance(a, b) + 1e-6 * np.abs(b)), lin.name
+
+
+def test_flat_clipping_block_f32():
+    w, data, dev = _block(dtype="f32", d=64, ffn=96, B=3, T=24, seed=8, lognormal=False)
+    C = 0.9
+    outs, norms, flat = _lib.dp_block_step(_layers(w, dev, C), mode="flat", C=C, sigma=0.0, seed=1)
+    ref = oracle.block_step(_oracle_layers(w, data, C), np.float32(C), 0.0, 1, 0, mode="flat")
+    assert rel_max(host(flat), ref["flat_norms"]) <= TOL["f32"]["norm"]
+    for k in range(len(w.linears)):
+        assert rel_fro(host(outs[k]), ref["layers"][k]["S"]) <= TOL["f32"]["sum"]
+
+
+def test_per_layer_block_equals_linear_steps():
+    w, data, dev = _block(seed=4)
+    C = 1.0 / math.sqrt(7.0)
+    outs, norms, _ = _lib.dp_block_step(_layers(w, dev, C), mode="per_layer", sigma=w.sigma, seed=w.seed,
+                                        step=2)
+    for k, lin in enumerate(w.linears):
+        G, n = _lib.dp_linear_step(dev["X"][lin.x_key], dev["dY"][lin.name], C, w.sigma, w.seed, 2,
+                                   lin.layer_id)
+        assert torch.equal(n, norms[k]), lin.name
+        assert rel_fro(host(outs[k]), host(G)) <= 1e-6, lin.name
+
+
+@pytest.mark.slow
+def test_flat_clipping_llama7b_block_sampled():
+    w = inputs.WORKLOADS["llama7b_block"]
+    data = inputs.generate(w)
+    dev = {"X": {k: v.cuda() for k, v in data["X"].items()},
+           "dY": {k: v.cuda() for k, v in data["dY"].items()}}
+    C = 1.0
+    outs, norms, flat = _lib.dp_block_step(_layers(w, dev, C), mode="flat", C=C, sigma=0.0, seed=w.seed)
+    torch.cuda.synchronize()
+    olayers = _oracle_layers(w, data, C)
+    n_layers = [oracle.per_sample_norms(l["X"], l["dY"]) for l in olayers]
+    flat_ref = np.sqrt(np.sum(np.stack(n_layers) ** 2, axis=0))
+    assert rel_max(host(flat), flat_ref) <= TOL["bf16"]["norm"]
+    c = oracle.clip_factors(flat_ref, C)
+    rng = np.random.default_rng(0)
+    for k, l in enumerate(olayers):
+        m, n = outs[k].shape
+        rows, cols = rng.integers(0, m, 256), rng.integers(0, n, 256)
+        want = oracle.clipped_sum_entries(l["X"], l["dY"], c, rows, cols)
+        assert rel_fro(host(outs[k])[rows, cols], want) <= TOL["bf16"]["sum"]
+
+
+@pytest.mark.parametrize("mode", ["per_layer", "flat"])
+def test_shared_x_gram_ghost_block(mode):
+    """q/k/v and gate/up read the same X: one X Gram per group, same norms as one linear at a time."""
+    w, data, dev = _block(d=256, ffn=384, B=3, T=384, seed=11)
+    C = 1.0 if mode == "flat" else 1.0 / math.sqrt(7.0)
+    _lib.profiling_enable(True)
+    _lib.profiling_collect()
+    outs, norms, flat = _lib.dp_block_step(_layers(w, dev, C), mode=mode, C=C, sigma=0.0, seed=w.seed, step=1,
+                                           method="ghost")
+    torch.cuda.synchronize()
+    kinds = _lib.profiling_collect()
+    _lib.profiling_enable(False)
+    # q/k/v share one launch, gate/up another; o and down each run the plain ghost kernel.
+    assert kinds["umma_ghost_shared"][1] == 2 and kinds["umma_ghost_norm"][1] == 2, kinds
+    for k, lin in enumerate(w.linears):
+        n1 = _lib.dp_per_sample_norms(dev["X"][lin.x_key], dev["dY"][lin.name], method="ghost")
+        assert torch.equal(norms[k], n1), lin.name      # same Gram tiles, same partial slots
+    ref = oracle.block_step(_oracle_layers(w, data, C), C, 0.0, w.seed, 1, mode=mode)
+    tol = TOL["bf16"]
+    if mode == "flat":
+        assert rel_max(host(flat), ref["flat_norms"]) <= tol["norm"]
+    for k, lin in enumerate(w.linears):
+        r = ref["layers"][k]
+        assert rel_max(host(norms[k]), r["norms"]) <= tol["norm"], lin.name
+        assert rel_fro(host(outs[k]), r["S"]) <= tol["sum"], lin.name

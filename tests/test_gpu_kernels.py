@@ -37,7 +37,8 @@ def test_philox_words_bit_exact(seed, step, layer, stream):
     assert np.array_equal(got, want)
 
 
-@pytest.mark.parametrize("rows,cols", [(1, 1), (3, 5), (64, 32), (257, 520), (1000, 1003), (768, 3072)])
+@pytest.mark.parametrize("rows,cols", [(1, 1), (3, 5), (64, 32), (257, 520), (1000, 1003), (768, 3072),
+                                       (2048, 2052)])   # the last stages the tables in shared memory
 @pytest.mark.parametrize("std", [1.0, 0.6 / math.sqrt(7.0)])
 def test_noise_on_zero_buffer(rows, cols, std):
     G = torch.zeros(rows, cols, dtype=torch.float32, device="cuda")
