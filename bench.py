@@ -1,8 +1,9 @@
 """Benchmark of the DP-SGD per-sample clip + sum + noise step on B200.
 
-One step = the whole hot path over one batch: dp_linear_step on every linear of the workload
-(Llama-7B-shaped block by default: 7 linears, B=8, T=2048, bf16).  Each call computes the
-per-sample norms, the clip factors, the clipped sum and the Gaussian noise.  The inputs are
+One step = the whole hot path over one batch: one dp_block_step over the linears of the
+workload (Llama-7B-shaped block by default: 7 linears, B=8, T=2048, bf16), or one
+dp_linear_step per linear for the projected variant.  It computes the per-sample norms, the
+clip factors, the clipped sum and the Gaussian noise of every linear.  The inputs are
 seeded synthetic tensors, resident in HBM.  They are larger than the 126 MB L2, and the 7
 linears cycle through 2.2 GB, so no L2 flush is needed between steps.
 
@@ -27,6 +28,20 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "DP clip+sum+noise tokens/s and TFLOP/s as % of B200 roofline, 1 GPU"
+
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of a step's dominant
+# kernel, averaged over the step's launches, from one ncu capture of the same command (the
+# ncu summaries in profiles/ give the capture).  Each entry records a hash of the sources that
+# define that kernel; when they change, the figure no longer describes the code and bench.py
+# reports traffic as null.
+KERNEL_SOURCES = ("sample_gradient_clipping_b200/csrc/ptx.cuh",
+                  "sample_gradient_clipping_b200/csrc/umma_gemm.cuh",
+                  "sample_gradient_clipping_b200/csrc/umma_gemm_2sm.cuh")
+# (workload, kernel) -> (bytes per launch, source hash)
+MEASURED_TRAFFIC = {
+    ("llama7b_block", "umma_explicit_store"): (878291712, "52573065ffda7a1c"),
+    ("llama13b_block", "umma_explicit_store"): (675981056, "52573065ffda7a1c"),
+}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -39,8 +54,12 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--method", default="auto", choices=["auto", "ghost", "explicit"])
+    ap.add_argument("--no-non-dp", action="store_true",
+                    help="skip the non-private comparison (plain bf16 weight-gradient GEMMs)")
+    ap.add_argument("--method", default="auto", choices=["auto", "ghost", "explicit", "once"])
     ap.add_argument("--linears", default="", help="comma-separated subset of the workload's linears")
+    ap.add_argument("--clip", default="per_layer", choices=["per_layer", "flat"],
+                    help="per-layer bounds C_l, or one flat bound sqrt(L) * C_l for the whole block")
     return ap.parse_args()
 
 
@@ -75,6 +94,23 @@ def workload_model(w):
         seen.add(lin.x_key)
         per_linear.append((lin, f, b))
     return flops, byts, x_shared_bytes, per_linear
+
+
+def kernel_source_hash():
+    import hashlib
+
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(workload, kernel):
+    entry = MEASURED_TRAFFIC.get((workload, kernel))
+    if entry is None or entry[1] != kernel_source_hash():
+        return None
+    return entry[0]
 
 
 def max_over_ranks(value, device, world):
@@ -247,16 +283,43 @@ def run_ours(args, w, rank, world):
     ws_bytes = max(_lib.workspace_size(w.B, w.T, l.d_in, l.d_out, r,
                                        _lib.DP_BF16 if w.dtype == "bf16" else _lib.DP_F32, args.method)
                    for l in w.linears)
-    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     G = {l.name: torch.empty(l.d_in, r or l.d_out, dtype=torch.float32, device=dev) for l in w.linears}
     norms = {l.name: torch.empty(w.B, dtype=torch.float32, device=dev) for l in w.linears}
     stream = torch.cuda.current_stream(dev)
+    # The projection depends on (seed, layer) only, not on the step: it is generated once per
+    # linear, as a training loop would, and passed to every step.
+    P = {l.name: _lib.dp_projection_matrix(torch.empty(l.d_out, r, dtype=X[l.x_key].dtype, device=dev),
+                                           w.seed, l.layer_id, stream=stream) for l in w.linears} if r else {}
+    flat_C = w.C * math.sqrt(len(w.linears))
+    block = [{"X": X[l.x_key], "dY": dY[l.name], "layer_id": l.layer_id, "C": w.C, "G_out": G[l.name],
+              "norms_out": norms[l.name]} for l in w.linears]
+    # Unprojected blocks go through the block call (per-layer or flat clipping); the projected
+    # variant runs one dp_linear_step per linear, each with its own P.
+    use_block = (r == 0)
+    if args.clip == "flat" and not use_block:
+        raise SystemExit("flat clipping is defined for unprojected blocks")
+    if use_block:
+        arr = (_lib.DpLayer * len(block))(*[
+            _lib.DpLayer(b["X"].data_ptr(), b["dY"].data_ptr(), b["X"].shape[2], b["dY"].shape[2],
+                         b["layer_id"], b["C"], b["G_out"].data_ptr(), b["norms_out"].data_ptr())
+            for b in block])
+        ws_bytes = _lib.lib().dp_block_workspace_size(arr, len(block), w.B, w.T,
+                                                      _lib.DP_BF16 if w.dtype == "bf16" else _lib.DP_F32,
+                                                      _lib.CLIP_MODES[args.clip], _lib.METHODS[args.method])
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    flat_norms = torch.empty(w.B, dtype=torch.float32, device=dev)
 
     def step(k):
+        if use_block:
+            _lib.dp_block_step(block, mode=args.clip, C=flat_C if args.clip == "flat" else w.C, sigma=w.sigma,
+                               seed=w.seed, step=w.step + k, method=args.method,
+                               flat_norms_out=flat_norms if args.clip == "flat" else None, workspace=ws,
+                               stream=stream)
+            return
         for l in w.linears:
             _lib.dp_linear_step(X[l.x_key], dY[l.name], w.C, w.sigma, w.seed, w.step + k, l.layer_id,
-                                r=r, method=args.method, norms_out=norms[l.name], G_out=G[l.name],
-                                workspace=ws, stream=stream)
+                                P=P.get(l.name), r=r, method=args.method, norms_out=norms[l.name],
+                                G_out=G[l.name], workspace=ws, stream=stream)
 
     for k in range(args.warmup):
         step(k)
@@ -291,10 +354,15 @@ def run_ours(args, w, rank, world):
         raise RuntimeError("an in-kernel wait timed out during the timed steps")
     ms = max_over_ranks(ms, dev, world)
 
+    # ---- the non-private step of the same shapes, for FlashDP's "share of non-DP throughput"
+    non_dp = None
+    if not args.no_non_dp and r == 0 and w.dtype == "bf16":
+        non_dp = run_non_dp(args, w, X, dY, dev, stream, torch, world, ms)
+
     # ---- end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(args, w, data, dev, stream, ws, r, _lib, torch, world)
+        e2e = run_e2e(args, w, data, dev, stream, r, P, _lib, torch, world)
 
     if rank != 0:
         return 0
@@ -326,7 +394,9 @@ def run_ours(args, w, rank, world):
                 achieved = work / (d_ms / 1e3) / 1e12
                 peak = pk["bf16_tflops_sustained"]
             roofline = {"bound": bound, "kernel": dominant, "achieved": achieved, "peak": peak,
-                        "unit": unit, "frac": achieved / peak, "traffic": None,
+                        "unit": unit, "frac": achieved / peak,
+                        "traffic": measured_traffic(w.name, dominant),
+                        "traffic_unit": "bytes per launch (DRAM read + write, ncu)",
                         "peak_kind": (f"{pk_kind} HBM copy bandwidth" if unit == "GB/s" else
                                       f"{pk_kind} sustained bf16 (kernel timed inside a long step)"),
                         "launches": d_n // args.steps, "avg_launch_ms": d_ms / d_n,
@@ -337,8 +407,10 @@ def run_ours(args, w, rank, world):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "T": w.T, "linears": len(w.linears),
-                   "method": args.method, "l2": "inputs larger than L2 (no flush)",
+                   "method": args.method, "clip": args.clip, "l2": "inputs larger than L2 (no flush)",
                    "parallelism": "replicas" if world > 1 else "1 GPU",
+                   **({"projection": f"P [d_out, {r}] generated once per linear before timing "
+                                     "(it depends on seed and layer only)"} if r else {}),
                    "description": w.description},
         "tflops_alg": flops * world / step_s / 1e12,
         "step_roofline": {"frac_of_burst": roof_t_burst / step_s, "frac_of_sustained": roof_t_sust / step_s,
@@ -351,6 +423,7 @@ def run_ours(args, w, rank, world):
         "gpu_launches": launches,
         "clocks": clocks,
         "e2e": e2e,
+        "non_dp": non_dp,
     }
     if world == 1 and not args.no_cpu_baseline:
         secs, toks = oracle_block_sample(w, data, list(w.linears))
@@ -362,10 +435,56 @@ def run_ours(args, w, rank, world):
     return 0
 
 
-def run_e2e(args, w, data, dev, stream, ws, r, _lib, torch, world):
-    """Same step through the public API from pinned host buffers, copies inside the timing."""
+def run_non_dp(args, w, X, dY, dev, stream, torch, world, dp_ms):
+    """Plain weight gradients X^T dY of every linear, bf16 in, fp32 out, by cuBLAS (torch.mm).
+
+    This is what a non-private step computes for these linears: no per-sample norms, no
+    clipping, no noise.  It is a comparison only; nothing of it is on the library's path.
+    """
+    outs = {l.name: torch.empty(l.d_in, l.d_out, dtype=torch.float32, device=dev) for l in w.linears}
+    Xf = {k: v.view(-1, v.shape[-1]) for k, v in X.items()}
+    dYf = {k: v.view(-1, v.shape[-1]) for k, v in dY.items()}
+
+    def step():
+        for l in w.linears:
+            torch.mm(Xf[l.x_key].t(), dYf[l.name], out_dtype=torch.float32, out=outs[l.name])
+
+    try:
+        step()
+    except (RuntimeError, NotImplementedError, TypeError) as e:  # no fp32-output bf16 mm here
+        return {"unavailable": f"torch.mm with out_dtype=float32: {type(e).__name__}"}
+
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            step()
+        torch.cuda.synchronize(dev)
+        steps = max(5, min(args.steps, 50))
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record(stream)
+        for _ in range(steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+    ms = max_over_ranks(ev0.elapsed_time(ev1) / steps, dev, world)
+    return {"what": "X^T dY per linear by cuBLAS (torch.mm, bf16 in, fp32 out); no norms, clipping or noise",
+            "ms_per_step": ms, "steps": steps, "tokens_per_s": job_tokens_per_second(w.tokens, world, ms),
+            "dp_share_of_non_dp_throughput": ms / dp_ms}
+
+
+def run_e2e(args, w, data, dev, stream, r, P, _lib, torch, world):
+    """Same step through the public API from pinned host buffers, copies inside the timing.
+
+    Three streams: host->device copies of each linear's inputs, dp_linear_step on the compute
+    stream, and device->host copies of its outputs.  They overlap layer by layer: linear l+1
+    uploads while l computes and l-1 downloads (PCIe is full duplex).  CUDA events order
+    every dependency, including the reuse of a device buffer by the next step.
+    """
     hX = {k: v.pin_memory() for k, v in data["X"].items()}
     hdY = {k: v.pin_memory() for k, v in data["dY"].items()}
+    # One linear at a time through dp_linear_step: its own workspace, sized for the largest.
+    ws = torch.empty(max(_lib.workspace_size(w.B, w.T, l.d_in, l.d_out, r,
+                                             _lib.DP_BF16 if w.dtype == "bf16" else _lib.DP_F32, args.method)
+                         for l in w.linears), dtype=torch.uint8, device=dev)
     dX = {k: torch.empty_like(v, device=dev) for k, v in hX.items()}
     ddY = {k: torch.empty_like(v, device=dev) for k, v in hdY.items()}
     G = {l.name: torch.empty(l.d_in, r or l.d_out, dtype=torch.float32, device=dev) for l in w.linears}
@@ -376,19 +495,42 @@ def run_e2e(args, w, data, dev, stream, ws, r, _lib, torch, world):
         sum(v.numel() * v.element_size() for v in hdY.values())
     bo = sum(v.numel() * v.element_size() for v in hG.values()) + \
         sum(v.numel() * v.element_size() for v in hn.values())
+    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event()
+    # last use of each device buffer (compute of the previous step) and of each output
+    x_free = {k: None for k in dX}
+    dy_free = {k: None for k in ddY}
+    out_free = {k: None for k in G}
 
     def step(k):
-        loaded = set()
+        loaded = {}
         for l in w.linears:
-            if l.x_key not in loaded:
-                dX[l.x_key].copy_(hX[l.x_key], non_blocking=True)
-                loaded.add(l.x_key)
-            ddY[l.name].copy_(hdY[l.name], non_blocking=True)
+            with torch.cuda.stream(up):
+                if l.x_key not in loaded:
+                    if x_free[l.x_key] is not None:
+                        up.wait_event(x_free[l.x_key])
+                    dX[l.x_key].copy_(hX[l.x_key], non_blocking=True)
+                    e = ev(); e.record(up); loaded[l.x_key] = e
+                if dy_free[l.name] is not None:
+                    up.wait_event(dy_free[l.name])
+                ddY[l.name].copy_(hdY[l.name], non_blocking=True)
+                dy_ready = ev(); dy_ready.record(up)
+            stream.wait_event(loaded[l.x_key])
+            stream.wait_event(dy_ready)
+            if out_free[l.name] is not None:
+                stream.wait_event(out_free[l.name])
             _lib.dp_linear_step(dX[l.x_key], ddY[l.name], w.C, w.sigma, w.seed, w.step + k, l.layer_id,
-                                r=r, method=args.method, norms_out=n[l.name], G_out=G[l.name],
-                                workspace=ws, stream=stream)
-            hG[l.name].copy_(G[l.name], non_blocking=True)
-            hn[l.name].copy_(n[l.name], non_blocking=True)
+                                P=P.get(l.name), r=r, method=args.method, norms_out=n[l.name],
+                                G_out=G[l.name], workspace=ws, stream=stream)
+            done = ev(); done.record(stream)
+            x_free[l.x_key] = done
+            dy_free[l.name] = done
+            with torch.cuda.stream(down):
+                down.wait_event(done)
+                hG[l.name].copy_(G[l.name], non_blocking=True)
+                hn[l.name].copy_(n[l.name], non_blocking=True)
+                read = ev(); read.record(down)
+                out_free[l.name] = read
 
     steps = max(1, min(args.steps, 5))
     for k in range(min(args.warmup, 2)):
@@ -398,14 +540,19 @@ def run_e2e(args, w, data, dev, stream, ws, r, _lib, torch, world):
         torch.distributed.barrier()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ev0.record(stream)
+    up.wait_event(ev0)
     for k in range(steps):
         step(k)
+    down.synchronize()
+    stream.wait_stream(down)
+    stream.wait_stream(up)
     ev1.record(stream)
     torch.cuda.synchronize(dev)
     ms = max_over_ranks(ev0.elapsed_time(ev1) / steps, dev, world)
     return {"value": job_tokens_per_second(w.tokens, world, ms), "unit": "tokens/s", "h2d_bytes_per_step": bi,
             "d2h_bytes_per_step": bo, "ms_per_step": ms, "steps": steps,
-            "result_read_back": "every linear's noisy clipped gradient and per-sample norms"}
+            "result_read_back": "every linear's noisy clipped gradient and per-sample norms",
+            "overlap": "uploads, compute and downloads on three streams, layer by layer"}
 
 
 def main():
