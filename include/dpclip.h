@@ -145,12 +145,29 @@ dp_status dp_projection_matrix(void* P, dp_dtype dt, int d_out, int r,
  *   C          : > 0.  +INF (no clipping) requires sigma = 0.
  *   sigma      : >= 0.
  *   norms_out  : NULL or DEVICE fp32 [B].
- *   G_out      : DEVICE fp32 [d_in, r or d_out], overwritten. */
+ *   G_out      : DEVICE fp32 [d_in, r or d_out], overwritten.  The gradients-once method
+ *                rounds sigma*C*z to fp32 before adding it to the fp32 sum (within one ulp
+ *                of rounding the fp64 sum once); the others add in fp64 and round once. */
 dp_status dp_linear_step(const void* X, const void* dY, const void* P, int r, dp_dtype dt,
                          int B, int T, int d_in, int d_out, float C, float sigma,
                          unsigned long long seed, unsigned long long step, unsigned layer_id,
                          dp_norm_method method, float* norms_out, float* G_out,
                          void* workspace, size_t ws_bytes, void* stream);
+
+/* dp_linear_step with the step number in device memory, read when the noise kernels run.
+ * One CUDA graph captured around this call then serves every training step: the caller
+ * advances *step_dev (on the device, or by a copy ordered on the stream) between replays.
+ * (The pages have no counterpart; the noise counter is the same (seed, step, layer_id).)
+ *   step_dev : DEVICE uint64, 8-byte aligned; only its low 32 bits enter the counter.
+ * Capture only after one ordinary call with the same shapes and method on that device: the
+ * first call of a kernel configuration sets its shared-memory attribute, which is not a
+ * stream operation.  The call itself allocates nothing and does not synchronise. */
+dp_status dp_linear_step_dev_step(const void* X, const void* dY, const void* P, int r,
+                                  dp_dtype dt, int B, int T, int d_in, int d_out, float C,
+                                  float sigma, unsigned long long seed,
+                                  const unsigned long long* step_dev, unsigned layer_id,
+                                  dp_norm_method method, float* norms_out, float* G_out,
+                                  void* workspace, size_t ws_bytes, void* stream);
 
 /* The raw Philox4x32-10 words behind every random number of the library (Salmon et al.,
  * "Parallel random numbers: as easy as 1, 2, 3", SC'11), exposed so that the uint32 stream
@@ -224,6 +241,13 @@ dp_status dp_block_step(const dp_layer* layers, int L, dp_dtype dt, int B, int T
                         dp_clip_mode mode, float C, float sigma, unsigned long long seed,
                         unsigned long long step, dp_norm_method method, float* flat_norms_out,
                         void* workspace, size_t ws_bytes, void* stream);
+
+/* dp_block_step with the step number in device memory (see dp_linear_step_dev_step). */
+dp_status dp_block_step_dev_step(const dp_layer* layers, int L, dp_dtype dt, int B, int T,
+                                 dp_clip_mode mode, float C, float sigma, unsigned long long seed,
+                                 const unsigned long long* step_dev, dp_norm_method method,
+                                 float* flat_norms_out, void* workspace, size_t ws_bytes,
+                                 void* stream);
 
 /* ------------------------------------------------------------------ projected Adam
  * One projected Adam update.  DP-GRAPE page, Methodology, "Projected Optimizer States": the

@@ -46,6 +46,9 @@ SIGNATURES = {
     "dp_linear_step": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_int, _c_int,
                                 _c_int, _c_int, _c_float, _c_float, _c_ull, _c_ull, _c_uint, _c_int,
                                 _c_void_p, _c_void_p, _c_void_p, _c_size_t, _c_void_p]),
+    "dp_linear_step_dev_step": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_int, _c_int,
+                                         _c_int, _c_int, _c_float, _c_float, _c_ull, _c_void_p, _c_uint,
+                                         _c_int, _c_void_p, _c_void_p, _c_void_p, _c_size_t, _c_void_p]),
     "dp_workspace_status": (_c_int, [_c_void_p, _c_void_p]),
     "dp_selftest_wait_timeout": (_c_int, [_c_void_p, _c_ull, _c_void_p]),
     "dp_per_sample_norms_static": (_c_int, [_c_void_p, _c_void_p, _c_int, _c_int, _c_int, _c_int, _c_int,
@@ -59,6 +62,9 @@ SIGNATURES = {
     "dp_block_step": (_c_int, [ctypes.POINTER(DpLayer), _c_int, _c_int, _c_int, _c_int, _c_int, _c_float,
                                _c_float, _c_ull, _c_ull, _c_int, _c_void_p, _c_void_p, _c_size_t,
                                _c_void_p]),
+    "dp_block_step_dev_step": (_c_int, [ctypes.POINTER(DpLayer), _c_int, _c_int, _c_int, _c_int, _c_int,
+                                        _c_float, _c_float, _c_ull, _c_void_p, _c_int, _c_void_p, _c_void_p,
+                                        _c_size_t, _c_void_p]),
     "dp_adam_workspace_size": (_c_size_t, [_c_int, _c_int]),
     "dp_projected_adam_step": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_int, _c_int,
                                         _c_int, _c_int, _c_float, _c_float, _c_float, _c_float, _c_float,
@@ -198,9 +204,24 @@ def dp_projection_matrix(P, seed, layer_id, stream=None):
     return P
 
 
+def _device_step(step):
+    """A device tensor holding the step (int64/uint64, one element), or None for a number."""
+    import torch
+
+    if not isinstance(step, torch.Tensor):
+        return None
+    if step.numel() != 1 or step.dtype not in (torch.int64, torch.uint64) or not step.is_cuda:
+        raise ValueError("a device step must be a one-element int64 CUDA tensor")
+    return step
+
+
 def dp_linear_step(X, dY, C, sigma, seed, step, layer_id, P=None, r=0, method="auto",
                    norms_out=None, G_out=None, workspace=None, stream=None):
-    """One privatised step; returns (G_out, norms_out)."""
+    """One privatised step; returns (G_out, norms_out).
+
+    ``step`` is a number, or a one-element int64 CUDA tensor read when the kernels run
+    (dp_linear_step_dev_step), so that a CUDA graph of this call serves every step.
+    """
     import torch
 
     B, T, d_in, d_out = _bt_dims(X, dY)
@@ -212,11 +233,19 @@ def dp_linear_step(X, dY, C, sigma, seed, step, layer_id, P=None, r=0, method="a
         G_out = torch.empty(d_in, width, dtype=torch.float32, device=X.device)
     if norms_out is None:
         norms_out = torch.empty(B, dtype=torch.float32, device=X.device)
-    check(lib().dp_linear_step(_ptr(X), _ptr(dY), _ptr(P), r, _dtype_code(X), B, T, d_in, d_out,
-                               float(C), float(sigma), int(seed), int(step), int(layer_id),
-                               METHODS[method], _ptr(norms_out), _ptr(G_out), _ptr(ws), ws.numel(),
-                               _stream(stream)),
-          "dp_linear_step")
+    dstep = _device_step(step)
+    if dstep is not None:
+        check(lib().dp_linear_step_dev_step(_ptr(X), _ptr(dY), _ptr(P), r, _dtype_code(X), B, T, d_in, d_out,
+                                            float(C), float(sigma), int(seed), _ptr(dstep), int(layer_id),
+                                            METHODS[method], _ptr(norms_out), _ptr(G_out), _ptr(ws),
+                                            ws.numel(), _stream(stream)),
+              "dp_linear_step_dev_step")
+    else:
+        check(lib().dp_linear_step(_ptr(X), _ptr(dY), _ptr(P), r, _dtype_code(X), B, T, d_in, d_out,
+                                   float(C), float(sigma), int(seed), int(step), int(layer_id),
+                                   METHODS[method], _ptr(norms_out), _ptr(G_out), _ptr(ws), ws.numel(),
+                                   _stream(stream)),
+              "dp_linear_step")
     return G_out, norms_out
 
 
@@ -263,6 +292,7 @@ def dp_block_step(layers, mode="per_layer", C=1.0, sigma=0.0, seed=0, step=0, me
     """One step for a block of linears sharing the batch.
 
     ``layers``: dicts with X, dY, layer_id, C (per-layer bound), and optional G_out, norms_out.
+    ``step``: a number, or a one-element int64 CUDA tensor read when the kernels run.
     Returns (list of G_out, list of norms_out or None, flat_norms_out or None).
     """
     import torch
@@ -289,10 +319,17 @@ def dp_block_step(layers, mode="per_layer", C=1.0, sigma=0.0, seed=0, step=0, me
         workspace = torch.empty(need, dtype=torch.uint8, device=first["X"].device)
     if mode == "flat" and flat_norms_out is None:
         flat_norms_out = torch.empty(B, dtype=torch.float32, device=first["X"].device)
-    check(lib().dp_block_step(arr, len(layers), dt, B, T, CLIP_MODES[mode], float(C), float(sigma), int(seed),
-                              int(step), METHODS[method], _ptr(flat_norms_out), _ptr(workspace),
-                              workspace.numel(), _stream(stream)),
-          "dp_block_step")
+    dstep = _device_step(step)
+    if dstep is not None:
+        check(lib().dp_block_step_dev_step(arr, len(layers), dt, B, T, CLIP_MODES[mode], float(C), float(sigma),
+                                           int(seed), _ptr(dstep), METHODS[method], _ptr(flat_norms_out),
+                                           _ptr(workspace), workspace.numel(), _stream(stream)),
+              "dp_block_step_dev_step")
+    else:
+        check(lib().dp_block_step(arr, len(layers), dt, B, T, CLIP_MODES[mode], float(C), float(sigma),
+                                  int(seed), int(step), METHODS[method], _ptr(flat_norms_out),
+                                  _ptr(workspace), workspace.numel(), _stream(stream)),
+              "dp_block_step")
     return outs, norms, flat_norms_out
 
 

@@ -128,21 +128,37 @@ WsLayout ws_layout(const Shape& s, dp_norm_method method) {
   return L;
 }
 
-// Roofline cost model of one step for each norm method (seconds at the rates below).
-constexpr double kModelFlops = 1.4e15;  // bf16 tensor flop/s
-constexpr double kModelBytes = 6.5e12;  // HBM byte/s
+// Cost model of one step for each norm method (seconds), a roofline with four corrections
+// calibrated on this B200 build:
+//   * per-sample tensor-core kernels run over a sample's T tokens per tile; below ~1024
+//     tokens their fixed cost per tile shows (measured: half rate at T = 512);
+//   * the clipped-sum contraction with its noise epilogue runs at about 65% of the rate of
+//     the per-sample pair kernel;
+//   * the gradients-once tile stores stream at ~3 TB/s, and its reduce is bound by the HBM
+//     stream or by the noise (~2.5e11 normals/s), whichever is slower;
+//   * each launch costs ~4 us, which decides the small shapes.
+constexpr double kModelFlops = 1.4e15;       // bf16 tensor flop/s (sustained)
+constexpr double kModelBytes = 6.5e12;       // HBM byte/s
+constexpr double kModelStoreBytes = 3.0e12;  // per-sample tile stores, byte/s
+constexpr double kModelNormals = 2.5e11;     // normals/s in the reduce
+constexpr double kModelClipSumEff = 0.65;
+constexpr double kModelLaunch = 4e-6;        // s per kernel launch
 
 double model_cost(const Shape& s, dp_norm_method m) {
   const double N = static_cast<double>(s.N()), d = s.m, ne = s.ne(), B = s.B;
   const double contraction = 2.0 * N * d * ne / kModelFlops;
+  const double per_sample = contraction / std::min(1.0, s.T / 1024.0);
+  const double clip_sum = contraction / kModelClipSumEff;
   const double scale_pass = N * (d < ne ? d : ne) * 4.0 / kModelBytes;
   if (m == DP_NORM_GHOST) {
     const double tt = std::ceil(s.T / 128.0);
-    return B * tt * (tt + 1) / 2 * 2.0 * 128 * 128 * (d + ne) / kModelFlops + scale_pass + contraction;
+    return B * tt * (tt + 1) / 2 * 2.0 * 128 * 128 * (d + ne) / kModelFlops + scale_pass + clip_sum +
+           4 * kModelLaunch;
   }
-  if (m == DP_NORM_EXPLICIT) return 2.0 * contraction + scale_pass;
-  const double store = B * d * ne * 2.0 / kModelBytes;  // written while the MMAs run
-  return (contraction > store ? contraction : store) + (B * d * ne * 2.0 + d * ne * 4.0) / kModelBytes;
+  if (m == DP_NORM_EXPLICIT) return per_sample + clip_sum + scale_pass + 4 * kModelLaunch;
+  const double store = B * d * ne * 2.0 / kModelStoreBytes;  // written while the MMAs run
+  const double reduce = std::max((B * d * ne * 2.0 + d * ne * 4.0) / kModelBytes, d * ne / kModelNormals);
+  return std::max(per_sample, store) + reduce + 3 * kModelLaunch;
 }
 
 dp_norm_method auto_method(const Shape& s) {
@@ -347,12 +363,12 @@ dp_status bf16_norms_ghost_shared(const Shape& s, const void* X, const void* con
 }
 
 dp_status launch_noise(float* G, unsigned long long total, double std_dev, unsigned long long seed,
-                       unsigned long long step, unsigned layer_id, cudaStream_t stream);
+                       StepRef step, unsigned layer_id, cudaStream_t stream);
 
 // out (+)= A^T Bm over all N rows (A: [N, m], Bm: [N, ne], both bf16, one already scaled by
 // c_i), plus noise when noise_std != 0.  `accumulate` = 0 overwrites out.
 dp_status bf16_clipsum(const Shape& s, const void* A, const void* Bm, float* out, int accumulate,
-                       double noise_std, unsigned long long seed, unsigned long long step,
+                       double noise_std, unsigned long long seed, StepRef step,
                        unsigned layer_id, uint32_t* status, cudaStream_t stream) {
   UmmaParams p = base_params(status);
   const int ne = s.ne();
@@ -393,7 +409,8 @@ dp_status bf16_clipsum(const Shape& s, const void* A, const void* Bm, float* out
   p.key0 = key.k0;
   p.key1 = key.k1;
   p.layer_id = layer_id;
-  p.step_lo = static_cast<uint32_t>(step & 0xFFFFFFFFull);
+  p.step_lo = step.lo;
+  p.step_dev = step.dev;
   dp_status st2 = (BN == 128) ? launch_umma<UmmaConfig<128, kEpiClipSum>>(p, stream)
                               : launch_umma<UmmaConfig<256, kEpiClipSum>>(p, stream);
   if (st2 != DP_OK || fused_noise || noise_std == 0.0) return st2;
@@ -402,17 +419,16 @@ dp_status bf16_clipsum(const Shape& s, const void* A, const void* Bm, float* out
 }
 
 dp_status launch_noise(float* G, unsigned long long total, double std_dev, unsigned long long seed,
-                       unsigned long long step, unsigned layer_id, cudaStream_t stream) {
+                       StepRef step, unsigned layer_id, cudaStream_t stream) {
   LaunchScope scope(kKindNoise, stream);
   // Large G: a persistent grid whose blocks stage the 32 KB of Box-Muller tables once each.
   const PhiloxKey key = philox_key_from_seed(seed);
-  const uint32_t step_lo = static_cast<uint32_t>(step & 0xFFFFFFFFull);
   if (total >= (1ull << 22)) {
     const int grid = std::min(stream_grid((total + 3) / 4, 256), sm_count() * 4);
-    noise_add_kernel<true><<<grid, 256, 0, stream>>>(G, total, std_dev, key, layer_id, step_lo);
+    noise_add_kernel<true><<<grid, 256, 0, stream>>>(G, total, std_dev, key, layer_id, step);
   } else {
     noise_add_kernel<false><<<stream_grid((total + 3) / 4, 256), 256, 0, stream>>>(G, total, std_dev, key,
-                                                                                  layer_id, step_lo);
+                                                                                  layer_id, step);
   }
   DP_CHECK_LAUNCH("noise_add_kernel");
   return DP_OK;
@@ -486,15 +502,15 @@ dp_status launch_finalize(NormSource src, int B, float C, float* norms_out, floa
 template <int BU>
 void reduce_kernel_launch(int grid, size_t smem, cudaStream_t stream, const __nv_bfloat16* gs, int B,
                           long long mn, NormSource src, float C, float* out, double noise_std,
-                          PhiloxKey key, unsigned layer_id, uint32_t step_lo) {
+                          PhiloxKey key, unsigned layer_id, StepRef step) {
   clip_reduce_kernel<BU><<<grid, 256, smem, stream>>>(gs, B, mn, src, C, out, noise_std, key, layer_id,
-                                                      step_lo);
+                                                      step);
 }
 
 template <int BU>
 dp_status reduce_tma_launch(cudaStream_t stream, const __nv_bfloat16* gs, long long mn, NormSource src,
                             float C, float* out, double noise_std, PhiloxKey key, unsigned layer_id,
-                            uint32_t step_lo, uint32_t* status) {
+                            StepRef step, uint32_t* status) {
   using Cfg = ReduceTmaConfig<BU>;
   static bool configured[64] = {false};
   int dev = 0;
@@ -507,28 +523,27 @@ dp_status reduce_tma_launch(cudaStream_t stream, const __nv_bfloat16* gs, long l
   const long long chunks = (mn + kReduceChunk - 1) / kReduceChunk;
   const int grid = static_cast<int>(chunks < sm_count() ? chunks : sm_count());
   clip_reduce_tma_kernel<BU><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(gs, mn, src, C, out, noise_std,
-                                                                               key, layer_id, step_lo, status);
+                                                                               key, layer_id, step, status);
   return DP_OK;
 }
 
 dp_status launch_reduce(const __nv_bfloat16* gs, int B, long long mn, NormSource src, float C,
-                        float* out, double noise_std, unsigned long long seed, unsigned long long step,
+                        float* out, double noise_std, unsigned long long seed, StepRef step,
                         unsigned layer_id, cudaStream_t stream, uint32_t* status) {
   if (B <= 8) {
     // Warp-specialised bulk-copy reduce: noise generation overlaps the HBM stream.
     const PhiloxKey key = philox_key_from_seed(seed);
-    const uint32_t step_lo = static_cast<uint32_t>(step & 0xFFFFFFFFull);
     LaunchScope scope(kKindReduce, stream);
     dp_status st;
     switch (B) {
-      case 1: st = reduce_tma_launch<1>(stream, gs, mn, src, C, out, noise_std, key, layer_id, step_lo, status); break;
-      case 2: st = reduce_tma_launch<2>(stream, gs, mn, src, C, out, noise_std, key, layer_id, step_lo, status); break;
-      case 3: st = reduce_tma_launch<3>(stream, gs, mn, src, C, out, noise_std, key, layer_id, step_lo, status); break;
-      case 4: st = reduce_tma_launch<4>(stream, gs, mn, src, C, out, noise_std, key, layer_id, step_lo, status); break;
-      case 5: st = reduce_tma_launch<5>(stream, gs, mn, src, C, out, noise_std, key, layer_id, step_lo, status); break;
-      case 6: st = reduce_tma_launch<6>(stream, gs, mn, src, C, out, noise_std, key, layer_id, step_lo, status); break;
-      case 7: st = reduce_tma_launch<7>(stream, gs, mn, src, C, out, noise_std, key, layer_id, step_lo, status); break;
-      default: st = reduce_tma_launch<8>(stream, gs, mn, src, C, out, noise_std, key, layer_id, step_lo, status); break;
+      case 1: st = reduce_tma_launch<1>(stream, gs, mn, src, C, out, noise_std, key, layer_id, step, status); break;
+      case 2: st = reduce_tma_launch<2>(stream, gs, mn, src, C, out, noise_std, key, layer_id, step, status); break;
+      case 3: st = reduce_tma_launch<3>(stream, gs, mn, src, C, out, noise_std, key, layer_id, step, status); break;
+      case 4: st = reduce_tma_launch<4>(stream, gs, mn, src, C, out, noise_std, key, layer_id, step, status); break;
+      case 5: st = reduce_tma_launch<5>(stream, gs, mn, src, C, out, noise_std, key, layer_id, step, status); break;
+      case 6: st = reduce_tma_launch<6>(stream, gs, mn, src, C, out, noise_std, key, layer_id, step, status); break;
+      case 7: st = reduce_tma_launch<7>(stream, gs, mn, src, C, out, noise_std, key, layer_id, step, status); break;
+      default: st = reduce_tma_launch<8>(stream, gs, mn, src, C, out, noise_std, key, layer_id, step, status); break;
     }
     if (st != DP_OK) return st;
     DP_CHECK_LAUNCH("clip_reduce_tma_kernel");
@@ -538,18 +553,17 @@ dp_status launch_reduce(const __nv_bfloat16* gs, int B, long long mn, NormSource
   const int grid = std::min(stream_grid(static_cast<unsigned long long>(mn / 8), 256), sm_count() * 2);
   const size_t smem = kNoiseSharedBytes + cached * sizeof(float);
   const PhiloxKey key = philox_key_from_seed(seed);
-  const uint32_t step_lo = static_cast<uint32_t>(step & 0xFFFFFFFFull);
   LaunchScope scope(kKindReduce, stream);
   switch (B) {
-    case 1: reduce_kernel_launch<1>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step_lo); break;
-    case 2: reduce_kernel_launch<2>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step_lo); break;
-    case 3: reduce_kernel_launch<3>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step_lo); break;
-    case 4: reduce_kernel_launch<4>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step_lo); break;
-    case 5: reduce_kernel_launch<5>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step_lo); break;
-    case 6: reduce_kernel_launch<6>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step_lo); break;
-    case 7: reduce_kernel_launch<7>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step_lo); break;
-    case 8: reduce_kernel_launch<8>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step_lo); break;
-    default: reduce_kernel_launch<0>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step_lo); break;
+    case 1: reduce_kernel_launch<1>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step); break;
+    case 2: reduce_kernel_launch<2>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step); break;
+    case 3: reduce_kernel_launch<3>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step); break;
+    case 4: reduce_kernel_launch<4>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step); break;
+    case 5: reduce_kernel_launch<5>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step); break;
+    case 6: reduce_kernel_launch<6>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step); break;
+    case 7: reduce_kernel_launch<7>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step); break;
+    case 8: reduce_kernel_launch<8>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step); break;
+    default: reduce_kernel_launch<0>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step); break;
   }
   static_assert(kReduceUnrolled == 8, "the switch above unrolls up to 8 samples");
   DP_CHECK_LAUNCH("clip_reduce_kernel");
@@ -646,7 +660,7 @@ NormSource ws_norm_source(const Call& c) {
 // G_out (+)= sum_i c_i X_i^T Z_i (+ noise) for norms given by `src`.
 dp_status clipped_sum(Call& c, const void* X, const void* Z, NormSource src, float C, float* out,
                       int accumulate, double noise_std, unsigned long long seed,
-                      unsigned long long step, unsigned layer_id) {
+                      StepRef step, unsigned layer_id) {
   const Shape& s = c.s;
   if (s.dt == DP_F32) {
     dim3 grid(ceil_div(s.ne(), kF32Tile), ceil_div(s.m, kF32Tile));
@@ -654,7 +668,7 @@ dp_status clipped_sum(Call& c, const void* X, const void* Z, NormSource src, flo
     LaunchScope scope(kKindF32ClipSum, c.stream);
     f32_clipsum_kernel<<<grid, 256, 0, c.stream>>>(
         static_cast<const float*>(X), static_cast<const float*>(Z), s.N(), s.T, s.m, s.ne(), src, C,
-        out, accumulate, noise_std, key, layer_id, static_cast<uint32_t>(step & 0xFFFFFFFFull));
+        out, accumulate, noise_std, key, layer_id, step);
     DP_CHECK_LAUNCH("f32_clipsum_kernel");
     return DP_OK;
   }
@@ -837,7 +851,7 @@ dp_status block_group_norms(const dp_layer* layers, const std::vector<int>& g, d
 
 // Layer l's clipped sum with the clip factors of `src` and bound C, plus noise of std sigma C.
 dp_status block_layer_sum(const dp_layer* layers, int l, dp_dtype dt, int B, int T, NormSource src, float C,
-                          float sigma, unsigned long long seed, unsigned long long step, const BlockLayout& Lb,
+                          float sigma, unsigned long long seed, StepRef step, const BlockLayout& Lb,
                           uint8_t* ws, cudaStream_t stream) {
   const dp_layer& y = layers[l];
   const Shape s = layer_shape(y, B, T, dt);
@@ -865,7 +879,7 @@ NormSource layer_norm_source(const BlockLayout& Lb, uint8_t* ws, int l, int B, d
 }
 
 dp_status block_step(const dp_layer* layers, int L, dp_dtype dt, int B, int T, dp_clip_mode mode, float C,
-                     float sigma, unsigned long long seed, unsigned long long step, const BlockLayout& Lb,
+                     float sigma, unsigned long long seed, StepRef step, const BlockLayout& Lb,
                      float* flat_norms_out, uint8_t* ws, cudaStream_t stream) {
   dp_status st;
   // Status word, and the fp32 path's atomic norm accumulators, start at zero.
@@ -997,7 +1011,7 @@ dp_status dp_clip_accumulate(const void* X, const void* dY, const void* P, int r
   const void* Z;
   if ((st = clip_space_operand(c, dY, P, false, 0, 0, &Z)) != DP_OK) return st;
   NormSource src{nullptr, nullptr, norms};
-  return clipped_sum(c, X, Z, src, C, G_sum, 1, 0.0, 0, 0, 0);
+  return clipped_sum(c, X, Z, src, C, G_sum, 1, 0.0, 0, step_value(0), 0);
 }
 
 dp_status dp_add_noise(float* G, long long rows, long long cols, float std, unsigned long long seed,
@@ -1007,7 +1021,7 @@ dp_status dp_add_noise(float* G, long long rows, long long cols, float std, unsi
   if (rows > (1ll << 34) / cols) return DP_ERR_INVALID_ARG;
   const unsigned long long total = static_cast<unsigned long long>(rows) * static_cast<unsigned long long>(cols);
   if (std == 0.0f) return DP_OK;
-  return launch_noise(G, total, static_cast<double>(std), seed, step, layer_id,
+  return launch_noise(G, total, static_cast<double>(std), seed, step_value(step), layer_id,
                       static_cast<cudaStream_t>(stream));
 }
 
@@ -1020,10 +1034,10 @@ dp_status dp_projection_matrix(void* P, dp_dtype dt, int d_out, int r, unsigned 
   return launch_projection(P, dt, d_out, r, seed, layer_id, static_cast<cudaStream_t>(stream));
 }
 
-dp_status dp_linear_step(const void* X, const void* dY, const void* P, int r, dp_dtype dt, int B, int T,
-                         int d_in, int d_out, float C, float sigma, unsigned long long seed,
-                         unsigned long long step, unsigned layer_id, dp_norm_method method,
-                         float* norms_out, float* G_out, void* workspace, size_t ws_bytes, void* stream) {
+dp_status linear_step(const void* X, const void* dY, const void* P, int r, dp_dtype dt, int B, int T, int d_in,
+                      int d_out, float C, float sigma, unsigned long long seed, StepRef step, unsigned layer_id,
+                      dp_norm_method method, float* norms_out, float* G_out, void* workspace, size_t ws_bytes,
+                      void* stream) {
   Call c;
   if (method < DP_NORM_AUTO || method > DP_NORM_ONCE) return DP_ERR_INVALID_ARG;
   dp_status st = check_common(X, dY, P, r, dt, B, T, d_in, d_out, workspace, ws_bytes, true,
@@ -1053,6 +1067,24 @@ dp_status dp_linear_step(const void* X, const void* dY, const void* P, int r, dp
     return launch_reduce(reinterpret_cast<const __nv_bfloat16*>(c.ws + c.L.gs), B, mn, src, C, G_out,
                          noise_std, seed, step, layer_id, c.stream, c.status());
   return clipped_sum(c, X, Z, src, C, G_out, 0, noise_std, seed, step, layer_id);
+}
+
+dp_status dp_linear_step(const void* X, const void* dY, const void* P, int r, dp_dtype dt, int B, int T,
+                         int d_in, int d_out, float C, float sigma, unsigned long long seed,
+                         unsigned long long step, unsigned layer_id, dp_norm_method method,
+                         float* norms_out, float* G_out, void* workspace, size_t ws_bytes, void* stream) {
+  return linear_step(X, dY, P, r, dt, B, T, d_in, d_out, C, sigma, seed, step_value(step), layer_id, method,
+                     norms_out, G_out, workspace, ws_bytes, stream);
+}
+
+dp_status dp_linear_step_dev_step(const void* X, const void* dY, const void* P, int r, dp_dtype dt, int B,
+                                  int T, int d_in, int d_out, float C, float sigma, unsigned long long seed,
+                                  const unsigned long long* step_dev, unsigned layer_id, dp_norm_method method,
+                                  float* norms_out, float* G_out, void* workspace, size_t ws_bytes,
+                                  void* stream) {
+  if (!step_dev || (reinterpret_cast<uintptr_t>(step_dev) & 7u) != 0) return DP_ERR_INVALID_ARG;
+  return linear_step(X, dY, P, r, dt, B, T, d_in, d_out, C, sigma, seed, StepRef{0u, step_dev}, layer_id,
+                     method, norms_out, G_out, workspace, ws_bytes, stream);
 }
 
 dp_status dp_philox_blocks(unsigned* out, unsigned long long nblocks, unsigned long long seed,
@@ -1125,10 +1157,9 @@ size_t dp_block_workspace_size(const dp_layer* layers, int L, int B, int T, dp_d
   return block_layout(layers, L, B, T, dt, mode, methods).total;
 }
 
-dp_status dp_block_step(const dp_layer* layers, int L, dp_dtype dt, int B, int T, dp_clip_mode mode,
-                        float C, float sigma, unsigned long long seed, unsigned long long step,
-                        dp_norm_method method, float* flat_norms_out, void* workspace, size_t ws_bytes,
-                        void* stream) {
+dp_status block_step_entry(const dp_layer* layers, int L, dp_dtype dt, int B, int T, dp_clip_mode mode,
+                           float C, float sigma, unsigned long long seed, StepRef step, dp_norm_method method,
+                           float* flat_norms_out, void* workspace, size_t ws_bytes, void* stream) {
   if (!layers || L < 1 || !workspace) return DP_ERR_INVALID_ARG;
   if (mode != DP_CLIP_PER_LAYER && mode != DP_CLIP_FLAT) return DP_ERR_INVALID_ARG;
   if (method < DP_NORM_AUTO || method > DP_NORM_ONCE) return DP_ERR_INVALID_ARG;
@@ -1150,6 +1181,23 @@ dp_status dp_block_step(const dp_layer* layers, int L, dp_dtype dt, int B, int T
   if (dt == DP_BF16 && (st = get_encoder()) != DP_OK) return st;
   return block_step(layers, L, dt, B, T, mode, C, sigma, seed, step, Lb, flat_norms_out,
                     static_cast<uint8_t*>(workspace), static_cast<cudaStream_t>(stream));
+}
+
+dp_status dp_block_step(const dp_layer* layers, int L, dp_dtype dt, int B, int T, dp_clip_mode mode,
+                        float C, float sigma, unsigned long long seed, unsigned long long step,
+                        dp_norm_method method, float* flat_norms_out, void* workspace, size_t ws_bytes,
+                        void* stream) {
+  return block_step_entry(layers, L, dt, B, T, mode, C, sigma, seed, step_value(step), method, flat_norms_out,
+                          workspace, ws_bytes, stream);
+}
+
+dp_status dp_block_step_dev_step(const dp_layer* layers, int L, dp_dtype dt, int B, int T, dp_clip_mode mode,
+                                 float C, float sigma, unsigned long long seed,
+                                 const unsigned long long* step_dev, dp_norm_method method,
+                                 float* flat_norms_out, void* workspace, size_t ws_bytes, void* stream) {
+  if (!step_dev || (reinterpret_cast<uintptr_t>(step_dev) & 7u) != 0) return DP_ERR_INVALID_ARG;
+  return block_step_entry(layers, L, dt, B, T, mode, C, sigma, seed, StepRef{0u, step_dev}, method,
+                          flat_norms_out, workspace, ws_bytes, stream);
 }
 
 size_t dp_adam_workspace_size(int d_in, int r) {

@@ -36,6 +36,20 @@ struct PhiloxKey {
   uint32_t k0, k1;
 };
 
+// The step number of the noise counter: fixed at launch, or read from device memory when the
+// kernel runs, so that one CUDA graph captured once serves every training step.
+struct StepRef {
+  uint32_t lo;                      // step mod 2^32, used when dev is null
+  const unsigned long long* dev;    // DEVICE address of the step, or null
+  __device__ __forceinline__ uint32_t get() const {
+    return dev ? static_cast<uint32_t>(*dev & 0xFFFFFFFFull) : lo;
+  }
+};
+
+inline StepRef step_value(unsigned long long step) {
+  return StepRef{static_cast<uint32_t>(step & 0xFFFFFFFFull), nullptr};
+}
+
 __host__ __device__ inline PhiloxKey philox_key_from_seed(unsigned long long seed) {
   return PhiloxKey{static_cast<uint32_t>(seed & 0xFFFFFFFFull), static_cast<uint32_t>(seed >> 32)};
 }

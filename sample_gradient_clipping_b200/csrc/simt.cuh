@@ -21,8 +21,9 @@ namespace dpclip {
 // they are read through the read-only cache, which saves the copy's latency on small G.
 template <bool STAGED>
 __global__ void noise_add_kernel(float* __restrict__ G, unsigned long long total, double std_dev,
-                                 PhiloxKey key, uint32_t layer_id, uint32_t step_lo) {
+                                 PhiloxKey key, uint32_t layer_id, StepRef step) {
   __shared__ double2 tab_s[STAGED ? kNoiseSharedEntries : 1];
+  const uint32_t step_lo = step.get();
   if constexpr (STAGED) {
     stage_noise_tables(tab_s);
     __syncthreads();
@@ -200,7 +201,8 @@ __global__ void scale_rows_bf16_kernel(const __nv_bfloat16* __restrict__ in,
 template <int BU>  // compile-time sample count, or 0 for a runtime loop
 __global__ void __launch_bounds__(256, 2) clip_reduce_kernel(
     const __nv_bfloat16* __restrict__ Gs, int B, long long mn, NormSource src, float C,
-    float* __restrict__ out, double noise_std, PhiloxKey key, uint32_t layer_id, uint32_t step_lo) {
+    float* __restrict__ out, double noise_std, PhiloxKey key, uint32_t layer_id, StepRef step) {
+  const uint32_t step_lo = step.get();
   extern __shared__ double2 reduce_smem[];  // noise tables, then the cached clip factors
   float* c_smem = reinterpret_cast<float*>(reduce_smem + kNoiseSharedEntries);
   const int cached = B < kReduceCachedSamples ? B : kReduceCachedSamples;
@@ -308,7 +310,8 @@ struct ReduceTmaConfig {
 template <int BU>
 __global__ void __launch_bounds__(ReduceTmaConfig<BU>::THREADS, 1) clip_reduce_tma_kernel(
     const __nv_bfloat16* __restrict__ Gs, long long mn, NormSource src, float C, float* __restrict__ out,
-    double noise_std, PhiloxKey key, uint32_t layer_id, uint32_t step_lo, uint32_t* status) {
+    double noise_std, PhiloxKey key, uint32_t layer_id, StepRef step, uint32_t* status) {
+  const uint32_t step_lo = step.get();
   using Cfg = ReduceTmaConfig<BU>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -498,7 +501,8 @@ __global__ void __launch_bounds__(256) f32_norm_kernel(const float* __restrict__
 __global__ void __launch_bounds__(256) f32_clipsum_kernel(
     const float* __restrict__ X, const float* __restrict__ dY, long long N, int T, int m, int n,
     NormSource src, float C, float* __restrict__ out, int add_mode, double noise_std, PhiloxKey key,
-    uint32_t layer_id, uint32_t step_lo) {
+    uint32_t layer_id, StepRef step) {
+  const uint32_t step_lo = step.get();
   __shared__ float xs[kF32Tile][kF32Tile + 1];
   __shared__ float ds[kF32Tile][kF32Tile + 1];
   __shared__ float cs[kF32Tile];

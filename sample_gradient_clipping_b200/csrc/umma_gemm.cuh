@@ -72,6 +72,7 @@ struct alignas(64) UmmaParams {
   __nv_bfloat16* out_bf16;
   double noise_std;           // 0 disables the noise
   uint32_t key0, key1, layer_id, step_lo;
+  const unsigned long long* step_dev;  // non-null: the step is read here when the kernel runs
   float alpha;                // axpy: W += alpha * acc
   float* partials;            // [B][partial_stride] per-warp squared-norm partials
   int partial_stride;         // slots per sample: 4 per unit of that sample
@@ -235,6 +236,7 @@ __device__ __forceinline__ void epilogue_unit(const UmmaParams& p, const Unit& w
     const bool row_ok = grow < p.out_rows;
     const bool noisy = (p.noise_std != 0.0) && (w.split == 0);
     const PhiloxKey key{p.key0, p.key1};
+    const uint32_t step_lo = StepRef{p.step_lo, p.step_dev}.get();
 #pragma unroll 1
     for (int c0 = 0; c0 < Cfg::BN; c0 += 32) {
       float v[32];
@@ -251,7 +253,7 @@ __device__ __forceinline__ void epilogue_unit(const UmmaParams& p, const Unit& w
         if (noisy) {
           const unsigned long long k = static_cast<unsigned long long>(grow) * p.out_cols + gcol0 + 4 * q;
           double z[4];
-          normals4(static_cast<uint32_t>(k >> 2), p.layer_id, p.step_lo, kStreamNoise, key, z);
+          normals4(static_cast<uint32_t>(k >> 2), p.layer_id, step_lo, kStreamNoise, key, z);
           val.x = static_cast<float>(static_cast<double>(val.x) + p.noise_std * z[0]);
           val.y = static_cast<float>(static_cast<double>(val.y) + p.noise_std * z[1]);
           val.z = static_cast<float>(static_cast<double>(val.z) + p.noise_std * z[2]);
