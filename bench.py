@@ -54,6 +54,13 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--shard", action="store_true",
+                    help="under torchrun: each rank holds its own batch of the workload's size and "
+                         "the ranks run one sample-sharded step (NCCL all-reduce of every linear's "
+                         "sum, noise added once); default: independent replicas")
+    ap.add_argument("--graph", action="store_true",
+                    help="replay one CUDA graph per step; the step number lives in device memory and "
+                         "the graph advances it")
     ap.add_argument("--no-non-dp", action="store_true",
                     help="skip the non-private comparison (plain bf16 weight-gradient GEMMs)")
     ap.add_argument("--method", default="auto", choices=["auto", "ghost", "explicit", "once"])
@@ -143,7 +150,12 @@ def ghost_flops(w):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 100 ms during the timed region."""
+    """nvidia-smi clocks and throttle reasons sampled every 100 ms during the timed region.
+
+    start() returns once the first sample has arrived, so the sampler is live when timing
+    begins; stop() waits for one sample taken after the region, so a region shorter than the
+    sampling interval still has a sample on each side of it.
+    """
 
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
@@ -151,6 +163,8 @@ class ClockSampler:
 
     def __init__(self, device_index):
         self.proc = None
+        self.lines = []
+        self.reader = None
         try:
             import torch
 
@@ -160,7 +174,13 @@ class ClockSampler:
             target = str(device_index)
         self.target = target
 
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.monotonic(), line))
+
     def start(self):
+        import threading
+
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", self.target, f"--query-gpu={self.FIELDS}",
@@ -168,19 +188,30 @@ class ClockSampler:
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
+            return
+        self.reader = threading.Thread(target=self._read, daemon=True)
+        self.reader.start()
+        deadline = time.monotonic() + 5.0
+        while not self.lines and time.monotonic() < deadline and self.proc.poll() is None:
+            time.sleep(0.01)
 
     def stop(self):
         if self.proc is None:
             return None
+        t_stop = time.monotonic()
+        deadline = t_stop + 1.0
+        while time.monotonic() < deadline and not any(t > t_stop for t, _ in self.lines):
+            time.sleep(0.01)
         self.proc.terminate()
         try:
-            out, _ = self.proc.communicate(timeout=5)
+            self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
-            out, _ = self.proc.communicate()
+        if self.reader is not None:
+            self.reader.join(timeout=2)
         sm, mx, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in out.splitlines():
+        for _, line in self.lines:
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 7:
                 continue
@@ -276,7 +307,11 @@ def run_ours(args, w, rank, world):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     _lib.lib()
-    data = inputs.generate(w)
+    shard = args.shard and world > 1
+    if shard and (w.r or args.graph):
+        raise SystemExit("--shard runs unprojected workloads without --graph")
+    # Sharded: every rank draws its own samples (the noise seed stays the workload's).
+    data = inputs.generate(dataclasses.replace(w, seed=w.seed + 7919 * rank) if shard else w)
     X = {k: v.to(dev) for k, v in data["X"].items()}
     dY = {k: v.to(dev) for k, v in data["dY"].items()}
     r = w.r
@@ -285,7 +320,9 @@ def run_ours(args, w, rank, world):
                    for l in w.linears)
     G = {l.name: torch.empty(l.d_in, r or l.d_out, dtype=torch.float32, device=dev) for l in w.linears}
     norms = {l.name: torch.empty(w.B, dtype=torch.float32, device=dev) for l in w.linears}
-    stream = torch.cuda.current_stream(dev)
+    # A graph is captured on a side stream; everything then runs on that stream.
+    stream = torch.cuda.Stream(dev) if args.graph else torch.cuda.current_stream(dev)
+    torch.cuda.set_stream(stream)
     # The projection depends on (seed, layer) only, not on the step: it is generated once per
     # linear, as a training loop would, and passed to every step.
     P = {l.name: _lib.dp_projection_matrix(torch.empty(l.d_out, r, dtype=X[l.x_key].dtype, device=dev),
@@ -309,15 +346,24 @@ def run_ours(args, w, rank, world):
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     flat_norms = torch.empty(w.B, dtype=torch.float32, device=dev)
 
+    if shard:
+        from sample_gradient_clipping_b200 import sharded
+
+        shard_ops = sharded.LibraryOps(args.method)
+
     def step(k):
+        k = w.step + k if isinstance(k, int) else k   # a number, or the device step counter
+        if shard:
+            sharded.sharded_step(block, w.sigma, w.seed, k, mode=args.clip, C=flat_C, ops=shard_ops)
+            return
         if use_block:
             _lib.dp_block_step(block, mode=args.clip, C=flat_C if args.clip == "flat" else w.C, sigma=w.sigma,
-                               seed=w.seed, step=w.step + k, method=args.method,
+                               seed=w.seed, step=k, method=args.method,
                                flat_norms_out=flat_norms if args.clip == "flat" else None, workspace=ws,
                                stream=stream)
             return
         for l in w.linears:
-            _lib.dp_linear_step(X[l.x_key], dY[l.name], w.C, w.sigma, w.seed, w.step + k, l.layer_id,
+            _lib.dp_linear_step(X[l.x_key], dY[l.name], w.C, w.sigma, w.seed, k, l.layer_id,
                                 P=P.get(l.name), r=r, method=args.method, norms_out=norms[l.name],
                                 G_out=G[l.name], workspace=ws, stream=stream)
 
@@ -327,13 +373,26 @@ def run_ours(args, w, rank, world):
     if _lib.dp_workspace_status(ws, stream) != _lib.DP_OK:
         raise RuntimeError("an in-kernel wait timed out during warm-up")
 
+    graph, graph_launches = None, 0
+    if args.graph:
+        # The step counter starts where the ordinary steps of the timed pass would, and the
+        # graph increments it after each step, so every replay draws the next step's noise.
+        step_dev = torch.full((1,), w.step + args.warmup, dtype=torch.int64, device=dev)
+        graph = torch.cuda.CUDAGraph()
+        l0 = _lib.kernel_launches()
+        with torch.cuda.graph(graph, stream=stream):
+            step(step_dev)
+            step_dev.add_(1)
+        graph_launches = _lib.kernel_launches() - l0
+        graph.replay()
+        torch.cuda.synchronize(dev)
+        step_dev.fill_(w.step + args.warmup)
+
     def barrier():
         if world > 1:
             torch.distributed.barrier()
 
     sampler = ClockSampler(local)
-    _lib.profiling_enable(True)
-    _lib.profiling_collect()
     barrier()
     torch.cuda.synchronize(dev)
     sampler.start()
@@ -341,15 +400,32 @@ def run_ours(args, w, rank, world):
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ev0.record(stream)
     for k in range(args.steps):
-        step(args.warmup + k)
+        if graph is not None:
+            graph.replay()
+        else:
+            step(args.warmup + k)
     ev1.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
-    launches = _lib.kernel_launches() - launches0
+    # Graph replays launch the kernels the capture recorded; the host counter saw them once.
+    launches = graph_launches * args.steps if graph is not None else _lib.kernel_launches() - launches0
     clocks = sampler.stop()
+    ms = ev0.elapsed_time(ev1) / args.steps
+    # Per-kernel device times come from a second pass over the same steps with a CUDA event
+    # pair around every launch.  The events cost a few microseconds a launch, which is noise
+    # on the Llama blocks but a large share of the small workloads' steps, so they stay out of
+    # the pass that gives `value`.
+    _lib.profiling_enable(True)
+    _lib.profiling_collect()
+    pv0, pv1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    pv0.record(stream)
+    for k in range(args.steps):
+        step(args.warmup + k)
+    pv1.record(stream)
+    torch.cuda.synchronize(dev)
     prof = _lib.profiling_collect()
     _lib.profiling_enable(False)
-    ms = ev0.elapsed_time(ev1) / args.steps
+    profiled_ms = pv0.elapsed_time(pv1) / args.steps
     if _lib.dp_workspace_status(ws, stream) != _lib.DP_OK:
         raise RuntimeError("an in-kernel wait timed out during the timed steps")
     ms = max_over_ranks(ms, dev, world)
@@ -361,7 +437,9 @@ def run_ours(args, w, rank, world):
 
     # ---- end to end through the public API with host buffers
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and shard:
+        e2e = {"unavailable": "the end-to-end leg times the one-GPU call; run it without --shard"}
+    elif not args.no_e2e:
         e2e = run_e2e(args, w, data, dev, stream, r, P, _lib, torch, world)
 
     if rank != 0:
@@ -400,7 +478,7 @@ def run_ours(args, w, rank, world):
                         "peak_kind": (f"{pk_kind} HBM copy bandwidth" if unit == "GB/s" else
                                       f"{pk_kind} sustained bf16 (kernel timed inside a long step)"),
                         "launches": d_n // args.steps, "avg_launch_ms": d_ms / d_n,
-                        "share_of_step": d_ms / (ms * args.steps)}
+                        "share_of_step": d_ms / (profiled_ms * args.steps)}
     line = {
         "metric": METRIC, "value": job_tokens_per_second(w.tokens, world, ms), "unit": "tokens/s",
         "n_gpus": world,
@@ -408,7 +486,10 @@ def run_ours(args, w, rank, world):
         "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "T": w.T, "linears": len(w.linears),
                    "method": args.method, "clip": args.clip, "l2": "inputs larger than L2 (no flush)",
-                   "parallelism": "replicas" if world > 1 else "1 GPU",
+                   "launch": ("one CUDA graph replay per step (device-resident step counter)" if args.graph
+                              else "library calls from the host every step"),
+                   "parallelism": (f"dp{world}: samples sharded, one NCCL all-reduce per linear, noise "
+                                   "added once" if shard else "replicas" if world > 1 else "1 GPU"),
                    **({"projection": f"P [d_out, {r}] generated once per linear before timing "
                                      "(it depends on seed and layer only)"} if r else {}),
                    "description": w.description},
@@ -420,6 +501,9 @@ def run_ours(args, w, rank, world):
         "roofline": roofline,
         "kernels": {k: {"ms_per_step": v[0] / args.steps, "launches_per_step": v[1] / args.steps}
                     for k, v in sorted(kinds.items(), key=lambda kv: -kv[1][0])},
+        "kernel_timing": {"how": "CUDA events around every launch, in a second pass over the same steps"
+                                 + (" launched from the host (no graph)" if args.graph else ""),
+                          "ms_per_step_with_events": profiled_ms},
         "gpu_launches": launches,
         "clocks": clocks,
         "e2e": e2e,
