@@ -499,12 +499,10 @@ dp_status launch_finalize(NormSource src, int B, float C, float* norms_out, floa
   return DP_OK;
 }
 
-template <int BU>
 void reduce_kernel_launch(int grid, size_t smem, cudaStream_t stream, const __nv_bfloat16* gs, int B,
-                          long long mn, NormSource src, float C, float* out, double noise_std,
-                          PhiloxKey key, unsigned layer_id, StepRef step) {
-  clip_reduce_kernel<BU><<<grid, 256, smem, stream>>>(gs, B, mn, src, C, out, noise_std, key, layer_id,
-                                                      step);
+                          long long mn, NormSource src, float C, float* out, double noise_std, PhiloxKey key,
+                          unsigned layer_id, StepRef step) {
+  clip_reduce_kernel<<<grid, 256, smem, stream>>>(gs, B, mn, src, C, out, noise_std, key, layer_id, step);
 }
 
 template <int BU>
@@ -554,18 +552,8 @@ dp_status launch_reduce(const __nv_bfloat16* gs, int B, long long mn, NormSource
   const size_t smem = kNoiseSharedBytes + cached * sizeof(float);
   const PhiloxKey key = philox_key_from_seed(seed);
   LaunchScope scope(kKindReduce, stream);
-  switch (B) {
-    case 1: reduce_kernel_launch<1>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step); break;
-    case 2: reduce_kernel_launch<2>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step); break;
-    case 3: reduce_kernel_launch<3>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step); break;
-    case 4: reduce_kernel_launch<4>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step); break;
-    case 5: reduce_kernel_launch<5>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step); break;
-    case 6: reduce_kernel_launch<6>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step); break;
-    case 7: reduce_kernel_launch<7>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step); break;
-    case 8: reduce_kernel_launch<8>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step); break;
-    default: reduce_kernel_launch<0>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step); break;
-  }
-  static_assert(kReduceUnrolled == 8, "the switch above unrolls up to 8 samples");
+  // B > 8 here (smaller batches take the bulk-copy kernel above): a runtime sample loop.
+  reduce_kernel_launch(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step);
   DP_CHECK_LAUNCH("clip_reduce_kernel");
   return DP_OK;
 }

@@ -98,10 +98,8 @@ __global__ void projection_kernel(void* __restrict__ P, unsigned long long total
   }
 }
 
-// Clip factors that clip_reduce_kernel keeps in shared memory (the rest are recomputed), and
-// the largest sample count whose loads it unrolls.
+// Clip factors that clip_reduce_kernel keeps in shared memory (the rest are recomputed).
 constexpr int kReduceCachedSamples = 4096;
-constexpr int kReduceUnrolled = 8;
 
 // Clip factor of sample i from either squared-norm accumulators or final norms.
 __device__ __forceinline__ float clip_factor(float norm, float C) {
@@ -191,14 +189,13 @@ __global__ void scale_rows_bf16_kernel(const __nv_bfloat16* __restrict__ in,
 
 // out[e] = fp32(sum_i c_i Gs[i][e] + std * z_e) over the per-sample bf16 gradients that the
 // explicit-store pass left in the workspace: the clipped sum without forming any G_i again.
+// This is the kernel for B > 8 samples (smaller batches take clip_reduce_tma_kernel below).
 //
 // Each thread owns 8 consecutive elements: two Philox blocks and four independent fp64
 // Box-Muller pairs.  The noise sigma C z is rounded to fp32 once and added to the fp32 sum
 // (one conversion an element instead of two; the result is within 1 ulp of the fp64 sum
-// rounded once).  The loads of all samples are issued first (for B <= kReduceUnrolled the
-// loop is unrolled), the noise is computed while they are in flight, and then the sum is
-// formed.  This keeps both the fp64 pipe and HBM busy instead of alternating between them.
-template <int BU>  // compile-time sample count, or 0 for a runtime loop
+// rounded once).  A persistent grid of two blocks per SM; each block stages the Box-Muller
+// tables in shared memory once.
 __global__ void __launch_bounds__(256, 2) clip_reduce_kernel(
     const __nv_bfloat16* __restrict__ Gs, int B, long long mn, NormSource src, float C,
     float* __restrict__ out, double noise_std, PhiloxKey key, uint32_t layer_id, StepRef step) {
@@ -211,71 +208,29 @@ __global__ void __launch_bounds__(256, 2) clip_reduce_kernel(
   __syncthreads();
   const NoiseTablesShared tab{reduce_smem};
   const long long nvec = mn / 8;  // 16-byte vectors per sample
-  const long long v0 = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x;
-  uint4 pk_next[BU > 0 ? BU : 1];
-  if constexpr (BU > 0) {
-    if (v0 < nvec) {
-#pragma unroll
-      for (int i = 0; i < BU; ++i)
-        pk_next[i] = __ldcs(reinterpret_cast<const uint4*>(Gs) + v0 + static_cast<long long>(i) * nvec);
-    }
-  }
-  for (long long v = v0; v < nvec; v += static_cast<long long>(gridDim.x) * blockDim.x) {
+  for (long long v = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; v < nvec;
+       v += static_cast<long long>(gridDim.x) * blockDim.x) {
     const uint4* g = reinterpret_cast<const uint4*>(Gs) + v;
     float acc[8];
 #pragma unroll
     for (int q = 0; q < 8; ++q) acc[q] = 0.f;
-    double z[8];
-    if constexpr (BU > 0) {
-      // Software pipeline: this iteration's vectors were loaded by the previous iteration
-      // (or the prologue), and the next iteration's loads are issued before the noise of this
-      // one is computed, so HBM stays busy while the fp64 pipe works.
-      uint4 pk[BU > 0 ? BU : 1];
+    for (int i = 0; i < B; ++i) {
+      const float c = i < cached ? c_smem[i] : clip_factor(src.norm(i), C);
+      const uint4 pk = __ldcs(g + static_cast<long long>(i) * nvec);
+      const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&pk);
 #pragma unroll
-      for (int i = 0; i < BU; ++i) pk[i] = pk_next[i];
-      const long long vn = v + static_cast<long long>(gridDim.x) * blockDim.x;
-      if (vn < nvec) {
-        const uint4* gn = reinterpret_cast<const uint4*>(Gs) + vn;
-#pragma unroll
-        for (int i = 0; i < BU; ++i) pk_next[i] = __ldcs(gn + static_cast<long long>(i) * nvec);
-      }
-      if (noise_std != 0.0) {
-        normals4(static_cast<uint32_t>(2 * v), layer_id, step_lo, kStreamNoise, key,
-                 *reinterpret_cast<double(*)[4]>(z), tab);
-        normals4(static_cast<uint32_t>(2 * v + 1), layer_id, step_lo, kStreamNoise, key,
-                 *reinterpret_cast<double(*)[4]>(z + 4), tab);
-      }
-#pragma unroll
-      for (int i = 0; i < BU; ++i) {
-        const float c = c_smem[i];
-        const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&pk[i]);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 f = __bfloat1622float2(hv[e]);
-          acc[2 * e] = fmaf(c, f.x, acc[2 * e]);
-          acc[2 * e + 1] = fmaf(c, f.y, acc[2 * e + 1]);
-        }
-      }
-    } else {
-      for (int i = 0; i < B; ++i) {
-        const float c = i < cached ? c_smem[i] : clip_factor(src.norm(i), C);
-        const uint4 pk = __ldcs(g + static_cast<long long>(i) * nvec);
-        const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&pk);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 f = __bfloat1622float2(hv[e]);
-          acc[2 * e] = fmaf(c, f.x, acc[2 * e]);
-          acc[2 * e + 1] = fmaf(c, f.y, acc[2 * e + 1]);
-        }
-      }
-      if (noise_std != 0.0) {
-        normals4(static_cast<uint32_t>(2 * v), layer_id, step_lo, kStreamNoise, key,
-                 *reinterpret_cast<double(*)[4]>(z), tab);
-        normals4(static_cast<uint32_t>(2 * v + 1), layer_id, step_lo, kStreamNoise, key,
-                 *reinterpret_cast<double(*)[4]>(z + 4), tab);
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(hv[e]);
+        acc[2 * e] = fmaf(c, f.x, acc[2 * e]);
+        acc[2 * e + 1] = fmaf(c, f.y, acc[2 * e + 1]);
       }
     }
     if (noise_std != 0.0) {
+      double z[8];
+      normals4(static_cast<uint32_t>(2 * v), layer_id, step_lo, kStreamNoise, key,
+               *reinterpret_cast<double(*)[4]>(z), tab);
+      normals4(static_cast<uint32_t>(2 * v + 1), layer_id, step_lo, kStreamNoise, key,
+               *reinterpret_cast<double(*)[4]>(z + 4), tab);
 #pragma unroll
       for (int q = 0; q < 8; ++q) acc[q] = acc[q] + __double2float_rn(noise_std * z[q]);
     }
