@@ -65,6 +65,7 @@ def parse():
                     help="skip the non-private comparison (plain bf16 weight-gradient GEMMs)")
     ap.add_argument("--method", default="auto", choices=["auto", "ghost", "explicit", "once"])
     ap.add_argument("--linears", default="", help="comma-separated subset of the workload's linears")
+    ap.add_argument("--sigma", type=float, default=None, help="noise multiplier (default: the workload's)")
     ap.add_argument("--clip", default="per_layer", choices=["per_layer", "flat"],
                     help="per-layer bounds C_l, or one flat bound sqrt(L) * C_l for the whole block")
     return ap.parse_args()
@@ -650,6 +651,8 @@ def main():
         if not lins:
             raise SystemExit(f"no linear of {w.name} in {keep}")
         w = dataclasses.replace(w, name=f"{w.name}[{args.linears}]", linears=lins)
+    if args.sigma is not None:
+        w = dataclasses.replace(w, name=f"{w.name}[sigma={args.sigma:g}]", sigma=args.sigma)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if args.impl == "reference":

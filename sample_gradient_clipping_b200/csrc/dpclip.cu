@@ -237,7 +237,10 @@ dp_status launch_umma_pair(const UmmaParams& p, cudaStream_t stream) {
   if (p.num_units <= 0) return DP_OK;
   const int pairs_avail = sm_count() / 2;
   const int pairs = p.num_units < pairs_avail ? p.num_units : pairs_avail;
-  LaunchScope scope(Cfg::EPI == kEpiExplicitStore ? kKindExplicitStore : kKindExplicitNorm, stream);
+  constexpr int kind = Cfg::EPI == kEpiExplicitStore ? kKindExplicitStore
+                       : Cfg::EPI == kEpiClipSum     ? kKindClipSum
+                                                     : kKindExplicitNorm;
+  LaunchScope scope(kind, stream);
   umma_pair_kernel<Cfg><<<2 * pairs, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(p);
   DP_CHECK_LAUNCH("umma_pair_kernel");
   return DP_OK;
@@ -373,16 +376,20 @@ dp_status bf16_clipsum(const Shape& s, const void* A, const void* Bm, float* out
   UmmaParams p = base_params(status);
   const int ne = s.ne();
   const int BN = ne <= 128 ? 128 : 256;
+  // 256 x 256 tiles on SM pairs when both output dimensions fill them: half the operand
+  // traffic per SM of a 128 x 256 one-SM tile.
+  const bool pair = (s.m >= 256 && ne >= 256);
   dp_status st;
   if ((st = map_2d(&p.tmA0, A, s.N(), s.m, 64)) != DP_OK) return st;
   if ((st = map_2d(&p.tmB0, Bm, s.N(), ne, 64)) != DP_OK) return st;
-  p.m_tiles = ceil_div(s.m, 128);
+  p.m_tiles = pair ? ceil_div(s.m, 256) : ceil_div(s.m, 128);
   p.n_tiles = ceil_div(ne, BN);
   p.k_blocks = ceil_div(s.N(), 64);
   const int tiles = p.m_tiles * p.n_tiles;
+  const int slots = pair ? sm_count() / 2 : sm_count();  // CTAs (or pairs) that run at once
   int splits = 1;
-  if (tiles < sm_count()) {
-    splits = sm_count() / tiles;
+  if (tiles < slots) {
+    splits = slots / tiles;
     const int max_splits = p.k_blocks / 4 > 0 ? p.k_blocks / 4 : 1;
     if (splits > max_splits) splits = max_splits;
     if (splits < 1) splits = 1;
@@ -411,8 +418,9 @@ dp_status bf16_clipsum(const Shape& s, const void* A, const void* Bm, float* out
   p.layer_id = layer_id;
   p.step_lo = step.lo;
   p.step_dev = step.dev;
-  dp_status st2 = (BN == 128) ? launch_umma<UmmaConfig<128, kEpiClipSum>>(p, stream)
-                              : launch_umma<UmmaConfig<256, kEpiClipSum>>(p, stream);
+  dp_status st2 = pair        ? launch_umma_pair<Umma2Config<kEpiClipSum>>(p, stream)
+                  : (BN == 128) ? launch_umma<UmmaConfig<128, kEpiClipSum>>(p, stream)
+                                : launch_umma<UmmaConfig<256, kEpiClipSum>>(p, stream);
   if (st2 != DP_OK || fused_noise || noise_std == 0.0) return st2;
   return launch_noise(out, static_cast<unsigned long long>(s.m) * ne, noise_std, seed, step, layer_id,
                       stream);

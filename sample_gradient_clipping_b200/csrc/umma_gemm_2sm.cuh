@@ -1,6 +1,8 @@
-// Two-SM (cta_group::2) variant of the per-sample explicit contraction for sm_100a.
+// Two-SM (cta_group::2) variant of the per-sample explicit contraction and of the clipped
+// sum, for sm_100a.
 //
-// A cluster of two CTAs on two SMs computes one 256 x 256 tile of G_i = X_i^T dY_i.
+// A cluster of two CTAs on two SMs computes one 256 x 256 tile of G_i = X_i^T dY_i (per
+// sample), or of S = Xs^T dYs over all B*T tokens (clipped sum, one operand pre-scaled).
 //   * Each CTA loads half of A (its 128 rows of d_in) and half of B (its 128 columns of
 //     d_out).  So each SM moves 32 KB per 64-token K-block instead of the 48 KB of a
 //     128 x 256 one-SM tile, for twice the MMA work per pair.  With 32 KB stages the
@@ -12,8 +14,10 @@
 //     arrive on both CTAs' empty and accumulator-full barriers through a CTA mask.  Each
 //     CTA's epilogue reads its own 128 TMEM lanes and then arrives on the leader's
 //     accumulator-empty barrier, remotely in the peer's case.
-// The epilogues are those of the one-SM engine (explicit norm, explicit store), applied to
-// the CTA's 128 rows.  Every wait is bounded, as in the one-SM engine.
+// The epilogues are those of the one-SM engine (explicit norm, explicit store, clipped sum
+// with its noise), applied to the CTA's 128 rows.  The clipped sum streams the long token
+// dimension and asks TMA to pull k-blocks into L2 ahead of their loads, as the one-SM
+// engine does.  Every wait is bounded, as in the one-SM engine.
 #pragma once
 #include "umma_gemm.cuh"
 
@@ -37,6 +41,14 @@ __device__ __forceinline__ void cluster_sync_all() {
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
                : "memory");
+}
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* m, uint32_t bar_cluster,
+                                                 int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(bar_cluster), "r"(c0), "r"(c1)
+      : "memory");
 }
 __device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap* m, uint32_t bar_cluster,
                                                  int c0, int c1, int c2) {
@@ -90,7 +102,7 @@ struct Umma2Config {
   static constexpr int BN = 256;     // columns of the pair's tile (each CTA loads half)
   static constexpr int BK = 64;
   static constexpr int EPI = EPI_;
-  static constexpr bool PER_SAMPLE = true;
+  static constexpr bool PER_SAMPLE = (EPI_ != kEpiClipSum);
   static constexpr bool A_MN = true;
   static constexpr bool B_MN = true;
   static constexpr int A_BYTES = BM * BK * 2;         // 16 KB
@@ -102,17 +114,27 @@ struct Umma2Config {
   static constexpr int THREADS = 192;
   static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
   static constexpr uint32_t IDESC = umma_idesc_bf16(2 * BM, BN, true, true);
-  static_assert(EPI_ == kEpiExplicitNorm || EPI_ == kEpiExplicitStore, "per-sample kernels only");
+  static_assert(EPI_ == kEpiExplicitNorm || EPI_ == kEpiExplicitStore || EPI_ == kEpiClipSum,
+                "per-sample explicit kernels and the clipped sum");
 };
 
-// Units: (sample, 256-row tile, 256-column tile), sample-major; p.m_tiles counts 256-row tiles.
+// Units: (sample or K split, 256-row tile, 256-column tile), sample- or split-major; p.m_tiles
+// counts 256-row tiles.
 template <class Cfg>
 __device__ __forceinline__ Unit decode_unit_pair(const UmmaParams& p, int u) {
   Unit w{};
   const int tiles = p.m_tiles * p.n_tiles;
   const int r = u % tiles;
-  w.sample = u / tiles;
   w.local = r;
+  if (Cfg::PER_SAMPLE) {
+    w.sample = u / tiles;
+    w.kb_begin = 0;
+    w.kb_end = p.k_blocks;
+  } else {
+    w.split = u / tiles;
+    w.kb_begin = w.split * p.k_blocks_per_split;
+    w.kb_end = min(p.k_blocks, w.kb_begin + p.k_blocks_per_split);
+  }
   constexpr int G = 8;
   const int per_group = G * p.n_tiles;
   const int first_m = (r / per_group) * G;
@@ -120,8 +142,6 @@ __device__ __forceinline__ Unit decode_unit_pair(const UmmaParams& p, int u) {
   const int within = r % per_group;
   w.m_blk = first_m + within % gsz;
   w.n_blk = within / gsz;
-  w.kb_begin = 0;
-  w.kb_end = p.k_blocks;
   return w;
 }
 
@@ -192,12 +212,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
           const uint32_t bar_leader = map_to_rank(smem_addr(full + stage), 0);
           if (leader) mbar_arrive_expect_tx(smem_addr(full + stage), 2 * Cfg::STAGE_BYTES);
           const int k0 = kb * Cfg::BK;
+          if constexpr (Cfg::PER_SAMPLE) {
 #pragma unroll
-          for (int h = 0; h < Cfg::BM / 64; ++h)
-            tma_load_3d_pair(sA + h * (Cfg::BK * 128), &p.tmA0, bar_leader, a0 + 64 * h, k0, w.sample);
+            for (int h = 0; h < Cfg::BM / 64; ++h)
+              tma_load_3d_pair(sA + h * (Cfg::BK * 128), &p.tmA0, bar_leader, a0 + 64 * h, k0, w.sample);
 #pragma unroll
-          for (int h = 0; h < Cfg::BN / 128; ++h)
-            tma_load_3d_pair(sB + h * (Cfg::BK * 128), &p.tmB0, bar_leader, b0 + 64 * h, k0, w.sample);
+            for (int h = 0; h < Cfg::BN / 128; ++h)
+              tma_load_3d_pair(sB + h * (Cfg::BK * 128), &p.tmB0, bar_leader, b0 + 64 * h, k0, w.sample);
+          } else {
+#pragma unroll
+            for (int h = 0; h < Cfg::BM / 64; ++h)
+              tma_load_2d_pair(sA + h * (Cfg::BK * 128), &p.tmA0, bar_leader, a0 + 64 * h, k0);
+#pragma unroll
+            for (int h = 0; h < Cfg::BN / 128; ++h)
+              tma_load_2d_pair(sB + h * (Cfg::BK * 128), &p.tmB0, bar_leader, b0 + 64 * h, k0);
+            // Pull this CTA's boxes of later k-blocks into L2: the long token dimension is
+            // first touched here and re-read by the other pairs on the same panels.
+            auto prefetch = [&](int kq) {
+#pragma unroll
+              for (int h = 0; h < Cfg::BM / 64; ++h) tma_prefetch_l2_2d(&p.tmA0, a0 + 64 * h, kq * Cfg::BK);
+#pragma unroll
+              for (int h = 0; h < Cfg::BN / 128; ++h) tma_prefetch_l2_2d(&p.tmB0, b0 + 64 * h, kq * Cfg::BK);
+            };
+            if (kb == w.kb_begin) {
+              for (int d = 1; d <= kL2PrefetchDistance && kb + d < w.kb_end; ++d) prefetch(kb + d);
+            } else if (kb + kL2PrefetchDistance < w.kb_end) {
+              prefetch(kb + kL2PrefetchDistance);
+            }
+          }
           if (++stage == Cfg::STAGES) {
             stage = 0;
             phase ^= 1u;
