@@ -515,8 +515,8 @@ void reduce_kernel_launch(int grid, size_t smem, cudaStream_t stream, const __nv
 
 template <int BU>
 dp_status reduce_tma_launch(cudaStream_t stream, const __nv_bfloat16* gs, long long mn, NormSource src,
-                            float C, float* out, double noise_std, PhiloxKey key, unsigned layer_id,
-                            StepRef step, uint32_t* status) {
+                            const PartialsRef& pr, float C, float* out, double noise_std, PhiloxKey key,
+                            unsigned layer_id, StepRef step, uint32_t* status) {
   using Cfg = ReduceTmaConfig<BU>;
   static bool configured[64] = {false};
   int dev = 0;
@@ -528,32 +528,44 @@ dp_status reduce_tma_launch(cudaStream_t stream, const __nv_bfloat16* gs, long l
   }
   const long long chunks = (mn + kReduceChunk - 1) / kReduceChunk;
   const int grid = static_cast<int>(chunks < sm_count() ? chunks : sm_count());
-  clip_reduce_tma_kernel<BU><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(gs, mn, src, C, out, noise_std,
-                                                                               key, layer_id, step, status);
+  clip_reduce_tma_kernel<BU><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(gs, mn, src, pr, C, out,
+                                                                               noise_std, key, layer_id, step,
+                                                                               status);
   return DP_OK;
 }
 
 dp_status launch_reduce(const __nv_bfloat16* gs, int B, long long mn, NormSource src, float C,
                         float* out, double noise_std, unsigned long long seed, StepRef step,
-                        unsigned layer_id, cudaStream_t stream, uint32_t* status) {
+                        unsigned layer_id, cudaStream_t stream, uint32_t* status,
+                        const PartialsRef* partials = nullptr) {
+  // With `partials`, the clip factors come from the per-warp norm partials: the bulk-copy
+  // reduce sums them in its prologue (and block 0 writes norm2 / norms_out / c_out); the
+  // other reduce needs them summed first.
   if (B <= 8) {
     // Warp-specialised bulk-copy reduce: noise generation overlaps the HBM stream.
     const PhiloxKey key = philox_key_from_seed(seed);
+    const PartialsRef pr = partials ? *partials : PartialsRef{nullptr, 0, 0, nullptr, nullptr, nullptr};
     LaunchScope scope(kKindReduce, stream);
     dp_status st;
     switch (B) {
-      case 1: st = reduce_tma_launch<1>(stream, gs, mn, src, C, out, noise_std, key, layer_id, step, status); break;
-      case 2: st = reduce_tma_launch<2>(stream, gs, mn, src, C, out, noise_std, key, layer_id, step, status); break;
-      case 3: st = reduce_tma_launch<3>(stream, gs, mn, src, C, out, noise_std, key, layer_id, step, status); break;
-      case 4: st = reduce_tma_launch<4>(stream, gs, mn, src, C, out, noise_std, key, layer_id, step, status); break;
-      case 5: st = reduce_tma_launch<5>(stream, gs, mn, src, C, out, noise_std, key, layer_id, step, status); break;
-      case 6: st = reduce_tma_launch<6>(stream, gs, mn, src, C, out, noise_std, key, layer_id, step, status); break;
-      case 7: st = reduce_tma_launch<7>(stream, gs, mn, src, C, out, noise_std, key, layer_id, step, status); break;
-      default: st = reduce_tma_launch<8>(stream, gs, mn, src, C, out, noise_std, key, layer_id, step, status); break;
+      case 1: st = reduce_tma_launch<1>(stream, gs, mn, src, pr, C, out, noise_std, key, layer_id, step, status); break;
+      case 2: st = reduce_tma_launch<2>(stream, gs, mn, src, pr, C, out, noise_std, key, layer_id, step, status); break;
+      case 3: st = reduce_tma_launch<3>(stream, gs, mn, src, pr, C, out, noise_std, key, layer_id, step, status); break;
+      case 4: st = reduce_tma_launch<4>(stream, gs, mn, src, pr, C, out, noise_std, key, layer_id, step, status); break;
+      case 5: st = reduce_tma_launch<5>(stream, gs, mn, src, pr, C, out, noise_std, key, layer_id, step, status); break;
+      case 6: st = reduce_tma_launch<6>(stream, gs, mn, src, pr, C, out, noise_std, key, layer_id, step, status); break;
+      case 7: st = reduce_tma_launch<7>(stream, gs, mn, src, pr, C, out, noise_std, key, layer_id, step, status); break;
+      default: st = reduce_tma_launch<8>(stream, gs, mn, src, pr, C, out, noise_std, key, layer_id, step, status); break;
     }
     if (st != DP_OK) return st;
     DP_CHECK_LAUNCH("clip_reduce_tma_kernel");
     return DP_OK;
+  }
+  if (partials) {
+    dp_status st = launch_norm_partials(partials->partials, partials->stride, partials->count, B, C,
+                                        partials->norm2, partials->norms_out, partials->c_out, stream);
+    if (st != DP_OK) return st;
+    src = NormSource{partials->norm2, nullptr, nullptr};
   }
   const int cached = B < kReduceCachedSamples ? B : kReduceCachedSamples;
   const int grid = std::min(stream_grid(static_cast<unsigned long long>(mn / 8), 256), sm_count() * 2);
@@ -883,6 +895,25 @@ dp_status block_step(const dp_layer* layers, int L, dp_dtype dt, int B, int T, d
   if (mode == DP_CLIP_PER_LAYER) {
     // Each group: its norms, then each member's clipped sum with its own bound and noise.
     for (const auto& g : Lb.groups) {
+      if (dt == DP_BF16 && Lb.methods[g[0]] == DP_NORM_ONCE) {
+        // Gradients once: tiles and norm partials, then the reduce that sums the partials.
+        const dp_layer& y = layers[g[0]];
+        const Shape s = layer_shape(y, B, T, dt);
+        float* partials = reinterpret_cast<float*>(ws + Lb.partials);
+        __nv_bfloat16* tiles = reinterpret_cast<__nv_bfloat16*>(ws + Lb.tiles[g[0]]);
+        int count = 0;
+        if ((st = bf16_norms(s, y.X, y.dY, DP_NORM_EXPLICIT, partials, Lb.partial_stride, &count,
+                             reinterpret_cast<uint32_t*>(ws), stream, tiles)) != DP_OK)
+          return st;
+        float* n2 = reinterpret_cast<float*>(ws + Lb.norm2) + static_cast<size_t>(g[0]) * B;
+        const PartialsRef pr{partials, Lb.partial_stride, count, n2, y.norms_out, nullptr};
+        const double noise_std = (sigma == 0.0f) ? 0.0 : static_cast<double>(sigma) * static_cast<double>(y.C);
+        if ((st = launch_reduce(tiles, B, static_cast<long long>(s.m) * s.n, layer_norm_source(Lb, ws, g[0], B, dt),
+                                y.C, y.G_out, noise_std, seed, step, y.layer_id, stream,
+                                reinterpret_cast<uint32_t*>(ws), &pr)) != DP_OK)
+          return st;
+        continue;
+      }
       if ((st = block_group_norms(layers, g, dt, B, T, Lb, ws, stream)) != DP_OK) return st;
       for (int l : g) {
         const NormSource src = layer_norm_source(Lb, ws, l, B, dt);
@@ -1053,15 +1084,23 @@ dp_status linear_step(const void* X, const void* dY, const void* P, int r, dp_dt
   // sigma = 0 means no noise, also for C = +inf (where sigma * C would be NaN).
   const double noise_std = (sigma == 0.0f) ? 0.0 : static_cast<double>(sigma) * static_cast<double>(C);
   const long long mn = static_cast<long long>(c.s.m) * c.s.ne();
-  if ((st = norms_into_ws(c, X, Z, once ? DP_NORM_EXPLICIT : m, C, dt == DP_BF16 ? norms_out : nullptr,
-                          once)) != DP_OK)
-    return st;
+  if (once) {
+    // Each G_i tile is formed once: squared on chip into per-warp partials and stored in bf16.
+    // The reduce sums the partials itself, then streams the tiles: sum_i c_i G_i + noise.
+    __nv_bfloat16* tiles = reinterpret_cast<__nv_bfloat16*>(c.ws + c.L.gs);
+    int count = 0;
+    if ((st = bf16_norms(c.s, X, Z, DP_NORM_EXPLICIT, c.partials(), c.L.partial_stride, &count, c.status(),
+                         c.stream, tiles)) != DP_OK)
+      return st;
+    const PartialsRef pr{c.partials(), c.L.partial_stride, count, c.norm2_f32(), norms_out,
+                         norms_out ? c.c() : nullptr};
+    return launch_reduce(tiles, B, mn, ws_norm_source(c), C, G_out, noise_std, seed, step, layer_id, c.stream,
+                         c.status(), &pr);
+  }
+  if ((st = norms_into_ws(c, X, Z, m, C, dt == DP_BF16 ? norms_out : nullptr)) != DP_OK) return st;
   const NormSource src = ws_norm_source(c);
   if (dt == DP_F32 && norms_out && (st = launch_finalize(src, B, C, norms_out, c.c(), c.stream)) != DP_OK)
     return st;
-  if (once)
-    return launch_reduce(reinterpret_cast<const __nv_bfloat16*>(c.ws + c.L.gs), B, mn, src, C, G_out,
-                         noise_std, seed, step, layer_id, c.stream, c.status());
   return clipped_sum(c, X, Z, src, C, G_out, 0, noise_std, seed, step, layer_id);
 }
 

@@ -117,21 +117,39 @@ struct NormSource {
   }
 };
 
-// norm2[i] = the sum of sample i's `count` per-warp partials, in a fixed order and in fp64,
-// so the norms (and the clip factors that follow from them) are reproducible bit for bit.
-// One warp per sample.  Also writes norms_out[i] = n_i and c_out[i] = c_i when given.
+// Sample i's squared norm from its `count` per-warp partials, summed by one warp in a fixed
+// order in fp64 (lane-strided, then a butterfly), so the norms and the clip factors that follow
+// from them are reproducible bit for bit.  Every lane returns the same value.
+__device__ __forceinline__ float warp_norm2_from_partials(const float* __restrict__ partials, int stride,
+                                                          int count, int i, int lane) {
+  double acc = 0.0;
+  for (int k = lane; k < count; k += 32) acc += static_cast<double>(partials[static_cast<long long>(i) * stride + k]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
+  return static_cast<float>(acc);
+}
+
+// Partials that the bulk-copy reduce sums itself in its prologue (partials == null: the clip
+// factors come from its NormSource instead).  Block 0 also writes norm2, norms_out and c_out
+// when they are given.
+struct PartialsRef {
+  const float* partials;
+  int stride, count;
+  float* norm2;
+  float* norms_out;
+  float* c_out;
+};
+
+// norm2[i] = warp_norm2_from_partials(sample i), one warp per sample.  Also writes
+// norms_out[i] = n_i and c_out[i] = c_i when given.
 __global__ void reduce_norm_partials_kernel(const float* __restrict__ partials, int stride, int count,
                                             int B, float C, float* __restrict__ norm2,
                                             float* __restrict__ norms_out, float* __restrict__ c_out) {
   const int i = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
   if (i >= B) return;
-  double acc = 0.0;
-  for (int k = lane; k < count; k += 32) acc += static_cast<double>(partials[static_cast<long long>(i) * stride + k]);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
+  const float n2 = warp_norm2_from_partials(partials, stride, count, i, lane);
   if (lane == 0) {
-    const float n2 = static_cast<float>(acc);
     norm2[i] = n2;
     const float n = sqrtf(n2);
     if (norms_out) norms_out[i] = n;
@@ -250,6 +268,7 @@ __global__ void __launch_bounds__(256, 2) clip_reduce_kernel(
 // the compute warps saturate the fp64 pipe.  Waits are bounded as in the tensor-core engine.
 constexpr int kReduceComputeWarps = 23;  // 24 warps at 80 registers fill the register file
 constexpr int kReduceChunk = 8 * 32 * kReduceComputeWarps;
+static_assert(kReduceComputeWarps >= 8, "one compute warp per sample sums the norm partials");
 
 template <int BU>
 struct ReduceTmaConfig {
@@ -264,8 +283,9 @@ struct ReduceTmaConfig {
 
 template <int BU>
 __global__ void __launch_bounds__(ReduceTmaConfig<BU>::THREADS, 1) clip_reduce_tma_kernel(
-    const __nv_bfloat16* __restrict__ Gs, long long mn, NormSource src, float C, float* __restrict__ out,
-    double noise_std, PhiloxKey key, uint32_t layer_id, StepRef step, uint32_t* status) {
+    const __nv_bfloat16* __restrict__ Gs, long long mn, NormSource src, PartialsRef pr, float C,
+    float* __restrict__ out, double noise_std, PhiloxKey key, uint32_t layer_id, StepRef step,
+    uint32_t* status) {
   const uint32_t step_lo = step.get();
   using Cfg = ReduceTmaConfig<BU>;
   extern __shared__ uint8_t smem_raw[];
@@ -285,7 +305,7 @@ __global__ void __launch_bounds__(ReduceTmaConfig<BU>::THREADS, 1) clip_reduce_t
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (threadIdx.x < BU) c_s[threadIdx.x] = clip_factor(src.norm(threadIdx.x), C);
+  if (pr.partials == nullptr && threadIdx.x < BU) c_s[threadIdx.x] = clip_factor(src.norm(threadIdx.x), C);
   double2* tab_s = reinterpret_cast<double2*>(smem + Cfg::TABLE_OFFSET);
   if (noise_std != 0.0) stage_noise_tables(tab_s);
   __syncthreads();
@@ -314,6 +334,21 @@ __global__ void __launch_bounds__(ReduceTmaConfig<BU>::THREADS, 1) clip_reduce_t
     }
   } else {
     const int t = threadIdx.x - 32;  // 0 .. 32 * kReduceComputeWarps - 1
+    if (pr.partials != nullptr && warp - 1 < BU) {
+      // Warp 1 + i sums sample i's norm partials while the producer starts streaming.
+      const int i = warp - 1;
+      const float n2 = warp_norm2_from_partials(pr.partials, pr.stride, pr.count, i, static_cast<int>(lane));
+      const float n = sqrtf(n2);
+      if (lane == 0) {
+        c_s[i] = clip_factor(n, C);
+        if (blockIdx.x == 0) {
+          if (pr.norm2) pr.norm2[i] = n2;
+          if (pr.norms_out) pr.norms_out[i] = n;
+          if (pr.c_out) pr.c_out[i] = c_s[i];
+        }
+      }
+    }
+    bool need_c = (pr.partials != nullptr);  // c_s is read first after the first chunk's noise
     int stage = 0;
     uint32_t phase = 0;
     for (long long ch = blockIdx.x; ch < chunks; ch += gridDim.x) {
@@ -324,6 +359,12 @@ __global__ void __launch_bounds__(ReduceTmaConfig<BU>::THREADS, 1) clip_reduce_t
                  *reinterpret_cast<double(*)[4]>(z), tab);
         normals4(static_cast<uint32_t>((e >> 2) + 1), layer_id, step_lo, kStreamNoise, key,
                  *reinterpret_cast<double(*)[4]>(z + 4), tab);
+      }
+      if (need_c) {
+        // Every compute warp passes here in its first iteration (the trip count is the same
+        // for all of them), before any wait that could end the loop early.
+        asm volatile("bar.sync 1, %0;" ::"r"(32 * kReduceComputeWarps) : "memory");
+        need_c = false;
       }
       if (!mbar_wait_bounded(smem_addr(full + stage), phase, abort_flag, status, 22u)) break;
       if (e < mn) {
