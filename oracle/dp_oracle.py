@@ -260,8 +260,9 @@ def linear_step(X, dY, C, sigma, seed, step, layer_id, P=None):
 def block_step(layers, C, sigma, seed, step, mode="per_layer"):
     """One privatised step for a block of linear layers that see the same samples.
 
-    ``layers`` is a list of dicts with X [B,T,d_in], dY [B,T,d_out], layer_id and, for
-    per-layer clipping, C (the layer's bound; ``C`` is then ignored).
+    ``layers`` is a list of dicts with X [B,T,d_in], dY [B,T,d_out], layer_id, optionally P
+    [d_out, r] (the layer is then clipped, summed and noised in the projected space, as in
+    ``linear_step``), and, for per-layer clipping, C (the layer's bound; ``C`` is then ignored).
     * mode "per_layer": each layer is clipped with its own bound, as in ``linear_step``
       (FlashDP Abstract: per-layer clipped DP-SGD).
     * mode "flat": one clip factor per sample for the whole block,
@@ -270,18 +271,18 @@ def block_step(layers, C, sigma, seed, step, mode="per_layer"):
     Returns {"layers": [per-layer dicts like linear_step], "flat_norms": [B] or None}.
     """
     if mode == "per_layer":
-        return {"layers": [linear_step(l["X"], l["dY"], l["C"], sigma, seed, step, l["layer_id"])
+        return {"layers": [linear_step(l["X"], l["dY"], l["C"], sigma, seed, step, l["layer_id"], l.get("P"))
                            for l in layers], "flat_norms": None}
     if mode != "flat":
         raise ValueError(mode)
     if sigma != 0 and not np.isfinite(C):
         raise ValueError("noise std sigma*C is infinite when C = inf; use sigma = 0")
-    per_layer_norms = [per_sample_norms(l["X"], l["dY"]) for l in layers]
+    per_layer_norms = [per_sample_norms(l["X"], l["dY"], l.get("P")) for l in layers]
     flat = np.sqrt(np.sum(np.stack(per_layer_norms) ** 2, axis=0))
     c = clip_factors(flat, C)
     out = []
     for l, n_l in zip(layers, per_layer_norms):
-        S = clipped_sum(l["X"], l["dY"], c)
+        S = clipped_sum(l["X"], l["dY"], c, l.get("P"))
         z = (noise(S.shape[0], S.shape[1], float(sigma) * float(C), seed, step, l["layer_id"])
              if sigma != 0 else np.zeros_like(S))
         out.append({"norms": n_l, "c": c, "S": S, "noise": z, "out": S + z})

@@ -334,10 +334,34 @@ def pin_projected_adam(o, seed=10):
     assert np.allclose(W1, W0 - lr * np.sign(R) @ P.T, rtol=1e-12, atol=1e-12)
 
 
+def pin_block_projection(o, seed=21):
+    """Projected layers in the block step.  With P = 2 Pi (Pi a permutation matrix), G P doubles
+    every entry of G and permutes its columns, so each clip-space norm doubles, and with no
+    clipping the sum is twice the plain batch gradient (einsum) with its columns permuted."""
+    rng = np.random.default_rng(seed)
+    B, T = 3, 5
+    X = rng.standard_normal((B, T, 6))
+    layers = [{"X": X, "dY": rng.standard_normal((B, T, 4)), "layer_id": 0, "C": np.inf},
+              {"X": rng.standard_normal((B, T, 5)), "dY": rng.standard_normal((B, T, 7)), "layer_id": 1,
+               "C": np.inf}]
+    perms = [np.array([2, 0, 3, 1]), np.array([4, 6, 0, 2, 5, 1, 3])]   # not involutions
+    for l, pm in zip(layers, perms):
+        n = len(pm)
+        P = np.zeros((n, n))
+        P[pm, np.arange(n)] = 2.0            # column j of G P is 2 * column pm[j] of G
+        l["P"] = P
+    for mode in ("per_layer", "flat"):
+        out = o.block_step(layers, np.inf, 0.0, 0, 0, mode=mode)
+        for l, pm, r in zip(layers, perms, out["layers"]):
+            G = np.einsum("bta,btc->bac", l["X"], l["dY"])
+            assert np.allclose(r["S"], 2.0 * G.sum(axis=0)[:, pm], rtol=1e-12, atol=1e-12), mode
+            assert np.allclose(r["norms"], 2.0 * np.sqrt(np.sum(G * G, axis=(1, 2))), rtol=1e-12), mode
+
+
 ALL_PINS = [
     pin_philox_kat, pin_box_muller_closed_forms, pin_box_muller_mpmath, pin_counter_layout,
     pin_gradient_brute_force, pin_gradient_finite_difference, pin_ghost_identity,
     pin_clip_invariants, pin_sigma_zero_deterministic, pin_noise_is_added_once,
     pin_projection, pin_normal_statistics, pin_bf16_rounding, pin_flat_clipping,
-    pin_projected_adam,
+    pin_projected_adam, pin_block_projection,
 ]

@@ -166,12 +166,29 @@ def _mut_adam_back_projection_transposed(m):
     m.projected_adam = bad
 
 
+def _mut_block_ignores_projection(m):
+    orig = m.block_step
+
+    def bad(layers, C, sigma, seed, step, mode="per_layer"):
+        return orig([{k: v for k, v in l.items() if k != "P"} for l in layers], C, sigma, seed, step, mode)
+    m.block_step = bad
+
+
+def _mut_block_projection_transposed(m):
+    orig = m.block_step
+
+    def bad(layers, C, sigma, seed, step, mode="per_layer"):
+        flipped = [dict(l, P=np.asarray(l["P"]).T) if "P" in l else l for l in layers]
+        return orig(flipped, C, sigma, seed, step, mode)
+    m.block_step = bad
+
+
 MUTANTS = [
     _mut_transposed_gradient, _mut_shifted_token, _mut_no_clip, _mut_clip_by_squared_norm,
     _mut_sin_cos_swap, _mut_key_bump_first, _mut_u1_without_offset, _mut_projection_unscaled,
     _mut_project_after_clip, _mut_noise_scaled_by_sigma_only, _mut_bf16_truncates,
     _mut_flat_without_square, _mut_adam_without_bias_correction,
-    _mut_adam_back_projection_transposed,
+    _mut_adam_back_projection_transposed, _mut_block_ignores_projection, _mut_block_projection_transposed,
 ]
 
 _FAST_PINS = [p for p in pins.ALL_PINS if p is not pins.pin_normal_statistics]
