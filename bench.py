@@ -1,9 +1,9 @@
 """Benchmark of the DP-SGD per-sample clip + sum + noise step on B200.
 
 One step = the whole hot path over one batch: one dp_block_step over the linears of the
-workload (Llama-7B-shaped block by default: 7 linears, B=8, T=2048, bf16), or one
-dp_linear_step per linear for the projected variant.  It computes the per-sample norms, the
-clip factors, the clipped sum and the Gaussian noise of every linear.  The inputs are
+workload (Llama-7B-shaped block by default: 7 linears, B=8, T=2048, bf16; the projected
+variant passes each linear's P).  It computes the per-sample norms, the clip factors, the
+clipped sum and the Gaussian noise of every linear.  The inputs are
 seeded synthetic tensors, resident in HBM.  They are larger than the 126 MB L2, and the 7
 linears cycle through 2.2 GB, so no L2 flush is needed between steps.
 
@@ -309,16 +309,13 @@ def run_ours(args, w, rank, world):
     dev = torch.device("cuda", local)
     _lib.lib()
     shard = args.shard and world > 1
-    if shard and (w.r or args.graph):
-        raise SystemExit("--shard runs unprojected workloads without --graph")
+    if shard and args.graph:
+        raise SystemExit("--shard runs without --graph")
     # Sharded: every rank draws its own samples (the noise seed stays the workload's).
     data = inputs.generate(dataclasses.replace(w, seed=w.seed + 7919 * rank) if shard else w)
     X = {k: v.to(dev) for k, v in data["X"].items()}
     dY = {k: v.to(dev) for k, v in data["dY"].items()}
     r = w.r
-    ws_bytes = max(_lib.workspace_size(w.B, w.T, l.d_in, l.d_out, r,
-                                       _lib.DP_BF16 if w.dtype == "bf16" else _lib.DP_F32, args.method)
-                   for l in w.linears)
     G = {l.name: torch.empty(l.d_in, r or l.d_out, dtype=torch.float32, device=dev) for l in w.linears}
     norms = {l.name: torch.empty(w.B, dtype=torch.float32, device=dev) for l in w.linears}
     # A graph is captured on a side stream; everything then runs on that stream.
@@ -330,20 +327,18 @@ def run_ours(args, w, rank, world):
                                            w.seed, l.layer_id, stream=stream) for l in w.linears} if r else {}
     flat_C = w.C * math.sqrt(len(w.linears))
     block = [{"X": X[l.x_key], "dY": dY[l.name], "layer_id": l.layer_id, "C": w.C, "G_out": G[l.name],
-              "norms_out": norms[l.name]} for l in w.linears]
-    # Unprojected blocks go through the block call (per-layer or flat clipping); the projected
-    # variant runs one dp_linear_step per linear, each with its own P.
-    use_block = (r == 0)
-    if args.clip == "flat" and not use_block:
-        raise SystemExit("flat clipping is defined for unprojected blocks")
-    if use_block:
-        arr = (_lib.DpLayer * len(block))(*[
-            _lib.DpLayer(b["X"].data_ptr(), b["dY"].data_ptr(), b["X"].shape[2], b["dY"].shape[2],
-                         b["layer_id"], b["C"], b["G_out"].data_ptr(), b["norms_out"].data_ptr())
-            for b in block])
-        ws_bytes = _lib.lib().dp_block_workspace_size(arr, len(block), w.B, w.T,
-                                                      _lib.DP_BF16 if w.dtype == "bf16" else _lib.DP_F32,
-                                                      _lib.CLIP_MODES[args.clip], _lib.METHODS[args.method])
+              "norms_out": norms[l.name], **({"P": P[l.name]} if r else {})} for l in w.linears]
+    # One block call per step (per-layer or flat clipping; projected layers carry their P).
+    if shard and r:
+        raise SystemExit("--shard runs unprojected workloads")
+    arr = (_lib.DpLayer * len(block))(*[
+        _lib.DpLayer(b["X"].data_ptr(), b["dY"].data_ptr(), b["X"].shape[2], b["dY"].shape[2],
+                     b["layer_id"], b["C"], b["G_out"].data_ptr(), b["norms_out"].data_ptr(),
+                     b["P"].data_ptr() if "P" in b else None, r)
+        for b in block])
+    ws_bytes = _lib.lib().dp_block_workspace_size(arr, len(block), w.B, w.T,
+                                                  _lib.DP_BF16 if w.dtype == "bf16" else _lib.DP_F32,
+                                                  _lib.CLIP_MODES[args.clip], _lib.METHODS[args.method])
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     flat_norms = torch.empty(w.B, dtype=torch.float32, device=dev)
 
@@ -357,16 +352,10 @@ def run_ours(args, w, rank, world):
         if shard:
             sharded.sharded_step(block, w.sigma, w.seed, k, mode=args.clip, C=flat_C, ops=shard_ops)
             return
-        if use_block:
-            _lib.dp_block_step(block, mode=args.clip, C=flat_C if args.clip == "flat" else w.C, sigma=w.sigma,
-                               seed=w.seed, step=k, method=args.method,
-                               flat_norms_out=flat_norms if args.clip == "flat" else None, workspace=ws,
-                               stream=stream)
-            return
-        for l in w.linears:
-            _lib.dp_linear_step(X[l.x_key], dY[l.name], w.C, w.sigma, w.seed, k, l.layer_id,
-                                P=P.get(l.name), r=r, method=args.method, norms_out=norms[l.name],
-                                G_out=G[l.name], workspace=ws, stream=stream)
+        _lib.dp_block_step(block, mode=args.clip, C=flat_C if args.clip == "flat" else w.C, sigma=w.sigma,
+                           seed=w.seed, step=k, method=args.method,
+                           flat_norms_out=flat_norms if args.clip == "flat" else None, workspace=ws,
+                           stream=stream)
 
     for k in range(args.warmup):
         step(k)

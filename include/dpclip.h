@@ -212,18 +212,24 @@ dp_status dp_per_sample_norms_static(const void* X, const void* dY, dp_dtype dt,
  *                       c_i = min(1, C / sqrt(sum_l n_{i,l}^2)).  The sample's gradient over
  *                       all the block's weights is clipped as one vector, as in textbook
  *                       DP-SGD.  Every layer's output gets noise of std sigma * C.
- * Each layer's noise uses its own layer_id in the Philox counter.  Unprojected only.
+ * Each layer's noise uses its own layer_id in the Philox counter.  A layer with P clips,
+ * sums and noises its projected gradient (the noise then has the [d_in, r] shape); its P is
+ * given, not regenerated (make it once with dp_projection_matrix).
  * Layers whose norm method resolves to DP_NORM_GHOST and that point at the same X with the
- * same d_in and d_out (q/k/v; gate/up) are grouped, up to three, and share one X Gram per
- * pair of 128-token blocks; their norms are bitwise those of one layer at a time. */
+ * same d_in and the same clip-space width (d_out, or r when projected; q/k/v, gate/up) are
+ * grouped, up to three, and share one X Gram per pair of 128-token blocks; their norms are
+ * bitwise those of one layer at a time. */
 typedef struct {
     const void* X;        /* DEVICE [B, T, d_in] in dtype dt */
     const void* dY;       /* DEVICE [B, T, d_out] in dtype dt */
     int d_in, d_out;
     unsigned layer_id;
     float C;              /* the layer's bound (per-layer mode; ignored in flat mode) */
-    float* G_out;         /* DEVICE fp32 [d_in, d_out], overwritten */
+    float* G_out;         /* DEVICE fp32 [d_in, r or d_out], overwritten */
     float* norms_out;     /* NULL or DEVICE fp32 [B]: the layer's own per-sample norms */
+    const void* P;        /* NULL, or DEVICE [d_out, r] in dtype dt: clip and noise the
+                             projected gradient G_i P (DP-GRAPE), as dp_linear_step does */
+    int r;                /* 0 without P; with P, a multiple of 8 (bf16) or 4 (fp32) */
 } dp_layer;
 
 typedef enum { DP_CLIP_PER_LAYER = 0, DP_CLIP_FLAT = 1 } dp_clip_mode;

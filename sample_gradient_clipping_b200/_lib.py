@@ -27,7 +27,8 @@ class DpLayer(ctypes.Structure):
     """Mirror of the C struct dp_layer (include/dpclip.h)."""
     _fields_ = [("X", ctypes.c_void_p), ("dY", ctypes.c_void_p), ("d_in", ctypes.c_int),
                 ("d_out", ctypes.c_int), ("layer_id", ctypes.c_uint), ("C", ctypes.c_float),
-                ("G_out", ctypes.c_void_p), ("norms_out", ctypes.c_void_p)]
+                ("G_out", ctypes.c_void_p), ("norms_out", ctypes.c_void_p), ("P", ctypes.c_void_p),
+                ("r", ctypes.c_int)]
 
 
 DP_CLIP_PER_LAYER, DP_CLIP_FLAT = 0, 1
@@ -291,7 +292,8 @@ def dp_block_step(layers, mode="per_layer", C=1.0, sigma=0.0, seed=0, step=0, me
                   flat_norms_out=None, workspace=None, stream=None):
     """One step for a block of linears sharing the batch.
 
-    ``layers``: dicts with X, dY, layer_id, C (per-layer bound), and optional G_out, norms_out.
+    ``layers``: dicts with X, dY, layer_id, C (per-layer bound), and optional G_out, norms_out and
+    P (a [d_out, r] projection: the layer then clips and noises G_i P).
     ``step``: a number, or a one-element int64 CUDA tensor read when the kernels run.
     Returns (list of G_out, list of norms_out or None, flat_norms_out or None).
     """
@@ -304,12 +306,14 @@ def dp_block_step(layers, mode="per_layer", C=1.0, sigma=0.0, seed=0, step=0, me
     outs, norms = [], []
     for k, l in enumerate(layers):
         _, _, d_in, d_out = _bt_dims(l["X"], l["dY"])
+        P = l.get("P")
+        r = int(P.shape[1]) if P is not None else 0
         G = l.get("G_out")
         if G is None:
-            G = torch.empty(d_in, d_out, dtype=torch.float32, device=l["X"].device)
+            G = torch.empty(d_in, r or d_out, dtype=torch.float32, device=l["X"].device)
         n = l.get("norms_out")
         arr[k] = DpLayer(_ptr(l["X"]), _ptr(l["dY"]), d_in, d_out, int(l["layer_id"]), float(l.get("C", C)),
-                         _ptr(G), _ptr(n))
+                         _ptr(G), _ptr(n), _ptr(P), r)
         outs.append(G)
         norms.append(n)
     need = int(lib().dp_block_workspace_size(arr, len(layers), B, T, dt, CLIP_MODES[mode], METHODS[method]))

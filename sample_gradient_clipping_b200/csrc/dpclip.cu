@@ -716,6 +716,7 @@ dp_status resolve_method(const Shape& s, dp_norm_method method, dp_norm_method* 
 // for the largest serves them all.
 struct BlockLayout {
   size_t flat = 0, norm2 = 0, c = 0, partials = 0, scaled = 0, total = 0;
+  std::vector<size_t> z;                 // per layer: its projected operand Z = dY P, or 0
   int partial_stride = 0;
   long long partial_op_stride = 0;       // floats between the partial sets of a shared group
   std::vector<size_t> tiles;             // per layer; 0 when the layer does not keep tiles
@@ -723,7 +724,9 @@ struct BlockLayout {
   std::vector<std::vector<int>> groups;  // layers in call order, grouped as described above
 };
 
-Shape layer_shape(const dp_layer& l, int B, int T, dp_dtype dt) { return Shape{B, T, l.d_in, l.d_out, 0, dt}; }
+Shape layer_shape(const dp_layer& l, int B, int T, dp_dtype dt) {
+  return Shape{B, T, l.d_in, l.d_out, l.P ? l.r : 0, dt};
+}
 
 dp_status block_methods(const dp_layer* layers, int L, int B, int T, dp_dtype dt, dp_norm_method method,
                         std::vector<dp_norm_method>* out) {
@@ -750,7 +753,8 @@ std::vector<std::vector<int>> block_groups(const dp_layer* layers, int L, dp_dty
     if (dt != DP_BF16 || methods[l] != DP_NORM_GHOST) continue;
     for (int j = l + 1; j < L && static_cast<int>(groups.back().size()) < kGhostSharedMaxOps; ++j) {
       if (!taken[j] && methods[j] == DP_NORM_GHOST && layers[j].X == layers[l].X &&
-          layers[j].d_in == layers[l].d_in && layers[j].d_out == layers[l].d_out) {
+          layers[j].d_in == layers[l].d_in &&
+          (layers[j].P ? layers[j].r : layers[j].d_out) == (layers[l].P ? layers[l].r : layers[l].d_out)) {
         groups.back().push_back(j);
         taken[j] = true;
       }
@@ -777,10 +781,10 @@ BlockLayout block_layout(const dp_layer* layers, int L, int B, int T, dp_dtype d
     if (dt == DP_BF16) {
       const int ps = partial_slots(s);
       if (ps > Lb.partial_stride) Lb.partial_stride = ps;
-      const size_t sc = static_cast<size_t>(s.N()) * static_cast<size_t>(s.m < s.n ? s.m : s.n) * 2;
+      const size_t sc = static_cast<size_t>(s.N()) * static_cast<size_t>(s.m < s.ne() ? s.m : s.ne()) * 2;
       if (methods[l] != DP_NORM_ONCE && sc > scaled) scaled = sc;
       if (methods[l] == DP_NORM_ONCE)
-        tiles_most = std::max(tiles_most, static_cast<size_t>(B) * layers[l].d_in * layers[l].d_out * 2);
+        tiles_most = std::max(tiles_most, static_cast<size_t>(B) * s.m * s.ne() * 2);
     }
   }
   int sets = 1;
@@ -801,12 +805,42 @@ BlockLayout block_layout(const dp_layer* layers, int L, int B, int T, dp_dtype d
     for (int l = 0; l < L; ++l) {
       if (dt == DP_BF16 && methods[l] == DP_NORM_ONCE) {
         Lb.tiles[l] = off;
-        off += align256(static_cast<size_t>(B) * layers[l].d_in * layers[l].d_out * 2);
+        off += align256(static_cast<size_t>(B) * layers[l].d_in * layer_shape(layers[l], B, T, dt).ne() * 2);
       }
+    }
+  }
+  // Each projected layer keeps its Z = dY P from its norms to its clipped sum.
+  Lb.z.assign(L, 0);
+  for (int l = 0; l < L; ++l) {
+    if (layers[l].P) {
+      Lb.z[l] = off;
+      off += align256(static_cast<size_t>(B) * T * layers[l].r * (dt == DP_BF16 ? 2 : 4));
     }
   }
   Lb.total = off;
   return Lb;
+}
+
+// Layer l's clip-space operand: dY, or Z = dY P formed into the workspace when `form` is set
+// (the norms pass forms it; the clipped sum reuses it).
+dp_status block_operand(const dp_layer* layers, int l, dp_dtype dt, int B, int T, const BlockLayout& Lb,
+                        uint8_t* ws, cudaStream_t stream, bool form, const void** Z) {
+  const dp_layer& y = layers[l];
+  if (!y.P) {
+    *Z = y.dY;
+    return DP_OK;
+  }
+  void* z = ws + Lb.z[l];
+  *Z = z;
+  if (!form) return DP_OK;
+  const Shape s = layer_shape(y, B, T, dt);
+  if (dt == DP_BF16) return bf16_project(s, y.dY, y.P, z, reinterpret_cast<uint32_t*>(ws), stream);
+  const long long total = s.N() * s.r;
+  LaunchScope scope(kKindF32Project, stream);
+  f32_project_kernel<<<stream_grid(total, 256), 256, 0, stream>>>(
+      static_cast<const float*>(y.dY), static_cast<const float*>(y.P), static_cast<float*>(z), s.N(), s.n, s.r);
+  DP_CHECK_LAUNCH("f32_project_kernel");
+  return DP_OK;
 }
 
 // Squared norms of the layers of one group into their [B] rows of the norm2 block, and each
@@ -817,13 +851,16 @@ dp_status block_group_norms(const dp_layer* layers, const std::vector<int>& g, d
   uint32_t* status = reinterpret_cast<uint32_t*>(ws);
   const dp_layer& y0 = layers[g[0]];
   const Shape s = layer_shape(y0, B, T, dt);
+  const void* Zs[kGhostSharedMaxOps] = {};
+  for (size_t j = 0; j < g.size(); ++j)
+    if ((st = block_operand(layers, g[j], dt, B, T, Lb, ws, stream, true, &Zs[j])) != DP_OK) return st;
   if (dt == DP_F32) {
     double* n2 = reinterpret_cast<double*>(ws + Lb.norm2) + static_cast<size_t>(g[0]) * B;
-    dim3 grid(ceil_div(s.n, kF32Tile), ceil_div(s.m, kF32Tile), B);
+    dim3 grid(ceil_div(s.ne(), kF32Tile), ceil_div(s.m, kF32Tile), B);
     {
       LaunchScope scope(kKindF32Norm, stream);
-      f32_norm_kernel<<<grid, 256, 0, stream>>>(static_cast<const float*>(y0.X), static_cast<const float*>(y0.dY),
-                                                 T, s.m, s.n, n2);
+      f32_norm_kernel<<<grid, 256, 0, stream>>>(static_cast<const float*>(y0.X), static_cast<const float*>(Zs[0]),
+                                                 T, s.m, s.ne(), n2);
       DP_CHECK_LAUNCH("f32_norm_kernel");
     }
     if (y0.norms_out) {
@@ -835,14 +872,12 @@ dp_status block_group_norms(const dp_layer* layers, const std::vector<int>& g, d
   float* partials = reinterpret_cast<float*>(ws + Lb.partials);
   int count = 0;
   if (g.size() > 1) {
-    const void* Zs[kGhostSharedMaxOps] = {};
-    for (size_t j = 0; j < g.size(); ++j) Zs[j] = layers[g[j]].dY;
     if ((st = bf16_norms_ghost_shared(s, y0.X, Zs, static_cast<int>(g.size()), partials, Lb.partial_stride,
                                       Lb.partial_op_stride, &count, status, stream)) != DP_OK)
       return st;
   } else {
     const bool once = (Lb.methods[g[0]] == DP_NORM_ONCE);
-    if ((st = bf16_norms(s, y0.X, y0.dY, once ? DP_NORM_EXPLICIT : Lb.methods[g[0]], partials,
+    if ((st = bf16_norms(s, y0.X, Zs[0], once ? DP_NORM_EXPLICIT : Lb.methods[g[0]], partials,
                          Lb.partial_stride, &count, status, stream,
                          once ? reinterpret_cast<__nv_bfloat16*>(ws + Lb.tiles[g[0]]) : nullptr)) != DP_OK)
       return st;
@@ -866,7 +901,7 @@ dp_status block_layer_sum(const dp_layer* layers, int l, dp_dtype dt, int B, int
   const double noise_std = (sigma == 0.0f) ? 0.0 : static_cast<double>(sigma) * static_cast<double>(C);
   if (dt == DP_BF16 && Lb.methods[l] == DP_NORM_ONCE)
     return launch_reduce(reinterpret_cast<const __nv_bfloat16*>(ws + Lb.tiles[l]), B,
-                         static_cast<long long>(s.m) * s.n, src, C, y.G_out, noise_std, seed, step, y.layer_id,
+                         static_cast<long long>(s.m) * s.ne(), src, C, y.G_out, noise_std, seed, step, y.layer_id,
                          stream, reinterpret_cast<uint32_t*>(ws));
   Call c;
   c.s = s;
@@ -874,7 +909,10 @@ dp_status block_layer_sum(const dp_layer* layers, int l, dp_dtype dt, int B, int
   c.L.scaled = Lb.scaled;
   c.ws = ws;
   c.stream = stream;
-  return clipped_sum(c, y.X, y.dY, src, C, y.G_out, 0, noise_std, seed, step, y.layer_id);
+  const void* Z;
+  dp_status st = block_operand(layers, l, dt, B, T, Lb, ws, stream, false, &Z);  // formed by the norms
+  if (st != DP_OK) return st;
+  return clipped_sum(c, y.X, Z, src, C, y.G_out, 0, noise_std, seed, step, y.layer_id);
 }
 
 NormSource layer_norm_source(const BlockLayout& Lb, uint8_t* ws, int l, int B, dp_dtype dt) {
@@ -901,14 +939,16 @@ dp_status block_step(const dp_layer* layers, int L, dp_dtype dt, int B, int T, d
         const Shape s = layer_shape(y, B, T, dt);
         float* partials = reinterpret_cast<float*>(ws + Lb.partials);
         __nv_bfloat16* tiles = reinterpret_cast<__nv_bfloat16*>(ws + Lb.tiles[g[0]]);
+        const void* Z;
+        if ((st = block_operand(layers, g[0], dt, B, T, Lb, ws, stream, true, &Z)) != DP_OK) return st;
         int count = 0;
-        if ((st = bf16_norms(s, y.X, y.dY, DP_NORM_EXPLICIT, partials, Lb.partial_stride, &count,
+        if ((st = bf16_norms(s, y.X, Z, DP_NORM_EXPLICIT, partials, Lb.partial_stride, &count,
                              reinterpret_cast<uint32_t*>(ws), stream, tiles)) != DP_OK)
           return st;
         float* n2 = reinterpret_cast<float*>(ws + Lb.norm2) + static_cast<size_t>(g[0]) * B;
         const PartialsRef pr{partials, Lb.partial_stride, count, n2, y.norms_out, nullptr};
         const double noise_std = (sigma == 0.0f) ? 0.0 : static_cast<double>(sigma) * static_cast<double>(y.C);
-        if ((st = launch_reduce(tiles, B, static_cast<long long>(s.m) * s.n, layer_norm_source(Lb, ws, g[0], B, dt),
+        if ((st = launch_reduce(tiles, B, static_cast<long long>(s.m) * s.ne(), layer_norm_source(Lb, ws, g[0], B, dt),
                                 y.C, y.G_out, noise_std, seed, step, y.layer_id, stream,
                                 reinterpret_cast<uint32_t*>(ws), &pr)) != DP_OK)
           return st;
@@ -1204,6 +1244,8 @@ dp_status block_step_entry(const dp_layer* layers, int L, dp_dtype dt, int B, in
     const dp_layer& y = layers[l];
     if (!y.X || !y.dY || !y.G_out || !aligned16(y.X) || !aligned16(y.dY) || !aligned16(y.G_out))
       return DP_ERR_INVALID_ARG;
+    // A projection is given with its width; r without P is refused (P is not regenerated).
+    if ((y.P && (y.r < 1 || !aligned16(y.P))) || (!y.P && y.r != 0)) return DP_ERR_INVALID_ARG;
     if (mode == DP_CLIP_PER_LAYER && (!(y.C > 0.0f) || (std::isinf(y.C) && sigma != 0.0f)))
       return DP_ERR_INVALID_ARG;
   }

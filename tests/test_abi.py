@@ -179,6 +179,17 @@ def test_block_workspace_size_and_host_rejections(L):
     assert call(ws_bytes=4096) == _lib.DP_ERR_WORKSPACE
     bad = (DpLayer * 1)(DpLayer(ODD, FAKE, 64, 64, 0, 1.0, FAKE, None))
     assert L.dp_block_step(bad, 1, _lib.DP_BF16, 2, 4, 1, 1.0, 0.0, 0, 0, 0, None, FAKE, 1 << 30, None) == E
+    # A projection width without P, a misaligned P, or a width not a multiple of 8 is refused.
+    for P, r in ((None, 64), (ODD, 64), (FAKE, 12)):
+        proj = (DpLayer * 1)(DpLayer(FAKE, FAKE, 64, 64, 0, 1.0, FAKE, None, P, r))
+        assert L.dp_block_step(proj, 1, _lib.DP_BF16, 2, 4, 0, 1.0, 0.0, 0, 0, 0, None, FAKE, 1 << 30, None) == E
+    # With P the workspace also holds Z = dY P (2 x 64 tokens x r bf16), and the scaled copy
+    # of the narrower operand is r wide instead of d_out.
+    sizes = {}
+    for r in (16, 32):
+        proj = (DpLayer * 1)(DpLayer(FAKE, FAKE, 64, 64, 0, 1.0, FAKE, None, FAKE, r))
+        sizes[r] = L.dp_block_workspace_size(proj, 1, 2, 64, _lib.DP_BF16, 0, _lib.DP_NORM_GHOST)
+    assert sizes[32] - sizes[16] == 2 * 128 * 16 * 2
 
 
 def test_projected_adam_rejects_on_host(L):

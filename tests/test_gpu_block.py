@@ -135,3 +135,64 @@ def test_shared_x_gram_ghost_block(mode):
         r = ref["layers"][k]
         assert rel_max(host(norms[k]), r["norms"]) <= tol["norm"], lin.name
         assert rel_fro(host(outs[k]), r["S"]) <= tol["sum"], lin.name
+
+
+def _projected_block(r=64, B=4, T=128, seed=17):
+    w = inputs.Workload("pblk", B=B, T=T, dtype="bf16", linears=inputs._block(0, 256, 512),
+                        C=1.0, sigma=0.7, seed=seed, dy_var="per_layer")
+    data = inputs.generate(w)
+    X = {k: v.cuda() for k, v in data["X"].items()}
+    dY = {k: v.cuda() for k, v in data["dY"].items()}
+    P = {l.name: _lib.dp_projection_matrix(torch.empty(l.d_out, r, dtype=torch.bfloat16, device="cuda"),
+                                           w.seed, l.layer_id) for l in w.linears}
+    return w, data, X, dY, P
+
+
+@pytest.mark.parametrize("mode", ["per_layer", "flat"])
+def test_projected_block_against_oracle(mode):
+    """DP-GRAPE layers in one block call: each clips, sums and noises G_i P; q/k/v and gate/up
+    share their X Grams (equal widths r)."""
+    w, data, X, dY, P = _projected_block()
+    C = 0.8
+    layers = [{"X": X[l.x_key], "dY": dY[l.name], "P": P[l.name], "layer_id": l.layer_id, "C": C,
+               "norms_out": torch.empty(w.B, dtype=torch.float32, device="cuda")} for l in w.linears]
+    _lib.profiling_enable(True)
+    _lib.profiling_collect()
+    outs, norms, flat = _lib.dp_block_step(layers, mode=mode, C=C, sigma=0.0, seed=w.seed, step=2, method="ghost")
+    torch.cuda.synchronize()
+    kinds = _lib.profiling_collect()
+    _lib.profiling_enable(False)
+    assert kinds["umma_ghost_shared"][1] == 2, kinds
+    olayers = [{"X": inputs.as_f64(data["X"][l.x_key]), "dY": inputs.as_f64(data["dY"][l.name]),
+                "P": host(P[l.name]), "layer_id": l.layer_id, "C": C} for l in w.linears]
+    ref = oracle.block_step(olayers, C, 0.0, w.seed, 2, mode=mode)
+    tol = TOL["bf16"]
+    if mode == "flat":
+        assert rel_max(host(flat), ref["flat_norms"]) <= tol["norm"]
+    for k, lin in enumerate(w.linears):
+        r = ref["layers"][k]
+        assert outs[k].shape == (lin.d_in, 64)
+        assert rel_max(host(norms[k]), r["norms"]) <= tol["norm"], lin.name
+        assert rel_fro(host(outs[k]), r["S"]) <= tol["sum"], lin.name
+    # The noise of a projected layer has the [d_in, r] shape and is added once.
+    outs1, _, _ = _lib.dp_block_step(layers, mode=mode, C=C, sigma=w.sigma, seed=w.seed, step=2, method="ghost")
+    torch.cuda.synchronize()
+    for k, lin in enumerate(w.linears):
+        a, b = host(outs1[k]), host(outs[k])
+        want = oracle.noise(a.shape[0], a.shape[1], float(np.float32(w.sigma)) * float(np.float32(C)), w.seed, 2,
+                            lin.layer_id)
+        assert np.all(np.abs((a - b) - want) <= noise_tolerance(a, b) + 1e-6 * np.abs(b)), lin.name
+
+
+@pytest.mark.parametrize("method", ["ghost", "once", "explicit"])
+def test_projected_block_equals_projected_linear_steps(method):
+    w, data, X, dY, P = _projected_block(seed=19)
+    layers = [{"X": X[l.x_key], "dY": dY[l.name], "P": P[l.name], "layer_id": l.layer_id, "C": 0.5,
+               "norms_out": torch.empty(w.B, dtype=torch.float32, device="cuda")} for l in w.linears]
+    outs, norms, _ = _lib.dp_block_step(layers, mode="per_layer", sigma=w.sigma, seed=w.seed, step=4,
+                                        method=method)
+    for k, lin in enumerate(w.linears):
+        G, n = _lib.dp_linear_step(X[lin.x_key], dY[lin.name], 0.5, w.sigma, w.seed, 4, lin.layer_id,
+                                   P=P[lin.name], method=method)
+        assert torch.equal(n, norms[k]), lin.name
+        assert rel_fro(host(outs[k]), host(G)) <= 1e-6, lin.name
