@@ -15,9 +15,11 @@
 //     CTA's epilogue reads its own 128 TMEM lanes and then arrives on the leader's
 //     accumulator-empty barrier, remotely in the peer's case.
 // The epilogues are those of the one-SM engine (explicit norm, explicit store, clipped sum
-// with its noise), applied to the CTA's 128 rows.  The clipped sum streams the long token
-// dimension and asks TMA to pull k-blocks into L2 ahead of their loads, as the one-SM
-// engine does.  Every wait is bounded, as in the one-SM engine.
+// with its noise), applied to the CTA's 128 rows.  (An L2 prefetch of later k-blocks along
+// the clipped sum's long token dimension was measured and dropped: 8, 16 or 32 blocks ahead
+// it made that kernel 5% slower than no prefetch.  256 x 128 pair tiles, which fill the last
+// wave of a 4096 x 4096 output better, were 10% slower there and 40% slower on GPT-2's
+// 768 x 3072.)  Every wait is bounded, as in the one-SM engine.
 #pragma once
 #include "umma_gemm.cuh"
 
@@ -226,19 +228,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
 #pragma unroll
             for (int h = 0; h < Cfg::BN / 128; ++h)
               tma_load_2d_pair(sB + h * (Cfg::BK * 128), &p.tmB0, bar_leader, b0 + 64 * h, k0);
-            // Pull this CTA's boxes of later k-blocks into L2: the long token dimension is
-            // first touched here and re-read by the other pairs on the same panels.
-            auto prefetch = [&](int kq) {
-#pragma unroll
-              for (int h = 0; h < Cfg::BM / 64; ++h) tma_prefetch_l2_2d(&p.tmA0, a0 + 64 * h, kq * Cfg::BK);
-#pragma unroll
-              for (int h = 0; h < Cfg::BN / 128; ++h) tma_prefetch_l2_2d(&p.tmB0, b0 + 64 * h, kq * Cfg::BK);
-            };
-            if (kb == w.kb_begin) {
-              for (int d = 1; d <= kL2PrefetchDistance && kb + d < w.kb_end; ++d) prefetch(kb + d);
-            } else if (kb + kL2PrefetchDistance < w.kb_end) {
-              prefetch(kb + kL2PrefetchDistance);
-            }
           }
           if (++stage == Cfg::STAGES) {
             stage = 0;
