@@ -39,8 +39,8 @@ KERNEL_SOURCES = ("sample_gradient_clipping_b200/csrc/ptx.cuh",
                   "sample_gradient_clipping_b200/csrc/umma_gemm_2sm.cuh")
 # (workload, kernel) -> (bytes per launch, source hash)
 MEASURED_TRAFFIC = {
-    ("llama7b_block", "umma_explicit_store"): (877514715, "89a6f5392dd9fa40"),
-    ("llama13b_block", "umma_explicit_store"): (677310976, "89a6f5392dd9fa40"),
+    ("llama7b_block", "umma_explicit_store"): (872185966, "e18278725ee2db47"),
+    ("llama13b_block", "umma_explicit_store"): (674696229, "e18278725ee2db47"),
 }
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
