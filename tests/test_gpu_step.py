@@ -40,7 +40,9 @@ def _step(w, lin, X, dY, sigma, method="auto", ws=None):
                                method=method, workspace=ws)
 
 
-def check_linear(w, lin, data, dev, method="auto", sample_entries=None, check_noise=True):
+def check_linear(w, lin, data, dev, method="auto", sample_entries=None, check_noise=True, got=None):
+    """Checks one linear's step against the oracle; ``got`` = (G at sigma 0, norms, G at sigma)
+    from a call made elsewhere (the block call), else the linear's own dp_linear_step."""
     tol = TOL[w.dtype]
     Xh = inputs.as_f64(data["X"][lin.x_key])
     dYh = inputs.as_f64(data["dY"][lin.name])
@@ -48,7 +50,10 @@ def check_linear(w, lin, data, dev, method="auto", sample_entries=None, check_no
     P = oracle_projection(w, lin) if w.r else None
     C = _f32(w.C)
 
-    G0, n0 = _step(w, lin, Xd, dYd, 0.0, method)
+    if got is not None:
+        G0, n0, G1 = got
+    else:
+        G0, n0 = _step(w, lin, Xd, dYd, 0.0, method)
     torch.cuda.synchronize()
     norms = oracle.per_sample_norms(Xh, dYh, P)
     assert rel_max(host(n0), norms) <= tol["norm"], (lin.name, host(n0), norms)
@@ -66,7 +71,8 @@ def check_linear(w, lin, data, dev, method="auto", sample_entries=None, check_no
         got = host(G0)[rows, cols]
         assert rel_fro(got, want) <= tol["sum"], (lin.name, rel_fro(got, want))
     if check_noise and w.sigma > 0:
-        G1, n1 = _step(w, lin, Xd, dYd, w.sigma, method)
+        if got is None:
+            G1, n1 = _step(w, lin, Xd, dYd, w.sigma, method)
         torch.cuda.synchronize()
         a, b = host(G1), host(G0)
         std = _f32(w.sigma) * C
@@ -111,11 +117,23 @@ def test_roberta_projected_workload(method):
 @pytest.mark.parametrize("name,method", [("llama7b_block", "auto"), ("llama13b_block", "auto"),
                                          ("llama13b_block", "ghost")])
 def test_llama_block_full_size_sampled(name, method):
-    """Full-size blocks, in the launch configuration the benchmark times (auto method)."""
+    """Full-size blocks in the launch configuration the benchmark times: one per-layer
+    dp_block_step over the block (auto method: gradients once), at sigma 0 and sigma."""
     w = inputs.WORKLOADS[name]
     data, dev = draw(w)
-    for lin in w.linears:
-        norms = check_linear(w, lin, data, dev, method=method, sample_entries=512)
+
+    def block(sigma):
+        layers = [{"X": dev["X"][l.x_key], "dY": dev["dY"][l.name], "layer_id": l.layer_id, "C": w.C,
+                   "norms_out": torch.empty(w.B, dtype=torch.float32, device="cuda")} for l in w.linears]
+        outs, norms, _ = _lib.dp_block_step(layers, mode="per_layer", sigma=sigma, seed=w.seed, step=w.step,
+                                            method=method)
+        return outs, norms
+
+    outs0, norms0 = block(0.0)
+    outs1, _ = block(w.sigma)
+    for k, lin in enumerate(w.linears):
+        norms = check_linear(w, lin, data, dev, method=method, sample_entries=512,
+                             got=(outs0[k], norms0[k], outs1[k]))
         if name == "llama13b_block":
             # s_i ~ LogNormal(0,1) makes samples 0 and 2 clip and 1 and 3 pass unclipped.
             assert list(norms > w.C) == [True, False, True, False], norms
