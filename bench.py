@@ -31,16 +31,16 @@ METRIC = "DP clip+sum+noise tokens/s and TFLOP/s as % of B200 roofline, 1 GPU"
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of a step's dominant
 # kernel, averaged over the step's launches, from one ncu capture of the same command (the
-# ncu summaries in profiles/ give the capture).  Each entry records a hash of the sources that
-# define that kernel; when they change, the figure no longer describes the code and bench.py
-# reports traffic as null.
+# ncu summaries in profiles/ give the capture).  Each entry records a hash of the code that
+# defines that kernel (comments and blank space excluded); when the code changes, the figure
+# no longer describes it and bench.py reports traffic as null.
 KERNEL_SOURCES = ("sample_gradient_clipping_b200/csrc/ptx.cuh",
                   "sample_gradient_clipping_b200/csrc/umma_gemm.cuh",
                   "sample_gradient_clipping_b200/csrc/umma_gemm_2sm.cuh")
 # (workload, kernel) -> (bytes per launch, source hash)
 MEASURED_TRAFFIC = {
-    ("llama7b_block", "umma_explicit_store"): (872185966, "e18278725ee2db47"),
-    ("llama13b_block", "umma_explicit_store"): (674696229, "e18278725ee2db47"),
+    ("llama7b_block", "umma_explicit_store"): (872185966, "ee30b8916c2920d7"),
+    ("llama13b_block", "umma_explicit_store"): (674696229, "ee30b8916c2920d7"),
 }
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -105,12 +105,18 @@ def workload_model(w):
 
 
 def kernel_source_hash():
+    """Hash of the dominant kernel's code: its sources with comments and blank space removed,
+    so that a comment edit does not void a measurement of unchanged code."""
     import hashlib
+    import re
 
     h = hashlib.sha256()
     for rel in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, rel)) as f:
+            text = f.read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        h.update(" ".join(text.split()).encode())
     return h.hexdigest()[:16]
 
 

@@ -1,8 +1,9 @@
 // CUDA-core kernels of the step: Gaussian noise, the projection matrix, the clip-factor
 // row scaling, and the fp32 path.
 //
-// The noise, projection and scaling kernels are HBM-bound streams: 16-byte vector loads and
-// stores, and grids sized in multiples of the SM count.  The fp32 path keeps fp64
+// The scaling kernel is an HBM-bound stream; the noise and projection kernels are bound by
+// their Box-Muller arithmetic.  All use 16-byte vector loads and stores and grids sized in
+// multiples of the SM count.  The fp32 path keeps fp64
 // accumulators.  A product of two fp32 values is exact in fp64, so the fp32 parity bounds
 // (1e-5 on the sum, 1e-6 on the norms) hold at any T.
 #pragma once
@@ -265,7 +266,8 @@ __global__ void __launch_bounds__(256, 2) clip_reduce_kernel(
 //                 their fp64 noise, which needs no data, then waits for the stage, forms
 //                 sum_i c_i G_i from shared memory, adds the noise and stores fp32.
 // The copies are issued by one thread with a few instructions each, so HBM stays busy while
-// the compute warps saturate the fp64 pipe.  Waits are bounded as in the tensor-core engine.
+// the compute warps spend their issue slots on the noise.  Waits are bounded as in the
+// tensor-core engine.
 constexpr int kReduceComputeWarps = 23;  // 24 warps at 80 registers fill the register file
 constexpr int kReduceChunk = 8 * 32 * kReduceComputeWarps;
 static_assert(kReduceComputeWarps >= 8, "one compute warp per sample sums the norm partials");

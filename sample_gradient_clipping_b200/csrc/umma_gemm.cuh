@@ -4,12 +4,13 @@
 //   warp 0      TMA producer: loads 128-byte-swizzled A/B tiles into a STAGES-deep smem ring;
 //   warp 1      MMA issuer: allocates all 512 TMEM columns, one lane issues tcgen05.mma
 //               (M = 128, N = BN, K = 16 per instruction) into a TMEM accumulator;
-//               accumulators are double-buffered so the epilogue of unit u overlaps the
-//               mainloop of unit u + 1;
+//               accumulators are double-buffered (all but kEpiGhostShared, whose four
+//               accumulators fill TMEM) so the epilogue of unit u overlaps the mainloop of
+//               unit u + 1;
 //   warps 2..5  epilogue: each thread owns one accumulator row (TMEM lane) and reads it
 //               back 32 columns at a time with tcgen05.ld.
 //
-// The same engine serves the four contractions of the step:
+// The same engine serves these contractions of the step:
 //   kEpiClipSum      S[a, b] = sum_t Xs[t, a] dYs[t, b] over all B*T tokens (both operands
 //                    MN-major; the clip factor is already folded into one operand), with the
 //                    Philox/Box-Muller noise added in the epilogue before the fp32 store;
