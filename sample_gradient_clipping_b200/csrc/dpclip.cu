@@ -370,9 +370,12 @@ dp_status launch_noise(float* G, unsigned long long total, double std_dev, unsig
 
 // out (+)= A^T Bm over all N rows (A: [N, m], Bm: [N, ne], both bf16, one already scaled by
 // c_i), plus noise when noise_std != 0.  `accumulate` = 0 overwrites out.
+// With `defer` (a block step), noise that cannot ride in the epilogue (split K) is queued
+// there instead of launched.
 dp_status bf16_clipsum(const Shape& s, const void* A, const void* Bm, float* out, int accumulate,
                        double noise_std, unsigned long long seed, StepRef step,
-                       unsigned layer_id, uint32_t* status, cudaStream_t stream) {
+                       unsigned layer_id, uint32_t* status, cudaStream_t stream,
+                       NoiseBatch* defer = nullptr) {
   UmmaParams p = base_params(status);
   const int ne = s.ne();
   const int BN = ne <= 128 ? 128 : 256;
@@ -422,8 +425,23 @@ dp_status bf16_clipsum(const Shape& s, const void* A, const void* Bm, float* out
                   : (BN == 128) ? launch_umma<UmmaConfig<128, kEpiClipSum>>(p, stream)
                                 : launch_umma<UmmaConfig<256, kEpiClipSum>>(p, stream);
   if (st2 != DP_OK || fused_noise || noise_std == 0.0) return st2;
+  if (defer && defer->count < kMaxNoiseSegments) {
+    defer->seg[defer->count++] = NoiseSegment{out, static_cast<unsigned long long>(s.m) * ne, noise_std,
+                                              static_cast<uint32_t>(layer_id)};
+    return DP_OK;
+  }
   return launch_noise(out, static_cast<unsigned long long>(s.m) * ne, noise_std, seed, step, layer_id,
                       stream);
+}
+
+dp_status launch_noise_batch(const NoiseBatch& b, unsigned long long seed, StepRef step, cudaStream_t stream) {
+  if (b.count == 0) return DP_OK;
+  unsigned long long nblk = 0;
+  for (int q = 0; q < b.count; ++q) nblk += (b.seg[q].total + 3) / 4;
+  LaunchScope scope(kKindNoise, stream);
+  noise_add_batch_kernel<<<stream_grid(nblk, 256), 256, 0, stream>>>(b, philox_key_from_seed(seed), step);
+  DP_CHECK_LAUNCH("noise_add_batch_kernel");
+  return DP_OK;
 }
 
 dp_status launch_noise(float* G, unsigned long long total, double std_dev, unsigned long long seed,
@@ -668,7 +686,7 @@ NormSource ws_norm_source(const Call& c) {
 // G_out (+)= sum_i c_i X_i^T Z_i (+ noise) for norms given by `src`.
 dp_status clipped_sum(Call& c, const void* X, const void* Z, NormSource src, float C, float* out,
                       int accumulate, double noise_std, unsigned long long seed,
-                      StepRef step, unsigned layer_id) {
+                      StepRef step, unsigned layer_id, NoiseBatch* defer = nullptr) {
   const Shape& s = c.s;
   if (s.dt == DP_F32) {
     dim3 grid(ceil_div(s.ne(), kF32Tile), ceil_div(s.m, kF32Tile));
@@ -685,10 +703,12 @@ dp_status clipped_sum(Call& c, const void* X, const void* Z, NormSource src, flo
   dp_status st;
   if (s.ne() <= s.m) {
     if ((st = launch_scale(Z, scaled, s.N(), s.ne(), s.T, src, C, c.stream)) != DP_OK) return st;
-    return bf16_clipsum(s, X, scaled, out, accumulate, noise_std, seed, step, layer_id, c.status(), c.stream);
+    return bf16_clipsum(s, X, scaled, out, accumulate, noise_std, seed, step, layer_id, c.status(), c.stream,
+                        defer);
   }
   if ((st = launch_scale(X, scaled, s.N(), s.m, s.T, src, C, c.stream)) != DP_OK) return st;
-  return bf16_clipsum(s, scaled, Z, out, accumulate, noise_std, seed, step, layer_id, c.status(), c.stream);
+  return bf16_clipsum(s, scaled, Z, out, accumulate, noise_std, seed, step, layer_id, c.status(), c.stream,
+                      defer);
 }
 
 dp_status resolve_method(const Shape& s, dp_norm_method method, dp_norm_method* out) {
@@ -895,7 +915,7 @@ dp_status block_group_norms(const dp_layer* layers, const std::vector<int>& g, d
 // Layer l's clipped sum with the clip factors of `src` and bound C, plus noise of std sigma C.
 dp_status block_layer_sum(const dp_layer* layers, int l, dp_dtype dt, int B, int T, NormSource src, float C,
                           float sigma, unsigned long long seed, StepRef step, const BlockLayout& Lb,
-                          uint8_t* ws, cudaStream_t stream) {
+                          uint8_t* ws, cudaStream_t stream, NoiseBatch* defer) {
   const dp_layer& y = layers[l];
   const Shape s = layer_shape(y, B, T, dt);
   const double noise_std = (sigma == 0.0f) ? 0.0 : static_cast<double>(sigma) * static_cast<double>(C);
@@ -912,7 +932,7 @@ dp_status block_layer_sum(const dp_layer* layers, int l, dp_dtype dt, int B, int
   const void* Z;
   dp_status st = block_operand(layers, l, dt, B, T, Lb, ws, stream, false, &Z);  // formed by the norms
   if (st != DP_OK) return st;
-  return clipped_sum(c, y.X, Z, src, C, y.G_out, 0, noise_std, seed, step, y.layer_id);
+  return clipped_sum(c, y.X, Z, src, C, y.G_out, 0, noise_std, seed, step, y.layer_id, defer);
 }
 
 NormSource layer_norm_source(const BlockLayout& Lb, uint8_t* ws, int l, int B, dp_dtype dt) {
@@ -930,6 +950,9 @@ dp_status block_step(const dp_layer* layers, int L, dp_dtype dt, int B, int T, d
   dp_status st;
   // Status word, and the fp32 path's atomic norm accumulators, start at zero.
   DP_CUDA(cudaMemsetAsync(ws, 0, Lb.c, stream));
+  // Noise of split-K clipped sums, added in one launch at the end of the step.
+  NoiseBatch deferred;
+  deferred.count = 0;
   if (mode == DP_CLIP_PER_LAYER) {
     // Each group: its norms, then each member's clipped sum with its own bound and noise.
     for (const auto& g : Lb.groups) {
@@ -957,12 +980,13 @@ dp_status block_step(const dp_layer* layers, int L, dp_dtype dt, int B, int T, d
       if ((st = block_group_norms(layers, g, dt, B, T, Lb, ws, stream)) != DP_OK) return st;
       for (int l : g) {
         const NormSource src = layer_norm_source(Lb, ws, l, B, dt);
-        if ((st = block_layer_sum(layers, l, dt, B, T, src, layers[l].C, sigma, seed, step, Lb, ws, stream)) !=
+        if ((st = block_layer_sum(layers, l, dt, B, T, src, layers[l].C, sigma, seed, step, Lb, ws, stream,
+                                  &deferred)) !=
             DP_OK)
           return st;
       }
     }
-    return DP_OK;
+    return launch_noise_batch(deferred, seed, step, stream);
   }
   // 1. Every layer's per-sample norms (gradients-once layers also keep their tiles).
   for (const auto& g : Lb.groups)
@@ -986,9 +1010,10 @@ dp_status block_step(const dp_layer* layers, int L, dp_dtype dt, int B, int T, d
   }
   // 3. Every layer's clipped sum with the shared clip factors, plus its own noise.
   for (int l = 0; l < L; ++l)
-    if ((st = block_layer_sum(layers, l, dt, B, T, src, C, sigma, seed, step, Lb, ws, stream)) != DP_OK)
+    if ((st = block_layer_sum(layers, l, dt, B, T, src, C, sigma, seed, step, Lb, ws, stream, &deferred)) !=
+        DP_OK)
       return st;
-  return DP_OK;
+  return launch_noise_batch(deferred, seed, step, stream);
 }
 
 // ---------------------------------------------------------------- allocation-free norms

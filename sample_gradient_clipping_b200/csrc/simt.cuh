@@ -53,6 +53,43 @@ __global__ void noise_add_kernel(float* __restrict__ G, unsigned long long total
   }
 }
 
+// The noise of several fp32 outputs in one launch: G_s[k] = fp32(G_s[k] + std_s * z_k) with
+// z from stream 0 under each segment's own layer_id.  A block step defers to this the noise of
+// every linear whose clipped sum was split over K (small outputs), so a block pays one small
+// launch instead of one per linear.  The values are those of noise_add_kernel.
+constexpr int kMaxNoiseSegments = 16;
+struct NoiseSegment {
+  float* G;
+  unsigned long long total;   // elements
+  double std_dev;
+  uint32_t layer_id;
+};
+struct NoiseBatch {
+  NoiseSegment seg[kMaxNoiseSegments];
+  int count;
+};
+
+__global__ void noise_add_batch_kernel(NoiseBatch b, PhiloxKey key, StepRef step) {
+  const uint32_t step_lo = step.get();
+  unsigned long long nblk_total = 0;
+  for (int q = 0; q < b.count; ++q) nblk_total += (b.seg[q].total + 3) / 4;
+  for (unsigned long long j = blockIdx.x * static_cast<unsigned long long>(blockDim.x) + threadIdx.x;
+       j < nblk_total; j += static_cast<unsigned long long>(gridDim.x) * blockDim.x) {
+    unsigned long long jj = j;
+    int q = 0;
+    while ((b.seg[q].total + 3) / 4 <= jj) {  // the segment holding global block j
+      jj -= (b.seg[q].total + 3) / 4;
+      ++q;
+    }
+    const NoiseSegment& sg = b.seg[q];
+    double z[4];
+    normals4(static_cast<uint32_t>(jj), sg.layer_id, step_lo, kStreamNoise, key, z);
+    const unsigned long long k0 = 4 * jj;
+    for (int e = 0; e < 4 && k0 + e < sg.total; ++e)
+      sg.G[k0 + e] = static_cast<float>(static_cast<double>(sg.G[k0 + e]) + sg.std_dev * z[e]);
+  }
+}
+
 // out[4 j + q] = word q of Philox block j (verification of the raw uint32 stream).
 __global__ void philox_blocks_kernel(uint4* __restrict__ out, unsigned long long nblocks,
                                      PhiloxKey key, uint32_t layer_id, uint32_t step_lo,
