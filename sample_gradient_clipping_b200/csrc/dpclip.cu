@@ -498,12 +498,32 @@ dp_status launch_projection(void* P, dp_dtype dt, int d_out, int r, unsigned lon
   return DP_OK;
 }
 
+dp_status launch_norm_partials(const float* partials, int stride, int count, int B, float C,
+                               float* norm2, float* norms_out, float* c_out, cudaStream_t stream);
+
+// With `partials` (B samples), the scaling kernel forms the clip factors itself when B <= 8
+// and B * count is small; otherwise the partials kernel runs first.
 dp_status launch_scale(const void* in, void* out, long long rows, int cols, int T, NormSource src,
-                       float C, cudaStream_t stream) {
+                       float C, cudaStream_t stream, const PartialsRef* partials = nullptr, int B = 0) {
   const unsigned long long vecs = static_cast<unsigned long long>(rows) * (cols / 8);
+  PartialsRef pr{nullptr, 0, 0, nullptr, nullptr, nullptr};
+  size_t smem = 0;
+  if (partials) {
+    // One warp per sample in each 256-thread block: with more samples than warps, the serial
+    // rounds of partial sums cost more in every block than the separate launch (measured).
+    if (B <= 8 && static_cast<long long>(B) * partials->count <= kScaleFusedPartialSlots) {
+      pr = *partials;
+      smem = static_cast<size_t>(B) * sizeof(float);
+    } else {
+      dp_status st = launch_norm_partials(partials->partials, partials->stride, partials->count, B, C,
+                                          partials->norm2, partials->norms_out, partials->c_out, stream);
+      if (st != DP_OK) return st;
+      src = NormSource{partials->norm2, nullptr, nullptr};
+    }
+  }
   LaunchScope scope(kKindScale, stream);
-  scale_rows_bf16_kernel<<<stream_grid(vecs, 256), 256, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(in), static_cast<__nv_bfloat16*>(out), rows, cols, T, src, C);
+  scale_rows_bf16_kernel<<<stream_grid(vecs, 256), 256, smem, stream>>>(
+      static_cast<const __nv_bfloat16*>(in), static_cast<__nv_bfloat16*>(out), rows, cols, T, src, pr, B, C);
   DP_CHECK_LAUNCH("scale_rows_bf16_kernel");
   return DP_OK;
 }
@@ -686,7 +706,8 @@ NormSource ws_norm_source(const Call& c) {
 // G_out (+)= sum_i c_i X_i^T Z_i (+ noise) for norms given by `src`.
 dp_status clipped_sum(Call& c, const void* X, const void* Z, NormSource src, float C, float* out,
                       int accumulate, double noise_std, unsigned long long seed,
-                      StepRef step, unsigned layer_id, NoiseBatch* defer = nullptr) {
+                      StepRef step, unsigned layer_id, NoiseBatch* defer = nullptr,
+                      const PartialsRef* partials = nullptr) {
   const Shape& s = c.s;
   if (s.dt == DP_F32) {
     dim3 grid(ceil_div(s.ne(), kF32Tile), ceil_div(s.m, kF32Tile));
@@ -702,11 +723,11 @@ dp_status clipped_sum(Call& c, const void* X, const void* Z, NormSource src, flo
   void* scaled = c.ws + c.L.scaled;
   dp_status st;
   if (s.ne() <= s.m) {
-    if ((st = launch_scale(Z, scaled, s.N(), s.ne(), s.T, src, C, c.stream)) != DP_OK) return st;
+    if ((st = launch_scale(Z, scaled, s.N(), s.ne(), s.T, src, C, c.stream, partials, s.B)) != DP_OK) return st;
     return bf16_clipsum(s, X, scaled, out, accumulate, noise_std, seed, step, layer_id, c.status(), c.stream,
                         defer);
   }
-  if ((st = launch_scale(X, scaled, s.N(), s.m, s.T, src, C, c.stream)) != DP_OK) return st;
+  if ((st = launch_scale(X, scaled, s.N(), s.m, s.T, src, C, c.stream, partials, s.B)) != DP_OK) return st;
   return bf16_clipsum(s, scaled, Z, out, accumulate, noise_std, seed, step, layer_id, c.status(), c.stream,
                       defer);
 }
@@ -866,7 +887,7 @@ dp_status block_operand(const dp_layer* layers, int l, dp_dtype dt, int B, int T
 // Squared norms of the layers of one group into their [B] rows of the norm2 block, and each
 // layer's norms_out when given (gradients-once layers also keep their tiles).
 dp_status block_group_norms(const dp_layer* layers, const std::vector<int>& g, dp_dtype dt, int B, int T,
-                            const BlockLayout& Lb, uint8_t* ws, cudaStream_t stream) {
+                            const BlockLayout& Lb, uint8_t* ws, cudaStream_t stream, int* count_out = nullptr) {
   dp_status st;
   uint32_t* status = reinterpret_cast<uint32_t*>(ws);
   const dp_layer& y0 = layers[g[0]];
@@ -902,6 +923,10 @@ dp_status block_group_norms(const dp_layer* layers, const std::vector<int>& g, d
                          once ? reinterpret_cast<__nv_bfloat16*>(ws + Lb.tiles[g[0]]) : nullptr)) != DP_OK)
       return st;
   }
+  if (count_out) {  // the caller sums the partials later (in the row-scaling kernel)
+    *count_out = count;
+    return DP_OK;
+  }
   for (size_t j = 0; j < g.size(); ++j) {
     const dp_layer& y = layers[g[j]];
     float* n2 = reinterpret_cast<float*>(ws + Lb.norm2) + static_cast<size_t>(g[j]) * B;
@@ -915,7 +940,8 @@ dp_status block_group_norms(const dp_layer* layers, const std::vector<int>& g, d
 // Layer l's clipped sum with the clip factors of `src` and bound C, plus noise of std sigma C.
 dp_status block_layer_sum(const dp_layer* layers, int l, dp_dtype dt, int B, int T, NormSource src, float C,
                           float sigma, unsigned long long seed, StepRef step, const BlockLayout& Lb,
-                          uint8_t* ws, cudaStream_t stream, NoiseBatch* defer) {
+                          uint8_t* ws, cudaStream_t stream, NoiseBatch* defer,
+                          const PartialsRef* partials = nullptr) {
   const dp_layer& y = layers[l];
   const Shape s = layer_shape(y, B, T, dt);
   const double noise_std = (sigma == 0.0f) ? 0.0 : static_cast<double>(sigma) * static_cast<double>(C);
@@ -932,7 +958,7 @@ dp_status block_layer_sum(const dp_layer* layers, int l, dp_dtype dt, int B, int
   const void* Z;
   dp_status st = block_operand(layers, l, dt, B, T, Lb, ws, stream, false, &Z);  // formed by the norms
   if (st != DP_OK) return st;
-  return clipped_sum(c, y.X, Z, src, C, y.G_out, 0, noise_std, seed, step, y.layer_id, defer);
+  return clipped_sum(c, y.X, Z, src, C, y.G_out, 0, noise_std, seed, step, y.layer_id, defer, partials);
 }
 
 NormSource layer_norm_source(const BlockLayout& Lb, uint8_t* ws, int l, int B, dp_dtype dt) {
@@ -977,12 +1003,19 @@ dp_status block_step(const dp_layer* layers, int L, dp_dtype dt, int B, int T, d
           return st;
         continue;
       }
-      if ((st = block_group_norms(layers, g, dt, B, T, Lb, ws, stream)) != DP_OK) return st;
-      for (int l : g) {
+      // bf16: the row-scaling kernel of each member's clipped sum sums its norm partials.
+      int count = 0;
+      if ((st = block_group_norms(layers, g, dt, B, T, Lb, ws, stream, dt == DP_BF16 ? &count : nullptr)) !=
+          DP_OK)
+        return st;
+      for (size_t j = 0; j < g.size(); ++j) {
+        const int l = g[j];
         const NormSource src = layer_norm_source(Lb, ws, l, B, dt);
+        const PartialsRef pr{reinterpret_cast<float*>(ws + Lb.partials) + j * Lb.partial_op_stride,
+                             Lb.partial_stride, count, reinterpret_cast<float*>(ws + Lb.norm2) + static_cast<size_t>(l) * B,
+                             layers[l].norms_out, nullptr};
         if ((st = block_layer_sum(layers, l, dt, B, T, src, layers[l].C, sigma, seed, step, Lb, ws, stream,
-                                  &deferred)) !=
-            DP_OK)
+                                  &deferred, dt == DP_BF16 ? &pr : nullptr)) != DP_OK)
           return st;
       }
     }
@@ -1162,7 +1195,17 @@ dp_status linear_step(const void* X, const void* dY, const void* P, int r, dp_dt
     return launch_reduce(tiles, B, mn, ws_norm_source(c), C, G_out, noise_std, seed, step, layer_id, c.stream,
                          c.status(), &pr);
   }
-  if ((st = norms_into_ws(c, X, Z, m, C, dt == DP_BF16 ? norms_out : nullptr)) != DP_OK) return st;
+  if (dt == DP_BF16) {
+    // The norm partials are summed by the row-scaling kernel of the clipped sum.
+    int count = 0;
+    if ((st = bf16_norms(c.s, X, Z, m, c.partials(), c.L.partial_stride, &count, c.status(), c.stream)) !=
+        DP_OK)
+      return st;
+    const PartialsRef pr{c.partials(), c.L.partial_stride, count, c.norm2_f32(), norms_out,
+                         norms_out ? c.c() : nullptr};
+    return clipped_sum(c, X, Z, ws_norm_source(c), C, G_out, 0, noise_std, seed, step, layer_id, nullptr, &pr);
+  }
+  if ((st = norms_into_ws(c, X, Z, m, C, nullptr)) != DP_OK) return st;
   const NormSource src = ws_norm_source(c);
   if (dt == DP_F32 && norms_out && (st = launch_finalize(src, B, C, norms_out, c.c(), c.stream)) != DP_OK)
     return st;

@@ -221,15 +221,38 @@ __global__ void finalize_norms_kernel(NormSource src, int B, float C, float* __r
 
 // out[row, :] = bf16(c_{row / T} * in[row, :]) for a [rows, cols] bf16 matrix, 8 elements per
 // thread (cols is a multiple of 8, rows are 16-byte aligned).
+// With pr.partials, every block first turns the per-warp norm partials of all B samples into
+// clip factors in shared memory (one warp per sample, the fixed-order routine above), and
+// block 0 writes norm2 / norms_out / c_out: the separate partials kernel is not needed.
+constexpr long long kScaleFusedPartialSlots = 1 << 16;  // B * count up to which blocks do that
+
 __global__ void scale_rows_bf16_kernel(const __nv_bfloat16* __restrict__ in,
                                        __nv_bfloat16* __restrict__ out, long long rows, int cols,
-                                       int T, NormSource src, float C) {
+                                       int T, NormSource src, PartialsRef pr, int B, float C) {
+  extern __shared__ float scale_c[];  // [B] with pr.partials
+  if (pr.partials != nullptr) {
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32, warps = blockDim.x / 32;
+    for (int i = warp; i < B; i += warps) {
+      const float n2 = warp_norm2_from_partials(pr.partials, pr.stride, pr.count, i, lane);
+      if (lane == 0) {
+        const float n = sqrtf(n2);
+        scale_c[i] = clip_factor(n, C);
+        if (blockIdx.x == 0) {
+          if (pr.norm2) pr.norm2[i] = n2;
+          if (pr.norms_out) pr.norms_out[i] = n;
+          if (pr.c_out) pr.c_out[i] = scale_c[i];
+        }
+      }
+    }
+    __syncthreads();
+  }
   const int vec_per_row = cols / 8;
   const long long total = rows * vec_per_row;
   for (long long v = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; v < total;
        v += static_cast<long long>(gridDim.x) * blockDim.x) {
     const long long row = v / vec_per_row;
-    const float c = clip_factor(src.norm(static_cast<int>(row / T)), C);
+    const int i = static_cast<int>(row / T);
+    const float c = pr.partials != nullptr ? scale_c[i] : clip_factor(src.norm(i), C);
     const uint4 pk = reinterpret_cast<const uint4*>(in)[v];
     const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&pk);
     uint4 res;
