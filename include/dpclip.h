@@ -178,6 +178,16 @@ dp_status dp_philox_blocks(unsigned* out, unsigned long long nblocks, unsigned l
                            unsigned long long step, unsigned layer_id, unsigned stream_id,
                            void* stream);
 
+/* The Gaussian transform behind the gradient noise, exposed so that it can be checked on
+ * chosen words (the noise itself reaches it only through Philox output).  Box and Muller
+ * (1958) in fp64, evaluated exactly as the noise kernels evaluate it, before the scaling by
+ * sigma*C: for q < npairs, with u1 = (words[2q] + 1) 2^-32 and u2 = words[2q+1] 2^-32,
+ *   z[2q] = sqrt(-2 ln u1) cos(2 pi u2),  z[2q+1] = sqrt(-2 ln u1) sin(2 pi u2).
+ * The evaluation is table-driven and agrees with the exact values to about 2e-12.
+ *   words : DEVICE uint32 [npairs, 2]; z : DEVICE fp64 [npairs, 2], overwritten;
+ *   both 16-byte aligned; 1 <= npairs <= 2^40. */
+dp_status dp_box_muller(const unsigned* words, long long npairs, double* z, void* stream);
+
 /* dp_per_sample_norms without a workspace, for callers that cannot allocate device memory.
  * Some callers cannot: code that runs inside another framework's allocator hook or a memory
  * budget it does not own, or a real-time loop that forbids new device allocations after

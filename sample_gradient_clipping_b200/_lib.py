@@ -55,6 +55,7 @@ SIGNATURES = {
     "dp_per_sample_norms_static": (_c_int, [_c_void_p, _c_void_p, _c_int, _c_int, _c_int, _c_int, _c_int,
                                             _c_int, _c_void_p, _c_void_p]),
     "dp_philox_blocks": (_c_int, [_c_void_p, _c_ull, _c_ull, _c_ull, _c_uint, _c_uint, _c_void_p]),
+    "dp_box_muller": (_c_int, [_c_void_p, _c_ll, _c_void_p, _c_void_p]),
     "dp_auto_norm_method": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_int]),
     "dp_status_string": (ctypes.c_char_p, [_c_int]),
     "dp_last_cuda_error": (ctypes.c_char_p, []),
@@ -259,6 +260,18 @@ def dp_philox_blocks(nblocks, seed, step, layer_id, stream_id, out=None, device=
     check(lib().dp_philox_blocks(_ptr(out), int(nblocks), int(seed), int(step), int(layer_id),
                                  int(stream_id), _stream(stream)),
           "dp_philox_blocks")
+    return out
+
+
+def dp_box_muller(words, out=None, stream=None):
+    """The noise's Box-Muller transform of word pairs: words int32/uint32 [n, 2] on the device
+    (the uint32 bits) -> fp64 [n, 2] (z_even, z_odd) before the sigma*C scaling."""
+    import torch
+
+    n = int(words.shape[0])
+    if out is None:
+        out = torch.empty(n, 2, dtype=torch.float64, device=words.device)
+    check(lib().dp_box_muller(_ptr(words), n, _ptr(out), _stream(stream)), "dp_box_muller")
     return out
 
 

@@ -1242,6 +1242,17 @@ dp_status dp_philox_blocks(unsigned* out, unsigned long long nblocks, unsigned l
   return DP_OK;
 }
 
+dp_status dp_box_muller(const unsigned* words, long long npairs, double* z, void* stream) {
+  if (!words || !z || !aligned16(words) || !aligned16(z) || npairs < 1 || npairs > (1ll << 40))
+    return DP_ERR_INVALID_ARG;
+  LaunchScope scope(kKindNoise, static_cast<cudaStream_t>(stream));
+  const unsigned long long n = static_cast<unsigned long long>(npairs);
+  box_muller_words_kernel<<<stream_grid(n, 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      reinterpret_cast<const uint2*>(words), reinterpret_cast<double2*>(z), n);
+  DP_CHECK_LAUNCH("box_muller_words_kernel");
+  return DP_OK;
+}
+
 dp_status dp_per_sample_norms_static(const void* X, const void* dY, dp_dtype dt, int B, int T,
                                      int d_in, int d_out, dp_norm_method method, float* norms,
                                      void* stream) {

@@ -74,9 +74,13 @@ __device__ __forceinline__ uint4 philox4x32_10(uint4 c, PhiloxKey k) {
 // IEEE floating-point arithmetic", ACM TOMS 1990; sine and cosine by the addition formula
 // around tabulated angles).  Every breakpoint value is the double nearest its exact value
 // (gen_noise_tables.py), so each piece is a short polynomial on a small interval.  The noise is
-// issue-bound where it is generated, and this form needs about 40 fp64 operations per pair.
-// Against 50-digit arithmetic on all edge words and 6500 random pairs, |z - z_exact| stays
-// below 5e-13.  The largest errors come at u1 just below 1, where the radius is ~2e-5.
+// issue-bound where it is generated, so the form is cut to about 30 fp64 operations a pair:
+// polynomial degrees only as high as a 1e-12 result needs, the factor -2 of -2 ln u1 and the
+// angle unit 2 pi 2^-32 folded into the tables and coefficients, one Newton step for the square
+// root, and the caller's scale (the noise std) folded into the radius.  Against CUDA's
+// full-precision log, sqrt and sincospi, |z - z_ref| stayed below 2.1e-12 on all edge words
+// (every table breakpoint of both words and its neighbours, u1 = 1, u1 = 2^-32) and on 2^30
+// random pairs; the largest errors come at u1 just below 1, where the radius is ~2e-5.
 
 // Where the transform reads its tables.  Global: the module's arrays through the read-only
 // cache.  Shared: eight copies, entry j of copy c at [8 j + c], each thread reading copy
@@ -123,77 +127,68 @@ __device__ __forceinline__ double u32_minus(uint32_t u, double offset) {
   return __hiloint2double(0x43300000, static_cast<int>(u)) - (kTwo52 + offset);
 }
 
-// Exact double <-> float moves by bit manipulation for normal, positive values in the float
-// range (2^-126 <= a < 2^128); the float is the double truncated to 24 bits.
-__device__ __forceinline__ float f32_trunc_from_pos_f64(double a) {
-  const int hi = __double2hiint(a);
-  const uint32_t lo = static_cast<uint32_t>(__double2loint(a));
-  return __int_as_float(((hi - (896 << 20)) << 3) | static_cast<int>(lo >> 29));
-}
-__device__ __forceinline__ double f64_from_pos_f32(float f) {
-  const int b = __float_as_int(f);
-  return __hiloint2double((b >> 3) + (896 << 20), b << 29);
-}
-
-// -2 ln(u1), u1 = (x + 1) 2^-32.  x + 1 = 2^k m exactly, m in [1, 2), and with (F, L) the
-// table entry of m's top 7 fraction bits, ln m = L + ln(1 + r) where r = m F - 1 comes from
-// one fused multiply-add and |r| <= 2^-8.  ln(1 + r) is its Taylor series to r^6 (the next
-// term is below 2e-18).  ln 2 is split so that (k - 32) ln 2 adds without rounding error.
+// -2 ln(u1), u1 = (x + 1) 2^-32.  x + 1 = 2^k m exactly, m in [1, 2).  With (F, L) the table
+// entry of m's top 7 fraction bits, ln m = L + ln(1 + r), r = m F - 1, |r| <= 2^-8.  The table
+// holds (-2F, -2L), so one fused multiply-add gives r' = -2r exactly as -2 times the rounded r,
+// and -2 ln(1 + r) = r' + r'^2/4 + r'^3/12 + r'^4/32 + r'^5/80 (the next term is below 2e-15).
+// ln 2 is split so that (k - 32)(-2 ln 2) adds without rounding error.
 template <class Tab>
 __device__ __forceinline__ double minus_two_ln_u1(uint32_t x, const Tab& tab) {
   const double d = u32_minus(x, -1.0);             // x + 1, exact
   const int hi = __double2hiint(d);                // biased exponent 1023 + k, k = 0 .. 32
   const double m = __hiloint2double((hi & 0x000FFFFF) | 0x3FF00000, __double2loint(d));
-  const double2 FL = tab.ln((static_cast<uint32_t>(hi) >> 13) & (kNoiseTableSize - 1));
-  const double r = fma(m, FL.x, -1.0);
-  double q = fma(r, -1.0 / 6.0, 1.0 / 5.0);
-  q = fma(r, q, -0.25);
-  q = fma(r, q, 1.0 / 3.0);
-  q = fma(r, q, -0.5);
-  const double ln1p_r = fma(r * r, q, r);
+  const double2 GH = tab.ln((static_cast<uint32_t>(hi) >> 13) & (kNoiseTableSize - 1));
+  const double rp = fma(m, GH.x, 2.0);
+  double q = fma(rp, 1.0 / 80.0, 1.0 / 32.0);
+  q = fma(rp, q, 1.0 / 12.0);
+  q = fma(rp, q, 0.25);
+  const double p = fma(rp * rp, q, rp);
   const double kk = u32_minus(static_cast<uint32_t>(hi) >> 20, 1055.0);  // k - 32
-  return -2.0 * (fma(kk, kLn2Hi, FL.y) + fma(kk, kLn2Lo, ln1p_r));
+  return fma(kk, kMinus2Ln2Hi, GH.y) + fma(kk, kMinus2Ln2Lo, p);
 }
 
-// sqrt(y) for 2^-126 <= y < 2^128: fp32 reciprocal-square-root seed (relative error ~2^-22),
-// one coupled Newton step on s ~ sqrt(y) and h ~ 1/(2 sqrt(y)) (Goldschmidt), then the
-// residual correction s + (y - s^2) h.
+// sqrt(y) for 2^-126 <= y < 2^128: an fp32 reciprocal-square-root seed r0 (relative error
+// e ~ 2^-22) moved into fp64 by bit manipulation, s = y r0, then one Newton step on the
+// residual, s + (y - s^2) r0 / 2, whose relative error is about e^2.
 __device__ __forceinline__ double sqrt_pos_f64(double y) {
-  const double r0 = f64_from_pos_f32(rsqrt_approx(f32_trunc_from_pos_f64(y)));
-  double s = y * r0, h = 0.5 * r0;
-  const double e = fma(-s, h, 0.5);
-  s = fma(s, e, s);
-  h = fma(h, e, h);
-  return fma(fma(-s, s, y), h, s);
+  const int yh = __double2hiint(y);
+  const uint32_t yl = static_cast<uint32_t>(__double2loint(y));
+  // y truncated to fp32: exponent rebased from 1023 to 127, 23 fraction bits.
+  const float f = __int_as_float(static_cast<int>(__funnelshift_l(yl, static_cast<uint32_t>(yh), 3)) - (896 << 23));
+  const int rb = __float_as_int(rsqrt_approx(f));
+  const int rl = rb << 29;
+  const double r0 = __hiloint2double((rb >> 3) + (896 << 20), rl);
+  const double half_r0 = __hiloint2double((rb >> 3) + (895 << 20), rl);
+  const double s = y * r0;
+  return fma(fma(-s, s, y), half_r0, s);
 }
 
 // (cos, sin) of 2 pi x 2^-32.  The top 7 bits of x pick the sector centre a_j = 2 pi (j + 1/2)
-// / 128; the other 25 bits, centred, give delta = angle - a_j exactly as an integer times
-// 2 pi 2^-32, |delta| <= pi/128.  sin(delta) to delta^7 and 1 - cos(delta) to delta^6 (next
-// terms below 1e-20 and 4e-18) then enter the addition formulas, written so that the small
-// corrections are added to the tabulated values last.
+// / 128; the other 25 bits, centred, give the integer k with angle - a_j = k a, a = 2 pi 2^-32,
+// |k a| <= pi/128.  sin(k a) to (k a)^5 and 1 - cos(k a) to (k a)^4 are polynomials in the
+// exact k^2 (next terms below 6e-16 and 3e-13), and enter the addition formulas as
+// S (1 - (1 - cos)) + C sin and C (1 - (1 - cos)) - S sin.
 template <class Tab>
 __device__ __forceinline__ void sincos_turn(uint32_t x, const Tab& tab, double& c, double& s) {
-  const double delta = u32_minus(x & 0x1FFFFFFu, 16777216.0) * kTurnToRad;
-  const double d2 = delta * delta;
-  double sp = fma(d2, -1.0 / 5040.0, 1.0 / 120.0);
-  sp = fma(d2, sp, -1.0 / 6.0);
-  const double sin_d = fma(delta * d2, sp, delta);
-  double cp = fma(d2, 1.0 / 720.0, -1.0 / 24.0);
-  cp = fma(d2, cp, 0.5);
-  const double one_minus_cos_d = d2 * cp;
+  const double k = u32_minus(x & 0x1FFFFFFu, 16777216.0);
+  const double k2 = k * k;                          // exact: |k| <= 2^24
+  double t = fma(k2, kSinK5, kSinK3);
+  t = fma(k2, t, kSinK1);
+  const double sin_d = k * t;
+  const double one_minus_cos_d = k2 * fma(k2, kCosK4, kCosK2);
   const double2 SC = tab.sincos(x >> 25);
-  s = SC.x + fma(SC.y, sin_d, -(SC.x * one_minus_cos_d));
-  c = SC.y - fma(SC.x, sin_d, SC.y * one_minus_cos_d);
+  s = fma(SC.y, sin_d, fma(-SC.x, one_minus_cos_d, SC.x));
+  c = fma(-SC.x, sin_d, fma(-SC.y, one_minus_cos_d, SC.y));
 }
 
+// (z_even, z_odd) times `scale`.
 template <class Tab>
-__device__ __forceinline__ void box_muller_f64(uint32_t x_even, uint32_t x_odd, const Tab& tab,
+__device__ __forceinline__ void box_muller_f64(uint32_t x_even, uint32_t x_odd, const Tab& tab, double scale,
                                                double& z_even, double& z_odd) {
-  const double y = minus_two_ln_u1(x_even, tab);
-  // u1 = 1 exactly (x_even = 2^32 - 1) has radius 0; y there is a rounding residue.  Every
-  // other word gives y >= 4.6e-10, inside the range of sqrt_pos_f64.
-  const double radius = x_even == 0xFFFFFFFFu ? 0.0 : sqrt_pos_f64(y);
+  // Every word but x_even = 2^32 - 1 gives y >= 4.6e-10; there u1 = 1, the radius is 0 and y
+  // is a rounding residue, which the clamp turns into a radius of 2^-50 instead.
+  const double y = fmax(minus_two_ln_u1(x_even, tab), 0x1p-100);
+  const double radius = sqrt_pos_f64(y) * scale;
   double c, s;
   sincos_turn(x_odd, tab, c, s);
   z_even = radius * c;
@@ -222,14 +217,15 @@ __device__ __forceinline__ void normals4_precise(uint32_t j, uint32_t layer_id, 
   box_muller_f64_precise(x.z, x.w, z[2], z[3]);
 }
 
-// The four standard normals of Philox block j: elements 4j .. 4j+3 of the stream.
+// The four standard normals of Philox block j (elements 4j .. 4j+3 of the stream), times
+// `scale`.
 template <class Tab = NoiseTablesGlobal>
 __device__ __forceinline__ void normals4(uint32_t j, uint32_t layer_id, uint32_t step_lo,
                                          uint32_t stream, PhiloxKey key, double (&z)[4],
-                                         const Tab& tab = Tab{}) {
+                                         const Tab& tab = Tab{}, double scale = 1.0) {
   const uint4 x = philox4x32_10(make_uint4(j, layer_id, step_lo, stream), key);
-  box_muller_f64(x.x, x.y, tab, z[0], z[1]);
-  box_muller_f64(x.z, x.w, tab, z[2], z[3]);
+  box_muller_f64(x.x, x.y, tab, scale, z[0], z[1]);
+  box_muller_f64(x.z, x.w, tab, scale, z[2], z[3]);
 }
 
 }  // namespace dpclip

@@ -36,19 +36,19 @@ __global__ void noise_add_kernel(float* __restrict__ G, unsigned long long total
   for (unsigned long long j = blockIdx.x * static_cast<unsigned long long>(blockDim.x) + threadIdx.x;
        j < nblk; j += static_cast<unsigned long long>(gridDim.x) * blockDim.x) {
     double z[4];
-    normals4(static_cast<uint32_t>(j), layer_id, step_lo, kStreamNoise, key, z, tab);
+    normals4(static_cast<uint32_t>(j), layer_id, step_lo, kStreamNoise, key, z, tab, std_dev);
     const unsigned long long k0 = 4 * j;
     if (k0 + 3 < total) {
       float4* p = reinterpret_cast<float4*>(G + k0);
       float4 g = *p;
-      g.x = static_cast<float>(static_cast<double>(g.x) + std_dev * z[0]);
-      g.y = static_cast<float>(static_cast<double>(g.y) + std_dev * z[1]);
-      g.z = static_cast<float>(static_cast<double>(g.z) + std_dev * z[2]);
-      g.w = static_cast<float>(static_cast<double>(g.w) + std_dev * z[3]);
+      g.x = static_cast<float>(static_cast<double>(g.x) + z[0]);
+      g.y = static_cast<float>(static_cast<double>(g.y) + z[1]);
+      g.z = static_cast<float>(static_cast<double>(g.z) + z[2]);
+      g.w = static_cast<float>(static_cast<double>(g.w) + z[3]);
       *p = g;
     } else {
       for (int q = 0; q < 4 && k0 + q < total; ++q)
-        G[k0 + q] = static_cast<float>(static_cast<double>(G[k0 + q]) + std_dev * z[q]);
+        G[k0 + q] = static_cast<float>(static_cast<double>(G[k0 + q]) + z[q]);
     }
   }
 }
@@ -83,10 +83,24 @@ __global__ void noise_add_batch_kernel(NoiseBatch b, PhiloxKey key, StepRef step
     }
     const NoiseSegment& sg = b.seg[q];
     double z[4];
-    normals4(static_cast<uint32_t>(jj), sg.layer_id, step_lo, kStreamNoise, key, z);
+    normals4(static_cast<uint32_t>(jj), sg.layer_id, step_lo, kStreamNoise, key, z, NoiseTablesGlobal{},
+             sg.std_dev);
     const unsigned long long k0 = 4 * jj;
     for (int e = 0; e < 4 && k0 + e < sg.total; ++e)
-      sg.G[k0 + e] = static_cast<float>(static_cast<double>(sg.G[k0 + e]) + sg.std_dev * z[e]);
+      sg.G[k0 + e] = static_cast<float>(static_cast<double>(sg.G[k0 + e]) + z[e]);
+  }
+}
+
+// (z[2q], z[2q+1]) = the noise's Box-Muller transform of words (2q, 2q+1), unscaled
+// (verification of the transform on chosen words).
+__global__ void box_muller_words_kernel(const uint2* __restrict__ words, double2* __restrict__ z,
+                                        unsigned long long npairs) {
+  for (unsigned long long q = blockIdx.x * static_cast<unsigned long long>(blockDim.x) + threadIdx.x;
+       q < npairs; q += static_cast<unsigned long long>(gridDim.x) * blockDim.x) {
+    const uint2 w = words[q];
+    double a, b;
+    box_muller_f64(w.x, w.y, NoiseTablesGlobal{}, 1.0, a, b);
+    z[q] = make_double2(a, b);
   }
 }
 
@@ -307,11 +321,11 @@ __global__ void __launch_bounds__(256, 2) clip_reduce_kernel(
     if (noise_std != 0.0) {
       double z[8];
       normals4(static_cast<uint32_t>(2 * v), layer_id, step_lo, kStreamNoise, key,
-               *reinterpret_cast<double(*)[4]>(z), tab);
+               *reinterpret_cast<double(*)[4]>(z), tab, noise_std);
       normals4(static_cast<uint32_t>(2 * v + 1), layer_id, step_lo, kStreamNoise, key,
-               *reinterpret_cast<double(*)[4]>(z + 4), tab);
+               *reinterpret_cast<double(*)[4]>(z + 4), tab, noise_std);
 #pragma unroll
-      for (int q = 0; q < 8; ++q) acc[q] = acc[q] + __double2float_rn(noise_std * z[q]);
+      for (int q = 0; q < 8; ++q) acc[q] = acc[q] + __double2float_rn(z[q]);
     }
     float4* o = reinterpret_cast<float4*>(out) + 2 * v;
     o[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
@@ -418,9 +432,9 @@ __global__ void __launch_bounds__(ReduceTmaConfig<BU>::THREADS, 1) clip_reduce_t
       double z[8];
       if (noise_std != 0.0 && e < mn) {
         normals4(static_cast<uint32_t>(e >> 2), layer_id, step_lo, kStreamNoise, key,
-                 *reinterpret_cast<double(*)[4]>(z), tab);
+                 *reinterpret_cast<double(*)[4]>(z), tab, noise_std);
         normals4(static_cast<uint32_t>((e >> 2) + 1), layer_id, step_lo, kStreamNoise, key,
-                 *reinterpret_cast<double(*)[4]>(z + 4), tab);
+                 *reinterpret_cast<double(*)[4]>(z + 4), tab, noise_std);
       }
       if (need_c) {
         // Every compute warp passes here in its first iteration (the trip count is the same
@@ -446,7 +460,7 @@ __global__ void __launch_bounds__(ReduceTmaConfig<BU>::THREADS, 1) clip_reduce_t
         }
         if (noise_std != 0.0) {
 #pragma unroll
-          for (int q = 0; q < 8; ++q) acc[q] = acc[q] + __double2float_rn(noise_std * z[q]);
+          for (int q = 0; q < 8; ++q) acc[q] = acc[q] + __double2float_rn(z[q]);
         }
         float4* o = reinterpret_cast<float4*>(out + e);
         o[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
@@ -597,8 +611,8 @@ __global__ void __launch_bounds__(256) f32_clipsum_kernel(
   if (noise_std != 0.0) {
     const unsigned long long k = static_cast<unsigned long long>(a) * n + b;
     double z[4];
-    normals4(static_cast<uint32_t>(k >> 2), layer_id, step_lo, kStreamNoise, key, z);
-    for (int q = 0; q < 4; ++q) acc[q] += noise_std * z[q];
+    normals4(static_cast<uint32_t>(k >> 2), layer_id, step_lo, kStreamNoise, key, z, NoiseTablesGlobal{}, noise_std);
+    for (int q = 0; q < 4; ++q) acc[q] += z[q];
   }
   for (int q = 0; q < 4; ++q) dst[q] = static_cast<float>(acc[q]);
 }

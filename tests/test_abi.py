@@ -152,6 +152,16 @@ def test_philox_blocks_rejects_on_host(L):
     assert L.dp_philox_blocks(FAKE, (1 << 32) + 1, 0, 0, 0, 0, None) == E
 
 
+def test_box_muller_rejects_on_host(L):
+    E = _lib.DP_ERR_INVALID_ARG
+    assert L.dp_box_muller(None, 4, FAKE, None) == E
+    assert L.dp_box_muller(FAKE, 4, None, None) == E
+    assert L.dp_box_muller(ODD, 4, FAKE, None) == E
+    assert L.dp_box_muller(FAKE, 4, ODD, None) == E
+    assert L.dp_box_muller(FAKE, 0, FAKE, None) == E
+    assert L.dp_box_muller(FAKE, (1 << 40) + 1, FAKE, None) == E
+
+
 def test_block_workspace_size_and_host_rejections(L):
     from sample_gradient_clipping_b200._lib import DpLayer
     lay = (DpLayer * 2)(DpLayer(FAKE, FAKE, 4096, 4096, 0, 0.3, FAKE, None),

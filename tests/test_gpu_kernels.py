@@ -37,6 +37,43 @@ def test_philox_words_bit_exact(seed, step, layer, stream):
     assert np.array_equal(got, want)
 
 
+def _edge_words():
+    """Words at every breakpoint of the transform's tables, their neighbours and the extremes:
+    x_even where x + 1 = 2^k (1 + j/128) starts a ln-table interval (and its centre), x_odd at
+    the start, centre and end of every 1/128-turn sector."""
+    xe = {0, 1, 2, 3, 0x7FFFFFFF, 0x80000000, 0xFFFFFFFD, 0xFFFFFFFE, 0xFFFFFFFF}
+    for k in (0, 1, 2, 5, 12, 20, 26, 30, 31):
+        for j in range(128):
+            for num in (2 * j, 2 * j + 1):           # interval start and centre, in 1/256 steps
+                v = ((256 + num) << k) // 256 - 1
+                for d in (-1, 0, 1):
+                    if 0 <= v + d < 1 << 32:
+                        xe.add(v + d)
+    xo = set()
+    for j in range(128):
+        for off in (0, 1, (1 << 24) - 1, 1 << 24, (1 << 24) + 1, (1 << 25) - 1):
+            xo.add((j << 25) + off)
+    return np.array(sorted(xe), np.uint32), np.array(sorted(xo), np.uint32)
+
+
+def test_box_muller_transform_on_edge_words():
+    # The transform alone, on chosen words, against the oracle's fp64 Box-Muller (itself within
+    # 1e-13 of 40-digit arithmetic): far tighter than the 1e-6 noise tolerance.
+    xe, xo = _edge_words()
+    pe, po = np.repeat(xe, xo.size), np.tile(xo, xe.size)
+    rng = np.random.default_rng(11)
+    pe = np.concatenate([pe, rng.integers(0, 1 << 32, 1 << 20, dtype=np.uint64).astype(np.uint32)])
+    po = np.concatenate([po, rng.integers(0, 1 << 32, 1 << 20, dtype=np.uint64).astype(np.uint32)])
+    words = torch.from_numpy(np.stack([pe, po], axis=1).view(np.int32)).cuda()
+    got = _lib.dp_box_muller(words).cpu().numpy()
+    ze, zo = oracle.box_muller(pe, po)
+    err = max(np.max(np.abs(got[:, 0] - ze)), np.max(np.abs(got[:, 1] - zo)))
+    assert err <= 1e-11, err
+    # u1 = 1: radius 0 (the transform returns a radius of 2^-50 there)
+    last = np.flatnonzero(pe == 0xFFFFFFFF)
+    assert np.all(np.abs(got[last]) <= 1e-14)
+
+
 @pytest.mark.parametrize("rows,cols", [(1, 1), (3, 5), (64, 32), (257, 520), (1000, 1003), (768, 3072),
                                        (2048, 2052)])   # the last stages the tables in shared memory
 @pytest.mark.parametrize("std", [1.0, 0.6 / math.sqrt(7.0)])
