@@ -39,8 +39,8 @@ KERNEL_SOURCES = ("sample_gradient_clipping_b200/csrc/ptx.cuh",
                   "sample_gradient_clipping_b200/csrc/umma_gemm_2sm.cuh")
 # (workload, kernel) -> (bytes per launch, source hash)
 MEASURED_TRAFFIC = {
-    ("llama7b_block", "umma_explicit_store"): (872185966, "ee30b8916c2920d7"),
-    ("llama13b_block", "umma_explicit_store"): (674696229, "ee30b8916c2920d7"),
+    ("llama7b_block", "umma_explicit_store"): (878553015, "574fbf108032c9c0"),
+    ("llama13b_block", "umma_explicit_store"): (676394167, "574fbf108032c9c0"),
 }
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 

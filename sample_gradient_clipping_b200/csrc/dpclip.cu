@@ -11,6 +11,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <utility>
 #include <vector>
 
 #include "dpclip.h"
@@ -37,10 +38,31 @@ dp_status cuda_fail(cudaError_t e, const char* what) {
     if (e_ != cudaSuccess) return cuda_fail(e_, #call); \
   } while (0)
 
-#define DP_CHECK_LAUNCH(what)                          \
-  do {                                                 \
-    cudaError_t e_ = cudaGetLastError();               \
-    if (e_ != cudaSuccess) return cuda_fail(e_, what); \
+// Every kernel is launched with programmatic stream serialization: it may be scheduled while
+// the previous kernel in the stream drains, runs its local prologue, and waits for that kernel
+// (griddep_wait in ptx.cuh) before its first access to global memory.  This hides most of the
+// launch gap between the short kernels of a step.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                          cudaStream_t stream, Args&&... args) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+#define DP_LAUNCH(what, ...)                             \
+  do {                                                   \
+    cudaError_t e_ = launch_kernel(__VA_ARGS__);         \
+    if (e_ == cudaSuccess) e_ = cudaGetLastError();      \
+    if (e_ != cudaSuccess) return cuda_fail(e_, what);   \
   } while (0)
 
 inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -241,8 +263,7 @@ dp_status launch_umma_pair(const UmmaParams& p, cudaStream_t stream) {
                        : Cfg::EPI == kEpiClipSum     ? kKindClipSum
                                                      : kKindExplicitNorm;
   LaunchScope scope(kind, stream);
-  umma_pair_kernel<Cfg><<<2 * pairs, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(p);
-  DP_CHECK_LAUNCH("umma_pair_kernel");
+  DP_LAUNCH("umma_pair_kernel", umma_pair_kernel<Cfg>, 2 * pairs, Cfg::THREADS, Cfg::SMEM_BYTES, stream, p);
   return DP_OK;
 }
 
@@ -266,8 +287,7 @@ dp_status launch_umma(const UmmaParams& p, cudaStream_t stream) {
                        : Cfg::EPI == kEpiGhostShared   ? kKindGhostShared
                                                        : kKindProject;
   LaunchScope scope(kind, stream);
-  umma_kernel<Cfg><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(p);
-  DP_CHECK_LAUNCH("umma_kernel");
+  DP_LAUNCH("umma_kernel", umma_kernel<Cfg>, grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream, p);
   return DP_OK;
 }
 
@@ -439,8 +459,8 @@ dp_status launch_noise_batch(const NoiseBatch& b, unsigned long long seed, StepR
   unsigned long long nblk = 0;
   for (int q = 0; q < b.count; ++q) nblk += (b.seg[q].total + 3) / 4;
   LaunchScope scope(kKindNoise, stream);
-  noise_add_batch_kernel<<<stream_grid(nblk, 256), 256, 0, stream>>>(b, philox_key_from_seed(seed), step);
-  DP_CHECK_LAUNCH("noise_add_batch_kernel");
+  DP_LAUNCH("noise_add_batch_kernel", noise_add_batch_kernel, stream_grid(nblk, 256), 256, 0, stream, b,
+            philox_key_from_seed(seed), step);
   return DP_OK;
 }
 
@@ -451,12 +471,12 @@ dp_status launch_noise(float* G, unsigned long long total, double std_dev, unsig
   const PhiloxKey key = philox_key_from_seed(seed);
   if (total >= (1ull << 22)) {
     const int grid = std::min(stream_grid((total + 3) / 4, 256), sm_count() * 4);
-    noise_add_kernel<true><<<grid, 256, 0, stream>>>(G, total, std_dev, key, layer_id, step);
+    DP_LAUNCH("noise_add_kernel", noise_add_kernel<true>, grid, 256, 0, stream, G, total, std_dev, key,
+              layer_id, step);
   } else {
-    noise_add_kernel<false><<<stream_grid((total + 3) / 4, 256), 256, 0, stream>>>(G, total, std_dev, key,
-                                                                                  layer_id, step);
+    DP_LAUNCH("noise_add_kernel", noise_add_kernel<false>, stream_grid((total + 3) / 4, 256), 256, 0, stream,
+              G, total, std_dev, key, layer_id, step);
   }
-  DP_CHECK_LAUNCH("noise_add_kernel");
   return DP_OK;
 }
 
@@ -491,29 +511,33 @@ dp_status launch_projection(void* P, dp_dtype dt, int d_out, int r, unsigned lon
   const PhiloxKey key = philox_key_from_seed(seed);
   LaunchScope scope(kKindProjection, stream);
   if (dt == DP_BF16)
-    projection_kernel<true><<<grid, 256, 0, stream>>>(P, total, r, key, layer_id);
+    DP_LAUNCH("projection_kernel", projection_kernel<true>, grid, 256, 0, stream, P, total, r, key, layer_id);
   else
-    projection_kernel<false><<<grid, 256, 0, stream>>>(P, total, r, key, layer_id);
-  DP_CHECK_LAUNCH("projection_kernel");
+    DP_LAUNCH("projection_kernel", projection_kernel<false>, grid, 256, 0, stream, P, total, r, key,
+              layer_id);
   return DP_OK;
 }
 
 dp_status launch_norm_partials(const float* partials, int stride, int count, int B, float C,
                                float* norm2, float* norms_out, float* c_out, cudaStream_t stream);
 
-// With `partials` (B samples), the scaling kernel forms the clip factors itself when B <= 8
-// and B * count is small; otherwise the partials kernel runs first.
+// With `partials` (B samples), the scaling kernel forms the clip factors of the samples each
+// of its blocks covers, unless a block would cover too many samples or partial slots; then the
+// partials kernel runs first.
 dp_status launch_scale(const void* in, void* out, long long rows, int cols, int T, NormSource src,
                        float C, cudaStream_t stream, const PartialsRef* partials = nullptr, int B = 0) {
   const unsigned long long vecs = static_cast<unsigned long long>(rows) * (cols / 8);
+  const int grid = stream_grid(vecs, 256);
   PartialsRef pr{nullptr, 0, 0, nullptr, nullptr, nullptr};
   size_t smem = 0;
   if (partials) {
-    // One warp per sample in each 256-thread block: with more samples than warps, the serial
-    // rounds of partial sums cost more in every block than the separate launch (measured).
-    if (B <= 8 && static_cast<long long>(B) * partials->count <= kScaleFusedPartialSlots) {
+    // A block's contiguous range of `per` vectors touches at most this many samples.
+    const unsigned long long per = (vecs + grid - 1) / grid;
+    const unsigned long long sample_vecs = static_cast<unsigned long long>(T) * (cols / 8);
+    const long long smax = static_cast<long long>(std::min<unsigned long long>((per - 1) / sample_vecs + 2, B));
+    if (smax <= kScaleFusedMaxSamples && smax * partials->count <= kScaleFusedPartialSlots) {
       pr = *partials;
-      smem = static_cast<size_t>(B) * sizeof(float);
+      smem = static_cast<size_t>(smax) * sizeof(float);
     } else {
       dp_status st = launch_norm_partials(partials->partials, partials->stride, partials->count, B, C,
                                           partials->norm2, partials->norms_out, partials->c_out, stream);
@@ -522,33 +546,34 @@ dp_status launch_scale(const void* in, void* out, long long rows, int cols, int 
     }
   }
   LaunchScope scope(kKindScale, stream);
-  scale_rows_bf16_kernel<<<stream_grid(vecs, 256), 256, smem, stream>>>(
-      static_cast<const __nv_bfloat16*>(in), static_cast<__nv_bfloat16*>(out), rows, cols, T, src, pr, B, C);
-  DP_CHECK_LAUNCH("scale_rows_bf16_kernel");
+  DP_LAUNCH("scale_rows_bf16_kernel", scale_rows_bf16_kernel, grid, 256, smem, stream,
+            static_cast<const __nv_bfloat16*>(in), static_cast<__nv_bfloat16*>(out), rows, cols, T, src, pr,
+            C);
   return DP_OK;
 }
 
 dp_status launch_norm_partials(const float* partials, int stride, int count, int B, float C,
                                float* norm2, float* norms_out, float* c_out, cudaStream_t stream) {
   LaunchScope scope(kKindFinalize, stream);
-  reduce_norm_partials_kernel<<<ceil_div(B, 8), 256, 0, stream>>>(partials, stride, count, B, C, norm2,
-                                                                   norms_out, c_out);
-  DP_CHECK_LAUNCH("reduce_norm_partials_kernel");
+  DP_LAUNCH("reduce_norm_partials_kernel", reduce_norm_partials_kernel, ceil_div(B, 8), 256, 0, stream,
+            partials, stride, count, B, C, norm2, norms_out, c_out);
   return DP_OK;
 }
 
 dp_status launch_finalize(NormSource src, int B, float C, float* norms_out, float* c_out,
                           cudaStream_t stream) {
   LaunchScope scope(kKindFinalize, stream);
-  finalize_norms_kernel<<<ceil_div(B, 256), 256, 0, stream>>>(src, B, C, norms_out, c_out);
-  DP_CHECK_LAUNCH("finalize_norms_kernel");
+  DP_LAUNCH("finalize_norms_kernel", finalize_norms_kernel, ceil_div(B, 256), 256, 0, stream, src, B, C,
+            norms_out, c_out);
   return DP_OK;
 }
 
-void reduce_kernel_launch(int grid, size_t smem, cudaStream_t stream, const __nv_bfloat16* gs, int B,
+dp_status reduce_kernel_launch(int grid, size_t smem, cudaStream_t stream, const __nv_bfloat16* gs, int B,
                           long long mn, NormSource src, float C, float* out, double noise_std, PhiloxKey key,
                           unsigned layer_id, StepRef step) {
-  clip_reduce_kernel<<<grid, 256, smem, stream>>>(gs, B, mn, src, C, out, noise_std, key, layer_id, step);
+  DP_LAUNCH("clip_reduce_kernel", clip_reduce_kernel, grid, 256, smem, stream, gs, B, mn, src, C, out,
+            noise_std, key, layer_id, step);
+  return DP_OK;
 }
 
 template <int BU>
@@ -566,9 +591,8 @@ dp_status reduce_tma_launch(cudaStream_t stream, const __nv_bfloat16* gs, long l
   }
   const long long chunks = (mn + kReduceChunk - 1) / kReduceChunk;
   const int grid = static_cast<int>(chunks < sm_count() ? chunks : sm_count());
-  clip_reduce_tma_kernel<BU><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(gs, mn, src, pr, C, out,
-                                                                               noise_std, key, layer_id, step,
-                                                                               status);
+  DP_LAUNCH("clip_reduce_tma_kernel", clip_reduce_tma_kernel<BU>, grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream,
+            gs, mn, src, pr, C, out, noise_std, key, layer_id, step, status);
   return DP_OK;
 }
 
@@ -596,7 +620,6 @@ dp_status launch_reduce(const __nv_bfloat16* gs, int B, long long mn, NormSource
       default: st = reduce_tma_launch<8>(stream, gs, mn, src, pr, C, out, noise_std, key, layer_id, step, status); break;
     }
     if (st != DP_OK) return st;
-    DP_CHECK_LAUNCH("clip_reduce_tma_kernel");
     return DP_OK;
   }
   if (partials) {
@@ -611,9 +634,7 @@ dp_status launch_reduce(const __nv_bfloat16* gs, int B, long long mn, NormSource
   const PhiloxKey key = philox_key_from_seed(seed);
   LaunchScope scope(kKindReduce, stream);
   // B > 8 here (smaller batches take the bulk-copy kernel above): a runtime sample loop.
-  reduce_kernel_launch(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step);
-  DP_CHECK_LAUNCH("clip_reduce_kernel");
-  return DP_OK;
+  return reduce_kernel_launch(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step);
 }
 
 // ---------------------------------------------------------------- common front end
@@ -665,10 +686,9 @@ dp_status clip_space_operand(Call& c, const void* dY, const void* P, bool p_from
   } else {
     const long long total = c.s.N() * c.s.r;
     LaunchScope scope(kKindF32Project, c.stream);
-    f32_project_kernel<<<stream_grid(total, 256), 256, 0, c.stream>>>(
-        static_cast<const float*>(dY), static_cast<const float*>(Pd), static_cast<float*>(Z), c.s.N(),
-        c.s.n, c.s.r);
-    DP_CHECK_LAUNCH("f32_project_kernel");
+    DP_LAUNCH("f32_project_kernel", f32_project_kernel, stream_grid(total, 256), 256, 0, c.stream,
+              static_cast<const float*>(dY), static_cast<const float*>(Pd), static_cast<float*>(Z), c.s.N(),
+              c.s.n, c.s.r);
   }
   *Zout = Z;
   return DP_OK;
@@ -681,9 +701,8 @@ dp_status norms_into_ws(Call& c, const void* X, const void* Z, dp_norm_method me
   if (c.s.dt == DP_F32) {
     dim3 grid(ceil_div(c.s.ne(), kF32Tile), ceil_div(c.s.m, kF32Tile), c.s.B);
     LaunchScope scope(kKindF32Norm, c.stream);
-    f32_norm_kernel<<<grid, 256, 0, c.stream>>>(static_cast<const float*>(X), static_cast<const float*>(Z),
-                                                 c.s.T, c.s.m, c.s.ne(), c.norm2_f64());
-    DP_CHECK_LAUNCH("f32_norm_kernel");
+    DP_LAUNCH("f32_norm_kernel", f32_norm_kernel, grid, 256, 0, c.stream, static_cast<const float*>(X),
+              static_cast<const float*>(Z), c.s.T, c.s.m, c.s.ne(), c.norm2_f64());
     return DP_OK;
   }
   int count = 0;
@@ -713,10 +732,9 @@ dp_status clipped_sum(Call& c, const void* X, const void* Z, NormSource src, flo
     dim3 grid(ceil_div(s.ne(), kF32Tile), ceil_div(s.m, kF32Tile));
     const PhiloxKey key = philox_key_from_seed(seed);
     LaunchScope scope(kKindF32ClipSum, c.stream);
-    f32_clipsum_kernel<<<grid, 256, 0, c.stream>>>(
-        static_cast<const float*>(X), static_cast<const float*>(Z), s.N(), s.T, s.m, s.ne(), src, C,
-        out, accumulate, noise_std, key, layer_id, step);
-    DP_CHECK_LAUNCH("f32_clipsum_kernel");
+    DP_LAUNCH("f32_clipsum_kernel", f32_clipsum_kernel, grid, 256, 0, c.stream, static_cast<const float*>(X),
+              static_cast<const float*>(Z), s.N(), s.T, s.m, s.ne(), src, C, out, accumulate, noise_std, key,
+              layer_id, step);
     return DP_OK;
   }
   // Fold c_i into the narrower operand: one extra read + write of N * min(m, ne) bf16.
@@ -878,9 +896,9 @@ dp_status block_operand(const dp_layer* layers, int l, dp_dtype dt, int B, int T
   if (dt == DP_BF16) return bf16_project(s, y.dY, y.P, z, reinterpret_cast<uint32_t*>(ws), stream);
   const long long total = s.N() * s.r;
   LaunchScope scope(kKindF32Project, stream);
-  f32_project_kernel<<<stream_grid(total, 256), 256, 0, stream>>>(
-      static_cast<const float*>(y.dY), static_cast<const float*>(y.P), static_cast<float*>(z), s.N(), s.n, s.r);
-  DP_CHECK_LAUNCH("f32_project_kernel");
+  DP_LAUNCH("f32_project_kernel", f32_project_kernel, stream_grid(total, 256), 256, 0, stream,
+            static_cast<const float*>(y.dY), static_cast<const float*>(y.P), static_cast<float*>(z), s.N(),
+            s.n, s.r);
   return DP_OK;
 }
 
@@ -900,9 +918,8 @@ dp_status block_group_norms(const dp_layer* layers, const std::vector<int>& g, d
     dim3 grid(ceil_div(s.ne(), kF32Tile), ceil_div(s.m, kF32Tile), B);
     {
       LaunchScope scope(kKindF32Norm, stream);
-      f32_norm_kernel<<<grid, 256, 0, stream>>>(static_cast<const float*>(y0.X), static_cast<const float*>(Zs[0]),
-                                                 T, s.m, s.ne(), n2);
-      DP_CHECK_LAUNCH("f32_norm_kernel");
+      DP_LAUNCH("f32_norm_kernel", f32_norm_kernel, grid, 256, 0, stream, static_cast<const float*>(y0.X),
+                static_cast<const float*>(Zs[0]), T, s.m, s.ne(), n2);
     }
     if (y0.norms_out) {
       NormSource src{nullptr, n2, nullptr};
@@ -1030,16 +1047,15 @@ dp_status block_step(const dp_layer* layers, int L, dp_dtype dt, int B, int T, d
     LaunchScope scope(kKindFinalize, stream);
     if (dt == DP_F32) {
       double* flat = reinterpret_cast<double*>(ws + Lb.flat);
-      flat_norm2_kernel<double><<<ceil_div(B, 256), 256, 0, stream>>>(
-          reinterpret_cast<const double*>(ws + Lb.norm2), L, B, flat, flat_norms_out);
+      DP_LAUNCH("flat_norm2_kernel", flat_norm2_kernel<double>, ceil_div(B, 256), 256, 0, stream,
+                reinterpret_cast<const double*>(ws + Lb.norm2), L, B, flat, flat_norms_out);
       src.norm2_f64 = flat;
     } else {
       float* flat = reinterpret_cast<float*>(ws + Lb.flat);
-      flat_norm2_kernel<float><<<ceil_div(B, 256), 256, 0, stream>>>(
-          reinterpret_cast<const float*>(ws + Lb.norm2), L, B, flat, flat_norms_out);
+      DP_LAUNCH("flat_norm2_kernel", flat_norm2_kernel<float>, ceil_div(B, 256), 256, 0, stream,
+                reinterpret_cast<const float*>(ws + Lb.norm2), L, B, flat, flat_norms_out);
       src.norm2_f32 = flat;
     }
-    DP_CHECK_LAUNCH("flat_norm2_kernel");
   }
   // 3. Every layer's clipped sum with the shared clip factors, plus its own noise.
   for (int l = 0; l < L; ++l)
@@ -1235,10 +1251,9 @@ dp_status dp_philox_blocks(unsigned* out, unsigned long long nblocks, unsigned l
                            void* stream) {
   if (!out || !aligned16(out) || nblocks < 1 || nblocks > (1ull << 32)) return DP_ERR_INVALID_ARG;
   LaunchScope scope(kKindPhilox, static_cast<cudaStream_t>(stream));
-  philox_blocks_kernel<<<stream_grid(nblocks, 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      reinterpret_cast<uint4*>(out), nblocks, philox_key_from_seed(seed), layer_id,
-      static_cast<uint32_t>(step & 0xFFFFFFFFull), stream_id);
-  DP_CHECK_LAUNCH("philox_blocks_kernel");
+  DP_LAUNCH("philox_blocks_kernel", philox_blocks_kernel, stream_grid(nblocks, 256), 256, 0,
+            static_cast<cudaStream_t>(stream), reinterpret_cast<uint4*>(out), nblocks,
+            philox_key_from_seed(seed), layer_id, static_cast<uint32_t>(step & 0xFFFFFFFFull), stream_id);
   return DP_OK;
 }
 
@@ -1247,9 +1262,9 @@ dp_status dp_box_muller(const unsigned* words, long long npairs, double* z, void
     return DP_ERR_INVALID_ARG;
   LaunchScope scope(kKindNoise, static_cast<cudaStream_t>(stream));
   const unsigned long long n = static_cast<unsigned long long>(npairs);
-  box_muller_words_kernel<<<stream_grid(n, 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      reinterpret_cast<const uint2*>(words), reinterpret_cast<double2*>(z), n);
-  DP_CHECK_LAUNCH("box_muller_words_kernel");
+  DP_LAUNCH("box_muller_words_kernel", box_muller_words_kernel, stream_grid(n, 256), 256, 0,
+            static_cast<cudaStream_t>(stream), reinterpret_cast<const uint2*>(words),
+            reinterpret_cast<double2*>(z), n);
   return DP_OK;
 }
 
@@ -1287,9 +1302,8 @@ dp_status dp_per_sample_norms_static(const void* X, const void* dY, dp_dtype dt,
     dim3 grid(ceil_div(d_out, kF32Tile), ceil_div(d_in, kF32Tile), B);
     {
       LaunchScope scope(kKindF32Norm, cs);
-      f32_norm_kernel<<<grid, 256, 0, cs>>>(static_cast<const float*>(X), static_cast<const float*>(dY), T,
-                                            d_in, d_out, norm2);
-      DP_CHECK_LAUNCH("f32_norm_kernel");
+      DP_LAUNCH("f32_norm_kernel", f32_norm_kernel, grid, 256, 0, cs, static_cast<const float*>(X),
+                static_cast<const float*>(dY), T, d_in, d_out, norm2);
     }
     NormSource src{nullptr, norm2, nullptr};
     return launch_finalize(src, B, INFINITY, norms, nullptr, cs);
@@ -1386,9 +1400,9 @@ dp_status dp_projected_adam_step(float* W, const float* R, float* m, float* v, c
   const float bc2 = 1.0f - static_cast<float>(std::pow(static_cast<double>(beta2), t));
   {
     LaunchScope scope(kKindAdam, cs);
-    adam_rspace_kernel<<<stream_grid(static_cast<unsigned long long>(n / 4), 256), 256, 0, cs>>>(
-        R, m, v, U, n, grad_scale, beta1, beta2, eps, bc1, bc2);
-    DP_CHECK_LAUNCH("adam_rspace_kernel");
+    DP_LAUNCH("adam_rspace_kernel", adam_rspace_kernel,
+              stream_grid(static_cast<unsigned long long>(n / 4), 256), 256, 0, cs, R, m, v, U, n, grad_scale,
+              beta1, beta2, eps, bc1, bc2);
   }
   if (lr == 0.0f) return DP_OK;
   UmmaParams p = base_params(reinterpret_cast<uint32_t*>(ws));
@@ -1412,8 +1426,8 @@ dp_status dp_selftest_wait_timeout(void* workspace, unsigned long long limit_ns,
   if (limit_ns < 1000ull || limit_ns > kWaitLimitNs) return DP_ERR_INVALID_ARG;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   DP_CUDA(cudaMemsetAsync(workspace, 0, 256, cs));
-  wait_timeout_selftest_kernel<<<1, 32, 0, cs>>>(static_cast<uint32_t*>(workspace), limit_ns);
-  DP_CHECK_LAUNCH("wait_timeout_selftest_kernel");
+  DP_LAUNCH("wait_timeout_selftest_kernel", wait_timeout_selftest_kernel, 1, 32, 0, cs,
+            static_cast<uint32_t*>(workspace), limit_ns);
   return DP_OK;
 }
 

@@ -28,6 +28,24 @@ __device__ __forceinline__ uint32_t lane_id() {
   return l;
 }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+// Every kernel of the library is launched so that it may start while the previous kernel in
+// its stream drains.  griddep_wait() returns once every kernel this one depends on in stream
+// order has completed and its writes are visible (at once when there is none); each kernel
+// calls it before its first access to global memory, so stream order holds for all data, and
+// transitively across kernels.  griddep_launch_dependents() lets the next kernel's blocks be
+// scheduled (they run their own prologue and wait in turn): the short CUDA-core kernels call
+// it at once (griddep_enter), the tensor-core kernels only after their main loops, so that
+// waiting blocks do not sit beside them on their SMs (measured faster on the small workloads).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_enter() {
+  griddep_wait();
+  griddep_launch_dependents();
+}
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");

@@ -23,6 +23,7 @@ namespace dpclip {
 template <bool STAGED>
 __global__ void noise_add_kernel(float* __restrict__ G, unsigned long long total, double std_dev,
                                  PhiloxKey key, uint32_t layer_id, StepRef step) {
+  griddep_enter();
   __shared__ double2 tab_s[STAGED ? kNoiseSharedEntries : 1];
   const uint32_t step_lo = step.get();
   if constexpr (STAGED) {
@@ -70,6 +71,7 @@ struct NoiseBatch {
 };
 
 __global__ void noise_add_batch_kernel(NoiseBatch b, PhiloxKey key, StepRef step) {
+  griddep_enter();
   const uint32_t step_lo = step.get();
   unsigned long long nblk_total = 0;
   for (int q = 0; q < b.count; ++q) nblk_total += (b.seg[q].total + 3) / 4;
@@ -95,6 +97,7 @@ __global__ void noise_add_batch_kernel(NoiseBatch b, PhiloxKey key, StepRef step
 // (verification of the transform on chosen words).
 __global__ void box_muller_words_kernel(const uint2* __restrict__ words, double2* __restrict__ z,
                                         unsigned long long npairs) {
+  griddep_enter();
   for (unsigned long long q = blockIdx.x * static_cast<unsigned long long>(blockDim.x) + threadIdx.x;
        q < npairs; q += static_cast<unsigned long long>(gridDim.x) * blockDim.x) {
     const uint2 w = words[q];
@@ -108,6 +111,7 @@ __global__ void box_muller_words_kernel(const uint2* __restrict__ words, double2
 __global__ void philox_blocks_kernel(uint4* __restrict__ out, unsigned long long nblocks,
                                      PhiloxKey key, uint32_t layer_id, uint32_t step_lo,
                                      uint32_t stream_id) {
+  griddep_enter();
   for (unsigned long long j = blockIdx.x * static_cast<unsigned long long>(blockDim.x) + threadIdx.x;
        j < nblocks; j += static_cast<unsigned long long>(gridDim.x) * blockDim.x)
     out[j] = philox4x32_10(make_uint4(static_cast<uint32_t>(j), layer_id, step_lo, stream_id), key);
@@ -117,6 +121,7 @@ __global__ void philox_blocks_kernel(uint4* __restrict__ out, unsigned long long
 template <bool BF16>
 __global__ void projection_kernel(void* __restrict__ P, unsigned long long total, int r,
                                   PhiloxKey key, uint32_t layer_id) {
+  griddep_enter();
   const double scale = sqrt(static_cast<double>(r));
   const unsigned long long nblk = (total + 3) / 4;
   for (unsigned long long j = blockIdx.x * static_cast<unsigned long long>(blockDim.x) + threadIdx.x;
@@ -197,6 +202,7 @@ struct PartialsRef {
 __global__ void reduce_norm_partials_kernel(const float* __restrict__ partials, int stride, int count,
                                             int B, float C, float* __restrict__ norm2,
                                             float* __restrict__ norms_out, float* __restrict__ c_out) {
+  griddep_enter();
   const int i = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
   if (i >= B) return;
@@ -215,6 +221,7 @@ __global__ void reduce_norm_partials_kernel(const float* __restrict__ partials, 
 template <typename T>
 __global__ void flat_norm2_kernel(const T* __restrict__ norm2_layers, int L, int B, T* __restrict__ flat,
                                   float* __restrict__ flat_norms_out) {
+  griddep_enter();
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < B; i += gridDim.x * blockDim.x) {
     double acc = 0.0;
     for (int l = 0; l < L; ++l) acc += static_cast<double>(norm2_layers[static_cast<long long>(l) * B + i]);
@@ -226,6 +233,7 @@ __global__ void flat_norm2_kernel(const T* __restrict__ norm2_layers, int L, int
 // norms_out[i] = n_i and c_out[i] = c_i for i < B (either may be null).
 __global__ void finalize_norms_kernel(NormSource src, int B, float C, float* __restrict__ norms_out,
                                       float* __restrict__ c_out) {
+  griddep_enter();
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < B; i += gridDim.x * blockDim.x) {
     const float n = src.norm(i);
     if (norms_out) norms_out[i] = n;
@@ -235,38 +243,57 @@ __global__ void finalize_norms_kernel(NormSource src, int B, float C, float* __r
 
 // out[row, :] = bf16(c_{row / T} * in[row, :]) for a [rows, cols] bf16 matrix, 8 elements per
 // thread (cols is a multiple of 8, rows are 16-byte aligned).
-// With pr.partials, every block first turns the per-warp norm partials of all B samples into
-// clip factors in shared memory (one warp per sample, the fixed-order routine above), and
-// block 0 writes norm2 / norms_out / c_out: the separate partials kernel is not needed.
-constexpr long long kScaleFusedPartialSlots = 1 << 16;  // B * count up to which blocks do that
+// With pr.partials, each block takes one contiguous range of the matrix, which covers the rows
+// of one or a few samples, and first turns the per-warp norm partials of just those samples into
+// clip factors in shared memory (one warp per sample, the fixed-order routine above, so every
+// block gets the same bits).  The block that holds a sample's first row writes its norm2 /
+// norms_out / c_out.  The separate partials kernel is then not needed.
+constexpr long long kScaleFusedPartialSlots = 1 << 16;  // samples * count per block, at most
+constexpr int kScaleFusedMaxSamples = 4096;              // samples one block may cover
 
 __global__ void scale_rows_bf16_kernel(const __nv_bfloat16* __restrict__ in,
                                        __nv_bfloat16* __restrict__ out, long long rows, int cols,
-                                       int T, NormSource src, PartialsRef pr, int B, float C) {
-  extern __shared__ float scale_c[];  // [B] with pr.partials
+                                       int T, NormSource src, PartialsRef pr, float C) {
+  griddep_enter();
+  extern __shared__ float scale_c[];  // with pr.partials: c of samples s_lo .. s_hi
+  const int vec_per_row = cols / 8;
+  const long long total = rows * vec_per_row;
+  long long v_begin = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x;
+  long long v_end = total;
+  long long v_step = static_cast<long long>(gridDim.x) * blockDim.x;
+  int s_lo = 0;
   if (pr.partials != nullptr) {
-    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32, warps = blockDim.x / 32;
-    for (int i = warp; i < B; i += warps) {
-      const float n2 = warp_norm2_from_partials(pr.partials, pr.stride, pr.count, i, lane);
-      if (lane == 0) {
-        const float n = sqrtf(n2);
-        scale_c[i] = clip_factor(n, C);
-        if (blockIdx.x == 0) {
-          if (pr.norm2) pr.norm2[i] = n2;
-          if (pr.norms_out) pr.norms_out[i] = n;
-          if (pr.c_out) pr.c_out[i] = scale_c[i];
+    const long long per = (total + gridDim.x - 1) / gridDim.x;
+    const long long v0 = blockIdx.x * per < total ? blockIdx.x * per : total;
+    const long long v1 = v0 + per < total ? v0 + per : total;
+    const long long sample_vecs = static_cast<long long>(T) * vec_per_row;
+    if (v0 < v1) {
+      const int warp = threadIdx.x / 32, lane = threadIdx.x % 32, warps = blockDim.x / 32;
+      s_lo = static_cast<int>(v0 / sample_vecs);
+      const int s_hi = static_cast<int>((v1 - 1) / sample_vecs);
+      for (int i = s_lo + warp; i <= s_hi; i += warps) {
+        const float n2 = warp_norm2_from_partials(pr.partials, pr.stride, pr.count, i, lane);
+        if (lane == 0) {
+          const float n = sqrtf(n2);
+          const float c = clip_factor(n, C);
+          scale_c[i - s_lo] = c;
+          if (static_cast<long long>(i) * sample_vecs >= v0) {  // the sample's first row is here
+            if (pr.norm2) pr.norm2[i] = n2;
+            if (pr.norms_out) pr.norms_out[i] = n;
+            if (pr.c_out) pr.c_out[i] = c;
+          }
         }
       }
     }
     __syncthreads();
+    v_begin = v0 + threadIdx.x;
+    v_end = v1;
+    v_step = blockDim.x;
   }
-  const int vec_per_row = cols / 8;
-  const long long total = rows * vec_per_row;
-  for (long long v = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; v < total;
-       v += static_cast<long long>(gridDim.x) * blockDim.x) {
+  for (long long v = v_begin; v < v_end; v += v_step) {
     const long long row = v / vec_per_row;
     const int i = static_cast<int>(row / T);
-    const float c = pr.partials != nullptr ? scale_c[i] : clip_factor(src.norm(i), C);
+    const float c = pr.partials != nullptr ? scale_c[i - s_lo] : clip_factor(src.norm(i), C);
     const uint4 pk = reinterpret_cast<const uint4*>(in)[v];
     const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&pk);
     uint4 res;
@@ -292,6 +319,7 @@ __global__ void scale_rows_bf16_kernel(const __nv_bfloat16* __restrict__ in,
 __global__ void __launch_bounds__(256, 2) clip_reduce_kernel(
     const __nv_bfloat16* __restrict__ Gs, int B, long long mn, NormSource src, float C,
     float* __restrict__ out, double noise_std, PhiloxKey key, uint32_t layer_id, StepRef step) {
+  griddep_enter();
   const uint32_t step_lo = step.get();
   extern __shared__ double2 reduce_smem[];  // noise tables, then the cached clip factors
   float* c_smem = reinterpret_cast<float*>(reduce_smem + kNoiseSharedEntries);
@@ -362,6 +390,7 @@ __global__ void __launch_bounds__(ReduceTmaConfig<BU>::THREADS, 1) clip_reduce_t
     const __nv_bfloat16* __restrict__ Gs, long long mn, NormSource src, PartialsRef pr, float C,
     float* __restrict__ out, double noise_std, PhiloxKey key, uint32_t layer_id, StepRef step,
     uint32_t* status) {
+  griddep_enter();
   const uint32_t step_lo = step.get();
   using Cfg = ReduceTmaConfig<BU>;
   extern __shared__ uint8_t smem_raw[];
@@ -483,6 +512,7 @@ __global__ void __launch_bounds__(ReduceTmaConfig<BU>::THREADS, 1) clip_reduce_t
 __global__ void adam_rspace_kernel(const float* __restrict__ R, float* __restrict__ m, float* __restrict__ v,
                                    __nv_bfloat16* __restrict__ U, long long n, float scale, float b1, float b2,
                                    float eps, float bc1, float bc2) {
+  griddep_enter();
   for (long long q = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; 4 * q < n;
        q += static_cast<long long>(gridDim.x) * blockDim.x) {
     const float4 r4 = reinterpret_cast<const float4*>(R)[q];
@@ -514,6 +544,7 @@ __global__ void adam_rspace_kernel(const float* __restrict__ R, float* __restric
 // on an mbarrier that nothing ever arrives at.  After `limit_ns` the wait gives up, records
 // its site (code 99) in the status word and the kernel returns; the GPU stays usable.
 __global__ void wait_timeout_selftest_kernel(uint32_t* status, unsigned long long limit_ns) {
+  griddep_enter();
   __shared__ uint64_t bar;
   __shared__ int abort_flag;
   if (threadIdx.x != 0) return;
@@ -532,6 +563,7 @@ constexpr int kF32Tile = 32;
 __global__ void __launch_bounds__(256) f32_norm_kernel(const float* __restrict__ X,
                                                        const float* __restrict__ dY, int T, int m,
                                                        int n, double* __restrict__ norm2) {
+  griddep_enter();
   __shared__ float xs[kF32Tile][kF32Tile + 1];  // [t][a]
   __shared__ float ds[kF32Tile][kF32Tile + 1];  // [t][b]
   __shared__ double red[8];
@@ -574,6 +606,7 @@ __global__ void __launch_bounds__(256) f32_clipsum_kernel(
     const float* __restrict__ X, const float* __restrict__ dY, long long N, int T, int m, int n,
     NormSource src, float C, float* __restrict__ out, int add_mode, double noise_std, PhiloxKey key,
     uint32_t layer_id, StepRef step) {
+  griddep_enter();
   const uint32_t step_lo = step.get();
   __shared__ float xs[kF32Tile][kF32Tile + 1];
   __shared__ float ds[kF32Tile][kF32Tile + 1];
@@ -620,6 +653,7 @@ __global__ void __launch_bounds__(256) f32_clipsum_kernel(
 // Z[t, j] = fp32(sum_b dY[t, b] P[b, j]) in fp64, one thread per output.
 __global__ void f32_project_kernel(const float* __restrict__ dY, const float* __restrict__ P,
                                    float* __restrict__ Z, long long N, int n, int r) {
+  griddep_enter();
   const long long total = N * r;
   for (long long e = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; e < total;
        e += static_cast<long long>(gridDim.x) * blockDim.x) {

@@ -447,6 +447,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1) umma_kernel(const __grid_cons
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  griddep_wait();  // barriers and TMEM are ready; global memory only from here
   const int nphases = (Cfg::EPI == kEpiGhostNorm) ? 2 : (Cfg::EPI == kEpiGhostShared) ? 1 + p.ghost_ops : 1;
 
   if (warp == 0) {
@@ -563,6 +564,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1) umma_kernel(const __grid_cons
     }
   }
   __syncthreads();
+  griddep_launch_dependents();  // every role is done: the next kernel may take the SM
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, 512);

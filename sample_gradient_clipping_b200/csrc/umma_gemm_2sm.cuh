@@ -193,6 +193,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
   cluster_sync_all();  // both CTAs' barriers exist before any remote arrival
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  griddep_wait();  // barriers and TMEM are ready; global memory only from here
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer (both CTAs)
@@ -315,6 +316,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
   }
   __syncthreads();
   cluster_sync_all();  // no CTA leaves while its peer may still signal it or use its smem
+  griddep_launch_dependents();  // every role is done: the next kernel may take the SM
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc_pair(tmem_base, 512);
