@@ -23,7 +23,9 @@
  *     is row i*T + t.
  *   - P is [d_out, r] in dtype `dt`.  Every output is fp32.
  *   - Work is enqueued asynchronously on `stream`, a cudaStream_t passed as void*; NULL is
- *     the legacy default stream.
+ *     the legacy default stream.  Kernels are launched with programmatic dependent launch: a
+ *     kernel may be scheduled while the work before it on the stream finishes, but it touches
+ *     no memory until that work has completed, so stream order holds as for plain launches.
  *   - The library allocates no device memory.  Scratch comes from the caller's `workspace`,
  *     sized by dp_workspace_size.
  *   - Arguments are checked on the host before anything is enqueued.  On failure nothing on
