@@ -1,0 +1,55 @@
+"""Source invariants of the CUDA library that no GPU is needed to check.
+
+Every kernel is launched with programmatic stream serialization, which lets it be scheduled
+before the previous kernel on the stream has finished.  Stream order then rests on two rules:
+every launch goes through the one launch helper, and every kernel waits for its predecessor
+(griddep_wait, or griddep_enter which includes it) before touching global memory.  A kernel
+added without the wait would read or overwrite data of a kernel still running.
+"""
+import os
+import re
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+CSRC = os.path.join(ROOT, "sample_gradient_clipping_b200", "csrc")
+
+
+def _kernel_bodies():
+    """(name, body) of every __global__ function in the CUDA sources."""
+    out = []
+    for fn in sorted(os.listdir(CSRC)):
+        if not fn.endswith((".cu", ".cuh")):
+            continue
+        text = open(os.path.join(CSRC, fn)).read()
+        text = re.sub(r"//[^\n]*", "", text)
+        for m in re.finditer(r"__global__", text):
+            brace = text.index("{", m.end())
+            depth, j = 0, brace
+            while True:
+                depth += {"{": 1, "}": -1}.get(text[j], 0)
+                if depth == 0:
+                    break
+                j += 1
+            head = text[m.end():brace]
+            name = re.findall(r"([A-Za-z_][A-Za-z0-9_]*)\s*\(", head)
+            name = [n for n in name if n != "__launch_bounds__" and n != "__cluster_dims__"][0]
+            out.append((f"{fn}:{name}", text[brace + 1:j]))
+    return out
+
+
+def test_every_kernel_waits_for_its_predecessor():
+    bodies = _kernel_bodies()
+    assert len(bodies) >= 18
+    for name, body in bodies:
+        m = re.search(r"\bgriddep_(enter|wait)\(\)", body)
+        assert m, f"{name} never waits for the previous kernel"
+        before = body[:m.start()]
+        # Before the wait only kernel-local work: no pointer parameters dereferenced, no
+        # global loads or stores through the usual access forms, no device step read.
+        assert "step.get()" not in before and "__ldg" not in before and "atomic" not in before, name
+
+
+def test_every_launch_goes_through_the_helper():
+    text = open(os.path.join(CSRC, "dpclip.cu")).read()
+    text = re.sub(r"//[^\n]*", "", text)
+    assert "<<<" not in text, "a kernel is launched without programmatic stream serialization"
+    assert "cudaLaunchAttributeProgrammaticStreamSerialization" in text
