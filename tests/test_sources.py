@@ -53,3 +53,15 @@ def test_every_launch_goes_through_the_helper():
     text = re.sub(r"//[^\n]*", "", text)
     assert "<<<" not in text, "a kernel is launched without programmatic stream serialization"
     assert "cudaLaunchAttributeProgrammaticStreamSerialization" in text
+
+
+def test_noise_tables_match_their_generator():
+    """The committed Box-Muller tables are exactly what gen_noise_tables.py writes (mpmath at
+    60 digits, each value rounded once), so the transform's constants cannot drift."""
+    import importlib.util
+
+    spec = importlib.util.spec_from_file_location("gen_noise_tables", os.path.join(CSRC, "gen_noise_tables.py"))
+    gen = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(gen)
+    with open(os.path.join(CSRC, "noise_tables.cuh")) as f:
+        assert f.read() == gen.render()
