@@ -262,11 +262,14 @@ __global__ void scale_rows_bf16_kernel(const __nv_bfloat16* __restrict__ in,
   long long v_end = total;
   long long v_step = static_cast<long long>(gridDim.x) * blockDim.x;
   int s_lo = 0;
+  uint4 first = make_uint4(0u, 0u, 0u, 0u);  // fused path: this thread's first vector, loaded early
   if (pr.partials != nullptr) {
     const long long per = (total + gridDim.x - 1) / gridDim.x;
     const long long v0 = blockIdx.x * per < total ? blockIdx.x * per : total;
     const long long v1 = v0 + per < total ? v0 + per : total;
     const long long sample_vecs = static_cast<long long>(T) * vec_per_row;
+    // The load is in flight while one warp per sample sums the partials.
+    if (v0 + threadIdx.x < v1) first = reinterpret_cast<const uint4*>(in)[v0 + threadIdx.x];
     if (v0 < v1) {
       const int warp = threadIdx.x / 32, lane = threadIdx.x % 32, warps = blockDim.x / 32;
       s_lo = static_cast<int>(v0 / sample_vecs);
@@ -294,7 +297,7 @@ __global__ void scale_rows_bf16_kernel(const __nv_bfloat16* __restrict__ in,
     const long long row = v / vec_per_row;
     const int i = static_cast<int>(row / T);
     const float c = pr.partials != nullptr ? scale_c[i - s_lo] : clip_factor(src.norm(i), C);
-    const uint4 pk = reinterpret_cast<const uint4*>(in)[v];
+    const uint4 pk = (pr.partials != nullptr && v == v_begin) ? first : reinterpret_cast<const uint4*>(in)[v];
     const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&pk);
     uint4 res;
     __nv_bfloat162* o = reinterpret_cast<__nv_bfloat162*>(&res);
