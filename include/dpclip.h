@@ -61,7 +61,7 @@ extern "C" {
 typedef enum {
     DP_OK = 0,
     DP_ERR_INVALID_ARG = 1,   /* null pointer, bad shape, misalignment, C <= 0, sigma < 0 ... */
-    DP_ERR_UNSUPPORTED = 2,   /* valid request this build does not implement (e.g. fp32 ghost) */
+    DP_ERR_UNSUPPORTED = 2,   /* valid request the library does not implement (e.g. fp32 ghost) */
     DP_ERR_WORKSPACE = 3,     /* workspace smaller than dp_workspace_size() */
     DP_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed; see dp_last_cuda_error */
     DP_ERR_TIMEOUT = 5        /* a bounded in-kernel wait ran out (reported by dp_workspace_status) */
