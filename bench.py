@@ -7,6 +7,10 @@ clipped sum and the Gaussian noise of every linear.  The inputs are
 seeded synthetic tensors, resident in HBM.  They are larger than the 126 MB L2, and the 7
 linears cycle through 2.2 GB, so no L2 flush is needed between steps.
 
+The main line is the 7B block.  The Llama-13B-shaped block (B=4, T=2048) is timed after it in
+the same run, with the same steps and warm-up, and reported under "legs" with its own step
+time, roofline fractions and per-kernel split.
+
 Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
 Under torchrun every rank runs an independent replica (the step has no cross-GPU exchange).
 Rank 0 prints one JSON line.
@@ -43,6 +47,9 @@ MEASURED_TRAFFIC = {
     ("llama13b_block", "umma_explicit_store"): (676394167, "574fbf108032c9c0"),
 }
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# A timed region at least this long runs under the sustained (power-capped) clock; a shorter
+# one is compared with the burst peak.
+SUSTAINED_REGION_S = 2.0
 
 
 def parse():
@@ -66,6 +73,10 @@ def parse():
     ap.add_argument("--method", default="auto", choices=["auto", "ghost", "explicit", "once"])
     ap.add_argument("--linears", default="", help="comma-separated subset of the workload's linears")
     ap.add_argument("--sigma", type=float, default=None, help="noise multiplier (default: the workload's)")
+    ap.add_argument("--also", default="auto",
+                    help="comma-separated workloads timed after the main one in the same run and "
+                         "reported under 'legs' (default: the Llama-13B block beside the 7B one; "
+                         "'none' for none)")
     ap.add_argument("--clip", default="per_layer", choices=["per_layer", "flat"],
                     help="per-layer bounds C_l, or one flat bound sqrt(L) * C_l for the whole block")
     return ap.parse_args()
@@ -305,35 +316,30 @@ def run_reference(args, w, rank):
 
 # ---------------------------------------------------------------------------- our arm
 
-def run_ours(args, w, rank, world):
+class Prepared:
+    """Device tensors and the step function of one workload (one dp_block_step per step)."""
+
+
+def prepare(args, w, rank, world, dev, stream, shard):
     import torch
 
     from sample_gradient_clipping_b200 import _lib, inputs
 
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    _lib.lib()
-    shard = args.shard and world > 1
-    if shard and args.graph:
-        raise SystemExit("--shard runs without --graph")
+    ctx = Prepared()
     # Sharded: every rank draws its own samples (the noise seed stays the workload's).
-    data = inputs.generate(dataclasses.replace(w, seed=w.seed + 7919 * rank) if shard else w)
-    X = {k: v.to(dev) for k, v in data["X"].items()}
-    dY = {k: v.to(dev) for k, v in data["dY"].items()}
+    ctx.data = inputs.generate(dataclasses.replace(w, seed=w.seed + 7919 * rank) if shard else w)
+    ctx.X = {k: v.to(dev) for k, v in ctx.data["X"].items()}
+    ctx.dY = {k: v.to(dev) for k, v in ctx.data["dY"].items()}
     r = w.r
-    G = {l.name: torch.empty(l.d_in, r or l.d_out, dtype=torch.float32, device=dev) for l in w.linears}
-    norms = {l.name: torch.empty(w.B, dtype=torch.float32, device=dev) for l in w.linears}
-    # A graph is captured on a side stream; everything then runs on that stream.
-    stream = torch.cuda.Stream(dev) if args.graph else torch.cuda.current_stream(dev)
-    torch.cuda.set_stream(stream)
+    ctx.G = {l.name: torch.empty(l.d_in, r or l.d_out, dtype=torch.float32, device=dev) for l in w.linears}
+    ctx.norms = {l.name: torch.empty(w.B, dtype=torch.float32, device=dev) for l in w.linears}
     # The projection depends on (seed, layer) only, not on the step: it is generated once per
     # linear, as a training loop would, and passed to every step.
-    P = {l.name: _lib.dp_projection_matrix(torch.empty(l.d_out, r, dtype=X[l.x_key].dtype, device=dev),
-                                           w.seed, l.layer_id, stream=stream) for l in w.linears} if r else {}
+    ctx.P = {l.name: _lib.dp_projection_matrix(torch.empty(l.d_out, r, dtype=ctx.X[l.x_key].dtype, device=dev),
+                                               w.seed, l.layer_id, stream=stream) for l in w.linears} if r else {}
     flat_C = w.C * math.sqrt(len(w.linears))
-    block = [{"X": X[l.x_key], "dY": dY[l.name], "layer_id": l.layer_id, "C": w.C, "G_out": G[l.name],
-              "norms_out": norms[l.name], **({"P": P[l.name]} if r else {})} for l in w.linears]
+    block = [{"X": ctx.X[l.x_key], "dY": ctx.dY[l.name], "layer_id": l.layer_id, "C": w.C, "G_out": ctx.G[l.name],
+              "norms_out": ctx.norms[l.name], **({"P": ctx.P[l.name]} if r else {})} for l in w.linears]
     # One block call per step (per-layer or flat clipping; projected layers carry their P).
     if shard and r:
         raise SystemExit("--shard runs unprojected workloads")
@@ -345,9 +351,8 @@ def run_ours(args, w, rank, world):
     ws_bytes = _lib.lib().dp_block_workspace_size(arr, len(block), w.B, w.T,
                                                   _lib.DP_BF16 if w.dtype == "bf16" else _lib.DP_F32,
                                                   _lib.CLIP_MODES[args.clip], _lib.METHODS[args.method])
-    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    ctx.ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     flat_norms = torch.empty(w.B, dtype=torch.float32, device=dev)
-
     if shard:
         from sample_gradient_clipping_b200 import sharded
 
@@ -360,13 +365,26 @@ def run_ours(args, w, rank, world):
             return
         _lib.dp_block_step(block, mode=args.clip, C=flat_C if args.clip == "flat" else w.C, sigma=w.sigma,
                            seed=w.seed, step=k, method=args.method,
-                           flat_norms_out=flat_norms if args.clip == "flat" else None, workspace=ws,
+                           flat_norms_out=flat_norms if args.clip == "flat" else None, workspace=ctx.ws,
                            stream=stream)
 
+    ctx.step = step
+    return ctx
+
+
+def measure(args, w, ctx, world, dev, stream, local):
+    """Warm-up, then K timed steps (CUDA events on the launching stream, barrier and
+    synchronize on both sides), then a second pass over the same steps with an event pair
+    around every launch for the per-kernel split.  Returns the measurements of this rank."""
+    import torch
+
+    from sample_gradient_clipping_b200 import _lib
+
+    step = ctx.step
     for k in range(args.warmup):
         step(k)
     torch.cuda.synchronize(dev)
-    if _lib.dp_workspace_status(ws, stream) != _lib.DP_OK:
+    if _lib.dp_workspace_status(ctx.ws, stream) != _lib.DP_OK:
         raise RuntimeError("an in-kernel wait timed out during warm-up")
 
     graph, graph_launches = None, 0
@@ -422,30 +440,28 @@ def run_ours(args, w, rank, world):
     prof = _lib.profiling_collect()
     _lib.profiling_enable(False)
     profiled_ms = pv0.elapsed_time(pv1) / args.steps
-    if _lib.dp_workspace_status(ws, stream) != _lib.DP_OK:
+    if _lib.dp_workspace_status(ctx.ws, stream) != _lib.DP_OK:
         raise RuntimeError("an in-kernel wait timed out during the timed steps")
-    ms = max_over_ranks(ms, dev, world)
+    if graph is not None:
+        del graph
+    return {"ms": max_over_ranks(ms, dev, world), "launches": launches, "clocks": clocks, "prof": prof,
+            "profiled_ms": profiled_ms}
 
-    # ---- the non-private step of the same shapes, for FlashDP's "share of non-DP throughput"
-    non_dp = None
-    if not args.no_non_dp and r == 0 and w.dtype == "bf16":
-        non_dp = run_non_dp(args, w, X, dY, dev, stream, torch, world, ms)
 
-    # ---- end to end through the public API with host buffers
-    e2e = None
-    if not args.no_e2e and shard:
-        e2e = {"unavailable": "the end-to-end leg times the one-GPU call; run it without --shard"}
-    elif not args.no_e2e:
-        e2e = run_e2e(args, w, data, dev, stream, r, P, _lib, torch, world)
+def roofline_report(args, w, meas, world):
+    """tflops_alg, step_roofline, the dominant kernel's roofline and the per-kernel split.
 
-    if rank != 0:
-        return 0
+    A tensor-bound kernel is divided by the measured burst bf16 peak unless the timed region
+    itself lasts seconds (then the sustained, power-capped figure applies); both fractions
+    are printed, each labelled."""
     pk, pk_kind = peaks()
     flops, byts, xbytes, per_linear = workload_model(w)
+    ms = meas["ms"]
     roof_t_burst = max(flops / (pk["bf16_tflops"] * 1e12), byts / (pk["hbm_gbs"] * 1e9))
     roof_t_sust = max(flops / (pk["bf16_tflops_sustained"] * 1e12), byts / (pk["hbm_gbs"] * 1e9))
     step_s = ms / 1e3
-    kinds = {k: v for k, v in prof.items()}
+    region_s = step_s * args.steps
+    kinds = dict(meas["prof"])
     dominant = max(kinds, key=lambda k: kinds[k][0]) if kinds else None
     roofline = None
     if dominant:
@@ -463,48 +479,128 @@ def run_ours(args, w, rank, world):
         if work is not None:
             if unit == "GB/s":
                 achieved = work / (d_ms / 1e3) / 1e9
-                peak = pk["hbm_gbs"]
+                peak, peak_kind = pk["hbm_gbs"], f"{pk_kind} HBM copy bandwidth"
+                extra = {}
             else:
                 achieved = work / (d_ms / 1e3) / 1e12
-                peak = pk["bf16_tflops_sustained"]
+                long_region = region_s >= SUSTAINED_REGION_S
+                burst, sust = pk["bf16_tflops"], pk["bf16_tflops_sustained"]
+                peak = sust if long_region else burst
+                peak_kind = (f"{pk_kind} sustained bf16 (timed region {region_s:.2f} s, seconds long)" if long_region
+                             else f"{pk_kind} burst bf16 (timed region {region_s:.2f} s, under "
+                                  f"{SUSTAINED_REGION_S:g} s)")
+                extra = {"frac_of_burst": achieved / burst, "peak_burst": burst,
+                         "frac_of_sustained": achieved / sust, "peak_sustained": sust}
             roofline = {"bound": bound, "kernel": dominant, "achieved": achieved, "peak": peak,
-                        "unit": unit, "frac": achieved / peak,
+                        "unit": unit, "frac": achieved / peak, **extra,
                         "traffic": measured_traffic(w.name, dominant),
                         "traffic_unit": "bytes per launch (DRAM read + write, ncu)",
-                        "peak_kind": (f"{pk_kind} HBM copy bandwidth" if unit == "GB/s" else
-                                      f"{pk_kind} sustained bf16 (kernel timed inside a long step)"),
+                        "peak_kind": peak_kind,
                         "launches": d_n // args.steps, "avg_launch_ms": d_ms / d_n,
-                        "share_of_step": d_ms / (profiled_ms * args.steps)}
-    line = {
-        "metric": METRIC, "value": job_tokens_per_second(w.tokens, world, ms), "unit": "tokens/s",
-        "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "T": w.T, "linears": len(w.linears),
-                   "method": args.method, "clip": args.clip, "l2": "inputs larger than L2 (no flush)",
-                   "launch": ("one CUDA graph replay per step (device-resident step counter)" if args.graph
-                              else "library calls from the host every step"),
-                   "parallelism": (f"dp{world}: samples sharded, one NCCL all-reduce per linear, noise "
-                                   "added once" if shard else "replicas" if world > 1 else "1 GPU"),
-                   **({"projection": f"P [d_out, {r}] generated once per linear before timing "
-                                     "(it depends on seed and layer only)"} if r else {}),
-                   "description": w.description},
+                        "share_of_step": d_ms / (meas["profiled_ms"] * args.steps)}
+    return {
         "tflops_alg": flops * world / step_s / 1e12,
         "step_roofline": {"frac_of_burst": roof_t_burst / step_s, "frac_of_sustained": roof_t_sust / step_s,
-                          "roofline_ms_burst": roof_t_burst * 1e3, "peaks": pk_kind,
-                          "bytes_alg": byts, "bytes_alg_x_shared": xbytes, "flops_alg": flops,
+                          "roofline_ms_burst": roof_t_burst * 1e3, "roofline_ms_sustained": roof_t_sust * 1e3,
+                          "peaks": pk_kind, "bytes_alg": byts, "bytes_alg_x_shared": xbytes, "flops_alg": flops,
                           "executed_ghost_flops": ghost_flops(w)},
         "roofline": roofline,
         "kernels": {k: {"ms_per_step": v[0] / args.steps, "launches_per_step": v[1] / args.steps}
                     for k, v in sorted(kinds.items(), key=lambda kv: -kv[1][0])},
         "kernel_timing": {"how": "CUDA events around every launch, in a second pass over the same steps"
                                  + (" launched from the host (no graph)" if args.graph else ""),
-                          "ms_per_step_with_events": profiled_ms},
-        "gpu_launches": launches,
-        "clocks": clocks,
+                          "ms_per_step_with_events": meas["profiled_ms"]},
+    }
+
+
+def workload_config(args, w, world, shard):
+    return {"workload": w.name, "B": w.B, "T": w.T, "linears": len(w.linears),
+            "method": args.method, "clip": args.clip, "l2": "inputs larger than L2 (no flush)",
+            "launch": ("one CUDA graph replay per step (device-resident step counter)" if args.graph
+                       else "library calls from the host every step"),
+            "parallelism": (f"dp{world}: samples sharded, one NCCL all-reduce per linear, noise "
+                            "added once" if shard else "replicas" if world > 1 else "1 GPU"),
+            **({"projection": f"P [d_out, {w.r}] generated once per linear before timing "
+                              "(it depends on seed and layer only)"} if w.r else {}),
+            "description": w.description}
+
+
+def extra_legs(args, w, shard):
+    """Workloads timed after the main one in the same run (same steps and warm-up)."""
+    if shard or args.also == "none":
+        return []
+    if args.also == "auto":
+        return ["llama13b_block"] if w.name == "llama7b_block" else []
+    return [n for n in args.also.split(",") if n and n != w.name]
+
+
+def run_ours(args, w, rank, world):
+    import torch
+
+    from sample_gradient_clipping_b200 import _lib, inputs
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    _lib.lib()
+    shard = args.shard and world > 1
+    if shard and args.graph:
+        raise SystemExit("--shard runs without --graph")
+    # A graph is captured on a side stream; everything then runs on that stream.
+    stream = torch.cuda.Stream(dev) if args.graph else torch.cuda.current_stream(dev)
+    torch.cuda.set_stream(stream)
+    ctx = prepare(args, w, rank, world, dev, stream, shard)
+    meas = measure(args, w, ctx, world, dev, stream, local)
+    ms = meas["ms"]
+
+    # ---- the non-private step of the same shapes, for FlashDP's "share of non-DP throughput"
+    non_dp = None
+    if not args.no_non_dp and w.r == 0 and w.dtype == "bf16":
+        non_dp = run_non_dp(args, w, ctx.X, ctx.dY, dev, stream, torch, world, ms)
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e and shard:
+        e2e = {"unavailable": "the end-to-end leg times the one-GPU call; run it without --shard"}
+    elif not args.no_e2e:
+        e2e = run_e2e(args, w, ctx.data, dev, stream, w.r, ctx.P, _lib, torch, world)
+
+    data = ctx.data
+    del ctx
+    torch.cuda.empty_cache()
+
+    # ---- further workloads in the same run (the Llama-13B block beside the 7B one)
+    legs = {}
+    for name in extra_legs(args, w, shard):
+        lw = inputs.WORKLOADS[name]
+        lctx = prepare(args, lw, rank, world, dev, stream, shard)
+        lmeas = measure(args, lw, lctx, world, dev, stream, local)
+        lnon = None
+        if not args.no_non_dp and lw.r == 0 and lw.dtype == "bf16":
+            lnon = run_non_dp(args, lw, lctx.X, lctx.dY, dev, stream, torch, world, lmeas["ms"])
+        legs[name] = {"value": job_tokens_per_second(lw.tokens, world, lmeas["ms"]), "unit": "tokens/s",
+                      "ms_per_step": lmeas["ms"], "config": workload_config(args, lw, world, shard),
+                      **roofline_report(args, lw, lmeas, world), "gpu_launches": lmeas["launches"],
+                      "clocks": lmeas["clocks"], "non_dp": lnon}
+        del lctx
+        torch.cuda.empty_cache()
+
+    if rank != 0:
+        return 0
+    line = {
+        "metric": METRIC, "value": job_tokens_per_second(w.tokens, world, ms), "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": workload_config(args, w, world, shard),
+        **roofline_report(args, w, meas, world),
+        "gpu_launches": meas["launches"],
+        "clocks": meas["clocks"],
         "e2e": e2e,
         "non_dp": non_dp,
     }
+    if legs:
+        line["legs"] = legs
     if world == 1 and not args.no_cpu_baseline:
         secs, toks = oracle_block_sample(w, data, list(w.linears))
         line["cpu_baseline"] = {

@@ -64,7 +64,9 @@ typedef enum {
     DP_ERR_UNSUPPORTED = 2,   /* valid request the library does not implement (e.g. fp32 ghost) */
     DP_ERR_WORKSPACE = 3,     /* workspace smaller than dp_workspace_size() */
     DP_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed; see dp_last_cuda_error */
-    DP_ERR_TIMEOUT = 5        /* a bounded in-kernel wait ran out (reported by dp_workspace_status) */
+    DP_ERR_TIMEOUT = 5,       /* a bounded in-kernel wait ran out (reported by dp_workspace_status) */
+    DP_ERR_DEVICE_CHECK = 6   /* a device-side index check of a DPCLIP_DEBUG build failed; the access
+                                 was skipped (reported by dp_workspace_status) */
 } dp_status;
 
 typedef enum { DP_F32 = 0, DP_BF16 = 1 } dp_dtype;
@@ -204,7 +206,10 @@ dp_status dp_box_muller(const unsigned* words, long long npairs, double* z, void
  *     2 ceil(T/128) (ceil(T/128) + 1); e.g. B <= 63 for 4096 x 4096 linears.
  *   - It calls no cudaMalloc, cudaFree or other allocating routine.  The first call on each
  *     device looks up the array's device address (cudaGetSymbolAddress) with that device
- *     current.  Make that first call before any stream capture.
+ *     current.  Make that first call before any stream capture.  The address belongs to the
+ *     CUDA context it was looked up in; a call in another context (after cudaDeviceReset, or
+ *     with another driver context current) looks it up again, so make one such call before
+ *     any capture in that context too.
  *   - Every call shares the one array, and each call clears what must start at zero.  Calls
  *     that overlap on the GPU (other streams, other host threads) race on it and give wrong
  *     norms: serialise them.
@@ -298,8 +303,14 @@ dp_status dp_selftest_wait_timeout(void* workspace, unsigned long long limit_ns,
 
 /* Synchronises `stream`, then reads the status word that the kernels of earlier calls wrote
  * into `workspace`.  Returns DP_OK, DP_ERR_TIMEOUT (a bounded in-kernel wait ran out; the
- * results of that call are invalid) or DP_ERR_CUDA.  The word is cleared at the start of
- * every call that takes a workspace. */
+ * results of that call are invalid), DP_ERR_DEVICE_CHECK or DP_ERR_CUDA.  The word is cleared
+ * at the start of every call that takes a workspace.
+ * Debug build: the library compiled with -DDPCLIP_DEBUG (libdpclip_debug.so) checks, before each
+ * main-loop store or load of its kernels, that the index lies inside the buffer the host
+ * described.  A failed check never traps: it skips the access and records its site, here and
+ * in a word of the module that this call also reads (that word is never cleared), and this
+ * call then returns DP_ERR_DEVICE_CHECK with the site in dp_last_cuda_error().  In the normal
+ * build the checks compile away. */
 dp_status dp_workspace_status(const void* workspace, void* stream);
 
 /* Norm method that DP_NORM_AUTO picks for these shapes (GHOST, EXPLICIT or ONCE). */

@@ -12,8 +12,11 @@ import os
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libdpclip.so")
+# The same library built with -DDPCLIP_DEBUG: device-side index checks (see dp_workspace_status).
+DEBUG_LIB_PATH = os.path.join(PKG, "libdpclip_debug.so")
 
-DP_OK, DP_ERR_INVALID_ARG, DP_ERR_UNSUPPORTED, DP_ERR_WORKSPACE, DP_ERR_CUDA, DP_ERR_TIMEOUT = range(6)
+(DP_OK, DP_ERR_INVALID_ARG, DP_ERR_UNSUPPORTED, DP_ERR_WORKSPACE, DP_ERR_CUDA, DP_ERR_TIMEOUT,
+ DP_ERR_DEVICE_CHECK) = range(7)
 DP_F32, DP_BF16 = 0, 1
 DP_NORM_AUTO, DP_NORM_GHOST, DP_NORM_EXPLICIT, DP_NORM_ONCE = 0, 1, 2, 3
 METHODS = {"auto": DP_NORM_AUTO, "ghost": DP_NORM_GHOST, "explicit": DP_NORM_EXPLICIT,
@@ -79,23 +82,56 @@ SIGNATURES = {
 }
 
 _lib = None
+_debug_lib = None
+
+
+def load(path):
+    """A ctypes handle of the library at ``path`` with every entry point's signature set."""
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"{path} is missing: build it with "
+            "`python -m sample_gradient_clipping_b200.build` (nvcc, sm_100a)")
+    handle = ctypes.CDLL(path)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(handle, name)
+        fn.restype = res
+        fn.argtypes = args
+    return handle
 
 
 def lib():
     """The loaded library (raises if it has not been built)."""
     global _lib
     if _lib is None:
-        if not os.path.exists(LIB_PATH):
-            raise RuntimeError(
-                f"{LIB_PATH} is missing: build it with "
-                "`python -m sample_gradient_clipping_b200.build` (nvcc, sm_100a)")
-        handle = ctypes.CDLL(LIB_PATH)
-        for name, (res, args) in SIGNATURES.items():
-            fn = getattr(handle, name)
-            fn.restype = res
-            fn.argtypes = args
-        _lib = handle
+        _lib = load(LIB_PATH)
     return _lib
+
+
+def debug_lib():
+    """The checked build of the library (libdpclip_debug.so), loaded beside the normal one."""
+    global _debug_lib
+    if _debug_lib is None:
+        _debug_lib = load(DEBUG_LIB_PATH)
+    return _debug_lib
+
+
+class using:
+    """Context manager: the functions of this module call ``handle`` (e.g. debug_lib())
+    instead of the normal library while it is active."""
+
+    def __init__(self, handle):
+        self.handle = handle
+
+    def __enter__(self):
+        global _lib
+        lib()
+        self.saved, _lib = _lib, self.handle
+        return self.handle
+
+    def __exit__(self, *exc):
+        global _lib
+        _lib = self.saved
+        return False
 
 
 class DPError(RuntimeError):

@@ -11,6 +11,9 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libdpclip.so")
+# The same sources with -DDPCLIP_DEBUG: device-side index checks that record a failed check in
+# the status word and skip the access (never a trap).
+DEBUG_LIB = os.path.join(PKG, "libdpclip_debug.so")
 SOURCES = [os.path.join(CSRC, "dpclip.cu")]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
@@ -29,26 +32,29 @@ def _deps():
     return files
 
 
-def up_to_date():
-    if not os.path.exists(LIB):
+def up_to_date(path=LIB):
+    if not os.path.exists(path):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(path)
     return all(os.path.getmtime(f) <= t for f in _deps())
 
 
-def build(force=False, verbose=False, extra=()):
-    """Compile the library unless it is newer than every source; returns its path."""
-    if not force and up_to_date():
-        return LIB
+def build(force=False, verbose=False, extra=(), debug=False):
+    """Compile the library (or, with ``debug``, its checked variant) unless it is newer than
+    every source; returns its path."""
+    out = DEBUG_LIB if debug else LIB
+    if not force and up_to_date(out):
+        return out
     cmd = [_nvcc(), "-O3", "-std=c++17", *ARCH, "-lineinfo", "-Xcompiler", "-fPIC", "-shared",
-           "-I", INCLUDE, "-I", CSRC, *extra, "-o", LIB + ".tmp", *SOURCES]
+           "-I", INCLUDE, "-I", CSRC, *(["-DDPCLIP_DEBUG"] if debug else []), *extra, "-o", out + ".tmp",
+           *SOURCES]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     subprocess.run(cmd, check=True)
-    os.replace(LIB + ".tmp", LIB)
-    return LIB
+    os.replace(out + ".tmp", out)
+    return out
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose=True,
+    build(force="--force" in sys.argv, verbose=True, debug="--debug" in sys.argv,
           extra=["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else [])

@@ -16,6 +16,7 @@
 
 #include "dpclip.h"
 #include "launch_profiler.h"
+#include "nvtx_range.h"
 #include "rng.cuh"
 #include "simt.cuh"
 #include "umma_gemm.cuh"
@@ -313,7 +314,9 @@ dp_status bf16_norms(const Shape& s, const void* X, const void* Z, dp_norm_metho
   UmmaParams p = base_params(status);
   p.partials = partials;
   p.partial_stride = stride;
+  p.partials_elems = static_cast<long long>(s.B) * stride;
   const int ne = s.ne();
+  if (store) p.out_elems = static_cast<long long>(s.B) * s.m * ne;
   if (method == DP_NORM_GHOST) {
     using Cfg = UmmaConfig<128, kEpiGhostNorm>;
     dp_status st;
@@ -369,6 +372,7 @@ dp_status bf16_norms_ghost_shared(const Shape& s, const void* X, const void* con
   p.partials = partials;
   p.partial_stride = stride;
   p.partial_op_stride = op_stride;
+  p.partials_elems = (k - 1) * op_stride + static_cast<long long>(s.B) * stride;
   p.ghost_ops = k;
   const int ne = s.ne();
   dp_status st;
@@ -424,6 +428,7 @@ dp_status bf16_clipsum(const Shape& s, const void* A, const void* Bm, float* out
   p.out_rows = s.m;
   p.out_cols = ne;
   p.out_f32 = out;
+  p.out_elems = static_cast<long long>(s.m) * ne;
   if (splits > 1 || accumulate) {
     p.out_mode = (splits > 1) ? kOutAtomicAdd : kOutAdd;
     if (!accumulate)
@@ -494,6 +499,7 @@ dp_status bf16_project(const Shape& s, const void* dY, const void* P, void* Z, u
   p.out_rows = static_cast<int>(s.N());
   p.out_cols = s.r;
   p.out_bf16 = static_cast<__nv_bfloat16*>(Z);
+  p.out_elems = s.N() * s.r;
   if (s.r <= 128) {
     p.n_tiles = ceil_div(s.r, 128);
     p.num_units = p.m_tiles * p.n_tiles;
@@ -1071,20 +1077,52 @@ dp_status block_step(const dp_layer* layers, int L, dp_dtype dt, int B, int T, d
 constexpr size_t kStaticScratchBytes = size_t(1) << 20;
 static __device__ __align__(256) unsigned char g_norms_scratch[kStaticScratchBytes];
 
-// Device address of g_norms_scratch on the current device.  In host code the array's name is
-// only a host-side stand-in, so the address must come from cudaGetSymbolAddress, resolved
-// once per device with that device current.
+// Unique ID of the CUDA context current on this thread (cuCtxGetId: IDs are never reused in a
+// process, unlike context handles), or 0 when it cannot be read.
+unsigned long long current_context_id() {
+  using GetCurrent = CUresult (*)(CUcontext*);
+  using GetId = CUresult (*)(CUcontext, unsigned long long*);
+  static GetCurrent get_current = nullptr;
+  static GetId get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &fn, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<GetCurrent>(fn);
+    fn = nullptr;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &fn, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<GetId>(fn);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
+// Device address of g_norms_scratch in the current context.  In host code the array's name is
+// only a host-side stand-in, so the address must come from cudaGetSymbolAddress, resolved with
+// the device current.  It is looked up once per device and context: a device reset, or another
+// context made current, gives a new context ID, and the address is looked up again (the module,
+// and so the array, is loaded anew in every context).  Without a readable context ID it is
+// looked up on every call.
 dp_status static_scratch(unsigned char** out) {
   static std::mutex mu;
   static unsigned char* addr[64] = {nullptr};
+  static unsigned long long ctx_id[64] = {0};
   int dev = 0;
   DP_CUDA(cudaGetDevice(&dev));
   if (dev < 0 || dev >= 64) return DP_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> g(mu);
-  if (!addr[dev]) {
+  const unsigned long long id = current_context_id();
+  if (!addr[dev] || id == 0 || id != ctx_id[dev]) {
     void* p = nullptr;
     DP_CUDA(cudaGetSymbolAddress(&p, g_norms_scratch));
     addr[dev] = static_cast<unsigned char*>(p);
+    ctx_id[dev] = current_context_id();  // the lookup makes the primary context current if none was
   }
   *out = addr[dev];
   return DP_OK;
@@ -1119,6 +1157,7 @@ dp_norm_method dp_auto_norm_method(int B, int T, int d_in, int d_out, int r, dp_
 dp_status dp_per_sample_norms(const void* X, const void* dY, const void* P, int r, dp_dtype dt, int B,
                               int T, int d_in, int d_out, dp_norm_method method, float* norms,
                               void* workspace, size_t ws_bytes, void* stream) {
+  DP_NVTX_RANGE();
   Call c;
   dp_status st = check_common(X, dY, P, r, dt, B, T, d_in, d_out, workspace, ws_bytes, false,
                               DP_NORM_GHOST, &c);
@@ -1140,6 +1179,7 @@ dp_status dp_per_sample_norms(const void* X, const void* dY, const void* P, int 
 dp_status dp_clip_accumulate(const void* X, const void* dY, const void* P, int r, dp_dtype dt, int B,
                              int T, int d_in, int d_out, const float* norms, float C, float* G_sum,
                              void* workspace, size_t ws_bytes, void* stream) {
+  DP_NVTX_RANGE();
   Call c;
   dp_status st = check_common(X, dY, P, r, dt, B, T, d_in, d_out, workspace, ws_bytes, false,
                               DP_NORM_GHOST, &c);
@@ -1157,6 +1197,7 @@ dp_status dp_clip_accumulate(const void* X, const void* dY, const void* P, int r
 
 dp_status dp_add_noise(float* G, long long rows, long long cols, float std, unsigned long long seed,
                        unsigned long long step, unsigned layer_id, void* stream) {
+  DP_NVTX_RANGE();
   if (!G || !aligned16(G) || rows < 1 || cols < 1) return DP_ERR_INVALID_ARG;
   if (!(std >= 0.0f) || std::isinf(std)) return DP_ERR_INVALID_ARG;
   if (rows > (1ll << 34) / cols) return DP_ERR_INVALID_ARG;
@@ -1168,6 +1209,7 @@ dp_status dp_add_noise(float* G, long long rows, long long cols, float std, unsi
 
 dp_status dp_projection_matrix(void* P, dp_dtype dt, int d_out, int r, unsigned long long seed,
                                unsigned layer_id, void* stream) {
+  DP_NVTX_RANGE();
   if (!P || !aligned16(P) || !valid_dtype(dt) || d_out < 1 || r < 1) return DP_ERR_INVALID_ARG;
   const int q = (dt == DP_BF16) ? 8 : 4;
   if (d_out % q || r % q) return DP_ERR_INVALID_ARG;
@@ -1232,6 +1274,7 @@ dp_status dp_linear_step(const void* X, const void* dY, const void* P, int r, dp
                          int d_in, int d_out, float C, float sigma, unsigned long long seed,
                          unsigned long long step, unsigned layer_id, dp_norm_method method,
                          float* norms_out, float* G_out, void* workspace, size_t ws_bytes, void* stream) {
+  DP_NVTX_RANGE();
   return linear_step(X, dY, P, r, dt, B, T, d_in, d_out, C, sigma, seed, step_value(step), layer_id, method,
                      norms_out, G_out, workspace, ws_bytes, stream);
 }
@@ -1241,6 +1284,7 @@ dp_status dp_linear_step_dev_step(const void* X, const void* dY, const void* P, 
                                   const unsigned long long* step_dev, unsigned layer_id, dp_norm_method method,
                                   float* norms_out, float* G_out, void* workspace, size_t ws_bytes,
                                   void* stream) {
+  DP_NVTX_RANGE();
   if (!step_dev || (reinterpret_cast<uintptr_t>(step_dev) & 7u) != 0) return DP_ERR_INVALID_ARG;
   return linear_step(X, dY, P, r, dt, B, T, d_in, d_out, C, sigma, seed, StepRef{0u, step_dev}, layer_id,
                      method, norms_out, G_out, workspace, ws_bytes, stream);
@@ -1249,6 +1293,7 @@ dp_status dp_linear_step_dev_step(const void* X, const void* dY, const void* P, 
 dp_status dp_philox_blocks(unsigned* out, unsigned long long nblocks, unsigned long long seed,
                            unsigned long long step, unsigned layer_id, unsigned stream_id,
                            void* stream) {
+  DP_NVTX_RANGE();
   if (!out || !aligned16(out) || nblocks < 1 || nblocks > (1ull << 32)) return DP_ERR_INVALID_ARG;
   LaunchScope scope(kKindPhilox, static_cast<cudaStream_t>(stream));
   DP_LAUNCH("philox_blocks_kernel", philox_blocks_kernel, stream_grid(nblocks, 256), 256, 0,
@@ -1258,6 +1303,7 @@ dp_status dp_philox_blocks(unsigned* out, unsigned long long nblocks, unsigned l
 }
 
 dp_status dp_box_muller(const unsigned* words, long long npairs, double* z, void* stream) {
+  DP_NVTX_RANGE();
   if (!words || !z || !aligned16(words) || !aligned16(z) || npairs < 1 || npairs > (1ll << 40))
     return DP_ERR_INVALID_ARG;
   LaunchScope scope(kKindNoise, static_cast<cudaStream_t>(stream));
@@ -1271,6 +1317,7 @@ dp_status dp_box_muller(const unsigned* words, long long npairs, double* z, void
 dp_status dp_per_sample_norms_static(const void* X, const void* dY, dp_dtype dt, int B, int T,
                                      int d_in, int d_out, dp_norm_method method, float* norms,
                                      void* stream) {
+  DP_NVTX_RANGE();
   if (!X || !dY || !norms || !aligned16(X) || !aligned16(dY)) return DP_ERR_INVALID_ARG;
   const Shape s{B, T, d_in, d_out, 0, dt};
   if (!valid_shape(s)) return DP_ERR_INVALID_ARG;
@@ -1357,6 +1404,7 @@ dp_status dp_block_step(const dp_layer* layers, int L, dp_dtype dt, int B, int T
                         float C, float sigma, unsigned long long seed, unsigned long long step,
                         dp_norm_method method, float* flat_norms_out, void* workspace, size_t ws_bytes,
                         void* stream) {
+  DP_NVTX_RANGE();
   return block_step_entry(layers, L, dt, B, T, mode, C, sigma, seed, step_value(step), method, flat_norms_out,
                           workspace, ws_bytes, stream);
 }
@@ -1365,6 +1413,7 @@ dp_status dp_block_step_dev_step(const dp_layer* layers, int L, dp_dtype dt, int
                                  float C, float sigma, unsigned long long seed,
                                  const unsigned long long* step_dev, dp_norm_method method,
                                  float* flat_norms_out, void* workspace, size_t ws_bytes, void* stream) {
+  DP_NVTX_RANGE();
   if (!step_dev || (reinterpret_cast<uintptr_t>(step_dev) & 7u) != 0) return DP_ERR_INVALID_ARG;
   return block_step_entry(layers, L, dt, B, T, mode, C, sigma, seed, StepRef{0u, step_dev}, method,
                           flat_norms_out, workspace, ws_bytes, stream);
@@ -1378,6 +1427,7 @@ size_t dp_adam_workspace_size(int d_in, int r) {
 dp_status dp_projected_adam_step(float* W, const float* R, float* m, float* v, const void* P, dp_dtype dt,
                                  int d_in, int d_out, int r, float lr, float beta1, float beta2, float eps,
                                  float grad_scale, int t, void* workspace, size_t ws_bytes, void* stream) {
+  DP_NVTX_RANGE();
   if (!W || !R || !m || !v || !P || !workspace) return DP_ERR_INVALID_ARG;
   if (!aligned16(W) || !aligned16(R) || !aligned16(m) || !aligned16(v) || !aligned16(P)) return DP_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return DP_ERR_INVALID_ARG;
@@ -1417,11 +1467,13 @@ dp_status dp_projected_adam_step(float* W, const float* R, float* m, float* v, c
   p.out_rows = d_in;
   p.out_cols = d_out;
   p.out_f32 = W;
+  p.out_elems = static_cast<long long>(d_in) * d_out;
   p.alpha = -lr;
   return launch_umma<UmmaConfig<256, kEpiAxpy>>(p, cs);
 }
 
 dp_status dp_selftest_wait_timeout(void* workspace, unsigned long long limit_ns, void* stream) {
+  DP_NVTX_RANGE();
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return DP_ERR_INVALID_ARG;
   if (limit_ns < 1000ull || limit_ns > kWaitLimitNs) return DP_ERR_INVALID_ARG;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
@@ -1432,10 +1484,24 @@ dp_status dp_selftest_wait_timeout(void* workspace, unsigned long long limit_ns,
 }
 
 dp_status dp_workspace_status(const void* workspace, void* stream) {
+  DP_NVTX_RANGE();
   if (!workspace) return DP_ERR_INVALID_ARG;
   DP_CUDA(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
   uint32_t word = 0;
   DP_CUDA(cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost));
+#ifdef DPCLIP_DEBUG
+  // Checks of kernels without a workspace status word land in the module's debug word only.
+  uint32_t dbg = 0;
+  DP_CUDA(cudaMemcpyFromSymbol(&dbg, g_debug_word, sizeof(dbg)));
+  if (dbg >= kDebugCheckBase) {
+    snprintf(g_cuda_error, sizeof(g_cuda_error), "device-side check %u failed", dbg - kDebugCheckBase);
+    return DP_ERR_DEVICE_CHECK;
+  }
+#endif
+  if (word >= kDebugCheckBase) {
+    snprintf(g_cuda_error, sizeof(g_cuda_error), "device-side check %u failed", word - kDebugCheckBase);
+    return DP_ERR_DEVICE_CHECK;
+  }
   return word ? DP_ERR_TIMEOUT : DP_OK;
 }
 
@@ -1447,6 +1513,7 @@ const char* dp_status_string(dp_status s) {
     case DP_ERR_WORKSPACE: return "workspace too small";
     case DP_ERR_CUDA: return "CUDA error";
     case DP_ERR_TIMEOUT: return "in-kernel wait timed out";
+    case DP_ERR_DEVICE_CHECK: return "device-side check failed (debug build)";
   }
   return "unknown status";
 }

@@ -28,6 +28,38 @@ __device__ __forceinline__ uint32_t lane_id() {
   return l;
 }
 
+// ---------------------------------------------------------------- device-side checks (debug build)
+// A build with -DDPCLIP_DEBUG checks, before each store or load of a kernel's main loops, that
+// its index lies inside the buffer the host described.  A failed check never traps: it records
+// kDebugCheckBase + site in g_debug_word (and in the workspace status word when the kernel has
+// one), and the access is skipped.  dp_workspace_status reports it as DP_ERR_DEVICE_CHECK.  In
+// the normal build DP_DCHECK is the constant true and the checks compile away.
+constexpr uint32_t kDebugCheckBase = 1000u;
+#ifdef DPCLIP_DEBUG
+__device__ uint32_t g_debug_word;
+__device__ __forceinline__ bool debug_check(bool ok, uint32_t site, uint32_t* status) {
+  if (!ok) {
+    atomicCAS(&g_debug_word, 0u, kDebugCheckBase + site);
+    if (status) atomicCAS(status, 0u, kDebugCheckBase + site);
+  }
+  return ok;
+}
+#define DP_DCHECK(cond, site, status) ::dpclip::debug_check((cond), (site), (status))
+#else
+#define DP_DCHECK(cond, site, status) true
+#endif
+// An index range [first, first + count) inside a buffer of `size` elements; size 0 = unknown.
+__host__ __device__ __forceinline__ bool in_buffer(long long first, long long count, long long size) {
+  return size == 0 || (first >= 0 && first + count <= size);
+}
+
+// Bytes of dynamic shared memory this block was launched with.
+__device__ __forceinline__ uint32_t dynamic_smem_bytes() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %dynamic_smem_size;" : "=r"(r));
+  return r;
+}
+
 // ---------------------------------------------------------------- programmatic dependent launch
 // Every kernel of the library is launched so that it may start while the previous kernel in
 // its stream drains.  griddep_wait() returns once every kernel this one depends on in stream

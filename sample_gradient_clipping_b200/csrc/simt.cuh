@@ -40,6 +40,7 @@ __global__ void noise_add_kernel(float* __restrict__ G, unsigned long long total
     normals4(static_cast<uint32_t>(j), layer_id, step_lo, kStreamNoise, key, z, tab, std_dev);
     const unsigned long long k0 = 4 * j;
     if (k0 + 3 < total) {
+      if (!DP_DCHECK(in_buffer(static_cast<long long>(k0), 4, static_cast<long long>(total)), 20u, nullptr)) continue;
       float4* p = reinterpret_cast<float4*>(G + k0);
       float4 g = *p;
       g.x = static_cast<float>(static_cast<double>(g.x) + z[0]);
@@ -179,6 +180,7 @@ struct NormSource {
 // from them are reproducible bit for bit.  Every lane returns the same value.
 __device__ __forceinline__ float warp_norm2_from_partials(const float* __restrict__ partials, int stride,
                                                           int count, int i, int lane) {
+  if (!DP_DCHECK(count <= stride && i >= 0, 26u, nullptr)) return 0.0f;
   double acc = 0.0;
   for (int k = lane; k < count; k += 32) acc += static_cast<double>(partials[static_cast<long long>(i) * stride + k]);
 #pragma unroll
@@ -296,6 +298,10 @@ __global__ void scale_rows_bf16_kernel(const __nv_bfloat16* __restrict__ in,
   for (long long v = v_begin; v < v_end; v += v_step) {
     const long long row = v / vec_per_row;
     const int i = static_cast<int>(row / T);
+    if (pr.partials != nullptr &&
+        !DP_DCHECK(i >= s_lo && (i - s_lo + 1) * sizeof(float) <= dynamic_smem_bytes(), 21u, nullptr))
+      break;
+    if (!DP_DCHECK(v >= 0 && v < total, 22u, nullptr)) break;
     const float c = pr.partials != nullptr ? scale_c[i - s_lo] : clip_factor(src.norm(i), C);
     const uint4 pk = (pr.partials != nullptr && v == v_begin) ? first : reinterpret_cast<const uint4*>(in)[v];
     const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&pk);
@@ -358,6 +364,7 @@ __global__ void __launch_bounds__(256, 2) clip_reduce_kernel(
 #pragma unroll
       for (int q = 0; q < 8; ++q) acc[q] = acc[q] + __double2float_rn(z[q]);
     }
+    if (!DP_DCHECK(in_buffer(8 * v, 8, mn), 23u, nullptr)) break;
     float4* o = reinterpret_cast<float4*>(out) + 2 * v;
     o[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
     o[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
@@ -429,11 +436,15 @@ __global__ void __launch_bounds__(ReduceTmaConfig<BU>::THREADS, 1) clip_reduce_t
         const long long n = (mn - e0) < kReduceChunk ? (mn - e0) : kReduceChunk;  // multiple of 8
         const uint32_t bytes = static_cast<uint32_t>(n * 2);
         const uint32_t bar = smem_addr(full + stage);
-        mbar_arrive_expect_tx(bar, BU * bytes);
-        const uint32_t dst = smem_addr(smem + stage * Cfg::STAGE_BYTES);
+        if (DP_DCHECK(n > 0 && n % 8 == 0 && in_buffer((BU - 1) * mn + e0, n, BU * mn), 24u, status)) {
+          mbar_arrive_expect_tx(bar, BU * bytes);
+          const uint32_t dst = smem_addr(smem + stage * Cfg::STAGE_BYTES);
 #pragma unroll
-        for (int i = 0; i < BU; ++i)
-          bulk_load(dst + i * kReduceChunk * 2, Gs + static_cast<long long>(i) * mn + e0, bytes, bar);
+          for (int i = 0; i < BU; ++i)
+            bulk_load(dst + i * kReduceChunk * 2, Gs + static_cast<long long>(i) * mn + e0, bytes, bar);
+        } else {
+          mbar_arrive(bar);  // no copy: the stage completes empty, nothing is left in flight
+        }
         if (++stage == Cfg::STAGES) {
           stage = 0;
           phase ^= 1u;
@@ -494,9 +505,11 @@ __global__ void __launch_bounds__(ReduceTmaConfig<BU>::THREADS, 1) clip_reduce_t
 #pragma unroll
           for (int q = 0; q < 8; ++q) acc[q] = acc[q] + __double2float_rn(z[q]);
         }
-        float4* o = reinterpret_cast<float4*>(out + e);
-        o[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-        o[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+        if (DP_DCHECK(in_buffer(e, 8, mn), 25u, status)) {
+          float4* o = reinterpret_cast<float4*>(out + e);
+          o[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+          o[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+        }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_addr(empty + stage));

@@ -80,6 +80,8 @@ struct alignas(64) UmmaParams {
   int ghost_ops;              // shared ghost: dY operands (1..3); phase 1 + k reads operand k
   long long partial_op_stride;  // shared ghost: floats between the operands' partial arrays
   uint32_t* status;
+  long long out_elems;        // elements of the output buffer (device-side checks; 0 = unknown)
+  long long partials_elems;   // floats of the partials buffer (device-side checks; 0 = unknown)
 };
 
 template <int BN_, int EPI_>
@@ -260,6 +262,7 @@ __device__ __forceinline__ void epilogue_unit(const UmmaParams& p, const Unit& w
           val.z = static_cast<float>(static_cast<double>(val.z) + p.noise_std * z[2]);
           val.w = static_cast<float>(static_cast<double>(val.w) + p.noise_std * z[3]);
         }
+        if (!DP_DCHECK(in_buffer(grow * p.out_cols + gcol0 + 4 * q, 4, p.out_elems), 1u, p.status)) break;
         float4* d4 = reinterpret_cast<float4*>(dst + 4 * q);
         if (p.out_mode == kOutStore) {
           *d4 = val;
@@ -295,12 +298,18 @@ __device__ __forceinline__ void epilogue_unit(const UmmaParams& p, const Unit& w
           __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&pk);
 #pragma unroll
           for (int e = 0; e < 4; ++e) h[e] = __floats2bfloat162_rn(v[8 * q + 2 * e], v[8 * q + 2 * e + 1]);
+          if (!DP_DCHECK(in_buffer((static_cast<long long>(w.sample) * p.out_rows + grow) * p.out_cols + gcol0 + 8 * q,
+                                   8, p.out_elems), 2u, p.status))
+            break;
           *reinterpret_cast<uint4*>(dst + 8 * q) = pk;
         }
       }
     }
     ss = warp_sum(ss);
-    if (lane == 0) p.partials[static_cast<long long>(w.sample) * p.partial_stride + 4 * w.local + wq] = ss;
+    const long long slot = static_cast<long long>(w.sample) * p.partial_stride + 4 * w.local + wq;
+    if (lane == 0 && DP_DCHECK(4 * w.local + wq < p.partial_stride && in_buffer(slot, 1, p.partials_elems), 3u,
+                               p.status))
+      p.partials[slot] = ss;
   } else if (Cfg::EPI == kEpiGhostNorm) {
     // Rows and columns past T were zero-filled by TMA, so their Gram entries are 0.
     const int t = w.m_blk * Cfg::BM + row;
@@ -320,7 +329,10 @@ __device__ __forceinline__ void epilogue_unit(const UmmaParams& p, const Unit& w
       }
     }
     ss = warp_sum(ss);
-    if (lane == 0) p.partials[static_cast<long long>(w.sample) * p.partial_stride + 4 * w.local + wq] = ss;
+    const long long slot = static_cast<long long>(w.sample) * p.partial_stride + 4 * w.local + wq;
+    if (lane == 0 && DP_DCHECK(4 * w.local + wq < p.partial_stride && in_buffer(slot, 1, p.partials_elems), 4u,
+                               p.status))
+      p.partials[slot] = ss;
   } else if (Cfg::EPI == kEpiGhostShared) {
     const int t = w.m_blk * Cfg::BM + row;
     float ss[kGhostSharedMaxOps] = {0.f, 0.f, 0.f};
@@ -350,9 +362,11 @@ __device__ __forceinline__ void epilogue_unit(const UmmaParams& p, const Unit& w
     for (int op = 0; op < kGhostSharedMaxOps; ++op) {
       if (op < p.ghost_ops) {
         const float v = warp_sum(ss[op]);
-        if (lane == 0)
-          p.partials[op * p.partial_op_stride + static_cast<long long>(w.sample) * p.partial_stride +
-                     4 * w.local + wq] = v;
+        const long long slot = op * p.partial_op_stride + static_cast<long long>(w.sample) * p.partial_stride +
+                               4 * w.local + wq;
+        if (lane == 0 && DP_DCHECK(4 * w.local + wq < p.partial_stride && in_buffer(slot, 1, p.partials_elems), 5u,
+                                   p.status))
+          p.partials[slot] = v;
       }
     }
   } else if (Cfg::EPI == kEpiAxpy) {
@@ -370,6 +384,7 @@ __device__ __forceinline__ void epilogue_unit(const UmmaParams& p, const Unit& w
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
         if (gcol0 + 4 * q >= p.out_cols) break;  // out_cols is a multiple of 4
+        if (!DP_DCHECK(in_buffer(grow * p.out_cols + gcol0 + 4 * q, 4, p.out_elems), 6u, p.status)) break;
         float4* d4 = reinterpret_cast<float4*>(dst + 4 * q);
         float4 o = *d4;
         o.x = fmaf(p.alpha, v[4 * q], o.x);
@@ -397,6 +412,7 @@ __device__ __forceinline__ void epilogue_unit(const UmmaParams& p, const Unit& w
         __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&pk);
 #pragma unroll
         for (int e = 0; e < 4; ++e) h[e] = __floats2bfloat162_rn(v[8 * q + 2 * e], v[8 * q + 2 * e + 1]);
+        if (!DP_DCHECK(in_buffer(grow * p.out_cols + gcol0 + 8 * q, 8, p.out_elems), 7u, p.status)) break;
         *reinterpret_cast<uint4*>(dst + 8 * q) = pk;
       }
     }

@@ -40,10 +40,32 @@ def check_clip_decisions(norms_gpu, norms_oracle, C):
         assert (ng > C) == (no > C), f"clip decision of sample {i}: gpu {ng} oracle {no} C {C}"
 
 
+def rounding_allowance(out_a, out_b):
+    """fp32 rounding of the two outputs whose difference is compared with the noise: at most
+    half an ulp of each, written as two ulps of the larger magnitude."""
+    mag = np.maximum(np.abs(out_a), np.abs(out_b))
+    return 2.0 * np.spacing(mag.astype(np.float32)).astype(np.float64)
+
+
 def noise_tolerance(out_a, out_b):
     """1e-6 plus the fp32 rounding of adding the noise to values of this magnitude."""
-    mag = np.maximum(np.abs(out_a), np.abs(out_b))
-    return NOISE_ABS + 2.0 * np.spacing(mag.astype(np.float32)).astype(np.float64)
+    return NOISE_ABS + rounding_allowance(out_a, out_b)
+
+
+def noise_excess(out_a, out_b, want):
+    """Largest error of (out_a - out_b) against the exact noise beyond the fp32 rounding
+    allowance: the figure that the 1e-6 bound applies to."""
+    err = np.abs((np.asarray(out_a, np.float64) - np.asarray(out_b, np.float64)) - want)
+    return float(np.max(err - rounding_allowance(out_a, out_b))) if err.size else 0.0
+
+
+# Measured parity errors of this session, (test, item, quantity, value, bound); the summary
+# hook in conftest.py prints them so that each run records how close it came to each bound.
+MARGINS = []
+
+
+def record(test, item, quantity, value, bound):
+    MARGINS.append((test, str(item), quantity, float(value), float(bound)))
 
 
 def draw(w, linears=None, device="cuda"):

@@ -33,9 +33,19 @@ def test_exports_every_declared_symbol(L):
 
 
 def test_status_strings(L):
-    for code in range(6):
-        assert L.dp_status_string(code)
+    for code in range(7):
+        assert L.dp_status_string(code) and L.dp_status_string(code) != b"unknown status"
     assert L.dp_status_string(0) == b"ok"
+
+
+def test_debug_build_compiles_and_exports_every_symbol():
+    """The checked variant (-DDPCLIP_DEBUG) builds from the same sources and exports the same
+    entry points; its device-side checks are exercised by the GPU tests."""
+    path = build.build(debug=True)
+    D = _lib.load(path)
+    for name in declared_functions():
+        assert hasattr(D, name), name
+    assert D.dp_status_string(_lib.DP_ERR_DEVICE_CHECK) == b"device-side check failed (debug build)"
 
 
 def test_workspace_size(L):

@@ -3,9 +3,9 @@
 dp_per_sample_norms_static serves callers that cannot allocate device memory: code inside
 another framework's allocator hook, or a real-time loop that forbids allocations after
 start-up.  Its scratch is a fixed device array inside the library instead of a caller
-workspace.  These tests call it through the C ABI and check that its norms equal those of
-dp_per_sample_norms, within the parity tolerance, on consecutive calls.  The calls use
-different shapes and methods, so stale contents of the shared array would show up.
+workspace.  These tests call it through the C ABI and check its norms, on consecutive calls, against
+those of dp_per_sample_norms and against the fp64 oracle, within the parity tolerance.  The
+calls use different shapes and methods, so stale contents of the shared array would show up.
 
 This file is collected last on purpose: a run that stops at the first failure has then
 already run every other test.
@@ -15,8 +15,9 @@ from __future__ import annotations
 import pytest
 import torch
 
+import oracle
 from sample_gradient_clipping_b200 import _lib, inputs
-from tests.gpu_helpers import TOL, host, rel_max
+from tests.gpu_helpers import TOL, host, record, rel_max
 
 pytestmark = pytest.mark.gpu
 
@@ -28,10 +29,11 @@ def _cuda():
     _lib.lib()
 
 
-def _draw(B, T, m, n, dtype, seed):
+def _draw(B, T, m, n, dtype, seed, with_host=False):
     w = inputs.custom("static", B=B, T=T, d_in=m, d_out=n, dtype=dtype, seed=seed)
     d = inputs.generate(w)
-    return d["X"]["in"].cuda(), d["dY"]["linear"].cuda()
+    dev = d["X"]["in"].cuda(), d["dY"]["linear"].cuda()
+    return (dev, (d["X"]["in"], d["dY"]["linear"])) if with_host else dev
 
 
 def _static_norms(X, dY, method):
@@ -58,10 +60,14 @@ CALLS = [  # consecutive calls: shapes and methods change between them
 
 def test_static_scratch_norms_match_workspace_norms_on_consecutive_calls():
     for k, (shape, dtype, method) in enumerate(CALLS):
-        X, dY = _draw(*shape, dtype, seed=50 + k)
+        (X, dY), (Xh, dYh) = _draw(*shape, dtype, seed=50 + k, with_host=True)
         want = host(_lib.dp_per_sample_norms(X, dY, method=method))
         got = host(_static_norms(X, dY, method))
         assert rel_max(got, want) <= TOL[dtype]["norm"], (k, shape, method, got, want)
+        exact = oracle.per_sample_norms(inputs.as_f64(Xh), inputs.as_f64(dYh))
+        err = rel_max(got, exact)
+        record("static-scratch norms", f"call {k} {shape} {method}", "norm", err, TOL[dtype]["norm"])
+        assert err <= TOL[dtype]["norm"], (k, shape, method, got, exact)
 
 
 def test_static_scratch_refuses_shapes_beyond_its_size():
