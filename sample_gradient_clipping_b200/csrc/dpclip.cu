@@ -500,6 +500,14 @@ dp_status bf16_project(const Shape& s, const void* dY, const void* P, void* Z, u
   p.out_cols = s.r;
   p.out_bf16 = static_cast<__nv_bfloat16*>(Z);
   p.out_elems = s.N() * s.r;
+  if (s.r <= 64 || (s.r <= 128 && p.m_tiles * 2 <= sm_count())) {
+    // 128 x 64 tiles when 128 x 128 tiles would leave more than half the SMs idle (e.g.
+    // N = 8192 tokens, r = 128: 64 tiles; 128 with this split).  The two CTAs of a row block
+    // read the same dY tile at about the same time, so the second read comes from L2.
+    p.n_tiles = ceil_div(s.r, 64);
+    p.num_units = p.m_tiles * p.n_tiles;
+    return launch_umma<UmmaConfig<64, kEpiStoreBf16>>(p, stream);
+  }
   if (s.r <= 128) {
     p.n_tiles = ceil_div(s.r, 128);
     p.num_units = p.m_tiles * p.n_tiles;
@@ -574,11 +582,14 @@ dp_status launch_finalize(NormSource src, int B, float C, float* norms_out, floa
   return DP_OK;
 }
 
+// Precision of the Box-Muller evaluation in the gradients-once reduce.
+constexpr int kReduceNoise = kGradientNoise;
+
 dp_status reduce_kernel_launch(int grid, size_t smem, cudaStream_t stream, const __nv_bfloat16* gs, int B,
                           long long mn, NormSource src, float C, float* out, double noise_std, PhiloxKey key,
                           unsigned layer_id, StepRef step) {
-  DP_LAUNCH("clip_reduce_kernel", clip_reduce_kernel, grid, 256, smem, stream, gs, B, mn, src, C, out,
-            noise_std, key, layer_id, step);
+  DP_LAUNCH("clip_reduce_kernel", clip_reduce_kernel<kReduceNoise>, grid, 256, smem, stream, gs, B, mn, src, C,
+            out, noise_std, key, layer_id, step);
   return DP_OK;
 }
 
@@ -591,14 +602,14 @@ dp_status reduce_tma_launch(cudaStream_t stream, const __nv_bfloat16* gs, long l
   int dev = 0;
   DP_CUDA(cudaGetDevice(&dev));
   if (dev >= 0 && dev < 64 && !configured[dev]) {
-    DP_CUDA(cudaFuncSetAttribute(clip_reduce_tma_kernel<BU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 Cfg::SMEM_BYTES));
+    DP_CUDA(cudaFuncSetAttribute(clip_reduce_tma_kernel<BU, kReduceNoise>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES));
     configured[dev] = true;
   }
   const long long chunks = (mn + kReduceChunk - 1) / kReduceChunk;
   const int grid = static_cast<int>(chunks < sm_count() ? chunks : sm_count());
-  DP_LAUNCH("clip_reduce_tma_kernel", clip_reduce_tma_kernel<BU>, grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream,
-            gs, mn, src, pr, C, out, noise_std, key, layer_id, step, status);
+  DP_LAUNCH("clip_reduce_tma_kernel", clip_reduce_tma_kernel<BU, kReduceNoise>, grid, Cfg::THREADS,
+            Cfg::SMEM_BYTES, stream, gs, mn, src, pr, C, out, noise_std, key, layer_id, step, status);
   return DP_OK;
 }
 

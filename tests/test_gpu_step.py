@@ -215,6 +215,17 @@ def test_given_projection_equals_seeded_projection():
     check_linear(w, lin, data, dev)
 
 
+@pytest.mark.parametrize("B,T,r", [(64, 128, 128),    # 64 row tiles: 128 x 64 projection tiles
+                                   (80, 128, 128),    # 80 row tiles: 128 x 128 tiles
+                                   (3, 100, 256),     # r > 128: 128 x 256 tiles, ragged N
+                                   (5, 72, 40)])      # r < 64: one 64-wide tile, ragged
+def test_projection_tile_shapes(B, T, r):
+    """Every tile shape of the projection GEMM Z = dY P, checked through the projected step."""
+    w = inputs.custom("ptile", B=B, T=T, d_in=256, d_out=512, r=r, C=0.3, sigma=0.9, seed=41)
+    data, dev = draw(w)
+    check_linear(w, w.linears[0], data, dev, method="ghost")
+
+
 def test_norms_entry_matches_step_norms():
     w, lin, data, dev = _custom(4, 160, 264, 520, C=0.5, sigma=0.0, seed=37)
     X, dY = dev["X"]["in"], dev["dY"]["linear"]
