@@ -7,6 +7,7 @@
 
 #include <algorithm>
 #include <cmath>
+#include <cstdlib>
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
@@ -587,9 +588,13 @@ constexpr int kReduceNoise = kGradientNoise;
 
 dp_status reduce_kernel_launch(int grid, size_t smem, cudaStream_t stream, const __nv_bfloat16* gs, int B,
                           long long mn, NormSource src, float C, float* out, double noise_std, PhiloxKey key,
-                          unsigned layer_id, StepRef step) {
-  DP_LAUNCH("clip_reduce_kernel", clip_reduce_kernel<kReduceNoise>, grid, 256, smem, stream, gs, B, mn, src, C,
-            out, noise_std, key, layer_id, step);
+                          unsigned layer_id, StepRef step, bool staged) {
+  if (staged)
+    DP_LAUNCH("clip_reduce_kernel", clip_reduce_kernel<kReduceNoise, true>, grid, 256, smem, stream, gs, B, mn,
+              src, C, out, noise_std, key, layer_id, step);
+  else
+    DP_LAUNCH("clip_reduce_kernel", clip_reduce_kernel<kReduceNoise, false>, grid, 256, smem, stream, gs, B, mn,
+              src, C, out, noise_std, key, layer_id, step);
   return DP_OK;
 }
 
@@ -616,11 +621,14 @@ dp_status reduce_tma_launch(cudaStream_t stream, const __nv_bfloat16* gs, long l
 dp_status launch_reduce(const __nv_bfloat16* gs, int B, long long mn, NormSource src, float C,
                         float* out, double noise_std, unsigned long long seed, StepRef step,
                         unsigned layer_id, cudaStream_t stream, uint32_t* status,
-                        const PartialsRef* partials = nullptr) {
+                        const PartialsRef* partials = nullptr, bool coresident = false) {
   // With `partials`, the clip factors come from the per-warp norm partials: the bulk-copy
   // reduce sums them in its prologue (and block 0 writes norm2 / norms_out / c_out); the
   // other reduce needs them summed first.
-  if (B <= 8) {
+  // `coresident`: the reduce runs beside a tensor-core pass (the overlapped block step), so it
+  // takes the plain kernel with its tables read through the cache, whose blocks fit on an SM
+  // next to a tensor-core CTA; the bulk-copy kernel fills a whole SM's shared memory.
+  if (B <= 8 && !coresident) {
     // Warp-specialised bulk-copy reduce: noise generation overlaps the HBM stream.
     const PhiloxKey key = philox_key_from_seed(seed);
     const PartialsRef pr = partials ? *partials : PartialsRef{nullptr, 0, 0, nullptr, nullptr, nullptr};
@@ -646,12 +654,16 @@ dp_status launch_reduce(const __nv_bfloat16* gs, int B, long long mn, NormSource
     src = NormSource{partials->norm2, nullptr, nullptr};
   }
   const int cached = B < kReduceCachedSamples ? B : kReduceCachedSamples;
-  const int grid = std::min(stream_grid(static_cast<unsigned long long>(mn / 8), 256), sm_count() * 2);
-  const size_t smem = kNoiseSharedBytes + cached * sizeof(float);
+  // Beside a tensor-core pass one block per SM: two would take more registers than an SM has
+  // next to a tensor-core CTA, and the next pass would wait for them.
+  const int grid = std::min(stream_grid(static_cast<unsigned long long>(mn / 8), 256),
+                            coresident ? sm_count() : sm_count() * 2);
+  const size_t smem = (coresident ? 0 : kNoiseSharedBytes) + cached * sizeof(float);
   const PhiloxKey key = philox_key_from_seed(seed);
   LaunchScope scope(kKindReduce, stream);
-  // B > 8 here (smaller batches take the bulk-copy kernel above): a runtime sample loop.
-  return reduce_kernel_launch(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step);
+  // B > 8, or beside a tensor-core pass: a runtime sample loop.
+  return reduce_kernel_launch(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step,
+                              !coresident);
 }
 
 // ---------------------------------------------------------------- common front end
@@ -797,11 +809,80 @@ struct BlockLayout {
   long long partial_op_stride = 0;       // floats between the partial sets of a shared group
   std::vector<size_t> tiles;             // per layer; 0 when the layer does not keep tiles
   std::vector<dp_norm_method> methods;   // resolved per layer
-  std::vector<std::vector<int>> groups;  // layers in call order, grouped as described above
+  std::vector<std::vector<int>> groups;  // layers grouped as described above, in processing order
+  // Per-layer mode with two or more gradients-once layers: the reduce of one such layer runs on
+  // a second stream beside the next layer's tensor-core pass, so consecutive gradients-once
+  // layers alternate between two tile regions and two norm-partial sets.
+  bool overlap = false;
+  size_t tiles_alt = 0;                  // the second tile region (overlap only)
 };
+
+// Whether a per-layer block step overlaps each gradients-once reduce with the next layer's
+// tensor-core pass (environment DPCLIP_OVERLAP_REDUCE=0 turns it off; read at every call, so
+// a workspace size query and the step that uses it must see the same setting).
+bool overlap_reduce_enabled() {
+  const char* v = getenv("DPCLIP_OVERLAP_REDUCE");
+  return !(v && v[0] == '0');
+}
 
 Shape layer_shape(const dp_layer& l, int B, int T, dp_dtype dt) {
   return Shape{B, T, l.d_in, l.d_out, l.P ? l.r : 0, dt};
+}
+
+// The second stream of the current device on which overlapped reduces run, created on the
+// first call that needs it (non-blocking, so it never waits on the legacy default stream).
+dp_status side_stream(cudaStream_t* out) {
+  static std::mutex mu;
+  static cudaStream_t streams[64] = {nullptr};
+  int dev = 0;
+  DP_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return DP_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> g(mu);
+  if (!streams[dev]) DP_CUDA(cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking));
+  *out = streams[dev];
+  return DP_OK;
+}
+
+// Ordering events of one host thread on the current device, reused round-robin.  A stream's
+// wait on an event takes the event's state when the wait is enqueued, so reuse is safe once
+// every wait on the earlier record has been enqueued (a block step waits at most two layers
+// after a record, far fewer than the ring's size).
+class EventRing {
+ public:
+  dp_status next(cudaEvent_t* out) {
+    int dev = 0;
+    DP_CUDA(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= 64) return DP_ERR_UNSUPPORTED;
+    auto& ring = rings_[dev];
+    if (ring.empty()) {
+      ring.resize(kSize, nullptr);
+      for (auto& e : ring) DP_CUDA(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
+    }
+    *out = ring[pos_[dev]];
+    pos_[dev] = (pos_[dev] + 1) % kSize;
+    return DP_OK;
+  }
+
+ private:
+  static constexpr int kSize = 64;
+  std::vector<cudaEvent_t> rings_[64];
+  int pos_[64] = {0};
+};
+
+EventRing& event_ring() {
+  static thread_local EventRing ring;
+  return ring;
+}
+
+// Makes `waiter` wait for everything enqueued on `signaller` so far.
+dp_status stream_after(cudaStream_t waiter, cudaStream_t signaller, cudaEvent_t* recorded = nullptr) {
+  cudaEvent_t e;
+  dp_status st = event_ring().next(&e);
+  if (st != DP_OK) return st;
+  DP_CUDA(cudaEventRecord(e, signaller));
+  DP_CUDA(cudaStreamWaitEvent(waiter, e, 0));
+  if (recorded) *recorded = e;
+  return DP_OK;
 }
 
 dp_status block_methods(const dp_layer* layers, int L, int B, int T, dp_dtype dt, dp_norm_method method,
@@ -844,6 +925,23 @@ BlockLayout block_layout(const dp_layer* layers, int L, int B, int T, dp_dtype d
   BlockLayout Lb;
   Lb.methods = methods;
   Lb.groups = block_groups(layers, L, dt, methods);
+  int once_groups = 0;
+  for (const auto& g : Lb.groups) once_groups += (dt == DP_BF16 && methods[g[0]] == DP_NORM_ONCE) ? 1 : 0;
+  Lb.overlap = (mode == DP_CLIP_PER_LAYER && once_groups >= 2 && overlap_reduce_enabled());
+  if (Lb.overlap) {
+    // Gradients-once layers first, largest reduce first, so that the one reduce no tensor-core
+    // pass follows is the smallest; then the other groups.  Per-layer clipping makes the layers
+    // independent, so the order changes no result.
+    auto size_of = [&](const std::vector<int>& g) {
+      const Shape s = layer_shape(layers[g[0]], B, T, dt);
+      return static_cast<long long>(s.m) * s.ne();
+    };
+    auto is_once = [&](const std::vector<int>& g) { return methods[g[0]] == DP_NORM_ONCE; };
+    std::stable_sort(Lb.groups.begin(), Lb.groups.end(), [&](const std::vector<int>& a, const std::vector<int>& b) {
+      if (is_once(a) != is_once(b)) return is_once(a);
+      return is_once(a) && size_of(a) > size_of(b);
+    });
+  }
   size_t off = 256;
   Lb.flat = off;
   off += align256(static_cast<size_t>(B) * 8);
@@ -863,7 +961,7 @@ BlockLayout block_layout(const dp_layer* layers, int L, int B, int T, dp_dtype d
         tiles_most = std::max(tiles_most, static_cast<size_t>(B) * s.m * s.ne() * 2);
     }
   }
-  int sets = 1;
+  int sets = Lb.overlap ? 2 : 1;
   for (const auto& g : Lb.groups) sets = std::max(sets, static_cast<int>(g.size()));
   Lb.partial_op_stride = static_cast<long long>(align256(static_cast<size_t>(B) * Lb.partial_stride * 4) / 4);
   Lb.partials = off;
@@ -876,6 +974,10 @@ BlockLayout block_layout(const dp_layer* layers, int L, int B, int T, dp_dtype d
       for (int l = 0; l < L; ++l)
         if (dt == DP_BF16 && methods[l] == DP_NORM_ONCE) Lb.tiles[l] = off;
       off += align256(tiles_most);
+      if (Lb.overlap) {
+        Lb.tiles_alt = off;
+        off += align256(tiles_most);
+      }
     }
   } else {
     for (int l = 0; l < L; ++l) {
@@ -1014,14 +1116,26 @@ dp_status block_step(const dp_layer* layers, int L, dp_dtype dt, int B, int T, d
   NoiseBatch deferred;
   deferred.count = 0;
   if (mode == DP_CLIP_PER_LAYER) {
+    // Overlap: gradients-once layer k's reduce runs on the side stream beside layer k+1's
+    // tensor-core pass.  Layer k alternates between tile region / partial set k mod 2, and the
+    // pass of layer k+2, which reuses them, waits for reduce k.  The side stream joins the
+    // caller's stream before the call returns, so the call keeps plain stream semantics (and a
+    // CUDA graph captured around it stays one fork-join).
+    cudaStream_t side = stream;
+    if (Lb.overlap && (st = side_stream(&side)) != DP_OK) return st;
+    cudaEvent_t reduce_done[2] = {nullptr, nullptr};
+    int once_k = 0;
+    bool side_pending = false;  // reduces on the side stream the caller's stream has not joined
     // Each group: its norms, then each member's clipped sum with its own bound and noise.
     for (const auto& g : Lb.groups) {
       if (dt == DP_BF16 && Lb.methods[g[0]] == DP_NORM_ONCE) {
         // Gradients once: tiles and norm partials, then the reduce that sums the partials.
         const dp_layer& y = layers[g[0]];
         const Shape s = layer_shape(y, B, T, dt);
-        float* partials = reinterpret_cast<float*>(ws + Lb.partials);
-        __nv_bfloat16* tiles = reinterpret_cast<__nv_bfloat16*>(ws + Lb.tiles[g[0]]);
+        const int par = Lb.overlap ? (once_k & 1) : 0;
+        float* partials = reinterpret_cast<float*>(ws + Lb.partials) + par * Lb.partial_op_stride;
+        __nv_bfloat16* tiles = reinterpret_cast<__nv_bfloat16*>(ws + (par ? Lb.tiles_alt : Lb.tiles[g[0]]));
+        if (reduce_done[par]) DP_CUDA(cudaStreamWaitEvent(stream, reduce_done[par], 0));
         const void* Z;
         if ((st = block_operand(layers, g[0], dt, B, T, Lb, ws, stream, true, &Z)) != DP_OK) return st;
         int count = 0;
@@ -1031,11 +1145,23 @@ dp_status block_step(const dp_layer* layers, int L, dp_dtype dt, int B, int T, d
         float* n2 = reinterpret_cast<float*>(ws + Lb.norm2) + static_cast<size_t>(g[0]) * B;
         const PartialsRef pr{partials, Lb.partial_stride, count, n2, y.norms_out, nullptr};
         const double noise_std = (sigma == 0.0f) ? 0.0 : static_cast<double>(sigma) * static_cast<double>(y.C);
+        if (Lb.overlap && (st = stream_after(side, stream)) != DP_OK) return st;
         if ((st = launch_reduce(tiles, B, static_cast<long long>(s.m) * s.ne(), layer_norm_source(Lb, ws, g[0], B, dt),
-                                y.C, y.G_out, noise_std, seed, step, y.layer_id, stream,
-                                reinterpret_cast<uint32_t*>(ws), &pr)) != DP_OK)
+                                y.C, y.G_out, noise_std, seed, step, y.layer_id, side,
+                                reinterpret_cast<uint32_t*>(ws), &pr, Lb.overlap)) != DP_OK)
           return st;
+        if (Lb.overlap) {
+          if ((st = event_ring().next(&reduce_done[par])) != DP_OK) return st;
+          DP_CUDA(cudaEventRecord(reduce_done[par], side));
+          side_pending = true;
+        }
+        ++once_k;
         continue;
+      }
+      // The other groups reuse the norm-partial sets: join the side stream first.
+      if (side_pending) {
+        if ((st = stream_after(stream, side)) != DP_OK) return st;
+        side_pending = false;
       }
       // bf16: the row-scaling kernel of each member's clipped sum sums its norm partials.
       int count = 0;
@@ -1053,6 +1179,7 @@ dp_status block_step(const dp_layer* layers, int L, dp_dtype dt, int B, int T, d
           return st;
       }
     }
+    if (side_pending && (st = stream_after(stream, side)) != DP_OK) return st;  // join
     return launch_noise_batch(deferred, seed, step, stream);
   }
   // 1. Every layer's per-sample norms (gradients-once layers also keep their tiles).

@@ -346,20 +346,25 @@ __device__ __forceinline__ void noise8_f32(uint32_t blk0, uint32_t layer_id, uin
   for (int q = 0; q < 4; ++q) n[4 + q] = z.rounded(q);
 }
 
-template <int NP>
+// STAGED: the Box-Muller tables are staged in shared memory (32 KB); otherwise they are read
+// through the read-only cache and the block needs only the clip factors' few bytes of shared
+// memory, so it fits on an SM beside a running tensor-core CTA (the overlapped block step).
+template <int NP, bool STAGED>
 __global__ void __launch_bounds__(256, 2) clip_reduce_kernel(
     const __nv_bfloat16* __restrict__ Gs, int B, long long mn, NormSource src, float C,
     float* __restrict__ out, double noise_std, PhiloxKey key, uint32_t layer_id, StepRef step) {
   griddep_enter();
   const uint32_t step_lo = step.get();
   using NT = NoiseTables<NP>;
-  extern __shared__ double2 reduce_smem[];  // noise tables, then the cached clip factors
-  float* c_smem = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(reduce_smem) + NT::kBytes);
+  extern __shared__ double2 reduce_smem[];  // noise tables (STAGED), then the cached clip factors
+  float* c_smem = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(reduce_smem) + (STAGED ? NT::kBytes : 0));
   const int cached = B < kReduceCachedSamples ? B : kReduceCachedSamples;
   for (int i = threadIdx.x; i < cached; i += blockDim.x) c_smem[i] = clip_factor(src.norm(i), C);
-  if (noise_std != 0.0) NT::stage(reduce_smem);
+  if (STAGED && noise_std != 0.0) NT::stage(reduce_smem);
   __syncthreads();
-  const auto tab = NT::shared(reduce_smem);
+  using Tab = typename std::conditional<STAGED, typename NT::Shared, typename NT::Global>::type;
+  Tab tab;
+  if constexpr (STAGED) tab = NT::shared(reduce_smem);
   const ScaleF2 sc = scale_f2(noise_std);
   const long long nvec = mn / 8;  // 16-byte vectors per sample
   for (long long v = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; v < nvec;

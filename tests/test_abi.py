@@ -178,10 +178,16 @@ def test_block_workspace_size_and_host_rejections(L):
                         DpLayer(FAKE, FAKE, 4096, 11008, 1, 0.3, FAKE, None))
     per = L.dp_block_workspace_size(lay, 2, 8, 2048, _lib.DP_BF16, 0, _lib.DP_NORM_ONCE)
     flat = L.dp_block_workspace_size(lay, 2, 8, 2048, _lib.DP_BF16, 1, _lib.DP_NORM_ONCE)
-    # per-layer mode reuses one tile region sized for the largest layer; flat once keeps every
-    # layer's tiles
-    assert 8 * 2 * 4096 * 11008 <= per <= L.dp_workspace_size_for(8, 2048, 4096, 11008, 0, _lib.DP_BF16,
-                                                                   _lib.DP_NORM_ONCE)
+    # per-layer mode alternates two tile regions sized for the largest layer (each reduce runs
+    # beside the next layer's tensor-core pass); flat once keeps every layer's tiles
+    tiles = 8 * 2 * 4096 * 11008
+    one = L.dp_workspace_size_for(8, 2048, 4096, 11008, 0, _lib.DP_BF16, _lib.DP_NORM_ONCE)
+    assert 2 * tiles <= per <= one + tiles
+    os.environ["DPCLIP_OVERLAP_REDUCE"] = "0"        # serial schedule: one region
+    try:
+        assert tiles <= L.dp_block_workspace_size(lay, 2, 8, 2048, _lib.DP_BF16, 0, _lib.DP_NORM_ONCE) <= one
+    finally:
+        del os.environ["DPCLIP_OVERLAP_REDUCE"]
     assert flat >= 8 * 2 * (4096 * 4096 + 4096 * 11008)
     assert L.dp_block_workspace_size(lay, 2, 8, 2048, _lib.DP_BF16, 7, 0) == 0
     assert L.dp_block_workspace_size(lay, 0, 8, 2048, _lib.DP_BF16, 0, 0) == 0

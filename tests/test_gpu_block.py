@@ -94,6 +94,28 @@ def test_per_layer_block_equals_linear_steps():
         assert rel_fro(host(outs[k]), host(G)) <= 1e-6, lin.name
 
 
+@pytest.mark.parametrize("sigma", [0.0, 0.6])
+def test_overlapped_reduces_equal_serial_order(sigma, monkeypatch):
+    """Per-layer gradients-once block: each reduce runs on a second stream beside the next
+    layer's tensor-core pass, in a different layer order, with alternating tile regions.  The
+    results must be bitwise those of the serial schedule (DPCLIP_OVERLAP_REDUCE=0)."""
+    w, data, dev = _block(seed=6)
+    C = 1.0 / math.sqrt(7.0)
+    outs_o, norms_o, _ = _lib.dp_block_step(_layers(w, dev, C), mode="per_layer", sigma=sigma, seed=w.seed,
+                                            step=3, method="once")
+    monkeypatch.setenv("DPCLIP_OVERLAP_REDUCE", "0")
+    outs_s, norms_s, _ = _lib.dp_block_step(_layers(w, dev, C), mode="per_layer", sigma=sigma, seed=w.seed,
+                                            step=3, method="once")
+    torch.cuda.synchronize()
+    for k, lin in enumerate(w.linears):
+        assert torch.equal(norms_o[k], norms_s[k]), lin.name
+        assert torch.equal(outs_o[k], outs_s[k]), lin.name
+    ref = oracle.block_step(_oracle_layers(w, data, C), C, 0.0, w.seed, 3, mode="per_layer")
+    if sigma == 0:
+        for k, lin in enumerate(w.linears):
+            assert rel_fro(host(outs_o[k]), ref["layers"][k]["S"]) <= TOL["bf16"]["sum"], lin.name
+
+
 @pytest.mark.slow
 def test_flat_clipping_llama7b_block_full():
     """Flat clipping over the full 7B block, every entry of every linear's sum compared."""

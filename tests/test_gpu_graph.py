@@ -63,7 +63,8 @@ def test_linear_step_graph_replays_each_step(method, r):
     assert _lib.dp_workspace_status(ws) == _lib.DP_OK
 
 
-def test_block_step_graph_replays_each_step():
+@pytest.mark.parametrize("method", ["ghost", "once"])   # once: reduces on a second stream, joined
+def test_block_step_graph_replays_each_step(method):
     w = inputs.Workload("gblk", B=3, T=256, dtype="bf16", linears=inputs._block(0, 256, 384),
                         C=1.0 / math.sqrt(7.0), sigma=0.6, seed=5, dy_var="per_layer")
     d = inputs.generate(w)
@@ -76,20 +77,20 @@ def test_block_step_graph_replays_each_step():
         _lib.DpLayer(l["X"].data_ptr(), l["dY"].data_ptr(), l["X"].shape[2], l["dY"].shape[2], l["layer_id"],
                      l["C"], l["G_out"].data_ptr(), l["norms_out"].data_ptr()) for l in layers])
     ws = torch.empty(_lib.lib().dp_block_workspace_size(arr, len(layers), w.B, w.T, _lib.DP_BF16,
-                                                         _lib.DP_CLIP_PER_LAYER, _lib.DP_NORM_GHOST),
+                                                         _lib.DP_CLIP_PER_LAYER, _lib.METHODS[method]),
                      dtype=torch.uint8, device="cuda")
     s = torch.cuda.Stream()
     eager = {}
     with torch.cuda.stream(s):
         for k in (7, 8):
-            _lib.dp_block_step(layers, mode="per_layer", sigma=w.sigma, seed=w.seed, step=k, method="ghost",
+            _lib.dp_block_step(layers, mode="per_layer", sigma=w.sigma, seed=w.seed, step=k, method=method,
                                workspace=ws, stream=s)
             s.synchronize()
             eager[k] = [l["G_out"].clone() for l in layers]
     step = torch.zeros(1, dtype=torch.int64, device="cuda")
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=s):
-        _lib.dp_block_step(layers, mode="per_layer", sigma=w.sigma, seed=w.seed, step=step, method="ghost",
+        _lib.dp_block_step(layers, mode="per_layer", sigma=w.sigma, seed=w.seed, step=step, method=method,
                            workspace=ws, stream=s)
     for k in (8, 7):
         with torch.cuda.stream(s):
