@@ -586,16 +586,32 @@ dp_status launch_finalize(NormSource src, int B, float C, float* norms_out, floa
 // Precision of the Box-Muller evaluation in the gradients-once reduce.
 constexpr int kReduceNoise = kGradientNoise;
 
+// The plain reduce: staged tables and a runtime sample loop (B > 8), or, beside a tensor-core
+// pass, tables through the cache and the sample loop unrolled for B <= 8.
+template <int BU>
+dp_status reduce_plain_launch(int grid, size_t smem, cudaStream_t stream, const __nv_bfloat16* gs, int B,
+                              long long mn, NormSource src, float C, float* out, double noise_std, PhiloxKey key,
+                              unsigned layer_id, StepRef step) {
+  constexpr bool kStaged = (BU == 0);
+  DP_LAUNCH("clip_reduce_kernel", clip_reduce_kernel<kReduceNoise, kStaged, BU>, grid, 256, smem, stream, gs, B, mn,
+            src, C, out, noise_std, key, layer_id, step);
+  return DP_OK;
+}
+
 dp_status reduce_kernel_launch(int grid, size_t smem, cudaStream_t stream, const __nv_bfloat16* gs, int B,
                           long long mn, NormSource src, float C, float* out, double noise_std, PhiloxKey key,
                           unsigned layer_id, StepRef step, bool staged) {
-  if (staged)
-    DP_LAUNCH("clip_reduce_kernel", clip_reduce_kernel<kReduceNoise, true>, grid, 256, smem, stream, gs, B, mn,
-              src, C, out, noise_std, key, layer_id, step);
-  else
-    DP_LAUNCH("clip_reduce_kernel", clip_reduce_kernel<kReduceNoise, false>, grid, 256, smem, stream, gs, B, mn,
-              src, C, out, noise_std, key, layer_id, step);
-  return DP_OK;
+  if (staged) return reduce_plain_launch<0>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step);
+  switch (B) {  // coresident: B <= 8 (larger batches keep the staged runtime loop)
+    case 1: return reduce_plain_launch<1>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step);
+    case 2: return reduce_plain_launch<2>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step);
+    case 3: return reduce_plain_launch<3>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step);
+    case 4: return reduce_plain_launch<4>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step);
+    case 5: return reduce_plain_launch<5>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step);
+    case 6: return reduce_plain_launch<6>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step);
+    case 7: return reduce_plain_launch<7>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step);
+    default: return reduce_plain_launch<8>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step);
+  }
 }
 
 template <int BU>
@@ -656,14 +672,14 @@ dp_status launch_reduce(const __nv_bfloat16* gs, int B, long long mn, NormSource
   const int cached = B < kReduceCachedSamples ? B : kReduceCachedSamples;
   // Beside a tensor-core pass one block per SM: two would take more registers than an SM has
   // next to a tensor-core CTA, and the next pass would wait for them.
+  const bool unrolled = coresident && B <= 8;
   const int grid = std::min(stream_grid(static_cast<unsigned long long>(mn / 8), 256),
                             coresident ? sm_count() : sm_count() * 2);
-  const size_t smem = (coresident ? 0 : kNoiseSharedBytes) + cached * sizeof(float);
+  const size_t smem = (unrolled ? 0 : kNoiseSharedBytes) + cached * sizeof(float);
   const PhiloxKey key = philox_key_from_seed(seed);
   LaunchScope scope(kKindReduce, stream);
-  // B > 8, or beside a tensor-core pass: a runtime sample loop.
   return reduce_kernel_launch(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step,
-                              !coresident);
+                              !unrolled);
 }
 
 // ---------------------------------------------------------------- common front end

@@ -349,7 +349,10 @@ __device__ __forceinline__ void noise8_f32(uint32_t blk0, uint32_t layer_id, uin
 // STAGED: the Box-Muller tables are staged in shared memory (32 KB); otherwise they are read
 // through the read-only cache and the block needs only the clip factors' few bytes of shared
 // memory, so it fits on an SM beside a running tensor-core CTA (the overlapped block step).
-template <int NP, bool STAGED>
+// BU > 0: exactly BU samples, unrolled: each thread issues all BU loads of its 8 elements,
+// computes their noise while the loads are in flight, then forms the weighted sum.  BU = 0: a
+// runtime loop over B samples.
+template <int NP, bool STAGED, int BU>
 __global__ void __launch_bounds__(256, 2) clip_reduce_kernel(
     const __nv_bfloat16* __restrict__ Gs, int B, long long mn, NormSource src, float C,
     float* __restrict__ out, double noise_std, PhiloxKey key, uint32_t layer_id, StepRef step) {
@@ -373,20 +376,40 @@ __global__ void __launch_bounds__(256, 2) clip_reduce_kernel(
     float acc[8];
 #pragma unroll
     for (int q = 0; q < 8; ++q) acc[q] = 0.f;
-    for (int i = 0; i < B; ++i) {
-      const float c = i < cached ? c_smem[i] : clip_factor(src.norm(i), C);
-      const uint4 pk = __ldcs(g + static_cast<long long>(i) * nvec);
-      const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&pk);
+    float z[8];
+    if constexpr (BU > 0) {
+      uint4 pk[BU];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 f = __bfloat1622float2(hv[e]);
-        acc[2 * e] = fmaf(c, f.x, acc[2 * e]);
-        acc[2 * e + 1] = fmaf(c, f.y, acc[2 * e + 1]);
+      for (int i = 0; i < BU; ++i) pk[i] = __ldcs(g + static_cast<long long>(i) * nvec);
+      if (noise_std != 0.0)
+        noise8_f32<NP>(static_cast<uint32_t>(2 * v), layer_id, step_lo, key, tab, noise_std, sc, z);
+#pragma unroll
+      for (int i = 0; i < BU; ++i) {
+        const float c = c_smem[i];
+        const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&pk[i]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(hv[e]);
+          acc[2 * e] = fmaf(c, f.x, acc[2 * e]);
+          acc[2 * e + 1] = fmaf(c, f.y, acc[2 * e + 1]);
+        }
       }
+    } else {
+      for (int i = 0; i < B; ++i) {
+        const float c = i < cached ? c_smem[i] : clip_factor(src.norm(i), C);
+        const uint4 pk = __ldcs(g + static_cast<long long>(i) * nvec);
+        const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&pk);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(hv[e]);
+          acc[2 * e] = fmaf(c, f.x, acc[2 * e]);
+          acc[2 * e + 1] = fmaf(c, f.y, acc[2 * e + 1]);
+        }
+      }
+      if (noise_std != 0.0)
+        noise8_f32<NP>(static_cast<uint32_t>(2 * v), layer_id, step_lo, key, tab, noise_std, sc, z);
     }
     if (noise_std != 0.0) {
-      float z[8];
-      noise8_f32<NP>(static_cast<uint32_t>(2 * v), layer_id, step_lo, key, tab, noise_std, sc, z);
 #pragma unroll
       for (int q = 0; q < 8; ++q) acc[q] = acc[q] + z[q];
     }
