@@ -831,7 +831,16 @@ struct BlockLayout {
   // layers alternate between two tile regions and two norm-partial sets.
   bool overlap = false;
   size_t tiles_alt = 0;                  // the second tile region (overlap only)
+  // Per-layer mode, bf16, two or more ghost/explicit layers whose scaled copies fit
+  // kBatchScaleBytes: every such layer's norm pass first (each into its own norm-partial set),
+  // then one row-scaling launch for all of them (each into its own scaled copy), then their
+  // clipped sums.  One launch replaces one per layer.
+  bool batched_scale = false;
+  std::vector<size_t> scaled_l;          // per layer: its scaled copy (batched schedule), or 0
+  std::vector<long long> partial_set;    // per layer: its norm-partial set (batched schedule)
 };
+
+constexpr size_t kBatchScaleBytes = size_t(256) << 20;
 
 // Whether a per-layer block step overlaps each gradients-once reduce with the next layer's
 // tensor-core pass (environment DPCLIP_OVERLAP_REDUCE=0 turns it off; read at every call, so
@@ -979,6 +988,28 @@ BlockLayout block_layout(const dp_layer* layers, int L, int B, int T, dp_dtype d
   }
   int sets = Lb.overlap ? 2 : 1;
   for (const auto& g : Lb.groups) sets = std::max(sets, static_cast<int>(g.size()));
+  // The batched row-scaling schedule (see BlockLayout).
+  size_t scaled_all = 0;
+  int scaled_layers = 0;
+  for (const auto& g : Lb.groups) {
+    if (dt != DP_BF16 || methods[g[0]] == DP_NORM_ONCE) continue;
+    for (int l : g) {
+      const Shape s = layer_shape(layers[l], B, T, dt);
+      scaled_all += align256(static_cast<size_t>(s.N()) * static_cast<size_t>(std::min(s.m, s.ne())) * 2);
+      ++scaled_layers;
+    }
+  }
+  Lb.batched_scale = (mode == DP_CLIP_PER_LAYER && scaled_layers >= 2 && scaled_layers <= kMaxScaleSegments &&
+                      scaled_all <= kBatchScaleBytes);
+  Lb.partial_set.assign(L, 0);
+  if (Lb.batched_scale) {
+    int next = 2;  // sets 0 and 1 serve the gradients-once layers
+    for (const auto& g : Lb.groups) {
+      if (methods[g[0]] == DP_NORM_ONCE) continue;
+      for (int l : g) Lb.partial_set[l] = next++;
+    }
+    sets = std::max(sets, next);
+  }
   Lb.partial_op_stride = static_cast<long long>(align256(static_cast<size_t>(B) * Lb.partial_stride * 4) / 4);
   Lb.partials = off;
   off += static_cast<size_t>(sets) * Lb.partial_op_stride * 4;
@@ -1000,6 +1031,17 @@ BlockLayout block_layout(const dp_layer* layers, int L, int B, int T, dp_dtype d
       if (dt == DP_BF16 && methods[l] == DP_NORM_ONCE) {
         Lb.tiles[l] = off;
         off += align256(static_cast<size_t>(B) * layers[l].d_in * layer_shape(layers[l], B, T, dt).ne() * 2);
+      }
+    }
+  }
+  Lb.scaled_l.assign(L, 0);
+  if (Lb.batched_scale) {
+    for (const auto& g : Lb.groups) {
+      if (methods[g[0]] == DP_NORM_ONCE) continue;
+      for (int l : g) {
+        const Shape s = layer_shape(layers[l], B, T, dt);
+        Lb.scaled_l[l] = off;
+        off += align256(static_cast<size_t>(s.N()) * static_cast<size_t>(std::min(s.m, s.ne())) * 2);
       }
     }
   }
@@ -1040,7 +1082,8 @@ dp_status block_operand(const dp_layer* layers, int l, dp_dtype dt, int B, int T
 // Squared norms of the layers of one group into their [B] rows of the norm2 block, and each
 // layer's norms_out when given (gradients-once layers also keep their tiles).
 dp_status block_group_norms(const dp_layer* layers, const std::vector<int>& g, dp_dtype dt, int B, int T,
-                            const BlockLayout& Lb, uint8_t* ws, cudaStream_t stream, int* count_out = nullptr) {
+                            const BlockLayout& Lb, uint8_t* ws, cudaStream_t stream, int* count_out = nullptr,
+                            float* partials_base = nullptr) {
   dp_status st;
   uint32_t* status = reinterpret_cast<uint32_t*>(ws);
   const dp_layer& y0 = layers[g[0]];
@@ -1062,7 +1105,7 @@ dp_status block_group_norms(const dp_layer* layers, const std::vector<int>& g, d
     }
     return DP_OK;
   }
-  float* partials = reinterpret_cast<float*>(ws + Lb.partials);
+  float* partials = partials_base ? partials_base : reinterpret_cast<float*>(ws + Lb.partials);
   int count = 0;
   if (g.size() > 1) {
     if ((st = bf16_norms_ghost_shared(s, y0.X, Zs, static_cast<int>(g.size()), partials, Lb.partial_stride,
@@ -1122,6 +1165,64 @@ NormSource layer_norm_source(const BlockLayout& Lb, uint8_t* ws, int l, int B, d
   return src;
 }
 
+// One launch of the row scalings of the layers in `ls` (batched schedule): layer l's narrower
+// operand (Z, or X when X is narrower) scaled by its clip factors into its own copy.  Each
+// layer's blocks sum their samples' norm partials themselves, unless a block would cover too
+// many samples or slots; that layer's partials are then summed first.
+dp_status launch_scale_batch(const dp_layer* layers, const std::vector<int>& ls, const std::vector<int>& counts,
+                             dp_dtype dt, int B, int T, const BlockLayout& Lb, uint8_t* ws, cudaStream_t stream) {
+  ScaleBatch b;
+  memset(&b, 0, sizeof(b));
+  b.T = T;
+  b.count = static_cast<int>(ls.size());
+  unsigned long long total_vecs = 0;
+  std::vector<unsigned long long> vecs(ls.size());
+  for (size_t q = 0; q < ls.size(); ++q) {
+    const Shape s = layer_shape(layers[ls[q]], B, T, dt);
+    vecs[q] = static_cast<unsigned long long>(s.N()) * (std::min(s.m, s.ne()) / 8);
+    total_vecs += vecs[q];
+  }
+  const int grid = stream_grid(total_vecs, 256);
+  int first = 0;
+  size_t smem = 0;
+  dp_status st;
+  for (size_t q = 0; q < ls.size(); ++q) {
+    const int l = ls[q];
+    const dp_layer& y = layers[l];
+    const Shape s = layer_shape(y, B, T, dt);
+    const void* Z;
+    if ((st = block_operand(layers, l, dt, B, T, Lb, ws, stream, false, &Z)) != DP_OK) return st;
+    ScaleSegment& sg = b.seg[q];
+    sg.in = static_cast<const __nv_bfloat16*>(s.ne() <= s.m ? Z : y.X);
+    sg.out = reinterpret_cast<__nv_bfloat16*>(ws + Lb.scaled_l[l]);
+    sg.rows = s.N();
+    sg.cols = std::min(s.m, s.ne());
+    sg.C = y.C;
+    sg.first_block = first;
+    sg.blocks = static_cast<int>(std::max<unsigned long long>(1, (vecs[q] * grid + total_vecs - 1) / total_vecs));
+    first += sg.blocks;
+    float* partials = reinterpret_cast<float*>(ws + Lb.partials) + Lb.partial_set[l] * Lb.partial_op_stride;
+    float* n2 = reinterpret_cast<float*>(ws + Lb.norm2) + static_cast<size_t>(l) * B;
+    const unsigned long long per = (vecs[q] + sg.blocks - 1) / sg.blocks;
+    const unsigned long long sample_vecs = static_cast<unsigned long long>(T) * (sg.cols / 8);
+    const long long smax = static_cast<long long>(std::min<unsigned long long>((per - 1) / sample_vecs + 2, B));
+    if (smax <= kScaleFusedMaxSamples && smax * counts[q] <= kScaleFusedPartialSlots) {
+      sg.pr = PartialsRef{partials, Lb.partial_stride, counts[q], n2, y.norms_out, nullptr};
+      smem = std::max(smem, static_cast<size_t>(smax) * sizeof(float));
+    } else {
+      // Too many samples or slots for one block: sum this layer's partials first.
+      if ((st = launch_norm_partials(partials, Lb.partial_stride, counts[q], B, y.C, n2, y.norms_out, nullptr,
+                                     stream)) != DP_OK)
+        return st;
+      sg.pr = PartialsRef{nullptr, 0, 0, nullptr, nullptr, nullptr};
+      sg.src = NormSource{n2, nullptr, nullptr};
+    }
+  }
+  LaunchScope scope(kKindScale, stream);
+  DP_LAUNCH("scale_rows_bf16_batch_kernel", scale_rows_bf16_batch_kernel, first, 256, smem, stream, b);
+  return DP_OK;
+}
+
 dp_status block_step(const dp_layer* layers, int L, dp_dtype dt, int B, int T, dp_clip_mode mode, float C,
                      float sigma, unsigned long long seed, StepRef step, const BlockLayout& Lb,
                      float* flat_norms_out, uint8_t* ws, cudaStream_t stream) {
@@ -1142,6 +1243,7 @@ dp_status block_step(const dp_layer* layers, int L, dp_dtype dt, int B, int T, d
     cudaEvent_t reduce_done[2] = {nullptr, nullptr};
     int once_k = 0;
     bool side_pending = false;  // reduces on the side stream the caller's stream has not joined
+    std::vector<int> batch_layers, batch_counts;  // batched schedule: layers waiting for their sums
     // Each group: its norms, then each member's clipped sum with its own bound and noise.
     for (const auto& g : Lb.groups) {
       if (dt == DP_BF16 && Lb.methods[g[0]] == DP_NORM_ONCE) {
@@ -1179,6 +1281,18 @@ dp_status block_step(const dp_layer* layers, int L, dp_dtype dt, int B, int T, d
         if ((st = stream_after(stream, side)) != DP_OK) return st;
         side_pending = false;
       }
+      if (Lb.batched_scale) {
+        // Batched schedule: this group's norm pass now, its row scaling and clipped sums after
+        // every group's norm pass.
+        int count = 0;
+        float* base = reinterpret_cast<float*>(ws + Lb.partials) + Lb.partial_set[g[0]] * Lb.partial_op_stride;
+        if ((st = block_group_norms(layers, g, dt, B, T, Lb, ws, stream, &count, base)) != DP_OK) return st;
+        for (int l : g) {
+          batch_layers.push_back(l);
+          batch_counts.push_back(count);
+        }
+        continue;
+      }
       // bf16: the row-scaling kernel of each member's clipped sum sums its norm partials.
       int count = 0;
       if ((st = block_group_norms(layers, g, dt, B, T, Lb, ws, stream, dt == DP_BF16 ? &count : nullptr)) !=
@@ -1192,6 +1306,20 @@ dp_status block_step(const dp_layer* layers, int L, dp_dtype dt, int B, int T, d
                              layers[l].norms_out, nullptr};
         if ((st = block_layer_sum(layers, l, dt, B, T, src, layers[l].C, sigma, seed, step, Lb, ws, stream,
                                   &deferred, dt == DP_BF16 ? &pr : nullptr)) != DP_OK)
+          return st;
+      }
+    }
+    if (!batch_layers.empty()) {
+      if ((st = launch_scale_batch(layers, batch_layers, batch_counts, dt, B, T, Lb, ws, stream)) != DP_OK) return st;
+      for (int l : batch_layers) {
+        const dp_layer& y = layers[l];
+        const Shape s = layer_shape(y, B, T, dt);
+        const void* Z;
+        if ((st = block_operand(layers, l, dt, B, T, Lb, ws, stream, false, &Z)) != DP_OK) return st;
+        const void* scaled = ws + Lb.scaled_l[l];
+        const double noise_std = (sigma == 0.0f) ? 0.0 : static_cast<double>(sigma) * static_cast<double>(y.C);
+        if ((st = bf16_clipsum(s, s.ne() <= s.m ? y.X : scaled, s.ne() <= s.m ? scaled : Z, y.G_out, 0, noise_std,
+                               seed, step, y.layer_id, reinterpret_cast<uint32_t*>(ws), stream, &deferred)) != DP_OK)
           return st;
       }
     }

@@ -260,21 +260,22 @@ __global__ void finalize_norms_kernel(NormSource src, int B, float C, float* __r
 constexpr long long kScaleFusedPartialSlots = 1 << 16;  // samples * count per block, at most
 constexpr int kScaleFusedMaxSamples = 4096;              // samples one block may cover
 
-__global__ void scale_rows_bf16_kernel(const __nv_bfloat16* __restrict__ in,
-                                       __nv_bfloat16* __restrict__ out, long long rows, int cols,
-                                       int T, NormSource src, PartialsRef pr, float C) {
-  griddep_enter();
+// The work of block `blk` of `nblk` blocks (the kernel's own grid, or a segment's share of a
+// batched grid).
+__device__ __forceinline__ void scale_rows_body(const __nv_bfloat16* __restrict__ in, __nv_bfloat16* __restrict__ out,
+                                                long long rows, int cols, int T, const NormSource& src,
+                                                const PartialsRef& pr, float C, long long blk, long long nblk) {
   extern __shared__ float scale_c[];  // with pr.partials: c of samples s_lo .. s_hi
   const int vec_per_row = cols / 8;
   const long long total = rows * vec_per_row;
-  long long v_begin = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x;
+  long long v_begin = blk * static_cast<long long>(blockDim.x) + threadIdx.x;
   long long v_end = total;
-  long long v_step = static_cast<long long>(gridDim.x) * blockDim.x;
+  long long v_step = nblk * blockDim.x;
   int s_lo = 0;
   uint4 first = make_uint4(0u, 0u, 0u, 0u);  // fused path: this thread's first vector, loaded early
   if (pr.partials != nullptr) {
-    const long long per = (total + gridDim.x - 1) / gridDim.x;
-    const long long v0 = blockIdx.x * per < total ? blockIdx.x * per : total;
+    const long long per = (total + nblk - 1) / nblk;
+    const long long v0 = blk * per < total ? blk * per : total;
     const long long v1 = v0 + per < total ? v0 + per : total;
     const long long sample_vecs = static_cast<long long>(T) * vec_per_row;
     // The load is in flight while one warp per sample sums the partials.
@@ -321,6 +322,43 @@ __global__ void scale_rows_bf16_kernel(const __nv_bfloat16* __restrict__ in,
     }
     reinterpret_cast<uint4*>(out)[v] = res;
   }
+}
+
+__global__ void scale_rows_bf16_kernel(const __nv_bfloat16* __restrict__ in,
+                                       __nv_bfloat16* __restrict__ out, long long rows, int cols,
+                                       int T, NormSource src, PartialsRef pr, float C) {
+  griddep_enter();
+  scale_rows_body(in, out, rows, cols, T, src, pr, C, blockIdx.x, gridDim.x);
+}
+
+// The row scalings of several layers in one launch (a per-layer block step scales every
+// layer's narrower operand after all the norm passes): segment q takes blocks
+// [first_block, first_block + blocks) of the grid and is scaled as scale_rows_bf16_kernel
+// would with that many blocks, each block summing its samples' norm partials itself.
+constexpr int kMaxScaleSegments = 16;
+struct ScaleSegment {
+  const __nv_bfloat16* in;
+  __nv_bfloat16* out;
+  long long rows;
+  int cols;
+  PartialsRef pr;   // pr.partials null: the clip factors come from src
+  NormSource src;
+  float C;
+  int first_block, blocks;
+};
+struct ScaleBatch {
+  ScaleSegment seg[kMaxScaleSegments];
+  int count;
+  int T;
+};
+
+__global__ void scale_rows_bf16_batch_kernel(ScaleBatch b) {
+  griddep_enter();
+  int q = 0;
+  while (q + 1 < b.count && static_cast<int>(blockIdx.x) >= b.seg[q + 1].first_block) ++q;
+  const ScaleSegment& sg = b.seg[q];
+  if (!DP_DCHECK(static_cast<int>(blockIdx.x) - sg.first_block < sg.blocks, 27u, nullptr)) return;
+  scale_rows_body(sg.in, sg.out, sg.rows, sg.cols, b.T, sg.src, sg.pr, sg.C, blockIdx.x - sg.first_block, sg.blocks);
 }
 
 // out[e] = fp32(sum_i c_i Gs[i][e] + std * z_e) over the per-sample bf16 gradients that the
@@ -414,9 +452,11 @@ __global__ void __launch_bounds__(256, 2) clip_reduce_kernel(
       for (int q = 0; q < 8; ++q) acc[q] = acc[q] + z[q];
     }
     if (!DP_DCHECK(in_buffer(8 * v, 8, mn), 23u, nullptr)) break;
+    // Streaming stores (evict first), like the loads: beside a tensor-core pass they should not
+    // push that pass's operand tiles out of L2.
     float4* o = reinterpret_cast<float4*>(out) + 2 * v;
-    o[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-    o[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+    __stcs(o, make_float4(acc[0], acc[1], acc[2], acc[3]));
+    __stcs(o + 1, make_float4(acc[4], acc[5], acc[6], acc[7]));
   }
 }
 
