@@ -293,6 +293,23 @@ dp_status launch_umma(const UmmaParams& p, cudaStream_t stream) {
   return DP_OK;
 }
 
+template <class Cfg>
+dp_status launch_umma_group(const UmmaParams& p, const UmmaGroup& g, cudaStream_t stream) {
+  static bool configured[64] = {false};
+  int dev = 0;
+  DP_CUDA(cudaGetDevice(&dev));
+  if (dev >= 0 && dev < 64 && !configured[dev]) {
+    DP_CUDA(cudaFuncSetAttribute(umma_group_kernel<Cfg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Cfg::SMEM_BYTES));
+    configured[dev] = true;
+  }
+  if (p.num_units <= 0) return DP_OK;
+  const int grid = p.num_units < sm_count() ? p.num_units : sm_count();
+  LaunchScope scope(kKindProject, stream);
+  DP_LAUNCH("umma_group_kernel", umma_group_kernel<Cfg>, grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream, p, g);
+  return DP_OK;
+}
+
 UmmaParams base_params(uint32_t* status) {
   UmmaParams p;
   memset(&p, 0, sizeof(p));
@@ -590,28 +607,33 @@ constexpr int kReduceNoise = kGradientNoise;
 // pass, tables through the cache and the sample loop unrolled for B <= 8.
 template <int BU>
 dp_status reduce_plain_launch(int grid, size_t smem, cudaStream_t stream, const __nv_bfloat16* gs, int B,
-                              long long mn, NormSource src, float C, float* out, double noise_std, PhiloxKey key,
-                              unsigned layer_id, StepRef step) {
+                              long long mn, NormSource src, const PartialsRef& pr, float C, float* out,
+                              double noise_std, PhiloxKey key, unsigned layer_id, StepRef step) {
   constexpr bool kStaged = (BU == 0);
   DP_LAUNCH("clip_reduce_kernel", clip_reduce_kernel<kReduceNoise, kStaged, BU>, grid, 256, smem, stream, gs, B, mn,
-            src, C, out, noise_std, key, layer_id, step);
+            src, pr, C, out, noise_std, key, layer_id, step);
   return DP_OK;
 }
 
+// `pr` is used by the unrolled form only (its blocks sum the partials themselves).
 dp_status reduce_kernel_launch(int grid, size_t smem, cudaStream_t stream, const __nv_bfloat16* gs, int B,
-                          long long mn, NormSource src, float C, float* out, double noise_std, PhiloxKey key,
-                          unsigned layer_id, StepRef step, bool staged) {
-  if (staged) return reduce_plain_launch<0>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step);
+                          long long mn, NormSource src, const PartialsRef& pr, float C, float* out,
+                          double noise_std, PhiloxKey key, unsigned layer_id, StepRef step, bool staged) {
+  const PartialsRef none{nullptr, 0, 0, nullptr, nullptr, nullptr};
+#define DP_REDUCE_PLAIN(BU_, PR_) \
+  reduce_plain_launch<BU_>(grid, smem, stream, gs, B, mn, src, PR_, C, out, noise_std, key, layer_id, step)
+  if (staged) return DP_REDUCE_PLAIN(0, none);
   switch (B) {  // coresident: B <= 8 (larger batches keep the staged runtime loop)
-    case 1: return reduce_plain_launch<1>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step);
-    case 2: return reduce_plain_launch<2>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step);
-    case 3: return reduce_plain_launch<3>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step);
-    case 4: return reduce_plain_launch<4>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step);
-    case 5: return reduce_plain_launch<5>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step);
-    case 6: return reduce_plain_launch<6>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step);
-    case 7: return reduce_plain_launch<7>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step);
-    default: return reduce_plain_launch<8>(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step);
+    case 1: return DP_REDUCE_PLAIN(1, pr);
+    case 2: return DP_REDUCE_PLAIN(2, pr);
+    case 3: return DP_REDUCE_PLAIN(3, pr);
+    case 4: return DP_REDUCE_PLAIN(4, pr);
+    case 5: return DP_REDUCE_PLAIN(5, pr);
+    case 6: return DP_REDUCE_PLAIN(6, pr);
+    case 7: return DP_REDUCE_PLAIN(7, pr);
+    default: return DP_REDUCE_PLAIN(8, pr);
   }
+#undef DP_REDUCE_PLAIN
 }
 
 template <int BU>
@@ -663,7 +685,11 @@ dp_status launch_reduce(const __nv_bfloat16* gs, int B, long long mn, NormSource
     if (st != DP_OK) return st;
     return DP_OK;
   }
-  if (partials) {
+  const bool unrolled = coresident && B <= 8;
+  PartialsRef pr{nullptr, 0, 0, nullptr, nullptr, nullptr};
+  if (partials && unrolled) {
+    pr = *partials;  // the unrolled reduce sums them in its prologue
+  } else if (partials) {
     dp_status st = launch_norm_partials(partials->partials, partials->stride, partials->count, B, C,
                                         partials->norm2, partials->norms_out, partials->c_out, stream);
     if (st != DP_OK) return st;
@@ -672,13 +698,12 @@ dp_status launch_reduce(const __nv_bfloat16* gs, int B, long long mn, NormSource
   const int cached = B < kReduceCachedSamples ? B : kReduceCachedSamples;
   // Beside a tensor-core pass one block per SM: two would take more registers than an SM has
   // next to a tensor-core CTA, and the next pass would wait for them.
-  const bool unrolled = coresident && B <= 8;
   const int grid = std::min(stream_grid(static_cast<unsigned long long>(mn / 8), 256),
                             coresident ? sm_count() : sm_count() * 2);
   const size_t smem = (unrolled ? 0 : kNoiseSharedBytes) + cached * sizeof(float);
   const PhiloxKey key = philox_key_from_seed(seed);
   LaunchScope scope(kKindReduce, stream);
-  return reduce_kernel_launch(grid, smem, stream, gs, B, mn, src, C, out, noise_std, key, layer_id, step,
+  return reduce_kernel_launch(grid, smem, stream, gs, B, mn, src, pr, C, out, noise_std, key, layer_id, step,
                               !unrolled);
 }
 
@@ -838,6 +863,7 @@ struct BlockLayout {
   bool batched_scale = false;
   std::vector<size_t> scaled_l;          // per layer: its scaled copy (batched schedule), or 0
   std::vector<long long> partial_set;    // per layer: its norm-partial set (batched schedule)
+  bool z_grouped = false;                // bf16 projected layers: every Z formed in grouped launches
 };
 
 constexpr size_t kBatchScaleBytes = size_t(256) << 20;
@@ -1047,6 +1073,8 @@ BlockLayout block_layout(const dp_layer* layers, int L, int B, int T, dp_dtype d
   }
   // Each projected layer keeps its Z = dY P from its norms to its clipped sum.
   Lb.z.assign(L, 0);
+  Lb.z_grouped = false;
+  for (int l = 0; l < L; ++l) Lb.z_grouped = Lb.z_grouped || (dt == DP_BF16 && layers[l].P);
   for (int l = 0; l < L; ++l) {
     if (layers[l].P) {
       Lb.z[l] = off;
@@ -1068,7 +1096,7 @@ dp_status block_operand(const dp_layer* layers, int l, dp_dtype dt, int B, int T
   }
   void* z = ws + Lb.z[l];
   *Z = z;
-  if (!form) return DP_OK;
+  if (!form || Lb.z_grouped) return DP_OK;  // grouped: formed at the start of the step
   const Shape s = layer_shape(y, B, T, dt);
   if (dt == DP_BF16) return bf16_project(s, y.dY, y.P, z, reinterpret_cast<uint32_t*>(ws), stream);
   const long long total = s.N() * s.r;
@@ -1076,6 +1104,55 @@ dp_status block_operand(const dp_layer* layers, int l, dp_dtype dt, int B, int T
   DP_LAUNCH("f32_project_kernel", f32_project_kernel, stream_grid(total, 256), 256, 0, stream,
             static_cast<const float*>(y.dY), static_cast<const float*>(y.P), static_cast<float*>(z), s.N(),
             s.n, s.r);
+  return DP_OK;
+}
+
+// Z_l = dY_l P_l of every bf16 projected layer, in one grouped tensor-core launch per chunk of
+// up to kMaxGroup layers with the same r (the DP-GRAPE projection of a block, formed once).
+dp_status block_projections(const dp_layer* layers, int L, dp_dtype dt, int B, int T, const BlockLayout& Lb,
+                            uint8_t* ws, cudaStream_t stream) {
+  if (!Lb.z_grouped) return DP_OK;
+  std::vector<bool> done(L, false);
+  const long long N = static_cast<long long>(B) * T;
+  const int m_tiles = ceil_div(N, 128);
+  for (int l0 = 0; l0 < L; ++l0) {
+    if (done[l0] || !layers[l0].P) continue;
+    const int r = layers[l0].r;
+    std::vector<int> chunk;
+    for (int l = l0; l < L && static_cast<int>(chunk.size()) < kMaxGroup; ++l)
+      if (!done[l] && layers[l].P && layers[l].r == r) chunk.push_back(l);
+    const int count = static_cast<int>(chunk.size());
+    // 128 x 64 tiles when 128 x 128 tiles would leave more than half the SMs idle.
+    const int bn = (r <= 64 || (r <= 128 && count * m_tiles * 2 <= sm_count())) ? 64 : (r <= 128 ? 128 : 256);
+    UmmaParams p = base_params(reinterpret_cast<uint32_t*>(ws));
+    UmmaGroup g;
+    memset(&g, 0, sizeof(g));
+    g.count = count;
+    p.m_tiles = m_tiles;
+    p.n_tiles = ceil_div(r, bn);
+    p.k_splits = 1;
+    p.out_rows = static_cast<int>(N);
+    p.out_cols = r;
+    p.out_elems = N * r;
+    int units = 0;
+    dp_status st;
+    for (int q = 0; q < count; ++q) {
+      const dp_layer& y = layers[chunk[q]];
+      if ((st = map_2d(&g.tmA[q], y.dY, N, y.d_out, 128)) != DP_OK) return st;
+      if ((st = map_2d(&g.tmB[q], y.P, y.d_out, r, 64)) != DP_OK) return st;
+      g.out_bf16[q] = reinterpret_cast<__nv_bfloat16*>(ws + Lb.z[chunk[q]]);
+      g.k_blocks[q] = ceil_div(y.d_out, 64);
+      g.unit_begin[q] = units;
+      units += p.m_tiles * p.n_tiles;
+      done[chunk[q]] = true;
+    }
+    g.unit_begin[count] = units;
+    p.num_units = units;
+    if (bn == 64) st = launch_umma_group<UmmaConfig<64, kEpiStoreBf16, true>>(p, g, stream);
+    else if (bn == 128) st = launch_umma_group<UmmaConfig<128, kEpiStoreBf16, true>>(p, g, stream);
+    else st = launch_umma_group<UmmaConfig<256, kEpiStoreBf16, true>>(p, g, stream);
+    if (st != DP_OK) return st;
+  }
   return DP_OK;
 }
 
@@ -1229,6 +1306,8 @@ dp_status block_step(const dp_layer* layers, int L, dp_dtype dt, int B, int T, d
   dp_status st;
   // Status word, and the fp32 path's atomic norm accumulators, start at zero.
   DP_CUDA(cudaMemsetAsync(ws, 0, Lb.c, stream));
+  // Every projected layer's Z = dY P, grouped (bf16).
+  if ((st = block_projections(layers, L, dt, B, T, Lb, ws, stream)) != DP_OK) return st;
   // Noise of split-K clipped sums, added in one launch at the end of the step.
   NoiseBatch deferred;
   deferred.count = 0;

@@ -390,9 +390,12 @@ __device__ __forceinline__ void noise8_f32(uint32_t blk0, uint32_t layer_id, uin
 // BU > 0: exactly BU samples, unrolled: each thread issues all BU loads of its 8 elements,
 // computes their noise while the loads are in flight, then forms the weighted sum.  BU = 0: a
 // runtime loop over B samples.
+// With pr.partials (BU > 0 only), warp i of every block first sums sample i's norm partials
+// (the fixed-order routine, so every block gets the same bits) and block 0 writes norm2 /
+// norms_out / c_out, as the bulk-copy reduce does: no separate partials kernel.
 template <int NP, bool STAGED, int BU>
 __global__ void __launch_bounds__(256, 2) clip_reduce_kernel(
-    const __nv_bfloat16* __restrict__ Gs, int B, long long mn, NormSource src, float C,
+    const __nv_bfloat16* __restrict__ Gs, int B, long long mn, NormSource src, PartialsRef pr, float C,
     float* __restrict__ out, double noise_std, PhiloxKey key, uint32_t layer_id, StepRef step) {
   griddep_enter();
   const uint32_t step_lo = step.get();
@@ -400,7 +403,23 @@ __global__ void __launch_bounds__(256, 2) clip_reduce_kernel(
   extern __shared__ double2 reduce_smem[];  // noise tables (STAGED), then the cached clip factors
   float* c_smem = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(reduce_smem) + (STAGED ? NT::kBytes : 0));
   const int cached = B < kReduceCachedSamples ? B : kReduceCachedSamples;
-  for (int i = threadIdx.x; i < cached; i += blockDim.x) c_smem[i] = clip_factor(src.norm(i), C);
+  if (BU > 0 && pr.partials != nullptr) {
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    if (warp < BU) {
+      const float n2 = warp_norm2_from_partials(pr.partials, pr.stride, pr.count, warp, lane);
+      if (lane == 0) {
+        const float n = sqrtf(n2);
+        c_smem[warp] = clip_factor(n, C);
+        if (blockIdx.x == 0) {
+          if (pr.norm2) pr.norm2[warp] = n2;
+          if (pr.norms_out) pr.norms_out[warp] = n;
+          if (pr.c_out) pr.c_out[warp] = c_smem[warp];
+        }
+      }
+    }
+  } else {
+    for (int i = threadIdx.x; i < cached; i += blockDim.x) c_smem[i] = clip_factor(src.norm(i), C);
+  }
   if (STAGED && noise_std != 0.0) NT::stage(reduce_smem);
   __syncthreads();
   using Tab = typename std::conditional<STAGED, typename NT::Shared, typename NT::Global>::type;

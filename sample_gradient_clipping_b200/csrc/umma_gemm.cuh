@@ -84,8 +84,22 @@ struct alignas(64) UmmaParams {
   long long partials_elems;   // floats of the partials buffer (device-side checks; 0 = unknown)
 };
 
-template <int BN_, int EPI_>
+// Several independent problems of one contraction kind in one launch (the projections
+// Z_l = dY_l P_l of a block's projected linears): problem q has its own operand maps, output
+// and K depth, and the units [unit_begin[q], unit_begin[q + 1]) of the launch.  Passed as a
+// second __grid_constant__ parameter, so launches of one problem keep their parameter size.
+constexpr int kMaxGroup = 8;
+struct alignas(64) UmmaGroup {
+  CUtensorMap tmA[kMaxGroup], tmB[kMaxGroup];
+  __nv_bfloat16* out_bf16[kMaxGroup];
+  int k_blocks[kMaxGroup];
+  int unit_begin[kMaxGroup + 1];
+  int count;
+};
+
+template <int BN_, int EPI_, bool GROUPED_ = false>
 struct UmmaConfig {
+  static constexpr bool GROUPED = GROUPED_;  // problems from a UmmaGroup (kEpiStoreBf16 only)
   static constexpr int BM = 128;
   static constexpr int BN = BN_;
   static constexpr int BK = 64;  // 64 bf16 = 128 bytes: one swizzle atom row
@@ -108,16 +122,30 @@ struct UmmaConfig {
   static constexpr uint32_t IDESC = umma_idesc_bf16(BM, BN, A_MN, B_MN);
   static_assert(NUM_BUFS >= 1, "TMEM budget");
   static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN");
+  static_assert(!GROUPED_ || EPI_ == kEpiStoreBf16, "grouped launches serve the projection");
 };
 
 struct Unit {
   int m_blk, n_blk, kb_begin, kb_end, sample, split;
   int local;  // index of the unit among the units of its sample (norm partial slots)
+  int prob;   // grouped launch: the problem of the unit
 };
 
 template <class Cfg>
-__device__ __forceinline__ Unit decode_unit(const UmmaParams& p, int u) {
+__device__ __forceinline__ Unit decode_unit(const UmmaParams& p, int u, const UmmaGroup* grp = nullptr) {
   Unit w{};
+  if constexpr (Cfg::GROUPED) {
+    // Problem q owns units unit_begin[q] .. unit_begin[q+1]-1, row-tile-major, n_tiles each row.
+    int q = 0;
+    while (q + 1 < grp->count && u >= grp->unit_begin[q + 1]) ++q;
+    const int r = u - grp->unit_begin[q];
+    w.prob = q;
+    w.m_blk = r / p.n_tiles;
+    w.n_blk = r % p.n_tiles;
+    w.kb_begin = 0;
+    w.kb_end = grp->k_blocks[q];
+    return w;
+  }
   if (Cfg::GHOST) {
     w.sample = u / p.pairs_per_sample;
     int r = u % p.pairs_per_sample;
@@ -164,8 +192,15 @@ __device__ __forceinline__ Unit decode_unit(const UmmaParams& p, int u) {
 template <class Cfg>
 __device__ __forceinline__ void issue_stage_loads(const UmmaParams& p, const Unit& w, int phase,
                                                   int kb, uint32_t sA, uint32_t sB,
-                                                  uint32_t bar) {
+                                                  uint32_t bar, const UmmaGroup* grp = nullptr) {
   const int k0 = kb * Cfg::BK;
+  if constexpr (Cfg::GROUPED) {  // kEpiStoreBf16 per problem: A = dY rows (K-major), B = P (MN-major)
+    tma_load_2d(sA, &grp->tmA[w.prob], bar, k0, w.m_blk * Cfg::BM);
+#pragma unroll
+    for (int h = 0; h < Cfg::BN / 64; ++h)
+      tma_load_2d(sB + h * (Cfg::BK * 128), &grp->tmB[w.prob], bar, w.n_blk * Cfg::BN + 64 * h, k0);
+    return;
+  }
   if (Cfg::EPI == kEpiClipSum) {
 #pragma unroll
     for (int h = 0; h < Cfg::BM / 64; ++h)
@@ -232,7 +267,7 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 template <class Cfg>
 __device__ __forceinline__ void epilogue_unit(const UmmaParams& p, const Unit& w, uint32_t tacc,
-                                              int wq, uint32_t lane) {
+                                              int wq, uint32_t lane, const UmmaGroup* grp = nullptr) {
   const int row = wq * 32 + static_cast<int>(lane);
   if (Cfg::EPI == kEpiClipSum) {
     const long long grow = static_cast<long long>(w.m_blk) * Cfg::BM + row;
@@ -405,7 +440,7 @@ __device__ __forceinline__ void epilogue_unit(const UmmaParams& p, const Unit& w
       tmem_ld_wait();
       const long long gcol0 = static_cast<long long>(w.n_blk) * Cfg::BN + c0;
       if (grow >= p.out_rows) continue;  // the next tmem_ld32 reconverges first
-      __nv_bfloat16* dst = p.out_bf16 + grow * p.out_cols + gcol0;
+      __nv_bfloat16* dst = (Cfg::GROUPED ? grp->out_bf16[w.prob] : p.out_bf16) + grow * p.out_cols + gcol0;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         if (gcol0 + 8 * q >= p.out_cols) break;  // out_cols is a multiple of 8
@@ -421,7 +456,7 @@ __device__ __forceinline__ void epilogue_unit(const UmmaParams& p, const Unit& w
 }
 
 template <class Cfg>
-__global__ void __launch_bounds__(Cfg::THREADS, 1) umma_kernel(const __grid_constant__ UmmaParams p) {
+__device__ __forceinline__ void umma_body(const UmmaParams& p, const UmmaGroup* grp) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -449,8 +484,15 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1) umma_kernel(const __grid_cons
     mbar_init(smem_addr(drain), 1);
     *abort_flag = 0;
     fence_mbar_init();
-    tma_prefetch_desc(&p.tmA0);
-    tma_prefetch_desc(&p.tmB0);
+    if constexpr (Cfg::GROUPED) {
+      for (int q = 0; q < grp->count; ++q) {
+        tma_prefetch_desc(&grp->tmA[q]);
+        tma_prefetch_desc(&grp->tmB[q]);
+      }
+    } else {
+      tma_prefetch_desc(&p.tmA0);
+      tma_prefetch_desc(&p.tmB0);
+    }
     if (Cfg::GHOST) {
       tma_prefetch_desc(&p.tmA1);
       tma_prefetch_desc(&p.tmB1);
@@ -474,7 +516,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1) umma_kernel(const __grid_cons
       uint32_t phase = 0;
       bool ok = true;
       for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
-        const Unit w = decode_unit<Cfg>(p, u);
+        const Unit w = decode_unit<Cfg>(p, u, grp);
         for (int ph = 0; ok && ph < nphases; ++ph) {
           const int kb_end = ph ? p.k_blocks1 : w.kb_end;
           const int kb_begin = ph ? 0 : w.kb_begin;
@@ -486,7 +528,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1) umma_kernel(const __grid_cons
             const uint32_t sA = smem_addr(smem + stage * Cfg::STAGE_BYTES);
             const uint32_t bar = smem_addr(full + stage);
             mbar_arrive_expect_tx(bar, Cfg::STAGE_BYTES);
-            issue_stage_loads<Cfg>(p, w, ph, kb, sA, sA + Cfg::A_BYTES, bar);
+            issue_stage_loads<Cfg>(p, w, ph, kb, sA, sA + Cfg::A_BYTES, bar, grp);
             if (Cfg::EPI == kEpiClipSum) {
               if (kb == kb_begin) {
                 for (int d = 1; d <= kL2PrefetchDistance && kb + d < kb_end; ++d)
@@ -512,7 +554,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1) umma_kernel(const __grid_cons
       uint32_t buf_phase = 0;
       bool ok = true;
       for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
-        const Unit w = decode_unit<Cfg>(p, u);
+        const Unit w = decode_unit<Cfg>(p, u, grp);
         if (!mbar_wait_bounded(smem_addr(acc_empty + buf), buf_phase ^ 1u, abort_flag, p.status, 2u)) {
           ok = false;
           break;
@@ -566,11 +608,11 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1) umma_kernel(const __grid_cons
     int buf = 0;
     uint32_t buf_phase = 0;
     for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
-      const Unit w = decode_unit<Cfg>(p, u);
+      const Unit w = decode_unit<Cfg>(p, u, grp);
       if (!mbar_wait_bounded(smem_addr(acc_full + buf), buf_phase, abort_flag, p.status, 4u)) break;
       tc_fence_after();
       const uint32_t tacc = tmem_base + buf * Cfg::ACC_COLS + (static_cast<uint32_t>(wq * 32) << 16);
-      epilogue_unit<Cfg>(p, w, tacc, wq, lane);
+      epilogue_unit<Cfg>(p, w, tacc, wq, lane, grp);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_addr(acc_empty + buf));
@@ -586,6 +628,17 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1) umma_kernel(const __grid_cons
     tc_fence_after();
     tmem_dealloc(tmem_base, 512);
   }
+}
+
+template <class Cfg>
+__global__ void __launch_bounds__(Cfg::THREADS, 1) umma_kernel(const __grid_constant__ UmmaParams p) {
+  umma_body<Cfg>(p, nullptr);
+}
+
+template <class Cfg>
+__global__ void __launch_bounds__(Cfg::THREADS, 1)
+    umma_group_kernel(const __grid_constant__ UmmaParams p, const __grid_constant__ UmmaGroup g) {
+  umma_body<Cfg>(p, &g);
 }
 
 }  // namespace dpclip

@@ -100,6 +100,7 @@ __device__ __forceinline__ void umma_commit_pair_local(uint32_t bar) {
 
 template <int EPI_>
 struct Umma2Config {
+  static constexpr bool GROUPED = false;
   static constexpr int BM = 128;     // rows per CTA (256 per pair)
   static constexpr int BN = 256;     // columns of the pair's tile (each CTA loads half)
   static constexpr int BK = 64;
