@@ -1320,7 +1320,8 @@ dp_status block_step(const dp_layer* layers, int L, dp_dtype dt, int B, int T, d
     cudaStream_t side = stream;
     if (Lb.overlap && (st = side_stream(&side)) != DP_OK) return st;
     cudaEvent_t reduce_done[2] = {nullptr, nullptr};
-    int once_k = 0;
+    int once_k = 0, once_n = 0;
+    for (const auto& g : Lb.groups) once_n += (dt == DP_BF16 && Lb.methods[g[0]] == DP_NORM_ONCE) ? 1 : 0;
     bool side_pending = false;  // reduces on the side stream the caller's stream has not joined
     std::vector<int> batch_layers, batch_counts;  // batched schedule: layers waiting for their sums
     // Each group: its norms, then each member's clipped sum with its own bound and noise.
@@ -1342,12 +1343,15 @@ dp_status block_step(const dp_layer* layers, int L, dp_dtype dt, int B, int T, d
         float* n2 = reinterpret_cast<float*>(ws + Lb.norm2) + static_cast<size_t>(g[0]) * B;
         const PartialsRef pr{partials, Lb.partial_stride, count, n2, y.norms_out, nullptr};
         const double noise_std = (sigma == 0.0f) ? 0.0 : static_cast<double>(sigma) * static_cast<double>(y.C);
-        if (Lb.overlap && (st = stream_after(side, stream)) != DP_OK) return st;
+        // The last gradients-once reduce has no tensor-core pass beside it: it takes the whole
+        // GPU, on the caller's stream, with the bulk-copy kernel.
+        const bool beside = Lb.overlap && once_k + 1 < once_n;
+        if (beside && (st = stream_after(side, stream)) != DP_OK) return st;
         if ((st = launch_reduce(tiles, B, static_cast<long long>(s.m) * s.ne(), layer_norm_source(Lb, ws, g[0], B, dt),
-                                y.C, y.G_out, noise_std, seed, step, y.layer_id, side,
-                                reinterpret_cast<uint32_t*>(ws), &pr, Lb.overlap)) != DP_OK)
+                                y.C, y.G_out, noise_std, seed, step, y.layer_id, beside ? side : stream,
+                                reinterpret_cast<uint32_t*>(ws), &pr, beside)) != DP_OK)
           return st;
-        if (Lb.overlap) {
+        if (beside) {
           if ((st = event_ring().next(&reduce_done[par])) != DP_OK) return st;
           DP_CUDA(cudaEventRecord(reduce_done[par], side));
           side_pending = true;
