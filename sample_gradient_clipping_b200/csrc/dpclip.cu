@@ -410,54 +410,79 @@ dp_status bf16_norms_ghost_shared(const Shape& s, const void* X, const void* con
 dp_status launch_noise(float* G, unsigned long long total, double std_dev, unsigned long long seed,
                        StepRef step, unsigned layer_id, cudaStream_t stream);
 
-// out (+)= A^T Bm over all N rows (A: [N, m], Bm: [N, ne], both bf16, one already scaled by
-// c_i), plus noise when noise_std != 0.  `accumulate` = 0 overwrites out.
-// With `defer` (a block step), noise that cannot ride in the epilogue (split K) is queued
-// there instead of launched.
-dp_status bf16_clipsum(const Shape& s, const void* A, const void* Bm, float* out, int accumulate,
-                       double noise_std, unsigned long long seed, StepRef step,
-                       unsigned layer_id, uint32_t* status, cudaStream_t stream,
-                       NoiseBatch* defer = nullptr) {
-  UmmaParams p = base_params(status);
+// How the clipped-sum contraction of shape s is tiled: SM-pair tiles or not, and into how many
+// K splits (a split-K sum lands by fp32 atomics).
+struct ClipSumPlan {
+  bool pair;
+  int bn, m_tiles, n_tiles, k_blocks, k_blocks_per_split, splits;
+};
+
+ClipSumPlan clipsum_plan(const Shape& s) {
+  ClipSumPlan c;
   const int ne = s.ne();
-  const int BN = ne <= 128 ? 128 : 256;
+  c.bn = ne <= 128 ? 128 : 256;
   // 256 x 256 tiles on SM pairs when both output dimensions fill them: half the operand
   // traffic per SM of a 128 x 256 one-SM tile.
-  const bool pair = (s.m >= 256 && ne >= 256);
-  dp_status st;
-  if ((st = map_2d(&p.tmA0, A, s.N(), s.m, 64)) != DP_OK) return st;
-  if ((st = map_2d(&p.tmB0, Bm, s.N(), ne, 64)) != DP_OK) return st;
-  p.m_tiles = pair ? ceil_div(s.m, 256) : ceil_div(s.m, 128);
-  p.n_tiles = ceil_div(ne, BN);
-  p.k_blocks = ceil_div(s.N(), 64);
-  const int tiles = p.m_tiles * p.n_tiles;
-  const int slots = pair ? sm_count() / 2 : sm_count();  // CTAs (or pairs) that run at once
+  c.pair = (s.m >= 256 && ne >= 256);
+  c.m_tiles = c.pair ? ceil_div(s.m, 256) : ceil_div(s.m, 128);
+  c.n_tiles = ceil_div(ne, c.bn);
+  c.k_blocks = ceil_div(s.N(), 64);
+  const int tiles = c.m_tiles * c.n_tiles;
+  const int slots = c.pair ? sm_count() / 2 : sm_count();  // CTAs (or pairs) that run at once
   int splits = 1;
   if (tiles < slots) {
     splits = slots / tiles;
-    const int max_splits = p.k_blocks / 4 > 0 ? p.k_blocks / 4 : 1;
+    const int max_splits = c.k_blocks / 4 > 0 ? c.k_blocks / 4 : 1;
     if (splits > max_splits) splits = max_splits;
     if (splits < 1) splits = 1;
   }
-  p.k_blocks_per_split = ceil_div(p.k_blocks, splits);
-  splits = ceil_div(p.k_blocks, p.k_blocks_per_split);  // every split non-empty
+  c.k_blocks_per_split = ceil_div(c.k_blocks, splits);
+  c.splits = ceil_div(c.k_blocks, c.k_blocks_per_split);  // every split non-empty
+  return c;
+}
+
+// out (+)= A^T Bm over all N rows (A: [N, m], Bm: [N, ne], both bf16, one already scaled by
+// c_i), plus noise when noise_std != 0.  `accumulate` = 0 overwrites out.
+// With `defer` (a block step), noise that cannot ride in the epilogue (split K) is queued
+// there instead of launched.  With `preset` (split K only), out already holds the noise
+// (written by a noise launch in SET mode) and the partial sums are added to it.
+dp_status bf16_clipsum(const Shape& s, const void* A, const void* Bm, float* out, int accumulate,
+                       double noise_std, unsigned long long seed, StepRef step,
+                       unsigned layer_id, uint32_t* status, cudaStream_t stream,
+                       NoiseBatch* defer = nullptr, bool preset = false) {
+  UmmaParams p = base_params(status);
+  const int ne = s.ne();
+  const ClipSumPlan plan = clipsum_plan(s);
+  const int BN = plan.bn;
+  const bool pair = plan.pair;
+  dp_status st;
+  if ((st = map_2d(&p.tmA0, A, s.N(), s.m, 64)) != DP_OK) return st;
+  if ((st = map_2d(&p.tmB0, Bm, s.N(), ne, 64)) != DP_OK) return st;
+  p.m_tiles = plan.m_tiles;
+  p.n_tiles = plan.n_tiles;
+  p.k_blocks = plan.k_blocks;
+  const int tiles = p.m_tiles * p.n_tiles;
+  const int splits = plan.splits;
+  p.k_blocks_per_split = plan.k_blocks_per_split;
   p.k_splits = splits;
   p.num_units = tiles * splits;
   p.out_rows = s.m;
   p.out_cols = ne;
   p.out_f32 = out;
   p.out_elems = static_cast<long long>(s.m) * ne;
+  if (preset && (splits == 1 || accumulate)) return DP_ERR_INVALID_ARG;  // the callers never ask this
   if (splits > 1 || accumulate) {
     p.out_mode = (splits > 1) ? kOutAtomicAdd : kOutAdd;
-    if (!accumulate)
+    if (!accumulate && !preset)
       DP_CUDA(cudaMemsetAsync(out, 0, static_cast<size_t>(s.m) * ne * sizeof(float), stream));
   } else {
     p.out_mode = kOutStore;
   }
-  // With split K the partial sums land by atomics; the noise is then added once, after the
-  // sum is complete, so that it is rounded once as in the unsplit epilogue.
+  // With split K the partial sums land by atomics; the noise is then added after the sum is
+  // complete (rounded once, as in the unsplit epilogue), or was written first (preset).
   const bool fused_noise = (splits == 1);
   p.noise_std = fused_noise ? noise_std : 0.0;
+  if (preset) noise_std = 0.0;  // already in out
   const PhiloxKey key = philox_key_from_seed(seed);
   p.key0 = key.k0;
   p.key1 = key.k1;
@@ -477,30 +502,44 @@ dp_status bf16_clipsum(const Shape& s, const void* A, const void* Bm, float* out
                       stream);
 }
 
-dp_status launch_noise_batch(const NoiseBatch& b, unsigned long long seed, StepRef step, cudaStream_t stream) {
+// `set`: write the noise instead of adding it (noise_add_kernel's SET mode).
+dp_status launch_noise_batch(const NoiseBatch& b, unsigned long long seed, StepRef step, cudaStream_t stream,
+                             bool set = false) {
   if (b.count == 0) return DP_OK;
   unsigned long long nblk = 0;
   for (int q = 0; q < b.count; ++q) nblk += (b.seg[q].total + 3) / 4;
   LaunchScope scope(kKindNoise, stream);
-  DP_LAUNCH("noise_add_batch_kernel", noise_add_batch_kernel, stream_grid(nblk, 256), 256, 0, stream, b,
-            philox_key_from_seed(seed), step);
+  if (set)
+    DP_LAUNCH("noise_add_batch_kernel", noise_add_batch_kernel<true>, stream_grid(nblk, 256), 256, 0, stream, b,
+              philox_key_from_seed(seed), step);
+  else
+    DP_LAUNCH("noise_add_batch_kernel", noise_add_batch_kernel<false>, stream_grid(nblk, 256), 256, 0, stream, b,
+              philox_key_from_seed(seed), step);
+  return DP_OK;
+}
+
+dp_status launch_noise(float* G, unsigned long long total, double std_dev, unsigned long long seed,
+                       StepRef step, unsigned layer_id, cudaStream_t stream, bool set) {
+  LaunchScope scope(kKindNoise, stream);
+  // Large G: a persistent grid whose blocks stage the 32 KB of Box-Muller tables once each.
+  const PhiloxKey key = philox_key_from_seed(seed);
+  const bool staged = total >= (1ull << 22);
+  const int grid = staged ? std::min(stream_grid((total + 3) / 4, 256), sm_count() * 4)
+                          : stream_grid((total + 3) / 4, 256);
+#define DP_NOISE(ST_, SET_)                                                                               \
+  DP_LAUNCH("noise_add_kernel", noise_add_kernel<ST_, SET_>, grid, 256, 0, stream, G, total, std_dev, key, \
+            layer_id, step)
+  if (staged && set) DP_NOISE(true, true);
+  else if (staged) DP_NOISE(true, false);
+  else if (set) DP_NOISE(false, true);
+  else DP_NOISE(false, false);
+#undef DP_NOISE
   return DP_OK;
 }
 
 dp_status launch_noise(float* G, unsigned long long total, double std_dev, unsigned long long seed,
                        StepRef step, unsigned layer_id, cudaStream_t stream) {
-  LaunchScope scope(kKindNoise, stream);
-  // Large G: a persistent grid whose blocks stage the 32 KB of Box-Muller tables once each.
-  const PhiloxKey key = philox_key_from_seed(seed);
-  if (total >= (1ull << 22)) {
-    const int grid = std::min(stream_grid((total + 3) / 4, 256), sm_count() * 4);
-    DP_LAUNCH("noise_add_kernel", noise_add_kernel<true>, grid, 256, 0, stream, G, total, std_dev, key,
-              layer_id, step);
-  } else {
-    DP_LAUNCH("noise_add_kernel", noise_add_kernel<false>, stream_grid((total + 3) / 4, 256), 256, 0, stream,
-              G, total, std_dev, key, layer_id, step);
-  }
-  return DP_OK;
+  return launch_noise(G, total, std_dev, seed, step, layer_id, stream, false);
 }
 
 // Z[N, r] = dY[N, n] P[n, r], bf16 out.
@@ -796,7 +835,9 @@ NormSource ws_norm_source(const Call& c) {
 dp_status clipped_sum(Call& c, const void* X, const void* Z, NormSource src, float C, float* out,
                       int accumulate, double noise_std, unsigned long long seed,
                       StepRef step, unsigned layer_id, NoiseBatch* defer = nullptr,
-                      const PartialsRef* partials = nullptr) {
+                      const PartialsRef* partials = nullptr, cudaEvent_t noise_written = nullptr) {
+  // noise_written: out already holds the noise (split K), written on another stream; the
+  // contraction waits for that event and adds its partial sums to it.
   const Shape& s = c.s;
   if (s.dt == DP_F32) {
     dim3 grid(ceil_div(s.ne(), kF32Tile), ceil_div(s.m, kF32Tile));
@@ -810,14 +851,17 @@ dp_status clipped_sum(Call& c, const void* X, const void* Z, NormSource src, flo
   // Fold c_i into the narrower operand: one extra read + write of N * min(m, ne) bf16.
   void* scaled = c.ws + c.L.scaled;
   dp_status st;
+  const bool preset = (noise_written != nullptr);
   if (s.ne() <= s.m) {
     if ((st = launch_scale(Z, scaled, s.N(), s.ne(), s.T, src, C, c.stream, partials, s.B)) != DP_OK) return st;
+    if (preset) DP_CUDA(cudaStreamWaitEvent(c.stream, noise_written, 0));
     return bf16_clipsum(s, X, scaled, out, accumulate, noise_std, seed, step, layer_id, c.status(), c.stream,
-                        defer);
+                        defer, preset);
   }
   if ((st = launch_scale(X, scaled, s.N(), s.m, s.T, src, C, c.stream, partials, s.B)) != DP_OK) return st;
+  if (preset) DP_CUDA(cudaStreamWaitEvent(c.stream, noise_written, 0));
   return bf16_clipsum(s, scaled, Z, out, accumulate, noise_std, seed, step, layer_id, c.status(), c.stream,
-                      defer);
+                      defer, preset);
 }
 
 dp_status resolve_method(const Shape& s, dp_norm_method method, dp_norm_method* out) {
@@ -1324,6 +1368,33 @@ dp_status block_step(const dp_layer* layers, int L, dp_dtype dt, int B, int T, d
     for (const auto& g : Lb.groups) once_n += (dt == DP_BF16 && Lb.methods[g[0]] == DP_NORM_ONCE) ? 1 : 0;
     bool side_pending = false;  // reduces on the side stream the caller's stream has not joined
     std::vector<int> batch_layers, batch_counts;  // batched schedule: layers waiting for their sums
+    // Batched schedule: the noise of every split-K clipped sum is written into its output first,
+    // in one launch on the second stream beside the norm passes; those sums then add to it.
+    std::vector<bool> preset(L, false);
+    cudaEvent_t noise_written = nullptr;
+    if (Lb.batched_scale && sigma != 0.0f) {
+      NoiseBatch nb;
+      nb.count = 0;
+      for (const auto& g : Lb.groups) {
+        if (Lb.methods[g[0]] == DP_NORM_ONCE) continue;
+        for (int l : g) {
+          const Shape s = layer_shape(layers[l], B, T, dt);
+          if (clipsum_plan(s).splits > 1 && nb.count < kMaxNoiseSegments) {
+            nb.seg[nb.count++] = NoiseSegment{layers[l].G_out, static_cast<unsigned long long>(s.m) * s.ne(),
+                                              static_cast<double>(sigma) * static_cast<double>(layers[l].C),
+                                              layers[l].layer_id};
+            preset[l] = true;
+          }
+        }
+      }
+      if (nb.count > 0) {
+        if (!Lb.overlap && (st = side_stream(&side)) != DP_OK) return st;
+        if ((st = stream_after(side, stream)) != DP_OK) return st;  // fork
+        if ((st = launch_noise_batch(nb, seed, step, side, true)) != DP_OK) return st;
+        if ((st = event_ring().next(&noise_written)) != DP_OK) return st;
+        DP_CUDA(cudaEventRecord(noise_written, side));
+      }
+    }
     // Each group: its norms, then each member's clipped sum with its own bound and noise.
     for (const auto& g : Lb.groups) {
       if (dt == DP_BF16 && Lb.methods[g[0]] == DP_NORM_ONCE) {
@@ -1401,8 +1472,13 @@ dp_status block_step(const dp_layer* layers, int L, dp_dtype dt, int B, int T, d
         if ((st = block_operand(layers, l, dt, B, T, Lb, ws, stream, false, &Z)) != DP_OK) return st;
         const void* scaled = ws + Lb.scaled_l[l];
         const double noise_std = (sigma == 0.0f) ? 0.0 : static_cast<double>(sigma) * static_cast<double>(y.C);
+        if (preset[l] && noise_written) {  // join the second stream once, before the first such sum
+          DP_CUDA(cudaStreamWaitEvent(stream, noise_written, 0));
+          noise_written = nullptr;
+        }
         if ((st = bf16_clipsum(s, s.ne() <= s.m ? y.X : scaled, s.ne() <= s.m ? scaled : Z, y.G_out, 0, noise_std,
-                               seed, step, y.layer_id, reinterpret_cast<uint32_t*>(ws), stream, &deferred)) != DP_OK)
+                               seed, step, y.layer_id, reinterpret_cast<uint32_t*>(ws), stream, &deferred,
+                               preset[l])) != DP_OK)
           return st;
       }
     }
@@ -1619,6 +1695,19 @@ dp_status linear_step(const void* X, const void* dY, const void* P, int r, dp_dt
                          c.status(), &pr);
   }
   if (dt == DP_BF16) {
+    // A clipped sum split over K adds its partial sums by atomics: its noise is written into
+    // G_out first, on the library's second stream beside the norm pass and the row scaling.
+    cudaEvent_t noise_written = nullptr;
+    if (noise_std != 0.0 && clipsum_plan(c.s).splits > 1) {
+      cudaStream_t side;
+      if ((st = side_stream(&side)) != DP_OK) return st;
+      if ((st = stream_after(side, c.stream)) != DP_OK) return st;  // fork
+      if ((st = launch_noise(G_out, static_cast<unsigned long long>(mn), noise_std, seed, step, layer_id, side,
+                             true)) != DP_OK)
+        return st;
+      if ((st = event_ring().next(&noise_written)) != DP_OK) return st;
+      DP_CUDA(cudaEventRecord(noise_written, side));
+    }
     // The norm partials are summed by the row-scaling kernel of the clipped sum.
     int count = 0;
     if ((st = bf16_norms(c.s, X, Z, m, c.partials(), c.L.partial_stride, &count, c.status(), c.stream)) !=
@@ -1626,7 +1715,8 @@ dp_status linear_step(const void* X, const void* dY, const void* P, int r, dp_dt
       return st;
     const PartialsRef pr{c.partials(), c.L.partial_stride, count, c.norm2_f32(), norms_out,
                          norms_out ? c.c() : nullptr};
-    return clipped_sum(c, X, Z, ws_norm_source(c), C, G_out, 0, noise_std, seed, step, layer_id, nullptr, &pr);
+    return clipped_sum(c, X, Z, ws_norm_source(c), C, G_out, 0, noise_std, seed, step, layer_id, nullptr, &pr,
+                       noise_written);  // the wait on noise_written joins the second stream
   }
   if ((st = norms_into_ws(c, X, Z, m, C, nullptr)) != DP_OK) return st;
   const NormSource src = ws_norm_source(c);

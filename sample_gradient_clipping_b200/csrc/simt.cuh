@@ -20,7 +20,9 @@ namespace dpclip {
 // G[k] = fp32(G[k] + std * z_k), z from stream 0.  One thread per Philox block of 4 elements.
 // STAGED: the Box-Muller tables are copied to shared memory once per block (large G); else
 // they are read through the read-only cache, which saves the copy's latency on small G.
-template <bool STAGED>
+// SET: G[k] = fp32(std * z_k) instead (the noise written into a buffer that a split-K sum then
+// adds its partial sums to).
+template <bool STAGED, bool SET = false>
 __global__ void noise_add_kernel(float* __restrict__ G, unsigned long long total, double std_dev,
                                  PhiloxKey key, uint32_t layer_id, StepRef step) {
   griddep_enter();
@@ -44,14 +46,18 @@ __global__ void noise_add_kernel(float* __restrict__ G, unsigned long long total
     if (k0 + 3 < total) {
       if (!DP_DCHECK(in_buffer(static_cast<long long>(k0), 4, static_cast<long long>(total)), 20u, nullptr)) continue;
       float4* p = reinterpret_cast<float4*>(G + k0);
-      float4 g = *p;
-      g.x = z.add_to(g.x, 0);
-      g.y = z.add_to(g.y, 1);
-      g.z = z.add_to(g.z, 2);
-      g.w = z.add_to(g.w, 3);
-      *p = g;
+      if constexpr (SET) {
+        *p = make_float4(z.rounded(0), z.rounded(1), z.rounded(2), z.rounded(3));
+      } else {
+        float4 g = *p;
+        g.x = z.add_to(g.x, 0);
+        g.y = z.add_to(g.y, 1);
+        g.z = z.add_to(g.z, 2);
+        g.w = z.add_to(g.w, 3);
+        *p = g;
+      }
     } else {
-      for (int q = 0; q < 4 && k0 + q < total; ++q) G[k0 + q] = z.add_to(G[k0 + q], q);
+      for (int q = 0; q < 4 && k0 + q < total; ++q) G[k0 + q] = SET ? z.rounded(q) : z.add_to(G[k0 + q], q);
     }
   }
 }
@@ -72,6 +78,7 @@ struct NoiseBatch {
   int count;
 };
 
+template <bool SET = false>
 __global__ void noise_add_batch_kernel(NoiseBatch b, PhiloxKey key, StepRef step) {
   griddep_enter();
   const uint32_t step_lo = step.get();
@@ -90,7 +97,7 @@ __global__ void noise_add_batch_kernel(NoiseBatch b, PhiloxKey key, StepRef step
     noise4(z, static_cast<uint32_t>(jj), sg.layer_id, step_lo, key, typename NoiseTables<kGradientNoise>::Global{},
            sg.std_dev, scale_f2(sg.std_dev));
     const unsigned long long k0 = 4 * jj;
-    for (int e = 0; e < 4 && k0 + e < sg.total; ++e) sg.G[k0 + e] = z.add_to(sg.G[k0 + e], e);
+    for (int e = 0; e < 4 && k0 + e < sg.total; ++e) sg.G[k0 + e] = SET ? z.rounded(e) : z.add_to(sg.G[k0 + e], e);
   }
 }
 
