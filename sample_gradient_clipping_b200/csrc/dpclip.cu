@@ -913,11 +913,14 @@ struct BlockLayout {
 constexpr size_t kBatchScaleBytes = size_t(256) << 20;
 
 // Whether a per-layer block step overlaps each gradients-once reduce with the next layer's
-// tensor-core pass (environment DPCLIP_OVERLAP_REDUCE=0 turns it off; read at every call, so
-// a workspace size query and the step that uses it must see the same setting).
+// tensor-core pass.  Off unless the environment sets DPCLIP_OVERLAP_REDUCE=1: measured on the
+// Llama blocks, the reduce beside the pass slows the pass by 7-17% (they share issue slots
+// and L2), which cancels the hidden reduce time (7B 5.59 against 5.61 ms serial, 13B 4.80
+// against 4.60 ms).  Read at every call, so a workspace size query and the step that uses it
+// must see the same setting.
 bool overlap_reduce_enabled() {
   const char* v = getenv("DPCLIP_OVERLAP_REDUCE");
-  return !(v && v[0] == '0');
+  return v && v[0] == '1';
 }
 
 Shape layer_shape(const dp_layer& l, int B, int T, dp_dtype dt) {

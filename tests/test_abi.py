@@ -182,10 +182,10 @@ def test_block_workspace_size_and_host_rejections(L):
     # beside the next layer's tensor-core pass); flat once keeps every layer's tiles
     tiles = 8 * 2 * 4096 * 11008
     one = L.dp_workspace_size_for(8, 2048, 4096, 11008, 0, _lib.DP_BF16, _lib.DP_NORM_ONCE)
-    assert 2 * tiles <= per <= one + tiles
-    os.environ["DPCLIP_OVERLAP_REDUCE"] = "0"        # serial schedule: one region
+    assert tiles <= per <= one                       # serial schedule (the default): one region
+    os.environ["DPCLIP_OVERLAP_REDUCE"] = "1"        # overlapped reduces: two regions
     try:
-        assert tiles <= L.dp_block_workspace_size(lay, 2, 8, 2048, _lib.DP_BF16, 0, _lib.DP_NORM_ONCE) <= one
+        assert 2 * tiles <= L.dp_block_workspace_size(lay, 2, 8, 2048, _lib.DP_BF16, 0, _lib.DP_NORM_ONCE) <= one + tiles
     finally:
         del os.environ["DPCLIP_OVERLAP_REDUCE"]
     assert flat >= 8 * 2 * (4096 * 4096 + 4096 * 11008)

@@ -101,6 +101,7 @@ def test_overlapped_reduces_equal_serial_order(sigma, monkeypatch):
     results must be bitwise those of the serial schedule (DPCLIP_OVERLAP_REDUCE=0)."""
     w, data, dev = _block(seed=6)
     C = 1.0 / math.sqrt(7.0)
+    monkeypatch.setenv("DPCLIP_OVERLAP_REDUCE", "1")
     outs_o, norms_o, _ = _lib.dp_block_step(_layers(w, dev, C), mode="per_layer", sigma=sigma, seed=w.seed,
                                             step=3, method="once")
     monkeypatch.setenv("DPCLIP_OVERLAP_REDUCE", "0")

@@ -63,8 +63,10 @@ def test_linear_step_graph_replays_each_step(method, r):
     assert _lib.dp_workspace_status(ws) == _lib.DP_OK
 
 
-@pytest.mark.parametrize("method", ["ghost", "once"])   # once: reduces on a second stream, joined
-def test_block_step_graph_replays_each_step(method):
+@pytest.mark.parametrize("method,overlap", [("ghost", "0"), ("once", "0"), ("once", "1")])
+def test_block_step_graph_replays_each_step(method, overlap, monkeypatch):
+    # overlap "1": the gradients-once reduces run on a second stream, forked and joined in the graph
+    monkeypatch.setenv("DPCLIP_OVERLAP_REDUCE", overlap)
     w = inputs.Workload("gblk", B=3, T=256, dtype="bf16", linears=inputs._block(0, 256, 384),
                         C=1.0 / math.sqrt(7.0), sigma=0.6, seed=5, dy_var="per_layer")
     d = inputs.generate(w)
