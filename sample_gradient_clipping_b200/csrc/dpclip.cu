@@ -639,9 +639,6 @@ dp_status launch_finalize(NormSource src, int B, float C, float* norms_out, floa
   return DP_OK;
 }
 
-// Precision of the Box-Muller evaluation in the gradients-once reduce.
-constexpr int kReduceNoise = kGradientNoise;
-
 // The plain reduce: staged tables and a runtime sample loop (B > 8), or, beside a tensor-core
 // pass, tables through the cache and the sample loop unrolled for B <= 8.
 template <int BU>
@@ -649,7 +646,7 @@ dp_status reduce_plain_launch(int grid, size_t smem, cudaStream_t stream, const 
                               long long mn, NormSource src, const PartialsRef& pr, float C, float* out,
                               double noise_std, PhiloxKey key, unsigned layer_id, StepRef step) {
   constexpr bool kStaged = (BU == 0);
-  DP_LAUNCH("clip_reduce_kernel", clip_reduce_kernel<kReduceNoise, kStaged, BU>, grid, 256, smem, stream, gs, B, mn,
+  DP_LAUNCH("clip_reduce_kernel", clip_reduce_kernel<kStaged, BU>, grid, 256, smem, stream, gs, B, mn,
             src, pr, C, out, noise_std, key, layer_id, step);
   return DP_OK;
 }
@@ -684,13 +681,13 @@ dp_status reduce_tma_launch(cudaStream_t stream, const __nv_bfloat16* gs, long l
   int dev = 0;
   DP_CUDA(cudaGetDevice(&dev));
   if (dev >= 0 && dev < 64 && !configured[dev]) {
-    DP_CUDA(cudaFuncSetAttribute(clip_reduce_tma_kernel<BU, kReduceNoise>,
+    DP_CUDA(cudaFuncSetAttribute(clip_reduce_tma_kernel<BU>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES));
     configured[dev] = true;
   }
   const long long chunks = (mn + kReduceChunk - 1) / kReduceChunk;
   const int grid = static_cast<int>(chunks < sm_count() ? chunks : sm_count());
-  DP_LAUNCH("clip_reduce_tma_kernel", clip_reduce_tma_kernel<BU, kReduceNoise>, grid, Cfg::THREADS,
+  DP_LAUNCH("clip_reduce_tma_kernel", clip_reduce_tma_kernel<BU>, grid, Cfg::THREADS,
             Cfg::SMEM_BYTES, stream, gs, mn, src, pr, C, out, noise_std, key, layer_id, step, status);
   return DP_OK;
 }

@@ -19,7 +19,6 @@
 // Counter layout: (j, layer_id, step mod 2^32, stream); key: (seed mod 2^32, seed >> 32).
 #pragma once
 #include <cstdint>
-#include <type_traits>
 
 #include "noise_tables.cuh"
 
@@ -194,207 +193,6 @@ __device__ __forceinline__ void box_muller_f64(uint32_t x_even, uint32_t x_odd, 
   sincos_turn(x_odd, tab, c, s);
   z_even = radius * c;
   z_odd = radius * s;
-}
-
-// ---------------------------------------------------------------- fp32 (float-float) form
-// The same transform on the fp32 and integer pipes only.  fp64 arithmetic on this part shares
-// issue with the tensor cores (a kernel that runs fp64 beside tcgen05 MMAs slows them), and
-// fp32 runs at twice its rate, so the noise is generated this way.  Values are carried as
-// unevaluated float-float sums hi + lo where a plain float would lose bits:
-//   * error-free transforms: Knuth's two-sum (TAOCP vol. 2, 4.2.2) for a + b, and the FMA
-//     product error a*b - fl(a*b) = fma(a, b, -fl(a*b)) (Dekker, "A floating-point technique
-//     for extending the available precision", Numer. Math. 1971);
-//   * -2 ln u1: x + 1 = 2^(31 - lz) M' exactly, M' = M 2^-31 in [1, 2); the top 7 fraction bits
-//     pick F_j = 1 + (j + 1/2)/128, the other 24 bits are the exact integer d = (M' - F_j) 2^31,
-//     |d| <= 2^23, so r' = -2 (M' - F_j)/F_j = d (-2^-30 / F_j) is formed in float-float and
-//     -2 ln u1 = 2 e ln 2 - 2 ln F_j + r' + r'^2/4 + r'^3/12 + r'^4/32 (e = lz + 1; the next
-//     term is below 4e-13).  The three large terms are summed with two-sums, so the
-//     cancellation when u1 is close to 1 costs nothing, and the result is renormalised;
-//   * sqrt: an rsqrt.approx seed and one Newton step on the float-float residual;
-//   * cos, sin of 2 pi x 2^-32: as in the fp64 form, the sector centre a_j from the top 7 bits
-//     (its sine and cosine as float-float pairs) and the exact integer k for the rest, with
-//     k a = k (a_hi + a_lo) in float-float and sin(k a) ~ k a - (k a)^3/6, 1 - cos(k a) ~
-//     (k a)^2/2 - (k a)^4/24 (next terms below 1e-10);
-//   * the products radius * cos and radius * sin keep their rounding error as a lo word.
-// Each output is returned as hi + lo; its error against the exact value is below about
-// 1e-8 * scale (measured over every table breakpoint of both words and 2^24 random pairs),
-// so rounding hi + lo to fp32 gives the nearest or next-nearest float.
-
-struct NoiseTablesF2Global {
-  __device__ __forceinline__ float4 ln(uint32_t j) const { return __ldg(&kLnTableF2[j]); }
-  __device__ __forceinline__ float4 sincos(uint32_t j) const { return __ldg(&kSinCosTableF2[j]); }
-};
-
-// Shared copies of the fp32 tables, laid out like NoiseTablesShared: entry j of copy c at
-// [8 j + c], each thread reading copy threadIdx.x mod 8 (8 KB per table pair and copy set).
-constexpr int kNoiseSharedEntriesF2 = 2 * kNoiseTableSize * kNoiseTableCopies;
-constexpr int kNoiseSharedBytesF2 = kNoiseSharedEntriesF2 * 16;  // 32 KB
-
-struct NoiseTablesF2Shared {
-  const float4* s;  // kNoiseSharedEntriesF2 entries, filled by stage_noise_tables_f2
-  __device__ __forceinline__ float4 ln(uint32_t j) const {
-    return s[j * kNoiseTableCopies + (threadIdx.x & (kNoiseTableCopies - 1))];
-  }
-  __device__ __forceinline__ float4 sincos(uint32_t j) const {
-    return s[(kNoiseTableSize + j) * kNoiseTableCopies + (threadIdx.x & (kNoiseTableCopies - 1))];
-  }
-};
-
-// Fills the shared copies; the caller synchronises the block before the first read.
-__device__ __forceinline__ void stage_noise_tables_f2(float4* s) {
-  for (int i = threadIdx.x; i < kNoiseSharedEntriesF2; i += blockDim.x) {
-    const int j = (i / kNoiseTableCopies) % kNoiseTableSize;
-    s[i] = i < kNoiseTableSize * kNoiseTableCopies ? kLnTableF2[j] : kSinCosTableF2[j];
-  }
-}
-
-__device__ __forceinline__ void two_sum_f(float a, float b, float& s, float& e) {
-  s = __fadd_rn(a, b);
-  const float bb = __fsub_rn(s, a);
-  e = __fadd_rn(__fsub_rn(a, __fsub_rn(s, bb)), __fsub_rn(b, bb));
-}
-
-// (z_even, z_odd) = scale * (sqrt(-2 ln u1) cos(2 pi u2), ... sin ...) as float-float pairs
-// {hi, lo}; scale = scale_hi + scale_lo.
-template <class Tab>
-__device__ __forceinline__ void box_muller_f32(uint32_t x_even, uint32_t x_odd, const Tab& tab, float scale_hi,
-                                               float scale_lo, float2& z_even, float2& z_odd) {
-  // ---- y = -2 ln u1, u1 = (x_even + 1) 2^-32
-  const uint32_t n = x_even + 1u;                        // 0 only for x_even = 2^32 - 1 (u1 = 1)
-  const uint32_t lz = static_cast<uint32_t>(__clz(n)) & 31u;
-  const uint32_t M = n << lz;
-  const float4 L = tab.ln((M >> 24) & (kNoiseTableSize - 1));   // {g_hi, g_lo, l_hi, l_lo}
-  const float d = __int2float_rn(static_cast<int>(M & 0xFFFFFFu) - 0x800000);
-  const float rh = __fmul_rn(d, L.x);                    // r' = d g, float-float
-  const float rl = __fmaf_rn(d, L.y, __fmaf_rn(d, L.x, -rh));
-  const float e = __int2float_rn(static_cast<int>(lz) + 1);
-  const float a = __fmul_rn(e, kF2Ln2x2Hi);              // exact
-  float s1, e1, s2, e2;
-  two_sum_f(a, L.z, s1, e1);
-  two_sum_f(s1, rh, s2, e2);
-  float p = __fmaf_rn(rh, 1.0f / 32.0f, 1.0f / 12.0f);
-  p = __fmaf_rn(rh, p, 0.25f);
-  p = __fmul_rn(__fmul_rn(rh, rh), p);
-  const float rest = __fadd_rn(__fadd_rn(__fadd_rn(e1, e2), __fmaf_rn(e, kF2Ln2x2Lo, L.w)), __fadd_rn(rl, p));
-  float yh, yl;
-  two_sum_f(s2, rest, yh, yl);                           // |yl| <= ulp(yh) / 2
-  // ---- radius = scale sqrt(y)
-  const float rs = rsqrt_approx(yh);
-  const float sh = __fmul_rn(yh, rs);
-  const float sl = __fmul_rn(__fadd_rn(__fmaf_rn(-sh, sh, yh), yl), __fmul_rn(0.5f, rs));
-  float Rh = __fmul_rn(sh, scale_hi);
-  float Rl = __fadd_rn(__fmaf_rn(sh, scale_lo, __fmaf_rn(sh, scale_hi, -Rh)), __fmul_rn(sl, scale_hi));
-  if (x_even == 0xFFFFFFFFu) {                           // u1 = 1: radius 0
-    Rh = 0.0f;
-    Rl = 0.0f;
-  }
-  // ---- cos, sin of 2 pi x_odd 2^-32
-  const float k = __int2float_rn(static_cast<int>(x_odd & 0x1FFFFFFu) - 0x1000000);   // |k| <= 2^24, exact
-  const float dh = __fmul_rn(k, kF2TurnHi);
-  const float dl = __fmaf_rn(k, kF2TurnLo, __fmaf_rn(k, kF2TurnHi, -dh));
-  const float d2 = __fmaf_rn(__fmul_rn(2.0f, dh), dl, __fmul_rn(dh, dh));
-  const float sdl = __fmaf_rn(-__fmul_rn(dh, d2), 1.0f / 6.0f, dl);          // sin(k a) - dh
-  const float cm = __fmul_rn(d2, __fmaf_rn(d2, -1.0f / 24.0f, 0.5f));       // 1 - cos(k a)
-  const float4 T = tab.sincos(x_odd >> 25);              // {s_hi, s_lo, c_hi, c_lo}
-  const float bs = __fadd_rn(T.y, __fmaf_rn(T.z, dh, __fsub_rn(__fmaf_rn(T.z, sdl, __fmul_rn(T.w, dh)),
-                                                                __fmul_rn(T.x, cm))));
-  const float bc = __fsub_rn(T.w, __fadd_rn(__fmaf_rn(T.x, dh, __fmaf_rn(T.x, sdl, __fmul_rn(T.y, dh))),
-                                            __fmul_rn(T.z, cm)));
-  // ---- products, each with its rounding error kept
-  const float ch = __fmul_rn(Rh, T.z);
-  z_even = make_float2(ch, __fadd_rn(__fmaf_rn(Rh, bc, __fmaf_rn(Rh, T.z, -ch)), __fmul_rn(Rl, T.z)));
-  const float sn = __fmul_rn(Rh, T.x);
-  z_odd = make_float2(sn, __fadd_rn(__fmaf_rn(Rh, bs, __fmaf_rn(Rh, T.x, -sn)), __fmul_rn(Rl, T.x)));
-}
-
-// The four normals of Philox block j times `scale` = scale_hi + scale_lo, each as {hi, lo}.
-template <class Tab = NoiseTablesF2Global>
-__device__ __forceinline__ void normals4_f32(uint32_t j, uint32_t layer_id, uint32_t step_lo, uint32_t stream,
-                                             PhiloxKey key, float2 (&z)[4], const Tab& tab, float scale_hi,
-                                             float scale_lo) {
-  const uint4 x = philox4x32_10(make_uint4(j, layer_id, step_lo, stream), key);
-  box_muller_f32(x.x, x.y, tab, scale_hi, scale_lo, z[0], z[1]);
-  box_muller_f32(x.z, x.w, tab, scale_hi, scale_lo, z[2], z[3]);
-}
-
-// fp32(g + (z.x + z.y)) rounded once: two-sum of g and z.x, then the low words.
-__device__ __forceinline__ float add_f2(float g, float2 z) {
-  float s, e;
-  two_sum_f(g, z.x, s, e);
-  return __fadd_rn(s, __fadd_rn(e, z.y));
-}
-
-// A scale given in fp64 (the noise std) as the float-float pair the fp32 transform takes.
-struct ScaleF2 {
-  float hi, lo;
-};
-__host__ __device__ inline ScaleF2 scale_f2(double v) {
-  const float hi = static_cast<float>(v);
-  return ScaleF2{hi, static_cast<float>(v - static_cast<double>(hi))};
-}
-
-// ---------------------------------------------------------------- the gradient noise
-// Which evaluation every gradient-noise site of the library uses (the reduce, the clipped-sum
-// epilogue, dp_add_noise and the transform exposed by dp_box_muller): fp64 (box_muller_f64)
-// or the fp32 float-float form (box_muller_f32).  Both are within about 1e-8 of the exact
-// transform before the result is rounded to fp32.
-enum NoisePrecision : int { kNoiseF64 = 0, kNoiseF32 = 1 };
-#ifndef DPCLIP_NOISE_PRECISION
-#define DPCLIP_NOISE_PRECISION 0
-#endif
-constexpr int kGradientNoise = DPCLIP_NOISE_PRECISION;
-
-// The tables of one precision: read through the read-only cache (Global) or from eight
-// shared copies (Shared, staged by stage(); 32 KB for either precision).
-template <int NP>
-struct NoiseTables {
-  using Entry = typename std::conditional<NP == kNoiseF32, float4, double2>::type;
-  using Global = typename std::conditional<NP == kNoiseF32, NoiseTablesF2Global, NoiseTablesGlobal>::type;
-  using Shared = typename std::conditional<NP == kNoiseF32, NoiseTablesF2Shared, NoiseTablesShared>::type;
-  static constexpr int kEntries = NP == kNoiseF32 ? kNoiseSharedEntriesF2 : kNoiseSharedEntries;
-  static constexpr int kBytes = NP == kNoiseF32 ? kNoiseSharedBytesF2 : kNoiseSharedBytes;
-  __device__ static void stage(void* s) {
-    if constexpr (NP == kNoiseF32) stage_noise_tables_f2(static_cast<float4*>(s));
-    else stage_noise_tables(static_cast<double2*>(s));
-  }
-  __device__ static Shared shared(const void* s) { return Shared{static_cast<const Entry*>(s)}; }
-};
-
-// The four noise values std * z_q of one Philox block, in the form the precision produces,
-// with the ways the kernels consume them.
-template <int NP>
-struct Noise4;
-template <>
-struct Noise4<kNoiseF64> {
-  double z[4];
-  __device__ __forceinline__ float add_to(float g, int q) const {   // fp32(g + n), one rounding
-    return static_cast<float>(static_cast<double>(g) + z[q]);
-  }
-  __device__ __forceinline__ float rounded(int q) const { return __double2float_rn(z[q]); }
-  __device__ __forceinline__ double value(int q) const { return z[q]; }
-};
-template <>
-struct Noise4<kNoiseF32> {
-  float2 z[4];
-  __device__ __forceinline__ float add_to(float g, int q) const { return add_f2(g, z[q]); }
-  __device__ __forceinline__ float rounded(int q) const { return __fadd_rn(z[q].x, z[q].y); }
-  __device__ __forceinline__ double value(int q) const {
-    return static_cast<double>(z[q].x) + static_cast<double>(z[q].y);
-  }
-};
-
-// Noise of Philox block j (elements 4j .. 4j+3 of the stream) scaled by std_dev.
-template <int NP, class Tab>
-__device__ __forceinline__ void noise4(Noise4<NP>& n, uint32_t j, uint32_t layer_id, uint32_t step_lo,
-                                       PhiloxKey key, const Tab& tab, double std_dev, ScaleF2 sc) {
-  const uint4 x = philox4x32_10(make_uint4(j, layer_id, step_lo, kStreamNoise), key);
-  if constexpr (NP == kNoiseF32) {
-    box_muller_f32(x.x, x.y, tab, sc.hi, sc.lo, n.z[0], n.z[1]);
-    box_muller_f32(x.z, x.w, tab, sc.hi, sc.lo, n.z[2], n.z[3]);
-  } else {
-    box_muller_f64(x.x, x.y, tab, std_dev, n.z[0], n.z[1]);
-    box_muller_f64(x.z, x.w, tab, std_dev, n.z[2], n.z[3]);
-  }
 }
 
 // Full-precision Box-Muller (CUDA's log, sqrt and sincospi, ~1e-16).  Used where the normals

@@ -26,38 +26,38 @@ template <bool STAGED, bool SET = false>
 __global__ void noise_add_kernel(float* __restrict__ G, unsigned long long total, double std_dev,
                                  PhiloxKey key, uint32_t layer_id, StepRef step) {
   griddep_enter();
-  using NT = NoiseTables<kGradientNoise>;
-  __shared__ typename NT::Entry tab_s[STAGED ? NT::kEntries : 1];
+  __shared__ double2 tab_s[STAGED ? kNoiseSharedEntries : 1];
   const uint32_t step_lo = step.get();
   if constexpr (STAGED) {
-    NT::stage(tab_s);
+    stage_noise_tables(tab_s);
     __syncthreads();
   }
-  using Tab = typename std::conditional<STAGED, typename NT::Shared, typename NT::Global>::type;
+  using Tab = typename std::conditional<STAGED, NoiseTablesShared, NoiseTablesGlobal>::type;
   Tab tab;
-  if constexpr (STAGED) tab = NT::shared(tab_s);
-  const ScaleF2 sc = scale_f2(std_dev);
+  if constexpr (STAGED) tab = NoiseTablesShared{tab_s};
   const unsigned long long nblk = (total + 3) / 4;
   for (unsigned long long j = blockIdx.x * static_cast<unsigned long long>(blockDim.x) + threadIdx.x;
        j < nblk; j += static_cast<unsigned long long>(gridDim.x) * blockDim.x) {
-    Noise4<kGradientNoise> z;
-    noise4(z, static_cast<uint32_t>(j), layer_id, step_lo, key, tab, std_dev, sc);
+    double z[4];
+    normals4(static_cast<uint32_t>(j), layer_id, step_lo, kStreamNoise, key, z, tab, std_dev);
     const unsigned long long k0 = 4 * j;
     if (k0 + 3 < total) {
       if (!DP_DCHECK(in_buffer(static_cast<long long>(k0), 4, static_cast<long long>(total)), 20u, nullptr)) continue;
       float4* p = reinterpret_cast<float4*>(G + k0);
       if constexpr (SET) {
-        *p = make_float4(z.rounded(0), z.rounded(1), z.rounded(2), z.rounded(3));
+        *p = make_float4(__double2float_rn(z[0]), __double2float_rn(z[1]), __double2float_rn(z[2]),
+                         __double2float_rn(z[3]));
       } else {
         float4 g = *p;
-        g.x = z.add_to(g.x, 0);
-        g.y = z.add_to(g.y, 1);
-        g.z = z.add_to(g.z, 2);
-        g.w = z.add_to(g.w, 3);
+        g.x = static_cast<float>(static_cast<double>(g.x) + z[0]);
+        g.y = static_cast<float>(static_cast<double>(g.y) + z[1]);
+        g.z = static_cast<float>(static_cast<double>(g.z) + z[2]);
+        g.w = static_cast<float>(static_cast<double>(g.w) + z[3]);
         *p = g;
       }
     } else {
-      for (int q = 0; q < 4 && k0 + q < total; ++q) G[k0 + q] = SET ? z.rounded(q) : z.add_to(G[k0 + q], q);
+      for (int q = 0; q < 4 && k0 + q < total; ++q)
+        G[k0 + q] = SET ? __double2float_rn(z[q]) : static_cast<float>(static_cast<double>(G[k0 + q]) + z[q]);
     }
   }
 }
@@ -93,11 +93,12 @@ __global__ void noise_add_batch_kernel(NoiseBatch b, PhiloxKey key, StepRef step
       ++q;
     }
     const NoiseSegment& sg = b.seg[q];
-    Noise4<kGradientNoise> z;
-    noise4(z, static_cast<uint32_t>(jj), sg.layer_id, step_lo, key, typename NoiseTables<kGradientNoise>::Global{},
-           sg.std_dev, scale_f2(sg.std_dev));
+    double z[4];
+    normals4(static_cast<uint32_t>(jj), sg.layer_id, step_lo, kStreamNoise, key, z, NoiseTablesGlobal{},
+             sg.std_dev);
     const unsigned long long k0 = 4 * jj;
-    for (int e = 0; e < 4 && k0 + e < sg.total; ++e) sg.G[k0 + e] = SET ? z.rounded(e) : z.add_to(sg.G[k0 + e], e);
+    for (int e = 0; e < 4 && k0 + e < sg.total; ++e)
+      sg.G[k0 + e] = SET ? __double2float_rn(z[e]) : static_cast<float>(static_cast<double>(sg.G[k0 + e]) + z[e]);
   }
 }
 
@@ -109,16 +110,9 @@ __global__ void box_muller_words_kernel(const uint2* __restrict__ words, double2
   for (unsigned long long q = blockIdx.x * static_cast<unsigned long long>(blockDim.x) + threadIdx.x;
        q < npairs; q += static_cast<unsigned long long>(gridDim.x) * blockDim.x) {
     const uint2 w = words[q];
-    if constexpr (kGradientNoise == kNoiseF32) {
-      float2 a, b;
-      box_muller_f32(w.x, w.y, NoiseTablesF2Global{}, 1.0f, 0.0f, a, b);
-      z[q] = make_double2(static_cast<double>(a.x) + static_cast<double>(a.y),
-                          static_cast<double>(b.x) + static_cast<double>(b.y));
-    } else {
-      double a, b;
-      box_muller_f64(w.x, w.y, NoiseTablesGlobal{}, 1.0, a, b);
-      z[q] = make_double2(a, b);
-    }
+    double a, b;
+    box_muller_f64(w.x, w.y, NoiseTablesGlobal{}, 1.0, a, b);
+    z[q] = make_double2(a, b);
   }
 }
 
@@ -379,16 +373,14 @@ __global__ void scale_rows_bf16_batch_kernel(ScaleBatch b) {
 // tables in shared memory once.
 // The eight noise values of elements 8 v2 .. 8 v2 + 7 (two Philox blocks), each rounded to
 // fp32 once, scaled by the std.
-template <int NP, class Tab>
+template <class Tab>
 __device__ __forceinline__ void noise8_f32(uint32_t blk0, uint32_t layer_id, uint32_t step_lo, PhiloxKey key,
-                                           const Tab& tab, double std_dev, ScaleF2 sc, float (&n)[8]) {
-  Noise4<NP> z;
-  noise4(z, blk0, layer_id, step_lo, key, tab, std_dev, sc);
+                                           const Tab& tab, double std_dev, float (&n)[8]) {
+  double z[8];
+  normals4(blk0, layer_id, step_lo, kStreamNoise, key, *reinterpret_cast<double(*)[4]>(z), tab, std_dev);
+  normals4(blk0 + 1u, layer_id, step_lo, kStreamNoise, key, *reinterpret_cast<double(*)[4]>(z + 4), tab, std_dev);
 #pragma unroll
-  for (int q = 0; q < 4; ++q) n[q] = z.rounded(q);
-  noise4(z, blk0 + 1u, layer_id, step_lo, key, tab, std_dev, sc);
-#pragma unroll
-  for (int q = 0; q < 4; ++q) n[4 + q] = z.rounded(q);
+  for (int q = 0; q < 8; ++q) n[q] = __double2float_rn(z[q]);
 }
 
 // STAGED: the Box-Muller tables are staged in shared memory (32 KB); otherwise they are read
@@ -400,15 +392,14 @@ __device__ __forceinline__ void noise8_f32(uint32_t blk0, uint32_t layer_id, uin
 // With pr.partials (BU > 0 only), warp i of every block first sums sample i's norm partials
 // (the fixed-order routine, so every block gets the same bits) and block 0 writes norm2 /
 // norms_out / c_out, as the bulk-copy reduce does: no separate partials kernel.
-template <int NP, bool STAGED, int BU>
+template <bool STAGED, int BU>
 __global__ void __launch_bounds__(256, 2) clip_reduce_kernel(
     const __nv_bfloat16* __restrict__ Gs, int B, long long mn, NormSource src, PartialsRef pr, float C,
     float* __restrict__ out, double noise_std, PhiloxKey key, uint32_t layer_id, StepRef step) {
   griddep_enter();
   const uint32_t step_lo = step.get();
-  using NT = NoiseTables<NP>;
   extern __shared__ double2 reduce_smem[];  // noise tables (STAGED), then the cached clip factors
-  float* c_smem = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(reduce_smem) + (STAGED ? NT::kBytes : 0));
+  float* c_smem = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(reduce_smem) + (STAGED ? kNoiseSharedBytes : 0));
   const int cached = B < kReduceCachedSamples ? B : kReduceCachedSamples;
   if (BU > 0 && pr.partials != nullptr) {
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -427,12 +418,11 @@ __global__ void __launch_bounds__(256, 2) clip_reduce_kernel(
   } else {
     for (int i = threadIdx.x; i < cached; i += blockDim.x) c_smem[i] = clip_factor(src.norm(i), C);
   }
-  if (STAGED && noise_std != 0.0) NT::stage(reduce_smem);
+  if (STAGED && noise_std != 0.0) stage_noise_tables(reduce_smem);
   __syncthreads();
-  using Tab = typename std::conditional<STAGED, typename NT::Shared, typename NT::Global>::type;
+  using Tab = typename std::conditional<STAGED, NoiseTablesShared, NoiseTablesGlobal>::type;
   Tab tab;
-  if constexpr (STAGED) tab = NT::shared(reduce_smem);
-  const ScaleF2 sc = scale_f2(noise_std);
+  if constexpr (STAGED) tab = NoiseTablesShared{reduce_smem};
   const long long nvec = mn / 8;  // 16-byte vectors per sample
   for (long long v = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; v < nvec;
        v += static_cast<long long>(gridDim.x) * blockDim.x) {
@@ -446,7 +436,7 @@ __global__ void __launch_bounds__(256, 2) clip_reduce_kernel(
 #pragma unroll
       for (int i = 0; i < BU; ++i) pk[i] = __ldcs(g + static_cast<long long>(i) * nvec);
       if (noise_std != 0.0)
-        noise8_f32<NP>(static_cast<uint32_t>(2 * v), layer_id, step_lo, key, tab, noise_std, sc, z);
+        noise8_f32(static_cast<uint32_t>(2 * v), layer_id, step_lo, key, tab, noise_std, z);
 #pragma unroll
       for (int i = 0; i < BU; ++i) {
         const float c = c_smem[i];
@@ -471,7 +461,7 @@ __global__ void __launch_bounds__(256, 2) clip_reduce_kernel(
         }
       }
       if (noise_std != 0.0)
-        noise8_f32<NP>(static_cast<uint32_t>(2 * v), layer_id, step_lo, key, tab, noise_std, sc, z);
+        noise8_f32(static_cast<uint32_t>(2 * v), layer_id, step_lo, key, tab, noise_std, z);
     }
     if (noise_std != 0.0) {
 #pragma unroll
@@ -505,13 +495,12 @@ struct ReduceTmaConfig {
   static constexpr int STAGES = (196608 / STAGE_BYTES) < 8 ? (196608 / STAGE_BYTES) : 8;
   static constexpr int THREADS = 32 * (1 + kReduceComputeWarps);
   static constexpr int TABLE_OFFSET = STAGES * STAGE_BYTES + 256;  // after the barriers
-  static_assert(kNoiseSharedBytes == kNoiseSharedBytesF2, "one table region serves both precisions");
   static constexpr int SMEM_BYTES = 1024 + TABLE_OFFSET + kNoiseSharedBytes;
   static_assert(SMEM_BYTES <= 232448, "dynamic shared memory per block");
   static_assert(kReduceChunk == 8 * 32 * kReduceComputeWarps, "8 elements per compute thread");
 };
 
-template <int BU, int NP>
+template <int BU>
 __global__ void __launch_bounds__(ReduceTmaConfig<BU>::THREADS, 1) clip_reduce_tma_kernel(
     const __nv_bfloat16* __restrict__ Gs, long long mn, NormSource src, PartialsRef pr, float C,
     float* __restrict__ out, double noise_std, PhiloxKey key, uint32_t layer_id, StepRef step,
@@ -537,11 +526,10 @@ __global__ void __launch_bounds__(ReduceTmaConfig<BU>::THREADS, 1) clip_reduce_t
     fence_mbar_init();
   }
   if (pr.partials == nullptr && threadIdx.x < BU) c_s[threadIdx.x] = clip_factor(src.norm(threadIdx.x), C);
-  using NT = NoiseTables<NP>;
-  if (noise_std != 0.0) NT::stage(smem + Cfg::TABLE_OFFSET);
+  double2* tab_s = reinterpret_cast<double2*>(smem + Cfg::TABLE_OFFSET);
+  if (noise_std != 0.0) stage_noise_tables(tab_s);
   __syncthreads();
-  const auto tab = NT::shared(smem + Cfg::TABLE_OFFSET);
-  const ScaleF2 sc = scale_f2(noise_std);
+  const NoiseTablesShared tab{tab_s};
   const long long chunks = (mn + kReduceChunk - 1) / kReduceChunk;
   if (warp == 0) {
     if (lane == 0) {
@@ -591,7 +579,7 @@ __global__ void __launch_bounds__(ReduceTmaConfig<BU>::THREADS, 1) clip_reduce_t
       const long long e = ch * kReduceChunk + 8 * t;  // first of this thread's 8 elements
       float z[8];
       if (noise_std != 0.0 && e < mn)
-        noise8_f32<NP>(static_cast<uint32_t>(e >> 2), layer_id, step_lo, key, tab, noise_std, sc, z);
+        noise8_f32(static_cast<uint32_t>(e >> 2), layer_id, step_lo, key, tab, noise_std, z);
       if (need_c) {
         // Every compute warp passes here in its first iteration (the trip count is the same
         // for all of them), before any wait that could end the loop early.
@@ -772,10 +760,9 @@ __global__ void __launch_bounds__(256) f32_clipsum_kernel(
   }
   if (noise_std != 0.0) {
     const unsigned long long k = static_cast<unsigned long long>(a) * n + b;
-    Noise4<kGradientNoise> z;
-    noise4(z, static_cast<uint32_t>(k >> 2), layer_id, step_lo, key, typename NoiseTables<kGradientNoise>::Global{},
-           noise_std, scale_f2(noise_std));
-    for (int q = 0; q < 4; ++q) acc[q] += z.value(q);
+    double z[4];
+    normals4(static_cast<uint32_t>(k >> 2), layer_id, step_lo, kStreamNoise, key, z, NoiseTablesGlobal{}, noise_std);
+    for (int q = 0; q < 4; ++q) acc[q] += z[q];
   }
   for (int q = 0; q < 4; ++q) dst[q] = static_cast<float>(acc[q]);
 }

@@ -290,13 +290,12 @@ __device__ __forceinline__ void epilogue_unit(const UmmaParams& p, const Unit& w
         float4 val = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
         if (noisy) {
           const unsigned long long k = static_cast<unsigned long long>(grow) * p.out_cols + gcol0 + 4 * q;
-          Noise4<kGradientNoise> z;
-          noise4(z, static_cast<uint32_t>(k >> 2), p.layer_id, step_lo, key,
-                 typename NoiseTables<kGradientNoise>::Global{}, p.noise_std, scale_f2(p.noise_std));
-          val.x = z.add_to(val.x, 0);
-          val.y = z.add_to(val.y, 1);
-          val.z = z.add_to(val.z, 2);
-          val.w = z.add_to(val.w, 3);
+          double z[4];
+          normals4(static_cast<uint32_t>(k >> 2), p.layer_id, step_lo, kStreamNoise, key, z);
+          val.x = static_cast<float>(static_cast<double>(val.x) + p.noise_std * z[0]);
+          val.y = static_cast<float>(static_cast<double>(val.y) + p.noise_std * z[1]);
+          val.z = static_cast<float>(static_cast<double>(val.z) + p.noise_std * z[2]);
+          val.w = static_cast<float>(static_cast<double>(val.w) + p.noise_std * z[3]);
         }
         if (!DP_DCHECK(in_buffer(grow * p.out_cols + gcol0 + 4 * q, 4, p.out_elems), 1u, p.status)) break;
         float4* d4 = reinterpret_cast<float4*>(dst + 4 * q);
