@@ -305,7 +305,7 @@ dp_status launch_umma_group(const UmmaParams& p, const UmmaGroup& g, cudaStream_
   }
   if (p.num_units <= 0) return DP_OK;
   const int grid = p.num_units < sm_count() ? p.num_units : sm_count();
-  LaunchScope scope(kKindProject, stream);
+  LaunchScope scope(Cfg::EPI == kEpiClipSum ? kKindClipSum : kKindProject, stream);
   DP_LAUNCH("umma_group_kernel", umma_group_kernel<Cfg>, grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream, p, g);
   return DP_OK;
 }
@@ -1286,6 +1286,77 @@ NormSource layer_norm_source(const BlockLayout& Lb, uint8_t* ws, int l, int B, d
   return src;
 }
 
+// Whether the clipped sums of the layers in `ls` can run as grouped launches: every one on the
+// one-SM engine with the same tile width (no SM-pair tiles), up to kMaxGroup a launch.
+bool clipsums_groupable(const dp_layer* layers, const std::vector<int>& ls, int B, int T, dp_dtype dt) {
+  if (ls.size() < 2) return false;
+  int bn = 0;
+  for (int l : ls) {
+    const ClipSumPlan c = clipsum_plan(layer_shape(layers[l], B, T, dt));
+    if (c.pair || (bn && c.bn != bn)) return false;
+    bn = c.bn;
+  }
+  return true;
+}
+
+// The clipped sums of the layers in `ls` (batched schedule, groupable) in grouped launches of
+// up to kMaxGroup problems.  One K split for the whole launch, chosen so that its units fill the
+// GPU about once; every output already holds its noise (or zeros) and the partial sums are
+// added to it by atomics.
+dp_status launch_clipsum_groups(const dp_layer* layers, const std::vector<int>& ls, dp_dtype dt, int B, int T,
+                                const BlockLayout& Lb, uint8_t* ws, cudaStream_t stream) {
+  dp_status st;
+  for (size_t c0 = 0; c0 < ls.size(); c0 += kMaxGroup) {
+    const int count = static_cast<int>(std::min<size_t>(kMaxGroup, ls.size() - c0));
+    UmmaParams p = base_params(reinterpret_cast<uint32_t*>(ws));
+    UmmaGroup g;
+    memset(&g, 0, sizeof(g));
+    g.count = count;
+    const ClipSumPlan plan0 = clipsum_plan(layer_shape(layers[ls[c0]], B, T, dt));
+    int tiles = 0;
+    for (int q = 0; q < count; ++q) {
+      const Shape s = layer_shape(layers[ls[c0 + q]], B, T, dt);
+      g.m_tiles[q] = ceil_div(s.m, 128);
+      tiles += g.m_tiles[q] * plan0.n_tiles;
+    }
+    const int k_blocks = plan0.k_blocks;
+    int splits = std::max(1, sm_count() / std::max(1, tiles));
+    splits = std::min(splits, std::max(1, k_blocks / 4));
+    g.k_blocks_per_split = ceil_div(k_blocks, splits);
+    splits = ceil_div(k_blocks, g.k_blocks_per_split);
+    int units = 0;
+    for (int q = 0; q < count; ++q) {
+      const int l = ls[c0 + q];
+      const dp_layer& y = layers[l];
+      const Shape s = layer_shape(y, B, T, dt);
+      const void* Z;
+      if ((st = block_operand(layers, l, dt, B, T, Lb, ws, stream, false, &Z)) != DP_OK) return st;
+      const void* scaled = ws + Lb.scaled_l[l];
+      const void* A = s.ne() <= s.m ? y.X : scaled;
+      const void* Bm = s.ne() <= s.m ? scaled : Z;
+      if ((st = map_2d(&g.tmA[q], A, s.N(), s.m, 64)) != DP_OK) return st;
+      if ((st = map_2d(&g.tmB[q], Bm, s.N(), s.ne(), 64)) != DP_OK) return st;
+      g.out_f32[q] = y.G_out;
+      g.out_rows[q] = s.m;
+      g.k_blocks[q] = k_blocks;
+      g.unit_begin[q] = units;
+      units += g.m_tiles[q] * plan0.n_tiles * splits;
+    }
+    g.unit_begin[count] = units;
+    p.num_units = units;
+    p.n_tiles = plan0.n_tiles;
+    p.k_blocks = k_blocks;
+    p.k_splits = splits;
+    p.out_cols = layer_shape(layers[ls[c0]], B, T, dt).ne();
+    p.out_mode = kOutAtomicAdd;
+    p.noise_std = 0.0;  // written into the outputs beforehand
+    if (plan0.bn == 128) st = launch_umma_group<UmmaConfig<128, kEpiClipSum, true>>(p, g, stream);
+    else st = launch_umma_group<UmmaConfig<256, kEpiClipSum, true>>(p, g, stream);
+    if (st != DP_OK) return st;
+  }
+  return DP_OK;
+}
+
 // One launch of the row scalings of the layers in `ls` (batched schedule): layer l's narrower
 // operand (Z, or X when X is narrower) scaled by its clip factors into its own copy.  Each
 // layer's blocks sum their samples' norm partials themselves, unless a block would cover too
@@ -1372,19 +1443,24 @@ dp_status block_step(const dp_layer* layers, int L, dp_dtype dt, int B, int T, d
     // in one launch on the second stream beside the norm passes; those sums then add to it.
     std::vector<bool> preset(L, false);
     cudaEvent_t noise_written = nullptr;
-    if (Lb.batched_scale && sigma != 0.0f) {
+    // Grouped clipped sums (batched schedule, all on the one-SM engine with one tile width):
+    // every output is prefilled, with its noise or with zeros, and added to by atomics.
+    std::vector<int> batch_all;
+    if (Lb.batched_scale)
+      for (const auto& g : Lb.groups)
+        if (Lb.methods[g[0]] != DP_NORM_ONCE) batch_all.insert(batch_all.end(), g.begin(), g.end());
+    const bool grouped_sums = Lb.batched_scale && dt == DP_BF16 && clipsums_groupable(layers, batch_all, B, T, dt);
+    if (Lb.batched_scale && (sigma != 0.0f || grouped_sums)) {
       NoiseBatch nb;
       nb.count = 0;
-      for (const auto& g : Lb.groups) {
-        if (Lb.methods[g[0]] == DP_NORM_ONCE) continue;
-        for (int l : g) {
-          const Shape s = layer_shape(layers[l], B, T, dt);
-          if (clipsum_plan(s).splits > 1 && nb.count < kMaxNoiseSegments) {
-            nb.seg[nb.count++] = NoiseSegment{layers[l].G_out, static_cast<unsigned long long>(s.m) * s.ne(),
-                                              static_cast<double>(sigma) * static_cast<double>(layers[l].C),
-                                              layers[l].layer_id};
-            preset[l] = true;
-          }
+      for (int l : batch_all) {
+        const Shape s = layer_shape(layers[l], B, T, dt);
+        if ((grouped_sums || clipsum_plan(s).splits > 1) && nb.count < kMaxNoiseSegments) {
+          nb.seg[nb.count++] = NoiseSegment{layers[l].G_out, static_cast<unsigned long long>(s.m) * s.ne(),
+                                            sigma == 0.0f ? 0.0
+                                                          : static_cast<double>(sigma) * static_cast<double>(layers[l].C),
+                                            layers[l].layer_id};
+          preset[l] = true;
         }
       }
       if (nb.count > 0) {
@@ -1465,7 +1541,12 @@ dp_status block_step(const dp_layer* layers, int L, dp_dtype dt, int B, int T, d
     }
     if (!batch_layers.empty()) {
       if ((st = launch_scale_batch(layers, batch_layers, batch_counts, dt, B, T, Lb, ws, stream)) != DP_OK) return st;
-      for (int l : batch_layers) {
+      if (grouped_sums) {
+        if (noise_written) DP_CUDA(cudaStreamWaitEvent(stream, noise_written, 0));  // join
+        noise_written = nullptr;
+        if ((st = launch_clipsum_groups(layers, batch_layers, dt, B, T, Lb, ws, stream)) != DP_OK) return st;
+      }
+      for (int l : grouped_sums ? std::vector<int>() : batch_layers) {
         const dp_layer& y = layers[l];
         const Shape s = layer_shape(y, B, T, dt);
         const void* Z;

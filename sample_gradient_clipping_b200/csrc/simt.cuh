@@ -93,9 +93,10 @@ __global__ void noise_add_batch_kernel(NoiseBatch b, PhiloxKey key, StepRef step
       ++q;
     }
     const NoiseSegment& sg = b.seg[q];
-    double z[4];
-    normals4(static_cast<uint32_t>(jj), sg.layer_id, step_lo, kStreamNoise, key, z, NoiseTablesGlobal{},
-             sg.std_dev);
+    double z[4] = {0.0, 0.0, 0.0, 0.0};
+    if (!SET || sg.std_dev != 0.0)  // SET with std 0: zeros (a prefill for atomic sums)
+      normals4(static_cast<uint32_t>(jj), sg.layer_id, step_lo, kStreamNoise, key, z, NoiseTablesGlobal{},
+               sg.std_dev);
     const unsigned long long k0 = 4 * jj;
     for (int e = 0; e < 4 && k0 + e < sg.total; ++e)
       sg.G[k0 + e] = SET ? __double2float_rn(z[e]) : static_cast<float>(static_cast<double>(sg.G[k0 + e]) + z[e]);

@@ -84,17 +84,23 @@ struct alignas(64) UmmaParams {
   long long partials_elems;   // floats of the partials buffer (device-side checks; 0 = unknown)
 };
 
-// Several independent problems of one contraction kind in one launch (the projections
-// Z_l = dY_l P_l of a block's projected linears): problem q has its own operand maps, output
-// and K depth, and the units [unit_begin[q], unit_begin[q + 1]) of the launch.  Passed as a
-// second __grid_constant__ parameter, so launches of one problem keep their parameter size.
+// Several independent problems of one contraction kind in one launch: the projections
+// Z_l = dY_l P_l of a block's projected linears (kEpiStoreBf16), or the clipped sums of a
+// block's ghost/explicit linears (kEpiClipSum, split over K, always added by atomics into an
+// output that already holds the noise or zeros).  Problem q has its own operand maps, output,
+// rows and K depth, and the units [unit_begin[q], unit_begin[q + 1]) of the launch.  Passed as
+// a second __grid_constant__ parameter, so launches of one problem keep their parameter size.
 constexpr int kMaxGroup = 8;
 struct alignas(64) UmmaGroup {
   CUtensorMap tmA[kMaxGroup], tmB[kMaxGroup];
-  __nv_bfloat16* out_bf16[kMaxGroup];
+  __nv_bfloat16* out_bf16[kMaxGroup];   // kEpiStoreBf16
+  float* out_f32[kMaxGroup];            // kEpiClipSum
+  int out_rows[kMaxGroup];              // kEpiClipSum: rows of problem q (m_tiles[q] 128-row tiles)
+  int m_tiles[kMaxGroup];               // kEpiClipSum
   int k_blocks[kMaxGroup];
   int unit_begin[kMaxGroup + 1];
   int count;
+  int k_blocks_per_split;               // kEpiClipSum: the group's K split
 };
 
 template <int BN_, int EPI_, bool GROUPED_ = false>
@@ -122,7 +128,8 @@ struct UmmaConfig {
   static constexpr uint32_t IDESC = umma_idesc_bf16(BM, BN, A_MN, B_MN);
   static_assert(NUM_BUFS >= 1, "TMEM budget");
   static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN");
-  static_assert(!GROUPED_ || EPI_ == kEpiStoreBf16, "grouped launches serve the projection");
+  static_assert(!GROUPED_ || EPI_ == kEpiStoreBf16 || EPI_ == kEpiClipSum,
+                "grouped launches serve the projection and the clipped sum");
 };
 
 struct Unit {
@@ -140,6 +147,15 @@ __device__ __forceinline__ Unit decode_unit(const UmmaParams& p, int u, const Um
     while (q + 1 < grp->count && u >= grp->unit_begin[q + 1]) ++q;
     const int r = u - grp->unit_begin[q];
     w.prob = q;
+    if (Cfg::EPI == kEpiClipSum) {  // split-major, then row tiles, then column tiles
+      const int tiles = grp->m_tiles[q] * p.n_tiles;
+      w.split = r / tiles;
+      w.m_blk = (r % tiles) / p.n_tiles;
+      w.n_blk = (r % tiles) % p.n_tiles;
+      w.kb_begin = w.split * grp->k_blocks_per_split;
+      w.kb_end = min(grp->k_blocks[q], w.kb_begin + grp->k_blocks_per_split);
+      return w;
+    }
     w.m_blk = r / p.n_tiles;
     w.n_blk = r % p.n_tiles;
     w.kb_begin = 0;
@@ -194,7 +210,15 @@ __device__ __forceinline__ void issue_stage_loads(const UmmaParams& p, const Uni
                                                   int kb, uint32_t sA, uint32_t sB,
                                                   uint32_t bar, const UmmaGroup* grp = nullptr) {
   const int k0 = kb * Cfg::BK;
-  if constexpr (Cfg::GROUPED) {  // kEpiStoreBf16 per problem: A = dY rows (K-major), B = P (MN-major)
+  if constexpr (Cfg::GROUPED && Cfg::EPI == kEpiClipSum) {  // both operands MN-major, per problem
+#pragma unroll
+    for (int h = 0; h < Cfg::BM / 64; ++h)
+      tma_load_2d(sA + h * (Cfg::BK * 128), &grp->tmA[w.prob], bar, w.m_blk * Cfg::BM + 64 * h, k0);
+#pragma unroll
+    for (int h = 0; h < Cfg::BN / 64; ++h)
+      tma_load_2d(sB + h * (Cfg::BK * 128), &grp->tmB[w.prob], bar, w.n_blk * Cfg::BN + 64 * h, k0);
+    return;
+  } else if constexpr (Cfg::GROUPED) {  // kEpiStoreBf16 per problem: A = dY rows (K-major), B = P (MN-major)
     tma_load_2d(sA, &grp->tmA[w.prob], bar, k0, w.m_blk * Cfg::BM);
 #pragma unroll
     for (int h = 0; h < Cfg::BN / 64; ++h)
@@ -271,7 +295,10 @@ __device__ __forceinline__ void epilogue_unit(const UmmaParams& p, const Unit& w
   const int row = wq * 32 + static_cast<int>(lane);
   if (Cfg::EPI == kEpiClipSum) {
     const long long grow = static_cast<long long>(w.m_blk) * Cfg::BM + row;
-    const bool row_ok = grow < p.out_rows;
+    const int out_rows = Cfg::GROUPED ? grp->out_rows[w.prob] : p.out_rows;
+    float* const out_base = Cfg::GROUPED ? grp->out_f32[w.prob] : p.out_f32;
+    const long long out_elems = Cfg::GROUPED ? static_cast<long long>(out_rows) * p.out_cols : p.out_elems;
+    const bool row_ok = grow < out_rows;
     const bool noisy = (p.noise_std != 0.0) && (w.split == 0);
     const PhiloxKey key{p.key0, p.key1};
     const uint32_t step_lo = StepRef{p.step_lo, p.step_dev}.get();
@@ -283,7 +310,7 @@ __device__ __forceinline__ void epilogue_unit(const UmmaParams& p, const Unit& w
       tmem_ld_wait();
       const long long gcol0 = static_cast<long long>(w.n_blk) * Cfg::BN + c0;
       if (!row_ok || gcol0 >= p.out_cols) continue;  // the next tmem_ld32 reconverges first
-      float* dst = p.out_f32 + grow * p.out_cols + gcol0;
+      float* dst = out_base + grow * p.out_cols + gcol0;
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
         if (gcol0 + 4 * q >= p.out_cols) break;  // out_cols is a multiple of 4
@@ -297,7 +324,7 @@ __device__ __forceinline__ void epilogue_unit(const UmmaParams& p, const Unit& w
           val.z = static_cast<float>(static_cast<double>(val.z) + p.noise_std * z[2]);
           val.w = static_cast<float>(static_cast<double>(val.w) + p.noise_std * z[3]);
         }
-        if (!DP_DCHECK(in_buffer(grow * p.out_cols + gcol0 + 4 * q, 4, p.out_elems), 1u, p.status)) break;
+        if (!DP_DCHECK(in_buffer(grow * p.out_cols + gcol0 + 4 * q, 4, out_elems), 1u, p.status)) break;
         float4* d4 = reinterpret_cast<float4*>(dst + 4 * q);
         if (p.out_mode == kOutStore) {
           *d4 = val;
@@ -528,7 +555,7 @@ __device__ __forceinline__ void umma_body(const UmmaParams& p, const UmmaGroup* 
             const uint32_t bar = smem_addr(full + stage);
             mbar_arrive_expect_tx(bar, Cfg::STAGE_BYTES);
             issue_stage_loads<Cfg>(p, w, ph, kb, sA, sA + Cfg::A_BYTES, bar, grp);
-            if (Cfg::EPI == kEpiClipSum) {
+            if (Cfg::EPI == kEpiClipSum && !Cfg::GROUPED) {
               if (kb == kb_begin) {
                 for (int d = 1; d <= kL2PrefetchDistance && kb + d < kb_end; ++d)
                   prefetch_stage_l2<Cfg>(p, w, kb + d);
