@@ -305,24 +305,38 @@ __device__ __forceinline__ void scale_rows_body(const __nv_bfloat16* __restrict_
     v_end = v1;
     v_step = blockDim.x;
   }
-  for (long long v = v_begin; v < v_end; v += v_step) {
-    const long long row = v / vec_per_row;
-    const int i = static_cast<int>(row / T);
-    if (pr.partials != nullptr &&
-        !DP_DCHECK(i >= s_lo && (i - s_lo + 1) * sizeof(float) <= dynamic_smem_bytes(), 21u, nullptr))
-      break;
-    if (!DP_DCHECK(v >= 0 && v < total, 22u, nullptr)) break;
-    const float c = pr.partials != nullptr ? scale_c[i - s_lo] : clip_factor(src.norm(i), C);
-    const uint4 pk = (pr.partials != nullptr && v == v_begin) ? first : reinterpret_cast<const uint4*>(in)[v];
-    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&pk);
-    uint4 res;
-    __nv_bfloat162* o = reinterpret_cast<__nv_bfloat162*>(&res);
+  // Four vectors per thread and iteration, all four loads issued before the first is used, so
+  // each thread keeps four 16-byte loads in flight (one at a time left the stream latency-bound).
+  constexpr int kU = 4;
+  for (long long v = v_begin; v < v_end; v += kU * v_step) {
+    uint4 pk[kU];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float2 f = __bfloat1622float2(h[e]);
-      o[e] = __floats2bfloat162_rn(c * f.x, c * f.y);
+    for (int u = 0; u < kU; ++u) {
+      const long long vu = v + u * v_step;
+      if (vu < v_end)
+        pk[u] = (pr.partials != nullptr && vu == v_begin) ? first : reinterpret_cast<const uint4*>(in)[vu];
     }
-    reinterpret_cast<uint4*>(out)[v] = res;
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const long long vu = v + u * v_step;
+      if (vu >= v_end) break;
+      const long long row = vu / vec_per_row;
+      const int i = static_cast<int>(row / T);
+      if (pr.partials != nullptr &&
+          !DP_DCHECK(i >= s_lo && (i - s_lo + 1) * sizeof(float) <= dynamic_smem_bytes(), 21u, nullptr))
+        break;
+      if (!DP_DCHECK(vu >= 0 && vu < total, 22u, nullptr)) break;
+      const float c = pr.partials != nullptr ? scale_c[i - s_lo] : clip_factor(src.norm(i), C);
+      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&pk[u]);
+      uint4 res;
+      __nv_bfloat162* o = reinterpret_cast<__nv_bfloat162*>(&res);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(h[e]);
+        o[e] = __floats2bfloat162_rn(c * f.x, c * f.y);
+      }
+      reinterpret_cast<uint4*>(out)[vu] = res;
+    }
   }
 }
 
@@ -404,15 +418,15 @@ __global__ void __launch_bounds__(256, 2) clip_reduce_kernel(
   const int cached = B < kReduceCachedSamples ? B : kReduceCachedSamples;
   if (BU > 0 && pr.partials != nullptr) {
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    if (warp < BU) {
-      const float n2 = warp_norm2_from_partials(pr.partials, pr.stride, pr.count, warp, lane);
+    for (int i = warp; i < BU; i += static_cast<int>(blockDim.x / 32)) {
+      const float n2 = warp_norm2_from_partials(pr.partials, pr.stride, pr.count, i, lane);
       if (lane == 0) {
         const float n = sqrtf(n2);
-        c_smem[warp] = clip_factor(n, C);
+        c_smem[i] = clip_factor(n, C);
         if (blockIdx.x == 0) {
-          if (pr.norm2) pr.norm2[warp] = n2;
-          if (pr.norms_out) pr.norms_out[warp] = n;
-          if (pr.c_out) pr.c_out[warp] = c_smem[warp];
+          if (pr.norm2) pr.norm2[i] = n2;
+          if (pr.norms_out) pr.norms_out[i] = n;
+          if (pr.c_out) pr.c_out[i] = c_smem[i];
         }
       }
     }
