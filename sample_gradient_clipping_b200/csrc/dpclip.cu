@@ -1442,7 +1442,19 @@ dp_status block_step(const dp_layer* layers, int L, dp_dtype dt, int B, int T, d
     // Batched schedule: the noise of every split-K clipped sum is written into its output first,
     // in one launch on the second stream beside the norm passes; those sums then add to it.
     std::vector<bool> preset(L, false);
-    cudaEvent_t noise_written = nullptr;
+    cudaEvent_t noise_written = nullptr, noise_fork = nullptr;
+    NoiseBatch noise_pending;
+    noise_pending.count = 0;
+    auto enqueue_preset_noise = [&]() -> dp_status {
+      if (noise_pending.count == 0) return DP_OK;
+      dp_status e;
+      DP_CUDA(cudaStreamWaitEvent(side, noise_fork, 0));
+      if ((e = launch_noise_batch(noise_pending, seed, step, side, true)) != DP_OK) return e;
+      if ((e = event_ring().next(&noise_written)) != DP_OK) return e;
+      DP_CUDA(cudaEventRecord(noise_written, side));
+      noise_pending.count = 0;
+      return DP_OK;
+    };
     // Grouped clipped sums (batched schedule, all on the one-SM engine with one tile width):
     // every output is prefilled, with its noise or with zeros, and added to by atomics.
     std::vector<int> batch_all;
@@ -1464,11 +1476,11 @@ dp_status block_step(const dp_layer* layers, int L, dp_dtype dt, int B, int T, d
         }
       }
       if (nb.count > 0) {
+        // Forked here; enqueued after the first norm pass (see the single-linear step).
         if (!Lb.overlap && (st = side_stream(&side)) != DP_OK) return st;
-        if ((st = stream_after(side, stream)) != DP_OK) return st;  // fork
-        if ((st = launch_noise_batch(nb, seed, step, side, true)) != DP_OK) return st;
-        if ((st = event_ring().next(&noise_written)) != DP_OK) return st;
-        DP_CUDA(cudaEventRecord(noise_written, side));
+        if ((st = event_ring().next(&noise_fork)) != DP_OK) return st;
+        DP_CUDA(cudaEventRecord(noise_fork, stream));
+        noise_pending = nb;
       }
     }
     // Each group: its norms, then each member's clipped sum with its own bound and noise.
@@ -1517,6 +1529,7 @@ dp_status block_step(const dp_layer* layers, int L, dp_dtype dt, int B, int T, d
         int count = 0;
         float* base = reinterpret_cast<float*>(ws + Lb.partials) + Lb.partial_set[g[0]] * Lb.partial_op_stride;
         if ((st = block_group_norms(layers, g, dt, B, T, Lb, ws, stream, &count, base)) != DP_OK) return st;
+        if ((st = enqueue_preset_noise()) != DP_OK) return st;  // after the first norm pass
         for (int l : g) {
           batch_layers.push_back(l);
           batch_counts.push_back(count);
@@ -1539,6 +1552,7 @@ dp_status block_step(const dp_layer* layers, int L, dp_dtype dt, int B, int T, d
           return st;
       }
     }
+    if ((st = enqueue_preset_noise()) != DP_OK) return st;  // (no norm pass enqueued it)
     if (!batch_layers.empty()) {
       if ((st = launch_scale_batch(layers, batch_layers, batch_counts, dt, B, T, Lb, ws, stream)) != DP_OK) return st;
       if (grouped_sums) {
@@ -1778,22 +1792,29 @@ dp_status linear_step(const void* X, const void* dY, const void* P, int r, dp_dt
   if (dt == DP_BF16) {
     // A clipped sum split over K adds its partial sums by atomics: its noise is written into
     // G_out first, on the library's second stream beside the norm pass and the row scaling.
-    cudaEvent_t noise_written = nullptr;
-    if (noise_std != 0.0 && clipsum_plan(c.s).splits > 1) {
-      cudaStream_t side;
-      if ((st = side_stream(&side)) != DP_OK) return st;
-      if ((st = stream_after(side, c.stream)) != DP_OK) return st;  // fork
-      if ((st = launch_noise(G_out, static_cast<unsigned long long>(mn), noise_std, seed, step, layer_id, side,
-                             true)) != DP_OK)
-        return st;
-      if ((st = event_ring().next(&noise_written)) != DP_OK) return st;
-      DP_CUDA(cudaEventRecord(noise_written, side));
+    // The fork point is recorded before the norm pass but the noise is enqueued after it, so that
+    // the norm pass's CTAs are placed first and the noise blocks take the thread slots left.
+    cudaEvent_t noise_written = nullptr, fork = nullptr;
+    const bool preset = (noise_std != 0.0 && clipsum_plan(c.s).splits > 1);
+    if (preset) {
+      if ((st = event_ring().next(&fork)) != DP_OK) return st;
+      DP_CUDA(cudaEventRecord(fork, c.stream));
     }
     // The norm partials are summed by the row-scaling kernel of the clipped sum.
     int count = 0;
     if ((st = bf16_norms(c.s, X, Z, m, c.partials(), c.L.partial_stride, &count, c.status(), c.stream)) !=
         DP_OK)
       return st;
+    if (preset) {
+      cudaStream_t side;
+      if ((st = side_stream(&side)) != DP_OK) return st;
+      DP_CUDA(cudaStreamWaitEvent(side, fork, 0));
+      if ((st = launch_noise(G_out, static_cast<unsigned long long>(mn), noise_std, seed, step, layer_id, side,
+                             true)) != DP_OK)
+        return st;
+      if ((st = event_ring().next(&noise_written)) != DP_OK) return st;
+      DP_CUDA(cudaEventRecord(noise_written, side));
+    }
     const PartialsRef pr{c.partials(), c.L.partial_stride, count, c.norm2_f32(), norms_out,
                          norms_out ? c.c() : nullptr};
     return clipped_sum(c, X, Z, ws_norm_source(c), C, G_out, 0, noise_std, seed, step, layer_id, nullptr, &pr,

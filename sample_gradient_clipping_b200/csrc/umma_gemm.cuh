@@ -297,7 +297,8 @@ __device__ __forceinline__ void epilogue_unit(const UmmaParams& p, const Unit& w
     const long long grow = static_cast<long long>(w.m_blk) * Cfg::BM + row;
     const int out_rows = Cfg::GROUPED ? grp->out_rows[w.prob] : p.out_rows;
     float* const out_base = Cfg::GROUPED ? grp->out_f32[w.prob] : p.out_f32;
-    const long long out_elems = Cfg::GROUPED ? static_cast<long long>(out_rows) * p.out_cols : p.out_elems;
+    [[maybe_unused]] const long long out_elems =
+        Cfg::GROUPED ? static_cast<long long>(out_rows) * p.out_cols : p.out_elems;
     const bool row_ok = grow < out_rows;
     const bool noisy = (p.noise_std != 0.0) && (w.split == 0);
     const PhiloxKey key{p.key0, p.key1};
