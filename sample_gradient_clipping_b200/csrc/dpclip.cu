@@ -305,7 +305,8 @@ dp_status launch_umma_group(const UmmaParams& p, const UmmaGroup& g, cudaStream_
   }
   if (p.num_units <= 0) return DP_OK;
   const int grid = p.num_units < sm_count() ? p.num_units : sm_count();
-  LaunchScope scope(Cfg::EPI == kEpiClipSum ? kKindClipSum : kKindProject, stream);
+  LaunchScope scope(Cfg::EPI == kEpiClipSum ? kKindClipSum : Cfg::EPI == kEpiGhostNorm ? kKindGhostNorm : kKindProject,
+                    stream);
   DP_LAUNCH("umma_group_kernel", umma_group_kernel<Cfg>, grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream, p, g);
   return DP_OK;
 }
@@ -328,7 +329,7 @@ int stream_grid(unsigned long long work_items, int threads) {
 // `store`, the explicit tiles of every G_i are also written there in bf16 ([B][d_in][ne]).
 dp_status bf16_norms(const Shape& s, const void* X, const void* Z, dp_norm_method method,
                      float* partials, int stride, int* count, uint32_t* status, cudaStream_t stream,
-                     __nv_bfloat16* store = nullptr) {
+                     __nv_bfloat16* store = nullptr, int x_splits = 1) {
   UmmaParams p = base_params(status);
   p.partials = partials;
   p.partial_stride = stride;
@@ -344,10 +345,11 @@ dp_status bf16_norms(const Shape& s, const void* X, const void* Z, dp_norm_metho
     p.tmB1 = p.tmA1;
     p.t_tiles = ceil_div(s.T, 128);
     p.pairs_per_sample = p.t_tiles * (p.t_tiles + 1) / 2;
-    p.num_units = s.B * p.pairs_per_sample;
-    *count = 4 * p.pairs_per_sample;
     p.k_blocks = ceil_div(s.m, 64);
     p.k_blocks1 = ceil_div(ne, 64);
+    p.x_splits = x_splits;
+    p.num_units = s.B * p.pairs_per_sample * x_splits;
+    *count = 4 * p.pairs_per_sample * x_splits;
     return launch_umma<Cfg>(p, stream);
   }
   dp_status st;
@@ -384,7 +386,7 @@ dp_status bf16_norms(const Shape& s, const void* X, const void* Z, dp_norm_metho
 // partials go to partials + j * op_stride, laid out as for bf16_norms.
 dp_status bf16_norms_ghost_shared(const Shape& s, const void* X, const void* const* Zs, int k,
                                   float* partials, int stride, long long op_stride, int* count,
-                                  uint32_t* status, cudaStream_t stream) {
+                                  uint32_t* status, cudaStream_t stream, int x_splits = 1) {
   if (k < 1 || k > kGhostSharedMaxOps) return DP_ERR_INVALID_ARG;
   UmmaParams p = base_params(status);
   p.partials = partials;
@@ -400,10 +402,11 @@ dp_status bf16_norms_ghost_shared(const Shape& s, const void* X, const void* con
     if ((st = map_3d(maps[j], Zs[j], s.B, s.T, ne, 128)) != DP_OK) return st;
   p.t_tiles = ceil_div(s.T, 128);
   p.pairs_per_sample = p.t_tiles * (p.t_tiles + 1) / 2;
-  p.num_units = s.B * p.pairs_per_sample;
-  *count = 4 * p.pairs_per_sample;
   p.k_blocks = ceil_div(s.m, 64);
   p.k_blocks1 = ceil_div(ne, 64);
+  p.x_splits = x_splits;
+  p.num_units = s.B * p.pairs_per_sample * x_splits;
+  *count = 4 * p.pairs_per_sample * x_splits;
   return launch_umma<UmmaConfig<128, kEpiGhostShared>>(p, stream);
 }
 
@@ -1200,11 +1203,63 @@ dp_status block_projections(const dp_layer* layers, int L, dp_dtype dt, int B, i
   return DP_OK;
 }
 
+// K splits of a ghost unit's X Gram (kx K blocks; its dY Grams take k1 blocks in all) so that
+// the units of a launch that would fill under a third of the SMs become more, shorter ones:
+// about 8 X blocks a split, no more than the partial slots hold (4 per split and pair).
+int ghost_x_splits(int kx, int k1, int units, int pairs, int stride) {
+  if (units * 3 >= sm_count()) return 1;
+  int xs = kx / std::max(8, k1);
+  xs = std::min(xs, stride / (4 * pairs));
+  xs = std::max(1, std::min(xs, kx));
+  return ceil_div(kx, ceil_div(kx, xs));  // every split non-empty
+}
+
+// Ghost-norm partials of single (unshared) ghost layers `ls` in grouped launches of up to
+// kMaxGroup problems, each with its own X and dY (or Z) maps, partial set and X-Gram split.
+dp_status launch_ghost_group(const dp_layer* layers, const std::vector<int>& ls, dp_dtype dt, int B, int T,
+                             const BlockLayout& Lb, uint8_t* ws, cudaStream_t stream, std::vector<int>* counts) {
+  dp_status st;
+  const int t_tiles = ceil_div(T, 128);
+  const int pairs = t_tiles * (t_tiles + 1) / 2;
+  int total_units = 0;
+  for (size_t i = 0; i < ls.size(); ++i) total_units += B * pairs;
+  for (size_t c0 = 0; c0 < ls.size(); c0 += kMaxGroup) {
+    const int count = static_cast<int>(std::min<size_t>(kMaxGroup, ls.size() - c0));
+    UmmaParams p = base_params(reinterpret_cast<uint32_t*>(ws));
+    UmmaGroup g;
+    memset(&g, 0, sizeof(g));
+    g.count = count;
+    p.t_tiles = t_tiles;
+    p.pairs_per_sample = pairs;
+    p.partial_stride = Lb.partial_stride;
+    int units = 0;
+    for (int q = 0; q < count; ++q) {
+      const int l = ls[c0 + q];
+      const Shape s = layer_shape(layers[l], B, T, dt);
+      const void* Z;
+      if ((st = block_operand(layers, l, dt, B, T, Lb, ws, stream, false, &Z)) != DP_OK) return st;
+      if ((st = map_3d(&g.tmA[q], layers[l].X, B, T, s.m, 128)) != DP_OK) return st;
+      if ((st = map_3d(&g.tmB[q], Z, B, T, s.ne(), 128)) != DP_OK) return st;
+      g.k_blocks[q] = ceil_div(s.m, 64);
+      g.k_blocks1[q] = ceil_div(s.ne(), 64);
+      g.x_splits[q] = ghost_x_splits(g.k_blocks[q], g.k_blocks1[q], total_units, pairs, Lb.partial_stride);
+      g.partials[q] = reinterpret_cast<float*>(ws + Lb.partials) + Lb.partial_set[l] * Lb.partial_op_stride;
+      g.unit_begin[q] = units;
+      units += B * pairs * g.x_splits[q];
+      (*counts)[c0 + q] = 4 * pairs * g.x_splits[q];
+    }
+    g.unit_begin[count] = units;
+    p.num_units = units;
+    if ((st = launch_umma_group<UmmaConfig<128, kEpiGhostNorm, true>>(p, g, stream)) != DP_OK) return st;
+  }
+  return DP_OK;
+}
+
 // Squared norms of the layers of one group into their [B] rows of the norm2 block, and each
 // layer's norms_out when given (gradients-once layers also keep their tiles).
 dp_status block_group_norms(const dp_layer* layers, const std::vector<int>& g, dp_dtype dt, int B, int T,
                             const BlockLayout& Lb, uint8_t* ws, cudaStream_t stream, int* count_out = nullptr,
-                            float* partials_base = nullptr) {
+                            float* partials_base = nullptr, int x_splits = 1) {
   dp_status st;
   uint32_t* status = reinterpret_cast<uint32_t*>(ws);
   const dp_layer& y0 = layers[g[0]];
@@ -1230,7 +1285,7 @@ dp_status block_group_norms(const dp_layer* layers, const std::vector<int>& g, d
   int count = 0;
   if (g.size() > 1) {
     if ((st = bf16_norms_ghost_shared(s, y0.X, Zs, static_cast<int>(g.size()), partials, Lb.partial_stride,
-                                      Lb.partial_op_stride, &count, status, stream)) != DP_OK)
+                                      Lb.partial_op_stride, &count, status, stream, x_splits)) != DP_OK)
       return st;
   } else {
     const bool once = (Lb.methods[g[0]] == DP_NORM_ONCE);
@@ -1439,6 +1494,7 @@ dp_status block_step(const dp_layer* layers, int L, dp_dtype dt, int B, int T, d
     for (const auto& g : Lb.groups) once_n += (dt == DP_BF16 && Lb.methods[g[0]] == DP_NORM_ONCE) ? 1 : 0;
     bool side_pending = false;  // reduces on the side stream the caller's stream has not joined
     std::vector<int> batch_layers, batch_counts;  // batched schedule: layers waiting for their sums
+    std::vector<int> ghost_single, ghost_single_at;  // batched schedule: single ghost layers, their slots
     // Batched schedule: the noise of every split-K clipped sum is written into its output first,
     // in one launch on the second stream beside the norm passes; those sums then add to it.
     std::vector<bool> preset(L, false);
@@ -1524,11 +1580,25 @@ dp_status block_step(const dp_layer* layers, int L, dp_dtype dt, int B, int T, d
         side_pending = false;
       }
       if (Lb.batched_scale) {
-        // Batched schedule: this group's norm pass now, its row scaling and clipped sums after
-        // every group's norm pass.
+        // Batched schedule: this group's norm pass now (single ghost layers: all in one grouped
+        // launch after the loop), its row scaling and clipped sums after every norm pass.
+        if (dt == DP_BF16 && g.size() == 1 && Lb.methods[g[0]] == DP_NORM_GHOST) {
+          ghost_single.push_back(g[0]);
+          ghost_single_at.push_back(static_cast<int>(batch_layers.size()));
+          batch_layers.push_back(g[0]);
+          batch_counts.push_back(0);  // set by the grouped launch
+          continue;
+        }
         int count = 0;
         float* base = reinterpret_cast<float*>(ws + Lb.partials) + Lb.partial_set[g[0]] * Lb.partial_op_stride;
-        if ((st = block_group_norms(layers, g, dt, B, T, Lb, ws, stream, &count, base)) != DP_OK) return st;
+        int xs = 1;
+        if (dt == DP_BF16 && g.size() > 1) {  // a shared X Gram: split it when its units are few
+          const Shape s0 = layer_shape(layers[g[0]], B, T, dt);
+          const int tt = ceil_div(T, 128), pairs = tt * (tt + 1) / 2;
+          xs = ghost_x_splits(ceil_div(s0.m, 64), static_cast<int>(g.size()) * ceil_div(s0.ne(), 64), B * pairs,
+                              pairs, Lb.partial_stride);
+        }
+        if ((st = block_group_norms(layers, g, dt, B, T, Lb, ws, stream, &count, base, xs)) != DP_OK) return st;
         if ((st = enqueue_preset_noise()) != DP_OK) return st;  // after the first norm pass
         for (int l : g) {
           batch_layers.push_back(l);
@@ -1552,7 +1622,12 @@ dp_status block_step(const dp_layer* layers, int L, dp_dtype dt, int B, int T, d
           return st;
       }
     }
-    if ((st = enqueue_preset_noise()) != DP_OK) return st;  // (no norm pass enqueued it)
+    if (!ghost_single.empty()) {
+      std::vector<int> counts(ghost_single.size(), 0);
+      if ((st = launch_ghost_group(layers, ghost_single, dt, B, T, Lb, ws, stream, &counts)) != DP_OK) return st;
+      for (size_t i = 0; i < ghost_single.size(); ++i) batch_counts[ghost_single_at[i]] = counts[i];
+    }
+    if ((st = enqueue_preset_noise()) != DP_OK) return st;  // (unless a norm pass enqueued it)
     if (!batch_layers.empty()) {
       if ((st = launch_scale_batch(layers, batch_layers, batch_counts, dt, B, T, Lb, ws, stream)) != DP_OK) return st;
       if (grouped_sums) {

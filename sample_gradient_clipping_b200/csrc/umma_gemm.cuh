@@ -82,6 +82,8 @@ struct alignas(64) UmmaParams {
   uint32_t* status;
   long long out_elems;        // elements of the output buffer (device-side checks; 0 = unknown)
   long long partials_elems;   // floats of the partials buffer (device-side checks; 0 = unknown)
+  int x_splits;               // ghost kinds: K splits of the X Gram (0 or 1: none).  The norm is
+                              // linear in the X Gram, so each split's partial sums add up.
 };
 
 // Several independent problems of one contraction kind in one launch: the projections
@@ -98,6 +100,9 @@ struct alignas(64) UmmaGroup {
   int out_rows[kMaxGroup];              // kEpiClipSum: rows of problem q (m_tiles[q] 128-row tiles)
   int m_tiles[kMaxGroup];               // kEpiClipSum
   int k_blocks[kMaxGroup];
+  int k_blocks1[kMaxGroup];             // kEpiGhostNorm: K blocks of the dY (or Z) Gram
+  int x_splits[kMaxGroup];              // kEpiGhostNorm: K splits of the X Gram
+  float* partials[kMaxGroup];           // kEpiGhostNorm: the problem's norm-partial set
   int unit_begin[kMaxGroup + 1];
   int count;
   int k_blocks_per_split;               // kEpiClipSum: the group's K split
@@ -128,15 +133,31 @@ struct UmmaConfig {
   static constexpr uint32_t IDESC = umma_idesc_bf16(BM, BN, A_MN, B_MN);
   static_assert(NUM_BUFS >= 1, "TMEM budget");
   static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN");
-  static_assert(!GROUPED_ || EPI_ == kEpiStoreBf16 || EPI_ == kEpiClipSum,
-                "grouped launches serve the projection and the clipped sum");
+  static_assert(!GROUPED_ || EPI_ == kEpiStoreBf16 || EPI_ == kEpiClipSum || EPI_ == kEpiGhostNorm,
+                "grouped launches serve the projection, the clipped sum and the ghost norm");
 };
 
 struct Unit {
   int m_blk, n_blk, kb_begin, kb_end, sample, split;
   int local;  // index of the unit among the units of its sample (norm partial slots)
   int prob;   // grouped launch: the problem of the unit
+  int kb1;    // ghost kinds: K blocks of the phases after the first (the dY Grams)
 };
+
+// Ghost units of one sample: upper-triangular pairs of 128-token blocks, each in `xs` K splits
+// of its X Gram.  Unit index r within the sample -> (row block, column block, split).
+__device__ __forceinline__ void ghost_pair(int r, int t_tiles, int xs, Unit& w) {
+  const int pair = r / xs;
+  w.split = r % xs;
+  w.local = r;  // = pair * xs + split: its four warps write slots 4 local .. 4 local + 3
+  int c = pair, row = 0;
+  while (c >= t_tiles - row) {
+    c -= t_tiles - row;
+    ++row;
+  }
+  w.m_blk = row;
+  w.n_blk = row + c;
+}
 
 template <class Cfg>
 __device__ __forceinline__ Unit decode_unit(const UmmaParams& p, int u, const UmmaGroup* grp = nullptr) {
@@ -156,6 +177,16 @@ __device__ __forceinline__ Unit decode_unit(const UmmaParams& p, int u, const Um
       w.kb_end = min(grp->k_blocks[q], w.kb_begin + grp->k_blocks_per_split);
       return w;
     }
+    if (Cfg::EPI == kEpiGhostNorm) {
+      const int xs = grp->x_splits[q];
+      w.sample = r / (p.pairs_per_sample * xs);
+      ghost_pair(r % (p.pairs_per_sample * xs), p.t_tiles, xs, w);
+      const int kbps = (grp->k_blocks[q] + xs - 1) / xs;
+      w.kb_begin = w.split * kbps;
+      w.kb_end = min(grp->k_blocks[q], w.kb_begin + kbps);
+      w.kb1 = grp->k_blocks1[q];
+      return w;
+    }
     w.m_blk = r / p.n_tiles;
     w.n_blk = r % p.n_tiles;
     w.kb_begin = 0;
@@ -163,19 +194,13 @@ __device__ __forceinline__ Unit decode_unit(const UmmaParams& p, int u, const Um
     return w;
   }
   if (Cfg::GHOST) {
-    w.sample = u / p.pairs_per_sample;
-    int r = u % p.pairs_per_sample;
-    int row = 0;
-    while (r >= p.t_tiles - row) {
-      r -= p.t_tiles - row;
-      ++row;
-    }
-    w.local = u % p.pairs_per_sample;
-    w.m_blk = row;
-    w.n_blk = row + r;
-    w.kb_begin = 0;
-    w.kb_end = p.k_blocks;
-    w.split = 0;
+    const int xs = p.x_splits > 1 ? p.x_splits : 1;
+    w.sample = u / (p.pairs_per_sample * xs);
+    ghost_pair(u % (p.pairs_per_sample * xs), p.t_tiles, xs, w);
+    const int kbps = (p.k_blocks + xs - 1) / xs;
+    w.kb_begin = w.split * kbps;
+    w.kb_end = min(p.k_blocks, w.kb_begin + kbps);
+    w.kb1 = p.k_blocks1;
     return w;
   }
   const int tiles = p.m_tiles * p.n_tiles;
@@ -218,7 +243,7 @@ __device__ __forceinline__ void issue_stage_loads(const UmmaParams& p, const Uni
     for (int h = 0; h < Cfg::BN / 64; ++h)
       tma_load_2d(sB + h * (Cfg::BK * 128), &grp->tmB[w.prob], bar, w.n_blk * Cfg::BN + 64 * h, k0);
     return;
-  } else if constexpr (Cfg::GROUPED) {  // kEpiStoreBf16 per problem: A = dY rows (K-major), B = P (MN-major)
+  } else if constexpr (Cfg::GROUPED && Cfg::EPI == kEpiStoreBf16) {  // per problem: A = dY rows (K-major), B = P (MN-major)
     tma_load_2d(sA, &grp->tmA[w.prob], bar, k0, w.m_blk * Cfg::BM);
 #pragma unroll
     for (int h = 0; h < Cfg::BN / 64; ++h)
@@ -242,8 +267,10 @@ __device__ __forceinline__ void issue_stage_loads(const UmmaParams& p, const Uni
       tma_load_3d(sB + h * (Cfg::BK * 128), &p.tmB0, bar, w.n_blk * Cfg::BN + 64 * h, k0,
                   w.sample);
   } else if (Cfg::EPI == kEpiGhostNorm) {
-    const CUtensorMap* ma = phase ? &p.tmA1 : &p.tmA0;
-    const CUtensorMap* mb = phase ? &p.tmB1 : &p.tmB0;
+    // Both operands of a Gram tile from one map (X, or dY / Z), at the pair's two token blocks.
+    const CUtensorMap* ma = Cfg::GROUPED ? (phase ? &grp->tmB[w.prob] : &grp->tmA[w.prob])
+                                         : (phase ? &p.tmA1 : &p.tmA0);
+    const CUtensorMap* mb = Cfg::GROUPED ? ma : (phase ? &p.tmB1 : &p.tmB0);
     tma_load_3d(sA, ma, bar, k0, w.m_blk * Cfg::BM, w.sample);
     tma_load_3d(sB, mb, bar, k0, w.n_blk * Cfg::BN, w.sample);
   } else if (Cfg::EPI == kEpiGhostShared) {
@@ -393,9 +420,10 @@ __device__ __forceinline__ void epilogue_unit(const UmmaParams& p, const Unit& w
     }
     ss = warp_sum(ss);
     const long long slot = static_cast<long long>(w.sample) * p.partial_stride + 4 * w.local + wq;
+    float* const partials = Cfg::GROUPED ? grp->partials[w.prob] : p.partials;
     if (lane == 0 && DP_DCHECK(4 * w.local + wq < p.partial_stride && in_buffer(slot, 1, p.partials_elems), 4u,
                                p.status))
-      p.partials[slot] = ss;
+      partials[slot] = ss;
   } else if (Cfg::EPI == kEpiGhostShared) {
     const int t = w.m_blk * Cfg::BM + row;
     float ss[kGhostSharedMaxOps] = {0.f, 0.f, 0.f};
@@ -545,7 +573,7 @@ __device__ __forceinline__ void umma_body(const UmmaParams& p, const UmmaGroup* 
       for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
         const Unit w = decode_unit<Cfg>(p, u, grp);
         for (int ph = 0; ok && ph < nphases; ++ph) {
-          const int kb_end = ph ? p.k_blocks1 : w.kb_end;
+          const int kb_end = ph ? w.kb1 : w.kb_end;
           const int kb_begin = ph ? 0 : w.kb_begin;
           for (int kb = kb_begin; kb < kb_end; ++kb) {
             if (!mbar_wait_bounded(smem_addr(empty + stage), phase ^ 1u, abort_flag, p.status, 1u)) {
@@ -589,7 +617,7 @@ __device__ __forceinline__ void umma_body(const UmmaParams& p, const UmmaGroup* 
         tc_fence_after();
         for (int ph = 0; ok && ph < nphases; ++ph) {
           const uint32_t d_tmem = tmem_base + buf * Cfg::ACC_COLS + ph * Cfg::BN;
-          const int kb_end = ph ? p.k_blocks1 : w.kb_end;
+          const int kb_end = ph ? w.kb1 : w.kb_end;
           const int kb_begin = ph ? 0 : w.kb_begin;
           for (int kb = kb_begin; kb < kb_end; ++kb) {
             if (!mbar_wait_bounded(smem_addr(full + stage), phase, abort_flag, p.status, 3u)) {

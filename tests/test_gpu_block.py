@@ -154,8 +154,10 @@ def test_shared_x_gram_ghost_block(mode):
     torch.cuda.synchronize()
     kinds = _lib.profiling_collect()
     _lib.profiling_enable(False)
-    # q/k/v share one launch, gate/up another; o and down each run the plain ghost kernel.
-    assert kinds["umma_ghost_shared"][1] == 2 and kinds["umma_ghost_norm"][1] == 2, kinds
+    # q/k/v share one launch, gate/up another; o and down run the plain ghost kernel: one grouped
+    # launch for both in per-layer mode (its batched schedule), one launch each in flat mode.
+    assert kinds["umma_ghost_shared"][1] == 2, kinds
+    assert kinds["umma_ghost_norm"][1] == (1 if mode == "per_layer" else 2), kinds
     for k, lin in enumerate(w.linears):
         n1 = _lib.dp_per_sample_norms(dev["X"][lin.x_key], dev["dY"][lin.name], method="ghost")
         assert torch.equal(norms[k], n1), lin.name      # same Gram tiles, same partial slots
@@ -214,6 +216,49 @@ def test_projected_block_against_oracle(mode):
         want = oracle.noise(a.shape[0], a.shape[1], float(np.float32(w.sigma)) * float(np.float32(C)), w.seed, 2,
                             lin.layer_id)
         record(f"projected block [{mode}]", lin.name, "noise", noise_excess(a, b, want), NOISE_ABS)
+        assert np.all(np.abs((a - b) - want) <= noise_tolerance(a, b)), lin.name
+
+
+def test_projected_block_with_split_x_grams_against_oracle():
+    """Few ghost units (B = 4, one 128-token block) over wide inputs (d = 1024, ffn = 2048): the
+    per-layer block step splits each X Gram over K (the shared q/k/v Gram in 2, o in 2, down in 4),
+    the single ghost layers run in one grouped launch, and the split partial sums must add up to
+    the oracle's norms; the clipped sums and the noise follow them."""
+    w = inputs.Workload("psplit", B=4, T=128, dtype="bf16", linears=inputs._block(0, 1024, 2048),
+                        C=0.9, sigma=0.8, seed=23, dy_var="per_layer")
+    data = inputs.generate(w)
+    X = {k: v.cuda() for k, v in data["X"].items()}
+    dY = {k: v.cuda() for k, v in data["dY"].items()}
+    r = 64
+    P = {l.name: _lib.dp_projection_matrix(torch.empty(l.d_out, r, dtype=torch.bfloat16, device="cuda"),
+                                           w.seed, l.layer_id) for l in w.linears}
+    layers = [{"X": X[l.x_key], "dY": dY[l.name], "P": P[l.name], "layer_id": l.layer_id, "C": w.C,
+               "norms_out": torch.empty(w.B, dtype=torch.float32, device="cuda")} for l in w.linears]
+    _lib.profiling_enable(True)
+    _lib.profiling_collect()
+    outs0, norms, _ = _lib.dp_block_step(layers, mode="per_layer", sigma=0.0, seed=w.seed, step=6, method="ghost")
+    torch.cuda.synchronize()
+    kinds = _lib.profiling_collect()
+    _lib.profiling_enable(False)
+    assert kinds["umma_ghost_shared"][1] == 2 and kinds["umma_ghost_norm"][1] == 1, kinds
+    outs1, _, _ = _lib.dp_block_step(layers, mode="per_layer", sigma=w.sigma, seed=w.seed, step=6, method="ghost")
+    torch.cuda.synchronize()
+    olayers = [{"X": inputs.as_f64(data["X"][l.x_key]), "dY": inputs.as_f64(data["dY"][l.name]),
+                "P": host(P[l.name]), "layer_id": l.layer_id, "C": float(np.float32(w.C))} for l in w.linears]
+    ref = oracle.block_step(olayers, None, 0.0, w.seed, 6, mode="per_layer")
+    tol = TOL["bf16"]
+    for k, lin in enumerate(w.linears):
+        rr = ref["layers"][k]
+        n_err, s_err = rel_max(host(norms[k]), rr["norms"]), rel_fro(host(outs0[k]), rr["S"])
+        record("projected block, split X Grams", lin.name, "norm", n_err, tol["norm"])
+        record("projected block, split X Grams", lin.name, "sum", s_err, tol["sum"])
+        assert n_err <= tol["norm"], (lin.name, n_err)
+        check_clip_decisions(host(norms[k]), rr["norms"], float(np.float32(w.C)))
+        assert s_err <= tol["sum"], (lin.name, s_err)
+        a, b = host(outs1[k]), host(outs0[k])
+        want = oracle.noise(a.shape[0], a.shape[1], float(np.float32(w.sigma)) * float(np.float32(w.C)), w.seed, 6,
+                            lin.layer_id)
+        record("projected block, split X Grams", lin.name, "noise", noise_excess(a, b, want), NOISE_ABS)
         assert np.all(np.abs((a - b) - want) <= noise_tolerance(a, b)), lin.name
 
 
