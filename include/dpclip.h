@@ -153,9 +153,9 @@ dp_status dp_projection_matrix(void* P, dp_dtype dt, int d_out, int r,
  *                rounds sigma*C*z to fp32 before adding it to the fp32 sum (within one ulp
  *                of rounding the fp64 sum once).  A ghost or explicit clipped sum that is
  *                split over K (small outputs) writes sigma*C*z rounded to fp32 first and adds
- *                its partial sums with fp32 atomics; an unsplit one adds the noise in its
- *                epilogue in fp64 and rounds once.  The noise is written on a second stream
- *                of the library beside the norm pass, joined before the call returns. */
+ *                its partial sums with fp32 atomics (the row-scaling launch before the sum
+ *                writes the noise); an unsplit one adds the noise in its epilogue in fp64 and
+ *                rounds once. */
 dp_status dp_linear_step(const void* X, const void* dY, const void* P, int r, dp_dtype dt,
                          int B, int T, int d_in, int d_out, float C, float sigma,
                          unsigned long long seed, unsigned long long step, unsigned layer_id,

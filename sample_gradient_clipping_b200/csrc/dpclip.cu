@@ -505,44 +505,30 @@ dp_status bf16_clipsum(const Shape& s, const void* A, const void* Bm, float* out
                       stream);
 }
 
-// `set`: write the noise instead of adding it (noise_add_kernel's SET mode).
-dp_status launch_noise_batch(const NoiseBatch& b, unsigned long long seed, StepRef step, cudaStream_t stream,
-                             bool set = false) {
+dp_status launch_noise_batch(const NoiseBatch& b, unsigned long long seed, StepRef step, cudaStream_t stream) {
   if (b.count == 0) return DP_OK;
   unsigned long long nblk = 0;
   for (int q = 0; q < b.count; ++q) nblk += (b.seg[q].total + 3) / 4;
   LaunchScope scope(kKindNoise, stream);
-  if (set)
-    DP_LAUNCH("noise_add_batch_kernel", noise_add_batch_kernel<true>, stream_grid(nblk, 256), 256, 0, stream, b,
-              philox_key_from_seed(seed), step);
-  else
-    DP_LAUNCH("noise_add_batch_kernel", noise_add_batch_kernel<false>, stream_grid(nblk, 256), 256, 0, stream, b,
-              philox_key_from_seed(seed), step);
-  return DP_OK;
-}
-
-dp_status launch_noise(float* G, unsigned long long total, double std_dev, unsigned long long seed,
-                       StepRef step, unsigned layer_id, cudaStream_t stream, bool set) {
-  LaunchScope scope(kKindNoise, stream);
-  // Large G: a persistent grid whose blocks stage the 32 KB of Box-Muller tables once each.
-  const PhiloxKey key = philox_key_from_seed(seed);
-  const bool staged = total >= (1ull << 22);
-  const int grid = staged ? std::min(stream_grid((total + 3) / 4, 256), sm_count() * 4)
-                          : stream_grid((total + 3) / 4, 256);
-#define DP_NOISE(ST_, SET_)                                                                               \
-  DP_LAUNCH("noise_add_kernel", noise_add_kernel<ST_, SET_>, grid, 256, 0, stream, G, total, std_dev, key, \
-            layer_id, step)
-  if (staged && set) DP_NOISE(true, true);
-  else if (staged) DP_NOISE(true, false);
-  else if (set) DP_NOISE(false, true);
-  else DP_NOISE(false, false);
-#undef DP_NOISE
+  DP_LAUNCH("noise_add_batch_kernel", noise_add_batch_kernel, stream_grid(nblk, 256), 256, 0, stream, b,
+            philox_key_from_seed(seed), step);
   return DP_OK;
 }
 
 dp_status launch_noise(float* G, unsigned long long total, double std_dev, unsigned long long seed,
                        StepRef step, unsigned layer_id, cudaStream_t stream) {
-  return launch_noise(G, total, std_dev, seed, step, layer_id, stream, false);
+  LaunchScope scope(kKindNoise, stream);
+  // Large G: a persistent grid whose blocks stage the 32 KB of Box-Muller tables once each.
+  const PhiloxKey key = philox_key_from_seed(seed);
+  if (total >= (1ull << 22)) {
+    const int grid = std::min(stream_grid((total + 3) / 4, 256), sm_count() * 4);
+    DP_LAUNCH("noise_add_kernel", noise_add_kernel<true>, grid, 256, 0, stream, G, total, std_dev, key,
+              layer_id, step);
+  } else {
+    DP_LAUNCH("noise_add_kernel", noise_add_kernel<false>, stream_grid((total + 3) / 4, 256), 256, 0, stream,
+              G, total, std_dev, key, layer_id, step);
+  }
+  return DP_OK;
 }
 
 // Z[N, r] = dY[N, n] P[n, r], bf16 out.
@@ -599,7 +585,8 @@ dp_status launch_norm_partials(const float* partials, int stride, int count, int
 // of its blocks covers, unless a block would cover too many samples or partial slots; then the
 // partials kernel runs first.
 dp_status launch_scale(const void* in, void* out, long long rows, int cols, int T, NormSource src,
-                       float C, cudaStream_t stream, const PartialsRef* partials = nullptr, int B = 0) {
+                       float C, cudaStream_t stream, const PartialsRef* partials = nullptr, int B = 0,
+                       const NoiseFill* fill = nullptr, unsigned long long seed = 0, StepRef step = StepRef{0u, nullptr}) {
   const unsigned long long vecs = static_cast<unsigned long long>(rows) * (cols / 8);
   const int grid = stream_grid(vecs, 256);
   PartialsRef pr{nullptr, 0, 0, nullptr, nullptr, nullptr};
@@ -620,9 +607,10 @@ dp_status launch_scale(const void* in, void* out, long long rows, int cols, int 
     }
   }
   LaunchScope scope(kKindScale, stream);
+  const NoiseFill nf = fill ? *fill : NoiseFill{nullptr, 0, 0.0, 0u};
   DP_LAUNCH("scale_rows_bf16_kernel", scale_rows_bf16_kernel, grid, 256, smem, stream,
             static_cast<const __nv_bfloat16*>(in), static_cast<__nv_bfloat16*>(out), rows, cols, T, src, pr,
-            C);
+            C, nf, philox_key_from_seed(seed), step);
   return DP_OK;
 }
 
@@ -835,9 +823,9 @@ NormSource ws_norm_source(const Call& c) {
 dp_status clipped_sum(Call& c, const void* X, const void* Z, NormSource src, float C, float* out,
                       int accumulate, double noise_std, unsigned long long seed,
                       StepRef step, unsigned layer_id, NoiseBatch* defer = nullptr,
-                      const PartialsRef* partials = nullptr, cudaEvent_t noise_written = nullptr) {
-  // noise_written: out already holds the noise (split K), written on another stream; the
-  // contraction waits for that event and adds its partial sums to it.
+                      const PartialsRef* partials = nullptr, bool prefill_noise = false) {
+  // prefill_noise (a clipped sum split over K, accumulate = 0): the row-scaling launch also
+  // writes the noise into out, and the contraction adds its partial sums to it.
   const Shape& s = c.s;
   if (s.dt == DP_F32) {
     dim3 grid(ceil_div(s.ne(), kF32Tile), ceil_div(s.m, kF32Tile));
@@ -851,17 +839,18 @@ dp_status clipped_sum(Call& c, const void* X, const void* Z, NormSource src, flo
   // Fold c_i into the narrower operand: one extra read + write of N * min(m, ne) bf16.
   void* scaled = c.ws + c.L.scaled;
   dp_status st;
-  const bool preset = (noise_written != nullptr);
+  const NoiseFill fill{out, static_cast<unsigned long long>(s.m) * s.ne(), noise_std, layer_id};
+  const NoiseFill* nf = prefill_noise ? &fill : nullptr;
   if (s.ne() <= s.m) {
-    if ((st = launch_scale(Z, scaled, s.N(), s.ne(), s.T, src, C, c.stream, partials, s.B)) != DP_OK) return st;
-    if (preset) DP_CUDA(cudaStreamWaitEvent(c.stream, noise_written, 0));
+    if ((st = launch_scale(Z, scaled, s.N(), s.ne(), s.T, src, C, c.stream, partials, s.B, nf, seed, step)) != DP_OK)
+      return st;
     return bf16_clipsum(s, X, scaled, out, accumulate, noise_std, seed, step, layer_id, c.status(), c.stream,
-                        defer, preset);
+                        defer, prefill_noise);
   }
-  if ((st = launch_scale(X, scaled, s.N(), s.m, s.T, src, C, c.stream, partials, s.B)) != DP_OK) return st;
-  if (preset) DP_CUDA(cudaStreamWaitEvent(c.stream, noise_written, 0));
+  if ((st = launch_scale(X, scaled, s.N(), s.m, s.T, src, C, c.stream, partials, s.B, nf, seed, step)) != DP_OK)
+    return st;
   return bf16_clipsum(s, scaled, Z, out, accumulate, noise_std, seed, step, layer_id, c.status(), c.stream,
-                      defer, preset);
+                      defer, prefill_noise);
 }
 
 dp_status resolve_method(const Shape& s, dp_norm_method method, dp_norm_method* out) {
@@ -1417,11 +1406,16 @@ dp_status launch_clipsum_groups(const dp_layer* layers, const std::vector<int>& 
 // layer's blocks sum their samples' norm partials themselves, unless a block would cover too
 // many samples or slots; that layer's partials are then summed first.
 dp_status launch_scale_batch(const dp_layer* layers, const std::vector<int>& ls, const std::vector<int>& counts,
-                             dp_dtype dt, int B, int T, const BlockLayout& Lb, uint8_t* ws, cudaStream_t stream) {
+                             dp_dtype dt, int B, int T, const BlockLayout& Lb, uint8_t* ws, cudaStream_t stream,
+                             const std::vector<NoiseFill>& fills, unsigned long long seed, StepRef step) {
   ScaleBatch b;
   memset(&b, 0, sizeof(b));
   b.T = T;
   b.count = static_cast<int>(ls.size());
+  b.fills = static_cast<int>(fills.size());
+  for (int q = 0; q < b.fills; ++q) b.fill[q] = fills[q];
+  b.key = philox_key_from_seed(seed);
+  b.step = step;
   unsigned long long total_vecs = 0;
   std::vector<unsigned long long> vecs(ls.size());
   for (size_t q = 0; q < ls.size(); ++q) {
@@ -1495,48 +1489,25 @@ dp_status block_step(const dp_layer* layers, int L, dp_dtype dt, int B, int T, d
     bool side_pending = false;  // reduces on the side stream the caller's stream has not joined
     std::vector<int> batch_layers, batch_counts;  // batched schedule: layers waiting for their sums
     std::vector<int> ghost_single, ghost_single_at;  // batched schedule: single ghost layers, their slots
-    // Batched schedule: the noise of every split-K clipped sum is written into its output first,
-    // in one launch on the second stream beside the norm passes; those sums then add to it.
+    // Batched schedule: the noise of every split-K clipped sum (of every clipped sum when they
+    // run grouped, zeros at sigma 0) is written into its output by the batched row-scaling
+    // launch; those sums then add their partial sums to it.
     std::vector<bool> preset(L, false);
-    cudaEvent_t noise_written = nullptr, noise_fork = nullptr;
-    NoiseBatch noise_pending;
-    noise_pending.count = 0;
-    auto enqueue_preset_noise = [&]() -> dp_status {
-      if (noise_pending.count == 0) return DP_OK;
-      dp_status e;
-      DP_CUDA(cudaStreamWaitEvent(side, noise_fork, 0));
-      if ((e = launch_noise_batch(noise_pending, seed, step, side, true)) != DP_OK) return e;
-      if ((e = event_ring().next(&noise_written)) != DP_OK) return e;
-      DP_CUDA(cudaEventRecord(noise_written, side));
-      noise_pending.count = 0;
-      return DP_OK;
-    };
-    // Grouped clipped sums (batched schedule, all on the one-SM engine with one tile width):
-    // every output is prefilled, with its noise or with zeros, and added to by atomics.
+    std::vector<NoiseFill> fills;
     std::vector<int> batch_all;
     if (Lb.batched_scale)
       for (const auto& g : Lb.groups)
         if (Lb.methods[g[0]] != DP_NORM_ONCE) batch_all.insert(batch_all.end(), g.begin(), g.end());
     const bool grouped_sums = Lb.batched_scale && dt == DP_BF16 && clipsums_groupable(layers, batch_all, B, T, dt);
     if (Lb.batched_scale && (sigma != 0.0f || grouped_sums)) {
-      NoiseBatch nb;
-      nb.count = 0;
       for (int l : batch_all) {
         const Shape s = layer_shape(layers[l], B, T, dt);
-        if ((grouped_sums || clipsum_plan(s).splits > 1) && nb.count < kMaxNoiseSegments) {
-          nb.seg[nb.count++] = NoiseSegment{layers[l].G_out, static_cast<unsigned long long>(s.m) * s.ne(),
-                                            sigma == 0.0f ? 0.0
-                                                          : static_cast<double>(sigma) * static_cast<double>(layers[l].C),
-                                            layers[l].layer_id};
+        if ((grouped_sums || clipsum_plan(s).splits > 1) && static_cast<int>(fills.size()) < kMaxScaleSegments) {
+          fills.push_back(NoiseFill{layers[l].G_out, static_cast<unsigned long long>(s.m) * s.ne(),
+                                    sigma == 0.0f ? 0.0 : static_cast<double>(sigma) * static_cast<double>(layers[l].C),
+                                    layers[l].layer_id});
           preset[l] = true;
         }
-      }
-      if (nb.count > 0) {
-        // Forked here; enqueued after the first norm pass (see the single-linear step).
-        if (!Lb.overlap && (st = side_stream(&side)) != DP_OK) return st;
-        if ((st = event_ring().next(&noise_fork)) != DP_OK) return st;
-        DP_CUDA(cudaEventRecord(noise_fork, stream));
-        noise_pending = nb;
       }
     }
     // Each group: its norms, then each member's clipped sum with its own bound and noise.
@@ -1599,7 +1570,6 @@ dp_status block_step(const dp_layer* layers, int L, dp_dtype dt, int B, int T, d
                               pairs, Lb.partial_stride);
         }
         if ((st = block_group_norms(layers, g, dt, B, T, Lb, ws, stream, &count, base, xs)) != DP_OK) return st;
-        if ((st = enqueue_preset_noise()) != DP_OK) return st;  // after the first norm pass
         for (int l : g) {
           batch_layers.push_back(l);
           batch_counts.push_back(count);
@@ -1627,14 +1597,12 @@ dp_status block_step(const dp_layer* layers, int L, dp_dtype dt, int B, int T, d
       if ((st = launch_ghost_group(layers, ghost_single, dt, B, T, Lb, ws, stream, &counts)) != DP_OK) return st;
       for (size_t i = 0; i < ghost_single.size(); ++i) batch_counts[ghost_single_at[i]] = counts[i];
     }
-    if ((st = enqueue_preset_noise()) != DP_OK) return st;  // (unless a norm pass enqueued it)
     if (!batch_layers.empty()) {
-      if ((st = launch_scale_batch(layers, batch_layers, batch_counts, dt, B, T, Lb, ws, stream)) != DP_OK) return st;
-      if (grouped_sums) {
-        if (noise_written) DP_CUDA(cudaStreamWaitEvent(stream, noise_written, 0));  // join
-        noise_written = nullptr;
-        if ((st = launch_clipsum_groups(layers, batch_layers, dt, B, T, Lb, ws, stream)) != DP_OK) return st;
-      }
+      if ((st = launch_scale_batch(layers, batch_layers, batch_counts, dt, B, T, Lb, ws, stream, fills, seed,
+                                   step)) != DP_OK)
+        return st;
+      if (grouped_sums && (st = launch_clipsum_groups(layers, batch_layers, dt, B, T, Lb, ws, stream)) != DP_OK)
+        return st;
       for (int l : grouped_sums ? std::vector<int>() : batch_layers) {
         const dp_layer& y = layers[l];
         const Shape s = layer_shape(y, B, T, dt);
@@ -1642,10 +1610,6 @@ dp_status block_step(const dp_layer* layers, int L, dp_dtype dt, int B, int T, d
         if ((st = block_operand(layers, l, dt, B, T, Lb, ws, stream, false, &Z)) != DP_OK) return st;
         const void* scaled = ws + Lb.scaled_l[l];
         const double noise_std = (sigma == 0.0f) ? 0.0 : static_cast<double>(sigma) * static_cast<double>(y.C);
-        if (preset[l] && noise_written) {  // join the second stream once, before the first such sum
-          DP_CUDA(cudaStreamWaitEvent(stream, noise_written, 0));
-          noise_written = nullptr;
-        }
         if ((st = bf16_clipsum(s, s.ne() <= s.m ? y.X : scaled, s.ne() <= s.m ? scaled : Z, y.G_out, 0, noise_std,
                                seed, step, y.layer_id, reinterpret_cast<uint32_t*>(ws), stream, &deferred,
                                preset[l])) != DP_OK)
@@ -1866,34 +1830,17 @@ dp_status linear_step(const void* X, const void* dY, const void* P, int r, dp_dt
   }
   if (dt == DP_BF16) {
     // A clipped sum split over K adds its partial sums by atomics: its noise is written into
-    // G_out first, on the library's second stream beside the norm pass and the row scaling.
-    // The fork point is recorded before the norm pass but the noise is enqueued after it, so that
-    // the norm pass's CTAs are placed first and the noise blocks take the thread slots left.
-    cudaEvent_t noise_written = nullptr, fork = nullptr;
-    const bool preset = (noise_std != 0.0 && clipsum_plan(c.s).splits > 1);
-    if (preset) {
-      if ((st = event_ring().next(&fork)) != DP_OK) return st;
-      DP_CUDA(cudaEventRecord(fork, c.stream));
-    }
+    // G_out first, by the row-scaling launch that precedes it.
+    const bool prefill = (noise_std != 0.0 && clipsum_plan(c.s).splits > 1);
     // The norm partials are summed by the row-scaling kernel of the clipped sum.
     int count = 0;
     if ((st = bf16_norms(c.s, X, Z, m, c.partials(), c.L.partial_stride, &count, c.status(), c.stream)) !=
         DP_OK)
       return st;
-    if (preset) {
-      cudaStream_t side;
-      if ((st = side_stream(&side)) != DP_OK) return st;
-      DP_CUDA(cudaStreamWaitEvent(side, fork, 0));
-      if ((st = launch_noise(G_out, static_cast<unsigned long long>(mn), noise_std, seed, step, layer_id, side,
-                             true)) != DP_OK)
-        return st;
-      if ((st = event_ring().next(&noise_written)) != DP_OK) return st;
-      DP_CUDA(cudaEventRecord(noise_written, side));
-    }
     const PartialsRef pr{c.partials(), c.L.partial_stride, count, c.norm2_f32(), norms_out,
                          norms_out ? c.c() : nullptr};
     return clipped_sum(c, X, Z, ws_norm_source(c), C, G_out, 0, noise_std, seed, step, layer_id, nullptr, &pr,
-                       noise_written);  // the wait on noise_written joins the second stream
+                       prefill);
   }
   if ((st = norms_into_ws(c, X, Z, m, C, nullptr)) != DP_OK) return st;
   const NormSource src = ws_norm_source(c);

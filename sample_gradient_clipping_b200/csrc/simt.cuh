@@ -20,9 +20,7 @@ namespace dpclip {
 // G[k] = fp32(G[k] + std * z_k), z from stream 0.  One thread per Philox block of 4 elements.
 // STAGED: the Box-Muller tables are copied to shared memory once per block (large G); else
 // they are read through the read-only cache, which saves the copy's latency on small G.
-// SET: G[k] = fp32(std * z_k) instead (the noise written into a buffer that a split-K sum then
-// adds its partial sums to).
-template <bool STAGED, bool SET = false>
+template <bool STAGED>
 __global__ void noise_add_kernel(float* __restrict__ G, unsigned long long total, double std_dev,
                                  PhiloxKey key, uint32_t layer_id, StepRef step) {
   griddep_enter();
@@ -44,20 +42,15 @@ __global__ void noise_add_kernel(float* __restrict__ G, unsigned long long total
     if (k0 + 3 < total) {
       if (!DP_DCHECK(in_buffer(static_cast<long long>(k0), 4, static_cast<long long>(total)), 20u, nullptr)) continue;
       float4* p = reinterpret_cast<float4*>(G + k0);
-      if constexpr (SET) {
-        *p = make_float4(__double2float_rn(z[0]), __double2float_rn(z[1]), __double2float_rn(z[2]),
-                         __double2float_rn(z[3]));
-      } else {
-        float4 g = *p;
-        g.x = static_cast<float>(static_cast<double>(g.x) + z[0]);
-        g.y = static_cast<float>(static_cast<double>(g.y) + z[1]);
-        g.z = static_cast<float>(static_cast<double>(g.z) + z[2]);
-        g.w = static_cast<float>(static_cast<double>(g.w) + z[3]);
-        *p = g;
-      }
+      float4 g = *p;
+      g.x = static_cast<float>(static_cast<double>(g.x) + z[0]);
+      g.y = static_cast<float>(static_cast<double>(g.y) + z[1]);
+      g.z = static_cast<float>(static_cast<double>(g.z) + z[2]);
+      g.w = static_cast<float>(static_cast<double>(g.w) + z[3]);
+      *p = g;
     } else {
       for (int q = 0; q < 4 && k0 + q < total; ++q)
-        G[k0 + q] = SET ? __double2float_rn(z[q]) : static_cast<float>(static_cast<double>(G[k0 + q]) + z[q]);
+        G[k0 + q] = static_cast<float>(static_cast<double>(G[k0 + q]) + z[q]);
     }
   }
 }
@@ -78,7 +71,6 @@ struct NoiseBatch {
   int count;
 };
 
-template <bool SET = false>
 __global__ void noise_add_batch_kernel(NoiseBatch b, PhiloxKey key, StepRef step) {
   griddep_enter();
   const uint32_t step_lo = step.get();
@@ -93,13 +85,12 @@ __global__ void noise_add_batch_kernel(NoiseBatch b, PhiloxKey key, StepRef step
       ++q;
     }
     const NoiseSegment& sg = b.seg[q];
-    double z[4] = {0.0, 0.0, 0.0, 0.0};
-    if (!SET || sg.std_dev != 0.0)  // SET with std 0: zeros (a prefill for atomic sums)
-      normals4(static_cast<uint32_t>(jj), sg.layer_id, step_lo, kStreamNoise, key, z, NoiseTablesGlobal{},
-               sg.std_dev);
+    double z[4];
+    normals4(static_cast<uint32_t>(jj), sg.layer_id, step_lo, kStreamNoise, key, z, NoiseTablesGlobal{},
+             sg.std_dev);
     const unsigned long long k0 = 4 * jj;
     for (int e = 0; e < 4 && k0 + e < sg.total; ++e)
-      sg.G[k0 + e] = SET ? __double2float_rn(z[e]) : static_cast<float>(static_cast<double>(sg.G[k0 + e]) + z[e]);
+      sg.G[k0 + e] = static_cast<float>(static_cast<double>(sg.G[k0 + e]) + z[e]);
   }
 }
 
@@ -340,11 +331,52 @@ __device__ __forceinline__ void scale_rows_body(const __nv_bfloat16* __restrict_
   }
 }
 
+// The noise of a clipped sum split over K, written into its output before the sum (which then
+// adds its partial sums by atomics): out[k] = fp32(std * z_k), z from stream 0 under the
+// layer's counter; std = 0 writes zeros.  The row-scaling kernel that precedes the sum carries
+// it: the scaling is an HBM stream with idle arithmetic pipes, and the sum needs both.
+struct NoiseFill {
+  float* G;                   // null: nothing to write
+  unsigned long long total;   // elements
+  double std_dev;
+  uint32_t layer_id;
+};
+
+// This block's share (block `blk` of `nblk`) of the Philox blocks of `fills` (count of them).
+__device__ __forceinline__ void noise_fill_share(const NoiseFill* fills, int count, PhiloxKey key, uint32_t step_lo,
+                                                 long long blk, long long nblk) {
+  unsigned long long total_blocks = 0;
+  for (int q = 0; q < count; ++q) total_blocks += (fills[q].total + 3) / 4;
+  for (unsigned long long j = blk * static_cast<unsigned long long>(blockDim.x) + threadIdx.x; j < total_blocks;
+       j += static_cast<unsigned long long>(nblk) * blockDim.x) {
+    unsigned long long jj = j;
+    int q = 0;
+    while ((fills[q].total + 3) / 4 <= jj) {  // the fill holding global block j
+      jj -= (fills[q].total + 3) / 4;
+      ++q;
+    }
+    const NoiseFill& f = fills[q];
+    double z[4] = {0.0, 0.0, 0.0, 0.0};
+    if (f.std_dev != 0.0)
+      normals4(static_cast<uint32_t>(jj), f.layer_id, step_lo, kStreamNoise, key, z, NoiseTablesGlobal{}, f.std_dev);
+    const unsigned long long k0 = 4 * jj;
+    if (k0 + 3 < f.total) {
+      if (!DP_DCHECK(in_buffer(static_cast<long long>(k0), 4, static_cast<long long>(f.total)), 28u, nullptr)) continue;
+      *reinterpret_cast<float4*>(f.G + k0) = make_float4(__double2float_rn(z[0]), __double2float_rn(z[1]),
+                                                         __double2float_rn(z[2]), __double2float_rn(z[3]));
+    } else {
+      for (int e = 0; e < 4 && k0 + e < f.total; ++e) f.G[k0 + e] = __double2float_rn(z[e]);
+    }
+  }
+}
+
 __global__ void scale_rows_bf16_kernel(const __nv_bfloat16* __restrict__ in,
                                        __nv_bfloat16* __restrict__ out, long long rows, int cols,
-                                       int T, NormSource src, PartialsRef pr, float C) {
+                                       int T, NormSource src, PartialsRef pr, float C, NoiseFill fill,
+                                       PhiloxKey key, StepRef step) {
   griddep_enter();
   scale_rows_body(in, out, rows, cols, T, src, pr, C, blockIdx.x, gridDim.x);
+  if (fill.G != nullptr) noise_fill_share(&fill, 1, key, step.get(), blockIdx.x, gridDim.x);
 }
 
 // The row scalings of several layers in one launch (a per-layer block step scales every
@@ -366,6 +398,10 @@ struct ScaleBatch {
   ScaleSegment seg[kMaxScaleSegments];
   int count;
   int T;
+  NoiseFill fill[kMaxScaleSegments];  // noise (or zeros) for the split-K sums that follow
+  int fills;
+  PhiloxKey key;
+  StepRef step;
 };
 
 __global__ void scale_rows_bf16_batch_kernel(ScaleBatch b) {
@@ -375,6 +411,7 @@ __global__ void scale_rows_bf16_batch_kernel(ScaleBatch b) {
   const ScaleSegment& sg = b.seg[q];
   if (!DP_DCHECK(static_cast<int>(blockIdx.x) - sg.first_block < sg.blocks, 27u, nullptr)) return;
   scale_rows_body(sg.in, sg.out, sg.rows, sg.cols, b.T, sg.src, sg.pr, sg.C, blockIdx.x - sg.first_block, sg.blocks);
+  if (b.fills > 0) noise_fill_share(b.fill, b.fills, b.key, b.step.get(), blockIdx.x, gridDim.x);
 }
 
 // out[e] = fp32(sum_i c_i Gs[i][e] + std * z_e) over the per-sample bf16 gradients that the
