@@ -1318,7 +1318,10 @@ dp_status block_layer_sum(const dp_layer* layers, int l, dp_dtype dt, int B, int
   const void* Z;
   dp_status st = block_operand(layers, l, dt, B, T, Lb, ws, stream, false, &Z);  // formed by the norms
   if (st != DP_OK) return st;
-  return clipped_sum(c, y.X, Z, src, C, y.G_out, 0, noise_std, seed, step, y.layer_id, defer, partials);
+  // A bf16 sum split over K: its row-scaling launch writes the noise first (as in one linear).
+  const bool prefill = (dt == DP_BF16 && noise_std != 0.0 && clipsum_plan(s).splits > 1);
+  return clipped_sum(c, y.X, Z, src, C, y.G_out, 0, noise_std, seed, step, y.layer_id, defer, partials,
+                     prefill);
 }
 
 NormSource layer_norm_source(const BlockLayout& Lb, uint8_t* ws, int l, int B, dp_dtype dt) {
@@ -1472,7 +1475,8 @@ dp_status block_step(const dp_layer* layers, int L, dp_dtype dt, int B, int T, d
   DP_CUDA(cudaMemsetAsync(ws, 0, Lb.c, stream));
   // Every projected layer's Z = dY P, grouped (bf16).
   if ((st = block_projections(layers, L, dt, B, T, Lb, ws, stream)) != DP_OK) return st;
-  // Noise of split-K clipped sums, added in one launch at the end of the step.
+  // Noise of split-K clipped sums that no row-scaling launch writes (past the batched launch's
+  // segment table), added in one launch at the end of the step.
   NoiseBatch deferred;
   deferred.count = 0;
   if (mode == DP_CLIP_PER_LAYER) {
