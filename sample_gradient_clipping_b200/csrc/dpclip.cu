@@ -121,6 +121,40 @@ int partial_slots(const Shape& s) {
   return static_cast<int>(most);
 }
 
+// The ghost units (one per sample and upper-triangular pair of 128-token blocks) that are cut
+// in parts, and how.  The ghost kernel is persistent, so the units of the last, partial wave
+// on the SMs would run alone while the other SMs wait; each of them is cut into parts over the
+// K of the deeper Gram (X over d_in, or dY over the clip-space width) when that Gram is at
+// least twice as deep as the other (each part still forms the other Gram whole).  With fewer
+// units than SMs every unit is such a tail unit.  A function of the shape alone (and the SM
+// count): every launch that forms this linear's ghost norm (alone, grouped with other linears,
+// or sharing its X Gram) cuts the same units the same way and writes the same partials, so the
+// norms are bitwise the same whichever entry point formed them.  At most
+// partial_slots(s) / (4 pairs) parts, so the partials fit every workspace layout.
+struct GhostSplit {
+  int full;     // units [0, full) whole
+  int parts;    // parts of each later unit (1: none)
+  bool over_x;  // parts of the X Gram's K (else of the dY Grams')
+};
+GhostSplit ghost_split(const Shape& s) {
+  const int t_tiles = (s.T + 127) / 128;
+  const int pairs = t_tiles * (t_tiles + 1) / 2;
+  const int units = s.B * pairs;
+  const int kx = (s.m + 63) / 64, k1 = (s.ne() + 63) / 64;
+  const int sms = sm_count();
+  const int tail = units % sms;
+  const bool over_x = kx >= 2 * k1;
+  if (tail == 0 || !(over_x || k1 >= 2 * kx)) return GhostSplit{units, 1, false};
+  const int kd = over_x ? kx : k1;
+  int parts = std::min(sms / tail, std::min(kd, partial_slots(s) / (4 * pairs)));
+  if (parts < 2) return GhostSplit{units, 1, false};
+  parts = ceil_div(kd, ceil_div(kd, parts));  // every part non-empty
+  return GhostSplit{units - tail, parts, over_x};
+}
+
+// Units of a ghost launch for one linear under its split, and its partial slots per sample.
+int ghost_units(const GhostSplit& g, int units) { return g.parts > 1 ? g.full + (units - g.full) * g.parts : units; }
+
 WsLayout ws_layout(const Shape& s, dp_norm_method method) {
   WsLayout L;
   size_t off = 256;  // status word(s)
@@ -329,7 +363,7 @@ int stream_grid(unsigned long long work_items, int threads) {
 // `store`, the explicit tiles of every G_i are also written there in bf16 ([B][d_in][ne]).
 dp_status bf16_norms(const Shape& s, const void* X, const void* Z, dp_norm_method method,
                      float* partials, int stride, int* count, uint32_t* status, cudaStream_t stream,
-                     __nv_bfloat16* store = nullptr, int x_splits = 1) {
+                     __nv_bfloat16* store = nullptr) {
   UmmaParams p = base_params(status);
   p.partials = partials;
   p.partial_stride = stride;
@@ -347,9 +381,12 @@ dp_status bf16_norms(const Shape& s, const void* X, const void* Z, dp_norm_metho
     p.pairs_per_sample = p.t_tiles * (p.t_tiles + 1) / 2;
     p.k_blocks = ceil_div(s.m, 64);
     p.k_blocks1 = ceil_div(ne, 64);
-    p.x_splits = x_splits;
-    p.num_units = s.B * p.pairs_per_sample * x_splits;
-    *count = 4 * p.pairs_per_sample * x_splits;
+    const GhostSplit g = ghost_split(s);
+    p.split_full_units = g.full;
+    p.split_parts = g.parts;
+    p.split_over_x = g.over_x ? 1 : 0;
+    p.num_units = ghost_units(g, s.B * p.pairs_per_sample);
+    *count = 4 * p.pairs_per_sample * g.parts;
     return launch_umma<Cfg>(p, stream);
   }
   dp_status st;
@@ -386,7 +423,7 @@ dp_status bf16_norms(const Shape& s, const void* X, const void* Z, dp_norm_metho
 // partials go to partials + j * op_stride, laid out as for bf16_norms.
 dp_status bf16_norms_ghost_shared(const Shape& s, const void* X, const void* const* Zs, int k,
                                   float* partials, int stride, long long op_stride, int* count,
-                                  uint32_t* status, cudaStream_t stream, int x_splits = 1) {
+                                  uint32_t* status, cudaStream_t stream) {
   if (k < 1 || k > kGhostSharedMaxOps) return DP_ERR_INVALID_ARG;
   UmmaParams p = base_params(status);
   p.partials = partials;
@@ -404,9 +441,12 @@ dp_status bf16_norms_ghost_shared(const Shape& s, const void* X, const void* con
   p.pairs_per_sample = p.t_tiles * (p.t_tiles + 1) / 2;
   p.k_blocks = ceil_div(s.m, 64);
   p.k_blocks1 = ceil_div(ne, 64);
-  p.x_splits = x_splits;
-  p.num_units = s.B * p.pairs_per_sample * x_splits;
-  *count = 4 * p.pairs_per_sample * x_splits;
+  const GhostSplit g = ghost_split(s);  // the split of one member alone: the members' partials are theirs
+  p.split_full_units = g.full;
+  p.split_parts = g.parts;
+  p.split_over_x = g.over_x ? 1 : 0;
+  p.num_units = ghost_units(g, s.B * p.pairs_per_sample);
+  *count = 4 * p.pairs_per_sample * g.parts;
   return launch_umma<UmmaConfig<128, kEpiGhostShared>>(p, stream);
 }
 
@@ -584,11 +624,29 @@ dp_status launch_norm_partials(const float* partials, int stride, int count, int
 // With `partials` (B samples), the scaling kernel forms the clip factors of the samples each
 // of its blocks covers, unless a block would cover too many samples or partial slots; then the
 // partials kernel runs first.
+// Blocks of a row-scaling kernel that are resident on one SM at once.  The scaling launches
+// are short (tens of microseconds): a grid of exactly one wave of resident blocks keeps every
+// block's prologue (its samples' clip factors) off the critical path of a second wave.
+int scale_blocks_per_sm(bool batch) {
+  static int cached[2][64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
+  int& c = cached[batch ? 1 : 0][dev & 63];
+  if (c == 0) {
+    int n = 0;
+    const cudaError_t e =
+        batch ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, scale_rows_bf16_batch_kernel, 256, 1024)
+              : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, scale_rows_bf16_kernel, 256, 1024);
+    c = (e == cudaSuccess && n > 0) ? n : 4;
+  }
+  return c;
+}
+
 dp_status launch_scale(const void* in, void* out, long long rows, int cols, int T, NormSource src,
                        float C, cudaStream_t stream, const PartialsRef* partials = nullptr, int B = 0,
                        const NoiseFill* fill = nullptr, unsigned long long seed = 0, StepRef step = StepRef{0u, nullptr}) {
   const unsigned long long vecs = static_cast<unsigned long long>(rows) * (cols / 8);
-  const int grid = stream_grid(vecs, 256);
+  const int grid = std::min(stream_grid(vecs, 256), sm_count() * scale_blocks_per_sm(false));
   PartialsRef pr{nullptr, 0, 0, nullptr, nullptr, nullptr};
   size_t smem = 0;
   if (partials) {
@@ -1192,26 +1250,13 @@ dp_status block_projections(const dp_layer* layers, int L, dp_dtype dt, int B, i
   return DP_OK;
 }
 
-// K splits of a ghost unit's X Gram (kx K blocks; its dY Grams take k1 blocks in all) so that
-// the units of a launch that would fill under a third of the SMs become more, shorter ones:
-// about 8 X blocks a split, no more than the partial slots hold (4 per split and pair).
-int ghost_x_splits(int kx, int k1, int units, int pairs, int stride) {
-  if (units * 3 >= sm_count()) return 1;
-  int xs = kx / std::max(8, k1);
-  xs = std::min(xs, stride / (4 * pairs));
-  xs = std::max(1, std::min(xs, kx));
-  return ceil_div(kx, ceil_div(kx, xs));  // every split non-empty
-}
-
 // Ghost-norm partials of single (unshared) ghost layers `ls` in grouped launches of up to
-// kMaxGroup problems, each with its own X and dY (or Z) maps, partial set and X-Gram split.
+// kMaxGroup problems, each with its own X and dY (or Z) maps, partial set and unit split.
 dp_status launch_ghost_group(const dp_layer* layers, const std::vector<int>& ls, dp_dtype dt, int B, int T,
                              const BlockLayout& Lb, uint8_t* ws, cudaStream_t stream, std::vector<int>* counts) {
   dp_status st;
   const int t_tiles = ceil_div(T, 128);
   const int pairs = t_tiles * (t_tiles + 1) / 2;
-  int total_units = 0;
-  for (size_t i = 0; i < ls.size(); ++i) total_units += B * pairs;
   for (size_t c0 = 0; c0 < ls.size(); c0 += kMaxGroup) {
     const int count = static_cast<int>(std::min<size_t>(kMaxGroup, ls.size() - c0));
     UmmaParams p = base_params(reinterpret_cast<uint32_t*>(ws));
@@ -1231,11 +1276,14 @@ dp_status launch_ghost_group(const dp_layer* layers, const std::vector<int>& ls,
       if ((st = map_3d(&g.tmB[q], Z, B, T, s.ne(), 128)) != DP_OK) return st;
       g.k_blocks[q] = ceil_div(s.m, 64);
       g.k_blocks1[q] = ceil_div(s.ne(), 64);
-      g.x_splits[q] = ghost_x_splits(g.k_blocks[q], g.k_blocks1[q], total_units, pairs, Lb.partial_stride);
       g.partials[q] = reinterpret_cast<float*>(ws + Lb.partials) + Lb.partial_set[l] * Lb.partial_op_stride;
       g.unit_begin[q] = units;
-      units += B * pairs * g.x_splits[q];
-      (*counts)[c0 + q] = 4 * pairs * g.x_splits[q];
+      const GhostSplit gs = ghost_split(s);
+      g.split_full_units[q] = gs.full;
+      g.split_parts[q] = gs.parts;
+      g.split_over_x[q] = gs.over_x ? 1 : 0;
+      units += ghost_units(gs, B * pairs);
+      (*counts)[c0 + q] = 4 * pairs * gs.parts;
     }
     g.unit_begin[count] = units;
     p.num_units = units;
@@ -1248,7 +1296,7 @@ dp_status launch_ghost_group(const dp_layer* layers, const std::vector<int>& ls,
 // layer's norms_out when given (gradients-once layers also keep their tiles).
 dp_status block_group_norms(const dp_layer* layers, const std::vector<int>& g, dp_dtype dt, int B, int T,
                             const BlockLayout& Lb, uint8_t* ws, cudaStream_t stream, int* count_out = nullptr,
-                            float* partials_base = nullptr, int x_splits = 1) {
+                            float* partials_base = nullptr) {
   dp_status st;
   uint32_t* status = reinterpret_cast<uint32_t*>(ws);
   const dp_layer& y0 = layers[g[0]];
@@ -1274,7 +1322,7 @@ dp_status block_group_norms(const dp_layer* layers, const std::vector<int>& g, d
   int count = 0;
   if (g.size() > 1) {
     if ((st = bf16_norms_ghost_shared(s, y0.X, Zs, static_cast<int>(g.size()), partials, Lb.partial_stride,
-                                      Lb.partial_op_stride, &count, status, stream, x_splits)) != DP_OK)
+                                      Lb.partial_op_stride, &count, status, stream)) != DP_OK)
       return st;
   } else {
     const bool once = (Lb.methods[g[0]] == DP_NORM_ONCE);
@@ -1426,7 +1474,7 @@ dp_status launch_scale_batch(const dp_layer* layers, const std::vector<int>& ls,
     vecs[q] = static_cast<unsigned long long>(s.N()) * (std::min(s.m, s.ne()) / 8);
     total_vecs += vecs[q];
   }
-  const int grid = stream_grid(total_vecs, 256);
+  const int grid = std::min(stream_grid(total_vecs, 256), sm_count() * scale_blocks_per_sm(true));
   int first = 0;
   size_t smem = 0;
   dp_status st;
@@ -1566,14 +1614,7 @@ dp_status block_step(const dp_layer* layers, int L, dp_dtype dt, int B, int T, d
         }
         int count = 0;
         float* base = reinterpret_cast<float*>(ws + Lb.partials) + Lb.partial_set[g[0]] * Lb.partial_op_stride;
-        int xs = 1;
-        if (dt == DP_BF16 && g.size() > 1) {  // a shared X Gram: split it when its units are few
-          const Shape s0 = layer_shape(layers[g[0]], B, T, dt);
-          const int tt = ceil_div(T, 128), pairs = tt * (tt + 1) / 2;
-          xs = ghost_x_splits(ceil_div(s0.m, 64), static_cast<int>(g.size()) * ceil_div(s0.ne(), 64), B * pairs,
-                              pairs, Lb.partial_stride);
-        }
-        if ((st = block_group_norms(layers, g, dt, B, T, Lb, ws, stream, &count, base, xs)) != DP_OK) return st;
+        if ((st = block_group_norms(layers, g, dt, B, T, Lb, ws, stream, &count, base)) != DP_OK) return st;
         for (int l : g) {
           batch_layers.push_back(l);
           batch_counts.push_back(count);

@@ -298,7 +298,13 @@ __device__ __forceinline__ void scale_rows_body(const __nv_bfloat16* __restrict_
   }
   // Four vectors per thread and iteration, all four loads issued before the first is used, so
   // each thread keeps four 16-byte loads in flight (one at a time left the stream latency-bound).
+  // A thread's vectors only move forward, so its sample index is advanced at each sample
+  // boundary instead of divided out per vector (a 64-bit division was most of the kernel's
+  // instructions).
   constexpr int kU = 4;
+  const long long sample_vecs = static_cast<long long>(T) * vec_per_row;
+  int i_cur = v_begin < v_end ? static_cast<int>(v_begin / sample_vecs) : 0;
+  long long next_sample = static_cast<long long>(i_cur + 1) * sample_vecs;  // first vector of sample i_cur + 1
   for (long long v = v_begin; v < v_end; v += kU * v_step) {
     uint4 pk[kU];
 #pragma unroll
@@ -311,8 +317,16 @@ __device__ __forceinline__ void scale_rows_body(const __nv_bfloat16* __restrict_
     for (int u = 0; u < kU; ++u) {
       const long long vu = v + u * v_step;
       if (vu >= v_end) break;
-      const long long row = vu / vec_per_row;
-      const int i = static_cast<int>(row / T);
+      if (vu >= next_sample) {
+        if (vu - next_sample < sample_vecs) {
+          ++i_cur;
+          next_sample += sample_vecs;
+        } else {
+          i_cur = static_cast<int>(vu / sample_vecs);
+          next_sample = static_cast<long long>(i_cur + 1) * sample_vecs;
+        }
+      }
+      const int i = i_cur;
       if (pr.partials != nullptr &&
           !DP_DCHECK(i >= s_lo && (i - s_lo + 1) * sizeof(float) <= dynamic_smem_bytes(), 21u, nullptr))
         break;
@@ -370,7 +384,7 @@ __device__ __forceinline__ void noise_fill_share(const NoiseFill* fills, int cou
   }
 }
 
-__global__ void scale_rows_bf16_kernel(const __nv_bfloat16* __restrict__ in,
+__global__ void __launch_bounds__(256, 4) scale_rows_bf16_kernel(const __nv_bfloat16* __restrict__ in,
                                        __nv_bfloat16* __restrict__ out, long long rows, int cols,
                                        int T, NormSource src, PartialsRef pr, float C, NoiseFill fill,
                                        PhiloxKey key, StepRef step) {
@@ -404,7 +418,7 @@ struct ScaleBatch {
   StepRef step;
 };
 
-__global__ void scale_rows_bf16_batch_kernel(ScaleBatch b) {
+__global__ void __launch_bounds__(256, 4) scale_rows_bf16_batch_kernel(ScaleBatch b) {
   griddep_enter();
   int q = 0;
   while (q + 1 < b.count && static_cast<int>(blockIdx.x) >= b.seg[q + 1].first_block) ++q;
@@ -414,15 +428,6 @@ __global__ void scale_rows_bf16_batch_kernel(ScaleBatch b) {
   if (b.fills > 0) noise_fill_share(b.fill, b.fills, b.key, b.step.get(), blockIdx.x, gridDim.x);
 }
 
-// out[e] = fp32(sum_i c_i Gs[i][e] + std * z_e) over the per-sample bf16 gradients that the
-// explicit-store pass left in the workspace: the clipped sum without forming any G_i again.
-// This is the kernel for B > 8 samples (smaller batches take clip_reduce_tma_kernel below).
-//
-// Each thread owns 8 consecutive elements: two Philox blocks and four independent fp64
-// Box-Muller pairs.  The noise sigma C z is rounded to fp32 once and added to the fp32 sum
-// (one conversion an element instead of two; the result is within 1 ulp of the fp64 sum
-// rounded once).  A persistent grid of two blocks per SM; each block stages the Box-Muller
-// tables in shared memory once.
 // The eight noise values of elements 8 v2 .. 8 v2 + 7 (two Philox blocks), each rounded to
 // fp32 once, scaled by the std.
 template <class Tab>
@@ -435,6 +440,16 @@ __device__ __forceinline__ void noise8_f32(uint32_t blk0, uint32_t layer_id, uin
   for (int q = 0; q < 8; ++q) n[q] = __double2float_rn(z[q]);
 }
 
+// out[e] = fp32(sum_i c_i Gs[i][e] + std * z_e) over the per-sample bf16 gradients that the
+// explicit-store pass left in the workspace: the clipped sum without forming any G_i again.
+// This is the kernel for B > 8 samples (smaller batches take clip_reduce_tma_kernel below).
+//
+// Each thread owns 8 consecutive elements: two Philox blocks and four independent fp64
+// Box-Muller pairs.  The noise sigma C z is rounded to fp32 once and added to the fp32 sum
+// (one conversion an element instead of two; the result is within 1 ulp of the fp64 sum
+// rounded once).  A persistent grid of two blocks per SM; each block stages the Box-Muller
+// tables in shared memory once.
+//
 // STAGED: the Box-Muller tables are staged in shared memory (32 KB); otherwise they are read
 // through the read-only cache and the block needs only the clip factors' few bytes of shared
 // memory, so it fits on an SM beside a running tensor-core CTA (the overlapped block step).

@@ -82,8 +82,10 @@ struct alignas(64) UmmaParams {
   uint32_t* status;
   long long out_elems;        // elements of the output buffer (device-side checks; 0 = unknown)
   long long partials_elems;   // floats of the partials buffer (device-side checks; 0 = unknown)
-  int x_splits;               // ghost kinds: K splits of the X Gram (0 or 1: none).  The norm is
-                              // linear in the X Gram, so each split's partial sums add up.
+  // Ghost kinds: (sample, pair) units [0, split_full_units) whole, each later one in
+  // split_parts parts of the K of the X Gram (split_over_x) or of the dY Grams.  The norm is
+  // linear in each Gram, so the parts' partial sums add up.  split_parts 0 or 1: none.
+  int split_full_units, split_parts, split_over_x;
 };
 
 // Several independent problems of one contraction kind in one launch: the projections
@@ -101,7 +103,9 @@ struct alignas(64) UmmaGroup {
   int m_tiles[kMaxGroup];               // kEpiClipSum
   int k_blocks[kMaxGroup];
   int k_blocks1[kMaxGroup];             // kEpiGhostNorm: K blocks of the dY (or Z) Gram
-  int x_splits[kMaxGroup];              // kEpiGhostNorm: K splits of the X Gram
+  int split_full_units[kMaxGroup];      // kEpiGhostNorm: as in UmmaParams, per problem
+  int split_parts[kMaxGroup];
+  int split_over_x[kMaxGroup];
   float* partials[kMaxGroup];           // kEpiGhostNorm: the problem's norm-partial set
   int unit_begin[kMaxGroup + 1];
   int count;
@@ -141,22 +145,51 @@ struct Unit {
   int m_blk, n_blk, kb_begin, kb_end, sample, split;
   int local;  // index of the unit among the units of its sample (norm partial slots)
   int prob;   // grouped launch: the problem of the unit
-  int kb1;    // ghost kinds: K blocks of the phases after the first (the dY Grams)
+  int kb1;    // ghost kinds: K blocks of the phases after the first (the dY Grams), end
+  int kb1_begin;   // ... and first (a unit split over the dY Grams' K)
+  int zero_slots;  // ghost kinds: partial slot groups after this unit's own to write as zero
 };
 
-// Ghost units of one sample: upper-triangular pairs of 128-token blocks, each in `xs` K splits
-// of its X Gram.  Unit index r within the sample -> (row block, column block, split).
-__device__ __forceinline__ void ghost_pair(int r, int t_tiles, int xs, Unit& w) {
-  const int pair = r / xs;
-  w.split = r % xs;
-  w.local = r;  // = pair * xs + split: its four warps write slots 4 local .. 4 local + 3
-  int c = pair, row = 0;
+// Pair r of one sample's upper-triangular pairs of 128-token blocks -> (row block, column
+// block); local = r.
+__device__ __forceinline__ void ghost_pair(int r, int t_tiles, Unit& w) {
+  w.local = r;
+  int c = r, row = 0;
   while (c >= t_tiles - row) {
     c -= t_tiles - row;
     ++row;
   }
   w.m_blk = row;
   w.n_blk = row + c;
+}
+
+// Ghost unit r of one problem (pairs per sample, X Gram K blocks kx, dY Gram K blocks k1).
+// With parts > 1, the (sample, pair) units from `full` on are each cut in `parts` parts of the
+// K of the X Gram (over_x) or of the dY Grams.  Every pair then owns `parts` groups of four
+// partial slots (one per epilogue warp), and a whole unit writes zeros into the groups it does
+// not use, so that no slot of a sample holds a stale value.
+__device__ __forceinline__ void ghost_unit(int r, int pairs, int t_tiles, int full, int parts, bool over_x,
+                                           int kx, int k1, Unit& w) {
+  const bool split = parts > 1 && r >= full;
+  const int base = split ? full + (r - full) / parts : r;
+  const int part = split ? (r - full) % parts : 0;
+  w.sample = base / pairs;
+  ghost_pair(base % pairs, t_tiles, w);
+  w.local = w.local * (parts > 1 ? parts : 1) + part;  // its warps write slots 4 local .. 4 local + 3
+  w.zero_slots = (parts > 1 && !split) ? parts - 1 : 0;
+  w.kb_begin = 0;
+  w.kb_end = kx;
+  w.kb1_begin = 0;
+  w.kb1 = k1;
+  if (split && over_x) {
+    const int per = (kx + parts - 1) / parts;
+    w.kb_begin = part * per;
+    w.kb_end = min(kx, w.kb_begin + per);
+  } else if (split) {
+    const int per = (k1 + parts - 1) / parts;
+    w.kb1_begin = part * per;
+    w.kb1 = min(k1, w.kb1_begin + per);
+  }
 }
 
 template <class Cfg>
@@ -178,13 +211,8 @@ __device__ __forceinline__ Unit decode_unit(const UmmaParams& p, int u, const Um
       return w;
     }
     if (Cfg::EPI == kEpiGhostNorm) {
-      const int xs = grp->x_splits[q];
-      w.sample = r / (p.pairs_per_sample * xs);
-      ghost_pair(r % (p.pairs_per_sample * xs), p.t_tiles, xs, w);
-      const int kbps = (grp->k_blocks[q] + xs - 1) / xs;
-      w.kb_begin = w.split * kbps;
-      w.kb_end = min(grp->k_blocks[q], w.kb_begin + kbps);
-      w.kb1 = grp->k_blocks1[q];
+      ghost_unit(r, p.pairs_per_sample, p.t_tiles, grp->split_full_units[q], grp->split_parts[q],
+                 grp->split_over_x[q] != 0, grp->k_blocks[q], grp->k_blocks1[q], w);
       return w;
     }
     w.m_blk = r / p.n_tiles;
@@ -194,13 +222,8 @@ __device__ __forceinline__ Unit decode_unit(const UmmaParams& p, int u, const Um
     return w;
   }
   if (Cfg::GHOST) {
-    const int xs = p.x_splits > 1 ? p.x_splits : 1;
-    w.sample = u / (p.pairs_per_sample * xs);
-    ghost_pair(u % (p.pairs_per_sample * xs), p.t_tiles, xs, w);
-    const int kbps = (p.k_blocks + xs - 1) / xs;
-    w.kb_begin = w.split * kbps;
-    w.kb_end = min(p.k_blocks, w.kb_begin + kbps);
-    w.kb1 = p.k_blocks1;
+    ghost_unit(u, p.pairs_per_sample, p.t_tiles, p.split_full_units, p.split_parts, p.split_over_x != 0,
+               p.k_blocks, p.k_blocks1, w);
     return w;
   }
   const int tiles = p.m_tiles * p.n_tiles;
@@ -421,9 +444,11 @@ __device__ __forceinline__ void epilogue_unit(const UmmaParams& p, const Unit& w
     ss = warp_sum(ss);
     const long long slot = static_cast<long long>(w.sample) * p.partial_stride + 4 * w.local + wq;
     float* const partials = Cfg::GROUPED ? grp->partials[w.prob] : p.partials;
-    if (lane == 0 && DP_DCHECK(4 * w.local + wq < p.partial_stride && in_buffer(slot, 1, p.partials_elems), 4u,
-                               p.status))
+    if (lane == 0 && DP_DCHECK(4 * (w.local + w.zero_slots) + wq < p.partial_stride &&
+                                   in_buffer(slot, 1 + 4 * w.zero_slots, p.partials_elems), 4u, p.status)) {
       partials[slot] = ss;
+      for (int z = 1; z <= w.zero_slots; ++z) partials[slot + 4 * z] = 0.f;
+    }
   } else if (Cfg::EPI == kEpiGhostShared) {
     const int t = w.m_blk * Cfg::BM + row;
     float ss[kGhostSharedMaxOps] = {0.f, 0.f, 0.f};
@@ -455,9 +480,11 @@ __device__ __forceinline__ void epilogue_unit(const UmmaParams& p, const Unit& w
         const float v = warp_sum(ss[op]);
         const long long slot = op * p.partial_op_stride + static_cast<long long>(w.sample) * p.partial_stride +
                                4 * w.local + wq;
-        if (lane == 0 && DP_DCHECK(4 * w.local + wq < p.partial_stride && in_buffer(slot, 1, p.partials_elems), 5u,
-                                   p.status))
+        if (lane == 0 && DP_DCHECK(4 * (w.local + w.zero_slots) + wq < p.partial_stride &&
+                                       in_buffer(slot, 1 + 4 * w.zero_slots, p.partials_elems), 5u, p.status)) {
           p.partials[slot] = v;
+          for (int z = 1; z <= w.zero_slots; ++z) p.partials[slot + 4 * z] = 0.f;
+        }
       }
     }
   } else if (Cfg::EPI == kEpiAxpy) {
@@ -574,7 +601,7 @@ __device__ __forceinline__ void umma_body(const UmmaParams& p, const UmmaGroup* 
         const Unit w = decode_unit<Cfg>(p, u, grp);
         for (int ph = 0; ok && ph < nphases; ++ph) {
           const int kb_end = ph ? w.kb1 : w.kb_end;
-          const int kb_begin = ph ? 0 : w.kb_begin;
+          const int kb_begin = ph ? w.kb1_begin : w.kb_begin;
           for (int kb = kb_begin; kb < kb_end; ++kb) {
             if (!mbar_wait_bounded(smem_addr(empty + stage), phase ^ 1u, abort_flag, p.status, 1u)) {
               ok = false;
@@ -618,7 +645,7 @@ __device__ __forceinline__ void umma_body(const UmmaParams& p, const UmmaGroup* 
         for (int ph = 0; ok && ph < nphases; ++ph) {
           const uint32_t d_tmem = tmem_base + buf * Cfg::ACC_COLS + ph * Cfg::BN;
           const int kb_end = ph ? w.kb1 : w.kb_end;
-          const int kb_begin = ph ? 0 : w.kb_begin;
+          const int kb_begin = ph ? w.kb1_begin : w.kb_begin;
           for (int kb = kb_begin; kb < kb_end; ++kb) {
             if (!mbar_wait_bounded(smem_addr(full + stage), phase, abort_flag, p.status, 3u)) {
               ok = false;

@@ -143,9 +143,17 @@ def test_flat_clipping_llama7b_block_full():
 
 
 @pytest.mark.parametrize("mode", ["per_layer", "flat"])
-def test_shared_x_gram_ghost_block(mode):
-    """q/k/v and gate/up read the same X: one X Gram per group, same norms as one linear at a time."""
-    w, data, dev = _block(d=256, ffn=384, B=3, T=384, seed=11)
+@pytest.mark.parametrize("shape", ["plain", "tail_split"])
+def test_shared_x_gram_ghost_block(mode, shape):
+    """q/k/v and gate/up read the same X: one X Gram per group, same norms as one linear at a time.
+
+    tail_split: gate/up (256 -> 1024, B = 5, T = 256) have 15 ghost units, fewer than the SMs, and
+    a dY Gram four times the X Gram's depth, so each unit is split in 4 parts over the dY Grams'
+    K, in the shared launch and in the one-linear launch alike: the norms stay bitwise equal."""
+    if shape == "plain":
+        w, data, dev = _block(d=256, ffn=384, B=3, T=384, seed=11)
+    else:
+        w, data, dev = _block(d=256, ffn=1024, B=5, T=256, seed=13)
     C = 1.0 if mode == "flat" else 1.0 / math.sqrt(7.0)
     _lib.profiling_enable(True)
     _lib.profiling_collect()
