@@ -261,18 +261,31 @@ __device__ __forceinline__ void scale_rows_body(const __nv_bfloat16* __restrict_
   extern __shared__ float scale_c[];  // with pr.partials: c of samples s_lo .. s_hi
   const int vec_per_row = cols / 8;
   const long long total = rows * vec_per_row;
+  const long long sample_vecs = static_cast<long long>(T) * vec_per_row;
+  // Plain: the block strides over all vectors.  With pr.partials: one contiguous range [v0, v1)
+  // per block, which touches few samples.
   long long v_begin = blk * static_cast<long long>(blockDim.x) + threadIdx.x;
   long long v_end = total;
   long long v_step = nblk * blockDim.x;
-  int s_lo = 0;
-  uint4 first = make_uint4(0u, 0u, 0u, 0u);  // fused path: this thread's first vector, loaded early
+  long long v0 = 0, v1 = 0;
   if (pr.partials != nullptr) {
     const long long per = (total + nblk - 1) / nblk;
-    const long long v0 = blk * per < total ? blk * per : total;
-    const long long v1 = v0 + per < total ? v0 + per : total;
-    const long long sample_vecs = static_cast<long long>(T) * vec_per_row;
-    // The load is in flight while one warp per sample sums the partials.
-    if (v0 + threadIdx.x < v1) first = reinterpret_cast<const uint4*>(in)[v0 + threadIdx.x];
+    v0 = blk * per < total ? blk * per : total;
+    v1 = v0 + per < total ? v0 + per : total;
+    v_begin = v0 + threadIdx.x;
+    v_end = v1;
+    v_step = blockDim.x;
+  }
+  // kU vectors per thread and iteration, all kU loads issued before the first is used (one at
+  // a time left the stream latency-bound).  The first iteration's loads are issued before the
+  // clip factors are formed, so they are in flight meanwhile.
+  constexpr int kU = 4;  // 8 measured slower (RoBERTa 0.118 against 0.116 ms a step)
+  uint4 pk[kU];
+#pragma unroll
+  for (int u = 0; u < kU; ++u)
+    if (v_begin + u * v_step < v_end) pk[u] = reinterpret_cast<const uint4*>(in)[v_begin + u * v_step];
+  int s_lo = 0;
+  if (pr.partials != nullptr) {
     if (v0 < v1) {
       const int warp = threadIdx.x / 32, lane = threadIdx.x % 32, warps = blockDim.x / 32;
       s_lo = static_cast<int>(v0 / sample_vecs);
@@ -292,26 +305,17 @@ __device__ __forceinline__ void scale_rows_body(const __nv_bfloat16* __restrict_
       }
     }
     __syncthreads();
-    v_begin = v0 + threadIdx.x;
-    v_end = v1;
-    v_step = blockDim.x;
   }
-  // Four vectors per thread and iteration, all four loads issued before the first is used, so
-  // each thread keeps four 16-byte loads in flight (one at a time left the stream latency-bound).
   // A thread's vectors only move forward, so its sample index is advanced at each sample
   // boundary instead of divided out per vector (a 64-bit division was most of the kernel's
   // instructions).
-  constexpr int kU = 4;
-  const long long sample_vecs = static_cast<long long>(T) * vec_per_row;
   int i_cur = v_begin < v_end ? static_cast<int>(v_begin / sample_vecs) : 0;
   long long next_sample = static_cast<long long>(i_cur + 1) * sample_vecs;  // first vector of sample i_cur + 1
   for (long long v = v_begin; v < v_end; v += kU * v_step) {
-    uint4 pk[kU];
+    if (v != v_begin) {
 #pragma unroll
-    for (int u = 0; u < kU; ++u) {
-      const long long vu = v + u * v_step;
-      if (vu < v_end)
-        pk[u] = (pr.partials != nullptr && vu == v_begin) ? first : reinterpret_cast<const uint4*>(in)[vu];
+      for (int u = 0; u < kU; ++u)
+        if (v + u * v_step < v_end) pk[u] = reinterpret_cast<const uint4*>(in)[v + u * v_step];
     }
 #pragma unroll
     for (int u = 0; u < kU; ++u) {
@@ -356,31 +360,34 @@ struct NoiseFill {
   uint32_t layer_id;
 };
 
-// This block's share (block `blk` of `nblk`) of the Philox blocks of `fills` (count of them).
+// This block's share (block `blk` of `nblk`) of the Philox blocks of `fills` (count of them):
+// global block j of the fills' concatenation goes to thread j mod (nblk * blockDim.x), which
+// walks each fill directly from its first such block.
 __device__ __forceinline__ void noise_fill_share(const NoiseFill* fills, int count, PhiloxKey key, uint32_t step_lo,
                                                  long long blk, long long nblk) {
-  unsigned long long total_blocks = 0;
-  for (int q = 0; q < count; ++q) total_blocks += (fills[q].total + 3) / 4;
-  for (unsigned long long j = blk * static_cast<unsigned long long>(blockDim.x) + threadIdx.x; j < total_blocks;
-       j += static_cast<unsigned long long>(nblk) * blockDim.x) {
-    unsigned long long jj = j;
-    int q = 0;
-    while ((fills[q].total + 3) / 4 <= jj) {  // the fill holding global block j
-      jj -= (fills[q].total + 3) / 4;
-      ++q;
+  const unsigned long long stride = static_cast<unsigned long long>(nblk) * blockDim.x;
+  const unsigned long long j0 = static_cast<unsigned long long>(blk) * blockDim.x + threadIdx.x;
+  unsigned long long seg_begin = 0;  // global index of the fill's first block
+  for (int q = 0; q < count; ++q) {
+    const NoiseFill f = fills[q];
+    const unsigned long long nb = (f.total + 3) / 4;
+    // This thread's first global block at or after seg_begin, as an index into the fill.
+    const unsigned long long first =
+        j0 >= seg_begin ? j0 - seg_begin : (stride - (seg_begin - j0) % stride) % stride;
+    for (unsigned long long jj = first; jj < nb; jj += stride) {
+      double z[4] = {0.0, 0.0, 0.0, 0.0};
+      if (f.std_dev != 0.0)
+        normals4(static_cast<uint32_t>(jj), f.layer_id, step_lo, kStreamNoise, key, z, NoiseTablesGlobal{}, f.std_dev);
+      const unsigned long long k0 = 4 * jj;
+      if (k0 + 3 < f.total) {
+        if (!DP_DCHECK(in_buffer(static_cast<long long>(k0), 4, static_cast<long long>(f.total)), 28u, nullptr)) break;
+        *reinterpret_cast<float4*>(f.G + k0) = make_float4(__double2float_rn(z[0]), __double2float_rn(z[1]),
+                                                           __double2float_rn(z[2]), __double2float_rn(z[3]));
+      } else {
+        for (int e = 0; e < 4 && k0 + e < f.total; ++e) f.G[k0 + e] = __double2float_rn(z[e]);
+      }
     }
-    const NoiseFill& f = fills[q];
-    double z[4] = {0.0, 0.0, 0.0, 0.0};
-    if (f.std_dev != 0.0)
-      normals4(static_cast<uint32_t>(jj), f.layer_id, step_lo, kStreamNoise, key, z, NoiseTablesGlobal{}, f.std_dev);
-    const unsigned long long k0 = 4 * jj;
-    if (k0 + 3 < f.total) {
-      if (!DP_DCHECK(in_buffer(static_cast<long long>(k0), 4, static_cast<long long>(f.total)), 28u, nullptr)) continue;
-      *reinterpret_cast<float4*>(f.G + k0) = make_float4(__double2float_rn(z[0]), __double2float_rn(z[1]),
-                                                         __double2float_rn(z[2]), __double2float_rn(z[3]));
-    } else {
-      for (int e = 0; e < 4 && k0 + e < f.total; ++e) f.G[k0 + e] = __double2float_rn(z[e]);
-    }
+    seg_begin += nb;
   }
 }
 
