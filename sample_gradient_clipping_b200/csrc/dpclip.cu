@@ -106,6 +106,8 @@ bool valid_shape(const Shape& s) {
 
 struct WsLayout {
   size_t status = 0, norm2 = 0, c = 0, partials = 0, scaled = 0, z = 0, p = 0, gs = 0, total = 0;
+  size_t fixup = 0;     // a clipped sum split over K: its split partials (0: none)
+  int fixup_splits = 0;  // splits that region holds
   int partial_stride = 0;  // floats per sample
 };
 
@@ -155,9 +157,49 @@ GhostSplit ghost_split(const Shape& s) {
 // Units of a ghost launch for one linear under its split, and its partial slots per sample.
 int ghost_units(const GhostSplit& g, int units) { return g.parts > 1 ? g.full + (units - g.full) * g.parts : units; }
 
+struct ClipSumPlan {
+  bool pair;
+  int bn, m_tiles, n_tiles, k_blocks, k_blocks_per_split, splits;
+};
+
+ClipSumPlan clipsum_plan(const Shape& s) {
+  ClipSumPlan c;
+  const int ne = s.ne();
+  c.bn = ne <= 128 ? 128 : 256;
+  // 256 x 256 tiles on SM pairs when both output dimensions fill them: half the operand
+  // traffic per SM of a 128 x 256 one-SM tile.
+  c.pair = (s.m >= 256 && ne >= 256);
+  c.m_tiles = c.pair ? ceil_div(s.m, 256) : ceil_div(s.m, 128);
+  c.n_tiles = ceil_div(ne, c.bn);
+  c.k_blocks = ceil_div(s.N(), 64);
+  const int tiles = c.m_tiles * c.n_tiles;
+  const int slots = c.pair ? sm_count() / 2 : sm_count();  // CTAs (or pairs) that run at once
+  int splits = 1;
+  if (tiles < slots) {
+    splits = slots / tiles;
+    const int max_splits = c.k_blocks / 4 > 0 ? c.k_blocks / 4 : 1;
+    if (splits > max_splits) splits = max_splits;
+    if (splits < 1) splits = 1;
+  }
+  c.k_blocks_per_split = ceil_div(c.k_blocks, splits);
+  c.splits = ceil_div(c.k_blocks, c.k_blocks_per_split);  // every split non-empty
+  return c;
+}
+
+// Where a clipped sum split over K keeps its split partials (kOutSplitPartials).
+struct FixupRef {
+  float* scratch;  // [splits][m][ne] fp32
+  int max_splits;  // splits the scratch holds
+};
+
 WsLayout ws_layout(const Shape& s, dp_norm_method method) {
   WsLayout L;
   size_t off = 256;  // status word(s)
+  // A bf16 clipped sum split over K keeps its split partials at the end.  Every method's
+  // layout holds them, so that the gradients-once layout stays the largest
+  // (dp_clip_accumulate runs the clipped sum whatever method sized the workspace).
+  const ClipSumPlan cp = clipsum_plan(s);
+  const bool fix = s.dt == DP_BF16 && cp.splits > 1;
   L.norm2 = off;
   off += align256(static_cast<size_t>(s.B) * 8);
   L.c = off;
@@ -181,6 +223,11 @@ WsLayout ws_layout(const Shape& s, dp_norm_method method) {
   if (method == DP_NORM_ONCE && s.dt == DP_BF16) {
     L.gs = off;  // per-sample gradient tiles, bf16 [B][d_in][ne]
     off += align256(static_cast<size_t>(s.B) * s.m * s.ne() * 2);
+  }
+  if (fix) {
+    L.fixup = off;
+    L.fixup_splits = cp.splits;
+    off += align256(static_cast<size_t>(cp.splits) * s.m * s.ne() * 4);
   }
   L.total = off;
   return L;
@@ -455,44 +502,28 @@ dp_status launch_noise(float* G, unsigned long long total, double std_dev, unsig
 
 // How the clipped-sum contraction of shape s is tiled: SM-pair tiles or not, and into how many
 // K splits (a split-K sum lands by fp32 atomics).
-struct ClipSumPlan {
-  bool pair;
-  int bn, m_tiles, n_tiles, k_blocks, k_blocks_per_split, splits;
-};
-
-ClipSumPlan clipsum_plan(const Shape& s) {
-  ClipSumPlan c;
-  const int ne = s.ne();
-  c.bn = ne <= 128 ? 128 : 256;
-  // 256 x 256 tiles on SM pairs when both output dimensions fill them: half the operand
-  // traffic per SM of a 128 x 256 one-SM tile.
-  c.pair = (s.m >= 256 && ne >= 256);
-  c.m_tiles = c.pair ? ceil_div(s.m, 256) : ceil_div(s.m, 128);
-  c.n_tiles = ceil_div(ne, c.bn);
-  c.k_blocks = ceil_div(s.N(), 64);
-  const int tiles = c.m_tiles * c.n_tiles;
-  const int slots = c.pair ? sm_count() / 2 : sm_count();  // CTAs (or pairs) that run at once
-  int splits = 1;
-  if (tiles < slots) {
-    splits = slots / tiles;
-    const int max_splits = c.k_blocks / 4 > 0 ? c.k_blocks / 4 : 1;
-    if (splits > max_splits) splits = max_splits;
-    if (splits < 1) splits = 1;
-  }
-  c.k_blocks_per_split = ceil_div(c.k_blocks, splits);
-  c.splits = ceil_div(c.k_blocks, c.k_blocks_per_split);  // every split non-empty
-  return c;
+// The combining launch of clipped sums split over K (combine_splits_kernel).
+dp_status launch_combine(const CombineBatch& b, cudaStream_t stream) {
+  if (b.count == 0) return DP_OK;
+  unsigned long long vecs = 0;
+  for (int q = 0; q < b.count; ++q) vecs += b.seg[q].elems / 4;
+  LaunchScope scope(kKindCombine, stream);
+  DP_LAUNCH("combine_splits_kernel", combine_splits_kernel, stream_grid(vecs, 256), 256, 0, stream, b);
+  return DP_OK;
 }
 
 // out (+)= A^T Bm over all N rows (A: [N, m], Bm: [N, ne], both bf16, one already scaled by
 // c_i), plus noise when noise_std != 0.  `accumulate` = 0 overwrites out.
 // With `defer` (a block step), noise that cannot ride in the epilogue (split K) is queued
 // there instead of launched.  With `preset` (split K only), out already holds the noise
-// (written by a noise launch in SET mode) and the partial sums are added to it.
+// (written by the row-scaling launch) and the sum is added to it.
+// Split over K with `fx`: each split stores its partial sum, and a combining launch adds them
+// in split order to out's contents in fp64 and rounds once (kOutSplitPartials).  Without it,
+// the splits add their partial sums into out by fp32 atomics.
 dp_status bf16_clipsum(const Shape& s, const void* A, const void* Bm, float* out, int accumulate,
                        double noise_std, unsigned long long seed, StepRef step,
                        unsigned layer_id, uint32_t* status, cudaStream_t stream,
-                       NoiseBatch* defer = nullptr, bool preset = false) {
+                       NoiseBatch* defer = nullptr, bool preset = false, const FixupRef* fx = nullptr) {
   UmmaParams p = base_params(status);
   const int ne = s.ne();
   const ClipSumPlan plan = clipsum_plan(s);
@@ -514,7 +545,11 @@ dp_status bf16_clipsum(const Shape& s, const void* A, const void* Bm, float* out
   p.out_f32 = out;
   p.out_elems = static_cast<long long>(s.m) * ne;
   if (preset && (splits == 1 || accumulate)) return DP_ERR_INVALID_ARG;  // the callers never ask this
-  if (splits > 1 || accumulate) {
+  const bool split_partials = splits > 1 && fx && fx->scratch && splits <= fx->max_splits;
+  if (split_partials) {
+    p.out_mode = kOutSplitPartials;
+    p.split_scratch = fx->scratch;
+  } else if (splits > 1 || accumulate) {
     p.out_mode = (splits > 1) ? kOutAtomicAdd : kOutAdd;
     if (!accumulate && !preset)
       DP_CUDA(cudaMemsetAsync(out, 0, static_cast<size_t>(s.m) * ne * sizeof(float), stream));
@@ -535,6 +570,14 @@ dp_status bf16_clipsum(const Shape& s, const void* A, const void* Bm, float* out
   dp_status st2 = pair        ? launch_umma_pair<Umma2Config<kEpiClipSum>>(p, stream)
                   : (BN == 128) ? launch_umma<UmmaConfig<128, kEpiClipSum>>(p, stream)
                                 : launch_umma<UmmaConfig<256, kEpiClipSum>>(p, stream);
+  if (st2 == DP_OK && split_partials) {
+    CombineBatch cb;
+    memset(&cb, 0, sizeof(cb));
+    cb.count = 1;
+    cb.seg[0] = CombineSegment{out, fx->scratch, static_cast<unsigned long long>(s.m) * ne, splits,
+                               (accumulate || preset) ? 1 : 0};
+    st2 = launch_combine(cb, stream);
+  }
   if (st2 != DP_OK || fused_noise || noise_std == 0.0) return st2;
   if (defer && defer->count < kMaxNoiseSegments) {
     defer->seg[defer->count++] = NoiseSegment{out, static_cast<unsigned long long>(s.m) * ne, noise_std,
@@ -899,16 +942,18 @@ dp_status clipped_sum(Call& c, const void* X, const void* Z, NormSource src, flo
   dp_status st;
   const NoiseFill fill{out, static_cast<unsigned long long>(s.m) * s.ne(), noise_std, layer_id};
   const NoiseFill* nf = prefill_noise ? &fill : nullptr;
+  // The layout's split-sum regions, when it has them (a shape whose clipped sum splits over K).
+  const FixupRef fx{c.L.fixup ? reinterpret_cast<float*>(c.ws + c.L.fixup) : nullptr, c.L.fixup_splits};
   if (s.ne() <= s.m) {
     if ((st = launch_scale(Z, scaled, s.N(), s.ne(), s.T, src, C, c.stream, partials, s.B, nf, seed, step)) != DP_OK)
       return st;
     return bf16_clipsum(s, X, scaled, out, accumulate, noise_std, seed, step, layer_id, c.status(), c.stream,
-                        defer, prefill_noise);
+                        defer, prefill_noise, &fx);
   }
   if ((st = launch_scale(X, scaled, s.N(), s.m, s.T, src, C, c.stream, partials, s.B, nf, seed, step)) != DP_OK)
     return st;
   return bf16_clipsum(s, scaled, Z, out, accumulate, noise_std, seed, step, layer_id, c.status(), c.stream,
-                      defer, prefill_noise);
+                      defer, prefill_noise, &fx);
 }
 
 dp_status resolve_method(const Shape& s, dp_norm_method method, dp_norm_method* out) {
@@ -955,6 +1000,9 @@ struct BlockLayout {
   std::vector<size_t> scaled_l;          // per layer: its scaled copy (batched schedule), or 0
   std::vector<long long> partial_set;    // per layer: its norm-partial set (batched schedule)
   bool z_grouped = false;                // bf16 projected layers: every Z formed in grouped launches
+  // Clipped sums split over K: per layer its split partials (0: none).
+  std::vector<size_t> fixup;
+  std::vector<int> fixup_splits;         // per layer: splits its partials region holds
 };
 
 constexpr size_t kBatchScaleBytes = size_t(256) << 20;
@@ -1065,6 +1113,37 @@ std::vector<std::vector<int>> block_groups(const dp_layer* layers, int L, dp_dty
   return groups;
 }
 
+// Whether the clipped sums of the layers in `ls` can run as grouped launches: every one on the
+// one-SM engine with the same tile width (no SM-pair tiles), up to kMaxGroup a launch.
+bool clipsums_groupable(const dp_layer* layers, const std::vector<int>& ls, int B, int T, dp_dtype dt) {
+  if (ls.size() < 2) return false;
+  int bn = 0;
+  for (int l : ls) {
+    const ClipSumPlan c = clipsum_plan(layer_shape(layers[l], B, T, dt));
+    if (c.pair || (bn && c.bn != bn)) return false;
+    bn = c.bn;
+  }
+  return true;
+}
+
+// The K split of each grouped launch of clipped sums over the layers `ls` (chunks of up to
+// kMaxGroup in order), per layer of `ls`: one split for a whole launch, chosen so that its
+// units fill the GPU about once.  The layout sizes each layer's split partials with it.
+std::vector<int> group_sum_splits(const dp_layer* layers, const std::vector<int>& ls, int B, int T, dp_dtype dt) {
+  std::vector<int> out;
+  for (size_t c0 = 0; c0 < ls.size(); c0 += kMaxGroup) {
+    const int count = static_cast<int>(std::min<size_t>(kMaxGroup, ls.size() - c0));
+    const ClipSumPlan plan0 = clipsum_plan(layer_shape(layers[ls[c0]], B, T, dt));
+    int tiles = 0;
+    for (int q = 0; q < count; ++q) tiles += ceil_div(layers[ls[c0 + q]].d_in, 128) * plan0.n_tiles;
+    int splits = std::max(1, sm_count() / std::max(1, tiles));
+    splits = std::min(splits, std::max(1, plan0.k_blocks / 4));
+    splits = ceil_div(plan0.k_blocks, ceil_div(plan0.k_blocks, splits));  // every split non-empty
+    for (int q = 0; q < count; ++q) out.push_back(splits);
+  }
+  return out;
+}
+
 BlockLayout block_layout(const dp_layer* layers, int L, int B, int T, dp_dtype dt, dp_clip_mode mode,
                          const std::vector<dp_norm_method>& methods) {
   BlockLayout Lb;
@@ -1173,6 +1252,31 @@ BlockLayout block_layout(const dp_layer* layers, int L, int B, int T, dp_dtype d
     if (layers[l].P) {
       Lb.z[l] = off;
       off += align256(static_cast<size_t>(B) * T * layers[l].r * (dt == DP_BF16 ? 2 : 4));
+    }
+  }
+  // Split partials of each bf16 ghost or explicit layer whose clipped sum splits over K: with
+  // the split of its grouped launch (batched schedule, groupable sums), else its own.
+  Lb.fixup.assign(L, 0);
+  Lb.fixup_splits.assign(L, 0);
+  if (dt == DP_BF16) {
+    std::vector<int> splits(L, 1);
+    for (int l = 0; l < L; ++l)
+      if (methods[l] != DP_NORM_ONCE) splits[l] = clipsum_plan(layer_shape(layers[l], B, T, dt)).splits;
+    if (Lb.batched_scale) {
+      std::vector<int> batch_all;
+      for (const auto& g : Lb.groups)
+        if (methods[g[0]] != DP_NORM_ONCE) batch_all.insert(batch_all.end(), g.begin(), g.end());
+      if (clipsums_groupable(layers, batch_all, B, T, dt)) {
+        const std::vector<int> gs = group_sum_splits(layers, batch_all, B, T, dt);
+        for (size_t i = 0; i < batch_all.size(); ++i) splits[batch_all[i]] = gs[i];
+      }
+    }
+    for (int l = 0; l < L; ++l) {
+      if (splits[l] < 2) continue;
+      const Shape s = layer_shape(layers[l], B, T, dt);
+      Lb.fixup[l] = off;
+      Lb.fixup_splits[l] = splits[l];
+      off += align256(static_cast<size_t>(splits[l]) * s.m * s.ne() * 4);
     }
   }
   Lb.total = off;
@@ -1361,6 +1465,8 @@ dp_status block_layer_sum(const dp_layer* layers, int l, dp_dtype dt, int B, int
   c.s = s;
   c.L = WsLayout();
   c.L.scaled = Lb.scaled;
+  c.L.fixup = Lb.fixup[l];
+  c.L.fixup_splits = Lb.fixup_splits[l];
   c.ws = ws;
   c.stream = stream;
   const void* Z;
@@ -1381,23 +1487,11 @@ NormSource layer_norm_source(const BlockLayout& Lb, uint8_t* ws, int l, int B, d
   return src;
 }
 
-// Whether the clipped sums of the layers in `ls` can run as grouped launches: every one on the
-// one-SM engine with the same tile width (no SM-pair tiles), up to kMaxGroup a launch.
-bool clipsums_groupable(const dp_layer* layers, const std::vector<int>& ls, int B, int T, dp_dtype dt) {
-  if (ls.size() < 2) return false;
-  int bn = 0;
-  for (int l : ls) {
-    const ClipSumPlan c = clipsum_plan(layer_shape(layers[l], B, T, dt));
-    if (c.pair || (bn && c.bn != bn)) return false;
-    bn = c.bn;
-  }
-  return true;
-}
-
 // The clipped sums of the layers in `ls` (batched schedule, groupable) in grouped launches of
-// up to kMaxGroup problems.  One K split for the whole launch, chosen so that its units fill the
-// GPU about once; every output already holds its noise (or zeros) and the partial sums are
-// added to it by atomics.
+// up to kMaxGroup problems.  One K split for the whole launch (group_sum_splits), chosen so
+// that its units fill the GPU about once; every output already holds its noise (or zeros).
+// The splits store their partial sums and one combining launch adds them to the outputs in
+// split order (kOutSplitPartials); without the layout's split partials they add by atomics.
 dp_status launch_clipsum_groups(const dp_layer* layers, const std::vector<int>& ls, dp_dtype dt, int B, int T,
                                 const BlockLayout& Lb, uint8_t* ws, cudaStream_t stream) {
   dp_status st;
@@ -1408,17 +1502,17 @@ dp_status launch_clipsum_groups(const dp_layer* layers, const std::vector<int>& 
     memset(&g, 0, sizeof(g));
     g.count = count;
     const ClipSumPlan plan0 = clipsum_plan(layer_shape(layers[ls[c0]], B, T, dt));
-    int tiles = 0;
+    bool fix = true;
     for (int q = 0; q < count; ++q) {
       const Shape s = layer_shape(layers[ls[c0 + q]], B, T, dt);
       g.m_tiles[q] = ceil_div(s.m, 128);
-      tiles += g.m_tiles[q] * plan0.n_tiles;
+      fix = fix && Lb.fixup[ls[c0 + q]] != 0;
     }
     const int k_blocks = plan0.k_blocks;
-    int splits = std::max(1, sm_count() / std::max(1, tiles));
-    splits = std::min(splits, std::max(1, k_blocks / 4));
+    int splits = group_sum_splits(layers, std::vector<int>(ls.begin() + c0, ls.begin() + c0 + count), B, T, dt)[0];
     g.k_blocks_per_split = ceil_div(k_blocks, splits);
     splits = ceil_div(k_blocks, g.k_blocks_per_split);
+    for (int q = 0; q < count; ++q) fix = fix && splits <= Lb.fixup_splits[ls[c0 + q]];
     int units = 0;
     for (int q = 0; q < count; ++q) {
       const int l = ls[c0 + q];
@@ -1432,6 +1526,7 @@ dp_status launch_clipsum_groups(const dp_layer* layers, const std::vector<int>& 
       if ((st = map_2d(&g.tmA[q], A, s.N(), s.m, 64)) != DP_OK) return st;
       if ((st = map_2d(&g.tmB[q], Bm, s.N(), s.ne(), 64)) != DP_OK) return st;
       g.out_f32[q] = y.G_out;
+      g.split_scratch[q] = fix ? reinterpret_cast<float*>(ws + Lb.fixup[l]) : nullptr;
       g.out_rows[q] = s.m;
       g.k_blocks[q] = k_blocks;
       g.unit_begin[q] = units;
@@ -1443,11 +1538,22 @@ dp_status launch_clipsum_groups(const dp_layer* layers, const std::vector<int>& 
     p.k_blocks = k_blocks;
     p.k_splits = splits;
     p.out_cols = layer_shape(layers[ls[c0]], B, T, dt).ne();
-    p.out_mode = kOutAtomicAdd;
+    p.out_mode = fix ? kOutSplitPartials : kOutAtomicAdd;
     p.noise_std = 0.0;  // written into the outputs beforehand
     if (plan0.bn == 128) st = launch_umma_group<UmmaConfig<128, kEpiClipSum, true>>(p, g, stream);
     else st = launch_umma_group<UmmaConfig<256, kEpiClipSum, true>>(p, g, stream);
     if (st != DP_OK) return st;
+    if (fix) {
+      CombineBatch cb;
+      memset(&cb, 0, sizeof(cb));
+      cb.count = count;
+      for (int q = 0; q < count; ++q) {
+        const Shape s = layer_shape(layers[ls[c0 + q]], B, T, dt);
+        cb.seg[q] = CombineSegment{g.out_f32[q], g.split_scratch[q], static_cast<unsigned long long>(s.m) * s.ne(),
+                                   splits, 1};
+      }
+      if ((st = launch_combine(cb, stream)) != DP_OK) return st;
+    }
   }
   return DP_OK;
 }
@@ -1655,9 +1761,10 @@ dp_status block_step(const dp_layer* layers, int L, dp_dtype dt, int B, int T, d
         if ((st = block_operand(layers, l, dt, B, T, Lb, ws, stream, false, &Z)) != DP_OK) return st;
         const void* scaled = ws + Lb.scaled_l[l];
         const double noise_std = (sigma == 0.0f) ? 0.0 : static_cast<double>(sigma) * static_cast<double>(y.C);
+        const FixupRef fx{Lb.fixup[l] ? reinterpret_cast<float*>(ws + Lb.fixup[l]) : nullptr, Lb.fixup_splits[l]};
         if ((st = bf16_clipsum(s, s.ne() <= s.m ? y.X : scaled, s.ne() <= s.m ? scaled : Z, y.G_out, 0, noise_std,
                                seed, step, y.layer_id, reinterpret_cast<uint32_t*>(ws), stream, &deferred,
-                               preset[l])) != DP_OK)
+                               preset[l], &fx)) != DP_OK)
           return st;
       }
     }

@@ -31,6 +31,7 @@ enum KernelKind : int {
   kKindAdam,          // projected Adam moments and update in r-space
   kKindAxpy,          // tcgen05 W += alpha U P^T
   kKindGhostShared,   // tcgen05 one X Gram shared by the dY Grams of up to three linears
+  kKindCombine,       // the split partials of clipped sums split over K, added in split order
   kNumKinds
 };
 
@@ -39,7 +40,7 @@ inline const char* kernel_kind_name(int k) {
       "noise_add",  "projection",   "philox_blocks", "scale_rows_bf16", "finalize_norms",
       "f32_norm",   "f32_clipsum",  "f32_project",   "umma_clipsum",    "umma_explicit_norm",
       "umma_ghost_norm", "umma_project", "umma_explicit_store", "clip_reduce", "adam_rspace",
-      "umma_axpy", "umma_ghost_shared"};
+      "umma_axpy", "umma_ghost_shared", "split_combine"};
   return (k >= 0 && k < kNumKinds) ? names[k] : "";
 }
 

@@ -447,6 +447,54 @@ __device__ __forceinline__ void noise8_f32(uint32_t blk0, uint32_t layer_id, uin
   for (int q = 0; q < 8; ++q) n[q] = __double2float_rn(z[q]);
 }
 
+// The last step of clipped sums split over K: out[e] = fp32(o + sum_k scratch[k][e]), the
+// split partials added in split order in fp64 and rounded once, where o is what out holds
+// (the noise written by the row-scaling launch, zeros, or the caller's accumulator) when
+// read_out, else 0.  The result is the same whatever order the split units ran in, and the
+// noise is added to the finished sum as in an unsplit epilogue.  Segments are walked as in
+// noise_fill_share: global vector j of their concatenation goes to thread j mod (grid size).
+constexpr int kMaxCombineSegments = 8;
+struct CombineSegment {
+  float* out;
+  const float* scratch;     // [splits][elems]
+  unsigned long long elems;  // a multiple of 4
+  int splits;
+  int read_out;
+};
+struct CombineBatch {
+  CombineSegment seg[kMaxCombineSegments];
+  int count;
+};
+
+__global__ void __launch_bounds__(256) combine_splits_kernel(CombineBatch b) {
+  griddep_enter();
+  const unsigned long long stride = static_cast<unsigned long long>(gridDim.x) * blockDim.x;
+  const unsigned long long j0 = static_cast<unsigned long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  unsigned long long seg_begin = 0;
+  for (int q = 0; q < b.count; ++q) {
+    const CombineSegment sg = b.seg[q];
+    const unsigned long long nv = sg.elems / 4;
+    const unsigned long long first =
+        j0 >= seg_begin ? j0 - seg_begin : (stride - (seg_begin - j0) % stride) % stride;
+    for (unsigned long long v = first; v < nv; v += stride) {
+      if (!DP_DCHECK(in_buffer(static_cast<long long>(4 * v), 4, static_cast<long long>(sg.elems)), 32u, nullptr))
+        break;
+      double a[4] = {0.0, 0.0, 0.0, 0.0};
+      if (sg.read_out) {
+        const float4 o = __ldcs(reinterpret_cast<const float4*>(sg.out) + v);
+        a[0] = o.x; a[1] = o.y; a[2] = o.z; a[3] = o.w;
+      }
+      for (int k = 0; k < sg.splits; ++k) {
+        const float4 pk = __ldcs(reinterpret_cast<const float4*>(sg.scratch + k * sg.elems) + v);
+        a[0] += pk.x; a[1] += pk.y; a[2] += pk.z; a[3] += pk.w;
+      }
+      reinterpret_cast<float4*>(sg.out)[v] = make_float4(static_cast<float>(a[0]), static_cast<float>(a[1]),
+                                                        static_cast<float>(a[2]), static_cast<float>(a[3]));
+    }
+    seg_begin += nv;
+  }
+}
+
 // out[e] = fp32(sum_i c_i Gs[i][e] + std * z_e) over the per-sample bf16 gradients that the
 // explicit-store pass left in the workspace: the clipped sum without forming any G_i again.
 // This is the kernel for B > 8 samples (smaller batches take clip_reduce_tma_kernel below).

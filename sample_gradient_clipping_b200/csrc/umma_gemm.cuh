@@ -56,7 +56,10 @@ constexpr int kGhostSharedMaxOps = 3;  // dY operands per shared X Gram (TMEM: 4
 // K-blocks ahead of the smem ring that the clipped-sum producer asks TMA to pull into L2.
 constexpr int kL2PrefetchDistance = 8;
 
-enum OutMode : int { kOutStore = 0, kOutAtomicAdd = 1, kOutAdd = 2 };
+// kOutSplitPartials (a sum split over K): each unit stores its partial sum into its split's
+// slot of a scratch array [k_splits][out_rows][out_cols]; a combining launch then adds the
+// slots in split order, so the result does not depend on the order in which units finish.
+enum OutMode : int { kOutStore = 0, kOutAtomicAdd = 1, kOutAdd = 2, kOutSplitPartials = 3 };
 
 struct alignas(64) UmmaParams {
   CUtensorMap tmA0, tmB0, tmA1, tmB1;  // phase-1 maps are used by the ghost norm only
@@ -86,6 +89,7 @@ struct alignas(64) UmmaParams {
   // split_parts parts of the K of the X Gram (split_over_x) or of the dY Grams.  The norm is
   // linear in each Gram, so the parts' partial sums add up.  split_parts 0 or 1: none.
   int split_full_units, split_parts, split_over_x;
+  float* split_scratch;  // kOutSplitPartials: [k_splits][out_rows][out_cols] fp32
 };
 
 // Several independent problems of one contraction kind in one launch: the projections
@@ -110,6 +114,7 @@ struct alignas(64) UmmaGroup {
   int unit_begin[kMaxGroup + 1];
   int count;
   int k_blocks_per_split;               // kEpiClipSum: the group's K split
+  float* split_scratch[kMaxGroup];      // kEpiClipSum, kOutSplitPartials: the problem's partials
 };
 
 template <int BN_, int EPI_, bool GROUPED_ = false>
@@ -353,6 +358,9 @@ __device__ __forceinline__ void epilogue_unit(const UmmaParams& p, const Unit& w
     const bool noisy = (p.noise_std != 0.0) && (w.split == 0);
     const PhiloxKey key{p.key0, p.key1};
     const uint32_t step_lo = StepRef{p.step_lo, p.step_dev}.get();
+    const bool partial = (p.out_mode == kOutSplitPartials);
+    float* const scratch = Cfg::GROUPED ? grp->split_scratch[w.prob] : p.split_scratch;
+    const long long split_stride = static_cast<long long>(out_rows) * p.out_cols;
 #pragma unroll 1
     for (int c0 = 0; c0 < Cfg::BN; c0 += 32) {
       float v[32];
@@ -377,7 +385,10 @@ __device__ __forceinline__ void epilogue_unit(const UmmaParams& p, const Unit& w
         }
         if (!DP_DCHECK(in_buffer(grow * p.out_cols + gcol0 + 4 * q, 4, out_elems), 1u, p.status)) break;
         float4* d4 = reinterpret_cast<float4*>(dst + 4 * q);
-        if (p.out_mode == kOutStore) {
+        if (partial) {
+          if (!DP_DCHECK(w.split >= 0 && w.split < p.k_splits, 30u, p.status)) break;
+          *reinterpret_cast<float4*>(scratch + w.split * split_stride + grow * p.out_cols + gcol0 + 4 * q) = val;
+        } else if (p.out_mode == kOutStore) {
           *d4 = val;
         } else if (p.out_mode == kOutAtomicAdd) {
           atomicAdd(d4, val);
