@@ -172,8 +172,11 @@ ClipSumPlan clipsum_plan(const Shape& s) {
   c.m_tiles = c.pair ? ceil_div(s.m, 256) : ceil_div(s.m, 128);
   c.n_tiles = ceil_div(ne, c.bn);
   c.k_blocks = ceil_div(s.N(), 64);
-  const int tiles = c.m_tiles * c.n_tiles;
+  // Measured and left out for GPT-2's 768x3072 output (58 us with 256x256 pair tiles split in
+  // two): unsplit 256x128 pair tiles (72 on 74 pairs) 96 us, unsplit one-SM 128x128 tiles (144
+  // on 148 SMs) 99 us.  Both read 1.5-2x the operand bytes per flop from L2.
   const int slots = c.pair ? sm_count() / 2 : sm_count();  // CTAs (or pairs) that run at once
+  const int tiles = c.m_tiles * c.n_tiles;
   int splits = 1;
   if (tiles < slots) {
     splits = slots / tiles;
@@ -184,6 +187,17 @@ ClipSumPlan clipsum_plan(const Shape& s) {
   c.k_blocks_per_split = ceil_div(c.k_blocks, splits);
   c.splits = ceil_div(c.k_blocks, c.k_blocks_per_split);  // every split non-empty
   return c;
+}
+
+// Whether a clipped sum takes its noise from the row-scaling launch before it (which writes
+// the noise into the output, each value rounded to fp32 once) instead of from its epilogue:
+// when it is split over K (the noise must go on the finished sum), or when all its units run
+// in one wave, where the epilogue's fp64 noise would run after every tile with nothing to
+// hide it (measured on unsplit 256x128 tiles of GPT-2's output: 100 against 96 us).  The sum
+// is then added to the noise.
+bool sum_prefills_noise(const ClipSumPlan& c) {
+  const int slots = c.pair ? sm_count() / 2 : sm_count();
+  return c.splits > 1 || c.m_tiles * c.n_tiles <= slots;
 }
 
 // Where a clipped sum split over K keeps its split partials (kOutSplitPartials).
@@ -508,7 +522,7 @@ dp_status launch_combine(const CombineBatch& b, cudaStream_t stream) {
   unsigned long long vecs = 0;
   for (int q = 0; q < b.count; ++q) vecs += b.seg[q].elems / 4;
   LaunchScope scope(kKindCombine, stream);
-  DP_LAUNCH("combine_splits_kernel", combine_splits_kernel, stream_grid(vecs, 256), 256, 0, stream, b);
+  DP_LAUNCH("combine_splits_kernel", combine_splits_kernel, stream_grid((vecs + 1) / 2, 256), 256, 0, stream, b);
   return DP_OK;
 }
 
@@ -544,23 +558,23 @@ dp_status bf16_clipsum(const Shape& s, const void* A, const void* Bm, float* out
   p.out_cols = ne;
   p.out_f32 = out;
   p.out_elems = static_cast<long long>(s.m) * ne;
-  if (preset && (splits == 1 || accumulate)) return DP_ERR_INVALID_ARG;  // the callers never ask this
+  if (preset && accumulate) return DP_ERR_INVALID_ARG;  // the callers never ask this
   const bool split_partials = splits > 1 && fx && fx->scratch && splits <= fx->max_splits;
   if (split_partials) {
     p.out_mode = kOutSplitPartials;
     p.split_scratch = fx->scratch;
-  } else if (splits > 1 || accumulate) {
+  } else if (splits > 1 || accumulate || preset) {
     p.out_mode = (splits > 1) ? kOutAtomicAdd : kOutAdd;
     if (!accumulate && !preset)
       DP_CUDA(cudaMemsetAsync(out, 0, static_cast<size_t>(s.m) * ne * sizeof(float), stream));
   } else {
     p.out_mode = kOutStore;
   }
-  // With split K the partial sums land by atomics; the noise is then added after the sum is
-  // complete (rounded once, as in the unsplit epilogue), or was written first (preset).
+  // With `preset` the noise is already in out.  Otherwise an unsplit sum adds it in its
+  // epilogue (fp64, rounded once), and a split one after the sum is complete.
+  if (preset) noise_std = 0.0;
   const bool fused_noise = (splits == 1);
   p.noise_std = fused_noise ? noise_std : 0.0;
-  if (preset) noise_std = 0.0;  // already in out
   const PhiloxKey key = philox_key_from_seed(seed);
   p.key0 = key.k0;
   p.key1 = key.k1;
@@ -1473,7 +1487,7 @@ dp_status block_layer_sum(const dp_layer* layers, int l, dp_dtype dt, int B, int
   dp_status st = block_operand(layers, l, dt, B, T, Lb, ws, stream, false, &Z);  // formed by the norms
   if (st != DP_OK) return st;
   // A bf16 sum split over K: its row-scaling launch writes the noise first (as in one linear).
-  const bool prefill = (dt == DP_BF16 && noise_std != 0.0 && clipsum_plan(s).splits > 1);
+  const bool prefill = (dt == DP_BF16 && noise_std != 0.0 && sum_prefills_noise(clipsum_plan(s)));
   return clipped_sum(c, y.X, Z, src, C, y.G_out, 0, noise_std, seed, step, y.layer_id, defer, partials,
                      prefill);
 }
@@ -1660,7 +1674,7 @@ dp_status block_step(const dp_layer* layers, int L, dp_dtype dt, int B, int T, d
     if (Lb.batched_scale && (sigma != 0.0f || grouped_sums)) {
       for (int l : batch_all) {
         const Shape s = layer_shape(layers[l], B, T, dt);
-        if ((grouped_sums || clipsum_plan(s).splits > 1) && static_cast<int>(fills.size()) < kMaxScaleSegments) {
+        if ((grouped_sums || sum_prefills_noise(clipsum_plan(s))) && static_cast<int>(fills.size()) < kMaxScaleSegments) {
           fills.push_back(NoiseFill{layers[l].G_out, static_cast<unsigned long long>(s.m) * s.ne(),
                                     sigma == 0.0f ? 0.0 : static_cast<double>(sigma) * static_cast<double>(layers[l].C),
                                     layers[l].layer_id});
@@ -1983,7 +1997,7 @@ dp_status linear_step(const void* X, const void* dY, const void* P, int r, dp_dt
   if (dt == DP_BF16) {
     // A clipped sum split over K adds its partial sums by atomics: its noise is written into
     // G_out first, by the row-scaling launch that precedes it.
-    const bool prefill = (noise_std != 0.0 && clipsum_plan(c.s).splits > 1);
+    const bool prefill = (noise_std != 0.0 && sum_prefills_noise(clipsum_plan(c.s)));
     // The norm partials are summed by the row-scaling kernel of the clipped sum.
     int count = 0;
     if ((st = bf16_norms(c.s, X, Z, m, c.partials(), c.L.partial_stride, &count, c.status(), c.stream)) !=

@@ -476,20 +476,37 @@ __global__ void __launch_bounds__(256) combine_splits_kernel(CombineBatch b) {
     const unsigned long long nv = sg.elems / 4;
     const unsigned long long first =
         j0 >= seg_begin ? j0 - seg_begin : (stride - (seg_begin - j0) % stride) % stride;
-    for (unsigned long long v = first; v < nv; v += stride) {
-      if (!DP_DCHECK(in_buffer(static_cast<long long>(4 * v), 4, static_cast<long long>(sg.elems)), 32u, nullptr))
-        break;
-      double a[4] = {0.0, 0.0, 0.0, 0.0};
-      if (sg.read_out) {
-        const float4 o = __ldcs(reinterpret_cast<const float4*>(sg.out) + v);
-        a[0] = o.x; a[1] = o.y; a[2] = o.z; a[3] = o.w;
+    // Two splits (the usual case): both partials and the output read before any add, for
+    // every vector of the iteration, so that each thread keeps several loads in flight.
+    constexpr int kV = 2;
+    for (unsigned long long v = first; v < nv; v += kV * stride) {
+      float4 o[kV], p0[kV], p1[kV];
+#pragma unroll
+      for (int u = 0; u < kV; ++u) {
+        const unsigned long long vu = v + u * stride;
+        if (vu >= nv) break;
+        o[u] = sg.read_out ? __ldcs(reinterpret_cast<const float4*>(sg.out) + vu) : make_float4(0.f, 0.f, 0.f, 0.f);
+        p0[u] = __ldcs(reinterpret_cast<const float4*>(sg.scratch) + vu);
+        p1[u] = sg.splits > 1 ? __ldcs(reinterpret_cast<const float4*>(sg.scratch + sg.elems) + vu)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
       }
-      for (int k = 0; k < sg.splits; ++k) {
-        const float4 pk = __ldcs(reinterpret_cast<const float4*>(sg.scratch + k * sg.elems) + v);
-        a[0] += pk.x; a[1] += pk.y; a[2] += pk.z; a[3] += pk.w;
+#pragma unroll
+      for (int u = 0; u < kV; ++u) {
+        const unsigned long long vu = v + u * stride;
+        if (vu >= nv) break;
+        if (!DP_DCHECK(in_buffer(static_cast<long long>(4 * vu), 4, static_cast<long long>(sg.elems)), 32u, nullptr))
+          break;
+        double a[4] = {static_cast<double>(o[u].x), static_cast<double>(o[u].y), static_cast<double>(o[u].z),
+                       static_cast<double>(o[u].w)};
+        a[0] += p0[u].x; a[1] += p0[u].y; a[2] += p0[u].z; a[3] += p0[u].w;
+        a[0] += p1[u].x; a[1] += p1[u].y; a[2] += p1[u].z; a[3] += p1[u].w;
+        for (int k = 2; k < sg.splits; ++k) {
+          const float4 pk = __ldcs(reinterpret_cast<const float4*>(sg.scratch + k * sg.elems) + vu);
+          a[0] += pk.x; a[1] += pk.y; a[2] += pk.z; a[3] += pk.w;
+        }
+        reinterpret_cast<float4*>(sg.out)[vu] = make_float4(static_cast<float>(a[0]), static_cast<float>(a[1]),
+                                                           static_cast<float>(a[2]), static_cast<float>(a[3]));
       }
-      reinterpret_cast<float4*>(sg.out)[v] = make_float4(static_cast<float>(a[0]), static_cast<float>(a[1]),
-                                                        static_cast<float>(a[2]), static_cast<float>(a[3]));
     }
     seg_begin += nv;
   }
