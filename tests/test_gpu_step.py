@@ -268,3 +268,19 @@ def test_norms_and_sums_are_reproducible(method):
     G2, n2 = _step(w, lin, X, dY, 0.0, method)
     assert torch.equal(n1, n2)
     assert torch.equal(G1, G2)
+
+
+@pytest.mark.parametrize("method", ["ghost", "explicit"])
+def test_split_k_sums_are_reproducible_with_noise(method):
+    # One 128 x 128 output tile over 4096 tokens: the clipped sum is split over K into many
+    # parts.  Each part stores its partial sum and one combining launch adds them in split
+    # order to the noise already in the output, so reruns give the same bits whatever order
+    # the parts ran in, and the result matches the oracle's sum and noise.
+    w, lin, data, dev = _custom(8, 512, 128, 128, C=0.3, sigma=1.0, seed=36)
+    X, dY = dev["X"]["in"], dev["dY"]["linear"]
+    G1, n1 = _step(w, lin, X, dY, w.sigma, method)
+    G2, n2 = _step(w, lin, X, dY, w.sigma, method)
+    torch.cuda.synchronize()
+    assert torch.equal(n1, n2)
+    assert torch.equal(G1, G2)
+    check_linear(w, lin, data, dev, method=method, tag=f"split-K reproducible[{method}]")
