@@ -130,6 +130,7 @@ struct UmmaConfig {
   static constexpr bool B_MN = (!GHOST && EPI != kEpiAxpy);
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = BN * BK * 2;
+  static_assert(!GHOST || BM == BN, "ghost tiles are square: a diagonal tile is its own B operand");
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int STAGES = (196608 / STAGE_BYTES) < 8 ? (196608 / STAGE_BYTES) : 8;
   static constexpr int ACCS = (EPI == kEpiGhostNorm)     ? 2
@@ -258,6 +259,14 @@ __device__ __forceinline__ Unit decode_unit(const UmmaParams& p, int u, const Um
   return w;
 }
 
+// A ghost unit on the diagonal (both token blocks the same) forms X_a X_a^T and dY_a dY_a^T:
+// its two operands are one tile, loaded once into the A slot and read by both descriptors.
+template <class Cfg>
+__device__ __forceinline__ bool ghost_diagonal(const Unit& w) {
+  if constexpr (Cfg::GHOST) return w.m_blk == w.n_blk;
+  return false;
+}
+
 template <class Cfg>
 __device__ __forceinline__ void issue_stage_loads(const UmmaParams& p, const Unit& w, int phase,
                                                   int kb, uint32_t sA, uint32_t sB,
@@ -300,13 +309,13 @@ __device__ __forceinline__ void issue_stage_loads(const UmmaParams& p, const Uni
                                          : (phase ? &p.tmA1 : &p.tmA0);
     const CUtensorMap* mb = Cfg::GROUPED ? ma : (phase ? &p.tmB1 : &p.tmB0);
     tma_load_3d(sA, ma, bar, k0, w.m_blk * Cfg::BM, w.sample);
-    tma_load_3d(sB, mb, bar, k0, w.n_blk * Cfg::BN, w.sample);
+    if (!ghost_diagonal<Cfg>(w)) tma_load_3d(sB, mb, bar, k0, w.n_blk * Cfg::BN, w.sample);
   } else if (Cfg::EPI == kEpiGhostShared) {
     // Phase 0 reads X (tmA0), phase 1 + k reads dY operand k (tmB0, tmA1, tmB1); both
     // operands of a Gram tile come from the same map, at the two token blocks of the pair.
     const CUtensorMap* m = phase == 0 ? &p.tmA0 : phase == 1 ? &p.tmB0 : phase == 2 ? &p.tmA1 : &p.tmB1;
     tma_load_3d(sA, m, bar, k0, w.m_blk * Cfg::BM, w.sample);
-    tma_load_3d(sB, m, bar, k0, w.n_blk * Cfg::BN, w.sample);
+    if (!ghost_diagonal<Cfg>(w)) tma_load_3d(sB, m, bar, k0, w.n_blk * Cfg::BN, w.sample);
   } else if (Cfg::EPI == kEpiAxpy) {  // A = U rows, B = P rows, both K-major
     tma_load_2d(sA, &p.tmA0, bar, k0, w.m_blk * Cfg::BM);
     tma_load_2d(sB, &p.tmB0, bar, k0, w.n_blk * Cfg::BN);
@@ -620,7 +629,7 @@ __device__ __forceinline__ void umma_body(const UmmaParams& p, const UmmaGroup* 
             }
             const uint32_t sA = smem_addr(smem + stage * Cfg::STAGE_BYTES);
             const uint32_t bar = smem_addr(full + stage);
-            mbar_arrive_expect_tx(bar, Cfg::STAGE_BYTES);
+            mbar_arrive_expect_tx(bar, ghost_diagonal<Cfg>(w) ? Cfg::A_BYTES : Cfg::STAGE_BYTES);
             issue_stage_loads<Cfg>(p, w, ph, kb, sA, sA + Cfg::A_BYTES, bar, grp);
             if (Cfg::EPI == kEpiClipSum && !Cfg::GROUPED) {
               if (kb == kb_begin) {
@@ -664,7 +673,7 @@ __device__ __forceinline__ void umma_body(const UmmaParams& p, const UmmaGroup* 
             }
             tc_fence_after();
             const uint32_t sA = smem_addr(smem + stage * Cfg::STAGE_BYTES);
-            const uint32_t sB = sA + Cfg::A_BYTES;
+            const uint32_t sB = ghost_diagonal<Cfg>(w) ? sA : sA + Cfg::A_BYTES;
 #pragma unroll
             for (int ks = 0; ks < Cfg::BK / 16; ++ks) {
               umma_bf16(d_tmem, operand_desc<Cfg>(sA, ks, Cfg::A_MN),
