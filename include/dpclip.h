@@ -305,6 +305,16 @@ dp_status dp_projected_adam_step(float* W, const float* R, float* m, float* v, c
  *   workspace : DEVICE, 256-byte aligned, at least 256 bytes. */
 dp_status dp_selftest_wait_timeout(void* workspace, unsigned long long limit_ns, void* stream);
 
+/* Host-side fault injection, for tests of the error paths (no device fault is involved): the
+ * library lets the next `skip` kernel launches of this process through, then makes the
+ * `count` launches after them fail with `cuda_error` (a cudaError_t value, e.g. 2 for
+ * cudaErrorMemoryAllocation) as if the runtime had refused them.  Nothing is enqueued for a
+ * failed launch; the call that made it returns DP_ERR_CUDA and dp_last_cuda_error() names the
+ * launch and the error.  count = 0 clears any pending injection.  The counters are global to
+ * the process and shared by all threads.  Returns DP_ERR_INVALID_ARG for a negative count or
+ * skip, or an error code <= 0 with count > 0. */
+dp_status dp_selftest_fail_launches(long long skip, long long count, int cuda_error);
+
 /* Synchronises `stream`, then reads the status word that the kernels of earlier calls wrote
  * into `workspace`.  Returns DP_OK, DP_ERR_TIMEOUT (a bounded in-kernel wait ran out; the
  * results of that call are invalid), DP_ERR_DEVICE_CHECK or DP_ERR_CUDA.  The word is cleared

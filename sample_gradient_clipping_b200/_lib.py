@@ -55,6 +55,7 @@ SIGNATURES = {
                                          _c_int, _c_void_p, _c_void_p, _c_void_p, _c_size_t, _c_void_p]),
     "dp_workspace_status": (_c_int, [_c_void_p, _c_void_p]),
     "dp_selftest_wait_timeout": (_c_int, [_c_void_p, _c_ull, _c_void_p]),
+    "dp_selftest_fail_launches": (_c_int, [_c_ll, _c_ll, _c_int]),
     "dp_per_sample_norms_static": (_c_int, [_c_void_p, _c_void_p, _c_int, _c_int, _c_int, _c_int, _c_int,
                                             _c_int, _c_void_p, _c_void_p]),
     "dp_philox_blocks": (_c_int, [_c_void_p, _c_ull, _c_ull, _c_ull, _c_uint, _c_uint, _c_void_p]),

@@ -6,6 +6,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdlib>
 #include <cstdint>
@@ -44,9 +45,25 @@ dp_status cuda_fail(cudaError_t e, const char* what) {
 // the previous kernel in the stream drains, runs its local prologue, and waits for that kernel
 // (griddep_wait in ptx.cuh) before its first access to global memory.  This hides most of the
 // launch gap between the short kernels of a step.
+// Host-side fault injection (dp_selftest_fail_launches): launches to let through before the
+// injected failures, the failures left, and the error they report.  Nothing is enqueued for a
+// failed launch, as when the runtime refuses one.
+std::atomic<long long> g_inject_skip{0};
+std::atomic<long long> g_inject_count{0};
+std::atomic<int> g_inject_error{0};
+
+cudaError_t injected_launch_error() {
+  if (g_inject_count.load(std::memory_order_relaxed) <= 0) return cudaSuccess;
+  if (g_inject_skip.fetch_sub(1) > 0) return cudaSuccess;
+  if (g_inject_count.fetch_sub(1) <= 0) return cudaSuccess;
+  return static_cast<cudaError_t>(g_inject_error.load());
+}
+
 template <typename... KArgs, typename... Args>
 cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
                           cudaStream_t stream, Args&&... args) {
+  const cudaError_t injected = injected_launch_error();
+  if (injected != cudaSuccess) return injected;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
@@ -2215,6 +2232,15 @@ dp_status dp_projected_adam_step(float* W, const float* R, float* m, float* v, c
   p.out_elems = static_cast<long long>(d_in) * d_out;
   p.alpha = -lr;
   return launch_umma<UmmaConfig<256, kEpiAxpy>>(p, cs);
+}
+
+dp_status dp_selftest_fail_launches(long long skip, long long count, int cuda_error) {
+  if (skip < 0 || count < 0 || (count > 0 && cuda_error <= 0)) return DP_ERR_INVALID_ARG;
+  g_inject_count.store(0);
+  g_inject_skip.store(skip);
+  g_inject_error.store(cuda_error);
+  g_inject_count.store(count);
+  return DP_OK;
 }
 
 dp_status dp_selftest_wait_timeout(void* workspace, unsigned long long limit_ns, void* stream) {

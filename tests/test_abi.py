@@ -124,6 +124,14 @@ def test_linear_step_rejects_on_host(L, kw, want):
     assert _step(L, **kw) == want
 
 
+def test_launch_fault_injection_arguments(L):
+    E = _lib.DP_ERR_INVALID_ARG
+    assert L.dp_selftest_fail_launches(-1, 1, 2) == E
+    assert L.dp_selftest_fail_launches(0, -1, 2) == E
+    assert L.dp_selftest_fail_launches(0, 1, 0) == E      # an error code is needed
+    assert L.dp_selftest_fail_launches(0, 0, 0) == _lib.DP_OK  # clears (nothing pending)
+
+
 def test_other_entry_points_reject_on_host(L):
     E = _lib.DP_ERR_INVALID_ARG
     assert L.dp_add_noise(None, 4, 4, 1.0, 0, 0, 0, None) == E

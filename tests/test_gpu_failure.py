@@ -35,3 +35,25 @@ def test_bounded_wait_timeout_is_reported_and_device_stays_usable():
     G, n = _lib.dp_linear_step(X, dY, 0.5, 0.0, 3, 0, 0, workspace=wsp)
     assert _lib.dp_workspace_status(wsp) == _lib.DP_OK
     assert torch.isfinite(G).all() and bool((n > 0).all())
+
+
+def test_refused_launch_is_reported_and_the_next_call_is_whole():
+    """Host-side fault injection: a launch the runtime refuses (here as out of memory, through
+    the library's fake of the launch call) makes the call return DP_ERR_CUDA with the launch
+    named; nothing was enqueued for it, and the next call gives the same bits as a clean run."""
+    L = _lib.lib()
+    w = inputs.custom("inject", B=2, T=256, d_in=256, d_out=512, C=0.5, sigma=0.7, seed=5)
+    d = inputs.generate(w)
+    X, dY = d["X"]["in"].cuda(), d["dY"]["linear"].cuda()
+    G_ref, n_ref = _lib.dp_linear_step(X, dY, 0.5, 0.7, 5, 1, 0, method="ghost")
+    torch.cuda.synchronize()
+    for skip in (0, 1, 2):  # the first, second or third kernel launch of the call is refused
+        assert L.dp_selftest_fail_launches(skip, 1, 2) == _lib.DP_OK  # 2: cudaErrorMemoryAllocation
+        with pytest.raises(_lib.DPError) as err:
+            _lib.dp_linear_step(X, dY, 0.5, 0.7, 5, 1, 0, method="ghost")
+        assert err.value.status == _lib.DP_ERR_CUDA
+        assert b"out of memory" in L.dp_last_cuda_error()
+        G, n = _lib.dp_linear_step(X, dY, 0.5, 0.7, 5, 1, 0, method="ghost")
+        torch.cuda.synchronize()
+        assert torch.equal(n, n_ref) and torch.equal(G, G_ref), skip
+    assert L.dp_selftest_fail_launches(0, 0, 0) == _lib.DP_OK
