@@ -132,7 +132,8 @@ struct UmmaConfig {
   static constexpr int B_BYTES = BN * BK * 2;
   static_assert(!GHOST || BM == BN, "ghost tiles are square: a diagonal tile is its own B operand");
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES = (196608 / STAGE_BYTES) < 8 ? (196608 / STAGE_BYTES) : 8;
+  // As many stages as the 227 KB of shared memory hold next to the barriers, up to 8.
+  static constexpr int STAGES = ((232448 - 1280) / STAGE_BYTES) < 8 ? ((232448 - 1280) / STAGE_BYTES) : 8;
   static constexpr int ACCS = (EPI == kEpiGhostNorm)     ? 2
                               : (EPI == kEpiGhostShared) ? 1 + kGhostSharedMaxOps
                                                          : 1;  // accumulators per unit
@@ -140,6 +141,7 @@ struct UmmaConfig {
   static constexpr int NUM_BUFS = 512 / ACC_COLS;
   static constexpr int THREADS = 192;
   static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
+  static_assert(SMEM_BYTES <= 232448, "dynamic shared memory per block");
   static constexpr uint32_t IDESC = umma_idesc_bf16(BM, BN, A_MN, B_MN);
   static_assert(NUM_BUFS >= 1, "TMEM budget");
   static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN");
