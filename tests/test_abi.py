@@ -64,6 +64,18 @@ def test_workspace_size(L):
     assert L.dp_workspace_size(1, 1, 12, 8, 0, _lib.DP_F32) > 0        # fp32 needs multiples of 4
 
 
+def test_workspace_holds_split_partials(L):
+    # GPT-2's 768 x 3072 output fills 36 of 74 SM pairs with 256 x 256 tiles, so its clipped
+    # sum is split in two over the tokens and each split's fp32 partial sum gets a slot.
+    ghost = L.dp_workspace_size_for(32, 512, 768, 3072, 0, _lib.DP_BF16, _lib.DP_NORM_GHOST)
+    scaled = 32 * 512 * 768 * 2                      # the narrower operand, X, scaled in bf16
+    partials = 2 * 768 * 3072 * 4
+    assert scaled + partials <= ghost < scaled + partials + (1 << 20)
+    # The gradients-once layout holds them too, so that it stays the largest.
+    once = L.dp_workspace_size_for(32, 512, 768, 3072, 0, _lib.DP_BF16, _lib.DP_NORM_ONCE)
+    assert once - ghost == 32 * 768 * 3072 * 2       # plus the bf16 per-sample tiles
+
+
 def test_auto_method_cost_model(L):
     # Long sequences over wide layers: forming each G_i once beats a second contraction.
     assert _lib.auto_norm_method(8, 2048, 4096, 4096) == "once"
