@@ -539,7 +539,10 @@ dp_status launch_combine(const CombineBatch& b, cudaStream_t stream) {
   unsigned long long vecs = 0;
   for (int q = 0; q < b.count; ++q) vecs += b.seg[q].elems / 4;
   LaunchScope scope(kKindCombine, stream);
-  DP_LAUNCH("combine_splits_kernel", combine_splits_kernel, stream_grid((vecs + 1) / 2, 256), 256, 0, stream, b);
+  // One wave of resident blocks (3 per SM at 80 registers): a short launch whose second wave
+  // would start after the first one's tail.
+  const int grid = std::min(stream_grid((vecs + 1) / 2, 256), sm_count() * 3);
+  DP_LAUNCH("combine_splits_kernel", combine_splits_kernel, grid, 256, 0, stream, b);
   return DP_OK;
 }
 
