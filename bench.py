@@ -43,8 +43,8 @@ KERNEL_SOURCES = ("sample_gradient_clipping_b200/csrc/ptx.cuh",
                   "sample_gradient_clipping_b200/csrc/umma_gemm_2sm.cuh")
 # (workload, kernel) -> (bytes per launch, source hash)
 MEASURED_TRAFFIC = {
-    ("llama7b_block", "umma_explicit_store"): (875895881, "f293da536260e71b"),
-    ("llama13b_block", "umma_explicit_store"): (675810048, "f293da536260e71b"),
+    ("llama7b_block", "umma_explicit_store"): (895072658, "f293da536260e71b"),
+    ("llama13b_block", "umma_explicit_store"): (683888274, "f293da536260e71b"),
 }
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # A timed region at least this long runs under the sustained (power-capped) clock; a shorter
