@@ -75,8 +75,8 @@ def parse():
     ap.add_argument("--sigma", type=float, default=None, help="noise multiplier (default: the workload's)")
     ap.add_argument("--also", default="auto",
                     help="comma-separated workloads timed after the main one in the same run and "
-                         "reported under 'legs' (default: the Llama-13B block beside the 7B one; "
-                         "'none' for none)")
+                         "reported under 'legs' (default beside the Llama-7B block: the Llama-13B "
+                         "block, GPT-2 MLP up and the projected RoBERTa block; 'none' for none)")
     ap.add_argument("--clip", default="per_layer", choices=["per_layer", "flat"],
                     help="per-layer bounds C_l, or one flat bound sqrt(L) * C_l for the whole block")
     return ap.parse_args()
@@ -530,7 +530,7 @@ def extra_legs(args, w, shard):
     if shard or args.also == "none":
         return []
     if args.also == "auto":
-        return ["llama13b_block"] if w.name == "llama7b_block" else []
+        return ["llama13b_block", "gpt2_mlp_up", "roberta_large_projected"] if w.name == "llama7b_block" else []
     return [n for n in args.also.split(",") if n and n != w.name]
 
 
@@ -569,7 +569,8 @@ def run_ours(args, w, rank, world):
     del ctx
     torch.cuda.empty_cache()
 
-    # ---- further workloads in the same run (the Llama-13B block beside the 7B one)
+    # ---- further workloads in the same run (the Llama-13B block and the two small
+    # configurations beside the 7B one)
     legs = {}
     for name in extra_legs(args, w, shard):
         lw = inputs.WORKLOADS[name]
