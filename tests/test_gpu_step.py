@@ -153,8 +153,12 @@ def _custom(B, T, m, n, dtype="bf16", **kw):
     return w, w.linears[0], data, dev
 
 
+# (3, 200, 128, 1000) and (3, 200, 1000, 128): 9 ghost units, fewer than the SMs, with one Gram
+# eight times the other's depth, so every unit is cut in two over the deeper Gram's K (ragged
+# last K block and ragged T included).
 @pytest.mark.parametrize("B,T,m,n", [(1, 1, 8, 8), (3, 200, 320, 392), (2, 257, 264, 136),
-                                     (7, 64, 1024, 128), (1, 4096, 128, 128)])
+                                     (7, 64, 1024, 128), (1, 4096, 128, 128),
+                                     (3, 200, 128, 1000), (3, 200, 1000, 128)])
 @pytest.mark.parametrize("method", ["ghost", "explicit", "once"])
 def test_ragged_shapes(B, T, m, n, method):
     w, lin, data, dev = _custom(B, T, m, n, C=0.5, sigma=0.7, seed=31)
