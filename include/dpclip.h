@@ -329,7 +329,10 @@ dp_status dp_selftest_fail_launches(long long skip, long long count, int cuda_er
  * build the checks compile away. */
 dp_status dp_workspace_status(const void* workspace, void* stream);
 
-/* Norm method that DP_NORM_AUTO picks for these shapes (GHOST, EXPLICIT or ONCE). */
+/* Norm method that DP_NORM_AUTO picks for these shapes (GHOST, EXPLICIT or ONCE).  For bf16,
+ * the environment variable DPCLIP_NORM=ghost|explicit|once, read at every call, overrides the
+ * cost model in every call made with DP_NORM_AUTO (and in dp_workspace_size); other values
+ * are ignored.  fp32 always takes EXPLICIT. */
 dp_norm_method dp_auto_norm_method(int B, int T, int d_in, int d_out, int r, dp_dtype dt);
 
 /* Launch accounting, for measurement.  dp_kernel_launches() is the number of kernels this

@@ -297,8 +297,23 @@ double model_cost(const Shape& s, dp_norm_method m) {
   return std::max(per_sample, store) + reduce + 3 * kModelLaunch;
 }
 
+// DPCLIP_NORM=ghost|explicit|once in the environment overrides the cost model for bf16 calls
+// with DP_NORM_AUTO (read at every call, so a workspace size query and the call that uses it
+// see the same setting); any other value, or none, leaves the choice to the model.
+bool env_norm_method(dp_norm_method* out) {
+  const char* v = getenv("DPCLIP_NORM");
+  if (!v) return false;
+  if (!strcmp(v, "ghost")) *out = DP_NORM_GHOST;
+  else if (!strcmp(v, "explicit")) *out = DP_NORM_EXPLICIT;
+  else if (!strcmp(v, "once")) *out = DP_NORM_ONCE;
+  else return false;
+  return true;
+}
+
 dp_norm_method auto_method(const Shape& s) {
   if (s.dt == DP_F32) return DP_NORM_EXPLICIT;
+  dp_norm_method forced;
+  if (env_norm_method(&forced)) return forced;
   dp_norm_method best = DP_NORM_GHOST;
   for (dp_norm_method m : {DP_NORM_EXPLICIT, DP_NORM_ONCE})
     if (model_cost(s, m) < model_cost(s, best)) best = m;

@@ -64,6 +64,22 @@ def test_workspace_size(L):
     assert L.dp_workspace_size(1, 1, 12, 8, 0, _lib.DP_F32) > 0        # fp32 needs multiples of 4
 
 
+def test_norm_method_environment_override(L):
+    try:
+        for name in ("ghost", "explicit", "once"):
+            os.environ["DPCLIP_NORM"] = name
+            assert _lib.auto_norm_method(8, 2048, 4096, 4096) == name
+            assert _lib.auto_norm_method(4, 16, 64, 32, dtype_code=_lib.DP_F32) == "explicit"
+        os.environ["DPCLIP_NORM"] = "once"      # the workspace query sees the same choice
+        assert L.dp_workspace_size(32, 512, 768, 3072, 0, _lib.DP_BF16) == \
+            L.dp_workspace_size_for(32, 512, 768, 3072, 0, _lib.DP_BF16, _lib.DP_NORM_ONCE)
+        os.environ["DPCLIP_NORM"] = "fastest"   # not a method: the cost model decides
+        assert _lib.auto_norm_method(32, 512, 768, 3072) == "ghost"
+    finally:
+        os.environ.pop("DPCLIP_NORM", None)
+    assert _lib.auto_norm_method(8, 2048, 4096, 4096) == "once"
+
+
 def test_workspace_holds_split_partials(L):
     # GPT-2's 768 x 3072 output fills 36 of 74 SM pairs with 256 x 256 tiles, so its clipped
     # sum is split in two over the tokens and each split's fp32 partial sum gets a slot.
