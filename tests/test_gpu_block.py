@@ -190,11 +190,16 @@ def _projected_block(r=64, B=4, T=128, seed=17):
     return w, data, X, dY, P
 
 
+# (r, B, T): the small block forms Z = dY P in 128 x 64 tiles (4 row tiles a linear); the larger ones have
+# 24 row tiles per linear, a ragged last one (N = 3000), and 128 x 128 tiles whose columns r = 96
+# only partly fill.
+@pytest.mark.parametrize("shape", [(64, 4, 128), (128, 6, 500), (96, 6, 500)], ids=["r64", "r128_ragged", "r96_ragged"])
 @pytest.mark.parametrize("mode", ["per_layer", "flat"])
-def test_projected_block_against_oracle(mode):
+def test_projected_block_against_oracle(mode, shape):
     """DP-GRAPE layers in one block call: each clips, sums and noises G_i P; q/k/v and gate/up
     share their X Grams (equal widths r)."""
-    w, data, X, dY, P = _projected_block()
+    r_width, B, T = shape
+    w, data, X, dY, P = _projected_block(r=r_width, B=B, T=T)
     C = 0.8
     layers = [{"X": X[l.x_key], "dY": dY[l.name], "P": P[l.name], "layer_id": l.layer_id, "C": C,
                "norms_out": torch.empty(w.B, dtype=torch.float32, device="cuda")} for l in w.linears]
@@ -213,7 +218,7 @@ def test_projected_block_against_oracle(mode):
         assert rel_max(host(flat), ref["flat_norms"]) <= tol["norm"]
     for k, lin in enumerate(w.linears):
         r = ref["layers"][k]
-        assert outs[k].shape == (lin.d_in, 64)
+        assert outs[k].shape == (lin.d_in, r_width)
         assert rel_max(host(norms[k]), r["norms"]) <= tol["norm"], lin.name
         assert rel_fro(host(outs[k]), r["S"]) <= tol["sum"], lin.name
     # The noise of a projected layer has the [d_in, r] shape and is added once.

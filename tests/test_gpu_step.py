@@ -116,6 +116,32 @@ def test_roberta_projected_workload(method):
         check_linear(w, lin, data, dev, method=method)
 
 
+@pytest.mark.parametrize("method", ["auto", "ghost"])
+def test_roberta_projected_block(method):
+    """The RoBERTa block in the call the benchmark times: one per-layer dp_block_step over the six
+    projected linears (their Z = dY P in one grouped launch, the grouped ghost norms and clipped
+    sums split over the tokens), at sigma 0 and sigma; every linear's norms, clipped sum and noise
+    are compared with the oracle."""
+    w = inputs.WORKLOADS["roberta_large_projected"]
+    data, dev = draw(w)
+    P = {l.name: _lib.dp_projection_matrix(torch.empty(l.d_out, w.r, dtype=torch.bfloat16, device="cuda"),
+                                           w.seed, l.layer_id) for l in w.linears}
+
+    def block(sigma):
+        layers = [{"X": dev["X"][l.x_key], "dY": dev["dY"][l.name], "P": P[l.name], "layer_id": l.layer_id,
+                   "C": w.C, "norms_out": torch.empty(w.B, dtype=torch.float32, device="cuda")}
+                  for l in w.linears]
+        outs, norms, _ = _lib.dp_block_step(layers, mode="per_layer", sigma=sigma, seed=w.seed, step=w.step,
+                                            method=method)
+        return outs, norms
+
+    outs0, norms0 = block(0.0)
+    outs1, _ = block(w.sigma)
+    for k, lin in enumerate(w.linears):
+        check_linear(w, lin, data, dev, method=method, got=(outs0[k], norms0[k], outs1[k]),
+                     tag=f"roberta_large_projected[{method}] block")
+
+
 @pytest.mark.slow
 @pytest.mark.parametrize("name,method", [("llama7b_block", "auto"), ("llama13b_block", "auto"),
                                          ("llama13b_block", "ghost")])
