@@ -151,13 +151,14 @@ dp_status dp_projection_matrix(void* P, dp_dtype dt, int d_out, int r,
  *   norms_out  : NULL or DEVICE fp32 [B].
  *   G_out      : DEVICE fp32 [d_in, r or d_out], overwritten.  The gradients-once method
  *                rounds sigma*C*z to fp32 before adding it to the fp32 sum (within one ulp
- *                of rounding the fp64 sum once).  A ghost or explicit clipped sum that runs
- *                in one wave or is split over K (small outputs) gets sigma*C*z rounded to fp32
- *                from the row-scaling launch before the sum; a split sum stores each split's
- *                partial sum in the workspace and a combining launch adds them to the noise
- *                in split order in fp64, rounding once, so the result does not depend on the
- *                order the splits ran in.  Otherwise the epilogue adds the noise in fp64 and
- *                rounds once.  bf16 results are the same bits on every run. */
+ *                of rounding the fp64 sum once).  A ghost or explicit clipped sum split over
+ *                K (small outputs) stores each split's partial sum in the workspace, and a
+ *                combining launch adds sigma*C*z and the partials in split order in fp64,
+ *                rounding once, so the result does not depend on the order the splits ran
+ *                in.  An unsplit sum that runs in one wave gets sigma*C*z rounded to fp32 from
+ *                the row-scaling launch before it and adds itself to that.  Otherwise the
+ *                epilogue adds the noise in fp64 and rounds once.  bf16 results are the same
+ *                bits on every run. */
 dp_status dp_linear_step(const void* X, const void* dY, const void* P, int r, dp_dtype dt,
                          int B, int T, int d_in, int d_out, float C, float sigma,
                          unsigned long long seed, unsigned long long step, unsigned layer_id,

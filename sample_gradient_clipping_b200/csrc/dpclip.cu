@@ -207,14 +207,17 @@ ClipSumPlan clipsum_plan(const Shape& s) {
 }
 
 // Whether a clipped sum takes its noise from the row-scaling launch before it (which writes
-// the noise into the output, each value rounded to fp32 once) instead of from its epilogue:
-// when it is split over K (the noise must go on the finished sum), or when all its units run
-// in one wave, where the epilogue's fp64 noise would run after every tile with nothing to
-// hide it (measured on unsplit 256x128 tiles of GPT-2's output: 100 against 96 us).  The sum
-// is then added to the noise.
-bool sum_prefills_noise(const ClipSumPlan& c) {
+// the noise into the output, each value rounded to fp32 once) instead of from its epilogue or
+// its combining launch: when all its units run in one unsplit wave, where the epilogue's fp64
+// noise would run after every tile with nothing to hide it (measured on unsplit 256x128 tiles
+// of GPT-2's output: 100 against 96 us), or when it is split over K into more splits than the
+// workspace holds partials for (`fixup_splits`), so that its splits add by atomics.  The sum
+// is then added to the noise.  A sum split over K with its split partials takes its noise in
+// the combining launch, on the finished sum.
+bool sum_prefills_noise(const ClipSumPlan& c, int fixup_splits) {
   const int slots = c.pair ? sm_count() / 2 : sm_count();
-  return c.splits > 1 || c.m_tiles * c.n_tiles <= slots;
+  if (c.splits > 1) return c.splits > fixup_splits;
+  return c.m_tiles * c.n_tiles <= slots;
 }
 
 // Where a clipped sum split over K keeps its split partials (kOutSplitPartials).
@@ -566,9 +569,10 @@ dp_status launch_combine(const CombineBatch& b, cudaStream_t stream) {
 // With `defer` (a block step), noise that cannot ride in the epilogue (split K) is queued
 // there instead of launched.  With `preset` (split K only), out already holds the noise
 // (written by the row-scaling launch) and the sum is added to it.
-// Split over K with `fx`: each split stores its partial sum, and a combining launch adds them
-// in split order to out's contents in fp64 and rounds once (kOutSplitPartials).  Without it,
-// the splits add their partial sums into out by fp32 atomics.
+// Split over K with `fx`: each split stores its partial sum, and a combining launch adds the
+// noise and them, in split order, to out's contents (accumulate or preset) in fp64 and rounds
+// once (kOutSplitPartials).  Without it, the splits add their partial sums into out by fp32
+// atomics and the noise follows.
 dp_status bf16_clipsum(const Shape& s, const void* A, const void* Bm, float* out, int accumulate,
                        double noise_std, unsigned long long seed, StepRef step,
                        unsigned layer_id, uint32_t* status, cudaStream_t stream,
@@ -623,9 +627,11 @@ dp_status bf16_clipsum(const Shape& s, const void* A, const void* Bm, float* out
     CombineBatch cb;
     memset(&cb, 0, sizeof(cb));
     cb.count = 1;
+    cb.key = key;
+    cb.step = step;
     cb.seg[0] = CombineSegment{out, fx->scratch, static_cast<unsigned long long>(s.m) * ne, splits,
-                               (accumulate || preset) ? 1 : 0};
-    st2 = launch_combine(cb, stream);
+                               (accumulate || preset) ? 1 : 0, noise_std, static_cast<uint32_t>(layer_id)};
+    return launch_combine(cb, stream);
   }
   if (st2 != DP_OK || fused_noise || noise_std == 0.0) return st2;
   if (defer && defer->count < kMaxNoiseSegments) {
@@ -1521,8 +1527,10 @@ dp_status block_layer_sum(const dp_layer* layers, int l, dp_dtype dt, int B, int
   const void* Z;
   dp_status st = block_operand(layers, l, dt, B, T, Lb, ws, stream, false, &Z);  // formed by the norms
   if (st != DP_OK) return st;
-  // A bf16 sum split over K: its row-scaling launch writes the noise first (as in one linear).
-  const bool prefill = (dt == DP_BF16 && noise_std != 0.0 && sum_prefills_noise(clipsum_plan(s)));
+  // A bf16 sum that adds itself to its output: its row-scaling launch writes the noise first
+  // (as in one linear).
+  const bool prefill =
+      (dt == DP_BF16 && noise_std != 0.0 && sum_prefills_noise(clipsum_plan(s), Lb.fixup_splits[l]));
   return clipped_sum(c, y.X, Z, src, C, y.G_out, 0, noise_std, seed, step, y.layer_id, defer, partials,
                      prefill);
 }
@@ -1538,11 +1546,13 @@ NormSource layer_norm_source(const BlockLayout& Lb, uint8_t* ws, int l, int B, d
 
 // The clipped sums of the layers in `ls` (batched schedule, groupable) in grouped launches of
 // up to kMaxGroup problems.  One K split for the whole launch (group_sum_splits), chosen so
-// that its units fill the GPU about once; every output already holds its noise (or zeros).
-// The splits store their partial sums and one combining launch adds them to the outputs in
-// split order (kOutSplitPartials); without the layout's split partials they add by atomics.
+// that its units fill the GPU about once.  The splits store their partial sums and one
+// combining launch forms every output from its noise (std sigma C_l) and its partials, in
+// split order (kOutSplitPartials).  Without the layout's split partials the outputs are zeroed,
+// the splits add by atomics, and the noise is queued in `deferred`.
 dp_status launch_clipsum_groups(const dp_layer* layers, const std::vector<int>& ls, dp_dtype dt, int B, int T,
-                                const BlockLayout& Lb, uint8_t* ws, cudaStream_t stream) {
+                                const BlockLayout& Lb, uint8_t* ws, float sigma, unsigned long long seed,
+                                StepRef step, NoiseBatch* deferred, cudaStream_t stream) {
   dp_status st;
   for (size_t c0 = 0; c0 < ls.size(); c0 += kMaxGroup) {
     const int count = static_cast<int>(std::min<size_t>(kMaxGroup, ls.size() - c0));
@@ -1588,21 +1598,33 @@ dp_status launch_clipsum_groups(const dp_layer* layers, const std::vector<int>& 
     p.k_splits = splits;
     p.out_cols = layer_shape(layers[ls[c0]], B, T, dt).ne();
     p.out_mode = fix ? kOutSplitPartials : kOutAtomicAdd;
-    p.noise_std = 0.0;  // written into the outputs beforehand
+    p.noise_std = 0.0;  // added to the finished sums
+    if (!fix)
+      for (int q = 0; q < count; ++q) {
+        const Shape s = layer_shape(layers[ls[c0 + q]], B, T, dt);
+        DP_CUDA(cudaMemsetAsync(g.out_f32[q], 0, static_cast<size_t>(s.m) * s.ne() * sizeof(float), stream));
+      }
     if (plan0.bn == 128) st = launch_umma_group<UmmaConfig<128, kEpiClipSum, true>>(p, g, stream);
     else st = launch_umma_group<UmmaConfig<256, kEpiClipSum, true>>(p, g, stream);
     if (st != DP_OK) return st;
-    if (fix) {
-      CombineBatch cb;
-      memset(&cb, 0, sizeof(cb));
-      cb.count = count;
-      for (int q = 0; q < count; ++q) {
-        const Shape s = layer_shape(layers[ls[c0 + q]], B, T, dt);
-        cb.seg[q] = CombineSegment{g.out_f32[q], g.split_scratch[q], static_cast<unsigned long long>(s.m) * s.ne(),
-                                   splits, 1};
+    CombineBatch cb;
+    memset(&cb, 0, sizeof(cb));
+    cb.key = philox_key_from_seed(seed);
+    cb.step = step;
+    for (int q = 0; q < count; ++q) {
+      const dp_layer& y = layers[ls[c0 + q]];
+      const Shape s = layer_shape(y, B, T, dt);
+      const unsigned long long elems = static_cast<unsigned long long>(s.m) * s.ne();
+      const double std_dev = sigma == 0.0f ? 0.0 : static_cast<double>(sigma) * static_cast<double>(y.C);
+      if (fix) {
+        cb.seg[cb.count++] = CombineSegment{g.out_f32[q], g.split_scratch[q], elems, splits, 0, std_dev, y.layer_id};
+      } else if (std_dev != 0.0 && deferred->count < kMaxNoiseSegments) {
+        deferred->seg[deferred->count++] = NoiseSegment{g.out_f32[q], elems, std_dev, y.layer_id};
+      } else if (std_dev != 0.0 && (st = launch_noise(g.out_f32[q], elems, std_dev, seed, step, y.layer_id, stream)) != DP_OK) {
+        return st;
       }
-      if ((st = launch_combine(cb, stream)) != DP_OK) return st;
     }
+    if (fix && (st = launch_combine(cb, stream)) != DP_OK) return st;
   }
   return DP_OK;
 }
@@ -1696,9 +1718,10 @@ dp_status block_step(const dp_layer* layers, int L, dp_dtype dt, int B, int T, d
     bool side_pending = false;  // reduces on the side stream the caller's stream has not joined
     std::vector<int> batch_layers, batch_counts;  // batched schedule: layers waiting for their sums
     std::vector<int> ghost_single, ghost_single_at;  // batched schedule: single ghost layers, their slots
-    // Batched schedule: the noise of every split-K clipped sum (of every clipped sum when they
-    // run grouped, zeros at sigma 0) is written into its output by the batched row-scaling
-    // launch; those sums then add their partial sums to it.
+    // Batched schedule: the noise of every clipped sum that adds itself to its output (one
+    // unsplit wave, or splits without their partials' workspace) is written into that output by
+    // the batched row-scaling launch.  Grouped sums, and sums split with their partials, take
+    // their noise in the combining launch.
     std::vector<bool> preset(L, false);
     std::vector<NoiseFill> fills;
     std::vector<int> batch_all;
@@ -1706,13 +1729,12 @@ dp_status block_step(const dp_layer* layers, int L, dp_dtype dt, int B, int T, d
       for (const auto& g : Lb.groups)
         if (Lb.methods[g[0]] != DP_NORM_ONCE) batch_all.insert(batch_all.end(), g.begin(), g.end());
     const bool grouped_sums = Lb.batched_scale && dt == DP_BF16 && clipsums_groupable(layers, batch_all, B, T, dt);
-    if (Lb.batched_scale && (sigma != 0.0f || grouped_sums)) {
+    if (Lb.batched_scale && sigma != 0.0f && !grouped_sums) {
       for (int l : batch_all) {
         const Shape s = layer_shape(layers[l], B, T, dt);
-        if ((grouped_sums || sum_prefills_noise(clipsum_plan(s))) && static_cast<int>(fills.size()) < kMaxScaleSegments) {
+        if (sum_prefills_noise(clipsum_plan(s), Lb.fixup_splits[l]) && static_cast<int>(fills.size()) < kMaxScaleSegments) {
           fills.push_back(NoiseFill{layers[l].G_out, static_cast<unsigned long long>(s.m) * s.ne(),
-                                    sigma == 0.0f ? 0.0 : static_cast<double>(sigma) * static_cast<double>(layers[l].C),
-                                    layers[l].layer_id});
+                                    static_cast<double>(sigma) * static_cast<double>(layers[l].C), layers[l].layer_id});
           preset[l] = true;
         }
       }
@@ -1801,7 +1823,8 @@ dp_status block_step(const dp_layer* layers, int L, dp_dtype dt, int B, int T, d
       if ((st = launch_scale_batch(layers, batch_layers, batch_counts, dt, B, T, Lb, ws, stream, fills, seed,
                                    step)) != DP_OK)
         return st;
-      if (grouped_sums && (st = launch_clipsum_groups(layers, batch_layers, dt, B, T, Lb, ws, stream)) != DP_OK)
+      if (grouped_sums && (st = launch_clipsum_groups(layers, batch_layers, dt, B, T, Lb, ws, sigma, seed, step,
+                                                      &deferred, stream)) != DP_OK)
         return st;
       for (int l : grouped_sums ? std::vector<int>() : batch_layers) {
         const dp_layer& y = layers[l];
@@ -2030,9 +2053,9 @@ dp_status linear_step(const void* X, const void* dY, const void* P, int r, dp_dt
                          c.status(), &pr);
   }
   if (dt == DP_BF16) {
-    // A clipped sum split over K adds its partial sums by atomics: its noise is written into
-    // G_out first, by the row-scaling launch that precedes it.
-    const bool prefill = (noise_std != 0.0 && sum_prefills_noise(clipsum_plan(c.s)));
+    // A clipped sum that adds itself to G_out (one unsplit wave, or splits without their
+    // partials' workspace) finds its noise there, written by the row-scaling launch before it.
+    const bool prefill = (noise_std != 0.0 && sum_prefills_noise(clipsum_plan(c.s), c.L.fixup_splits));
     // The norm partials are summed by the row-scaling kernel of the clipped sum.
     int count = 0;
     if ((st = bf16_norms(c.s, X, Z, m, c.partials(), c.L.partial_stride, &count, c.status(), c.stream)) !=

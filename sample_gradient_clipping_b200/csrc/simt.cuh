@@ -349,10 +349,12 @@ __device__ __forceinline__ void scale_rows_body(const __nv_bfloat16* __restrict_
   }
 }
 
-// The noise of a clipped sum split over K, written into its output before the sum (which then
-// adds its partial sums by atomics): out[k] = fp32(std * z_k), z from stream 0 under the
-// layer's counter; std = 0 writes zeros.  The row-scaling kernel that precedes the sum carries
-// it: the scaling is an HBM stream with idle arithmetic pipes, and the sum needs both.
+// The noise of a clipped sum that adds its result to its output (an unsplit sum whose units
+// all run in one wave, or a sum split over K without workspace for its split partials, whose
+// splits then add by atomics), written into that output before the sum: out[k] = fp32(std *
+// z_k), z from stream 0 under the layer's counter; std = 0 writes zeros.  The row-scaling
+// kernel that precedes the sum carries it: the scaling is an HBM stream with idle arithmetic
+// pipes, and the sum needs both.
 struct NoiseFill {
   float* G;                   // null: nothing to write
   unsigned long long total;   // elements
@@ -447,12 +449,14 @@ __device__ __forceinline__ void noise8_f32(uint32_t blk0, uint32_t layer_id, uin
   for (int q = 0; q < 8; ++q) n[q] = __double2float_rn(z[q]);
 }
 
-// The last step of clipped sums split over K: out[e] = fp32(o + sum_k scratch[k][e]), the
-// split partials added in split order in fp64 and rounded once, where o is what out holds
-// (the noise written by the row-scaling launch, zeros, or the caller's accumulator) when
-// read_out, else 0.  The result is the same whatever order the split units ran in, and the
-// noise is added to the finished sum as in an unsplit epilogue.  Segments are walked as in
-// noise_fill_share: global vector j of their concatenation goes to thread j mod (grid size).
+// The last step of clipped sums split over K: out[e] = fp32(o + std z_e + sum_k scratch[k][e]),
+// added in fp64 (the split partials in split order) and rounded once, where o is what out
+// holds (the caller's accumulator, or noise written by a row-scaling launch) when read_out,
+// else 0, and z_e is the output's noise (stream 0 under the layer's counter; none at std 0).
+// The result is the same whatever order the split units ran in, and the noise goes on the
+// finished sum as in an unsplit epilogue.  Segments are walked as in noise_fill_share: global
+// vector j of their concatenation goes to thread j mod (grid size); vector j of a segment is
+// its Philox block j.
 constexpr int kMaxCombineSegments = 8;
 struct CombineSegment {
   float* out;
@@ -460,16 +464,21 @@ struct CombineSegment {
   unsigned long long elems;  // a multiple of 4
   int splits;
   int read_out;
+  double std_dev;            // 0: no noise
+  uint32_t layer_id;
 };
 struct CombineBatch {
   CombineSegment seg[kMaxCombineSegments];
   int count;
+  PhiloxKey key;
+  StepRef step;
 };
 
 __global__ void __launch_bounds__(256) combine_splits_kernel(CombineBatch b) {
   griddep_enter();
   const unsigned long long stride = static_cast<unsigned long long>(gridDim.x) * blockDim.x;
   const unsigned long long j0 = static_cast<unsigned long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const uint32_t step_lo = b.step.get();
   unsigned long long seg_begin = 0;
   for (int q = 0; q < b.count; ++q) {
     const CombineSegment sg = b.seg[q];
@@ -477,7 +486,8 @@ __global__ void __launch_bounds__(256) combine_splits_kernel(CombineBatch b) {
     const unsigned long long first =
         j0 >= seg_begin ? j0 - seg_begin : (stride - (seg_begin - j0) % stride) % stride;
     // Two splits (the usual case): both partials and the output read before any add, for
-    // every vector of the iteration, so that each thread keeps several loads in flight.
+    // every vector of the iteration, so that each thread keeps several loads in flight; the
+    // noise is formed while they land.
     constexpr int kV = 2;
     for (unsigned long long v = first; v < nv; v += kV * stride) {
       float4 o[kV], p0[kV], p1[kV];
@@ -496,8 +506,11 @@ __global__ void __launch_bounds__(256) combine_splits_kernel(CombineBatch b) {
         if (vu >= nv) break;
         if (!DP_DCHECK(in_buffer(static_cast<long long>(4 * vu), 4, static_cast<long long>(sg.elems)), 32u, nullptr))
           break;
-        double a[4] = {static_cast<double>(o[u].x), static_cast<double>(o[u].y), static_cast<double>(o[u].z),
-                       static_cast<double>(o[u].w)};
+        double a[4] = {0.0, 0.0, 0.0, 0.0};
+        if (sg.std_dev != 0.0)
+          normals4(static_cast<uint32_t>(vu), sg.layer_id, step_lo, kStreamNoise, b.key, a, NoiseTablesGlobal{},
+                   sg.std_dev);
+        a[0] += o[u].x; a[1] += o[u].y; a[2] += o[u].z; a[3] += o[u].w;
         a[0] += p0[u].x; a[1] += p0[u].y; a[2] += p0[u].z; a[3] += p0[u].w;
         a[0] += p1[u].x; a[1] += p1[u].y; a[2] += p1[u].z; a[3] += p1[u].w;
         for (int k = 2; k < sg.splits; ++k) {
