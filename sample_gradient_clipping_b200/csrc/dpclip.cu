@@ -557,9 +557,9 @@ dp_status launch_combine(const CombineBatch& b, cudaStream_t stream) {
   unsigned long long vecs = 0;
   for (int q = 0; q < b.count; ++q) vecs += b.seg[q].elems / 4;
   LaunchScope scope(kKindCombine, stream);
-  // One wave of resident blocks (3 per SM at 80 registers): a short launch whose second wave
+  // One wave of resident blocks (4 per SM at 64 registers): a short launch whose second wave
   // would start after the first one's tail.
-  const int grid = std::min(stream_grid((vecs + 1) / 2, 256), sm_count() * 3);
+  const int grid = std::min(stream_grid(vecs, 256), sm_count() * 4);
   DP_LAUNCH("combine_splits_kernel", combine_splits_kernel, grid, 256, 0, stream, b);
   return DP_OK;
 }

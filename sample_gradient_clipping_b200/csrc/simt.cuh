@@ -474,7 +474,7 @@ struct CombineBatch {
   StepRef step;
 };
 
-__global__ void __launch_bounds__(256) combine_splits_kernel(CombineBatch b) {
+__global__ void __launch_bounds__(256, 4) combine_splits_kernel(CombineBatch b) {
   griddep_enter();
   const unsigned long long stride = static_cast<unsigned long long>(gridDim.x) * blockDim.x;
   const unsigned long long j0 = static_cast<unsigned long long>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -485,10 +485,11 @@ __global__ void __launch_bounds__(256) combine_splits_kernel(CombineBatch b) {
     const unsigned long long nv = sg.elems / 4;
     const unsigned long long first =
         j0 >= seg_begin ? j0 - seg_begin : (stride - (seg_begin - j0) % stride) % stride;
-    // Two splits (the usual case): both partials and the output read before any add, for
-    // every vector of the iteration, so that each thread keeps several loads in flight; the
-    // noise is formed while they land.
-    constexpr int kV = 2;
+    // One vector an iteration: the output and the partials are read before any add, and the
+    // noise is formed while they land.  (Two vectors an iteration kept more loads in flight per
+    // thread but took 80 registers, 3 blocks per SM, and left a tail of one iteration in
+    // three: GPT-2 14.8 against 13.0 us at 64 registers and 4 blocks.)
+    constexpr int kV = 1;
     for (unsigned long long v = first; v < nv; v += kV * stride) {
       float4 o[kV], p0[kV], p1[kV];
 #pragma unroll
