@@ -980,8 +980,8 @@ dp_status clipped_sum(Call& c, const void* X, const void* Z, NormSource src, flo
                       int accumulate, double noise_std, unsigned long long seed,
                       StepRef step, unsigned layer_id, NoiseBatch* defer = nullptr,
                       const PartialsRef* partials = nullptr, bool prefill_noise = false) {
-  // prefill_noise (a clipped sum split over K, accumulate = 0): the row-scaling launch also
-  // writes the noise into out, and the contraction adds its partial sums to it.
+  // prefill_noise (a clipped sum that adds itself to out, accumulate = 0): the row-scaling
+  // launch also writes the noise into out, and the contraction adds its sum to it.
   const Shape& s = c.s;
   if (s.dt == DP_F32) {
     dim3 grid(ceil_div(s.ne(), kF32Tile), ceil_div(s.m, kF32Tile));

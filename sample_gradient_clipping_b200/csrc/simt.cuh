@@ -421,7 +421,7 @@ struct ScaleBatch {
   ScaleSegment seg[kMaxScaleSegments];
   int count;
   int T;
-  NoiseFill fill[kMaxScaleSegments];  // noise (or zeros) for the split-K sums that follow
+  NoiseFill fill[kMaxScaleSegments];  // noise for the one-wave sums that follow, which add to it
   int fills;
   PhiloxKey key;
   StepRef step;

@@ -94,8 +94,8 @@ struct alignas(64) UmmaParams {
 
 // Several independent problems of one contraction kind in one launch: the projections
 // Z_l = dY_l P_l of a block's projected linears (kEpiStoreBf16), or the clipped sums of a
-// block's ghost/explicit linears (kEpiClipSum, split over K, always added by atomics into an
-// output that already holds the noise or zeros).  Problem q has its own operand maps, output,
+// block's ghost/explicit linears (kEpiClipSum, split over K: each split stores its partial sum,
+// and a combining launch forms the outputs).  Problem q has its own operand maps, output,
 // rows and K depth, and the units [unit_begin[q], unit_begin[q + 1]) of the launch.  Passed as
 // a second __grid_constant__ parameter, so launches of one problem keep their parameter size.
 constexpr int kMaxGroup = 8;
