@@ -87,3 +87,36 @@ def test_noise_tables_match_their_generator():
     spec.loader.exec_module(gen)
     with open(os.path.join(CSRC, "noise_tables.cuh")) as f:
         assert f.read() == gen.render()
+
+
+def _profile_commands():
+    """(file, command) of every command in the fenced blocks of the ncu summaries in profiles/,
+    continuation lines joined and `&&` chains split."""
+    out = []
+    pdir = os.path.join(ROOT, "profiles")
+    for fn in sorted(os.listdir(pdir)):
+        text = open(os.path.join(pdir, fn)).read()
+        for block in re.findall(r"```[^\n]*\n(.*?)```", text, flags=re.S):
+            joined = re.sub(r"\\\n\s*", " ", block)
+            for line in joined.splitlines():
+                for cmd in line.split("&&"):
+                    if cmd.strip():
+                        out.append((fn, cmd.strip()))
+    return out
+
+
+def test_profiles_hold_summaries_whose_commands_run_committed_files():
+    """The ncu summaries are text, each gives the command that made it, every ncu command leaves
+    the clocks alone, and every script it runs is part of the repository."""
+    pdir = os.path.join(ROOT, "profiles")
+    assert all(fn.endswith((".md", ".txt")) for fn in os.listdir(pdir))
+    cmds = _profile_commands()
+    files = {fn for fn, _ in cmds}
+    assert files == {fn for fn in os.listdir(pdir)}, "a summary without its command"
+    for fn, cmd in cmds:
+        if cmd.startswith("ncu "):
+            assert "--clock-control none" in cmd, (fn, cmd)
+        for script in re.findall(r"\bpython\s+(?:-m\s+([\w.]+)|([\w./]+\.py))", cmd):
+            mod, path = script
+            target = os.path.join(ROOT, *mod.split(".")) + ".py" if mod else os.path.join(ROOT, path)
+            assert os.path.exists(target), (fn, cmd)
