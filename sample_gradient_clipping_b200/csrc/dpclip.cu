@@ -566,9 +566,9 @@ dp_status launch_combine(const CombineBatch& b, cudaStream_t stream) {
 
 // out (+)= A^T Bm over all N rows (A: [N, m], Bm: [N, ne], both bf16, one already scaled by
 // c_i), plus noise when noise_std != 0.  `accumulate` = 0 overwrites out.
-// With `defer` (a block step), noise that cannot ride in the epilogue (split K) is queued
-// there instead of launched.  With `preset` (split K only), out already holds the noise
-// (written by the row-scaling launch) and the sum is added to it.
+// With `defer` (a block step), noise that neither the epilogue nor a combining launch adds
+// (splits added by atomics) is queued there instead of launched.  With `preset`, out already
+// holds the noise (written by the row-scaling launch) and the sum is added to it.
 // Split over K with `fx`: each split stores its partial sum, and a combining launch adds the
 // noise and them, in split order, to out's contents (accumulate or preset) in fp64 and rounds
 // once (kOutSplitPartials).  Without it, the splits add their partial sums into out by fp32
