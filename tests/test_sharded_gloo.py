@@ -1,8 +1,8 @@
-"""The sample-sharded step's orchestration on two CPU ranks (gloo), with the fp64 oracle as
-each rank's local compute.
+"""The sample-sharded step's orchestration on two and three CPU ranks (gloo), with the fp64
+oracle as each rank's local compute.
 
-Two ranks each hold half of the batch, clip and sum their own samples, all-reduce the sums
-and add the noise once on every rank.  Every rank must end with the one-device result on the
+The ranks each hold a contiguous share of the batch, clip and sum their own samples,
+all-reduce the sums and add the noise once on every rank.  Every rank must end with the one-device result on the
 whole batch: the oracle's step, noise included.  This checks the sharding logic (which
 samples, which bound, noise added once, flat norms local to a sample); the GPU path plugs the
 CUDA library into the same function.
@@ -78,21 +78,31 @@ def _rank(rank, world, port, mode, out):
         dist.destroy_process_group()
 
 
+# Two ranks split the 5 samples 3 / 2; three ranks 2 / 2 / 1.
+@pytest.mark.parametrize("world", [2, 3])
 @pytest.mark.parametrize("mode", ["per_layer", "flat"])
-def test_two_ranks_match_one_device_step(mode):
+def test_ranks_match_one_device_step(mode, world):
     port = _free_port()
     out = mp.get_context("spawn").Manager().dict()
-    mp.start_processes(_rank, args=(2, port, mode, out), nprocs=2, join=True, start_method="spawn")
+    mp.start_processes(_rank, args=(world, port, mode, out), nprocs=world, join=True, start_method="spawn")
     full = _batch()
     want = oracle.block_step([dict(l) for l in full], 2.5, 0.8, 11, 4, mode=mode)
-    for rank in (0, 1):
+    covered = []
+    for rank in range(world):
         sums, norms, (lo, hi) = out[rank]
+        covered.append((lo, hi))
         for k, layer in enumerate(want["layers"]):
             np.testing.assert_allclose(sums[k], layer["out"], rtol=1e-12, atol=1e-12)
             np.testing.assert_allclose(norms[k], layer["norms"][lo:hi], rtol=1e-13)
-    # Both ranks hold identical noisy sums: the noise was drawn once from the shared counter.
-    for a, b in zip(out[0][0], out[1][0]):
-        assert np.array_equal(a, b)
+    assert sorted(covered) == sharded_spans(full[0]["X"].shape[0], world)
+    # Every rank holds identical noisy sums: the noise was drawn once from the shared counter.
+    for rank in range(1, world):
+        for a, b in zip(out[0][0], out[rank][0]):
+            assert np.array_equal(a, b)
+
+
+def sharded_spans(B, world):
+    return [sharded.shard_rows(B, r, world) for r in range(world)]
 
 
 def test_shard_rows_cover_the_batch():
