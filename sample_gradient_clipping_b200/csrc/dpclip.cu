@@ -549,8 +549,6 @@ dp_status bf16_norms_ghost_shared(const Shape& s, const void* X, const void* con
 dp_status launch_noise(float* G, unsigned long long total, double std_dev, unsigned long long seed,
                        StepRef step, unsigned layer_id, cudaStream_t stream);
 
-// How the clipped-sum contraction of shape s is tiled: SM-pair tiles or not, and into how many
-// K splits (a split-K sum lands by fp32 atomics).
 // The combining launch of clipped sums split over K (combine_splits_kernel).
 dp_status launch_combine(const CombineBatch& b, cudaStream_t stream) {
   if (b.count == 0) return DP_OK;
